@@ -1,0 +1,375 @@
+#!/usr/bin/env python
+"""Benchmark: EAGLE-3 tree-verification step on B200.
+
+Default workload (one GPU): Llama-3.1-8B-shaped bf16 random-init target,
+batch 1, prefix 2048 tokens, a 60-draft tree of depth 8 (per-level widths
+10,10,10,8,8,6,4,4, top-k 10 expansion) whose tokens are planted with
+acceptance probability 0.8.  A step is one whole verification: one target
+forward over the 61 tree nodes on top of the cache, argmax acceptance, bonus
+token, K/V compaction.  Every step replays the same step from the same cached
+state (the sequence is rolled back between steps, outside the timed region).
+
+Prints ONE JSON line (rank 0).  `--impl reference` times the float64 CPU
+oracle on a bounded sample of the same workload instead.
+
+    python bench.py [--gpus N] [--steps K] [--warmup W] [--impl ours|reference]
+"""
+
+from __future__ import annotations
+
+import argparse
+import json
+import os
+import statistics
+import subprocess
+import sys
+import tempfile
+import time
+
+import numpy as np
+
+ROOT = os.path.dirname(os.path.abspath(__file__))
+sys.path.insert(0, ROOT)
+
+import synth  # noqa: E402
+
+METRIC = "verify steps/s and accepted tokens/s at Llama-3.1-8B shape; % HBM roofline"
+UNIT = "verify steps/s"
+
+
+def workload_config(P=2048):
+    return {"workload": "llama3.1-8b-shape bf16, batch 1, prefix %d, 60-draft depth-8 tree (widths 10,10,10,8,8,6,4,4),"
+                        " planted acceptance p=0.8" % P,
+            "model_shape": "32 layers, d 4096, 32/8 heads x 128, ffn 14336, vocab 128256",
+            "batch": 1, "prefix": P, "tree_nodes": 61, "depth": 8, "accept_p": 0.8,
+            "l2": "inputs larger than L2 (15 GB of weights streamed per step)",
+            "parallelism": "replicas (one independent verifier per GPU)"}
+
+
+def measured_peaks():
+    p = os.path.join(ROOT, "MEASURED_PEAKS.json")
+    if os.path.exists(p):
+        j = json.load(open(p))
+        return float(j["hbm_gbs"]), float(j["bf16_tflops"]), "measured"
+    return 6650.0, 1590.0, "fallback"
+
+
+def step_bytes(d, P, n):
+    """Algorithmic bytes of one verification step (bf16): every weight once, the prefix K/V, the tree K/V."""
+    per_layer = 2 * (d.q_dim * d.hidden + 2 * d.kv_dim * d.hidden + d.hidden * d.q_dim + 3 * d.ffn * d.hidden)
+    weights = d.n_layers * per_layer + 2 * d.vocab * d.hidden
+    kv_tok = d.n_layers * 2 * d.kv_dim * 2
+    return weights + P * kv_tok + n * kv_tok + n * d.hidden * 2
+
+
+def class_bytes(d, M, P, n):
+    """Algorithmic bytes per launch of each GEMM class: weights + activations in + outputs."""
+    a = 2  # bf16
+    return {
+        "gemm_qkv": a * (d.q_dim + 2 * d.kv_dim) * d.hidden + a * M * d.hidden + 4 * M * (d.q_dim + 2 * d.kv_dim),
+        "gemm_o": a * d.hidden * d.q_dim + a * M * d.q_dim + 4 * M * d.hidden,
+        "gemm_gate_up": a * 2 * d.ffn * d.hidden + a * M * d.hidden + a * M * d.ffn,
+        "gemm_down": a * d.hidden * d.ffn + a * M * d.ffn + 4 * M * d.hidden,
+        "lm_head": a * d.vocab * d.hidden + a * M * d.hidden,
+        "attention": (P + n) * d.kv_dim * 2 * a + M * d.q_dim * a * 2,
+    }
+
+
+class ClockSampler:
+    """nvidia-smi clock / throttle sampling while the timed region runs."""
+
+    FIELDS = ("index,clocks.sm,clocks.max.sm,power.draw,clocks_event_reasons.active,"
+              "clocks_event_reasons.hw_slowdown,clocks_event_reasons.hw_thermal_slowdown,"
+              "clocks_event_reasons.sw_thermal_slowdown,clocks_event_reasons.sw_power_cap")
+
+    def __init__(self, gpu_id: str):
+        self.f = tempfile.NamedTemporaryFile("w+", suffix=".csv", delete=False)
+        try:
+            self.p = subprocess.Popen(["nvidia-smi", "-i", gpu_id, "--query-gpu=" + self.FIELDS,
+                                       "--format=csv,noheader,nounits", "-lms", "200"],
+                                      stdout=self.f, stderr=subprocess.DEVNULL)
+        except Exception:
+            self.p = None
+
+    def stop(self):
+        if self.p is None:
+            return None
+        self.p.terminate()
+        try:
+            self.p.wait(timeout=5)
+        except Exception:
+            self.p.kill()
+        self.f.flush()
+        rows = []
+        for ln in open(self.f.name):
+            parts = [x.strip() for x in ln.split(",")]
+            if len(parts) >= 9:
+                rows.append(parts)
+        os.unlink(self.f.name)
+        if not rows:
+            return None
+        sm = [float(r[1]) for r in rows if r[1].replace(".", "").isdigit()]
+        mx = [float(r[2]) for r in rows if r[2].replace(".", "").isdigit()]
+        names = ["hw_slowdown", "hw_thermal_slowdown", "sw_thermal_slowdown", "sw_power_cap"]
+        reasons = sorted({names[i] for r in rows for i in range(4) if r[5 + i].lower().startswith("active")})
+        return {"sm_mhz": statistics.median(sm) if sm else None, "sm_max_mhz": max(mx) if mx else None,
+                "reasons": reasons, "samples": len(rows)}
+
+
+def gpu_uuid(dev):
+    import torch
+    try:
+        return "GPU-" + str(torch.cuda.get_device_properties(dev).uuid)
+    except Exception:
+        return str(dev)
+
+
+# ---------------------------------------------------------------------------
+# CPU oracle timing (bounded sample)
+# ---------------------------------------------------------------------------
+
+def oracle_step_sample(dims, host_w, P, tokens, parents, n_layers_sample=2, seed=0):
+    """Time the float64 oracle's verification step on a bounded sample.
+
+    Sample: `n_layers_sample` of the decoder layers (each over the full tree and
+    a P-token prefix cache) plus the LM head over all tree nodes, timed with the
+    oracle's own layer and LM-head functions; a full step is extrapolated as
+    n_layers x (mean layer time) + LM-head time.  The prefix K/V values are
+    seeded random (the oracle's work does not depend on them).
+    """
+    import oracle
+    from oracle.model import OracleModel
+    from oracle.tree import tree_meta, ancestor_matrix
+    rng = np.random.default_rng(seed)
+    om = OracleModel(dims, host_w, cache_limit_bytes=0)
+    depth, _ = tree_meta(parents)
+    vis = ancestor_matrix(parents)
+    x = om.embed(tokens)
+    pos = P + depth
+    t_layers = []
+    t_all0 = time.perf_counter()
+    for l in range(n_layers_sample):
+        pk = rng.standard_normal((P, dims.n_kv_heads, dims.head_dim))
+        pv = rng.standard_normal((P, dims.n_kv_heads, dims.head_dim))
+        t0 = time.perf_counter()
+        x, _, _ = om.layer_forward(l, x, pos, pk, pv, vis)
+        t_layers.append(time.perf_counter() - t0)
+    t0 = time.perf_counter()
+    logits = om.lm_logits(x)
+    amax = np.argmax(logits, axis=1)
+    oracle.accept_walk(tokens, parents, amax)
+    t_lm = time.perf_counter() - t0
+    wall = time.perf_counter() - t_all0
+    per_step = dims.n_layers * float(np.mean(t_layers)) + t_lm
+    return per_step, wall
+
+
+def threads_used():
+    try:
+        from threadpoolctl import threadpool_info
+        return max([i.get("num_threads", 1) for i in threadpool_info()] + [1])
+    except Exception:
+        return len(os.sched_getaffinity(0))
+
+
+def host_sample_weights(wdev, n_layers_sample):
+    sub = {"embed": wdev["embed"], "lm_head": wdev["lm_head"], "final_norm": wdev["final_norm"],
+           "layers": wdev["layers"][:n_layers_sample]}
+    return synth.weights_to_host(sub)
+
+
+# ---------------------------------------------------------------------------
+# reference arm: the oracle
+# ---------------------------------------------------------------------------
+
+def run_reference(args, rank, world):
+    if rank != 0:
+        return 0
+    import torch
+    dims = synth.LLAMA8B
+    P = args.prefix
+    shape = synth.tree_from_widths(synth.TREE60_WIDTHS, stream=0)
+    draws = synth.plant_draws(shape.n, dims.vocab, stream=0)
+    # tokens: the planting rule needs the target's argmax, which only a full
+    # float64 prefill would give here; the oracle's cost does not depend on
+    # token values, so the timed sample uses the uniform draws directly
+    tokens = draws.rand_tok.copy()
+    dev = "cuda" if torch.cuda.is_available() else "cpu"
+    wsmall = synth.model_weights(synth.ModelDims(args.sample_layers, dims.hidden, dims.n_q_heads, dims.n_kv_heads,
+                                                 dims.head_dim, dims.ffn, dims.vocab, dims.rms_eps, dims.rope_theta,
+                                                 "bf16"), seed=0, device=dev)
+    host = synth.weights_to_host(wsmall)
+    times = []
+    for _ in range(min(1, args.warmup)):
+        oracle_step_sample(dims, host, P, tokens, shape.parents, args.sample_layers, seed=99)
+    for k in range(args.steps):
+        per_step, wall = oracle_step_sample(dims, host, P, tokens, shape.parents, args.sample_layers, seed=k)
+        times.append(per_step)
+    v = 1.0 / float(np.mean(times))
+    cores = len(os.sched_getaffinity(0))
+    line = {"impl": "reference", "metric": METRIC, "value": v, "unit": UNIT, "n_gpus": world, "steps": args.steps,
+            "warmup": args.warmup, "ms_per_step": 1000.0 * float(np.mean(times)), "higher_is_better": True,
+            "scaling": "weak", "vs_baseline": None, "dtype": "f64", "data": "synthetic",
+            "config": workload_config(P),
+            "cpu_baseline": {"value": v, "unit": UNIT, "cores": cores, "threads": threads_used(), "kind": "oracle",
+                             "sample": "%d of 32 decoder layers + LM head per step, extrapolated to 32 layers"
+                                       % args.sample_layers},
+            "e2e": {"value": v, "unit": UNIT, "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0}}
+    print(json.dumps(line))
+    return 0
+
+
+# ---------------------------------------------------------------------------
+# our arm
+# ---------------------------------------------------------------------------
+
+def run_ours(args, rank, world, local_rank):
+    import torch
+    from speculative_decoding_06_b200.engine import SpecEngine, pack_trees
+    from speculative_decoding_06_b200 import spec as S
+
+    torch.cuda.set_device(local_rank)
+    dist = None
+    if world > 1:
+        import datetime
+        import torch.distributed as dist
+        dist.init_process_group("nccl", timeout=datetime.timedelta(seconds=120), device_id=torch.device("cuda", local_rank))
+    dims = synth.LLAMA8B
+    P = args.prefix
+    w = synth.model_weights(dims, seed=0, device="cuda")
+    eng = SpecEngine(dims, w, max_batch=1, max_seq=P + 256, max_nodes=64)
+    prefix = synth.prefix_tokens(dims.vocab, P, seed=1)
+    pend = eng.prefill(0, prefix)
+    shape = synth.tree_from_widths(synth.TREE60_WIDTHS, stream=0)
+    draws = synth.plant_draws(shape.n, dims.vocab, stream=0)
+
+    def gpu_argmax(tokens, parents):
+        return eng.score([0], [(tokens, parents)])[0]
+
+    tokens = synth.plant_tree(shape, pend, 0.8, draws, gpu_argmax)
+    tk, pr, off = pack_trees([(tokens, shape.parents)])
+    ids = np.array([0], np.int32)
+    acc_dev = torch.zeros(1, dtype=torch.int32, device="cuda")
+    stream = torch.cuda.current_stream()
+
+    def one_step():
+        eng.verify_batch_device(ids, tk, pr, off, outputs=(acc_dev, None, None, None))
+
+    # warm-up (also captures the CUDA graph)
+    for _ in range(max(3, args.warmup)):
+        one_step()
+        eng.sync()
+        eng.truncate(0, P)
+    a_len, _, _ = eng.verify(0, tokens, shape.parents)
+    eng.truncate(0, P)
+    launches = eng.step_launches()
+
+    # ---- timed region: K steps, device time from CUDA events on the launching stream
+    clk = ClockSampler(gpu_uuid(local_rank))
+    if dist:
+        dist.barrier()
+    torch.cuda.synchronize()
+    times = []
+    for _ in range(args.steps):
+        e0 = torch.cuda.Event(enable_timing=True)
+        e1 = torch.cuda.Event(enable_timing=True)
+        e0.record(stream)
+        one_step()
+        e1.record(stream)
+        e1.synchronize()
+        times.append(e0.elapsed_time(e1))
+        eng.sync()
+        eng.truncate(0, P)
+    torch.cuda.synchronize()
+    if dist:
+        dist.barrier()
+    clocks = clk.stop()
+    t_total = float(sum(times))
+    if dist:
+        tt = torch.tensor([t_total], device="cuda")
+        dist.all_reduce(tt, op=dist.ReduceOp.MAX)
+        t_total = float(tt.item())
+    ms = t_total / args.steps
+    value = world * args.steps / (t_total / 1000.0)
+
+    # ---- end to end through the public API with host buffers (H2D + D2H inside)
+    e2e_times = []
+    for _ in range(args.steps):
+        torch.cuda.synchronize()
+        t0 = time.perf_counter()
+        eng.verify(0, tokens, shape.parents)
+        e2e_times.append(time.perf_counter() - t0)
+        eng.truncate(0, P)
+    h2d, d2h = eng.io_bytes()
+    e2e_value = world / float(np.mean(e2e_times))
+
+    # ---- per-kernel-class device time (event pair per launch, launch by launch)
+    eng.profile(True)
+    nprof = 3
+    for _ in range(nprof):
+        eng.verify_batch_device(ids, tk, pr, off)
+        eng.sync()
+        eng.truncate(0, P)
+    prof = eng.profile_read()
+    eng.profile(False)
+    hbm, tflops, peak_kind = measured_peaks()
+    M = shape.n
+    cb = class_bytes(dims, M, P, shape.n)
+    dom = max(cb, key=lambda k: prof[k][0])
+    dom_ms, dom_n = prof[dom]
+    achieved = cb[dom] / ((dom_ms / dom_n) / 1000.0) / 1e9
+    sb = step_bytes(dims, P, shape.n)
+    step_gbs = sb / (ms / 1000.0) / 1e9
+    kernel_share = {k: round(v[0] / nprof, 4) for k, v in prof.items()}
+
+    line = {
+        "metric": METRIC, "value": value, "unit": UNIT, "n_gpus": world, "steps": args.steps,
+        "warmup": max(3, args.warmup), "ms_per_step": ms, "higher_is_better": True, "scaling": "weak",
+        "vs_baseline": None, "dtype": "bf16", "data": "synthetic (random-init weights, uniform prefix, planted tree)",
+        "config": workload_config(P),
+        "accepted_tokens_per_s": value * (a_len + 1), "tau": a_len + 1,
+        "roofline": {"bound": "hbm", "kernel": dom, "achieved": achieved, "peak": hbm, "unit": "GB/s",
+                     "frac": achieved / hbm, "traffic": None, "peak_source": peak_kind,
+                     "bytes_per_launch": cb[dom], "ms_per_launch": dom_ms / dom_n},
+        "step_roofline": {"bound": "hbm", "bytes_per_step": sb, "achieved": step_gbs, "peak": hbm, "unit": "GB/s",
+                          "frac": step_gbs / hbm, "roofline_ms": sb / hbm / 1e6},
+        "kernel_ms_per_step": kernel_share,
+        "e2e": {"value": e2e_value, "unit": UNIT, "h2d_bytes_per_step": h2d, "d2h_bytes_per_step": d2h},
+        "gpu_launches": launches * args.steps,
+        "clocks": clocks,
+    }
+    if rank == 0 and world == 1 and not args.no_cpu_baseline:
+        hostw = host_sample_weights(w, args.sample_layers)
+        per_step, wall = oracle_step_sample(dims, hostw, P, tokens, shape.parents, args.sample_layers)
+        line["cpu_baseline"] = {"value": 1.0 / per_step, "unit": UNIT, "cores": len(os.sched_getaffinity(0)),
+                                "threads": threads_used(), "kind": "oracle",
+                                "sample": "%d of 32 decoder layers (61-node tree, prefix %d) + LM head, extrapolated"
+                                          " to 32 layers; %.1f s of CPU work" % (args.sample_layers, P, wall)}
+    if rank == 0:
+        print(json.dumps(line))
+    eng.close()
+    if dist:
+        dist.destroy_process_group()
+    return 0
+
+
+def main():
+    ap = argparse.ArgumentParser()
+    ap.add_argument("--gpus", type=int, default=1)
+    ap.add_argument("--steps", type=int, default=20)
+    ap.add_argument("--warmup", type=int, default=5)
+    ap.add_argument("--impl", default="ours", choices=["ours", "reference"])
+    ap.add_argument("--prefix", type=int, default=2048)
+    ap.add_argument("--sample-layers", type=int, default=2)
+    ap.add_argument("--no-cpu-baseline", action="store_true")
+    args = ap.parse_args()
+    rank = int(os.environ.get("RANK", "0"))
+    world = int(os.environ.get("WORLD_SIZE", "1"))
+    local_rank = int(os.environ.get("LOCAL_RANK", "0"))
+    if args.impl == "reference":
+        return run_reference(args, rank, world)
+    return run_ours(args, rank, world, local_rank)
+
+
+if __name__ == "__main__":
+    sys.exit(main())

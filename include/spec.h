@@ -1,0 +1,215 @@
+/*
+ * spec.h -- C ABI of a B200 (sm_100a) library for the tree-verification step
+ * of EAGLE-3 speculative decoding.
+ *
+ * What the step computes ("EAGLE-3投机解码：树验证器方法", fanquanpp.github.io,
+ * sections 验证-接受语义 and 树draft vs 链draft):
+ *   - the target model runs ONE forward pass over a whole draft tree, given as
+ *     a token array plus parent indices, on top of the sequence's K/V cache;
+ *   - every tree node attends to the cached prefix and to its own ancestors
+ *     only (the tree's structure is fixed before verification);
+ *   - a draft node is accepted iff its token equals the target's argmax at its
+ *     parent; the walk from the root keeps the longest accepted path (lowest
+ *     index child first) and emits one bonus token, the target's argmax at the
+ *     last accepted node -- so each step emits accepted_len + 1 tokens, exactly
+ *     what greedy autoregressive decoding would emit;
+ *   - only the root's and the accepted nodes' K/V stay in the cache, moved to
+ *     consecutive slots.
+ *
+ * Conventions for every function below:
+ *   - return value: SPEC_OK (0) or a negative SPEC_ERR_* code; on error the
+ *     cached state of every sequence is unchanged and spec_last_error() holds
+ *     a message;
+ *   - "device" pointers are CUDA device memory of the GPU that was current at
+ *     spec_init; "host" pointers are ordinary CPU memory;
+ *   - the library borrows every buffer it is given (weights, K/V cache,
+ *     workspace) and never frees one; they must outlive the handle;
+ *   - a handle is not thread-safe; all GPU work runs on the stream given to
+ *     spec_init.
+ */
+#ifndef SPEC_H
+#define SPEC_H
+
+#include <stddef.h>
+#include <stdint.h>
+
+#if defined(__GNUC__)
+#define SPEC_API __attribute__((visibility("default")))
+#else
+#define SPEC_API
+#endif
+
+#ifdef __cplusplus
+extern "C" {
+#endif
+
+/* return codes */
+#define SPEC_OK 0
+#define SPEC_ERR_ARG (-1)      /* null pointer, bad dimension, misaligned buffer */
+#define SPEC_ERR_TREE (-2)     /* parents[0] != -1, or some parents[i] outside [0, i) */
+#define SPEC_ERR_TOKEN (-3)    /* a token outside [0, vocab) */
+#define SPEC_ERR_CAPACITY (-4) /* n_nodes > max_nodes, batch > max_batch, length + n_nodes > max_seq, buffer too small */
+#define SPEC_ERR_ROOT (-5)     /* tokens[0] is not the sequence's pending token */
+#define SPEC_ERR_CUDA (-6)     /* a CUDA call failed; the message names the cudaError_t */
+#define SPEC_ERR_TIMEOUT (-7)  /* a bounded wait inside a kernel expired */
+#define SPEC_ERR_STATE (-8)    /* sequence not prefilled, or truncation beyond its length */
+
+/* model dtypes */
+#define SPEC_DTYPE_F32 0       /* weights, activations and K/V in fp32; plain FFMA arithmetic */
+#define SPEC_DTYPE_BF16 1      /* weights and K/V in bf16; fp32 accumulation, residual and softmax */
+
+/* flags of spec_verify_tree_batch */
+#define SPEC_DEVICE_OUTPUTS 1  /* outputs are device pointers (or NULL); return without synchronising */
+#define SPEC_DEBUG_LOGITS 2    /* also store fp32 logits [total nodes][vocab] to the buffer of spec_set_debug_logits */
+#define SPEC_NO_GRAPH 4        /* launch kernel by kernel instead of replaying a captured CUDA graph */
+
+typedef struct spec_config {
+  int32_t n_layers;
+  int32_t hidden;       /* d */
+  int32_t n_q_heads;    /* Hq */
+  int32_t n_kv_heads;   /* Hkv; Hq % Hkv == 0 (query head j reads kv head j / (Hq/Hkv)) */
+  int32_t head_dim;     /* hd; bf16 models need 128, fp32 models <= 128 and even */
+  int32_t ffn;          /* SwiGLU width */
+  int32_t vocab;
+  int32_t dtype;        /* SPEC_DTYPE_* */
+  float rms_eps;        /* RMSNorm epsilon */
+  float rope_theta;     /* rotary base (rotate-half pairing, no frequency scaling) */
+  int32_t max_batch;    /* sequences held in the cache */
+  int32_t max_seq;      /* cache slots per sequence */
+  int32_t max_nodes;    /* tree nodes per sequence per step, root included; <= 128 */
+  int32_t draft_head;   /* 1: also size buffers for the EAGLE-3 draft head (bf16 only) */
+} spec_config;
+
+/* Per-layer weights, device pointers, row-major [out][in] in the model dtype:
+ * wq [Hq*hd][d], wk/wv [Hkv*hd][d], wo [d][Hq*hd], w_gate/w_up [ffn][d],
+ * w_down [d][ffn]; attn_norm / mlp_norm [d]. */
+typedef struct spec_layer_weights {
+  const void* wq;
+  const void* wk;
+  const void* wv;
+  const void* wo;
+  const void* w_gate;
+  const void* w_up;
+  const void* w_down;
+  const void* attn_norm;
+  const void* mlp_norm;
+} spec_layer_weights;
+
+/* Model weights.  `layers` is a HOST array of n_layers entries (copied by
+ * spec_init); every weight pointer in it, and embed [vocab][d], final_norm [d],
+ * lm_head [vocab][d], are device pointers 16-byte aligned.  The draft-head
+ * fields may be NULL when cfg.draft_head == 0: draft_fc_fuse [d][3d],
+ * draft_fc_in [d][2d], draft_layer (host pointer to one entry), draft_final_norm [d]. */
+typedef struct spec_weights {
+  const void* embed;
+  const void* final_norm;
+  const void* lm_head;
+  const spec_layer_weights* layers;
+  const void* draft_fc_fuse;
+  const void* draft_fc_in;
+  const spec_layer_weights* draft_layer;
+  const void* draft_final_norm;
+} spec_weights;
+
+typedef struct spec_handle spec_handle;
+
+/* Bytes of device memory for the K/V cache (layout [layer][K|V][seq][kv head][slot][hd]). */
+SPEC_API size_t spec_kv_bytes(const spec_config* cfg);
+/* Bytes of device workspace (activations, split-K partials, per-sequence state). */
+SPEC_API size_t spec_workspace_bytes(const spec_config* cfg);
+
+/* Validate dimensions, record the borrowed device buffers, build the TMA
+ * descriptors.  kv_cache and workspace are device buffers of at least the
+ * sizes above; cuda_stream is a cudaStream_t (NULL: the legacy default stream).
+ * Every sequence starts empty. */
+SPEC_API int spec_init(const spec_config* cfg, const spec_weights* w, void* kv_cache, size_t kv_bytes, void* workspace,
+              size_t ws_bytes, void* cuda_stream, spec_handle** out);
+
+/* Reset sequence `seq` and run the prompt (host int32[n], n >= 1) through the
+ * target in causal chunks of at most max_nodes tokens, caching every position.
+ * *pending_token (host) receives the argmax at the last position: the root of
+ * the next tree.  Synchronises the stream. */
+SPEC_API int spec_prefill(spec_handle* h, int seq, const int32_t* tokens, int n, int32_t* pending_token);
+
+/* One verification step for one sequence (host pointers, synchronises).
+ * tokens[0] must be the pending token; parents[0] == -1 and 0 <= parents[i] < i.
+ * accepted_tokens needs room for n_nodes - 1 entries.  Emitted tokens are
+ * accepted_tokens[0 .. *accepted_len) followed by *bonus_token, which becomes
+ * the next pending token. */
+SPEC_API int spec_verify_tree(spec_handle* h, int seq, const int32_t* tokens, const int32_t* parents, int n_nodes,
+                     int32_t* accepted_len, int32_t* accepted_tokens, int32_t* bonus_token);
+
+/* Batched verification.  Host inputs: seq_ids[B] (distinct), node_offsets[B+1]
+ * (node_offsets[0] == 0), tokens / parents concatenated per sequence, parents
+ * local to their sequence.  Outputs per sequence b: accepted_len[b],
+ * accepted_nodes[b * max_nodes + k] (local node indices), accepted_tokens
+ * (same layout), bonus[b].  Without SPEC_DEVICE_OUTPUTS they are host pointers
+ * and the call synchronises; with it they are device pointers (or NULL) and the
+ * call returns once the work is queued -- errors found on the device are then
+ * reported by the next spec_sync. */
+SPEC_API int spec_verify_tree_batch(spec_handle* h, int B, const int32_t* seq_ids, const int32_t* tokens,
+                           const int32_t* parents, const int32_t* node_offsets, int32_t* accepted_len,
+                           int32_t* accepted_nodes, int32_t* accepted_tokens, int32_t* bonus, int flags);
+
+/* The target's argmax (and top-1 / top-2 logits) at every node of a batch of
+ * trees, without acceptance and without changing any cached state.  Inputs as
+ * in spec_verify_tree_batch; outputs are host arrays of node_offsets[B]
+ * entries.  Synchronises. */
+SPEC_API int spec_score_trees(spec_handle* h, int B, const int32_t* seq_ids, const int32_t* tokens, const int32_t* parents,
+                     const int32_t* node_offsets, int32_t* argmax, float* top1, float* top2, int flags);
+
+/* Device buffer (fp32, >= max_batch * max_nodes * vocab entries) for SPEC_DEBUG_LOGITS. */
+SPEC_API int spec_set_debug_logits(spec_handle* h, float* device_buf, size_t bytes);
+
+/* Roll sequence `seq` back to new_len cached positions (new_len < current
+ * length, or equal for a no-op); the token cached at new_len becomes pending. */
+SPEC_API int spec_truncate(spec_handle* h, int seq, int new_len);
+/* Cached length and pending token of `seq` (host outputs; synchronises). */
+SPEC_API int spec_seq_len(spec_handle* h, int seq, int32_t* len, int32_t* pending);
+/* Wait for queued work; report (and clear) errors recorded on the device. */
+SPEC_API int spec_sync(spec_handle* h);
+
+/* Host-only check of one tree, usable without a GPU or a handle: 1 <= n <=
+ * max_nodes (else SPEC_ERR_CAPACITY), parents[0] == -1 and 0 <= parents[i] < i
+ * (else SPEC_ERR_TREE), every token in [0, vocab) (else SPEC_ERR_TOKEN); null
+ * pointers give SPEC_ERR_ARG.  The verification calls apply the same checks. */
+SPEC_API int spec_validate_tree(const int32_t* tokens, const int32_t* parents, int n, int vocab, int max_nodes);
+
+/* Kernel classes timed by the profiler (index into spec_profile_read's arrays). */
+#define SPEC_PROF_EMBED_META 0   /* tree metadata + embedding + first RMSNorm */
+#define SPEC_PROF_GEMM_QKV 1
+#define SPEC_PROF_ROPE_KV 2      /* split-K sum + rotary + K/V cache store */
+#define SPEC_PROF_ATTENTION 3    /* tree attention chunks + merge */
+#define SPEC_PROF_GEMM_O 4
+#define SPEC_PROF_RESID_NORM 5   /* split-K sum + residual + RMSNorm */
+#define SPEC_PROF_GEMM_GATE_UP 6 /* gate/up GEMM with fused SwiGLU */
+#define SPEC_PROF_GEMM_DOWN 7
+#define SPEC_PROF_LM_HEAD 8      /* LM-head GEMM with fused argmax */
+#define SPEC_PROF_LM_REDUCE 9
+#define SPEC_PROF_WALK 10        /* acceptance walk + state update */
+#define SPEC_PROF_COMPACT 11     /* K/V compaction */
+#define SPEC_PROF_CLASSES 12
+
+/* enable != 0: subsequent steps launch kernel by kernel (no graph) with a CUDA
+ * event pair around every launch on the handle's stream. */
+SPEC_API int spec_profile(spec_handle* h, int enable);
+/* Synchronise, then add the recorded device milliseconds and launch counts per
+ * class into ms[SPEC_PROF_CLASSES] and launches[SPEC_PROF_CLASSES] (host
+ * arrays, either may be NULL) and forget the records. */
+SPEC_API int spec_profile_read(spec_handle* h, double* ms, int64_t* launches);
+/* Bytes one synchronous verification step copies host->device (parameter
+ * block) and device->host (outputs and error word). */
+SPEC_API int spec_io_bytes(spec_handle* h, size_t* h2d, size_t* d2h);
+/* Number of kernels the most recent step enqueued. */
+SPEC_API int spec_step_launches(spec_handle* h);
+
+/* Message of the last error on this handle ("" if none). */
+SPEC_API const char* spec_last_error(spec_handle* h);
+/* Free host-side state (graphs, descriptors); never frees borrowed buffers. */
+SPEC_API void spec_free(spec_handle* h);
+
+#ifdef __cplusplus
+}
+#endif
+
+#endif /* SPEC_H */

@@ -1,0 +1,139 @@
+// Internal kernel interfaces of the tree-verification library (host <-> device
+// argument structs and launchers).  Not part of the public C ABI.
+#pragma once
+
+#include <cstddef>
+#include <cstdint>
+#include <cuda.h>
+#include <cuda_bf16.h>
+#include <cuda_runtime.h>
+
+namespace spec {
+
+struct Top2;
+
+enum { GEMM_EPI_PARTIAL = 0, GEMM_EPI_SWIGLU = 1, GEMM_EPI_ARGMAX = 2 };
+
+struct GemmTcArgs {
+  int n_out;          // output features (weight rows) across all segments
+  int K;              // reduction length, multiple of 64
+  int M;              // valid tokens (columns); token rows >= M are ignored
+  int tiles_o, tiles_t, splits, kb_per_split;
+  int seg_rows[3];    // rows served by mA0, mA1, mA2 (PARTIAL); unused for SWIGLU
+  float* out_f32;     // PARTIAL: [splits][tokens][n_out]
+  size_t split_stride;
+  __nv_bfloat16* out_bf16;  // SWIGLU: [tokens][ld_out]
+  int ld_out;
+  Top2* top_part;     // ARGMAX: [tiles_o][top_ld]
+  int top_ld;
+  float* dbg_logits;  // ARGMAX: optional [M][n_out]
+  uint32_t* err;
+};
+
+struct GemmTcLaunch {
+  int bn, epi, grid;
+  const CUtensorMap *mA0, *mA1, *mA2, *mB;
+  GemmTcArgs args;
+};
+
+cudaError_t gemm_tc_launch(const GemmTcLaunch& L, cudaStream_t stream, bool pdl);
+uint32_t gemm_tc_smem_bytes(int bn, int epi);
+const void* gemm_tc_function(int bn, int epi);
+
+// One verification step, as seen by the kernels.  Node ("row") r in [0, M)
+// belongs to batch entry b with node_off[b] <= r < node_off[b+1]; its local
+// index is r - node_off[b]; parents hold local indices.
+struct StepView {
+  const int32_t* tokens;    // [M]
+  const int32_t* parents;   // [M]
+  const int32_t* node_off;  // [B+1]
+  const int32_t* seq_ids;   // [B]
+  int B, M;
+  int32_t* row_seq;         // [M] batch entry
+  int32_t* row_local;       // [M] local node index
+  int32_t* row_pos;         // [M] position P_b + depth
+  uint64_t* row_anc;        // [M][2] ancestor bits over local indices (self included)
+  float2* rope_cs;          // [M][head_dim/2] (cos, sin)
+  int32_t* P_step;          // [B] cached length at step start
+  int32_t* seq_len;         // [max_batch] persistent
+  int32_t* pending;         // [max_batch] persistent
+  int32_t* hist;            // [max_batch][max_seq] persistent token history
+  int max_seq;
+  uint32_t* err;            // this step's error bits
+  uint32_t* err_sticky;     // accumulated until read by the host
+};
+
+struct KvView {
+  void* base;               // [layer][2][max_batch][Hkv][max_seq][hd]
+  int max_batch, Hkv, max_seq, hd;
+  size_t elem;              // 2 (bf16) or 4 (fp32)
+  __host__ __device__ size_t head_stride() const { return (size_t)max_seq * hd; }
+  __host__ __device__ size_t seq_stride() const { return (size_t)Hkv * max_seq * hd; }
+  __host__ __device__ size_t kv_stride() const { return (size_t)max_batch * seq_stride(); }
+  __host__ __device__ size_t layer_stride() const { return 2 * kv_stride(); }
+};
+
+enum { STEP_VERIFY = 0, STEP_PREFILL = 1, STEP_SCORE = 2 };
+
+// metadata + embedding + first RMSNorm
+cudaError_t launch_embed_meta(int dtype, const StepView& sv, const void* embed, const void* norm_w, int d, float eps,
+                              float* x, void* xn, const double* inv_freq, int half, int mode, cudaStream_t s,
+                              bool pdl);
+// x += sum of split partials; xn = RMSNorm(x) * w
+cudaError_t launch_residual_norm(int dtype, int M, int d, int S, const float* partial, size_t split_stride, float* x,
+                                 void* xn, const void* w, float eps, cudaStream_t s, bool pdl);
+// sum partials, rotary on q and k, q -> q_out, k/v -> cache slots P_b + local
+cudaError_t launch_qkv_rope_store(int dtype, const StepView& sv, int S, const float* partial, size_t split_stride,
+                                  int Hq, int Hkv, int hd, void* q_out, const KvView& kv, int layer, cudaStream_t s,
+                                  bool pdl);
+// fp32 path: h = silu(gate) * up from a [M][2F] buffer
+cudaError_t launch_swiglu_f32(int M, int F, const float* gu, float* h, cudaStream_t s);
+// fp32 path SIMT GEMM: C[t][o] = sum_k A[t][k] W[o][k]
+cudaError_t launch_gemm_simt_f32(const float* A, int lda, const float* W, int K, float* C, int ldc, int M, int N,
+                                 cudaStream_t s);
+
+// attention
+struct AttnArgs {
+  StepView sv;
+  KvView kv;
+  int layer;
+  int Hq, hd;
+  const void* q;            // [M][Hq][hd]
+  void* out;                // [M][Hq*hd]
+  float* part_o;            // [M*Hq][n_chunks][hd]
+  float* part_lse;          // [M*Hq][n_chunks]
+  int n_chunks, chunk;      // key chunking of [0, P_b + n_b)
+  int max_rows;             // max over batch of n_b * (Hq/Hkv)
+};
+cudaError_t launch_attention(int dtype, const AttnArgs& a, cudaStream_t s, bool pdl);
+size_t attention_smem_bytes();
+cudaError_t attention_configure();
+
+// LM head reductions
+cudaError_t launch_top2_reduce(int M, int tiles, const Top2* part, int top_ld, int32_t* argmax, float* top1,
+                               float* top2, cudaStream_t s, bool pdl);
+cudaError_t launch_rows_top2_f32(int M, int V, const float* logits, int32_t* argmax, float* top1, float* top2,
+                                 cudaStream_t s);
+
+// acceptance walk (or commit-all for prefill chains) + state update
+struct WalkArgs {
+  StepView sv;
+  const int32_t* argmax;    // [M]
+  int32_t* acc_len;         // [B]
+  int32_t* acc_nodes;       // [B][max_nodes]
+  int32_t* acc_tokens;      // [B][max_nodes]
+  int32_t* bonus;           // [B]
+  int max_nodes;
+  int mode;
+};
+cudaError_t launch_accept_walk(const WalkArgs& w, cudaStream_t s, bool pdl);
+cudaError_t kv_compact_configure(size_t smem);
+// move accepted nodes' K/V to slots P+1..P+a (all layers, heads)
+cudaError_t launch_kv_compact(const StepView& sv, const KvView& kv, int n_layers, const int32_t* acc_len,
+                              const int32_t* acc_nodes, int max_nodes, cudaStream_t s, bool pdl);
+
+// draft-head pieces
+cudaError_t launch_gather_concat(int M, int d, const __nv_bfloat16* g, const int32_t* tokens,
+                                 const __nv_bfloat16* embed, __nv_bfloat16* out, cudaStream_t s);
+
+}  // namespace spec

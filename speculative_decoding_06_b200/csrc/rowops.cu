@@ -1,0 +1,358 @@
+// Row-wise kernels of the verification forward: tree metadata with the
+// embedding gather and first RMSNorm, split-K reduction fused with the
+// residual add and the next RMSNorm, rotary embedding fused with the K/V cache
+// store, the LM-head argmax reductions, and the fp32 (SIMT) GEMM used by the
+// fp32 model path.
+#include "common.cuh"
+#include "kernels.h"
+
+namespace spec {
+
+namespace {
+
+template <int NT>
+__device__ __forceinline__ float block_sum(float v, float* red) {
+  v = warp_sum(v);
+  const int w = threadIdx.x >> 5;
+  if ((threadIdx.x & 31) == 0) red[w] = v;
+  __syncthreads();
+  float t = 0.f;
+  if (threadIdx.x < 32) {
+    t = threadIdx.x < NT / 32 ? red[threadIdx.x] : 0.f;
+    t = warp_sum(t);
+    if (threadIdx.x == 0) red[0] = t;
+  }
+  __syncthreads();
+  t = red[0];
+  __syncthreads();
+  return t;
+}
+
+cudaLaunchConfig_t make_cfg(dim3 grid, dim3 block, size_t smem, cudaStream_t s, bool pdl, cudaLaunchAttribute* attr) {
+  cudaLaunchConfig_t cfg = {};
+  cfg.gridDim = grid;
+  cfg.blockDim = block;
+  cfg.dynamicSmemBytes = smem;
+  cfg.stream = s;
+  attr[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+  attr[0].val.programmaticStreamSerializationAllowed = 1;
+  cfg.attrs = attr;
+  cfg.numAttrs = pdl ? 1 : 0;
+  return cfg;
+}
+
+}  // namespace
+
+// ---------------------------------------------------------------------------
+// tree metadata + embedding + RMSNorm
+// ---------------------------------------------------------------------------
+// One CTA per node.  A node's depth and ancestor set come from walking its
+// parent links up to the root ("EAGLE-3投机解码：树验证器方法", section 树draft vs
+// 链draft: every token sees only its ancestors); its position is P_b + depth.
+template <typename T>
+__global__ void __launch_bounds__(256) embed_meta_kernel(StepView sv, const T* __restrict__ embed,
+                                                         const T* __restrict__ norm_w, int d, float eps,
+                                                         float* __restrict__ x, T* __restrict__ xn,
+                                                         const double* __restrict__ inv_freq, int half, int mode) {
+  __shared__ int s_pos;
+  __shared__ float red[8];
+  pdl_wait();
+  const int r = blockIdx.x;
+  if (threadIdx.x == 0) {
+    int b = 0;
+    while (b + 1 < sv.B && sv.node_off[b + 1] <= r) ++b;
+    const int base = sv.node_off[b];
+    const int n = sv.node_off[b + 1] - base;
+    const int i = r - base;
+    const int seq = sv.seq_ids[b];
+    const int P = sv.seq_len[seq];
+    uint64_t a0 = 0, a1 = 0;
+    int depth = -1;
+    int j = i;
+    int guard = 0;
+    while (j >= 0 && guard <= n) {
+      if (j < 64) a0 |= 1ull << j; else a1 |= 1ull << (j - 64);
+      const int pj = sv.parents[base + j];
+      if (pj >= j) {  // malformed links are rejected on the host; never follow one here
+        set_error(sv.err, SPEC_DEVERR_BOUNDS);
+        break;
+      }
+      j = pj;
+      ++depth;
+      ++guard;
+    }
+    sv.row_seq[r] = b;
+    sv.row_local[r] = i;
+    sv.row_pos[r] = P + depth;
+    sv.row_anc[2 * r] = a0;
+    sv.row_anc[2 * r + 1] = a1;
+    if (i == 0) {
+      sv.P_step[b] = P;
+      if (mode == STEP_VERIFY && sv.tokens[r] != sv.pending[seq]) set_error(sv.err, SPEC_DEVERR_ROOT);
+    }
+    s_pos = P + depth;
+  }
+  __syncthreads();
+  const int pos = s_pos;
+  for (int j = threadIdx.x; j < half; j += blockDim.x) {
+    double sn, cs;
+    sincos((double)pos * inv_freq[j], &sn, &cs);
+    sv.rope_cs[(size_t)r * half + j] = make_float2((float)cs, (float)sn);
+  }
+  const int tok = sv.tokens[r];
+  const T* e = embed + (size_t)tok * d;
+  float* xr = x + (size_t)r * d;
+  float ss = 0.f;
+  for (int k = threadIdx.x; k < d; k += blockDim.x) {
+    const float v = to_f32(e[k]);
+    xr[k] = v;
+    ss += v * v;
+  }
+  ss = block_sum<256>(ss, red);
+  const float inv = rsqrtf(ss / (float)d + eps);
+  T* o = xn + (size_t)r * d;
+  for (int k = threadIdx.x; k < d; k += blockDim.x) o[k] = from_f32<T>(xr[k] * inv * to_f32(norm_w[k]));
+  pdl_launch_dependents();
+}
+
+cudaError_t launch_embed_meta(int dtype, const StepView& sv, const void* embed, const void* norm_w, int d, float eps,
+                              float* x, void* xn, const double* inv_freq, int half, int mode, cudaStream_t s,
+                              bool pdl) {
+  cudaLaunchAttribute attr[1];
+  cudaLaunchConfig_t cfg = make_cfg(dim3(sv.M), dim3(256), 0, s, pdl, attr);
+  if (dtype == 0)
+    return cudaLaunchKernelEx(&cfg, embed_meta_kernel<float>, sv, (const float*)embed, (const float*)norm_w, d, eps, x,
+                              (float*)xn, inv_freq, half, mode);
+  return cudaLaunchKernelEx(&cfg, embed_meta_kernel<__nv_bfloat16>, sv, (const __nv_bfloat16*)embed,
+                            (const __nv_bfloat16*)norm_w, d, eps, x, (__nv_bfloat16*)xn, inv_freq, half, mode);
+}
+
+// ---------------------------------------------------------------------------
+// split-K reduction + residual + RMSNorm
+// ---------------------------------------------------------------------------
+// x[r] += sum_s partial[s][r] (fixed order, deterministic); xn[r] = x[r] * rsqrt(mean x^2 + eps) * w.
+template <typename T>
+__global__ void __launch_bounds__(256) residual_norm_kernel(int d, int S, const float* __restrict__ partial,
+                                                            size_t split_stride, float* __restrict__ x,
+                                                            T* __restrict__ xn, const T* __restrict__ w, float eps) {
+  __shared__ float red[8];
+  pdl_wait();
+  const int r = blockIdx.x;
+  float* xr = x + (size_t)r * d;
+  const float* pr = partial + (size_t)r * d;
+  float ss = 0.f;
+  for (int k = threadIdx.x * 4; k < d; k += blockDim.x * 4) {
+    float4 acc = *reinterpret_cast<const float4*>(xr + k);
+    for (int sp = 0; sp < S; ++sp) {
+      const float4 p = *reinterpret_cast<const float4*>(pr + sp * split_stride + k);
+      acc.x += p.x; acc.y += p.y; acc.z += p.z; acc.w += p.w;
+    }
+    *reinterpret_cast<float4*>(xr + k) = acc;
+    ss += acc.x * acc.x + acc.y * acc.y + acc.z * acc.z + acc.w * acc.w;
+  }
+  ss = block_sum<256>(ss, red);
+  const float inv = rsqrtf(ss / (float)d + eps);
+  T* o = xn + (size_t)r * d;
+  for (int k = threadIdx.x; k < d; k += blockDim.x) o[k] = from_f32<T>(xr[k] * inv * to_f32(w[k]));
+  pdl_launch_dependents();
+}
+
+cudaError_t launch_residual_norm(int dtype, int M, int d, int S, const float* partial, size_t split_stride, float* x,
+                                 void* xn, const void* w, float eps, cudaStream_t s, bool pdl) {
+  cudaLaunchAttribute attr[1];
+  cudaLaunchConfig_t cfg = make_cfg(dim3(M), dim3(256), 0, s, pdl, attr);
+  if (dtype == 0)
+    return cudaLaunchKernelEx(&cfg, residual_norm_kernel<float>, d, S, partial, split_stride, x, (float*)xn,
+                              (const float*)w, eps);
+  return cudaLaunchKernelEx(&cfg, residual_norm_kernel<__nv_bfloat16>, d, S, partial, split_stride, x,
+                            (__nv_bfloat16*)xn, (const __nv_bfloat16*)w, eps);
+}
+
+// ---------------------------------------------------------------------------
+// split-K reduction + rotary embedding + K/V cache store
+// ---------------------------------------------------------------------------
+// Rotate-half pairing: element j and element j + hd/2 of a head form one pair,
+// rotated by pos * theta^(-2j/hd) (table computed in double per step).
+template <typename T>
+__global__ void __launch_bounds__(256) qkv_rope_store_kernel(StepView sv, int S, const float* __restrict__ partial,
+                                                             size_t split_stride, int Hq, int Hkv, int hd,
+                                                             T* __restrict__ q_out, KvView kv, int layer) {
+  pdl_wait();
+  const int r = blockIdx.x;
+  const int half = hd / 2;
+  const int n_cols = (Hq + 2 * Hkv) * hd;
+  const float* pr = partial + (size_t)r * n_cols;
+  const int b = sv.row_seq[r];
+  const int slot = sv.P_step[b] + sv.row_local[r];
+  const int seq = sv.seq_ids[b];
+  const bool slot_ok = slot < kv.max_seq;
+  if (!slot_ok && threadIdx.x == 0) set_error(sv.err, SPEC_DEVERR_BOUNDS);
+  T* kbase = reinterpret_cast<T*>(kv.base) + layer * kv.layer_stride() + seq * kv.seq_stride() + (size_t)slot * hd;
+  T* vbase = kbase + kv.kv_stride();
+  const float2* cs = sv.rope_cs + (size_t)r * half;
+  const int pairs = (Hq + 2 * Hkv) * half;
+  for (int p = threadIdx.x; p < pairs; p += blockDim.x) {
+    const int h = p / half;
+    const int j = p - h * half;
+    const int c1 = h * hd + j;
+    const int c2 = c1 + half;
+    float v1 = 0.f, v2 = 0.f;
+    for (int sp = 0; sp < S; ++sp) {
+      v1 += pr[sp * split_stride + c1];
+      v2 += pr[sp * split_stride + c2];
+    }
+    if (h < Hq + Hkv) {
+      const float2 c = cs[j];
+      const float o1 = v1 * c.x - v2 * c.y;
+      const float o2 = v2 * c.x + v1 * c.y;
+      v1 = o1;
+      v2 = o2;
+    }
+    if (h < Hq) {
+      T* q = q_out + (size_t)r * Hq * hd;
+      q[c1] = from_f32<T>(v1);
+      q[c2] = from_f32<T>(v2);
+    } else if (slot_ok) {
+      const int kh = (h < Hq + Hkv) ? h - Hq : h - Hq - Hkv;
+      T* dst = ((h < Hq + Hkv) ? kbase : vbase) + kh * kv.head_stride();
+      dst[j] = from_f32<T>(v1);
+      dst[j + half] = from_f32<T>(v2);
+    }
+  }
+  pdl_launch_dependents();
+}
+
+cudaError_t launch_qkv_rope_store(int dtype, const StepView& sv, int S, const float* partial, size_t split_stride,
+                                  int Hq, int Hkv, int hd, void* q_out, const KvView& kv, int layer, cudaStream_t s,
+                                  bool pdl) {
+  cudaLaunchAttribute attr[1];
+  cudaLaunchConfig_t cfg = make_cfg(dim3(sv.M), dim3(256), 0, s, pdl, attr);
+  if (dtype == 0)
+    return cudaLaunchKernelEx(&cfg, qkv_rope_store_kernel<float>, sv, S, partial, split_stride, Hq, Hkv, hd,
+                              (float*)q_out, kv, layer);
+  return cudaLaunchKernelEx(&cfg, qkv_rope_store_kernel<__nv_bfloat16>, sv, S, partial, split_stride, Hq, Hkv, hd,
+                            (__nv_bfloat16*)q_out, kv, layer);
+}
+
+// ---------------------------------------------------------------------------
+// fp32 path: SwiGLU and a plain tiled SIMT GEMM (FFMA, no TF32)
+// ---------------------------------------------------------------------------
+__global__ void swiglu_f32_kernel(int M, int F, const float* __restrict__ gu, float* __restrict__ h) {
+  const size_t total = (size_t)M * F;
+  for (size_t i = blockIdx.x * (size_t)blockDim.x + threadIdx.x; i < total; i += (size_t)gridDim.x * blockDim.x) {
+    const size_t r = i / F, f = i - r * F;
+    const float g = gu[r * 2 * F + f];
+    const float u = gu[r * 2 * F + F + f];
+    h[i] = g / (1.0f + expf(-g)) * u;
+  }
+}
+
+cudaError_t launch_swiglu_f32(int M, int F, const float* gu, float* h, cudaStream_t s) {
+  const int blocks = (int)(((size_t)M * F + 255) / 256);
+  swiglu_f32_kernel<<<blocks < 4096 ? blocks : 4096, 256, 0, s>>>(M, F, gu, h);
+  return cudaGetLastError();
+}
+
+// C[t][o] = sum_k A[t][k] * W[o][k]; 16 tokens x 64 outputs per block, k ascending.
+__global__ void __launch_bounds__(256) gemm_simt_f32_kernel(const float* __restrict__ A, int lda,
+                                                            const float* __restrict__ W, int K,
+                                                            float* __restrict__ C, int ldc, int M, int N) {
+  __shared__ float sA[16][33];
+  __shared__ float sW[64][33];
+  const int t0 = blockIdx.y * 16, o0 = blockIdx.x * 64;
+  const int tx = threadIdx.x & 15;   // output column group
+  const int ty = threadIdx.x >> 4;   // token row
+  float acc[4] = {0.f, 0.f, 0.f, 0.f};
+  for (int k0 = 0; k0 < K; k0 += 32) {
+    for (int i = threadIdx.x; i < 16 * 32; i += 256) {
+      const int rr = i / 32, kk = i % 32;
+      const int t = t0 + rr, k = k0 + kk;
+      sA[rr][kk] = (t < M && k < K) ? A[(size_t)t * lda + k] : 0.f;
+    }
+    for (int i = threadIdx.x; i < 64 * 32; i += 256) {
+      const int rr = i / 32, kk = i % 32;
+      const int o = o0 + rr, k = k0 + kk;
+      sW[rr][kk] = (o < N && k < K) ? W[(size_t)o * K + k] : 0.f;
+    }
+    __syncthreads();
+#pragma unroll 8
+    for (int kk = 0; kk < 32; ++kk) {
+      const float a = sA[ty][kk];
+#pragma unroll
+      for (int j = 0; j < 4; ++j) acc[j] = fmaf(a, sW[tx + 16 * j][kk], acc[j]);
+    }
+    __syncthreads();
+  }
+  const int t = t0 + ty;
+  if (t < M) {
+#pragma unroll
+    for (int j = 0; j < 4; ++j) {
+      const int o = o0 + tx + 16 * j;
+      if (o < N) C[(size_t)t * ldc + o] = acc[j];
+    }
+  }
+}
+
+cudaError_t launch_gemm_simt_f32(const float* A, int lda, const float* W, int K, float* C, int ldc, int M, int N,
+                                 cudaStream_t s) {
+  dim3 grid((N + 63) / 64, (M + 15) / 16);
+  gemm_simt_f32_kernel<<<grid, 256, 0, s>>>(A, lda, W, K, C, ldc, M, N);
+  return cudaGetLastError();
+}
+
+// ---------------------------------------------------------------------------
+// LM-head reductions
+// ---------------------------------------------------------------------------
+// one warp per token: merge the per-tile (best, index, runner-up) in tile order
+__global__ void top2_reduce_kernel(int M, int tiles, const Top2* __restrict__ part, int top_ld,
+                                   int32_t* __restrict__ argmax, float* __restrict__ top1, float* __restrict__ top2) {
+  pdl_wait();
+  const int t = blockIdx.x * (blockDim.x >> 5) + (threadIdx.x >> 5);
+  const int lane = threadIdx.x & 31;
+  if (t >= M) return;
+  Top2 best;
+  best.v1 = -INFINITY; best.i1 = 0x7fffffff; best.v2 = -INFINITY;
+  for (int i = lane; i < tiles; i += 32) best = top2_merge(best, part[(size_t)i * top_ld + t]);
+  best = warp_top2(best);
+  if (lane == 0) {
+    argmax[t] = best.i1;
+    top1[t] = best.v1;
+    top2[t] = best.v2;
+  }
+  pdl_launch_dependents();
+}
+
+cudaError_t launch_top2_reduce(int M, int tiles, const Top2* part, int top_ld, int32_t* argmax, float* top1,
+                               float* top2, cudaStream_t s, bool pdl) {
+  cudaLaunchAttribute attr[1];
+  cudaLaunchConfig_t cfg = make_cfg(dim3((M + 7) / 8), dim3(256), 0, s, pdl, attr);
+  return cudaLaunchKernelEx(&cfg, top2_reduce_kernel, M, tiles, part, top_ld, argmax, top1, top2);
+}
+
+__global__ void rows_top2_f32_kernel(int M, int V, const float* __restrict__ logits, int32_t* __restrict__ argmax,
+                                     float* __restrict__ top1, float* __restrict__ top2) {
+  const int t = blockIdx.x * (blockDim.x >> 5) + (threadIdx.x >> 5);
+  const int lane = threadIdx.x & 31;
+  if (t >= M) return;
+  Top2 best;
+  best.v1 = -INFINITY; best.i1 = 0x7fffffff; best.v2 = -INFINITY;
+  for (int v = lane; v < V; v += 32) {
+    Top2 x;
+    x.v1 = logits[(size_t)t * V + v]; x.i1 = v; x.v2 = -INFINITY;
+    best = top2_merge(best, x);
+  }
+  best = warp_top2(best);
+  if (lane == 0) {
+    argmax[t] = best.i1;
+    top1[t] = best.v1;
+    top2[t] = best.v2;
+  }
+}
+
+cudaError_t launch_rows_top2_f32(int M, int V, const float* logits, int32_t* argmax, float* top1, float* top2,
+                                 cudaStream_t s) {
+  rows_top2_f32_kernel<<<(M + 7) / 8, 256, 0, s>>>(M, V, logits, argmax, top1, top2);
+  return cudaGetLastError();
+}
+
+}  // namespace spec

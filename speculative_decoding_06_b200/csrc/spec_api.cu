@@ -1,0 +1,973 @@
+// C ABI of the tree-verification library: argument validation, workspace
+// layout, TMA descriptors, the per-step kernel sequence and CUDA-graph replay.
+//
+// One verification step (all on the caller's stream):
+//   embed_meta      depth / position / ancestor bits per node, embedding, RMSNorm
+//   per layer:      QKV GEMM -> rotary + K/V store -> tree attention -> O GEMM ->
+//                   residual + RMSNorm -> gate/up GEMM + SwiGLU -> down GEMM ->
+//                   residual + RMSNorm
+//   LM head GEMM with a fused per-token argmax, then a small cross-tile reduction
+//   acceptance walk (one warp per tree) + sequence state update
+//   K/V compaction of the accepted path
+#include <cuda.h>
+#include <cuda_runtime.h>
+
+#include <algorithm>
+#include <cmath>
+#include <cstdarg>
+#include <cstdio>
+#include <cstring>
+#include <map>
+#include <string>
+#include <tuple>
+#include <vector>
+
+#include "../../include/spec.h"
+#include "common.cuh"
+#include "kernels.h"
+
+using namespace spec;
+
+namespace {
+
+constexpr int kMaxNodesLimit = 128;  // ancestor bitmask is two 64-bit words
+constexpr int kMaxSplits = 16;
+
+size_t align_up(size_t x, size_t a) { return (x + a - 1) / a * a; }
+int ceil_div(int a, int b) { return (a + b - 1) / b; }
+
+struct WsLayout {
+  size_t total = 0;
+  int Mmax = 0, Mpad = 0, splits_cap = 1, chunks_cap = 1;
+  // parameter block (one host->device copy per step)
+  size_t p_tokens, p_parents, p_node_off, p_seq_ids, p_err, p_end;
+  // per-row metadata
+  size_t row_seq, row_local, row_pos, row_anc, rope_cs, P_step;
+  // persistent state
+  size_t seq_len, pending, hist, err_sticky;
+  // activations
+  size_t x, xn, q, attn, hmlp, partial, part_o, part_lse, top_part, argmax, top1, top2, inv_freq;
+  size_t partial_bytes;
+  // outputs (one device->host copy per step)
+  size_t o_acc_len, o_acc_nodes, o_acc_tokens, o_bonus, o_end;
+};
+
+WsLayout make_layout(const spec_config& c) {
+  WsLayout L;
+  const size_t es = c.dtype == SPEC_DTYPE_BF16 ? 2 : 4;
+  L.Mmax = c.max_batch * c.max_nodes;
+  L.Mpad = (int)align_up(L.Mmax, 128);
+  L.splits_cap = L.Mpad <= 256 ? kMaxSplits : 2;
+  L.chunks_cap = std::max(2, std::min(32, 1184 / std::max(1, c.max_batch * c.n_kv_heads)));
+  const int qd = c.n_q_heads * c.head_dim;
+  const int nqkv = (c.n_q_heads + 2 * c.n_kv_heads) * c.head_dim;
+  size_t off = 0;
+  auto take = [&](size_t bytes) {
+    size_t o = off;
+    off = align_up(off + bytes, 256);
+    return o;
+  };
+  L.p_tokens = take(4 * (size_t)L.Mmax);
+  L.p_parents = take(4 * (size_t)L.Mmax);
+  L.p_node_off = take(4 * (size_t)(c.max_batch + 1));
+  L.p_seq_ids = take(4 * (size_t)c.max_batch);
+  L.p_err = take(16);
+  L.p_end = off;
+  L.row_seq = take(4 * (size_t)L.Mmax);
+  L.row_local = take(4 * (size_t)L.Mmax);
+  L.row_pos = take(4 * (size_t)L.Mmax);
+  L.row_anc = take(16 * (size_t)L.Mmax);
+  L.rope_cs = take(8 * (size_t)L.Mmax * (c.head_dim / 2));
+  L.P_step = take(4 * (size_t)c.max_batch);
+  L.seq_len = take(4 * (size_t)c.max_batch);
+  L.pending = take(4 * (size_t)c.max_batch);
+  L.hist = take(4 * (size_t)c.max_batch * c.max_seq);
+  L.err_sticky = take(16);
+  L.inv_freq = take(8 * (size_t)(c.head_dim / 2));
+  L.x = take(4 * (size_t)L.Mpad * c.hidden);
+  L.xn = take(es * (size_t)L.Mpad * c.hidden);
+  L.q = take(es * (size_t)L.Mpad * qd);
+  L.attn = take(es * (size_t)L.Mpad * qd);
+  L.hmlp = take(es * (size_t)L.Mpad * c.ffn);
+  size_t pcols = (size_t)std::max(nqkv, c.hidden) * (c.dtype == SPEC_DTYPE_BF16 ? L.splits_cap : 1);
+  if (c.dtype == SPEC_DTYPE_F32) pcols = std::max<size_t>(pcols, std::max<size_t>(2 * (size_t)c.ffn, c.vocab));
+  L.partial_bytes = 4 * (size_t)L.Mpad * pcols;
+  L.partial = take(L.partial_bytes);
+  L.part_o = take(4 * (size_t)L.Mmax * c.n_q_heads * L.chunks_cap * c.head_dim);
+  L.part_lse = take(4 * (size_t)L.Mmax * c.n_q_heads * L.chunks_cap);
+  L.top_part = take(sizeof(Top2) * (size_t)ceil_div(c.vocab, 128) * L.Mpad);
+  L.argmax = take(4 * (size_t)L.Mpad);
+  L.top1 = take(4 * (size_t)L.Mpad);
+  L.top2 = take(4 * (size_t)L.Mpad);
+  const size_t o0 = off;
+  L.o_acc_len = take(4 * (size_t)c.max_batch);
+  L.o_acc_nodes = take(4 * (size_t)c.max_batch * c.max_nodes);
+  L.o_acc_tokens = take(4 * (size_t)c.max_batch * c.max_nodes);
+  L.o_bonus = take(4 * (size_t)c.max_batch);
+  L.o_end = off;
+  (void)o0;
+  L.total = off;
+  return L;
+}
+
+size_t kv_bytes_of(const spec_config& c) {
+  const size_t es = c.dtype == SPEC_DTYPE_BF16 ? 2 : 4;
+  return (size_t)c.n_layers * 2 * c.max_batch * c.n_kv_heads * (size_t)c.max_seq * c.head_dim * es;
+}
+
+std::string check_config(const spec_config* c) {
+  if (!c) return "config is NULL";
+  if (c->n_layers < 1 || c->hidden < 1 || c->n_q_heads < 1 || c->n_kv_heads < 1 || c->head_dim < 2 || c->ffn < 1 ||
+      c->vocab < 2)
+    return "all model dimensions must be positive";
+  if (c->n_q_heads % c->n_kv_heads) return "n_q_heads must be a multiple of n_kv_heads";
+  if (c->dtype != SPEC_DTYPE_F32 && c->dtype != SPEC_DTYPE_BF16) return "dtype must be SPEC_DTYPE_F32 or SPEC_DTYPE_BF16";
+  if (c->max_batch < 1 || c->max_seq < 2 || c->max_nodes < 1) return "max_batch, max_seq, max_nodes must be positive";
+  if (c->max_nodes > kMaxNodesLimit) return "max_nodes must be <= 128";
+  if (c->max_nodes > c->max_seq) return "max_nodes must be <= max_seq";
+  if (!(c->rms_eps > 0.f) || !(c->rope_theta > 1.f)) return "rms_eps must be > 0 and rope_theta > 1";
+  if (c->dtype == SPEC_DTYPE_BF16) {
+    if (c->head_dim != 128) return "bf16 models need head_dim == 128";
+    if (c->hidden % 128) return "bf16 models need hidden % 128 == 0";
+    if (c->ffn % 64) return "bf16 models need ffn % 64 == 0";
+  } else {
+    if (c->head_dim > 128 || c->head_dim % 2) return "fp32 models need an even head_dim <= 128";
+    if (c->hidden % 4) return "fp32 models need hidden % 4 == 0";
+  }
+  if (c->draft_head && c->dtype != SPEC_DTYPE_BF16) return "the draft head is bf16 only";
+  return "";
+}
+
+typedef CUresult (*EncodeTiledFn)(CUtensorMap*, CUtensorMapDataType, cuuint32_t, void*, const cuuint64_t*,
+                                  const cuuint64_t*, const cuuint32_t*, const cuuint32_t*, CUtensorMapInterleave,
+                                  CUtensorMapSwizzle, CUtensorMapL2promotion, CUtensorMapFloatOOBfill);
+
+EncodeTiledFn get_encode_fn() {
+  static EncodeTiledFn fn = nullptr;
+  if (!fn) {
+    void* p = nullptr;
+    cudaDriverEntryPointQueryResult q;
+    if (cudaGetDriverEntryPointByVersion("cuTensorMapEncodeTiled", &p, 12000, cudaEnableDefault, &q) == cudaSuccess &&
+        q == cudaDriverEntryPointSuccess)
+      fn = reinterpret_cast<EncodeTiledFn>(p);
+  }
+  return fn;
+}
+
+// [rows][cols] bf16, row-major; boxes of 64 columns x box_rows rows, 128-byte swizzle
+bool make_tmap(CUtensorMap* m, const void* ptr, uint64_t rows, uint64_t cols, uint32_t box_rows) {
+  EncodeTiledFn enc = get_encode_fn();
+  if (!enc) return false;
+  cuuint64_t dims[2] = {cols, rows};
+  cuuint64_t strides[1] = {cols * 2};
+  cuuint32_t box[2] = {64, box_rows};
+  cuuint32_t estr[2] = {1, 1};
+  return enc(m, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, const_cast<void*>(ptr), dims, strides, box, estr,
+             CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
+             CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
+}
+
+struct LayerMaps {
+  CUtensorMap wq, wk, wv, wo, wg, wu, wd;
+};
+
+struct GemmPlan {
+  int bn, tiles_o, tiles_t, splits, kbps, grid;
+};
+
+struct StepPlan {
+  int B, M, max_n, max_lk, n_chunks, chunk, max_rows;
+  GemmPlan qkv, o, gu, down, lm;
+};
+
+using GraphKey = std::tuple<int, int, int, int, int, int, int, int>;
+
+}  // namespace
+
+struct spec_handle {
+  spec_config cfg{};
+  WsLayout lay;
+  int device = 0;
+  int sm_count = 148;
+  cudaStream_t stream = nullptr;
+  const void* embed = nullptr;
+  const void* final_norm = nullptr;
+  const void* lm_head = nullptr;
+  std::vector<spec_layer_weights> layers;
+  KvView kv{};
+  uint8_t* ws = nullptr;
+  std::vector<LayerMaps> maps;
+  CUtensorMap map_lm;
+  CUtensorMap map_xn[2], map_attn[2], map_h[2];  // B operands for BN = 64, 128
+  int resident[2][3] = {{0, 0, 0}, {0, 0, 0}};   // co-resident CTAs per SM [bn][epi]
+  // host mirror of per-sequence state
+  std::vector<int32_t> len, pending;
+  std::vector<int32_t> len_hi;  // upper bound while device-output steps are in flight
+  std::vector<uint8_t> ready;   // prefilled
+  bool stale = false;
+  // pinned staging
+  uint8_t* h_params = nullptr;
+  uint8_t* h_out = nullptr;
+  float* dbg_logits = nullptr;
+  size_t dbg_bytes = 0;
+  std::map<GraphKey, cudaGraphExec_t> graphs;
+  bool use_pdl = true;
+  std::string err;
+  // profiler: an event pair per launch
+  bool prof = false;
+  std::vector<cudaEvent_t> ev_pool;
+  std::vector<std::pair<int, int>> prof_marks;  // (class, index of first event of the pair)
+  int launches = 0;
+
+  template <typename T>
+  T* W(size_t off) const { return reinterpret_cast<T*>(ws + off); }
+};
+
+namespace {
+
+int fail(spec_handle* h, int code, const char* fmt, ...) {
+  char buf[512];
+  va_list ap;
+  va_start(ap, fmt);
+  vsnprintf(buf, sizeof(buf), fmt, ap);
+  va_end(ap);
+  if (h) h->err = buf;
+  return code;
+}
+
+#define CUDA_TRY(h, call)                                                                      \
+  do {                                                                                         \
+    cudaError_t e__ = (call);                                                                  \
+    if (e__ != cudaSuccess)                                                                    \
+      return fail(h, SPEC_ERR_CUDA, "%s failed: %s (%s)", #call, cudaGetErrorName(e__),        \
+                  cudaGetErrorString(e__));                                                    \
+  } while (0)
+
+// Launch wrapper: counts launches and, when profiling, brackets each one with events.
+template <typename F>
+cudaError_t launch_k(spec_handle* h, int cls, int n_kernels, F&& fn) {
+  int i0 = -1;
+  if (h->prof) {
+    i0 = (int)(2 * h->prof_marks.size());
+    while ((int)h->ev_pool.size() < i0 + 2) {
+      cudaEvent_t e;
+      cudaError_t r = cudaEventCreate(&e);
+      if (r != cudaSuccess) return r;
+      h->ev_pool.push_back(e);
+    }
+    cudaError_t r = cudaEventRecord(h->ev_pool[i0], h->stream);
+    if (r != cudaSuccess) return r;
+  }
+  cudaError_t e = fn();
+  if (e != cudaSuccess) return e;
+  h->launches += n_kernels;
+  if (h->prof) {
+    cudaError_t r = cudaEventRecord(h->ev_pool[i0 + 1], h->stream);
+    if (r != cudaSuccess) return r;
+    h->prof_marks.emplace_back(cls, i0);
+  }
+  return cudaSuccess;
+}
+
+GemmPlan plan_gemm(const spec_handle* h, int rows_per_tile, int n_out, int K, int M, int epi) {
+  GemmPlan p;
+  p.bn = M <= 64 ? 64 : 128;
+  const int bi = p.bn == 64 ? 0 : 1;
+  const int resident = std::max(1, h->resident[bi][epi]) * h->sm_count;
+  p.tiles_o = ceil_div(n_out, rows_per_tile);
+  p.tiles_t = ceil_div(M, p.bn);
+  const int KB = K / 64;
+  const int base = p.tiles_o * p.tiles_t;
+  int S = 1;
+  if (epi == GEMM_EPI_PARTIAL) {
+    const int cap = std::min(h->lay.splits_cap, std::max(1, KB / 4));
+    S = std::max(1, std::min(cap, resident / std::max(1, base)));
+  }
+  p.kbps = ceil_div(KB, S);
+  p.splits = ceil_div(KB, p.kbps);  // no empty split
+  p.grid = std::min(base * p.splits, resident);
+  return p;
+}
+
+StepPlan make_plan(const spec_handle* h, int B, int M, int max_n, int max_lk) {
+  const spec_config& c = h->cfg;
+  StepPlan s;
+  s.B = B;
+  s.M = M;
+  s.max_n = max_n;
+  s.max_lk = max_lk;
+  const int G = c.n_q_heads / c.n_kv_heads;
+  s.max_rows = max_n * G;
+  const int rowblocks = ceil_div(s.max_rows, 64);
+  const int ctas_per_chunk = B * c.n_kv_heads * rowblocks;
+  int want = std::max(1, ceil_div(2 * h->sm_count, ctas_per_chunk));
+  want = std::min(want, h->lay.chunks_cap);
+  int chunk = std::max(256, (int)align_up(ceil_div(max_lk, want), 64));
+  chunk = std::max(chunk, (int)align_up(ceil_div(max_lk, h->lay.chunks_cap), 64));
+  s.chunk = chunk;
+  s.n_chunks = ceil_div(max_lk, chunk);
+  const int nqkv = (c.n_q_heads + 2 * c.n_kv_heads) * c.head_dim;
+  const int qd = c.n_q_heads * c.head_dim;
+  s.qkv = plan_gemm(h, 128, nqkv, c.hidden, M, GEMM_EPI_PARTIAL);
+  s.o = plan_gemm(h, 128, c.hidden, qd, M, GEMM_EPI_PARTIAL);
+  s.gu = plan_gemm(h, 64, c.ffn, c.hidden, M, GEMM_EPI_SWIGLU);
+  s.down = plan_gemm(h, 128, c.hidden, c.ffn, M, GEMM_EPI_PARTIAL);
+  s.lm = plan_gemm(h, 128, c.vocab, c.hidden, M, GEMM_EPI_ARGMAX);
+  return s;
+}
+
+StepView make_view(spec_handle* h, int B, int M) {
+  const WsLayout& L = h->lay;
+  StepView v;
+  v.tokens = h->W<int32_t>(L.p_tokens);
+  v.parents = h->W<int32_t>(L.p_parents);
+  v.node_off = h->W<int32_t>(L.p_node_off);
+  v.seq_ids = h->W<int32_t>(L.p_seq_ids);
+  v.B = B;
+  v.M = M;
+  v.row_seq = h->W<int32_t>(L.row_seq);
+  v.row_local = h->W<int32_t>(L.row_local);
+  v.row_pos = h->W<int32_t>(L.row_pos);
+  v.row_anc = h->W<uint64_t>(L.row_anc);
+  v.rope_cs = h->W<float2>(L.rope_cs);
+  v.P_step = h->W<int32_t>(L.P_step);
+  v.seq_len = h->W<int32_t>(L.seq_len);
+  v.pending = h->W<int32_t>(L.pending);
+  v.hist = h->W<int32_t>(L.hist);
+  v.max_seq = h->cfg.max_seq;
+  v.err = h->W<uint32_t>(L.p_err);
+  v.err_sticky = h->W<uint32_t>(L.err_sticky);
+  return v;
+}
+
+GemmTcLaunch gemm_launch(const GemmPlan& p, int epi, int n_out, int K, int M, const CUtensorMap* a0,
+                         const CUtensorMap* a1, const CUtensorMap* a2, const CUtensorMap* b, int s0, int s1, int s2,
+                         uint32_t* err) {
+  GemmTcLaunch L{};
+  L.bn = p.bn;
+  L.epi = epi;
+  L.grid = p.grid;
+  L.mA0 = a0;
+  L.mA1 = a1 ? a1 : a0;
+  L.mA2 = a2 ? a2 : a0;
+  L.mB = b;
+  L.args.n_out = n_out;
+  L.args.K = K;
+  L.args.M = M;
+  L.args.tiles_o = p.tiles_o;
+  L.args.tiles_t = p.tiles_t;
+  L.args.splits = p.splits;
+  L.args.kb_per_split = p.kbps;
+  L.args.seg_rows[0] = s0;
+  L.args.seg_rows[1] = s1;
+  L.args.seg_rows[2] = s2;
+  L.args.err = err;
+  return L;
+}
+
+// Enqueue the whole step (everything after the parameter upload).
+#define LK(cls, nk, expr)                                                             \
+  do {                                                                                \
+    cudaError_t e_ = launch_k(h, cls, nk, [&]() { return (expr); });                  \
+    if (e_ != cudaSuccess) return e_;                                                 \
+  } while (0)
+
+cudaError_t enqueue_step(spec_handle* h, const StepPlan& sp, int mode, bool dbg) {
+  const spec_config& c = h->cfg;
+  const WsLayout& L = h->lay;
+  cudaStream_t st = h->stream;
+  const bool pdl = h->use_pdl && !h->prof;
+  StepView sv = make_view(h, sp.B, sp.M);
+  const int dt = c.dtype == SPEC_DTYPE_BF16 ? 1 : 0;
+  const int d = c.hidden, qd = c.n_q_heads * c.head_dim, kvd = c.n_kv_heads * c.head_dim;
+  const int nqkv = qd + 2 * kvd;
+  const int M = sp.M;
+  float* x = h->W<float>(L.x);
+  void* xn = h->ws + L.xn;
+  void* q = h->ws + L.q;
+  void* attn = h->ws + L.attn;
+  void* hm = h->ws + L.hmlp;
+  float* part = h->W<float>(L.partial);
+  h->launches = 0;
+
+  LK(SPEC_PROF_EMBED_META, 1,
+     launch_embed_meta(dt, sv, h->embed, h->layers[0].attn_norm, d, c.rms_eps, x, xn, h->W<double>(L.inv_freq),
+                       c.head_dim / 2, mode, st, pdl));
+
+  AttnArgs aa{};
+  aa.sv = sv;
+  aa.kv = h->kv;
+  aa.Hq = c.n_q_heads;
+  aa.hd = c.head_dim;
+  aa.q = q;
+  aa.out = attn;
+  aa.part_o = h->W<float>(L.part_o);
+  aa.part_lse = h->W<float>(L.part_lse);
+  aa.n_chunks = sp.n_chunks;
+  aa.chunk = sp.chunk;
+  aa.max_rows = sp.max_rows;
+
+  for (int l = 0; l < c.n_layers; ++l) {
+    const spec_layer_weights& lw = h->layers[l];
+    const void* next_norm = (l + 1 < c.n_layers) ? h->layers[l + 1].attn_norm : h->final_norm;
+    aa.layer = l;
+    if (dt == 1) {
+      const LayerMaps& mp = h->maps[l];
+      const int bi = sp.qkv.bn == 64 ? 0 : 1;
+      GemmTcLaunch g = gemm_launch(sp.qkv, GEMM_EPI_PARTIAL, nqkv, d, M, &mp.wq, &mp.wk, &mp.wv, &h->map_xn[bi], qd,
+                                   kvd, kvd, sv.err);
+      g.args.out_f32 = part;
+      g.args.split_stride = (size_t)L.Mpad * nqkv;
+      LK(SPEC_PROF_GEMM_QKV, 1, gemm_tc_launch(g, st, pdl));
+      LK(SPEC_PROF_ROPE_KV, 1,
+         launch_qkv_rope_store(dt, sv, sp.qkv.splits, part, (size_t)L.Mpad * nqkv, c.n_q_heads, c.n_kv_heads,
+                               c.head_dim, q, h->kv, l, st, pdl));
+      LK(SPEC_PROF_ATTENTION, 2, launch_attention(dt, aa, st, pdl));
+      GemmTcLaunch go = gemm_launch(sp.o, GEMM_EPI_PARTIAL, d, qd, M, &mp.wo, nullptr, nullptr, &h->map_attn[bi], d,
+                                    0, 0, sv.err);
+      go.args.out_f32 = part;
+      go.args.split_stride = (size_t)L.Mpad * d;
+      LK(SPEC_PROF_GEMM_O, 1, gemm_tc_launch(go, st, pdl));
+      LK(SPEC_PROF_RESID_NORM, 1,
+         launch_residual_norm(dt, M, d, sp.o.splits, part, (size_t)L.Mpad * d, x, xn, lw.mlp_norm, c.rms_eps, st,
+                              pdl));
+      GemmTcLaunch gg = gemm_launch(sp.gu, GEMM_EPI_SWIGLU, c.ffn, d, M, &mp.wg, &mp.wu, nullptr, &h->map_xn[bi], 0,
+                                    0, 0, sv.err);
+      gg.args.out_bf16 = reinterpret_cast<__nv_bfloat16*>(hm);
+      gg.args.ld_out = c.ffn;
+      LK(SPEC_PROF_GEMM_GATE_UP, 1, gemm_tc_launch(gg, st, pdl));
+      GemmTcLaunch gd = gemm_launch(sp.down, GEMM_EPI_PARTIAL, d, c.ffn, M, &mp.wd, nullptr, nullptr, &h->map_h[bi],
+                                    d, 0, 0, sv.err);
+      gd.args.out_f32 = part;
+      gd.args.split_stride = (size_t)L.Mpad * d;
+      LK(SPEC_PROF_GEMM_DOWN, 1, gemm_tc_launch(gd, st, pdl));
+      LK(SPEC_PROF_RESID_NORM, 1,
+         launch_residual_norm(dt, M, d, sp.down.splits, part, (size_t)L.Mpad * d, x, xn, next_norm, c.rms_eps, st,
+                              pdl));
+    } else {
+      const float* xf = reinterpret_cast<const float*>(xn);
+      LK(SPEC_PROF_GEMM_QKV, 1, launch_gemm_simt_f32(xf, d, (const float*)lw.wq, d, part, nqkv, M, qd, st));
+      LK(SPEC_PROF_GEMM_QKV, 1, launch_gemm_simt_f32(xf, d, (const float*)lw.wk, d, part + qd, nqkv, M, kvd, st));
+      LK(SPEC_PROF_GEMM_QKV, 1,
+         launch_gemm_simt_f32(xf, d, (const float*)lw.wv, d, part + qd + kvd, nqkv, M, kvd, st));
+      LK(SPEC_PROF_ROPE_KV, 1,
+         launch_qkv_rope_store(dt, sv, 1, part, 0, c.n_q_heads, c.n_kv_heads, c.head_dim, q, h->kv, l, st, false));
+      LK(SPEC_PROF_ATTENTION, 1, launch_attention(dt, aa, st, false));
+      LK(SPEC_PROF_GEMM_O, 1, launch_gemm_simt_f32((const float*)attn, qd, (const float*)lw.wo, qd, part, d, M, d, st));
+      LK(SPEC_PROF_RESID_NORM, 1, launch_residual_norm(dt, M, d, 1, part, 0, x, xn, lw.mlp_norm, c.rms_eps, st, false));
+      LK(SPEC_PROF_GEMM_GATE_UP, 1,
+         launch_gemm_simt_f32(xf, d, (const float*)lw.w_gate, d, part, 2 * c.ffn, M, c.ffn, st));
+      LK(SPEC_PROF_GEMM_GATE_UP, 1,
+         launch_gemm_simt_f32(xf, d, (const float*)lw.w_up, d, part + c.ffn, 2 * c.ffn, M, c.ffn, st));
+      LK(SPEC_PROF_GEMM_GATE_UP, 1, launch_swiglu_f32(M, c.ffn, part, (float*)hm, st));
+      LK(SPEC_PROF_GEMM_DOWN, 1,
+         launch_gemm_simt_f32((const float*)hm, c.ffn, (const float*)lw.w_down, c.ffn, part, d, M, d, st));
+      LK(SPEC_PROF_RESID_NORM, 1, launch_residual_norm(dt, M, d, 1, part, 0, x, xn, next_norm, c.rms_eps, st, false));
+    }
+  }
+
+  int32_t* amax = h->W<int32_t>(L.argmax);
+  if (dt == 1) {
+    const int bi = sp.lm.bn == 64 ? 0 : 1;
+    GemmTcLaunch g = gemm_launch(sp.lm, GEMM_EPI_ARGMAX, c.vocab, d, M, &h->map_lm, nullptr, nullptr, &h->map_xn[bi],
+                                 c.vocab, 0, 0, sv.err);
+    g.args.top_part = h->W<Top2>(L.top_part);
+    g.args.top_ld = L.Mpad;
+    g.args.dbg_logits = dbg ? h->dbg_logits : nullptr;
+    LK(SPEC_PROF_LM_HEAD, 1, gemm_tc_launch(g, st, pdl));
+    LK(SPEC_PROF_LM_REDUCE, 1,
+       launch_top2_reduce(M, sp.lm.tiles_o, h->W<Top2>(L.top_part), L.Mpad, amax, h->W<float>(L.top1),
+                          h->W<float>(L.top2), st, pdl));
+  } else {
+    LK(SPEC_PROF_LM_HEAD, 1,
+       launch_gemm_simt_f32((const float*)xn, d, (const float*)h->lm_head, d, part, c.vocab, M, c.vocab, st));
+    LK(SPEC_PROF_LM_REDUCE, 1, launch_rows_top2_f32(M, c.vocab, part, amax, h->W<float>(L.top1), h->W<float>(L.top2), st));
+    if (dbg && h->dbg_logits) {
+      cudaError_t e = cudaMemcpyAsync(h->dbg_logits, part, sizeof(float) * (size_t)M * c.vocab,
+                                      cudaMemcpyDeviceToDevice, st);
+      if (e != cudaSuccess) return e;
+    }
+  }
+
+  WalkArgs w{};
+  w.sv = sv;
+  w.argmax = amax;
+  w.acc_len = h->W<int32_t>(L.o_acc_len);
+  w.acc_nodes = h->W<int32_t>(L.o_acc_nodes);
+  w.acc_tokens = h->W<int32_t>(L.o_acc_tokens);
+  w.bonus = h->W<int32_t>(L.o_bonus);
+  w.max_nodes = c.max_nodes;
+  w.mode = mode;
+  LK(SPEC_PROF_WALK, 1, launch_accept_walk(w, st, pdl && dt == 1));
+  if (mode == STEP_VERIFY)
+    LK(SPEC_PROF_COMPACT, 1,
+       launch_kv_compact(sv, h->kv, c.n_layers, w.acc_len, w.acc_nodes, c.max_nodes, st, pdl && dt == 1));
+  return cudaSuccess;
+}
+
+// Validate a batch of trees on the host (before anything is queued).
+int validate_batch(spec_handle* h, int B, const int32_t* seq_ids, const int32_t* tokens, const int32_t* parents,
+                   const int32_t* node_off, int mode, int* M_out, int* max_n_out, int* max_lk_out) {
+  const spec_config& c = h->cfg;
+  if (B < 1 || B > c.max_batch) return fail(h, SPEC_ERR_CAPACITY, "batch %d outside [1, %d]", B, c.max_batch);
+  if (!seq_ids || !tokens || !parents || !node_off) return fail(h, SPEC_ERR_ARG, "null input pointer");
+  if (node_off[0] != 0) return fail(h, SPEC_ERR_ARG, "node_offsets[0] must be 0");
+  std::vector<uint8_t> seen(c.max_batch, 0);
+  int max_n = 0, max_lk = 0;
+  for (int b = 0; b < B; ++b) {
+    const int s = seq_ids[b];
+    if (s < 0 || s >= c.max_batch) return fail(h, SPEC_ERR_ARG, "seq id %d outside [0, %d)", s, c.max_batch);
+    if (seen[s]) return fail(h, SPEC_ERR_ARG, "seq id %d appears twice in one batch", s);
+    seen[s] = 1;
+    const int n = node_off[b + 1] - node_off[b];
+    if (n < 1) return fail(h, SPEC_ERR_ARG, "tree %d is empty", b);
+    if (n > c.max_nodes) return fail(h, SPEC_ERR_CAPACITY, "tree %d has %d nodes > max_nodes %d", b, n, c.max_nodes);
+    if (mode != STEP_PREFILL && !h->ready[s]) return fail(h, SPEC_ERR_STATE, "sequence %d has not been prefilled", s);
+    const int P = h->stale ? h->len_hi[s] : h->len[s];
+    if (P + n > c.max_seq)
+      return fail(h, SPEC_ERR_CAPACITY, "sequence %d: length %d + %d nodes exceeds max_seq %d", s, P, n, c.max_seq);
+    const int32_t* tk = tokens + node_off[b];
+    const int32_t* pr = parents + node_off[b];
+    const int vr = spec_validate_tree(tk, pr, n, c.vocab, c.max_nodes);
+    if (vr == SPEC_ERR_TREE) return fail(h, vr, "tree %d: parents[0] must be -1 and 0 <= parents[i] < i", b);
+    if (vr == SPEC_ERR_TOKEN) return fail(h, vr, "tree %d: a token is outside [0, %d)", b, c.vocab);
+    if (vr) return fail(h, vr, "tree %d rejected", b);
+    if (mode == STEP_VERIFY && !h->stale && tk[0] != h->pending[s])
+      return fail(h, SPEC_ERR_ROOT, "sequence %d: tokens[0] = %d is not the pending token %d", s, tk[0], h->pending[s]);
+    max_n = std::max(max_n, n);
+    max_lk = std::max(max_lk, P + n);
+  }
+  *M_out = node_off[B];
+  *max_n_out = max_n;
+  *max_lk_out = max_lk;
+  return SPEC_OK;
+}
+
+// Upload parameters and run one step; with `sync`, wait and read the outputs.
+int run_step(spec_handle* h, int B, const int32_t* seq_ids, const int32_t* tokens, const int32_t* parents,
+             const int32_t* node_off, int mode, int flags, bool sync) {
+  int M = 0, max_n = 0, max_lk = 0;
+  int rc = validate_batch(h, B, seq_ids, tokens, parents, node_off, mode, &M, &max_n, &max_lk);
+  if (rc) return rc;
+  const WsLayout& L = h->lay;
+  const bool dbg = (flags & SPEC_DEBUG_LOGITS) != 0;
+  if (dbg && (!h->dbg_logits || h->dbg_bytes < sizeof(float) * (size_t)M * h->cfg.vocab))
+    return fail(h, SPEC_ERR_CAPACITY, "SPEC_DEBUG_LOGITS needs a debug buffer of %zu bytes",
+                sizeof(float) * (size_t)M * h->cfg.vocab);
+  // pack the parameter block
+  uint8_t* pb = h->h_params;
+  std::memcpy(pb + L.p_tokens, tokens, 4 * (size_t)M);
+  std::memcpy(pb + L.p_parents, parents, 4 * (size_t)M);
+  std::memcpy(pb + L.p_node_off, node_off, 4 * (size_t)(B + 1));
+  std::memcpy(pb + L.p_seq_ids, seq_ids, 4 * (size_t)B);
+  std::memset(pb + L.p_err, 0, 16);
+  CUDA_TRY(h, cudaMemcpyAsync(h->ws, pb, L.p_end, cudaMemcpyHostToDevice, h->stream));
+
+  StepPlan sp = make_plan(h, B, M, max_n, max_lk);
+  const bool graph = !(flags & SPEC_NO_GRAPH) && !h->prof;
+  if (graph) {
+    GraphKey key{mode, B, M, max_n, sp.n_chunks, sp.chunk, dbg ? 1 : 0, h->use_pdl ? 1 : 0};
+    auto it = h->graphs.find(key);
+    if (it == h->graphs.end()) {
+      cudaGraph_t g = nullptr;
+      CUDA_TRY(h, cudaStreamBeginCapture(h->stream, cudaStreamCaptureModeThreadLocal));
+      cudaError_t e = enqueue_step(h, sp, mode, dbg);
+      cudaError_t e2 = cudaStreamEndCapture(h->stream, &g);
+      if (e != cudaSuccess || e2 != cudaSuccess) {
+        if (g) cudaGraphDestroy(g);
+        return fail(h, SPEC_ERR_CUDA, "graph capture failed: %s", cudaGetErrorString(e != cudaSuccess ? e : e2));
+      }
+      cudaGraphExec_t ex = nullptr;
+      e = cudaGraphInstantiate(&ex, g, 0);
+      cudaGraphDestroy(g);
+      if (e != cudaSuccess) return fail(h, SPEC_ERR_CUDA, "graph instantiate failed: %s", cudaGetErrorString(e));
+      it = h->graphs.emplace(key, ex).first;
+    }
+    CUDA_TRY(h, cudaGraphLaunch(it->second, h->stream));
+  } else {
+    cudaError_t e = enqueue_step(h, sp, mode, dbg);
+    if (e != cudaSuccess) return fail(h, SPEC_ERR_CUDA, "kernel launch failed: %s", cudaGetErrorString(e));
+  }
+
+  if (!sync) {
+    // device-output step: lengths are known only as upper bounds until spec_sync
+    for (int b = 0; b < B; ++b) {
+      const int s = seq_ids[b];
+      const int n = node_off[b + 1] - node_off[b];
+      const int base = h->stale ? h->len_hi[s] : h->len[s];
+      if (mode == STEP_VERIFY) h->len_hi[s] = base + n;
+      else if (mode == STEP_PREFILL) h->len_hi[s] = base + n;
+      else h->len_hi[s] = base;
+    }
+    if (mode != STEP_SCORE) h->stale = true;
+    return SPEC_OK;
+  }
+  CUDA_TRY(h, cudaMemcpyAsync(h->h_out, h->ws + L.o_acc_len, L.o_end - L.o_acc_len, cudaMemcpyDeviceToHost, h->stream));
+  uint32_t errw[2] = {0, 0};
+  CUDA_TRY(h, cudaMemcpyAsync(errw, h->ws + L.p_err, 4, cudaMemcpyDeviceToHost, h->stream));
+  CUDA_TRY(h, cudaStreamSynchronize(h->stream));
+  if (errw[0] & SPEC_DEVERR_TIMEOUT) return fail(h, SPEC_ERR_TIMEOUT, "a bounded wait expired on the device");
+  if (errw[0] & SPEC_DEVERR_ROOT) return fail(h, SPEC_ERR_ROOT, "tokens[0] is not the pending token (device check)");
+  if (errw[0]) return fail(h, SPEC_ERR_CUDA, "device reported error bits 0x%x", errw[0]);
+  // mirror the state update done on the device
+  if (mode != STEP_SCORE) {
+    const int32_t* acc_len = reinterpret_cast<const int32_t*>(h->h_out);
+    const int32_t* bonus = reinterpret_cast<const int32_t*>(h->h_out + (L.o_bonus - L.o_acc_len));
+    for (int b = 0; b < B; ++b) {
+      const int s = seq_ids[b];
+      h->len[s] += 1 + acc_len[b];
+      h->len_hi[s] = h->len[s];
+      h->pending[s] = bonus[b];
+    }
+  }
+  return SPEC_OK;
+}
+
+int refresh_state(spec_handle* h) {
+  const WsLayout& L = h->lay;
+  const int nb = h->cfg.max_batch;
+  std::vector<int32_t> buf(2 * (size_t)nb);
+  uint32_t sticky = 0;
+  CUDA_TRY(h, cudaMemcpyAsync(buf.data(), h->ws + L.seq_len, 4 * (size_t)nb, cudaMemcpyDeviceToHost, h->stream));
+  CUDA_TRY(h, cudaMemcpyAsync(buf.data() + nb, h->ws + L.pending, 4 * (size_t)nb, cudaMemcpyDeviceToHost, h->stream));
+  CUDA_TRY(h, cudaMemcpyAsync(&sticky, h->ws + L.err_sticky, 4, cudaMemcpyDeviceToHost, h->stream));
+  CUDA_TRY(h, cudaMemsetAsync(h->ws + L.err_sticky, 0, 4, h->stream));
+  CUDA_TRY(h, cudaStreamSynchronize(h->stream));
+  for (int s = 0; s < nb; ++s) {
+    h->len[s] = buf[s];
+    h->len_hi[s] = buf[s];
+    h->pending[s] = buf[nb + s];
+  }
+  h->stale = false;
+  if (sticky & SPEC_DEVERR_TIMEOUT) return fail(h, SPEC_ERR_TIMEOUT, "a bounded wait expired on the device");
+  if (sticky & SPEC_DEVERR_ROOT) return fail(h, SPEC_ERR_ROOT, "a queued step had tokens[0] != pending token");
+  if (sticky) return fail(h, SPEC_ERR_CUDA, "device reported error bits 0x%x", sticky);
+  return SPEC_OK;
+}
+
+bool aligned16(const void* p) { return (reinterpret_cast<uintptr_t>(p) & 15u) == 0; }
+
+}  // namespace
+
+// ===========================================================================
+// C ABI
+// ===========================================================================
+extern "C" {
+
+int spec_validate_tree(const int32_t* tokens, const int32_t* parents, int n, int vocab, int max_nodes) {
+  if (!tokens || !parents) return SPEC_ERR_ARG;
+  if (n < 1 || n > max_nodes || max_nodes > kMaxNodesLimit) return SPEC_ERR_CAPACITY;
+  if (parents[0] != -1) return SPEC_ERR_TREE;
+  for (int i = 1; i < n; ++i)
+    if (parents[i] < 0 || parents[i] >= i) return SPEC_ERR_TREE;
+  for (int i = 0; i < n; ++i)
+    if (tokens[i] < 0 || tokens[i] >= vocab) return SPEC_ERR_TOKEN;
+  return SPEC_OK;
+}
+
+size_t spec_kv_bytes(const spec_config* cfg) {
+  if (!check_config(cfg).empty()) return 0;
+  return kv_bytes_of(*cfg);
+}
+
+size_t spec_workspace_bytes(const spec_config* cfg) {
+  if (!check_config(cfg).empty()) return 0;
+  return make_layout(*cfg).total;
+}
+
+int spec_init(const spec_config* cfg, const spec_weights* w, void* kv_cache, size_t kv_bytes, void* workspace,
+              size_t ws_bytes, void* cuda_stream, spec_handle** out) {
+  if (!out) return SPEC_ERR_ARG;
+  *out = nullptr;
+  std::string why = check_config(cfg);
+  static std::string init_err;
+  if (!why.empty()) return SPEC_ERR_ARG;
+  if (!w || !w->embed || !w->final_norm || !w->lm_head || !w->layers || !kv_cache || !workspace) return SPEC_ERR_ARG;
+  const spec_config& c = *cfg;
+  if (kv_bytes < kv_bytes_of(c)) return SPEC_ERR_CAPACITY;
+  WsLayout lay = make_layout(c);
+  if (ws_bytes < lay.total) return SPEC_ERR_CAPACITY;
+  if (!aligned16(kv_cache) || !aligned16(workspace) || !aligned16(w->embed) || !aligned16(w->lm_head) ||
+      !aligned16(w->final_norm))
+    return SPEC_ERR_ARG;
+  for (int l = 0; l < c.n_layers; ++l) {
+    const spec_layer_weights& lw = w->layers[l];
+    const void* ps[9] = {lw.wq, lw.wk, lw.wv, lw.wo, lw.w_gate, lw.w_up, lw.w_down, lw.attn_norm, lw.mlp_norm};
+    for (const void* p : ps)
+      if (!p || !aligned16(p)) return SPEC_ERR_ARG;
+  }
+
+  spec_handle* h = new spec_handle();
+  h->cfg = c;
+  h->lay = lay;
+  h->stream = reinterpret_cast<cudaStream_t>(cuda_stream);
+  h->embed = w->embed;
+  h->final_norm = w->final_norm;
+  h->lm_head = w->lm_head;
+  h->layers.assign(w->layers, w->layers + c.n_layers);
+  h->ws = reinterpret_cast<uint8_t*>(workspace);
+  h->kv.base = kv_cache;
+  h->kv.max_batch = c.max_batch;
+  h->kv.Hkv = c.n_kv_heads;
+  h->kv.max_seq = c.max_seq;
+  h->kv.hd = c.head_dim;
+  h->kv.elem = c.dtype == SPEC_DTYPE_BF16 ? 2 : 4;
+  h->len.assign(c.max_batch, 0);
+  h->pending.assign(c.max_batch, -1);
+  h->len_hi.assign(c.max_batch, 0);
+  h->ready.assign(c.max_batch, 0);
+
+  auto bail = [&](int code, const char* msg) {
+    spec_free(h);
+    (void)msg;
+    return code;
+  };
+  if (cudaGetDevice(&h->device) != cudaSuccess) return bail(SPEC_ERR_CUDA, "cudaGetDevice");
+  cudaDeviceProp prop;
+  if (cudaGetDeviceProperties(&prop, h->device) != cudaSuccess) return bail(SPEC_ERR_CUDA, "props");
+  h->sm_count = prop.multiProcessorCount;
+  if (cudaMallocHost(&h->h_params, lay.p_end) != cudaSuccess) return bail(SPEC_ERR_CUDA, "pinned");
+  if (cudaMallocHost(&h->h_out, lay.o_end - lay.o_acc_len) != cudaSuccess) return bail(SPEC_ERR_CUDA, "pinned");
+
+  // per-sequence state starts empty; rotary frequencies theta^(-2j/hd) in double
+  std::vector<double> inv(c.head_dim / 2);
+  for (int j = 0; j < c.head_dim / 2; ++j) inv[j] = std::pow((double)c.rope_theta, -2.0 * j / c.head_dim);
+  if (cudaMemsetAsync(h->ws + lay.seq_len, 0, 4 * (size_t)c.max_batch, h->stream) != cudaSuccess ||
+      cudaMemsetAsync(h->ws + lay.pending, 0xff, 4 * (size_t)c.max_batch, h->stream) != cudaSuccess ||
+      cudaMemsetAsync(h->ws + lay.err_sticky, 0, 16, h->stream) != cudaSuccess ||
+      cudaMemcpyAsync(h->ws + lay.inv_freq, inv.data(), 8 * inv.size(), cudaMemcpyHostToDevice, h->stream) !=
+          cudaSuccess ||
+      cudaStreamSynchronize(h->stream) != cudaSuccess)
+    return bail(SPEC_ERR_CUDA, "state init");
+
+  if (kv_compact_configure((size_t)(c.max_nodes - 1) * c.head_dim * h->kv.elem + 16) != cudaSuccess)
+    return bail(SPEC_ERR_CUDA, "smem attribute");
+  if (c.dtype == SPEC_DTYPE_BF16) {
+    if (!get_encode_fn()) return bail(SPEC_ERR_CUDA, "cuTensorMapEncodeTiled unavailable");
+    if (attention_configure() != cudaSuccess) return bail(SPEC_ERR_CUDA, "smem attribute");
+    const int qd = c.n_q_heads * c.head_dim, kvd = c.n_kv_heads * c.head_dim;
+    h->maps.resize(c.n_layers);
+    for (int l = 0; l < c.n_layers; ++l) {
+      const spec_layer_weights& lw = h->layers[l];
+      LayerMaps& m = h->maps[l];
+      bool ok = make_tmap(&m.wq, lw.wq, qd, c.hidden, 128) && make_tmap(&m.wk, lw.wk, kvd, c.hidden, 128) &&
+                make_tmap(&m.wv, lw.wv, kvd, c.hidden, 128) && make_tmap(&m.wo, lw.wo, c.hidden, qd, 128) &&
+                make_tmap(&m.wg, lw.w_gate, c.ffn, c.hidden, 64) && make_tmap(&m.wu, lw.w_up, c.ffn, c.hidden, 64) &&
+                make_tmap(&m.wd, lw.w_down, c.hidden, c.ffn, 128);
+      if (!ok) return bail(SPEC_ERR_CUDA, "tensor map");
+    }
+    if (!make_tmap(&h->map_lm, h->lm_head, c.vocab, c.hidden, 128)) return bail(SPEC_ERR_CUDA, "tensor map");
+    const int bns[2] = {64, 128};
+    for (int i = 0; i < 2; ++i) {
+      if (!make_tmap(&h->map_xn[i], h->ws + lay.xn, lay.Mpad, c.hidden, bns[i]) ||
+          !make_tmap(&h->map_attn[i], h->ws + lay.attn, lay.Mpad, qd, bns[i]) ||
+          !make_tmap(&h->map_h[i], h->ws + lay.hmlp, lay.Mpad, c.ffn, bns[i]))
+        return bail(SPEC_ERR_CUDA, "tensor map");
+    }
+    for (int i = 0; i < 2; ++i)
+      for (int e = 0; e < 3; ++e) {
+        const void* fn = gemm_tc_function(bns[i], e);
+        const int smem = (int)gemm_tc_smem_bytes(bns[i], e);
+        if (cudaFuncSetAttribute(fn, cudaFuncAttributeMaxDynamicSharedMemorySize, smem) != cudaSuccess)
+          return bail(SPEC_ERR_CUDA, "smem attribute");
+        int nb = 0;
+        if (cudaOccupancyMaxActiveBlocksPerMultiprocessor(&nb, fn, 192, smem) != cudaSuccess || nb < 1)
+          return bail(SPEC_ERR_CUDA, "occupancy");
+        // tensor memory: two accumulators of BN columns per CTA, 512 columns per SM
+        h->resident[i][e] = std::min(nb, 512 / (2 * bns[i]));
+      }
+  }
+  *out = h;
+  return SPEC_OK;
+}
+
+int spec_prefill(spec_handle* h, int seq, const int32_t* tokens, int n, int32_t* pending_token) {
+  if (!h) return SPEC_ERR_ARG;
+  h->err.clear();
+  const spec_config& c = h->cfg;
+  if (!tokens || n < 1) return fail(h, SPEC_ERR_ARG, "prefill needs n >= 1 tokens");
+  if (seq < 0 || seq >= c.max_batch) return fail(h, SPEC_ERR_ARG, "seq %d outside [0, %d)", seq, c.max_batch);
+  if (n > c.max_seq) return fail(h, SPEC_ERR_CAPACITY, "prompt of %d tokens exceeds max_seq %d", n, c.max_seq);
+  for (int i = 0; i < n; ++i)
+    if (tokens[i] < 0 || tokens[i] >= c.vocab) return fail(h, SPEC_ERR_TOKEN, "token %d outside [0, %d)", tokens[i], c.vocab);
+  if (h->stale) {
+    int rc = refresh_state(h);
+    if (rc) return rc;
+  }
+  // reset the sequence
+  const int zero = 0;
+  CUDA_TRY(h, cudaMemcpyAsync(h->ws + h->lay.seq_len + 4 * (size_t)seq, &zero, 4, cudaMemcpyHostToDevice, h->stream));
+  CUDA_TRY(h, cudaStreamSynchronize(h->stream));
+  h->len[seq] = 0;
+  h->len_hi[seq] = 0;
+  h->ready[seq] = 0;
+  std::vector<int32_t> parents(c.max_nodes);
+  for (int i = 0; i < c.max_nodes; ++i) parents[i] = i - 1;
+  const int32_t ids[1] = {seq};
+  for (int s0 = 0; s0 < n; s0 += c.max_nodes) {
+    const int m = std::min(c.max_nodes, n - s0);
+    const int32_t off[2] = {0, m};
+    int rc = run_step(h, 1, ids, tokens + s0, parents.data(), off, STEP_PREFILL, 0, true);
+    if (rc) return rc;
+  }
+  h->ready[seq] = 1;
+  if (pending_token) *pending_token = h->pending[seq];
+  return SPEC_OK;
+}
+
+int spec_verify_tree_batch(spec_handle* h, int B, const int32_t* seq_ids, const int32_t* tokens,
+                           const int32_t* parents, const int32_t* node_offsets, int32_t* accepted_len,
+                           int32_t* accepted_nodes, int32_t* accepted_tokens, int32_t* bonus, int flags) {
+  if (!h) return SPEC_ERR_ARG;
+  h->err.clear();
+  const bool dev = (flags & SPEC_DEVICE_OUTPUTS) != 0;
+  int rc = run_step(h, B, seq_ids, tokens, parents, node_offsets, STEP_VERIFY, flags, !dev);
+  if (rc) return rc;
+  const WsLayout& L = h->lay;
+  const size_t nn = (size_t)B * h->cfg.max_nodes;
+  if (dev) {
+    if (accepted_len)
+      CUDA_TRY(h, cudaMemcpyAsync(accepted_len, h->ws + L.o_acc_len, 4 * (size_t)B, cudaMemcpyDeviceToDevice, h->stream));
+    if (accepted_nodes)
+      CUDA_TRY(h, cudaMemcpyAsync(accepted_nodes, h->ws + L.o_acc_nodes, 4 * nn, cudaMemcpyDeviceToDevice, h->stream));
+    if (accepted_tokens)
+      CUDA_TRY(h, cudaMemcpyAsync(accepted_tokens, h->ws + L.o_acc_tokens, 4 * nn, cudaMemcpyDeviceToDevice, h->stream));
+    if (bonus) CUDA_TRY(h, cudaMemcpyAsync(bonus, h->ws + L.o_bonus, 4 * (size_t)B, cudaMemcpyDeviceToDevice, h->stream));
+    return SPEC_OK;
+  }
+  const uint8_t* ho = h->h_out;
+  if (accepted_len) std::memcpy(accepted_len, ho + (L.o_acc_len - L.o_acc_len), 4 * (size_t)B);
+  if (accepted_nodes) std::memcpy(accepted_nodes, ho + (L.o_acc_nodes - L.o_acc_len), 4 * nn);
+  if (accepted_tokens) std::memcpy(accepted_tokens, ho + (L.o_acc_tokens - L.o_acc_len), 4 * nn);
+  if (bonus) std::memcpy(bonus, ho + (L.o_bonus - L.o_acc_len), 4 * (size_t)B);
+  return SPEC_OK;
+}
+
+int spec_verify_tree(spec_handle* h, int seq, const int32_t* tokens, const int32_t* parents, int n_nodes,
+                     int32_t* accepted_len, int32_t* accepted_tokens, int32_t* bonus_token) {
+  if (!h) return SPEC_ERR_ARG;
+  if (n_nodes < 1) return fail(h, SPEC_ERR_ARG, "n_nodes must be >= 1");
+  if (n_nodes > h->cfg.max_nodes)
+    return fail(h, SPEC_ERR_CAPACITY, "%d nodes > max_nodes %d", n_nodes, h->cfg.max_nodes);
+  const int32_t ids[1] = {seq};
+  const int32_t off[2] = {0, n_nodes};
+  int32_t len = 0, bon = 0;
+  std::vector<int32_t> toks(h->cfg.max_nodes);
+  int rc = spec_verify_tree_batch(h, 1, ids, tokens, parents, off, &len, nullptr, toks.data(), &bon, 0);
+  if (rc) return rc;
+  if (accepted_len) *accepted_len = len;
+  if (accepted_tokens) std::memcpy(accepted_tokens, toks.data(), 4 * (size_t)std::max(0, len));
+  if (bonus_token) *bonus_token = bon;
+  return SPEC_OK;
+}
+
+int spec_score_trees(spec_handle* h, int B, const int32_t* seq_ids, const int32_t* tokens, const int32_t* parents,
+                     const int32_t* node_offsets, int32_t* argmax, float* top1, float* top2, int flags) {
+  if (!h) return SPEC_ERR_ARG;
+  h->err.clear();
+  int rc = run_step(h, B, seq_ids, tokens, parents, node_offsets, STEP_SCORE, flags & ~SPEC_DEVICE_OUTPUTS, true);
+  if (rc) return rc;
+  const int M = node_offsets[B];
+  const WsLayout& L = h->lay;
+  if (argmax) CUDA_TRY(h, cudaMemcpy(argmax, h->ws + L.argmax, 4 * (size_t)M, cudaMemcpyDeviceToHost));
+  if (top1) CUDA_TRY(h, cudaMemcpy(top1, h->ws + L.top1, 4 * (size_t)M, cudaMemcpyDeviceToHost));
+  if (top2) CUDA_TRY(h, cudaMemcpy(top2, h->ws + L.top2, 4 * (size_t)M, cudaMemcpyDeviceToHost));
+  return SPEC_OK;
+}
+
+int spec_set_debug_logits(spec_handle* h, float* device_buf, size_t bytes) {
+  if (!h) return SPEC_ERR_ARG;
+  h->dbg_logits = device_buf;
+  h->dbg_bytes = device_buf ? bytes : 0;
+  // graphs bake the pointer in
+  for (auto& kv : h->graphs) cudaGraphExecDestroy(kv.second);
+  h->graphs.clear();
+  return SPEC_OK;
+}
+
+int spec_truncate(spec_handle* h, int seq, int new_len) {
+  if (!h) return SPEC_ERR_ARG;
+  h->err.clear();
+  if (seq < 0 || seq >= h->cfg.max_batch) return fail(h, SPEC_ERR_ARG, "seq %d outside [0, %d)", seq, h->cfg.max_batch);
+  if (h->stale) {
+    int rc = refresh_state(h);
+    if (rc) return rc;
+  }
+  if (!h->ready[seq]) return fail(h, SPEC_ERR_STATE, "sequence %d has not been prefilled", seq);
+  if (new_len == h->len[seq]) return SPEC_OK;
+  if (new_len < 1 || new_len > h->len[seq])
+    return fail(h, SPEC_ERR_STATE, "cannot truncate sequence %d from %d to %d", seq, h->len[seq], new_len);
+  int32_t tok = 0;
+  CUDA_TRY(h, cudaMemcpyAsync(&tok, h->ws + h->lay.hist + 4 * ((size_t)seq * h->cfg.max_seq + new_len), 4,
+                              cudaMemcpyDeviceToHost, h->stream));
+  CUDA_TRY(h, cudaStreamSynchronize(h->stream));
+  const int32_t vals[1] = {new_len};
+  CUDA_TRY(h, cudaMemcpyAsync(h->ws + h->lay.seq_len + 4 * (size_t)seq, vals, 4, cudaMemcpyHostToDevice, h->stream));
+  CUDA_TRY(h, cudaMemcpyAsync(h->ws + h->lay.pending + 4 * (size_t)seq, &tok, 4, cudaMemcpyHostToDevice, h->stream));
+  CUDA_TRY(h, cudaStreamSynchronize(h->stream));
+  h->len[seq] = new_len;
+  h->len_hi[seq] = new_len;
+  h->pending[seq] = tok;
+  return SPEC_OK;
+}
+
+int spec_seq_len(spec_handle* h, int seq, int32_t* len, int32_t* pending) {
+  if (!h) return SPEC_ERR_ARG;
+  h->err.clear();
+  if (seq < 0 || seq >= h->cfg.max_batch) return fail(h, SPEC_ERR_ARG, "seq %d outside [0, %d)", seq, h->cfg.max_batch);
+  if (h->stale) {
+    int rc = refresh_state(h);
+    if (rc) return rc;
+  }
+  if (len) *len = h->len[seq];
+  if (pending) *pending = h->pending[seq];
+  return SPEC_OK;
+}
+
+int spec_sync(spec_handle* h) {
+  if (!h) return SPEC_ERR_ARG;
+  h->err.clear();
+  return refresh_state(h);
+}
+
+int spec_profile(spec_handle* h, int enable) {
+  if (!h) return SPEC_ERR_ARG;
+  h->prof = enable != 0;
+  h->prof_marks.clear();
+  return SPEC_OK;
+}
+
+int spec_profile_read(spec_handle* h, double* ms, int64_t* launches) {
+  if (!h) return SPEC_ERR_ARG;
+  CUDA_TRY(h, cudaStreamSynchronize(h->stream));
+  for (const auto& m : h->prof_marks) {
+    float t = 0.f;
+    CUDA_TRY(h, cudaEventElapsedTime(&t, h->ev_pool[m.second], h->ev_pool[m.second + 1]));
+    if (ms) ms[m.first] += t;
+    if (launches) launches[m.first] += 1;
+  }
+  h->prof_marks.clear();
+  return SPEC_OK;
+}
+
+int spec_step_launches(spec_handle* h) { return h ? h->launches : 0; }
+
+int spec_io_bytes(spec_handle* h, size_t* h2d, size_t* d2h) {
+  if (!h) return SPEC_ERR_ARG;
+  if (h2d) *h2d = h->lay.p_end;
+  if (d2h) *d2h = (h->lay.o_end - h->lay.o_acc_len) + 4;
+  return SPEC_OK;
+}
+
+const char* spec_last_error(spec_handle* h) { return h ? h->err.c_str() : "null handle"; }
+
+void spec_free(spec_handle* h) {
+  if (!h) return;
+  for (auto& kv : h->graphs) cudaGraphExecDestroy(kv.second);
+  for (cudaEvent_t e : h->ev_pool) cudaEventDestroy(e);
+  if (h->h_params) cudaFreeHost(h->h_params);
+  if (h->h_out) cudaFreeHost(h->h_out);
+  delete h;
+}
+
+}  // extern "C"

@@ -1,0 +1,187 @@
+"""Convenience wrapper over the C ABI: device memory from torch, numpy in and out.
+
+Only marshalling happens here: buffers are allocated with torch (device memory
+and the stream are PyTorch's), arguments are packed into the C structs, and
+every computation is a call into libspec.so.
+"""
+
+from __future__ import annotations
+
+import ctypes
+from typing import Dict, List, Optional, Sequence, Tuple
+
+import numpy as np
+import torch
+
+from . import spec as S
+
+_LAYER_KEYS = ("wq", "wk", "wv", "wo", "w_gate", "w_up", "w_down", "attn_norm", "mlp_norm")
+
+
+def _i32(a) -> np.ndarray:
+    return np.ascontiguousarray(np.asarray(a, dtype=np.int32))
+
+
+def _ptr(a: np.ndarray):
+    return a.ctypes.data_as(ctypes.POINTER(ctypes.c_int32))
+
+
+def _fptr(a: np.ndarray):
+    return a.ctypes.data_as(ctypes.POINTER(ctypes.c_float))
+
+
+def pack_trees(trees: Sequence[Tuple[Sequence[int], Sequence[int]]]):
+    """[(tokens, parents), ...] -> concatenated tokens, parents and node offsets."""
+    toks = [_i32(t) for t, _ in trees]
+    pars = [_i32(p) for _, p in trees]
+    off = np.zeros(len(trees) + 1, np.int32)
+    off[1:] = np.cumsum([len(t) for t in toks])
+    return np.concatenate(toks), np.concatenate(pars), off
+
+
+class SpecEngine:
+    """One handle of the library over caller-owned (torch) device buffers."""
+
+    def __init__(self, dims, weights: Dict, max_batch: int, max_seq: int, max_nodes: int = 128,
+                 stream: Optional[torch.cuda.Stream] = None):
+        self.dims = dims
+        self.cfg = S.spec_config(
+            n_layers=dims.n_layers, hidden=dims.hidden, n_q_heads=dims.n_q_heads, n_kv_heads=dims.n_kv_heads,
+            head_dim=dims.head_dim, ffn=dims.ffn, vocab=dims.vocab,
+            dtype=S.SPEC_DTYPE_BF16 if dims.dtype == "bf16" else S.SPEC_DTYPE_F32,
+            rms_eps=dims.rms_eps, rope_theta=dims.rope_theta, max_batch=max_batch, max_seq=max_seq,
+            max_nodes=max_nodes, draft_head=0)
+        self.max_nodes = max_nodes
+        self.max_batch = max_batch
+        kvb = S.spec_kv_bytes(ctypes.byref(self.cfg))
+        wsb = S.spec_workspace_bytes(ctypes.byref(self.cfg))
+        if kvb == 0 or wsb == 0:
+            raise S.SpecError(S.SPEC_ERR_ARG, "configuration rejected")
+        self.kv = torch.empty(kvb, dtype=torch.uint8, device="cuda")
+        self.ws = torch.empty(wsb, dtype=torch.uint8, device="cuda")
+        self._weights = weights  # keep the tensors alive
+        self._layers = (S.spec_layer_weights * dims.n_layers)()
+        for l, lw in enumerate(weights["layers"]):
+            for k in _LAYER_KEYS:
+                setattr(self._layers[l], k, lw[k].data_ptr())
+        self._w = S.spec_weights(embed=weights["embed"].data_ptr(), final_norm=weights["final_norm"].data_ptr(),
+                                 lm_head=weights["lm_head"].data_ptr(), layers=self._layers)
+        self.stream = stream or torch.cuda.current_stream()
+        h = ctypes.c_void_p()
+        rc = S.spec_init(ctypes.byref(self.cfg), ctypes.byref(self._w), self.kv.data_ptr(), kvb,
+                         self.ws.data_ptr(), wsb, ctypes.c_void_p(self.stream.cuda_stream), ctypes.byref(h))
+        if rc != S.SPEC_OK:
+            raise S.SpecError(rc, "spec_init failed")
+        self.h = h
+        self._dbg = None
+
+    # ------------------------------------------------------------------ helpers
+    def _check(self, rc):
+        if rc != S.SPEC_OK:
+            raise S.SpecError(rc, S.spec_last_error(self.h).decode())
+
+    def close(self):
+        if getattr(self, "h", None):
+            S.spec_free(self.h)
+            self.h = None
+
+    def __del__(self):
+        try:
+            self.close()
+        except Exception:
+            pass
+
+    # ------------------------------------------------------------------ calls
+    def prefill(self, seq: int, tokens) -> int:
+        t = _i32(tokens)
+        pend = np.zeros(1, np.int32)
+        self._check(S.spec_prefill(self.h, seq, _ptr(t), len(t), _ptr(pend)))
+        return int(pend[0])
+
+    def verify(self, seq: int, tokens, parents):
+        t, p = _i32(tokens), _i32(parents)
+        acc_len = np.zeros(1, np.int32)
+        acc_tok = np.zeros(max(1, len(t)), np.int32)
+        bonus = np.zeros(1, np.int32)
+        self._check(S.spec_verify_tree(self.h, seq, _ptr(t), _ptr(p), len(t), _ptr(acc_len), _ptr(acc_tok),
+                                       _ptr(bonus)))
+        a = int(acc_len[0])
+        return a, [int(x) for x in acc_tok[:a]], int(bonus[0])
+
+    def verify_batch(self, seq_ids, trees, flags: int = 0):
+        """Host outputs: (accepted_len[B], accepted_nodes[B][max_nodes], accepted_tokens, bonus[B])."""
+        tok, par, off = pack_trees(trees)
+        ids = _i32(seq_ids)
+        B = len(ids)
+        acc_len = np.zeros(B, np.int32)
+        acc_nodes = np.zeros((B, self.max_nodes), np.int32)
+        acc_tok = np.zeros((B, self.max_nodes), np.int32)
+        bonus = np.zeros(B, np.int32)
+        self._check(S.spec_verify_tree_batch(self.h, B, _ptr(ids), _ptr(tok), _ptr(par), _ptr(off),
+                                             acc_len.ctypes.data, acc_nodes.ctypes.data, acc_tok.ctypes.data,
+                                             bonus.ctypes.data, flags & ~S.SPEC_DEVICE_OUTPUTS))
+        return acc_len, acc_nodes, acc_tok, bonus
+
+    def verify_batch_device(self, ids: np.ndarray, tok: np.ndarray, par: np.ndarray, off: np.ndarray,
+                            outputs: Optional[Tuple[torch.Tensor, ...]] = None, flags: int = 0):
+        """Queue a step without synchronising; outputs (if given) are int32 device tensors."""
+        ptrs = [None] * 4 if outputs is None else [o.data_ptr() if o is not None else None for o in outputs]
+        self._check(S.spec_verify_tree_batch(self.h, len(ids), _ptr(ids), _ptr(tok), _ptr(par), _ptr(off),
+                                             ptrs[0], ptrs[1], ptrs[2], ptrs[3], flags | S.SPEC_DEVICE_OUTPUTS))
+
+    def score(self, seq_ids, trees, flags: int = 0):
+        tok, par, off = pack_trees(trees)
+        ids = _i32(seq_ids)
+        M = int(off[-1])
+        if flags & S.SPEC_DEBUG_LOGITS and (self._dbg is None or self._dbg.numel() < M * self.dims.vocab):
+            self.enable_debug_logits(self.max_batch * self.max_nodes)
+        amax = np.zeros(M, np.int32)
+        t1 = np.zeros(M, np.float32)
+        t2 = np.zeros(M, np.float32)
+        self._check(S.spec_score_trees(self.h, len(ids), _ptr(ids), _ptr(tok), _ptr(par), _ptr(off), _ptr(amax),
+                                       _fptr(t1), _fptr(t2), flags))
+        return amax, t1, t2, off
+
+    def enable_debug_logits(self, rows: int):
+        self._dbg = torch.empty(rows * self.dims.vocab, dtype=torch.float32, device="cuda")
+        self._check(S.spec_set_debug_logits(self.h, self._dbg.data_ptr(), self._dbg.numel() * 4))
+        return self._dbg
+
+    def debug_logits(self, rows: int) -> np.ndarray:
+        torch.cuda.synchronize()
+        return self._dbg[: rows * self.dims.vocab].view(rows, self.dims.vocab).cpu().numpy()
+
+    def truncate(self, seq: int, new_len: int):
+        self._check(S.spec_truncate(self.h, seq, new_len))
+
+    def seq_len(self, seq: int):
+        ln = np.zeros(1, np.int32)
+        pd = np.zeros(1, np.int32)
+        self._check(S.spec_seq_len(self.h, seq, _ptr(ln), _ptr(pd)))
+        return int(ln[0]), int(pd[0])
+
+    def profile(self, enable: bool):
+        self._check(S.spec_profile(self.h, 1 if enable else 0))
+
+    def profile_read(self):
+        ms = (ctypes.c_double * len(S.PROF_CLASSES))()
+        n = (ctypes.c_int64 * len(S.PROF_CLASSES))()
+        self._check(S.spec_profile_read(self.h, ms, n))
+        return {k: (ms[i], n[i]) for i, k in enumerate(S.PROF_CLASSES)}
+
+    def step_launches(self) -> int:
+        return int(S.spec_step_launches(self.h))
+
+    def io_bytes(self):
+        a, b = ctypes.c_size_t(), ctypes.c_size_t()
+        self._check(S.spec_io_bytes(self.h, ctypes.byref(a), ctypes.byref(b)))
+        return int(a.value), int(b.value)
+
+    def sync(self):
+        self._check(S.spec_sync(self.h))
+
+    def kv_view(self) -> torch.Tensor:
+        """The cache as a tensor [layer][2][max_batch][Hkv][max_seq][hd] in the model dtype."""
+        d = self.dims
+        tdt = torch.bfloat16 if d.dtype == "bf16" else torch.float32
+        return self.kv.view(tdt).view(d.n_layers, 2, self.max_batch, d.n_kv_heads, -1, d.head_dim)

@@ -1,0 +1,162 @@
+"""GPU parity: the library (through its C ABI) against the float64 oracle.
+
+Compared element by element on the same seeded inputs: logits at every tree
+node (within 1e-4 for fp32 models, 2e-2 for bf16), the argmax at every node
+whose margin leaves no doubt, the step's outputs (accepted length, tokens,
+bonus), the compacted K/V cache and the sequence state.  Shapes span several
+GEMM and attention tiles, ragged tails, root-only trees, chains, 128-node
+trees and batches of sequences with different prefix lengths.
+"""
+
+import numpy as np
+import pytest
+
+import synth
+from oracle import oracle_verify, top2_margin
+from gpu_common import (DECISIVE, TOL, decisive_nodes, decisive_prefix, gpu_kv, kv_close, make_pair,
+                        planted_tree)
+
+pytestmark = pytest.mark.gpu
+
+
+def _check_step(eng, om, seq_id, seq, shape, tokens, dtype, check_kv=True):
+    """Score (logits), then verify; compare everything with the oracle."""
+    n = shape.n
+    tol = TOL[dtype]
+    amax, t1, t2, _ = eng.score([seq_id], [(tokens, shape.parents)], flags=2)
+    logits = eng.debug_logits(n)
+    P = seq.length
+    r = oracle_verify(om, seq, tokens, shape.parents)
+    err = float(np.max(np.abs(logits - r["logits"])))
+    assert err <= tol, "max |logit error| %.3g > %.3g" % (err, tol)
+    # argmax: exact wherever the oracle's margin exceeds twice the observed error
+    thr = min(DECISIVE, max(2.5 * err, 1e-6))
+    sure = r["margin"] > thr
+    assert np.array_equal(amax[sure], r["argmax"][sure])
+    np.testing.assert_allclose(t1, r["logits"].max(axis=1), atol=tol)
+    a, acc_tok, bonus = eng.verify(seq_id, tokens, shape.parents)
+    decided = bool(np.all(r["margin"][decisive_nodes(r, shape.parents)] > thr))
+    if decided:
+        assert a == r["accepted_len"]
+        assert acc_tok == r["accepted_tokens"]
+        assert bonus == r["bonus"]
+        ln, pend = eng.seq_len(seq_id)
+        assert ln == P + 1 + a and pend == bonus
+        if check_kv:
+            gk, gv = gpu_kv(eng, seq_id, ln)
+            for l in range(om.d.n_layers):
+                kt = 1e-5 if dtype == "f32" else 2e-2
+                assert kv_close(gk[l], seq.k[l], kt) <= kt, "layer %d K" % l
+                assert kv_close(gv[l], seq.v[l], kt) <= kt, "layer %d V" % l
+    return decided, err
+
+
+def test_tiny_fp32_config():
+    """fp32 tiny decoder: prefix 64, 8 drafts at depth 4 (widths 2,4,1,1), planted p = 0.8."""
+    eng, om = make_pair(synth.TINY, max_batch=1, max_seq=512, max_nodes=16)
+    prefix, seq = decisive_prefix(om, 64, min_margin=1e-3)
+    pend = eng.prefill(0, prefix)
+    assert pend == seq.pending
+    gk, gv = gpu_kv(eng, 0, 64)
+    assert kv_close(gk[0], seq.k[0], 1e-5) <= 1e-5
+    decided = 0
+    for step in range(4):
+        shape = synth.tiny_tree()
+        toks = planted_tree(om, seq, shape, 0.8, stream=step)
+        d, err = _check_step(eng, om, 0, seq, shape, toks, "f32")
+        decided += d
+        assert err < 1e-4
+    assert decided >= 3
+
+
+BF16_CASES = [
+    ("mini", 37, "root"),
+    ("mini", 37, "chain2"),
+    ("mini", 300, "tiny"),
+    ("mini", 1000, "tree60"),
+    ("mini", 129, "tree127"),
+    ("small", 700, "tree60"),
+    ("small", 64, "chain8"),
+]
+
+
+def _shape(kind):
+    if kind == "root":
+        return synth.chain(0)
+    if kind == "chain2":
+        return synth.chain(2)
+    if kind == "chain8":
+        return synth.chain(8)
+    if kind == "tiny":
+        return synth.tiny_tree()
+    if kind == "tree60":
+        return synth.tree_from_widths(synth.TREE60_WIDTHS, stream=4)
+    if kind == "tree127":
+        return synth.tree_from_widths((10, 12, 16, 20, 20, 20, 16, 13), stream=5)
+    raise KeyError(kind)
+
+
+_pairs = {}
+
+
+def _pair(which):
+    if which not in _pairs:
+        dims = synth.MINI_BF16 if which == "mini" else synth.SMALL_BF16
+        _pairs[which] = make_pair(dims, max_batch=4, max_seq=1400, max_nodes=128)
+    return _pairs[which]
+
+
+@pytest.mark.parametrize("which,P,kind", BF16_CASES)
+def test_bf16_verify_parity(which, P, kind):
+    eng, om = _pair(which)
+    prefix, seq = decisive_prefix(om, P, stream0=P)
+    pend = eng.prefill(0, prefix)
+    assert pend == seq.pending
+    gk, gv = gpu_kv(eng, 0, P)
+    for l in range(om.d.n_layers):
+        assert kv_close(gk[l], seq.k[l], 2e-2) <= 2e-2
+    shape = _shape(kind)
+    toks = planted_tree(om, seq, shape, 0.8, stream=P)
+    _check_step(eng, om, 0, seq, shape, toks, "bf16")
+
+
+def test_bf16_batch_of_sequences():
+    """Three sequences with different prefix lengths and trees in one batched step."""
+    eng, om = _pair("mini")
+    Ps = [45, 410, 130]
+    shapes = [synth.tree_from_widths((3, 3, 2), stream=1), synth.tiny_tree(), synth.chain(5)]
+    seqs, trees = [], []
+    for i, (P, sh) in enumerate(zip(Ps, shapes)):
+        prefix, seq = decisive_prefix(om, P, stream0=100 + 10 * i)
+        assert eng.prefill(i, prefix) == seq.pending
+        toks = planted_tree(om, seq, sh, 0.8, stream=50 + i)
+        seqs.append(seq)
+        trees.append((toks, sh.parents))
+    amax, t1, t2, off = eng.score([0, 1, 2], trees, flags=2)
+    logits = eng.debug_logits(int(off[-1]))
+    acc_len, acc_nodes, acc_tok, bonus = eng.verify_batch([0, 1, 2], trees)
+    for i, (seq, (toks, par)) in enumerate(zip(seqs, trees)):
+        r = oracle_verify(om, seq, toks, par)
+        lg = logits[off[i]:off[i + 1]]
+        err = float(np.max(np.abs(lg - r["logits"])))
+        assert err <= TOL["bf16"]
+        thr = min(DECISIVE, 2.5 * err)
+        if np.all(r["margin"][decisive_nodes(r, par)] > thr):
+            assert acc_len[i] == r["accepted_len"]
+            assert list(acc_nodes[i, :acc_len[i]]) == r["accepted_nodes"]
+            assert list(acc_tok[i, :acc_len[i]]) == r["accepted_tokens"]
+            assert bonus[i] == r["bonus"]
+            ln, _ = eng.seq_len(i)
+            gk, gv = gpu_kv(eng, i, ln)
+            for l in range(om.d.n_layers):
+                assert kv_close(gk[l], seq.k[l], 2e-2) <= 2e-2
+
+
+def test_wide_bf16_full_size_tiles():
+    """8B layer shapes (d 4096, 32/8 heads, ffn 14336), 2 layers, vocab 16384: full-size tiles and splits."""
+    eng, om = make_pair(synth.WIDE_BF16, max_batch=1, max_seq=512, max_nodes=64, device_gen=True)
+    prefix, seq = decisive_prefix(om, 200, stream0=7, tries=6)
+    assert eng.prefill(0, prefix) == seq.pending
+    shape = synth.tree_from_widths(synth.TREE60_WIDTHS, stream=0)
+    toks = planted_tree(om, seq, shape, 0.8, stream=9)
+    _check_step(eng, om, 0, seq, shape, toks, "bf16")
