@@ -37,10 +37,11 @@ METRIC = "verify steps/s and accepted tokens/s at Llama-3.1-8B shape; % HBM roof
 UNIT = "verify steps/s"
 
 
-def workload_config(P=2048):
+def workload_config(P=2048, layers=32):
     return {"workload": "llama3.1-8b-shape bf16, batch 1, prefix %d, 60-draft depth-8 tree (widths 10,10,10,8,8,6,4,4),"
-                        " planted acceptance p=0.8" % P,
-            "model_shape": "32 layers, d 4096, 32/8 heads x 128, ffn 14336, vocab 128256",
+                        " planted acceptance p=0.8%s" % (P, "" if layers == 32 else
+                                                          " [PROFILING CASE: %d of 32 layers]" % layers),
+            "model_shape": "%d layers, d 4096, 32/8 heads x 128, ffn 14336, vocab 128256" % layers,
             "batch": 1, "prefix": P, "tree_nodes": 61, "depth": 8, "accept_p": 0.8,
             "l2": "inputs larger than L2 (15 GB of weights streamed per step)",
             "parallelism": "replicas (one independent verifier per GPU)"}
@@ -234,7 +235,8 @@ def run_ours(args, rank, world, local_rank):
         import datetime
         import torch.distributed as dist
         dist.init_process_group("nccl", timeout=datetime.timedelta(seconds=120), device_id=torch.device("cuda", local_rank))
-    dims = synth.LLAMA8B
+    import dataclasses
+    dims = dataclasses.replace(synth.LLAMA8B, n_layers=args.layers)
     P = args.prefix
     w = synth.model_weights(dims, seed=0, device="cuda")
     eng = SpecEngine(dims, w, max_batch=1, max_seq=P + 256, max_nodes=64)
@@ -250,7 +252,7 @@ def run_ours(args, rank, world, local_rank):
     tk, pr, off = pack_trees([(tokens, shape.parents)])
     ids = np.array([0], np.int32)
     acc_dev = torch.zeros(1, dtype=torch.int32, device="cuda")
-    stream = torch.cuda.current_stream()
+    stream = eng.stream  # the library's stream: events must be recorded where its kernels run
 
     def one_step():
         eng.verify_batch_device(ids, tk, pr, off, outputs=(acc_dev, None, None, None))
@@ -273,9 +275,11 @@ def run_ours(args, rank, world, local_rank):
     for _ in range(args.steps):
         e0 = torch.cuda.Event(enable_timing=True)
         e1 = torch.cuda.Event(enable_timing=True)
+        torch.cuda.nvtx.range_push("timed_step")
         e0.record(stream)
         one_step()
         e1.record(stream)
+        torch.cuda.nvtx.range_pop()
         e1.synchronize()
         times.append(e0.elapsed_time(e1))
         eng.sync()
@@ -326,7 +330,7 @@ def run_ours(args, rank, world, local_rank):
         "metric": METRIC, "value": value, "unit": UNIT, "n_gpus": world, "steps": args.steps,
         "warmup": max(3, args.warmup), "ms_per_step": ms, "higher_is_better": True, "scaling": "weak",
         "vs_baseline": None, "dtype": "bf16", "data": "synthetic (random-init weights, uniform prefix, planted tree)",
-        "config": workload_config(P),
+        "config": workload_config(P, args.layers),
         "accepted_tokens_per_s": value * (a_len + 1), "tau": a_len + 1,
         "roofline": {"bound": "hbm", "kernel": dom, "achieved": achieved, "peak": hbm, "unit": "GB/s",
                      "frac": achieved / hbm, "traffic": None, "peak_source": peak_kind,
@@ -338,7 +342,7 @@ def run_ours(args, rank, world, local_rank):
         "gpu_launches": launches * args.steps,
         "clocks": clocks,
     }
-    if rank == 0 and world == 1 and not args.no_cpu_baseline:
+    if rank == 0 and world == 1 and not args.no_cpu_baseline and args.layers == 32:
         hostw = host_sample_weights(w, args.sample_layers)
         per_step, wall = oracle_step_sample(dims, hostw, P, tokens, shape.parents, args.sample_layers)
         line["cpu_baseline"] = {"value": 1.0 / per_step, "unit": UNIT, "cores": len(os.sched_getaffinity(0)),
@@ -362,6 +366,7 @@ def main():
     ap.add_argument("--prefix", type=int, default=2048)
     ap.add_argument("--sample-layers", type=int, default=2)
     ap.add_argument("--no-cpu-baseline", action="store_true")
+    ap.add_argument("--layers", type=int, default=32, help="decoder layers (32 = the 8B shape; fewer only for profiling)")
     args = ap.parse_args()
     rank = int(os.environ.get("RANK", "0"))
     world = int(os.environ.get("WORLD_SIZE", "1"))

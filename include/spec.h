@@ -56,7 +56,8 @@ extern "C" {
 
 /* model dtypes */
 #define SPEC_DTYPE_F32 0       /* weights, activations and K/V in fp32; plain FFMA arithmetic */
-#define SPEC_DTYPE_BF16 1      /* weights and K/V in bf16; fp32 accumulation, residual and softmax */
+#define SPEC_DTYPE_BF16 1      /* weights bf16; GEMM activations as split bf16 (hi + lo); q, K/V cache and
+                                  attention probabilities fp16; fp32 accumulation, residual and softmax */
 
 /* flags of spec_verify_tree_batch */
 #define SPEC_DEVICE_OUTPUTS 1  /* outputs are device pointers (or NULL); return without synchronising */
@@ -113,14 +114,17 @@ typedef struct spec_weights {
 
 typedef struct spec_handle spec_handle;
 
-/* Bytes of device memory for the K/V cache (layout [layer][K|V][seq][kv head][slot][hd]). */
+/* Bytes of device memory for the K/V cache (layout [layer][K|V][seq][kv head][slot][hd];
+ * fp16 elements for bf16 models, fp32 for fp32 models). */
 SPEC_API size_t spec_kv_bytes(const spec_config* cfg);
 /* Bytes of device workspace (activations, split-K partials, per-sequence state). */
 SPEC_API size_t spec_workspace_bytes(const spec_config* cfg);
 
 /* Validate dimensions, record the borrowed device buffers, build the TMA
  * descriptors.  kv_cache and workspace are device buffers of at least the
- * sizes above; cuda_stream is a cudaStream_t (NULL: the legacy default stream).
+ * sizes above; cuda_stream is a cudaStream_t (NULL: the legacy default stream,
+ * on which steps are launched kernel by kernel because it cannot be captured
+ * into a CUDA graph).
  * Every sequence starts empty. */
 SPEC_API int spec_init(const spec_config* cfg, const spec_weights* w, void* kv_cache, size_t kv_bytes, void* workspace,
               size_t ws_bytes, void* cuda_stream, spec_handle** out);

@@ -6,13 +6,16 @@
 // 树验证器方法", section 树draft vs 链draft).  Grouped-query attention: query head
 // h reads key/value head h / (Hq/Hkv).
 //
-// bf16 path (flash-decoding): the keys [0, P_b + n_b) are cut into chunks;
+// bf16-model path (flash-decoding): the keys [0, P_b + n_b) are cut into chunks;
 // one CTA handles one (sequence, kv head, chunk, block of 64 query rows).  The
 // query rows of a kv head are its G = Hq/Hkv heads for every tree node, so a
-// K/V chunk loaded once serves all of them.  Scores and P.V run on bf16
-// mma.sync tiles with an fp32 online softmax (quad shuffles); the ancestor
+// K/V chunk loaded once serves all of them.  q, the K/V cache and the
+// probabilities are fp16 (10 mantissa bits at 2 bytes); scores and P.V run on
+// fp16 mma.sync tiles with fp32 accumulation and an fp32 online softmax (quad
+// shuffles); the ancestor
 // mask applies only to keys at or beyond P_b.  Each CTA writes an fp32 partial
-// (normalised output + log-sum-exp); a merge kernel combines the chunks.
+// (normalised output + log-sum-exp); a merge kernel combines the chunks and
+// writes the output as split bf16 for the O-projection GEMM.
 //
 // fp32 path: one warp per (node, head), exact fp32 scalar arithmetic.
 #include "common.cuh"
@@ -44,15 +47,15 @@ __device__ __forceinline__ void ldsm_x4_t(uint32_t addr, uint32_t& r0, uint32_t&
                : "=r"(r0), "=r"(r1), "=r"(r2), "=r"(r3)
                : "r"(addr));
 }
-__device__ __forceinline__ void mma_bf16_16816(float* c, const uint32_t* a, uint32_t b0, uint32_t b1) {
+__device__ __forceinline__ void mma_f16_16816(float* c, const uint32_t* a, uint32_t b0, uint32_t b1) {
   asm volatile(
-      "mma.sync.aligned.m16n8k16.row.col.f32.bf16.bf16.f32 {%0,%1,%2,%3}, {%4,%5,%6,%7}, {%8,%9}, "
+      "mma.sync.aligned.m16n8k16.row.col.f32.f16.f16.f32 {%0,%1,%2,%3}, {%4,%5,%6,%7}, {%8,%9}, "
       "{%0,%1,%2,%3};"
       : "+f"(c[0]), "+f"(c[1]), "+f"(c[2]), "+f"(c[3])
       : "r"(a[0]), "r"(a[1]), "r"(a[2]), "r"(a[3]), "r"(b0), "r"(b1));
 }
-__device__ __forceinline__ uint32_t pack_bf16(float lo, float hi) {
-  __nv_bfloat162 v = __floats2bfloat162_rn(lo, hi);
+__device__ __forceinline__ uint32_t pack_f16(float lo, float hi) {
+  __half2 v = __floats2half2_rn(lo, hi);
   return *reinterpret_cast<uint32_t*>(&v);
 }
 
@@ -62,11 +65,11 @@ __device__ __forceinline__ bool anc_has(uint64_t a0, uint64_t a1, int j) {
 
 }  // namespace
 
-__global__ void __launch_bounds__(128) attn_chunk_bf16_kernel(AttnArgs a) {
+__global__ void __launch_bounds__(128) attn_chunk_f16_kernel(AttnArgs a) {
   extern __shared__ __align__(16) uint8_t smem_raw[];
-  __nv_bfloat16* sQ = reinterpret_cast<__nv_bfloat16*>(smem_raw);
-  __nv_bfloat16* sK = sQ + kRowsPerCta * kStride;          // [2][64][kStride]
-  __nv_bfloat16* sV = sK + 2 * kKeyBlock * kStride;        // [2][64][kStride]
+  __half* sQ = reinterpret_cast<__half*>(smem_raw);
+  __half* sK = sQ + kRowsPerCta * kStride;          // [2][64][kStride]
+  __half* sV = sK + 2 * kKeyBlock * kStride;        // [2][64][kStride]
 
   pdl_wait();
   const StepView& sv = a.sv;
@@ -89,10 +92,10 @@ __global__ void __launch_bounds__(128) attn_chunk_bf16_kernel(AttnArgs a) {
   const int c1 = min(c0 + a.chunk, Lk);
   const int seq = sv.seq_ids[b];
 
-  const __nv_bfloat16* kbase = reinterpret_cast<const __nv_bfloat16*>(a.kv.base) + a.layer * a.kv.layer_stride() +
-                               seq * a.kv.seq_stride() + kvh * a.kv.head_stride();
-  const __nv_bfloat16* vbase = kbase + a.kv.kv_stride();
-  const __nv_bfloat16* q = reinterpret_cast<const __nv_bfloat16*>(a.q);
+  const __half* kbase = reinterpret_cast<const __half*>(a.kv.base) + a.layer * a.kv.layer_stride() +
+                        seq * a.kv.seq_stride() + kvh * a.kv.head_stride();
+  const __half* vbase = kbase + a.kv.kv_stride();
+  const __half* q = reinterpret_cast<const __half*>(a.q);
 
   const int tid = threadIdx.x;
   const int warp = tid >> 5;
@@ -105,7 +108,7 @@ __global__ void __launch_bounds__(128) attn_chunk_bf16_kernel(AttnArgs a) {
     const bool ok = qr < rows;
     const int node = ok ? qr / G : 0;
     const int h = kvh * G + (ok ? qr - node * G : 0);
-    const __nv_bfloat16* src = q + ((size_t)(base + node) * a.Hq + h) * hd + ch * 8;
+    const __half* src = q + ((size_t)(base + node) * a.Hq + h) * hd + ch * 8;
     cp_async16(sQ + rr * kStride + ch * 8, src, ok);
   }
   auto load_kv = [&](int buf, int kstart) {
@@ -160,8 +163,8 @@ __global__ void __launch_bounds__(128) attn_chunk_bf16_kernel(AttnArgs a) {
         ldsm_x4(addr, qf[ks][0], qf[ks][1], qf[ks][2], qf[ks][3]);
       }
     }
-    const __nv_bfloat16* K_ = sK + buf * kKeyBlock * kStride;
-    const __nv_bfloat16* V_ = sV + buf * kKeyBlock * kStride;
+    const __half* K_ = sK + buf * kKeyBlock * kStride;
+    const __half* V_ = sV + buf * kKeyBlock * kStride;
     const int kstart = c0 + blk * kKeyBlock;
 
     // S = Q K^T  (16 rows x 64 keys per warp)
@@ -174,8 +177,8 @@ __global__ void __launch_bounds__(128) attn_chunk_bf16_kernel(AttnArgs a) {
         uint32_t b0, b1, b2, b3;
         const uint32_t addr = smem_u32(K_ + (nt * 8 + (lane & 7)) * kStride + ks * 16 + (lane >> 3) * 8);
         ldsm_x4(addr, b0, b1, b2, b3);
-        mma_bf16_16816(s[nt], qf[ks], b0, b1);
-        mma_bf16_16816(s[nt], qf[ks + 1], b2, b3);
+        mma_f16_16816(s[nt], qf[ks], b0, b1);
+        mma_f16_16816(s[nt], qf[ks + 1], b2, b3);
       }
     }
     // mask, scale, online softmax
@@ -228,10 +231,10 @@ __global__ void __launch_bounds__(128) attn_chunk_bf16_kernel(AttnArgs a) {
 #pragma unroll
     for (int kk = 0; kk < 4; ++kk) {
       uint32_t pa[4];
-      pa[0] = pack_bf16(s[2 * kk][0], s[2 * kk][1]);
-      pa[1] = pack_bf16(s[2 * kk][2], s[2 * kk][3]);
-      pa[2] = pack_bf16(s[2 * kk + 1][0], s[2 * kk + 1][1]);
-      pa[3] = pack_bf16(s[2 * kk + 1][2], s[2 * kk + 1][3]);
+      pa[0] = pack_f16(s[2 * kk][0], s[2 * kk][1]);
+      pa[1] = pack_f16(s[2 * kk][2], s[2 * kk][3]);
+      pa[2] = pack_f16(s[2 * kk + 1][0], s[2 * kk + 1][1]);
+      pa[3] = pack_f16(s[2 * kk + 1][2], s[2 * kk + 1][3]);
 #pragma unroll
       for (int nd = 0; nd < 16; nd += 2) {
         uint32_t b0, b1, b2, b3;
@@ -239,8 +242,8 @@ __global__ void __launch_bounds__(128) attn_chunk_bf16_kernel(AttnArgs a) {
         const uint32_t addr =
             smem_u32(V_ + (kk * 16 + (m & 1) * 8 + (lane & 7)) * kStride + (nd + (m >> 1)) * 8);
         ldsm_x4_t(addr, b0, b1, b2, b3);
-        mma_bf16_16816(o[nd], pa, b0, b1);
-        mma_bf16_16816(o[nd + 1], pa, b2, b3);
+        mma_f16_16816(o[nd], pa, b0, b1);
+        mma_f16_16816(o[nd + 1], pa, b2, b3);
       }
     }
     __syncthreads();
@@ -267,8 +270,9 @@ __global__ void __launch_bounds__(128) attn_chunk_bf16_kernel(AttnArgs a) {
   pdl_launch_dependents();
 }
 
-// one warp per (node, head): weights 2^(lse_c - max) over the sequence's chunks
-__global__ void attn_merge_bf16_kernel(AttnArgs a) {
+// one warp per (node, head): weights 2^(lse_c - max) over the sequence's chunks;
+// the result is written as split bf16 (hi and lo rows) for the O projection
+__global__ void attn_merge_kernel(AttnArgs a) {
   pdl_wait();
   const int hd = 128;
   const int w = blockIdx.x * (blockDim.x >> 5) + (threadIdx.x >> 5);
@@ -293,11 +297,13 @@ __global__ void attn_merge_bf16_kernel(AttnArgs a) {
     acc.x += wt * v.x; acc.y += wt * v.y; acc.z += wt * v.z; acc.w += wt * v.w;
   }
   const float inv = wsum > 0.f ? 1.f / wsum : 0.f;
-  __nv_bfloat16* out = reinterpret_cast<__nv_bfloat16*>(a.out) + (size_t)w * hd + lane * 4;
-  __nv_bfloat162 lo = __floats2bfloat162_rn(acc.x * inv, acc.y * inv);
-  __nv_bfloat162 hi = __floats2bfloat162_rn(acc.z * inv, acc.w * inv);
-  *reinterpret_cast<__nv_bfloat162*>(out) = lo;
-  *reinterpret_cast<__nv_bfloat162*>(out + 2) = hi;
+  __nv_bfloat16* out = reinterpret_cast<__nv_bfloat16*>(a.out);
+  const int ld = a.Hq * hd;
+  const int col = (w - r * a.Hq) * hd + lane * 4;
+  split_store(out, r, ld, col + 0, acc.x * inv);
+  split_store(out, r, ld, col + 1, acc.y * inv);
+  split_store(out, r, ld, col + 2, acc.z * inv);
+  split_store(out, r, ld, col + 3, acc.w * inv);
   pdl_launch_dependents();
 }
 
@@ -358,10 +364,10 @@ __global__ void attn_f32_kernel(AttnArgs a) {
   }
 }
 
-size_t attention_smem_bytes() { return (size_t)(kRowsPerCta + 4 * kKeyBlock) * kStride * sizeof(__nv_bfloat16); }
+size_t attention_smem_bytes() { return (size_t)(kRowsPerCta + 4 * kKeyBlock) * kStride * sizeof(__half); }
 
 cudaError_t attention_configure() {
-  return cudaFuncSetAttribute(attn_chunk_bf16_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
+  return cudaFuncSetAttribute(attn_chunk_f16_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
                               (int)attention_smem_bytes());
 }
 
@@ -382,14 +388,14 @@ cudaError_t launch_attention(int dtype, const AttnArgs& a, cudaStream_t s, bool 
   cfg.stream = s;
   cfg.attrs = attr;
   cfg.numAttrs = pdl ? 1 : 0;
-  cudaError_t e = cudaLaunchKernelEx(&cfg, attn_chunk_bf16_kernel, a);
+  cudaError_t e = cudaLaunchKernelEx(&cfg, attn_chunk_f16_kernel, a);
   if (e != cudaSuccess) return e;
   cudaLaunchConfig_t cfg2 = cfg;
   const int warps = a.sv.M * a.Hq;
   cfg2.gridDim = dim3((warps + 7) / 8);
   cfg2.blockDim = dim3(256);
   cfg2.dynamicSmemBytes = 0;
-  return cudaLaunchKernelEx(&cfg2, attn_merge_bf16_kernel, a);
+  return cudaLaunchKernelEx(&cfg2, attn_merge_kernel, a);
 }
 
 }  // namespace spec

@@ -9,6 +9,7 @@
 
 #include <cstdint>
 #include <cuda_bf16.h>
+#include <cuda_fp16.h>
 #include <cuda_runtime.h>
 
 namespace spec {
@@ -187,6 +188,47 @@ __device__ __forceinline__ void tmem_ld16(uint32_t taddr, float* v) {
   for (int i = 0; i < 16; ++i) v[i] = __uint_as_float(r[i]);
 }
 
+// Two tcgen05.ld of 16 columns each (two column blocks of the same lanes), one wait.
+__device__ __forceinline__ void tmem_ld16x2(uint32_t ta, uint32_t tb, float* va, float* vb) {
+  uint32_t r[16], q[16];
+  asm volatile(
+      "tcgen05.ld.sync.aligned.32x32b.x16.b32 {%0,%1,%2,%3,%4,%5,%6,%7,%8,%9,%10,%11,%12,%13,%14,%15}, [%16];"
+      : "=r"(r[0]), "=r"(r[1]), "=r"(r[2]), "=r"(r[3]), "=r"(r[4]), "=r"(r[5]), "=r"(r[6]), "=r"(r[7]),
+        "=r"(r[8]), "=r"(r[9]), "=r"(r[10]), "=r"(r[11]), "=r"(r[12]), "=r"(r[13]), "=r"(r[14]), "=r"(r[15])
+      : "r"(ta));
+  asm volatile(
+      "tcgen05.ld.sync.aligned.32x32b.x16.b32 {%0,%1,%2,%3,%4,%5,%6,%7,%8,%9,%10,%11,%12,%13,%14,%15}, [%16];"
+      : "=r"(q[0]), "=r"(q[1]), "=r"(q[2]), "=r"(q[3]), "=r"(q[4]), "=r"(q[5]), "=r"(q[6]), "=r"(q[7]),
+        "=r"(q[8]), "=r"(q[9]), "=r"(q[10]), "=r"(q[11]), "=r"(q[12]), "=r"(q[13]), "=r"(q[14]), "=r"(q[15])
+      : "r"(tb));
+  asm volatile("tcgen05.wait::ld.sync.aligned;" ::: "memory");
+#pragma unroll
+  for (int i = 0; i < 16; ++i) {
+    va[i] = __uint_as_float(r[i]);
+    vb[i] = __uint_as_float(q[i]);
+  }
+}
+
+// ---------------------------------------------------------------------------
+// split-bf16 activations
+// ---------------------------------------------------------------------------
+// A bf16 model's GEMM activations are stored as two bf16 parts, hi = bf16(v)
+// and lo = bf16(v - hi), which together carry ~16 mantissa bits; the weights
+// are exact bf16, so W.hi + W.lo reproduces W.v to fp32-accumulation accuracy.
+// Layout: tokens in groups of 64; group g occupies 128 rows, its 64 hi rows
+// followed by its 64 lo rows.  A GEMM tile of BN tokens (BN a multiple of 64)
+// is one contiguous box of 2*BN rows.
+constexpr int kSplitGroup = 64;
+__host__ __device__ __forceinline__ int split_row(int t, int part) {
+  return (t / kSplitGroup) * (2 * kSplitGroup) + part * kSplitGroup + (t % kSplitGroup);
+}
+__device__ __forceinline__ void split_store(__nv_bfloat16* base, int t, int ld, int col, float v) {
+  const __nv_bfloat16 hi = __float2bfloat16_rn(v);
+  const __nv_bfloat16 lo = __float2bfloat16_rn(v - __bfloat162float(hi));
+  base[(size_t)split_row(t, 0) * ld + col] = hi;
+  base[(size_t)split_row(t, 1) * ld + col] = lo;
+}
+
 // Shared-memory matrix descriptor for a K-major tile written by TMA with the
 // 128-byte swizzle: rows of 64 bf16 (128 B), 8-row swizzle atoms 1024 B apart.
 // Fields: start address >> 4 (bits 0-13), leading byte offset >> 4 (16-29,
@@ -260,8 +302,10 @@ __device__ __forceinline__ Top2 warp_top2(Top2 t) {
 template <typename T> __device__ __forceinline__ float to_f32(T v);
 template <> __device__ __forceinline__ float to_f32<float>(float v) { return v; }
 template <> __device__ __forceinline__ float to_f32<__nv_bfloat16>(__nv_bfloat16 v) { return __bfloat162float(v); }
+template <> __device__ __forceinline__ float to_f32<__half>(__half v) { return __half2float(v); }
 template <typename T> __device__ __forceinline__ T from_f32(float v);
 template <> __device__ __forceinline__ float from_f32<float>(float v) { return v; }
 template <> __device__ __forceinline__ __nv_bfloat16 from_f32<__nv_bfloat16>(float v) { return __float2bfloat16_rn(v); }
+template <> __device__ __forceinline__ __half from_f32<__half>(float v) { return __float2half_rn(v); }
 
 }  // namespace spec

@@ -5,19 +5,22 @@
 //
 // At tree-verification sizes the token count (tree nodes x batch) is small,
 // so the weights are put on the MMA's M = 128 side and the tokens on its N
-// side (BN = 64 or 128 columns): one CTA streams 128 weight rows per tile
-// while the few token rows come from L2.  The step is bound by streaming the
+// side: one CTA streams 128 weight rows per tile while the few token rows come
+// from L2.  The activations arrive as split bf16 (hi and lo parts, see
+// split_row): a tile of BN tokens is a box of 2*BN rows and one MMA of
+// N = 2*BN; the epilogue adds the hi and lo columns, so the product carries
+// ~16 mantissa bits of the activation instead of 8.  The step is bound by streaming the
 // weights once from HBM ("EAGLE-3投机解码：树验证器方法", section 问题: decode
 // is memory-bandwidth bound), so the kernel is a persistent, warp-specialised
 // weight streamer:
 //
-//   warp 0      TMA producer: weight tile (128 x 64) + token tile (BN x 64) per stage
+//   warp 0      TMA producer: weight tile (128 x 64) + token tile (2*BN x 64) per stage
 //   warp 1      MMA issuer: 4 x tcgen05.mma (K = 16 each) per stage into a TMEM
 //               accumulator; owns the tensor-memory allocation
 //   warps 2-5   epilogue: tcgen05.ld of their 32 accumulator lanes, then one of
 //               - PARTIAL: fp32 split-K partial sums  [split][tokens][out]
 //               - SWIGLU : tile rows 0-63 are gate rows, 64-127 the matching up rows;
-//                          writes silu(gate) * up as bf16 [tokens][ffn]
+//                          writes silu(gate) * up as split bf16 [tokens][ffn]
 //               - ARGMAX : per token, best / index / runner-up over the tile's
 //                          128 vocabulary rows (logits never reach HBM)
 //
@@ -41,7 +44,7 @@ constexpr uint32_t kABytes = kTileO * kTileK * 2;
 
 template <int BN, int STAGES, int EPI>
 struct SmemLayout {
-  static constexpr uint32_t kBBytes = BN * kTileK * 2;
+  static constexpr uint32_t kBBytes = 2 * BN * kTileK * 2;  // hi and lo rows
   static constexpr uint32_t a_off = 0;
   static constexpr uint32_t b_off = a_off + STAGES * kABytes;
   static constexpr uint32_t epi_off = b_off + STAGES * kBBytes;
@@ -53,7 +56,8 @@ struct SmemLayout {
   static constexpr uint32_t misc_off = bar_off + n_bars * 8;
   static constexpr uint32_t total = misc_off + 16;
   static constexpr uint32_t dyn_bytes = total + 1024;  // slack to align the base to 1024
-  static constexpr uint32_t tmem_cols = (2 * BN < 32) ? 32 : 2 * BN;
+  static constexpr uint32_t acc_cols = 2 * BN;             // one accumulator: hi and lo columns
+  static constexpr uint32_t tmem_cols = 2 * acc_cols;       // two accumulators
 };
 
 __device__ __forceinline__ void named_sync(int id, int n) {
@@ -149,7 +153,7 @@ __global__ void __launch_bounds__(kThreads, 1)
               tma_load_2d(sa, &mA2, &full[stage], kx, row - args.seg_rows[0] - args.seg_rows[1], pol_w);
             }
           }
-          tma_load_2d(sb, &mB, &full[stage], kx, tt * BN, pol_x);
+          tma_load_2d(sb, &mB, &full[stage], kx, tt * 2 * BN, pol_x);
           if (++stage == STAGES) {
             stage = 0;
             phase ^= 1;
@@ -168,7 +172,7 @@ __global__ void __launch_bounds__(kThreads, 1)
   } else if (warp == 1) {
     // ------------------------------------------------------------------ MMA issuer
     if (elect_one()) {
-      constexpr uint32_t idesc = idesc_bf16_f32(kTileO, BN);
+      constexpr uint32_t idesc = idesc_bf16_f32(kTileO, 2 * BN);
       int stage = 0;
       uint32_t phase = 0;
       int j = 0;
@@ -183,7 +187,7 @@ __global__ void __launch_bounds__(kThreads, 1)
         const uint32_t acc_phase = (j >> 1) & 1;
         if (!mbar_wait(&tempty[acc], acc_phase ^ 1, args.err, abort_flag)) break;
         tc_fence_after();
-        const uint32_t d_tmem = tmem_base + acc * BN;
+        const uint32_t d_tmem = tmem_base + acc * L::acc_cols;
         bool ok = true;
         for (int kb = kb0; kb < kb1; ++kb) {
           if (!mbar_wait(&full[stage], phase, args.err, abort_flag)) {
@@ -232,7 +236,7 @@ __global__ void __launch_bounds__(kThreads, 1)
       named_sync(2, 128);
       if (!*ep_ok) break;
       tc_fence_after();
-      const uint32_t taddr = tmem_base + ((uint32_t)(quarter * 32) << 16) + acc * BN;
+      const uint32_t taddr = tmem_base + ((uint32_t)(quarter * 32) << 16) + acc * L::acc_cols;
       const int t_base = tt * BN;
 
       if (EPI == GEMM_EPI_PARTIAL) {
@@ -240,12 +244,13 @@ __global__ void __launch_bounds__(kThreads, 1)
         float* out = args.out_f32 + (size_t)sp * args.split_stride + o;
 #pragma unroll 1
         for (int c0 = 0; c0 < BN; c0 += 16) {
-          float v[16];
-          tmem_ld16(taddr + c0, v);
+          float v[16], vl[16];
+          const uint32_t col = (c0 / 64) * 128 + (c0 % 64);
+          tmem_ld16x2(taddr + col, taddr + col + 64, v, vl);
 #pragma unroll
           for (int i = 0; i < 16; ++i) {
             const int t = t_base + c0 + i;
-            if (t < args.M) out[(size_t)t * args.n_out] = v[i];
+            if (t < args.M) out[(size_t)t * args.n_out] = v[i] + vl[i];
           }
         }
       } else if (EPI == GEMM_EPI_SWIGLU) {
@@ -253,8 +258,11 @@ __global__ void __launch_bounds__(kThreads, 1)
         const int f = to * 64 + (row_in_tile & 63);
 #pragma unroll 1
         for (int c0 = 0; c0 < BN; c0 += 16) {
-          float v[16];
-          tmem_ld16(taddr + c0, v);
+          float v[16], vl[16];
+          const uint32_t col = (c0 / 64) * 128 + (c0 % 64);
+          tmem_ld16x2(taddr + col, taddr + col + 64, v, vl);
+#pragma unroll
+          for (int i = 0; i < 16; ++i) v[i] += vl[i];
           if (quarter >= 2) {
 #pragma unroll
             for (int i = 0; i < 16; ++i) stage_up[(row_in_tile - 64) * 17 + i] = v[i];
@@ -267,7 +275,7 @@ __global__ void __launch_bounds__(kThreads, 1)
               const float g = v[i];
               const float up = stage_up[row_in_tile * 17 + i];
               const float h = g / (1.0f + expf(-g)) * up;
-              if (t < args.M) args.out_bf16[(size_t)t * args.ld_out + f] = __float2bfloat16_rn(h);
+              if (t < args.M) split_store(args.out_bf16, t, args.ld_out, f, h);
             }
           }
           named_sync(1, 128);
@@ -278,8 +286,11 @@ __global__ void __launch_bounds__(kThreads, 1)
         const bool row_ok = o < args.n_out;
 #pragma unroll 1
         for (int c0 = 0; c0 < BN; c0 += 16) {
-          float v[16];
-          tmem_ld16(taddr + c0, v);
+          float v[16], vl[16];
+          const uint32_t col = (c0 / 64) * 128 + (c0 % 64);
+          tmem_ld16x2(taddr + col, taddr + col + 64, v, vl);
+#pragma unroll
+          for (int i = 0; i < 16; ++i) v[i] += vl[i];
 #pragma unroll
           for (int i = 0; i < 16; ++i) {
             const int t = t_base + c0 + i;
@@ -338,31 +349,33 @@ static cudaError_t launch_impl(const GemmTcLaunch& L_, cudaStream_t stream, bool
   return cudaLaunchKernelEx(&cfg, kern, *L_.mA0, *L_.mA1, *L_.mA2, *L_.mB, L_.args);
 }
 
+// BN = 64 tokens: 3 stages of 32 KB (two CTAs per SM); BN = 128: 4 stages of 48 KB (one per SM)
+
 uint32_t gemm_tc_smem_bytes(int bn, int epi) {
   switch (epi) {
-    case GEMM_EPI_PARTIAL: return bn == 64 ? SmemLayout<64, 4, GEMM_EPI_PARTIAL>::dyn_bytes : SmemLayout<128, 4, GEMM_EPI_PARTIAL>::dyn_bytes;
-    case GEMM_EPI_SWIGLU: return bn == 64 ? SmemLayout<64, 4, GEMM_EPI_SWIGLU>::dyn_bytes : SmemLayout<128, 4, GEMM_EPI_SWIGLU>::dyn_bytes;
-    default: return bn == 64 ? SmemLayout<64, 4, GEMM_EPI_ARGMAX>::dyn_bytes : SmemLayout<128, 4, GEMM_EPI_ARGMAX>::dyn_bytes;
+    case GEMM_EPI_PARTIAL: return bn == 64 ? SmemLayout<64, 3, GEMM_EPI_PARTIAL>::dyn_bytes : SmemLayout<128, 4, GEMM_EPI_PARTIAL>::dyn_bytes;
+    case GEMM_EPI_SWIGLU: return bn == 64 ? SmemLayout<64, 3, GEMM_EPI_SWIGLU>::dyn_bytes : SmemLayout<128, 4, GEMM_EPI_SWIGLU>::dyn_bytes;
+    default: return bn == 64 ? SmemLayout<64, 3, GEMM_EPI_ARGMAX>::dyn_bytes : SmemLayout<128, 4, GEMM_EPI_ARGMAX>::dyn_bytes;
   }
 }
 
 const void* gemm_tc_function(int bn, int epi) {
   switch (epi) {
     case GEMM_EPI_PARTIAL:
-      return bn == 64 ? (const void*)gemm_tc_kernel<64, 4, GEMM_EPI_PARTIAL> : (const void*)gemm_tc_kernel<128, 4, GEMM_EPI_PARTIAL>;
+      return bn == 64 ? (const void*)gemm_tc_kernel<64, 3, GEMM_EPI_PARTIAL> : (const void*)gemm_tc_kernel<128, 4, GEMM_EPI_PARTIAL>;
     case GEMM_EPI_SWIGLU:
-      return bn == 64 ? (const void*)gemm_tc_kernel<64, 4, GEMM_EPI_SWIGLU> : (const void*)gemm_tc_kernel<128, 4, GEMM_EPI_SWIGLU>;
+      return bn == 64 ? (const void*)gemm_tc_kernel<64, 3, GEMM_EPI_SWIGLU> : (const void*)gemm_tc_kernel<128, 4, GEMM_EPI_SWIGLU>;
     default:
-      return bn == 64 ? (const void*)gemm_tc_kernel<64, 4, GEMM_EPI_ARGMAX> : (const void*)gemm_tc_kernel<128, 4, GEMM_EPI_ARGMAX>;
+      return bn == 64 ? (const void*)gemm_tc_kernel<64, 3, GEMM_EPI_ARGMAX> : (const void*)gemm_tc_kernel<128, 4, GEMM_EPI_ARGMAX>;
   }
 }
 
 cudaError_t gemm_tc_launch(const GemmTcLaunch& L, cudaStream_t stream, bool pdl) {
   if (L.bn == 64) {
     switch (L.epi) {
-      case GEMM_EPI_PARTIAL: return launch_impl<64, 4, GEMM_EPI_PARTIAL>(L, stream, pdl);
-      case GEMM_EPI_SWIGLU: return launch_impl<64, 4, GEMM_EPI_SWIGLU>(L, stream, pdl);
-      case GEMM_EPI_ARGMAX: return launch_impl<64, 4, GEMM_EPI_ARGMAX>(L, stream, pdl);
+      case GEMM_EPI_PARTIAL: return launch_impl<64, 3, GEMM_EPI_PARTIAL>(L, stream, pdl);
+      case GEMM_EPI_SWIGLU: return launch_impl<64, 3, GEMM_EPI_SWIGLU>(L, stream, pdl);
+      case GEMM_EPI_ARGMAX: return launch_impl<64, 3, GEMM_EPI_ARGMAX>(L, stream, pdl);
     }
   } else if (L.bn == 128) {
     switch (L.epi) {

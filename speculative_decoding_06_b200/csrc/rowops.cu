@@ -3,6 +3,8 @@
 // residual add and the next RMSNorm, rotary embedding fused with the K/V cache
 // store, the LM-head argmax reductions, and the fp32 (SIMT) GEMM used by the
 // fp32 model path.
+#include <cooperative_groups.h>
+
 #include "common.cuh"
 #include "kernels.h"
 
@@ -49,10 +51,11 @@ cudaLaunchConfig_t make_cfg(dim3 grid, dim3 block, size_t smem, cudaStream_t s, 
 // One CTA per node.  A node's depth and ancestor set come from walking its
 // parent links up to the root ("EAGLE-3投机解码：树验证器方法", section 树draft vs
 // 链draft: every token sees only its ancestors); its position is P_b + depth.
-template <typename T>
+// SPLIT: write the normalised row as split bf16 (bf16 models); else as T (fp32 models)
+template <typename T, bool SPLIT>
 __global__ void __launch_bounds__(256) embed_meta_kernel(StepView sv, const T* __restrict__ embed,
                                                          const T* __restrict__ norm_w, int d, float eps,
-                                                         float* __restrict__ x, T* __restrict__ xn,
+                                                         float* __restrict__ x, void* __restrict__ xn,
                                                          const double* __restrict__ inv_freq, int half, int mode) {
   __shared__ int s_pos;
   __shared__ float red[8];
@@ -110,8 +113,11 @@ __global__ void __launch_bounds__(256) embed_meta_kernel(StepView sv, const T* _
   }
   ss = block_sum<256>(ss, red);
   const float inv = rsqrtf(ss / (float)d + eps);
-  T* o = xn + (size_t)r * d;
-  for (int k = threadIdx.x; k < d; k += blockDim.x) o[k] = from_f32<T>(xr[k] * inv * to_f32(norm_w[k]));
+  for (int k = threadIdx.x; k < d; k += blockDim.x) {
+    const float v = xr[k] * inv * to_f32(norm_w[k]);
+    if (SPLIT) split_store(reinterpret_cast<__nv_bfloat16*>(xn), r, d, k, v);
+    else reinterpret_cast<T*>(xn)[(size_t)r * d + k] = from_f32<T>(v);
+  }
   pdl_launch_dependents();
 }
 
@@ -121,27 +127,37 @@ cudaError_t launch_embed_meta(int dtype, const StepView& sv, const void* embed, 
   cudaLaunchAttribute attr[1];
   cudaLaunchConfig_t cfg = make_cfg(dim3(sv.M), dim3(256), 0, s, pdl, attr);
   if (dtype == 0)
-    return cudaLaunchKernelEx(&cfg, embed_meta_kernel<float>, sv, (const float*)embed, (const float*)norm_w, d, eps, x,
-                              (float*)xn, inv_freq, half, mode);
-  return cudaLaunchKernelEx(&cfg, embed_meta_kernel<__nv_bfloat16>, sv, (const __nv_bfloat16*)embed,
-                            (const __nv_bfloat16*)norm_w, d, eps, x, (__nv_bfloat16*)xn, inv_freq, half, mode);
+    return cudaLaunchKernelEx(&cfg, embed_meta_kernel<float, false>, sv, (const float*)embed, (const float*)norm_w, d,
+                              eps, x, xn, inv_freq, half, mode);
+  return cudaLaunchKernelEx(&cfg, embed_meta_kernel<__nv_bfloat16, true>, sv, (const __nv_bfloat16*)embed,
+                            (const __nv_bfloat16*)norm_w, d, eps, x, xn, inv_freq, half, mode);
 }
 
 // ---------------------------------------------------------------------------
 // split-K reduction + residual + RMSNorm
 // ---------------------------------------------------------------------------
 // x[r] += sum_s partial[s][r] (fixed order, deterministic); xn[r] = x[r] * rsqrt(mean x^2 + eps) * w.
-template <typename T>
+// A row is shared by a cluster of CL CTAs, each owning d/CL columns; the CTAs
+// exchange their partial sums of squares through distributed shared memory and
+// add them in rank order, so every CTA applies the same normaliser.
+template <typename T, bool SPLIT>
 __global__ void __launch_bounds__(256) residual_norm_kernel(int d, int S, const float* __restrict__ partial,
                                                             size_t split_stride, float* __restrict__ x,
-                                                            T* __restrict__ xn, const T* __restrict__ w, float eps) {
+                                                            void* __restrict__ xn, const T* __restrict__ w, float eps) {
   __shared__ float red[8];
+  __shared__ float cta_ss;
+  namespace cg = cooperative_groups;
+  cg::cluster_group cluster = cg::this_cluster();
+  const int CL = (int)cluster.num_blocks();
+  const int rank = (int)cluster.block_rank();
   pdl_wait();
-  const int r = blockIdx.x;
+  const int r = blockIdx.x / CL;
+  const int cols = d / CL;
+  const int c0 = rank * cols;
   float* xr = x + (size_t)r * d;
   const float* pr = partial + (size_t)r * d;
   float ss = 0.f;
-  for (int k = threadIdx.x * 4; k < d; k += blockDim.x * 4) {
+  for (int k = c0 + threadIdx.x * 4; k < c0 + cols; k += blockDim.x * 4) {
     float4 acc = *reinterpret_cast<const float4*>(xr + k);
     for (int sp = 0; sp < S; ++sp) {
       const float4 p = *reinterpret_cast<const float4*>(pr + sp * split_stride + k);
@@ -151,28 +167,53 @@ __global__ void __launch_bounds__(256) residual_norm_kernel(int d, int S, const 
     ss += acc.x * acc.x + acc.y * acc.y + acc.z * acc.z + acc.w * acc.w;
   }
   ss = block_sum<256>(ss, red);
-  const float inv = rsqrtf(ss / (float)d + eps);
-  T* o = xn + (size_t)r * d;
-  for (int k = threadIdx.x; k < d; k += blockDim.x) o[k] = from_f32<T>(xr[k] * inv * to_f32(w[k]));
+  if (threadIdx.x == 0) cta_ss = ss;
+  cluster.sync();
+  float total = 0.f;
+  for (int q = 0; q < CL; ++q) total += *cluster.map_shared_rank(&cta_ss, q);
+  cluster.sync();  // keep every CTA's cta_ss alive until all have read it
+  const float inv = rsqrtf(total / (float)d + eps);
+  for (int k = c0 + threadIdx.x; k < c0 + cols; k += blockDim.x) {
+    const float v = xr[k] * inv * to_f32(w[k]);
+    if (SPLIT) split_store(reinterpret_cast<__nv_bfloat16*>(xn), r, d, k, v);
+    else reinterpret_cast<T*>(xn)[(size_t)r * d + k] = from_f32<T>(v);
+  }
   pdl_launch_dependents();
+}
+
+int residual_norm_cluster(int d) {
+  // 4 KB-wide slices (one float4 per thread) when the row is wide enough
+  if (d % 4096 == 0 && d >= 4096) return 4;
+  if (d % 2048 == 0 && d >= 2048) return 2;
+  return 1;
 }
 
 cudaError_t launch_residual_norm(int dtype, int M, int d, int S, const float* partial, size_t split_stride, float* x,
                                  void* xn, const void* w, float eps, cudaStream_t s, bool pdl) {
-  cudaLaunchAttribute attr[1];
-  cudaLaunchConfig_t cfg = make_cfg(dim3(M), dim3(256), 0, s, pdl, attr);
+  const int CL = residual_norm_cluster(d);
+  cudaLaunchAttribute attr[2];
+  cudaLaunchConfig_t cfg = make_cfg(dim3(M * CL), dim3(256), 0, s, pdl, attr);
+  attr[cfg.numAttrs].id = cudaLaunchAttributeClusterDimension;
+  attr[cfg.numAttrs].val.clusterDim.x = CL;
+  attr[cfg.numAttrs].val.clusterDim.y = 1;
+  attr[cfg.numAttrs].val.clusterDim.z = 1;
+  cfg.numAttrs += 1;
   if (dtype == 0)
-    return cudaLaunchKernelEx(&cfg, residual_norm_kernel<float>, d, S, partial, split_stride, x, (float*)xn,
+    return cudaLaunchKernelEx(&cfg, residual_norm_kernel<float, false>, d, S, partial, split_stride, x, xn,
                               (const float*)w, eps);
-  return cudaLaunchKernelEx(&cfg, residual_norm_kernel<__nv_bfloat16>, d, S, partial, split_stride, x,
-                            (__nv_bfloat16*)xn, (const __nv_bfloat16*)w, eps);
+  return cudaLaunchKernelEx(&cfg, residual_norm_kernel<__nv_bfloat16, true>, d, S, partial, split_stride, x, xn,
+                            (const __nv_bfloat16*)w, eps);
 }
 
 // ---------------------------------------------------------------------------
 // split-K reduction + rotary embedding + K/V cache store
 // ---------------------------------------------------------------------------
+// grid (node, group of 8 heads of q|k|v)
+constexpr int kRopeHeadsPerCta = 8;
 // Rotate-half pairing: element j and element j + hd/2 of a head form one pair,
 // rotated by pos * theta^(-2j/hd) (table computed in double per step).
+// T is the attention operand type: fp32 for fp32 models, fp16 for bf16 models
+// (q and the K/V cache; 10 mantissa bits at 2 bytes).
 template <typename T>
 __global__ void __launch_bounds__(256) qkv_rope_store_kernel(StepView sv, int S, const float* __restrict__ partial,
                                                              size_t split_stride, int Hq, int Hkv, int hd,
@@ -181,19 +222,21 @@ __global__ void __launch_bounds__(256) qkv_rope_store_kernel(StepView sv, int S,
   const int r = blockIdx.x;
   const int half = hd / 2;
   const int n_cols = (Hq + 2 * Hkv) * hd;
+  const int h_begin = blockIdx.y * kRopeHeadsPerCta;
+  const int h_end = min(Hq + 2 * Hkv, h_begin + kRopeHeadsPerCta);
   const float* pr = partial + (size_t)r * n_cols;
   const int b = sv.row_seq[r];
   const int slot = sv.P_step[b] + sv.row_local[r];
   const int seq = sv.seq_ids[b];
   const bool slot_ok = slot < kv.max_seq;
-  if (!slot_ok && threadIdx.x == 0) set_error(sv.err, SPEC_DEVERR_BOUNDS);
+  if (!slot_ok && threadIdx.x == 0 && blockIdx.y == 0) set_error(sv.err, SPEC_DEVERR_BOUNDS);
   T* kbase = reinterpret_cast<T*>(kv.base) + layer * kv.layer_stride() + seq * kv.seq_stride() + (size_t)slot * hd;
   T* vbase = kbase + kv.kv_stride();
   const float2* cs = sv.rope_cs + (size_t)r * half;
-  const int pairs = (Hq + 2 * Hkv) * half;
+  const int pairs = (h_end - h_begin) * half;
   for (int p = threadIdx.x; p < pairs; p += blockDim.x) {
-    const int h = p / half;
-    const int j = p - h * half;
+    const int h = h_begin + p / half;
+    const int j = p % half;
     const int c1 = h * hd + j;
     const int c2 = c1 + half;
     float v1 = 0.f, v2 = 0.f;
@@ -226,12 +269,13 @@ cudaError_t launch_qkv_rope_store(int dtype, const StepView& sv, int S, const fl
                                   int Hq, int Hkv, int hd, void* q_out, const KvView& kv, int layer, cudaStream_t s,
                                   bool pdl) {
   cudaLaunchAttribute attr[1];
-  cudaLaunchConfig_t cfg = make_cfg(dim3(sv.M), dim3(256), 0, s, pdl, attr);
+  const int groups = (Hq + 2 * Hkv + kRopeHeadsPerCta - 1) / kRopeHeadsPerCta;
+  cudaLaunchConfig_t cfg = make_cfg(dim3(sv.M, groups), dim3(256), 0, s, pdl, attr);
   if (dtype == 0)
     return cudaLaunchKernelEx(&cfg, qkv_rope_store_kernel<float>, sv, S, partial, split_stride, Hq, Hkv, hd,
                               (float*)q_out, kv, layer);
-  return cudaLaunchKernelEx(&cfg, qkv_rope_store_kernel<__nv_bfloat16>, sv, S, partial, split_stride, Hq, Hkv, hd,
-                            (__nv_bfloat16*)q_out, kv, layer);
+  return cudaLaunchKernelEx(&cfg, qkv_rope_store_kernel<__half>, sv, S, partial, split_stride, Hq, Hkv, hd,
+                            (__half*)q_out, kv, layer);
 }
 
 // ---------------------------------------------------------------------------

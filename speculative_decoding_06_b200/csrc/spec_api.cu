@@ -85,10 +85,12 @@ WsLayout make_layout(const spec_config& c) {
   L.err_sticky = take(16);
   L.inv_freq = take(8 * (size_t)(c.head_dim / 2));
   L.x = take(4 * (size_t)L.Mpad * c.hidden);
-  L.xn = take(es * (size_t)L.Mpad * c.hidden);
+  // bf16 models keep GEMM activations as split bf16 (hi and lo rows): 2 x Mpad rows of 2 bytes
+  const size_t arows = c.dtype == SPEC_DTYPE_BF16 ? 2 * (size_t)L.Mpad : (size_t)L.Mpad;
+  L.xn = take(es * arows * c.hidden);
   L.q = take(es * (size_t)L.Mpad * qd);
-  L.attn = take(es * (size_t)L.Mpad * qd);
-  L.hmlp = take(es * (size_t)L.Mpad * c.ffn);
+  L.attn = take(es * arows * qd);
+  L.hmlp = take(es * arows * c.ffn);
   size_t pcols = (size_t)std::max(nqkv, c.hidden) * (c.dtype == SPEC_DTYPE_BF16 ? L.splits_cap : 1);
   if (c.dtype == SPEC_DTYPE_F32) pcols = std::max<size_t>(pcols, std::max<size_t>(2 * (size_t)c.ffn, c.vocab));
   L.partial_bytes = 4 * (size_t)L.Mpad * pcols;
@@ -564,7 +566,8 @@ int run_step(spec_handle* h, int B, const int32_t* seq_ids, const int32_t* token
   CUDA_TRY(h, cudaMemcpyAsync(h->ws, pb, L.p_end, cudaMemcpyHostToDevice, h->stream));
 
   StepPlan sp = make_plan(h, B, M, max_n, max_lk);
-  const bool graph = !(flags & SPEC_NO_GRAPH) && !h->prof;
+  // the legacy default stream cannot be captured: launch directly there
+  const bool graph = !(flags & SPEC_NO_GRAPH) && !h->prof && h->stream != nullptr;
   if (graph) {
     GraphKey key{mode, B, M, max_n, sp.n_chunks, sp.chunk, dbg ? 1 : 0, h->use_pdl ? 1 : 0};
     auto it = h->graphs.find(key);
@@ -759,9 +762,10 @@ int spec_init(const spec_config* cfg, const spec_weights* w, void* kv_cache, siz
     if (!make_tmap(&h->map_lm, h->lm_head, c.vocab, c.hidden, 128)) return bail(SPEC_ERR_CUDA, "tensor map");
     const int bns[2] = {64, 128};
     for (int i = 0; i < 2; ++i) {
-      if (!make_tmap(&h->map_xn[i], h->ws + lay.xn, lay.Mpad, c.hidden, bns[i]) ||
-          !make_tmap(&h->map_attn[i], h->ws + lay.attn, lay.Mpad, qd, bns[i]) ||
-          !make_tmap(&h->map_h[i], h->ws + lay.hmlp, lay.Mpad, c.ffn, bns[i]))
+      // split activations: a tile of BN tokens is 2*BN rows (hi and lo)
+      if (!make_tmap(&h->map_xn[i], h->ws + lay.xn, 2 * (uint64_t)lay.Mpad, c.hidden, 2 * bns[i]) ||
+          !make_tmap(&h->map_attn[i], h->ws + lay.attn, 2 * (uint64_t)lay.Mpad, qd, 2 * bns[i]) ||
+          !make_tmap(&h->map_h[i], h->ws + lay.hmlp, 2 * (uint64_t)lay.Mpad, c.ffn, 2 * bns[i]))
         return bail(SPEC_ERR_CUDA, "tensor map");
     }
     for (int i = 0; i < 2; ++i)
@@ -773,8 +777,8 @@ int spec_init(const spec_config* cfg, const spec_weights* w, void* kv_cache, siz
         int nb = 0;
         if (cudaOccupancyMaxActiveBlocksPerMultiprocessor(&nb, fn, 192, smem) != cudaSuccess || nb < 1)
           return bail(SPEC_ERR_CUDA, "occupancy");
-        // tensor memory: two accumulators of BN columns per CTA, 512 columns per SM
-        h->resident[i][e] = std::min(nb, 512 / (2 * bns[i]));
+        // tensor memory: two accumulators of 2*BN columns (hi and lo) per CTA, 512 columns per SM
+        h->resident[i][e] = std::min(nb, 512 / (4 * bns[i]));
       }
   }
   *out = h;

@@ -66,7 +66,9 @@ class SpecEngine:
                 setattr(self._layers[l], k, lw[k].data_ptr())
         self._w = S.spec_weights(embed=weights["embed"].data_ptr(), final_norm=weights["final_norm"].data_ptr(),
                                  lm_head=weights["lm_head"].data_ptr(), layers=self._layers)
-        self.stream = stream or torch.cuda.current_stream()
+        # a dedicated stream: the legacy default stream cannot be captured into graphs
+        self.stream = stream or torch.cuda.Stream()
+        torch.cuda.synchronize()  # weights and buffers were written on torch's stream
         h = ctypes.c_void_p()
         rc = S.spec_init(ctypes.byref(self.cfg), ctypes.byref(self._w), self.kv.data_ptr(), kvb,
                          self.ws.data_ptr(), wsb, ctypes.c_void_p(self.stream.cuda_stream), ctypes.byref(h))
@@ -126,6 +128,8 @@ class SpecEngine:
                             outputs: Optional[Tuple[torch.Tensor, ...]] = None, flags: int = 0):
         """Queue a step without synchronising; outputs (if given) are int32 device tensors."""
         ptrs = [None] * 4 if outputs is None else [o.data_ptr() if o is not None else None for o in outputs]
+        if outputs is not None:
+            self.stream.wait_stream(torch.cuda.current_stream())
         self._check(S.spec_verify_tree_batch(self.h, len(ids), _ptr(ids), _ptr(tok), _ptr(par), _ptr(off),
                                              ptrs[0], ptrs[1], ptrs[2], ptrs[3], flags | S.SPEC_DEVICE_OUTPUTS))
 
@@ -181,7 +185,7 @@ class SpecEngine:
         self._check(S.spec_sync(self.h))
 
     def kv_view(self) -> torch.Tensor:
-        """The cache as a tensor [layer][2][max_batch][Hkv][max_seq][hd] in the model dtype."""
+        """The cache as a tensor [layer][2][max_batch][Hkv][max_seq][hd] (fp16 for bf16 models, else fp32)."""
         d = self.dims
-        tdt = torch.bfloat16 if d.dtype == "bf16" else torch.float32
+        tdt = torch.float16 if d.dtype == "bf16" else torch.float32
         return self.kv.view(tdt).view(d.n_layers, 2, self.max_batch, d.n_kv_heads, -1, d.head_dim)
