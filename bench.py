@@ -340,6 +340,7 @@ def run_ours(args, rank, world, local_rank):
         "kernel_ms_per_step": kernel_share,
         "e2e": {"value": e2e_value, "unit": UNIT, "h2d_bytes_per_step": h2d, "d2h_bytes_per_step": d2h},
         "gpu_launches": launches * args.steps,
+        "plan": eng.info(1, shape.n, P),
         "clocks": clocks,
     }
     if rank == 0 and world == 1 and not args.no_cpu_baseline and args.layers == 32:

@@ -204,6 +204,10 @@ SPEC_API int spec_profile_read(spec_handle* h, double* ms, int64_t* launches);
 /* Bytes one synchronous verification step copies host->device (parameter
  * block) and device->host (outputs and error word). */
 SPEC_API int spec_io_bytes(spec_handle* h, size_t* h2d, size_t* d2h);
+/* Human-readable execution plan (residency, GEMM tiling and split-K, attention
+ * chunking) for a batch of B trees of n_nodes nodes on prefixes of `prefix`
+ * tokens, written to buf (n bytes, NUL-terminated). */
+SPEC_API int spec_info(spec_handle* h, int B, int n_nodes, int prefix, char* buf, size_t n);
 /* Number of kernels the most recent step enqueued. */
 SPEC_API int spec_step_launches(spec_handle* h);
 

@@ -18,6 +18,7 @@ namespace spec {
 
 __global__ void accept_walk_kernel(WalkArgs w) {
   pdl_wait();
+  pdl_launch_dependents();
   const StepView& sv = w.sv;
   const int b = blockIdx.x;
   const int lane = threadIdx.x;
@@ -84,7 +85,6 @@ __global__ void accept_walk_kernel(WalkArgs w) {
     w.acc_len[b] = count;
     w.bonus[b] = bonus;
   }
-  pdl_launch_dependents();
 }
 
 cudaError_t launch_accept_walk(const WalkArgs& w, cudaStream_t s, bool pdl) {
@@ -105,6 +105,7 @@ __global__ void __launch_bounds__(256) kv_compact_kernel(StepView sv, KvView kv,
                                                          const int32_t* __restrict__ acc_nodes, int max_nodes) {
   extern __shared__ __align__(16) uint8_t stage[];
   pdl_wait();
+  pdl_launch_dependents();
   const int b = blockIdx.y;
   const int a = acc_len[b];
   if (a <= 0) return;
@@ -133,7 +134,6 @@ __global__ void __launch_bounds__(256) kv_compact_kernel(StepView sv, KvView kv,
     const int dst = P + 1 + d;
     *reinterpret_cast<uint4*>(base + (size_t)dst * row_bytes + c * 16) = *reinterpret_cast<const uint4*>(stage + (size_t)v * 16);
   }
-  pdl_launch_dependents();
 }
 
 cudaError_t kv_compact_configure(size_t smem) {

@@ -14,8 +14,9 @@
 // fp16 mma.sync tiles with fp32 accumulation and an fp32 online softmax (quad
 // shuffles); the ancestor
 // mask applies only to keys at or beyond P_b.  Each CTA writes an fp32 partial
-// (normalised output + log-sum-exp); a merge kernel combines the chunks and
-// writes the output as split bf16 for the O-projection GEMM.
+// (normalised output + log-sum-exp); the last CTA of each (sequence, kv head,
+// row block) to finish combines the chunks and writes the output as split bf16
+// for the O-projection GEMM.
 //
 // fp32 path: one warp per (node, head), exact fp32 scalar arithmetic.
 #include "common.cuh"
@@ -71,7 +72,13 @@ __global__ void __launch_bounds__(128) attn_chunk_f16_kernel(AttnArgs a) {
   __half* sK = sQ + kRowsPerCta * kStride;          // [2][64][kStride]
   __half* sV = sK + 2 * kKeyBlock * kStride;        // [2][64][kStride]
 
+  // The chunks of one (sequence, kv head, row block) form a thread-block
+  // cluster along x: each writes its partial, signals every peer, and the
+  // peers then merge disjoint row slices.
+  __shared__ __align__(8) uint64_t donebar;
+  __shared__ int s_ok;
   pdl_wait();
+  pdl_launch_dependents();
   const StepView& sv = a.sv;
   const int hd = 128;
   const int Hkv = a.kv.Hkv;
@@ -79,16 +86,22 @@ __global__ void __launch_bounds__(128) attn_chunk_f16_kernel(AttnArgs a) {
   const int bk = blockIdx.z;
   const int b = bk / Hkv;
   const int kvh = bk - b * Hkv;
-  if (b >= sv.B) return;
-  const int base = sv.node_off[b];
-  const int n_b = sv.node_off[b + 1] - base;
+  const bool b_ok = b < sv.B;
+  const int base = b_ok ? sv.node_off[b] : 0;
+  const int n_b = b_ok ? sv.node_off[b + 1] - base : 0;
   const int rows = n_b * G;
   const int row0 = blockIdx.y * kRowsPerCta;
-  if (row0 >= rows) return;
-  const int P = sv.P_step[b];
+  const int P = b_ok ? sv.P_step[b] : 0;
   const int Lk = P + n_b;
+  const int nc = (Lk + a.chunk - 1) / a.chunk;  // chunks this sequence needs (<= cluster size)
+  if (threadIdx.x == 0) {
+    mbar_init(&donebar, nc > 0 ? nc : 1);
+    fence_barrier_init();
+  }
+  cluster_sync_all();  // every barrier is initialised before any peer arrives
+  if (!b_ok || row0 >= rows) return;
   const int c0 = blockIdx.x * a.chunk;
-  if (c0 >= Lk) return;
+  if (c0 >= Lk) return;  // this chunk lies beyond the sequence: no partial, no signal
   const int c1 = min(c0 + a.chunk, Lk);
   const int seq = sv.seq_ids[b];
 
@@ -267,44 +280,50 @@ __global__ void __launch_bounds__(128) attn_chunk_f16_kernel(AttnArgs a) {
     }
     if (t4 == 0) a.part_lse[prow * a.n_chunks + blockIdx.x] = any ? m_run[hr] + log2f(l_run[hr]) : -INFINITY;
   }
-  pdl_launch_dependents();
-}
 
-// one warp per (node, head): weights 2^(lse_c - max) over the sequence's chunks;
-// the result is written as split bf16 (hi and lo rows) for the O projection
-__global__ void attn_merge_kernel(AttnArgs a) {
-  pdl_wait();
-  const int hd = 128;
-  const int w = blockIdx.x * (blockDim.x >> 5) + (threadIdx.x >> 5);
-  const int lane = threadIdx.x & 31;
-  const StepView& sv = a.sv;
-  if (w >= sv.M * a.Hq) return;
-  const int r = w / a.Hq;
-  const int b = sv.row_seq[r];
-  const int n_b = sv.node_off[b + 1] - sv.node_off[b];
-  const int Lk = sv.P_step[b] + n_b;
-  const int nc = min(a.n_chunks, (Lk + a.chunk - 1) / a.chunk);
-  const float* lse = a.part_lse + (size_t)w * a.n_chunks;
-  float mx = -INFINITY;
-  for (int c = 0; c < nc; ++c) mx = fmaxf(mx, lse[c]);
-  float4 acc = make_float4(0.f, 0.f, 0.f, 0.f);
-  float wsum = 0.f;
-  for (int c = 0; c < nc; ++c) {
-    if (lse[c] == -INFINITY) continue;
-    const float wt = exp2f(lse[c] - mx);
-    wsum += wt;
-    const float4 v = *reinterpret_cast<const float4*>(a.part_o + ((size_t)w * a.n_chunks + c) * hd + lane * 4);
-    acc.x += wt * v.x; acc.y += wt * v.y; acc.z += wt * v.z; acc.w += wt * v.w;
+  // ---- signal the nc chunk CTAs of this row block, wait for theirs, then merge
+  // this CTA's slice of the rows over all chunks, in chunk order:
+  // weights 2^(lse_c - max), output written as split bf16 for the O projection
+  __threadfence();
+  __syncthreads();
+  if (tid == 0) {
+    for (int r = 0; r < nc; ++r) mbar_arrive_remote(&donebar, (uint32_t)r);
+    s_ok = mbar_wait_cluster(&donebar, 0, sv.err) ? 1 : 0;
   }
-  const float inv = wsum > 0.f ? 1.f / wsum : 0.f;
+  __syncthreads();
+  if (!s_ok) return;
   __nv_bfloat16* out = reinterpret_cast<__nv_bfloat16*>(a.out);
   const int ld = a.Hq * hd;
-  const int col = (w - r * a.Hq) * hd + lane * 4;
-  split_store(out, r, ld, col + 0, acc.x * inv);
-  split_store(out, r, ld, col + 1, acc.y * inv);
-  split_store(out, r, ld, col + 2, acc.z * inv);
-  split_store(out, r, ld, col + 3, acc.w * inv);
-  pdl_launch_dependents();
+  const int rows_here = min(kRowsPerCta, rows - row0);
+  const int per = (rows_here + nc - 1) / nc;
+  const int r_begin = blockIdx.x * per;
+  const int r_end = min(rows_here, r_begin + per);
+  for (int rr = r_begin + warp; rr < r_end; rr += 4) {
+    const int qr = row0 + rr;
+    const int node = qr / G;
+    const int h = kvh * G + (qr - node * G);
+    const size_t prow = (size_t)(base + node) * a.Hq + h;
+    const float* lse = a.part_lse + prow * a.n_chunks;
+    float mx = -INFINITY;
+    for (int c = lane; c < nc; c += 32) mx = fmaxf(mx, __ldcg(lse + c));  // written by peer CTAs
+    mx = warp_max(mx);
+    float4 acc = make_float4(0.f, 0.f, 0.f, 0.f);
+    float wsum = 0.f;
+    for (int c = 0; c < nc; ++c) {
+      const float l = __ldcg(lse + c);
+      if (l == -INFINITY) continue;
+      const float wt = exp2f(l - mx);
+      wsum += wt;
+      const float4 v = __ldcg(reinterpret_cast<const float4*>(a.part_o + (prow * a.n_chunks + c) * hd + lane * 4));
+      acc.x += wt * v.x; acc.y += wt * v.y; acc.z += wt * v.z; acc.w += wt * v.w;
+    }
+    const float inv = wsum > 0.f ? 1.f / wsum : 0.f;
+    const int col = h * hd + lane * 4;
+    split_store(out, base + node, ld, col + 0, acc.x * inv);
+    split_store(out, base + node, ld, col + 1, acc.y * inv);
+    split_store(out, base + node, ld, col + 2, acc.z * inv);
+    split_store(out, base + node, ld, col + 3, acc.w * inv);
+  }
 }
 
 // fp32 path: one warp per (node, head); keys visited in slot order with an
@@ -367,8 +386,11 @@ __global__ void attn_f32_kernel(AttnArgs a) {
 size_t attention_smem_bytes() { return (size_t)(kRowsPerCta + 4 * kKeyBlock) * kStride * sizeof(__half); }
 
 cudaError_t attention_configure() {
-  return cudaFuncSetAttribute(attn_chunk_f16_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
-                              (int)attention_smem_bytes());
+  cudaError_t e = cudaFuncSetAttribute(attn_chunk_f16_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                       (int)attention_smem_bytes());
+  if (e != cudaSuccess) return e;
+  return cudaFuncSetAttribute(attn_chunk_f16_kernel, cudaFuncAttributePreferredSharedMemoryCarveout,
+                              (int)cudaSharedmemCarveoutMaxShared);
 }
 
 cudaError_t launch_attention(int dtype, const AttnArgs& a, cudaStream_t s, bool pdl) {
@@ -378,7 +400,7 @@ cudaError_t launch_attention(int dtype, const AttnArgs& a, cudaStream_t s, bool 
     return cudaGetLastError();
   }
   const size_t smem = attention_smem_bytes();
-  cudaLaunchAttribute attr[1];
+  cudaLaunchAttribute attr[2];
   attr[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
   attr[0].val.programmaticStreamSerializationAllowed = 1;
   cudaLaunchConfig_t cfg = {};
@@ -386,16 +408,15 @@ cudaError_t launch_attention(int dtype, const AttnArgs& a, cudaStream_t s, bool 
   cfg.blockDim = dim3(128);
   cfg.dynamicSmemBytes = smem;
   cfg.stream = s;
+  int na = pdl ? 1 : 0;
+  attr[na].id = cudaLaunchAttributeClusterDimension;
+  attr[na].val.clusterDim.x = a.n_chunks;
+  attr[na].val.clusterDim.y = 1;
+  attr[na].val.clusterDim.z = 1;
+  ++na;
   cfg.attrs = attr;
-  cfg.numAttrs = pdl ? 1 : 0;
-  cudaError_t e = cudaLaunchKernelEx(&cfg, attn_chunk_f16_kernel, a);
-  if (e != cudaSuccess) return e;
-  cudaLaunchConfig_t cfg2 = cfg;
-  const int warps = a.sv.M * a.Hq;
-  cfg2.gridDim = dim3((warps + 7) / 8);
-  cfg2.blockDim = dim3(256);
-  cfg2.dynamicSmemBytes = 0;
-  return cudaLaunchKernelEx(&cfg2, attn_merge_kernel, a);
+  cfg.numAttrs = na;
+  return cudaLaunchKernelEx(&cfg, attn_chunk_f16_kernel, a);
 }
 
 }  // namespace spec

@@ -48,9 +48,13 @@ struct SmemLayout {
   static constexpr uint32_t a_off = 0;
   static constexpr uint32_t b_off = a_off + STAGES * kABytes;
   static constexpr uint32_t epi_off = b_off + STAGES * kBBytes;
-  // SWIGLU stages up values [64][17] (padded row: conflict-free); ARGMAX keeps per-warp results [4][BN]
-  static constexpr uint32_t epi_bytes =
-      EPI == GEMM_EPI_SWIGLU ? 64 * 17 * 4 : (EPI == GEMM_EPI_ARGMAX ? 4 * BN * sizeof(Top2) : 0);
+  // per-token norm scale r[BN], then: SWIGLU stages up values [64][17] (padded
+  // row: conflict-free); ARGMAX keeps per-warp results [4][BN]; RESID keeps
+  // per-warp sums of squares [4][BN]
+  static constexpr uint32_t epi_extra =
+      EPI == GEMM_EPI_SWIGLU ? 64 * 17 * 4
+                             : (EPI == GEMM_EPI_ARGMAX ? 4 * BN * sizeof(Top2) : (EPI == GEMM_EPI_RESID ? 4 * BN * 4 : 0));
+  static constexpr uint32_t epi_bytes = BN * 4 + epi_extra;
   static constexpr uint32_t bar_off = (epi_off + epi_bytes + 7) & ~7u;
   static constexpr uint32_t n_bars = 2 * STAGES + 4;
   static constexpr uint32_t misc_off = bar_off + n_bars * 8;
@@ -82,12 +86,24 @@ __global__ void __launch_bounds__(kThreads, 1)
   uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(smem + L::misc_off);
   volatile int* abort_flag = reinterpret_cast<volatile int*>(smem + L::misc_off + 4);
   volatile int* ep_ok = reinterpret_cast<volatile int*>(smem + L::misc_off + 8);
+  volatile int* ep_last = reinterpret_cast<volatile int*>(smem + L::misc_off + 12);
 
   const int warp = threadIdx.x >> 5;
   const int lane = threadIdx.x & 31;
 
   const int KB = args.K / kTileK;
-  const int units = args.tiles_o * args.splits * args.tiles_t;
+  // Work: tiles (row tile, token tile).  With split-K (S = args.splits > 1)
+  // the grid is exactly tiles x S CTAs, all co-resident, and CTA b computes
+  // split b % S of tile b / S; the S CTAs of a tile meet at an arrival counter
+  // and then share the tile's finishing work.  Without split-K, CTAs step
+  // through the tiles round-robin.
+  const int S = args.splits;
+  const int sp = S > 1 ? (int)blockIdx.x % S : 0;
+  const int cid = S > 1 ? (int)blockIdx.x / S : (int)blockIdx.x;
+  const int ncl = S > 1 ? (int)gridDim.x / S : (int)gridDim.x;
+  const int tiles = args.tiles_o * args.tiles_t;
+  const int kb0 = sp * args.kb_per_split;
+  const int kb1 = min(kb0 + args.kb_per_split, KB);
 
   if (threadIdx.x == 0) {
     for (int s = 0; s < STAGES; ++s) {
@@ -116,42 +132,58 @@ __global__ void __launch_bounds__(kThreads, 1)
   tc_fence_after();
   const uint32_t tmem_base = *tmem_slot;
 
-  // everything above touched only this CTA's own state; activations written by
-  // the previous kernel are read only after this point
+  // Weights never depend on the previous kernel: the producer starts streaming
+  // the first stages' weight tiles before waiting for it (programmatic
+  // dependent launch), and adds the activation tiles once it has finished.
+  const bool producer = (warp == 0) && elect_one();
+  uint64_t pol_w = 0, pol_x = 0;
+  int pre = 0;  // stages whose weight tile was issued before the wait
+  auto load_a = [&](uint8_t* sa, uint64_t* bar, int kx, int to) {
+    if (EPI == GEMM_EPI_SWIGLU) {
+      tma_load_2d(sa, &mA0, bar, kx, to * 64, pol_w);
+      tma_load_2d(sa + kABytes / 2, &mA1, bar, kx, to * 64, pol_w);
+    } else {
+      const int row = to * kTileO;
+      if (row < args.seg_rows[0]) {
+        tma_load_2d(sa, &mA0, bar, kx, row, pol_w);
+      } else if (row < args.seg_rows[0] + args.seg_rows[1]) {
+        tma_load_2d(sa, &mA1, bar, kx, row - args.seg_rows[0], pol_w);
+      } else {
+        tma_load_2d(sa, &mA2, bar, kx, row - args.seg_rows[0] - args.seg_rows[1], pol_w);
+      }
+    }
+  };
+  if (producer && cid < tiles) {
+    pol_w = policy_evict_first();
+    pol_x = policy_evict_last();
+    const int to = cid / args.tiles_t;
+    pre = min(STAGES, kb1 - kb0);
+    for (int s = 0; s < pre; ++s) {
+      mbar_arrive_expect_tx(&full[s], kABytes + L::kBBytes);
+      load_a(smem + L::a_off + s * kABytes, &full[s], (kb0 + s) * kTileK, to);
+    }
+  }
+  // activations written by the previous kernel are read only after this point
   pdl_wait();
+  pdl_launch_dependents();
 
   if (warp == 0) {
     // ------------------------------------------------------------------ producer
-    if (elect_one()) {
-      const uint64_t pol_w = policy_evict_first();
-      const uint64_t pol_x = policy_evict_last();
+    if (producer) {
       int stage = 0;
       uint32_t phase = 0;
-      for (int u = blockIdx.x; u < units && !*abort_flag; u += gridDim.x) {
-        const int tt = u % args.tiles_t;
-        const int rest = u / args.tiles_t;
-        const int sp = rest % args.splits;
-        const int to = rest / args.splits;
-        const int kb0 = sp * args.kb_per_split;
-        const int kb1 = min(kb0 + args.kb_per_split, KB);
-        for (int kb = kb0; kb < kb1; ++kb) {
-          if (!mbar_wait(&empty[stage], phase ^ 1, args.err, abort_flag)) break;
+      int issued = 0;
+      for (int ut = cid; ut < tiles && !*abort_flag; ut += ncl) {
+        const int tt = ut % args.tiles_t;
+        const int to = ut / args.tiles_t;
+        for (int kb = kb0; kb < kb1; ++kb, ++issued) {
           uint8_t* sa = smem + L::a_off + stage * kABytes;
           uint8_t* sb = smem + L::b_off + stage * L::kBBytes;
-          mbar_arrive_expect_tx(&full[stage], kABytes + L::kBBytes);
           const int kx = kb * kTileK;
-          if (EPI == GEMM_EPI_SWIGLU) {
-            tma_load_2d(sa, &mA0, &full[stage], kx, to * 64, pol_w);
-            tma_load_2d(sa + kABytes / 2, &mA1, &full[stage], kx, to * 64, pol_w);
-          } else {
-            int row = to * kTileO;
-            if (row < args.seg_rows[0]) {
-              tma_load_2d(sa, &mA0, &full[stage], kx, row, pol_w);
-            } else if (row < args.seg_rows[0] + args.seg_rows[1]) {
-              tma_load_2d(sa, &mA1, &full[stage], kx, row - args.seg_rows[0], pol_w);
-            } else {
-              tma_load_2d(sa, &mA2, &full[stage], kx, row - args.seg_rows[0] - args.seg_rows[1], pol_w);
-            }
+          if (issued >= pre) {
+            if (!mbar_wait(&empty[stage], phase ^ 1, args.err, abort_flag)) break;
+            mbar_arrive_expect_tx(&full[stage], kABytes + L::kBBytes);
+            load_a(sa, &full[stage], kx, to);
           }
           tma_load_2d(sb, &mB, &full[stage], kx, tt * 2 * BN, pol_x);
           if (++stage == STAGES) {
@@ -178,11 +210,7 @@ __global__ void __launch_bounds__(kThreads, 1)
       int j = 0;
       int last_acc = -1;
       uint32_t last_phase = 0;
-      for (int u = blockIdx.x; u < units && !*abort_flag; u += gridDim.x, ++j) {
-        const int rest = u / args.tiles_t;
-        const int sp = rest % args.splits;
-        const int kb0 = sp * args.kb_per_split;
-        const int kb1 = min(kb0 + args.kb_per_split, KB);
+      for (int ut = cid; ut < tiles && !*abort_flag; ut += ncl, ++j) {
         const int acc = j & 1;
         const uint32_t acc_phase = (j >> 1) & 1;
         if (!mbar_wait(&tempty[acc], acc_phase ^ 1, args.err, abort_flag)) break;
@@ -222,14 +250,28 @@ __global__ void __launch_bounds__(kThreads, 1)
     const int quarter = warp & 3;  // TMEM lanes [32*quarter, 32*quarter + 32)
     const int row_in_tile = quarter * 32 + lane;
     const int ep_tid = threadIdx.x - 64;  // 0..127
+    const int ep_warp = ep_tid >> 5;
+    float* r_s = reinterpret_cast<float*>(smem + L::epi_off);  // [BN]
+    uint8_t* epx = smem + L::epi_off + BN * 4;
     int j = 0;
-    for (int u = blockIdx.x; u < units; u += gridDim.x, ++j) {
-      const int tt = u % args.tiles_t;
-      const int rest = u / args.tiles_t;
-      const int sp = rest % args.splits;
-      const int to = rest / args.splits;
+    for (int ut = cid; ut < tiles; ut += ncl, ++j) {
+      const int tt = ut % args.tiles_t;
+      const int to = ut / args.tiles_t;
       const int acc = j & 1;
       const uint32_t acc_phase = (j >> 1) & 1;
+      const int t_base = tt * BN;
+      const int t_end = min(t_base + BN, args.M);
+      // per-token scale of the folded RMSNorm (1 when the operand is not normalised)
+      for (int c = ep_tid; c < BN; c += 128) {
+        const int t = t_base + c;
+        float r = 1.f;
+        if (args.ss_in && t < args.M) {
+          float ssum = 0.f;
+          for (int i = 0; i < args.n_ss; ++i) ssum += args.ss_in[(size_t)i * args.ss_ld + t];
+          r = rsqrtf(ssum / (float)args.norm_d + args.eps);
+        }
+        r_s[c] = r;
+      }
       // one thread waits, the four epilogue warps then agree on the outcome, so
       // that no warp can be left alone at a named barrier
       if (ep_tid == 0) *ep_ok = mbar_wait(&tfull[acc], acc_phase, args.err, abort_flag) ? 1 : 0;
@@ -237,11 +279,11 @@ __global__ void __launch_bounds__(kThreads, 1)
       if (!*ep_ok) break;
       tc_fence_after();
       const uint32_t taddr = tmem_base + ((uint32_t)(quarter * 32) << 16) + acc * L::acc_cols;
-      const int t_base = tt * BN;
 
-      if (EPI == GEMM_EPI_PARTIAL) {
+      if (EPI == GEMM_EPI_QKV || EPI == GEMM_EPI_RESID) {
+        // 1) this split's partial sums
         const int o = to * kTileO + row_in_tile;
-        float* out = args.out_f32 + (size_t)sp * args.split_stride + o;
+        float* out = args.part + (size_t)sp * args.split_stride + o;
 #pragma unroll 1
         for (int c0 = 0; c0 < BN; c0 += 16) {
           float v[16], vl[16];
@@ -253,8 +295,117 @@ __global__ void __launch_bounds__(kThreads, 1)
             if (t < args.M) out[(size_t)t * args.n_out] = v[i] + vl[i];
           }
         }
+        tc_fence_before();
+        mbar_arrive(&tempty[acc]);  // the accumulator is free for the next unit
+        // 2) the S split CTAs of the tile meet at its arrival counter, then all of
+        //    them share the finishing work, each taking 1/S of the tile's tokens
+        int* ctr = args.counters + 2 * ut;
+        __threadfence();
+        named_sync(2, 128);
+        if (ep_tid == 0) {
+          atomicAdd(ctr, 1);
+          *ep_ok = spin_until_geq(ctr, S, args.err) ? 1 : 0;
+        }
+        named_sync(2, 128);
+        if (!*ep_ok) break;
+        const int per = (t_end - t_base + S - 1) / S;
+        const int t0s = t_base + sp * per;
+        const int t1s = min(t_end, t0s + per);
+        const float* part = args.part;
+        const size_t sst = args.split_stride;
+        if (EPI == GEMM_EPI_QKV) {
+          // tile `to` is one head of q|k|v (head_dim 128): rotate-half pairs (c, c+64)
+          const int hh = to;
+          const int c = ep_tid & 63;
+          const int par = ep_tid >> 6;
+          for (int tb = t0s; tb < t1s; tb += 8) {
+            float v1[4], v2[4];
+#pragma unroll
+            for (int i = 0; i < 4; ++i) v1[i] = v2[i] = 0.f;
+            for (int q = 0; q < S; ++q) {  // L2 loads: the peers wrote these
+#pragma unroll
+              for (int i = 0; i < 4; ++i) {
+                const int t = tb + 2 * i + par;
+                if (t < t1s) {
+                  const float* pr = part + q * sst + (size_t)t * args.n_out + hh * 128 + c;
+                  v1[i] += __ldcg(pr);
+                  v2[i] += __ldcg(pr + 64);
+                }
+              }
+            }
+#pragma unroll
+            for (int i = 0; i < 4; ++i) {
+              const int t = tb + 2 * i + par;
+              if (t >= t1s) continue;
+              const float r = r_s[t - t_base];
+              float a1 = v1[i] * r, a2 = v2[i] * r;
+              if (hh < args.Hq + args.Hkv) {
+                const float2 cs = args.rope_cs[(size_t)t * 64 + c];
+                const float o1 = a1 * cs.x - a2 * cs.y;
+                const float o2 = a2 * cs.x + a1 * cs.y;
+                a1 = o1;
+                a2 = o2;
+              }
+              if (hh < args.Hq) {
+                __half* qo = args.q_out + ((size_t)t * args.Hq + hh) * 128;
+                qo[c] = __float2half_rn(a1);
+                qo[c + 64] = __float2half_rn(a2);
+              } else {
+                const int b = args.row_seq[t];
+                const int slot = args.P_step[b] + args.row_local[t];
+                if (slot < args.max_seq) {
+                  const bool is_k = hh < args.Hq + args.Hkv;
+                  const int kvh = is_k ? hh - args.Hq : hh - args.Hq - args.Hkv;
+                  __half* dst = (is_k ? args.k_cache : args.v_cache) + args.seq_ids[b] * args.kv_seq_stride +
+                                kvh * args.kv_head_stride + (size_t)slot * 128;
+                  dst[c] = __float2half_rn(a1);
+                  dst[c + 64] = __float2half_rn(a2);
+                } else if (c == 0) {
+                  set_error(args.err, SPEC_DEVERR_BOUNDS);
+                }
+              }
+            }
+          }
+        } else {
+          // residual update of this tile's 128 columns for this CTA's tokens, the
+          // next operand x*w (split bf16) and per-token sums of squares of x
+          float* ssw = reinterpret_cast<float*>(epx);  // [4][BN]
+          const int col = to * kTileO + ep_tid;
+          const float w = __bfloat162float(args.norm_w_next[col]);
+          for (int tb = t0s; tb < t1s; tb += 8) {
+            float xv[8];
+#pragma unroll
+            for (int i = 0; i < 8; ++i)
+              xv[i] = (tb + i < t1s) ? args.x[(size_t)(tb + i) * args.n_out + col] : 0.f;
+            for (int q = 0; q < S; ++q) {
+#pragma unroll
+              for (int i = 0; i < 8; ++i)
+                if (tb + i < t1s) xv[i] += __ldcg(part + q * sst + (size_t)(tb + i) * args.n_out + col);
+            }
+#pragma unroll
+            for (int i = 0; i < 8; ++i) {
+              const int t = tb + i;
+              if (t >= t1s) continue;
+              args.x[(size_t)t * args.n_out + col] = xv[i];
+              split_store(args.xn_out, t, args.n_out, col, xv[i] * w);
+              const float sq = warp_sum(xv[i] * xv[i]);
+              if (lane == 0) ssw[ep_warp * BN + (t - t_base)] = sq;
+            }
+          }
+          named_sync(2, 128);
+          for (int t = t0s + ep_tid; t < t1s; t += 128) {
+            const int c = t - t_base;
+            args.ss_out[(size_t)to * args.ss_ld + t] = ssw[c] + ssw[BN + c] + ssw[2 * BN + c] + ssw[3 * BN + c];
+          }
+        }
+        // the last CTA of the tile to leave resets its counters for the next launch
+        named_sync(2, 128);
+        if (ep_tid == 0 && atomicAdd(ctr + 1, 1) == S - 1) {
+          ctr[0] = 0;
+          ctr[1] = 0;
+        }
       } else if (EPI == GEMM_EPI_SWIGLU) {
-        float* stage_up = reinterpret_cast<float*>(smem + L::epi_off);  // [64][17]
+        float* stage_up = reinterpret_cast<float*>(epx);  // [64][17]
         const int f = to * 64 + (row_in_tile & 63);
 #pragma unroll 1
         for (int c0 = 0; c0 < BN; c0 += 16) {
@@ -262,7 +413,7 @@ __global__ void __launch_bounds__(kThreads, 1)
           const uint32_t col = (c0 / 64) * 128 + (c0 % 64);
           tmem_ld16x2(taddr + col, taddr + col + 64, v, vl);
 #pragma unroll
-          for (int i = 0; i < 16; ++i) v[i] += vl[i];
+          for (int i = 0; i < 16; ++i) v[i] = (v[i] + vl[i]) * r_s[c0 + i];
           if (quarter >= 2) {
 #pragma unroll
             for (int i = 0; i < 16; ++i) stage_up[(row_in_tile - 64) * 17 + i] = v[i];
@@ -280,8 +431,10 @@ __global__ void __launch_bounds__(kThreads, 1)
           }
           named_sync(1, 128);
         }
+        tc_fence_before();
+        mbar_arrive(&tempty[acc]);
       } else {  // GEMM_EPI_ARGMAX
-        Top2* wres = reinterpret_cast<Top2*>(smem + L::epi_off);  // [4][BN]
+        Top2* wres = reinterpret_cast<Top2*>(epx);  // [4][BN]
         const int o = to * kTileO + row_in_tile;
         const bool row_ok = o < args.n_out;
 #pragma unroll 1
@@ -290,7 +443,7 @@ __global__ void __launch_bounds__(kThreads, 1)
           const uint32_t col = (c0 / 64) * 128 + (c0 % 64);
           tmem_ld16x2(taddr + col, taddr + col + 64, v, vl);
 #pragma unroll
-          for (int i = 0; i < 16; ++i) v[i] += vl[i];
+          for (int i = 0; i < 16; ++i) v[i] = (v[i] + vl[i]) * r_s[c0 + i];
 #pragma unroll
           for (int i = 0; i < 16; ++i) {
             const int t = t_base + c0 + i;
@@ -303,6 +456,8 @@ __global__ void __launch_bounds__(kThreads, 1)
             if (lane == i) wres[quarter * BN + c0 + i] = x;
           }
         }
+        tc_fence_before();
+        mbar_arrive(&tempty[acc]);
         named_sync(1, 128);
         for (int c = ep_tid; c < BN; c += 128) {
           Top2 r = wres[c];
@@ -311,21 +466,18 @@ __global__ void __launch_bounds__(kThreads, 1)
           const int t = t_base + c;
           if (t < args.M) args.top_part[(size_t)to * args.top_ld + t] = r;
         }
-        named_sync(1, 128);
       }
-      tc_fence_before();
-      mbar_arrive(&tempty[acc]);
+      named_sync(2, 128);  // r_s and the staging areas are reused by the next unit
     }
   }
 
-  // let the next kernel in the stream begin its prologue
-  pdl_launch_dependents();
   tc_fence_before();
   __syncthreads();
   if (warp == 1) {
     tc_fence_after();
     tmem_dealloc(tmem_base, L::tmem_cols);
   }
+
 }
 
 // ---------------------------------------------------------------------------
@@ -341,49 +493,48 @@ static cudaError_t launch_impl(const GemmTcLaunch& L_, cudaStream_t stream, bool
   cfg.blockDim = dim3(kThreads);
   cfg.dynamicSmemBytes = L::dyn_bytes;
   cfg.stream = stream;
-  cudaLaunchAttribute attr[1];
-  attr[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
-  attr[0].val.programmaticStreamSerializationAllowed = 1;
+  cudaLaunchAttribute attr[2];
+  int na = 0;
+  if (pdl) {
+    attr[na].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+    attr[na].val.programmaticStreamSerializationAllowed = 1;
+    ++na;
+  }
   cfg.attrs = attr;
-  cfg.numAttrs = pdl ? 1 : 0;
+  cfg.numAttrs = na;
   return cudaLaunchKernelEx(&cfg, kern, *L_.mA0, *L_.mA1, *L_.mA2, *L_.mB, L_.args);
 }
 
 // BN = 64 tokens: 3 stages of 32 KB (two CTAs per SM); BN = 128: 4 stages of 48 KB (one per SM)
 
-uint32_t gemm_tc_smem_bytes(int bn, int epi) {
-  switch (epi) {
-    case GEMM_EPI_PARTIAL: return bn == 64 ? SmemLayout<64, 3, GEMM_EPI_PARTIAL>::dyn_bytes : SmemLayout<128, 4, GEMM_EPI_PARTIAL>::dyn_bytes;
-    case GEMM_EPI_SWIGLU: return bn == 64 ? SmemLayout<64, 3, GEMM_EPI_SWIGLU>::dyn_bytes : SmemLayout<128, 4, GEMM_EPI_SWIGLU>::dyn_bytes;
-    default: return bn == 64 ? SmemLayout<64, 3, GEMM_EPI_ARGMAX>::dyn_bytes : SmemLayout<128, 4, GEMM_EPI_ARGMAX>::dyn_bytes;
+#define SPEC_GEMM_DISPATCH(BN, ST, EXPR_T)                      \
+  switch (epi) {                                               \
+    case GEMM_EPI_QKV: return EXPR_T(BN, ST, GEMM_EPI_QKV);       \
+    case GEMM_EPI_SWIGLU: return EXPR_T(BN, ST, GEMM_EPI_SWIGLU); \
+    case GEMM_EPI_ARGMAX: return EXPR_T(BN, ST, GEMM_EPI_ARGMAX); \
+    case GEMM_EPI_RESID: return EXPR_T(BN, ST, GEMM_EPI_RESID);   \
   }
+
+#define SPEC_SMEM_OF(BN, ST, E) SmemLayout<BN, ST, E>::dyn_bytes
+#define SPEC_FN_OF(BN, ST, E) (const void*)gemm_tc_kernel<BN, ST, E>
+#define SPEC_LAUNCH_OF(BN, ST, E) launch_impl<BN, ST, E>(L, stream, pdl)
+
+uint32_t gemm_tc_smem_bytes(int bn, int epi) {
+  if (bn == 64) { SPEC_GEMM_DISPATCH(64, 3, SPEC_SMEM_OF) }
+  else { SPEC_GEMM_DISPATCH(128, 4, SPEC_SMEM_OF) }
+  return 0;
 }
 
 const void* gemm_tc_function(int bn, int epi) {
-  switch (epi) {
-    case GEMM_EPI_PARTIAL:
-      return bn == 64 ? (const void*)gemm_tc_kernel<64, 3, GEMM_EPI_PARTIAL> : (const void*)gemm_tc_kernel<128, 4, GEMM_EPI_PARTIAL>;
-    case GEMM_EPI_SWIGLU:
-      return bn == 64 ? (const void*)gemm_tc_kernel<64, 3, GEMM_EPI_SWIGLU> : (const void*)gemm_tc_kernel<128, 4, GEMM_EPI_SWIGLU>;
-    default:
-      return bn == 64 ? (const void*)gemm_tc_kernel<64, 3, GEMM_EPI_ARGMAX> : (const void*)gemm_tc_kernel<128, 4, GEMM_EPI_ARGMAX>;
-  }
+  if (bn == 64) { SPEC_GEMM_DISPATCH(64, 3, SPEC_FN_OF) }
+  else { SPEC_GEMM_DISPATCH(128, 4, SPEC_FN_OF) }
+  return nullptr;
 }
 
 cudaError_t gemm_tc_launch(const GemmTcLaunch& L, cudaStream_t stream, bool pdl) {
-  if (L.bn == 64) {
-    switch (L.epi) {
-      case GEMM_EPI_PARTIAL: return launch_impl<64, 3, GEMM_EPI_PARTIAL>(L, stream, pdl);
-      case GEMM_EPI_SWIGLU: return launch_impl<64, 3, GEMM_EPI_SWIGLU>(L, stream, pdl);
-      case GEMM_EPI_ARGMAX: return launch_impl<64, 3, GEMM_EPI_ARGMAX>(L, stream, pdl);
-    }
-  } else if (L.bn == 128) {
-    switch (L.epi) {
-      case GEMM_EPI_PARTIAL: return launch_impl<128, 4, GEMM_EPI_PARTIAL>(L, stream, pdl);
-      case GEMM_EPI_SWIGLU: return launch_impl<128, 4, GEMM_EPI_SWIGLU>(L, stream, pdl);
-      case GEMM_EPI_ARGMAX: return launch_impl<128, 4, GEMM_EPI_ARGMAX>(L, stream, pdl);
-    }
-  }
+  const int epi = L.epi;
+  if (L.bn == 64) { SPEC_GEMM_DISPATCH(64, 3, SPEC_LAUNCH_OF) }
+  else if (L.bn == 128) { SPEC_GEMM_DISPATCH(128, 4, SPEC_LAUNCH_OF) }
   return cudaErrorInvalidValue;
 }
 

@@ -12,21 +12,58 @@ namespace spec {
 
 struct Top2;
 
-enum { GEMM_EPI_PARTIAL = 0, GEMM_EPI_SWIGLU = 1, GEMM_EPI_ARGMAX = 2 };
+// GEMM epilogues:
+//   QKV    split-K partials; the last CTA of each 128-feature tile (one head of
+//          q|k|v) sums the splits, applies the norm scale and the rotary
+//          embedding, and writes q (fp16) or the K/V cache slot (fp16)
+//   RESID  split-K partials; the last CTA of each tile adds the sum to the fp32
+//          residual stream for its 128 columns, writes the next GEMM's operand
+//          x*w (split bf16) and the tile's per-token sums of squares of x
+//   SWIGLU gate rows 0-63, up rows 64-127 of a tile; silu(g)*u as split bf16
+//   ARGMAX per-token (best, index, runner-up) of the tile's vocabulary rows
+enum { GEMM_EPI_QKV = 0, GEMM_EPI_SWIGLU = 1, GEMM_EPI_ARGMAX = 2, GEMM_EPI_RESID = 3 };
+
+struct StepView;
 
 struct GemmTcArgs {
   int n_out;          // output features (weight rows) across all segments
   int K;              // reduction length, multiple of 64
   int M;              // valid tokens (columns); token rows >= M are ignored
   int tiles_o, tiles_t, splits, kb_per_split;
-  int seg_rows[3];    // rows served by mA0, mA1, mA2 (PARTIAL); unused for SWIGLU
-  float* out_f32;     // PARTIAL: [splits][tokens][n_out]
+  int seg_rows[3];    // rows served by mA0, mA1, mA2; unused for SWIGLU
+  // RMSNorm folded into the epilogue: the operand rows are x*w, not yet
+  // normalised; the result is scaled per token by rsqrt(sum(ss)/norm_d + eps)
+  // with ss the n_ss partial sums of squares of x (null: no scaling)
+  const float* ss_in;
+  int n_ss, ss_ld, norm_d;
+  float eps;
+  // split-K partials [splits][tokens][n_out] and per-tile arrival counters
+  float* part;
   size_t split_stride;
-  __nv_bfloat16* out_bf16;  // SWIGLU: [tokens][ld_out]
+  int* counters;      // [tiles_o * tiles_t], zero between launches
+  // SWIGLU
+  __nv_bfloat16* out_bf16;  // split bf16 [2 x tokens][ld_out]
   int ld_out;
-  Top2* top_part;     // ARGMAX: [tiles_o][top_ld]
+  // ARGMAX
+  Top2* top_part;     // [tiles_o][top_ld]
   int top_ld;
-  float* dbg_logits;  // ARGMAX: optional [M][n_out]
+  float* dbg_logits;  // optional [M][n_out]
+  // QKV
+  const int32_t* row_seq;
+  const int32_t* row_local;
+  const int32_t* P_step;
+  const int32_t* seq_ids;
+  const float2* rope_cs;  // [tokens][64]
+  __half* q_out;          // [tokens][Hq][128]
+  __half* k_cache;        // this layer's K base: [max_batch][Hkv][max_seq][128]
+  __half* v_cache;
+  size_t kv_seq_stride, kv_head_stride;
+  int Hq, Hkv, max_seq;
+  // RESID
+  float* x;                         // [tokens][n_out]
+  const __nv_bfloat16* norm_w_next; // [n_out]
+  __nv_bfloat16* xn_out;            // split bf16 [2 x tokens][n_out]
+  float* ss_out;                    // [tiles_o][ss_ld]
   uint32_t* err;
 };
 
@@ -75,10 +112,11 @@ struct KvView {
 
 enum { STEP_VERIFY = 0, STEP_PREFILL = 1, STEP_SCORE = 2 };
 
-// metadata + embedding + first RMSNorm
+// metadata + embedding + first RMSNorm.  bf16 models: xn = split(x*w) (the
+// norm scale is applied by the next GEMM) and ss[0][r] = sum x^2, ss[i>0][r] = 0.
 cudaError_t launch_embed_meta(int dtype, const StepView& sv, const void* embed, const void* norm_w, int d, float eps,
-                              float* x, void* xn, const double* inv_freq, int half, int mode, cudaStream_t s,
-                              bool pdl);
+                              float* x, void* xn, float* ss, int n_ss, int ss_ld, const double* inv_freq, int half,
+                              int mode, cudaStream_t s, bool pdl);
 // x += sum of split partials; xn = RMSNorm(x) * w
 cudaError_t launch_residual_norm(int dtype, int M, int d, int S, const float* partial, size_t split_stride, float* x,
                                  void* xn, const void* w, float eps, cudaStream_t s, bool pdl);
@@ -104,6 +142,7 @@ struct AttnArgs {
   float* part_lse;          // [M*Hq][n_chunks]
   int n_chunks, chunk;      // key chunking of [0, P_b + n_b)
   int max_rows;             // max over batch of n_b * (Hq/Hkv)
+  int* counters;            // [B][Hkv][row blocks] chunk arrivals, zero between launches
 };
 cudaError_t launch_attention(int dtype, const AttnArgs& a, cudaStream_t s, bool pdl);
 size_t attention_smem_bytes();

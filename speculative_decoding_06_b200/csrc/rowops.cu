@@ -52,14 +52,18 @@ cudaLaunchConfig_t make_cfg(dim3 grid, dim3 block, size_t smem, cudaStream_t s, 
 // parent links up to the root ("EAGLE-3投机解码：树验证器方法", section 树draft vs
 // 链draft: every token sees only its ancestors); its position is P_b + depth.
 // SPLIT: write the normalised row as split bf16 (bf16 models); else as T (fp32 models)
+// bf16 models leave the normalisation to the next GEMM: xn = split(x*w) and
+// ss[0][r] = sum x^2 (the other n_ss-1 partial slots are zero).
 template <typename T, bool SPLIT>
 __global__ void __launch_bounds__(256) embed_meta_kernel(StepView sv, const T* __restrict__ embed,
                                                          const T* __restrict__ norm_w, int d, float eps,
                                                          float* __restrict__ x, void* __restrict__ xn,
+                                                         float* __restrict__ ss_out, int n_ss, int ss_ld,
                                                          const double* __restrict__ inv_freq, int half, int mode) {
   __shared__ int s_pos;
   __shared__ float red[8];
   pdl_wait();
+  pdl_launch_dependents();
   const int r = blockIdx.x;
   if (threadIdx.x == 0) {
     int b = 0;
@@ -112,25 +116,27 @@ __global__ void __launch_bounds__(256) embed_meta_kernel(StepView sv, const T* _
     ss += v * v;
   }
   ss = block_sum<256>(ss, red);
-  const float inv = rsqrtf(ss / (float)d + eps);
-  for (int k = threadIdx.x; k < d; k += blockDim.x) {
-    const float v = xr[k] * inv * to_f32(norm_w[k]);
-    if (SPLIT) split_store(reinterpret_cast<__nv_bfloat16*>(xn), r, d, k, v);
-    else reinterpret_cast<T*>(xn)[(size_t)r * d + k] = from_f32<T>(v);
+  if (SPLIT) {
+    for (int k = threadIdx.x; k < d; k += blockDim.x)
+      split_store(reinterpret_cast<__nv_bfloat16*>(xn), r, d, k, xr[k] * to_f32(norm_w[k]));
+    for (int i = threadIdx.x; i < n_ss; i += blockDim.x) ss_out[(size_t)i * ss_ld + r] = i == 0 ? ss : 0.f;
+  } else {
+    const float inv = rsqrtf(ss / (float)d + eps);
+    for (int k = threadIdx.x; k < d; k += blockDim.x)
+      reinterpret_cast<T*>(xn)[(size_t)r * d + k] = from_f32<T>(xr[k] * inv * to_f32(norm_w[k]));
   }
-  pdl_launch_dependents();
 }
 
 cudaError_t launch_embed_meta(int dtype, const StepView& sv, const void* embed, const void* norm_w, int d, float eps,
-                              float* x, void* xn, const double* inv_freq, int half, int mode, cudaStream_t s,
-                              bool pdl) {
+                              float* x, void* xn, float* ss, int n_ss, int ss_ld, const double* inv_freq, int half,
+                              int mode, cudaStream_t s, bool pdl) {
   cudaLaunchAttribute attr[1];
   cudaLaunchConfig_t cfg = make_cfg(dim3(sv.M), dim3(256), 0, s, pdl, attr);
   if (dtype == 0)
     return cudaLaunchKernelEx(&cfg, embed_meta_kernel<float, false>, sv, (const float*)embed, (const float*)norm_w, d,
-                              eps, x, xn, inv_freq, half, mode);
+                              eps, x, xn, ss, n_ss, ss_ld, inv_freq, half, mode);
   return cudaLaunchKernelEx(&cfg, embed_meta_kernel<__nv_bfloat16, true>, sv, (const __nv_bfloat16*)embed,
-                            (const __nv_bfloat16*)norm_w, d, eps, x, xn, inv_freq, half, mode);
+                            (const __nv_bfloat16*)norm_w, d, eps, x, xn, ss, n_ss, ss_ld, inv_freq, half, mode);
 }
 
 // ---------------------------------------------------------------------------
@@ -151,6 +157,7 @@ __global__ void __launch_bounds__(256) residual_norm_kernel(int d, int S, const 
   const int CL = (int)cluster.num_blocks();
   const int rank = (int)cluster.block_rank();
   pdl_wait();
+  pdl_launch_dependents();
   const int r = blockIdx.x / CL;
   const int cols = d / CL;
   const int c0 = rank * cols;
@@ -178,7 +185,6 @@ __global__ void __launch_bounds__(256) residual_norm_kernel(int d, int S, const 
     if (SPLIT) split_store(reinterpret_cast<__nv_bfloat16*>(xn), r, d, k, v);
     else reinterpret_cast<T*>(xn)[(size_t)r * d + k] = from_f32<T>(v);
   }
-  pdl_launch_dependents();
 }
 
 int residual_norm_cluster(int d) {
@@ -219,6 +225,7 @@ __global__ void __launch_bounds__(256) qkv_rope_store_kernel(StepView sv, int S,
                                                              size_t split_stride, int Hq, int Hkv, int hd,
                                                              T* __restrict__ q_out, KvView kv, int layer) {
   pdl_wait();
+  pdl_launch_dependents();
   const int r = blockIdx.x;
   const int half = hd / 2;
   const int n_cols = (Hq + 2 * Hkv) * hd;
@@ -262,7 +269,6 @@ __global__ void __launch_bounds__(256) qkv_rope_store_kernel(StepView sv, int S,
       dst[j + half] = from_f32<T>(v2);
     }
   }
-  pdl_launch_dependents();
 }
 
 cudaError_t launch_qkv_rope_store(int dtype, const StepView& sv, int S, const float* partial, size_t split_stride,
@@ -351,6 +357,7 @@ cudaError_t launch_gemm_simt_f32(const float* A, int lda, const float* W, int K,
 __global__ void top2_reduce_kernel(int M, int tiles, const Top2* __restrict__ part, int top_ld,
                                    int32_t* __restrict__ argmax, float* __restrict__ top1, float* __restrict__ top2) {
   pdl_wait();
+  pdl_launch_dependents();
   const int t = blockIdx.x * (blockDim.x >> 5) + (threadIdx.x >> 5);
   const int lane = threadIdx.x & 31;
   if (t >= M) return;
@@ -363,7 +370,6 @@ __global__ void top2_reduce_kernel(int M, int tiles, const Top2* __restrict__ pa
     top1[t] = best.v1;
     top2[t] = best.v2;
   }
-  pdl_launch_dependents();
 }
 
 cudaError_t launch_top2_reduce(int M, int tiles, const Top2* part, int top_ld, int32_t* argmax, float* top1,

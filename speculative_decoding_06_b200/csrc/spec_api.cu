@@ -16,6 +16,7 @@
 #include <cmath>
 #include <cstdarg>
 #include <cstdio>
+#include <cstdlib>
 #include <cstring>
 #include <map>
 #include <string>
@@ -32,6 +33,8 @@ namespace {
 
 constexpr int kMaxNodesLimit = 128;  // ancestor bitmask is two 64-bit words
 constexpr int kMaxSplits = 16;
+constexpr int kGemmCounters = 8192;  // per-tile arrival counters of the split-K GEMMs
+constexpr int kMaxAttnChunks = 8;     // key chunks of one row block = one portable cluster
 
 size_t align_up(size_t x, size_t a) { return (x + a - 1) / a * a; }
 int ceil_div(int a, int b) { return (a + b - 1) / b; }
@@ -47,6 +50,8 @@ struct WsLayout {
   size_t seq_len, pending, hist, err_sticky;
   // activations
   size_t x, xn, q, attn, hmlp, partial, part_o, part_lse, top_part, argmax, top1, top2, inv_freq;
+  size_t ss, gemm_ctr, attn_ctr;
+  int n_ss = 1, attn_ctr_n = 0;
   size_t partial_bytes;
   // outputs (one device->host copy per step)
   size_t o_acc_len, o_acc_nodes, o_acc_tokens, o_bonus, o_end;
@@ -58,7 +63,7 @@ WsLayout make_layout(const spec_config& c) {
   L.Mmax = c.max_batch * c.max_nodes;
   L.Mpad = (int)align_up(L.Mmax, 128);
   L.splits_cap = L.Mpad <= 256 ? kMaxSplits : 2;
-  L.chunks_cap = std::max(2, std::min(32, 1184 / std::max(1, c.max_batch * c.n_kv_heads)));
+  L.chunks_cap = kMaxAttnChunks;
   const int qd = c.n_q_heads * c.head_dim;
   const int nqkv = (c.n_q_heads + 2 * c.n_kv_heads) * c.head_dim;
   size_t off = 0;
@@ -98,6 +103,11 @@ WsLayout make_layout(const spec_config& c) {
   L.part_o = take(4 * (size_t)L.Mmax * c.n_q_heads * L.chunks_cap * c.head_dim);
   L.part_lse = take(4 * (size_t)L.Mmax * c.n_q_heads * L.chunks_cap);
   L.top_part = take(sizeof(Top2) * (size_t)ceil_div(c.vocab, 128) * L.Mpad);
+  L.n_ss = std::max(1, c.hidden / 128);
+  L.ss = take(4 * (size_t)L.n_ss * L.Mpad);
+  L.gemm_ctr = take(4 * (size_t)kGemmCounters);
+  L.attn_ctr_n = c.max_batch * c.n_kv_heads * ceil_div(c.max_nodes * (c.n_q_heads / c.n_kv_heads), 64);
+  L.attn_ctr = take(4 * (size_t)L.attn_ctr_n);
   L.argmax = take(4 * (size_t)L.Mpad);
   L.top1 = take(4 * (size_t)L.Mpad);
   L.top2 = take(4 * (size_t)L.Mpad);
@@ -201,7 +211,8 @@ struct spec_handle {
   std::vector<LayerMaps> maps;
   CUtensorMap map_lm;
   CUtensorMap map_xn[2], map_attn[2], map_h[2];  // B operands for BN = 64, 128
-  int resident[2][3] = {{0, 0, 0}, {0, 0, 0}};   // co-resident CTAs per SM [bn][epi]
+  int resident[2][4] = {{0, 0, 0, 0}, {0, 0, 0, 0}};   // co-resident CTAs per SM [bn][epi]
+  int occ_api[2][4] = {{0, 0, 0, 0}, {0, 0, 0, 0}};    // what the occupancy query reported
   // host mirror of per-sequence state
   std::vector<int32_t> len, pending;
   std::vector<int32_t> len_hi;  // upper bound while device-output steps are in flight
@@ -214,6 +225,9 @@ struct spec_handle {
   size_t dbg_bytes = 0;
   std::map<GraphKey, cudaGraphExec_t> graphs;
   bool use_pdl = true;
+  int max_splits = 16;    // split-K cap
+  int max_chunks = 8;     // attention key-chunk cap (one cluster per row block)
+  int resident_cap = 0;   // 0: as many CTAs per SM as fit
   std::string err;
   // profiler: an event pair per launch
   bool prof = false;
@@ -275,19 +289,23 @@ GemmPlan plan_gemm(const spec_handle* h, int rows_per_tile, int n_out, int K, in
   GemmPlan p;
   p.bn = M <= 64 ? 64 : 128;
   const int bi = p.bn == 64 ? 0 : 1;
-  const int resident = std::max(1, h->resident[bi][epi]) * h->sm_count;
+  int per_sm = std::max(1, h->resident[bi][epi]);
+  if (h->resident_cap > 0) per_sm = std::min(per_sm, h->resident_cap);
+  const int resident = per_sm * h->sm_count;
   p.tiles_o = ceil_div(n_out, rows_per_tile);
   p.tiles_t = ceil_div(M, p.bn);
   const int KB = K / 64;
   const int base = p.tiles_o * p.tiles_t;
   int S = 1;
-  if (epi == GEMM_EPI_PARTIAL) {
-    const int cap = std::min(h->lay.splits_cap, std::max(1, KB / 4));
+  if (epi == GEMM_EPI_QKV || epi == GEMM_EPI_RESID) {
+    // split-K only while every tile x split CTA can be resident at once: the
+    // splits of a tile wait for one another
+    const int cap = std::min(std::min(h->lay.splits_cap, h->max_splits), std::max(1, KB / 4));
     S = std::max(1, std::min(cap, resident / std::max(1, base)));
   }
   p.kbps = ceil_div(KB, S);
   p.splits = ceil_div(KB, p.kbps);  // no empty split
-  p.grid = std::min(base * p.splits, resident);
+  p.grid = p.splits > 1 ? base * p.splits : std::min(base, resident);
   return p;
 }
 
@@ -302,18 +320,19 @@ StepPlan make_plan(const spec_handle* h, int B, int M, int max_n, int max_lk) {
   s.max_rows = max_n * G;
   const int rowblocks = ceil_div(s.max_rows, 64);
   const int ctas_per_chunk = B * c.n_kv_heads * rowblocks;
+  const int ccap = std::min(h->lay.chunks_cap, h->max_chunks);
   int want = std::max(1, ceil_div(2 * h->sm_count, ctas_per_chunk));
-  want = std::min(want, h->lay.chunks_cap);
+  want = std::min(want, ccap);
   int chunk = std::max(256, (int)align_up(ceil_div(max_lk, want), 64));
-  chunk = std::max(chunk, (int)align_up(ceil_div(max_lk, h->lay.chunks_cap), 64));
+  chunk = std::max(chunk, (int)align_up(ceil_div(max_lk, ccap), 64));
   s.chunk = chunk;
   s.n_chunks = ceil_div(max_lk, chunk);
   const int nqkv = (c.n_q_heads + 2 * c.n_kv_heads) * c.head_dim;
   const int qd = c.n_q_heads * c.head_dim;
-  s.qkv = plan_gemm(h, 128, nqkv, c.hidden, M, GEMM_EPI_PARTIAL);
-  s.o = plan_gemm(h, 128, c.hidden, qd, M, GEMM_EPI_PARTIAL);
+  s.qkv = plan_gemm(h, 128, nqkv, c.hidden, M, GEMM_EPI_QKV);
+  s.o = plan_gemm(h, 128, c.hidden, qd, M, GEMM_EPI_RESID);
   s.gu = plan_gemm(h, 64, c.ffn, c.hidden, M, GEMM_EPI_SWIGLU);
-  s.down = plan_gemm(h, 128, c.hidden, c.ffn, M, GEMM_EPI_PARTIAL);
+  s.down = plan_gemm(h, 128, c.hidden, c.ffn, M, GEMM_EPI_RESID);
   s.lm = plan_gemm(h, 128, c.vocab, c.hidden, M, GEMM_EPI_ARGMAX);
   return s;
 }
@@ -392,9 +411,17 @@ cudaError_t enqueue_step(spec_handle* h, const StepPlan& sp, int mode, bool dbg)
   float* part = h->W<float>(L.partial);
   h->launches = 0;
 
+  float* ss = h->W<float>(L.ss);
+  int* gctr = h->W<int>(L.gemm_ctr);
+  if (dt == 1) {
+    // arrival counters start every step at zero, whatever an earlier failed step left behind
+    cudaError_t e0 = cudaMemsetAsync(gctr, 0, 4 * (size_t)kGemmCounters, st);
+    if (e0 == cudaSuccess) e0 = cudaMemsetAsync(h->ws + L.attn_ctr, 0, 4 * (size_t)L.attn_ctr_n, st);
+    if (e0 != cudaSuccess) return e0;
+  }
   LK(SPEC_PROF_EMBED_META, 1,
-     launch_embed_meta(dt, sv, h->embed, h->layers[0].attn_norm, d, c.rms_eps, x, xn, h->W<double>(L.inv_freq),
-                       c.head_dim / 2, mode, st, pdl));
+     launch_embed_meta(dt, sv, h->embed, h->layers[0].attn_norm, d, c.rms_eps, x, xn, ss, L.n_ss, L.Mpad,
+                       h->W<double>(L.inv_freq), c.head_dim / 2, mode, st, pdl));
 
   AttnArgs aa{};
   aa.sv = sv;
@@ -408,6 +435,7 @@ cudaError_t enqueue_step(spec_handle* h, const StepPlan& sp, int mode, bool dbg)
   aa.n_chunks = sp.n_chunks;
   aa.chunk = sp.chunk;
   aa.max_rows = sp.max_rows;
+  aa.counters = h->W<int>(L.attn_ctr);
 
   for (int l = 0; l < c.n_layers; ++l) {
     const spec_layer_weights& lw = h->layers[l];
@@ -416,36 +444,69 @@ cudaError_t enqueue_step(spec_handle* h, const StepPlan& sp, int mode, bool dbg)
     if (dt == 1) {
       const LayerMaps& mp = h->maps[l];
       const int bi = sp.qkv.bn == 64 ? 0 : 1;
-      GemmTcLaunch g = gemm_launch(sp.qkv, GEMM_EPI_PARTIAL, nqkv, d, M, &mp.wq, &mp.wk, &mp.wv, &h->map_xn[bi], qd,
+      __half* kc = reinterpret_cast<__half*>(h->kv.base) + (size_t)l * h->kv.layer_stride();
+      // QKV (+ norm scale, rotary, q and K/V cache store in the last CTA of each head)
+      GemmTcLaunch g = gemm_launch(sp.qkv, GEMM_EPI_QKV, nqkv, d, M, &mp.wq, &mp.wk, &mp.wv, &h->map_xn[bi], qd,
                                    kvd, kvd, sv.err);
-      g.args.out_f32 = part;
+      g.args.ss_in = ss;
+      g.args.n_ss = L.n_ss;
+      g.args.ss_ld = L.Mpad;
+      g.args.norm_d = d;
+      g.args.eps = c.rms_eps;
+      g.args.part = part;
       g.args.split_stride = (size_t)L.Mpad * nqkv;
+      g.args.counters = gctr;
+      g.args.row_seq = sv.row_seq;
+      g.args.row_local = sv.row_local;
+      g.args.P_step = sv.P_step;
+      g.args.seq_ids = sv.seq_ids;
+      g.args.rope_cs = sv.rope_cs;
+      g.args.q_out = reinterpret_cast<__half*>(q);
+      g.args.k_cache = kc;
+      g.args.v_cache = kc + h->kv.kv_stride();
+      g.args.kv_seq_stride = h->kv.seq_stride();
+      g.args.kv_head_stride = h->kv.head_stride();
+      g.args.Hq = c.n_q_heads;
+      g.args.Hkv = c.n_kv_heads;
+      g.args.max_seq = c.max_seq;
       LK(SPEC_PROF_GEMM_QKV, 1, gemm_tc_launch(g, st, pdl));
-      LK(SPEC_PROF_ROPE_KV, 1,
-         launch_qkv_rope_store(dt, sv, sp.qkv.splits, part, (size_t)L.Mpad * nqkv, c.n_q_heads, c.n_kv_heads,
-                               c.head_dim, q, h->kv, l, st, pdl));
-      LK(SPEC_PROF_ATTENTION, 2, launch_attention(dt, aa, st, pdl));
-      GemmTcLaunch go = gemm_launch(sp.o, GEMM_EPI_PARTIAL, d, qd, M, &mp.wo, nullptr, nullptr, &h->map_attn[bi], d,
+      // attention (chunks + merge in the last chunk's CTA)
+      LK(SPEC_PROF_ATTENTION, 1, launch_attention(dt, aa, st, pdl));
+      // O projection (+ residual, next operand x*w_mlp, sums of squares)
+      GemmTcLaunch go = gemm_launch(sp.o, GEMM_EPI_RESID, d, qd, M, &mp.wo, nullptr, nullptr, &h->map_attn[bi], d,
                                     0, 0, sv.err);
-      go.args.out_f32 = part;
+      go.args.part = part;
       go.args.split_stride = (size_t)L.Mpad * d;
+      go.args.counters = gctr;
+      go.args.x = x;
+      go.args.norm_w_next = reinterpret_cast<const __nv_bfloat16*>(lw.mlp_norm);
+      go.args.xn_out = reinterpret_cast<__nv_bfloat16*>(xn);
+      go.args.ss_out = ss;
+      go.args.ss_ld = L.Mpad;
       LK(SPEC_PROF_GEMM_O, 1, gemm_tc_launch(go, st, pdl));
-      LK(SPEC_PROF_RESID_NORM, 1,
-         launch_residual_norm(dt, M, d, sp.o.splits, part, (size_t)L.Mpad * d, x, xn, lw.mlp_norm, c.rms_eps, st,
-                              pdl));
+      // gate/up (+ norm scale, SwiGLU)
       GemmTcLaunch gg = gemm_launch(sp.gu, GEMM_EPI_SWIGLU, c.ffn, d, M, &mp.wg, &mp.wu, nullptr, &h->map_xn[bi], 0,
                                     0, 0, sv.err);
+      gg.args.ss_in = ss;
+      gg.args.n_ss = L.n_ss;
+      gg.args.ss_ld = L.Mpad;
+      gg.args.norm_d = d;
+      gg.args.eps = c.rms_eps;
       gg.args.out_bf16 = reinterpret_cast<__nv_bfloat16*>(hm);
       gg.args.ld_out = c.ffn;
       LK(SPEC_PROF_GEMM_GATE_UP, 1, gemm_tc_launch(gg, st, pdl));
-      GemmTcLaunch gd = gemm_launch(sp.down, GEMM_EPI_PARTIAL, d, c.ffn, M, &mp.wd, nullptr, nullptr, &h->map_h[bi],
+      // down (+ residual, next operand x*w_next, sums of squares)
+      GemmTcLaunch gd = gemm_launch(sp.down, GEMM_EPI_RESID, d, c.ffn, M, &mp.wd, nullptr, nullptr, &h->map_h[bi],
                                     d, 0, 0, sv.err);
-      gd.args.out_f32 = part;
+      gd.args.part = part;
       gd.args.split_stride = (size_t)L.Mpad * d;
+      gd.args.counters = gctr;
+      gd.args.x = x;
+      gd.args.norm_w_next = reinterpret_cast<const __nv_bfloat16*>(next_norm);
+      gd.args.xn_out = reinterpret_cast<__nv_bfloat16*>(xn);
+      gd.args.ss_out = ss;
+      gd.args.ss_ld = L.Mpad;
       LK(SPEC_PROF_GEMM_DOWN, 1, gemm_tc_launch(gd, st, pdl));
-      LK(SPEC_PROF_RESID_NORM, 1,
-         launch_residual_norm(dt, M, d, sp.down.splits, part, (size_t)L.Mpad * d, x, xn, next_norm, c.rms_eps, st,
-                              pdl));
     } else {
       const float* xf = reinterpret_cast<const float*>(xn);
       LK(SPEC_PROF_GEMM_QKV, 1, launch_gemm_simt_f32(xf, d, (const float*)lw.wq, d, part, nqkv, M, qd, st));
@@ -476,6 +537,11 @@ cudaError_t enqueue_step(spec_handle* h, const StepPlan& sp, int mode, bool dbg)
     g.args.top_part = h->W<Top2>(L.top_part);
     g.args.top_ld = L.Mpad;
     g.args.dbg_logits = dbg ? h->dbg_logits : nullptr;
+    g.args.ss_in = h->W<float>(L.ss);
+    g.args.n_ss = L.n_ss;
+    g.args.ss_ld = L.Mpad;
+    g.args.norm_d = d;
+    g.args.eps = c.rms_eps;
     LK(SPEC_PROF_LM_HEAD, 1, gemm_tc_launch(g, st, pdl));
     LK(SPEC_PROF_LM_REDUCE, 1,
        launch_top2_reduce(M, sp.lm.tiles_o, h->W<Top2>(L.top_part), L.Mpad, amax, h->W<float>(L.top1),
@@ -725,6 +791,14 @@ int spec_init(const spec_config* cfg, const spec_weights* w, void* kv_cache, siz
     (void)msg;
     return code;
   };
+  // Optional tuning knobs, e.g. SPEC_TUNE="splits=4,chunks=8,pdl=0,per_sm=1"
+  if (const char* t = getenv("SPEC_TUNE")) {
+    int v = 0;
+    if (const char* q = strstr(t, "splits=")) if (sscanf(q + 7, "%d", &v) == 1 && v >= 1 && v <= kMaxSplits) h->max_splits = v;
+    if (const char* q = strstr(t, "chunks=")) if (sscanf(q + 7, "%d", &v) == 1 && v >= 1 && v <= kMaxAttnChunks) h->max_chunks = v;
+    if (const char* q = strstr(t, "pdl=")) if (sscanf(q + 4, "%d", &v) == 1) h->use_pdl = v != 0;
+    if (const char* q = strstr(t, "per_sm=")) if (sscanf(q + 7, "%d", &v) == 1 && v >= 0) h->resident_cap = v;
+  }
   if (cudaGetDevice(&h->device) != cudaSuccess) return bail(SPEC_ERR_CUDA, "cudaGetDevice");
   cudaDeviceProp prop;
   if (cudaGetDeviceProperties(&prop, h->device) != cudaSuccess) return bail(SPEC_ERR_CUDA, "props");
@@ -738,6 +812,8 @@ int spec_init(const spec_config* cfg, const spec_weights* w, void* kv_cache, siz
   if (cudaMemsetAsync(h->ws + lay.seq_len, 0, 4 * (size_t)c.max_batch, h->stream) != cudaSuccess ||
       cudaMemsetAsync(h->ws + lay.pending, 0xff, 4 * (size_t)c.max_batch, h->stream) != cudaSuccess ||
       cudaMemsetAsync(h->ws + lay.err_sticky, 0, 16, h->stream) != cudaSuccess ||
+      cudaMemsetAsync(h->ws + lay.gemm_ctr, 0, 4 * (size_t)kGemmCounters, h->stream) != cudaSuccess ||
+      cudaMemsetAsync(h->ws + lay.attn_ctr, 0, 4 * (size_t)lay.attn_ctr_n, h->stream) != cudaSuccess ||
       cudaMemcpyAsync(h->ws + lay.inv_freq, inv.data(), 8 * inv.size(), cudaMemcpyHostToDevice, h->stream) !=
           cudaSuccess ||
       cudaStreamSynchronize(h->stream) != cudaSuccess)
@@ -769,16 +845,22 @@ int spec_init(const spec_config* cfg, const spec_weights* w, void* kv_cache, siz
         return bail(SPEC_ERR_CUDA, "tensor map");
     }
     for (int i = 0; i < 2; ++i)
-      for (int e = 0; e < 3; ++e) {
+      for (int e = 0; e < 4; ++e) {
         const void* fn = gemm_tc_function(bns[i], e);
         const int smem = (int)gemm_tc_smem_bytes(bns[i], e);
-        if (cudaFuncSetAttribute(fn, cudaFuncAttributeMaxDynamicSharedMemorySize, smem) != cudaSuccess)
+        if (cudaFuncSetAttribute(fn, cudaFuncAttributeMaxDynamicSharedMemorySize, smem) != cudaSuccess ||
+            cudaFuncSetAttribute(fn, cudaFuncAttributePreferredSharedMemoryCarveout,
+                                 (int)cudaSharedmemCarveoutMaxShared) != cudaSuccess)
           return bail(SPEC_ERR_CUDA, "smem attribute");
         int nb = 0;
         if (cudaOccupancyMaxActiveBlocksPerMultiprocessor(&nb, fn, 192, smem) != cudaSuccess || nb < 1)
           return bail(SPEC_ERR_CUDA, "occupancy");
+        // shared memory per SM (1 KB per CTA is reserved by the system)
+        const int by_smem = prop.sharedMemPerMultiprocessor / (smem + (int)prop.reservedSharedMemPerBlock);
+        h->occ_api[i][e] = nb;
+        nb = std::max(nb, by_smem);
         // tensor memory: two accumulators of 2*BN columns (hi and lo) per CTA, 512 columns per SM
-        h->resident[i][e] = std::min(nb, 512 / (4 * bns[i]));
+        h->resident[i][e] = std::max(1, std::min(nb, 512 / (4 * bns[i])));
       }
   }
   *out = h;
@@ -955,6 +1037,25 @@ int spec_profile_read(spec_handle* h, double* ms, int64_t* launches) {
 }
 
 int spec_step_launches(spec_handle* h) { return h ? h->launches : 0; }
+
+int spec_info(spec_handle* h, int B, int n_nodes, int prefix, char* buf, size_t n) {
+  if (!h || !buf || n == 0) return SPEC_ERR_ARG;
+  const StepPlan sp = make_plan(h, B, B * n_nodes, n_nodes, prefix + n_nodes);
+  auto g = [](const GemmPlan& p) {
+    char t[96];
+    snprintf(t, sizeof(t), "bn%d tiles%dx%d splits%d kb/split%d grid%d", p.bn, p.tiles_o, p.tiles_t, p.splits,
+             p.kbps, p.grid);
+    return std::string(t);
+  };
+  std::string s = "sms " + std::to_string(h->sm_count) + "; resident/SM [bn64|bn128][qkv,swiglu,argmax,resid] = ";
+  for (int i = 0; i < 2; ++i)
+    for (int e = 0; e < 4; ++e)
+      s += std::to_string(h->resident[i][e]) + "(" + std::to_string(h->occ_api[i][e]) + ")" + (e < 3 ? "," : "|");
+  s += "; qkv " + g(sp.qkv) + "; o " + g(sp.o) + "; gate_up " + g(sp.gu) + "; down " + g(sp.down) + "; lm " +
+       g(sp.lm) + "; attention chunks " + std::to_string(sp.n_chunks) + " x " + std::to_string(sp.chunk);
+  snprintf(buf, n, "%s", s.c_str());
+  return SPEC_OK;
+}
 
 int spec_io_bytes(spec_handle* h, size_t* h2d, size_t* d2h) {
   if (!h) return SPEC_ERR_ARG;

@@ -173,6 +173,11 @@ class SpecEngine:
         self._check(S.spec_profile_read(self.h, ms, n))
         return {k: (ms[i], n[i]) for i, k in enumerate(S.PROF_CLASSES)}
 
+    def info(self, B: int, n_nodes: int, prefix: int) -> str:
+        buf = ctypes.create_string_buffer(4096)
+        self._check(S.spec_info(self.h, B, n_nodes, prefix, buf, 4096))
+        return buf.value.decode()
+
     def step_launches(self) -> int:
         return int(S.spec_step_launches(self.h))
 

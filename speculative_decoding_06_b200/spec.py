@@ -85,6 +85,7 @@ _SIGNATURES = {
     "spec_profile": (ctypes.c_int, [_h, ctypes.c_int]),
     "spec_profile_read": (ctypes.c_int, [_h, ctypes.POINTER(ctypes.c_double), ctypes.POINTER(ctypes.c_int64)]),
     "spec_step_launches": (ctypes.c_int, [_h]),
+    "spec_info": (ctypes.c_int, [_h, ctypes.c_int, ctypes.c_int, ctypes.c_int, ctypes.c_char_p, ctypes.c_size_t]),
     "spec_io_bytes": (ctypes.c_int, [_h, ctypes.POINTER(ctypes.c_size_t), ctypes.POINTER(ctypes.c_size_t)]),
     "spec_last_error": (ctypes.c_char_p, [_h]),
     "spec_free": (None, [_h]),
@@ -140,6 +141,7 @@ spec_validate_tree = _bind("spec_validate_tree")
 spec_profile = _bind("spec_profile")
 spec_profile_read = _bind("spec_profile_read")
 spec_step_launches = _bind("spec_step_launches")
+spec_info = _bind("spec_info")
 spec_io_bytes = _bind("spec_io_bytes")
 spec_last_error = _bind("spec_last_error")
 spec_free = _bind("spec_free")
