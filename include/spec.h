@@ -211,6 +211,33 @@ SPEC_API int spec_info(spec_handle* h, int B, int n_nodes, int prefix, char* buf
 /* Number of kernels the most recent step enqueued. */
 SPEC_API int spec_step_launches(spec_handle* h);
 
+/* LM head with fused per-row argmax, for callers that cannot allocate device
+ * memory.  (The pages have no counterpart: this is a deployment variant of the
+ * step's last kernel.)  Some callers are not allowed to call cudaMalloc: code
+ * running inside a CUDA-graph capture, runtimes that own every buffer and hand
+ * out no allocation rights, plug-in hosts that forbid allocation after start-up.
+ * This entry point needs no allocation and no handle: its scratch (a split-bf16
+ * copy of the normalised rows and per-vocabulary-tile top-2 partials) is one
+ * fixed array of about 3.5 MiB inside the library, which every GPU that loads
+ * the library holds until the process exits.
+ *
+ * Computes, for each of M hidden rows h (device fp32 [M][d], before the final
+ * norm): RMSNorm(h) * final_norm (device bf16 [d]) times lm_head^T (device bf16
+ * [V][d], 16-byte aligned), and writes argmax[M] (lowest index on ties),
+ * top1[M] and top2[M] (device arrays).  Limits: 1 <= M <= 64, d a multiple of
+ * 128 up to 8192, V up to 262144; larger sizes return SPEC_ERR_CAPACITY before
+ * any GPU work.  Work is queued on cuda_stream (NULL: legacy default stream);
+ * the call does not synchronise.
+ *
+ * The first call on a device looks up the scratch array's device address and
+ * sets kernel attributes, so make that first call before any stream capture.
+ * Every call uses the same scratch and leaves its contents behind; nothing in
+ * it has to start at zero.  Calls that overlap on the GPU (on different
+ * streams, or from different threads) race on the scratch: serialise them. */
+SPEC_API int spec_lm_head_argmax_noalloc(const float* hidden, const void* final_norm, const void* lm_head, int M,
+                                         int d, int V, float eps, int32_t* argmax, float* top1, float* top2,
+                                         void* cuda_stream);
+
 /* Message of the last error on this handle ("" if none). */
 SPEC_API const char* spec_last_error(spec_handle* h);
 /* Free host-side state (graphs, descriptors); never frees borrowed buffers. */

@@ -87,6 +87,8 @@ _SIGNATURES = {
     "spec_step_launches": (ctypes.c_int, [_h]),
     "spec_info": (ctypes.c_int, [_h, ctypes.c_int, ctypes.c_int, ctypes.c_int, ctypes.c_char_p, ctypes.c_size_t]),
     "spec_io_bytes": (ctypes.c_int, [_h, ctypes.POINTER(ctypes.c_size_t), ctypes.POINTER(ctypes.c_size_t)]),
+    "spec_lm_head_argmax_noalloc": (ctypes.c_int, [_vp, _vp, _vp, ctypes.c_int, ctypes.c_int, ctypes.c_int,
+                                                    ctypes.c_float, _vp, _vp, _vp, _vp]),
     "spec_last_error": (ctypes.c_char_p, [_h]),
     "spec_free": (None, [_h]),
 }
@@ -143,5 +145,6 @@ spec_profile_read = _bind("spec_profile_read")
 spec_step_launches = _bind("spec_step_launches")
 spec_info = _bind("spec_info")
 spec_io_bytes = _bind("spec_io_bytes")
+spec_lm_head_argmax_noalloc = _bind("spec_lm_head_argmax_noalloc")
 spec_last_error = _bind("spec_last_error")
 spec_free = _bind("spec_free")
