@@ -1,0 +1,585 @@
+// Tree attention of bf16 models on the 5th-generation tensor cores.
+//
+// Node i of a tree (local index) sits at cache slot P_b + i and at position
+// P_b + depth(i).  A query row sees every prefix key (slots 0 .. P_b-1) and the
+// tree keys of its own ancestors, itself included ("EAGLE-3投机解码：
+// 树验证器方法", section 树draft vs 链draft).  Grouped-query attention: query
+// head h reads key/value head h / (Hq/Hkv).
+//
+// One CTA handles one (sequence, kv head, tile of 128 query rows, key chunk).
+// The query rows of a kv head are its G = Hq/Hkv heads for every tree node
+// (row = node * G + g), so one K/V block serves all of them.  q and the K/V
+// cache are fp16; the probabilities P are rounded to fp16 for the P.V product;
+// scores and outputs accumulate in fp32 in tensor memory.
+//
+//   warp 4 (one thread): TMA loads of Q and of 128-key K/V blocks (two stages),
+//                        S_j = Q K_j^T into one of two 128-column TMEM buffers,
+//                        O += P_j V_j into a third (V is read MN-major);
+//   warps 0-3:           thread r owns query row r: reads S_j from its TMEM
+//                        lane, applies the ancestor mask and the online softmax
+//                        (the running max only moves when it grows by more than
+//                        2^8, which keeps every p <= 256 and rescales O rarely),
+//                        writes P_j into shared memory as the next MMA's A
+//                        operand, and at the end normalises O.
+//
+// A sequence's keys are cut into chunks so that short-prefix, small-batch steps
+// still occupy the GPU; the chunk CTAs of one (sequence, kv head, row tile)
+// are co-resident (the plan keeps the grid within one CTA per SM), publish
+// fp32 partials (normalised O and log2-sum-exp), meet at a bounded counter, and
+// each merges a slice of the rows.  With one chunk the CTA writes its rows
+// directly.  The output is split bf16 (hi, lo) for the O-projection GEMM.
+#include <cuda.h>
+
+#include "common.cuh"
+#include "kernels.h"
+
+namespace spec {
+
+namespace {
+
+constexpr int kRows = 128;                   // query rows per CTA (the MMA M)
+constexpr int kKeys = 128;                   // keys per block (S's N, P.V's K)
+constexpr int kThreads = 160;                // warps 0-3 rows, warp 4 issue
+constexpr uint32_t kHalf = 128 * 128;        // [128 rows][64 fp16] swizzled: 16 KB
+constexpr uint32_t kTile = 2 * kHalf;        // 128 x 128 fp16: 32 KB
+constexpr float kRescaleLog2 = 8.f;          // running-max slack (log2 units)
+
+enum { B_QFULL = 0, B_KVFULL = 1, B_KVEMPTY = 3, B_SFULL = 5, B_SFREE = 7, B_PFULL = 9, B_PEMPTY = 10, B_OFULL = 11,
+       B_DRAIN = 12, kNumBars = 13 };
+
+struct Smem {
+  static constexpr uint32_t q = 0;
+  static constexpr uint32_t k = q + kTile;          // 2 stages
+  static constexpr uint32_t v = k + 2 * kTile;      // 2 stages
+  static constexpr uint32_t p = v + 2 * kTile;
+  static constexpr uint32_t bars = p + kTile;
+  static constexpr uint32_t misc = bars + kNumBars * 8;  // tmem slot, abort flag, merge flag
+  static constexpr uint32_t end = misc + 16;
+  static constexpr uint32_t dyn = end + 1024;            // 1024-byte alignment slack
+};
+static_assert(Smem::dyn <= 227 * 1024, "shared memory");
+
+// tensor-memory columns: S buffers at 0 and 128, O at 256
+constexpr uint32_t kTmemCols = 512;
+constexpr uint32_t kColO = 256;
+
+// fp16 A and B, f32 D, M = 128, N = 128; bit 16 marks B as MN-major
+constexpr uint32_t kIdescS = (1u << 4) | ((uint32_t)(kKeys >> 3) << 17) | ((uint32_t)(kRows >> 4) << 24);
+constexpr uint32_t kIdescPV = kIdescS | (1u << 16);
+
+// MN-major operand with the 128-byte swizzle: 64 fp16 along N per 128-byte row,
+// 8-row (K) groups 1024 B apart (stride byte offset), N atoms `lbo` bytes apart
+// (leading byte offset).
+__device__ __forceinline__ uint64_t sw128_mnmajor_desc(uint32_t smem_addr, uint32_t lbo) {
+  uint64_t d = 0;
+  d |= (uint64_t)((smem_addr & 0x3FFFF) >> 4);
+  d |= (uint64_t)((lbo >> 4) & 0x3FFF) << 16;
+  d |= (uint64_t)(1024 >> 4) << 32;
+  d |= (uint64_t)1 << 46;
+  d |= (uint64_t)2 << 61;
+  return d;
+}
+
+// optional timeline: trace[cta][k] = %globaltimer at mark k (thread 0 of the
+// softmax warps, or the issuing thread for marks 1, 2, 11, 12)
+constexpr int kTraceMarks = 16;
+__device__ __forceinline__ void stamp_at(uint64_t* trace, int k) {
+  if (!trace) return;
+  const unsigned cta = (blockIdx.z * gridDim.y + blockIdx.y) * gridDim.x + blockIdx.x;
+  if (cta < (unsigned)kAttnPartCtas) trace[cta * kTraceMarks + k] = global_ns();
+}
+
+__device__ __forceinline__ void named_sync_rows() { asm volatile("bar.sync 1, 128;" ::: "memory"); }
+
+// keep uses of TMEM-loaded registers after the wait
+__device__ __forceinline__ void reg_fence32(uint32_t* r) {
+#pragma unroll
+  for (int i = 0; i < 32; ++i) asm volatile("" : "+r"(r[i]));
+}
+
+
+// 2^x on the special-function unit (PTX ex2.approx: relative error about
+// 2^-22, 2^-inf = +0); the probabilities are rounded to fp16 right after.
+__device__ __forceinline__ float fast_exp2(float x) {
+  float y;
+  asm("ex2.approx.ftz.f32 %0, %1;" : "=f"(y) : "f"(x));
+  return y;
+}
+
+// Bits j = 0..31 of the 128-bit ancestor set (a1:a0) starting at bit s, with
+// zeros for bit positions outside [0, 128); s in [-31, 127].
+__device__ __forceinline__ uint32_t anc_window(uint64_t a0, uint64_t a1, int s) {
+  if (s < 0) return (uint32_t)(a0 << (-s));
+  const uint64_t lo = s < 64 ? a0 : a1;
+  const uint64_t hi = s < 64 ? a1 : 0ull;
+  const int sh = s & 63;
+  return (uint32_t)(sh ? (lo >> sh) | (hi << (64 - sh)) : lo);
+}
+
+// Visible keys among key0 .. key0+31 for one query row: keys below c1, and
+// either prefix keys (below P) or tree keys whose node is an ancestor of the
+// row's node (bit key - P of the ancestor set).
+__device__ __forceinline__ uint32_t visible_word(int key0, int P, int c1, uint64_t a0, uint64_t a1) {
+  const int nv = c1 - key0;
+  const uint32_t lim = nv >= 32 ? 0xffffffffu : (nv <= 0 ? 0u : (1u << nv) - 1u);
+  const int np = P - key0;
+  const uint32_t pre = np >= 32 ? 0xffffffffu : (np <= 0 ? 0u : (1u << np) - 1u);
+  const int s = key0 - P;
+  const uint32_t tree = (s <= -32 || s >= 128) ? 0u : anc_window(a0, a1, s);
+  return lim & (pre | tree);
+}
+
+// Partial / output staging in shared memory: 128 rows x 32 float4 chunks,
+// chunk k of row r at position k ^ (r & 7) within its group of eight, so that
+// per-row writes by 32 threads and per-row reads by one warp are both free of
+// bank conflicts.
+__device__ __forceinline__ float4* stage_at(uint8_t* base, int r, int k) {
+  return reinterpret_cast<float4*>(base) + r * 32 + (k ^ (r & 7));
+}
+
+}  // namespace
+
+__global__ void __launch_bounds__(kThreads, 1) attn_tc_kernel(const __grid_constant__ AttnTcMaps maps, AttnArgs a) {
+  extern __shared__ uint8_t smem_raw[];
+  uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
+  uint64_t* bar = reinterpret_cast<uint64_t*>(smem + Smem::bars);
+  uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(smem + Smem::misc);
+  volatile int* abort_flag = reinterpret_cast<volatile int*>(smem + Smem::misc + 4);
+  volatile int* merge_ok = reinterpret_cast<volatile int*>(smem + Smem::misc + 8);
+
+  // The step's row metadata was written kernels ago (every kernel in between
+  // waited for its predecessor), so it may be read before this launch waits for
+  // the previous kernel; q, the tree's K/V and every output come after the wait.
+  const StepView& sv = a.sv;
+  const int Hkv = a.kv.Hkv;
+  const int G = a.Hq / Hkv;
+  const int bk = blockIdx.z;
+  const int b = bk / Hkv;
+  const int kvh = bk - b * Hkv;
+  const int tid = threadIdx.x;
+  const int warp = tid >> 5;
+  const int lane = tid & 31;
+  if (b >= sv.B) {
+    pdl_wait();
+    pdl_launch_dependents();
+    return;
+  }
+  const int base = sv.node_off[b];
+  const int n_b = sv.node_off[b + 1] - base;
+  const int rows = n_b * G;
+  const int row0 = blockIdx.y * kRows;
+  const int P = sv.P_step[b];
+  const int Lk = P + n_b;
+  const int c0 = blockIdx.x * a.chunk;
+  if (row0 >= rows || c0 >= Lk) {  // nothing here: no partial, no arrival
+    pdl_wait();
+    pdl_launch_dependents();
+    return;
+  }
+  const int c1 = min(c0 + a.chunk, Lk);
+  const int nc_b = (Lk + a.chunk - 1) / a.chunk;  // chunk CTAs of this sequence
+  const int nb = (c1 - c0 + kKeys - 1) / kKeys;
+  const int seq = sv.seq_ids[b];
+  uint32_t* err = sv.err;
+  auto stamp = [&](uint64_t* trace, int k) {
+    if (tid == 0) stamp_at(trace, k);
+  };
+  stamp(a.trace, 0);
+
+  if (warp == 4) {
+    tmem_alloc(tmem_slot, kTmemCols);
+    tmem_relinquish();
+  }
+  if (tid == 0) {
+    mbar_init(&bar[B_QFULL], 1);
+    for (int s = 0; s < 2; ++s) {
+      mbar_init(&bar[B_KVFULL + s], 1);
+      mbar_init(&bar[B_KVEMPTY + s], 1);
+      mbar_init(&bar[B_SFULL + s], 1);
+      mbar_init(&bar[B_SFREE + s], 4);
+    }
+    mbar_init(&bar[B_PFULL], 4);
+    mbar_init(&bar[B_PEMPTY], 1);
+    mbar_init(&bar[B_OFULL], 1);
+    mbar_init(&bar[B_DRAIN], 1);
+    *abort_flag = 0;
+    fence_barrier_init();
+  }
+  tc_fence_before();
+  __syncthreads();
+  tc_fence_after();
+  const uint32_t tmem = *tmem_slot;
+
+  if (warp == 4) {
+    // ------------------------------------------------------------ TMA + MMA issue
+    if (elect_one()) {
+      tma_prefetch_desc(&maps.q);
+      tma_prefetch_desc(&maps.kv);
+      // cache rows: [layer][K/V][max_batch][Hkv][max_seq]
+      const int krow = (((a.layer * 2 + 0) * a.kv.max_batch + seq) * Hkv + kvh) * a.kv.max_seq;
+      const int vrow = (((a.layer * 2 + 1) * a.kv.max_batch + seq) * Hkv + kvh) * a.kv.max_seq;
+      const int qrow = kvh * a.q_rows + base * G + row0;
+      const uint64_t pol_q = policy_evict_first();
+      const uint64_t pol = policy_evict_normal();  // the other row tiles read the same K/V blocks
+      int loaded = 0;
+      auto load_kv = [&](int j) {
+        const int st = j & 1;
+        const int key = c0 + j * kKeys;
+        uint8_t* sk = smem + Smem::k + st * kTile;
+        uint8_t* svb = smem + Smem::v + st * kTile;
+        mbar_arrive_expect_tx(&bar[B_KVFULL + st], 2 * kTile);
+        tma_load_2d(sk, &maps.kv, &bar[B_KVFULL + st], 0, krow + key, pol);
+        tma_load_2d(sk + kHalf, &maps.kv, &bar[B_KVFULL + st], 64, krow + key, pol);
+        tma_load_2d(svb, &maps.kv, &bar[B_KVFULL + st], 0, vrow + key, pol);
+        tma_load_2d(svb + kHalf, &maps.kv, &bar[B_KVFULL + st], 64, vrow + key, pol);
+        loaded = j + 1;
+      };
+      // blocks made only of prefix keys were written by earlier steps: load
+      // them before waiting for the previous kernel
+      const int first = min(nb, 2);
+      int pre = 0;
+      while (pre < first && c0 + (pre + 1) * kKeys <= P) load_kv(pre++);
+      pdl_wait();
+      pdl_launch_dependents();
+      mbar_arrive_expect_tx(&bar[B_QFULL], kTile);
+      tma_load_2d(smem + Smem::q, &maps.q, &bar[B_QFULL], 0, qrow, pol_q);
+      tma_load_2d(smem + Smem::q + kHalf, &maps.q, &bar[B_QFULL], 64, qrow, pol_q);
+      for (int j = pre; j < first; ++j) load_kv(j);
+      const uint32_t sq = smem_u32(smem + Smem::q);
+      const uint32_t sp = smem_u32(smem + Smem::p);
+      auto issue_pv = [&](int j) {
+        const uint32_t svv = smem_u32(smem + Smem::v + (j & 1) * kTile);
+#pragma unroll
+        for (int kk = 0; kk < kKeys / 16; ++kk) {
+          const uint64_t ad = sw128_kmajor_desc(sp + (kk >> 2) * kHalf + (kk & 3) * 32);
+          const uint64_t bd = sw128_mnmajor_desc(svv + kk * 16 * 128, kHalf);
+          tc_mma_bf16(tmem + kColO, ad, bd, kIdescPV, (j > 0 || kk > 0) ? 1u : 0u);
+        }
+      };
+      bool ok = mbar_wait(&bar[B_QFULL], 0, err, abort_flag);
+      stamp_at(a.trace, 1);
+      int waited = 0;  // K/V blocks whose arrival this thread has seen
+      for (int j = 0; j < nb && ok; ++j) {
+        const int st = j & 1;
+        ok = mbar_wait(&bar[B_KVFULL + st], (j >> 1) & 1, err, abort_flag);
+        if (!ok) break;
+        waited = j + 1;
+        if (j == 0) stamp_at(a.trace, 2);
+        if (j >= 2) ok = mbar_wait(&bar[B_SFREE + st], ((j - 2) >> 1) & 1, err, abort_flag);
+        if (!ok) break;
+        tc_fence_after();
+        const uint32_t sk = smem_u32(smem + Smem::k + st * kTile);
+#pragma unroll
+        for (int ks = 0; ks < 8; ++ks) {
+          const uint32_t off = (ks >> 2) * kHalf + (ks & 3) * 32;
+          tc_mma_bf16(tmem + st * kKeys, sw128_kmajor_desc(sq + off), sw128_kmajor_desc(sk + off), kIdescS,
+                      ks > 0 ? 1u : 0u);
+        }
+        tc_commit(&bar[B_SFULL + st]);
+        if (j == 0) stamp_at(a.trace, 11);
+        if (j >= 1) {
+          ok = mbar_wait(&bar[B_PFULL], (j - 1) & 1, err, abort_flag);
+          if (!ok) break;
+          tc_fence_after();
+          issue_pv(j - 1);
+          tc_commit(&bar[B_PEMPTY]);
+          tc_commit(&bar[B_KVEMPTY + ((j - 1) & 1)]);
+          if (j + 1 < nb) {
+            ok = mbar_wait(&bar[B_KVEMPTY + ((j - 1) & 1)], ((j - 1) >> 1) & 1, err, abort_flag);
+            if (!ok) break;
+            load_kv(j + 1);
+          }
+        }
+      }
+      if (ok) ok = mbar_wait(&bar[B_PFULL], (nb - 1) & 1, err, abort_flag);
+      stamp_at(a.trace, 12);
+      if (ok) {
+        tc_fence_after();
+        issue_pv(nb - 1);
+        tc_commit(&bar[B_OFULL]);
+      } else {
+        *abort_flag = 1;
+        // let issued MMAs and copies finish before the CTA's memory is released
+        tc_commit(&bar[B_DRAIN]);
+        mbar_wait(&bar[B_DRAIN], 0, nullptr, nullptr);
+        for (int j = waited; j < loaded; ++j) mbar_wait(&bar[B_KVFULL + (j & 1)], (j >> 1) & 1, nullptr, nullptr);
+      }
+    } else {
+      pdl_wait();
+      pdl_launch_dependents();
+    }
+    __syncwarp();
+  } else {
+    // ------------------------------------------------------------ softmax rows
+    pdl_wait();
+    pdl_launch_dependents();
+    const int r = warp * 32 + lane;
+    const int qr = row0 + r;
+    const bool row_ok = qr < rows;
+    const int node = row_ok ? qr / G : 0;
+    const uint64_t anc0 = sv.row_anc[2 * (base + node)];
+    const uint64_t anc1 = sv.row_anc[2 * (base + node) + 1];
+    const uint32_t tl = tmem + ((uint32_t)(warp * 32) << 16);  // this warp's TMEM lanes
+    const float sl2 = 1.4426950408889634f * 0.08838834764831845f;  // log2(e) / sqrt(128)
+    uint8_t* prow = smem + Smem::p + r * 128;
+    float m = -INFINITY, l = 0.f;
+    bool ok = true;
+    for (int j = 0; j < nb; ++j) {
+      const int st = j & 1;
+      const int key0 = c0 + j * kKeys;
+      const uint32_t ts = tl + st * kKeys;
+      ok = mbar_wait(&bar[B_SFULL + st], (j >> 1) & 1, err, abort_flag);
+      if (!__all_sync(0xffffffffu, ok)) {
+        ok = false;
+        *abort_flag = 1;
+        break;
+      }
+      if (j == 0) stamp(a.trace, 3);
+      tc_fence_after();
+      // visibility word of each 32-key piece (all ones when the whole block is
+      // prefix keys of this chunk)
+      const bool full = row_ok && key0 + kKeys <= min(P, c1);
+      auto vis = [&](int i) {
+        return full ? 0xffffffffu : (row_ok ? visible_word(key0 + 32 * i, P, c1, anc0, anc1) : 0u);
+      };
+      // pass 1: the block's row max (raw scores; the scale is positive)
+      float mx4[4] = {-INFINITY, -INFINITY, -INFINITY, -INFINITY};
+#pragma unroll 1
+      for (int i = 0; i < 4; ++i) {
+        uint32_t x[32];
+        tmem_ld32_async(ts + 32 * i, x);
+        tmem_wait_ld();
+        reg_fence32(x);
+        const uint32_t w = vis(i);
+#pragma unroll
+        for (int c = 0; c < 32; ++c) {
+          const float v = ((w >> c) & 1u) ? __uint_as_float(x[c]) : -INFINITY;
+          mx4[c & 3] = fmaxf(mx4[c & 3], v);
+        }
+      }
+      const float mblk = fmaxf(fmaxf(mx4[0], mx4[1]), fmaxf(mx4[2], mx4[3])) * sl2;
+      if (j == 0) stamp(a.trace, 8);
+      float corr = 1.f;
+      if (mblk > m + kRescaleLog2) {
+        corr = fast_exp2(m - mblk);  // 0 while nothing was visible
+        m = mblk;
+      }
+      const float nm = (m == -INFINITY) ? 0.f : -m;
+      if (j >= 1) {
+        // P.V of the previous block has finished: the P buffer is free and O is current
+        ok = mbar_wait(&bar[B_PEMPTY], (j - 1) & 1, err, abort_flag);
+        if (!__all_sync(0xffffffffu, ok)) {
+          ok = false;
+          *abort_flag = 1;
+          break;
+        }
+        tc_fence_after();
+        if (__any_sync(0xffffffffu, corr != 1.f)) {
+#pragma unroll 1
+          for (int i = 0; i < 4; ++i) {
+            uint32_t o[32];
+            tmem_ld32_async(tl + kColO + 32 * i, o);
+            tmem_wait_ld();
+            reg_fence32(o);
+#pragma unroll
+            for (int c = 0; c < 32; ++c) o[c] = __float_as_uint(__uint_as_float(o[c]) * corr);
+            tmem_st32_async(tl + kColO + 32 * i, o);
+          }
+          tmem_wait_st();
+        }
+      }
+      // pass 2: P = 2^(s - m) in fp16 into the K-major, 128-byte-swizzled A
+      // operand (16-byte chunk c of a 128-byte row lands at chunk c ^ (row & 7))
+      float ls4[4] = {0.f, 0.f, 0.f, 0.f};
+#pragma unroll 1
+      for (int i = 0; i < 4; ++i) {
+        uint32_t x[32];
+        tmem_ld32_async(ts + 32 * i, x);
+        tmem_wait_ld();
+        reg_fence32(x);
+        const uint32_t w = vis(i);
+        uint32_t pk[16];
+#pragma unroll
+        for (int c = 0; c < 16; ++c) {
+          const float s0 = ((w >> (2 * c)) & 1u) ? __uint_as_float(x[2 * c]) : -INFINITY;
+          const float s1 = ((w >> (2 * c + 1)) & 1u) ? __uint_as_float(x[2 * c + 1]) : -INFINITY;
+          const float p0 = fast_exp2(fmaf(s0, sl2, nm));
+          const float p1 = fast_exp2(fmaf(s1, sl2, nm));
+          ls4[c & 3] += p0 + p1;
+          const __half2 h2 = __floats2half2_rn(p0, p1);
+          pk[c] = *reinterpret_cast<const uint32_t*>(&h2);
+        }
+        uint8_t* dst = prow + (i >> 1) * kHalf;
+#pragma unroll
+        for (int q4 = 0; q4 < 4; ++q4) {
+          const int chunk = (i & 1) * 4 + q4;
+          *reinterpret_cast<uint4*>(dst + ((chunk ^ (r & 7)) << 4)) =
+              make_uint4(pk[4 * q4], pk[4 * q4 + 1], pk[4 * q4 + 2], pk[4 * q4 + 3]);
+        }
+      }
+      if (j == 0) stamp(a.trace, 9);
+      tc_fence_before();
+      fence_proxy_async_smem();
+      __syncwarp();
+      if (lane == 0) {
+        mbar_arrive(&bar[B_SFREE + st]);
+        mbar_arrive(&bar[B_PFULL]);
+      }
+      l = l * corr + ((ls4[0] + ls4[1]) + (ls4[2] + ls4[3]));
+    }
+    // ---- normalised output of this chunk, staged in shared memory (the K/V
+    // ring is idle once the last P.V has completed)
+    if (ok) ok = mbar_wait(&bar[B_OFULL], 0, err, abort_flag);
+    ok = __all_sync(0xffffffffu, ok);
+    stamp(a.trace, 4);
+    const bool any = l > 0.f;
+    const float inv = any ? 1.f / l : 0.f;
+    uint8_t* stg = smem + Smem::k;  // 128 rows x 512 B
+    if (ok) {
+      tc_fence_after();
+#pragma unroll 1
+      for (int i = 0; i < 4; ++i) {
+        uint32_t o[32];
+        tmem_ld32_async(tl + kColO + 32 * i, o);
+        tmem_wait_ld();
+        reg_fence32(o);
+#pragma unroll
+        for (int q4 = 0; q4 < 8; ++q4)
+          *stage_at(stg, r, i * 8 + q4) =
+              make_float4(__uint_as_float(o[4 * q4]) * inv, __uint_as_float(o[4 * q4 + 1]) * inv,
+                          __uint_as_float(o[4 * q4 + 2]) * inv, __uint_as_float(o[4 * q4 + 3]) * inv);
+      }
+    }
+    const int grp = (b * Hkv + kvh) * gridDim.y + blockIdx.y;
+    const size_t slot = (size_t)grp * a.n_chunks + blockIdx.x;
+    float* part_lse = a.part_lse + slot * kRows;
+    if (nc_b > 1 && ok) part_lse[r] = any ? m + __log2f(l) : -INFINITY;
+    named_sync_rows();
+    __nv_bfloat16* out = reinterpret_cast<__nv_bfloat16*>(a.out);
+    const int ld = a.Hq * 128;
+    const int valid = min(kRows, rows - row0);
+    if (nc_b == 1) {
+      // one chunk: each warp writes whole rows, lane = 4 columns, as split bf16
+      if (ok) {
+        for (int rr = warp; rr < valid; rr += 4) {
+          const float4 v = *stage_at(stg, rr, lane);
+          const int q2 = row0 + rr;
+          const int nd = q2 / G;
+          const int col = (kvh * G + (q2 - nd * G)) * 128 + lane * 4;
+          split_store4(out, base + nd, ld, col, v);
+        }
+      }
+    } else {
+      // partial rows, coalesced: lane = 4 columns of one row
+      float4* po = reinterpret_cast<float4*>(a.part_o + slot * kRows * 128);
+      if (ok)
+        for (int rr = warp; rr < valid; rr += 4) __stcg(po + rr * 32 + lane, *stage_at(stg, rr, lane));
+      __threadfence();
+      named_sync_rows();
+      stamp(a.trace, 5);
+      int* ctr = a.counters + 2 * grp;
+      if (tid == 0) {
+        bool met = false;
+        if (!*abort_flag) {
+          atomicAdd(ctr, 1);
+          met = spin_until_geq(ctr, nc_b, err);
+        }
+        *merge_ok = met ? 1 : 0;
+      }
+      named_sync_rows();
+      stamp(a.trace, 6);
+      if (*merge_ok) {
+        const int per = (valid + nc_b - 1) / nc_b;
+        const int rb = blockIdx.x * per;
+        const int R = max(0, min(valid, rb + per) - rb);
+        const float* lse0 = a.part_lse + (size_t)grp * a.n_chunks * kRows;
+        const float4* po0 = reinterpret_cast<const float4*>(a.part_o + (size_t)grp * a.n_chunks * kRows * 128);
+        // chunk weights 2^(lse_c - max) / sum per slice row, in shared memory [R][nc_b]
+        float* wsm = reinterpret_cast<float*>(smem + Smem::v);
+        for (int i = r; i < R * nc_b; i += 128) {
+          const int rr = i / nc_b, c = i - rr * nc_b;
+          wsm[i] = __ldcg(lse0 + c * kRows + rb + rr);
+        }
+        named_sync_rows();
+        if (r < R) {
+          float* wr = wsm + r * nc_b;
+          float mx = -INFINITY;
+          for (int c = 0; c < nc_b; ++c) mx = fmaxf(mx, wr[c]);
+          float sum = 0.f;
+          for (int c = 0; c < nc_b; ++c) {
+            const float w = fast_exp2(wr[c] - mx);  // 2^-inf = 0 for empty chunks
+            wr[c] = w;
+            sum += w;
+          }
+          const float wi = sum > 0.f ? 1.f / sum : 0.f;
+          for (int c = 0; c < nc_b; ++c) wr[c] *= wi;
+        }
+        named_sync_rows();
+        // warp per slice row, lane = 4 columns; all chunks' loads issued together
+        constexpr int kMaxMerge = 16;
+        for (int rr = warp; rr < R; rr += 4) {
+          const float* wr = wsm + rr * nc_b;
+          float4 acc = make_float4(0.f, 0.f, 0.f, 0.f);
+          for (int cb = 0; cb < nc_b; cb += kMaxMerge) {
+            float4 v[kMaxMerge];
+#pragma unroll
+            for (int u = 0; u < kMaxMerge; ++u)
+              v[u] = (cb + u < nc_b) ? __ldcg(po0 + ((size_t)(cb + u) * kRows + rb + rr) * 32 + lane)
+                                     : make_float4(0.f, 0.f, 0.f, 0.f);
+#pragma unroll
+            for (int u = 0; u < kMaxMerge; ++u) {
+              const float w = (cb + u < nc_b) ? wr[cb + u] : 0.f;
+              acc.x = fmaf(w, v[u].x, acc.x);
+              acc.y = fmaf(w, v[u].y, acc.y);
+              acc.z = fmaf(w, v[u].z, acc.z);
+              acc.w = fmaf(w, v[u].w, acc.w);
+            }
+          }
+          const int q2 = row0 + rb + rr;
+          const int nd = q2 / G;
+          const int col = (kvh * G + (q2 - nd * G)) * 128 + lane * 4;
+          split_store4(out, base + nd, ld, col, acc);
+        }
+        named_sync_rows();
+        stamp(a.trace, 7);
+        // the last chunk CTA to leave resets the group's counters for the next layer
+        if (tid == 0 && atomicAdd(ctr + 1, 1) == nc_b - 1) {
+          ctr[0] = 0;
+          ctr[1] = 0;
+        }
+      }
+    }
+  }
+  tc_fence_before();
+  __syncthreads();
+  if (warp == 4) {
+    tc_fence_after();
+    tmem_dealloc(tmem, kTmemCols);
+  }
+}
+
+size_t attention_tc_smem_bytes() { return Smem::dyn; }
+
+cudaError_t attention_tc_configure() {
+  cudaError_t e = cudaFuncSetAttribute(attn_tc_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                       (int)attention_tc_smem_bytes());
+  if (e != cudaSuccess) return e;
+  return cudaFuncSetAttribute(attn_tc_kernel, cudaFuncAttributePreferredSharedMemoryCarveout,
+                              (int)cudaSharedmemCarveoutMaxShared);
+}
+
+cudaError_t launch_attention_tc(const AttnArgs& a, const AttnTcMaps& maps, cudaStream_t s, bool pdl) {
+  cudaLaunchAttribute attr[1];
+  attr[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+  attr[0].val.programmaticStreamSerializationAllowed = 1;
+  cudaLaunchConfig_t cfg = {};
+  cfg.gridDim = dim3(a.n_chunks, (a.max_rows + kRows - 1) / kRows, a.sv.B * a.kv.Hkv);
+  cfg.blockDim = dim3(kThreads);
+  cfg.dynamicSmemBytes = attention_tc_smem_bytes();
+  cfg.stream = s;
+  cfg.attrs = attr;
+  cfg.numAttrs = pdl ? 1 : 0;
+  return cudaLaunchKernelEx(&cfg, attn_tc_kernel, maps, a);
+}
+
+}  // namespace spec

@@ -54,7 +54,8 @@ struct GemmTcArgs {
   const int32_t* P_step;
   const int32_t* seq_ids;
   const float2* rope_cs;  // [tokens][64]
-  __half* q_out;          // [tokens][Hq][128]
+  __half* q_out;          // [Hkv][q_rows][128]: row t*G + g holds head kvh*G + g of token t
+  int q_rows;             // rows per kv head in q_out (>= tokens * G)
   __half* k_cache;        // this layer's K base: [max_batch][Hkv][max_seq][128]
   __half* v_cache;
   size_t kv_seq_stride, kv_head_stride;
@@ -67,15 +68,49 @@ struct GemmTcArgs {
   uint32_t* err;
 };
 
+constexpr int kMaxGemmPhases = 4;
+
+// kernel parameters: the tensor maps of every phase (a0, a1, a2, b) and the phases
+struct GemmMaps {
+  CUtensorMap m[4 * kMaxGemmPhases];
+};
+struct GemmPhases {
+  int n_phases;
+  int epi[kMaxGemmPhases];
+  int* phase_bar;  // [n_phases - 1] CTAs done with each phase, zero at launch
+  uint32_t* err;
+  uint64_t* trace; // optional [grid][kMaxGemmPhases][8] %globaltimer stamps (see gemm_tc.cu)
+  int pf_next;     // k-blocks of the next phase each CTA brings into L2 once its loads for a phase are issued
+  int pf_ahead;    // within a phase, L2 prefetch distance in k-blocks ahead of the shared-memory ring (0: off)
+  GemmTcArgs ph[kMaxGemmPhases];
+};
+
+struct GemmPhase {
+  int epi;
+  const CUtensorMap *mA0, *mA1, *mA2, *mB;
+  GemmTcArgs args;
+};
+// One launch, a list of phases separated by grid-wide barriers.  The grid must
+// be co-resident in full when n_phases > 1 or any phase uses split-K.
+struct GemmMultiLaunch {
+  int bn, grid, n_phases;
+  int* phase_bar;
+  uint32_t* err;
+  uint64_t* trace;
+  int pf_next, pf_ahead;
+  GemmPhase ph[kMaxGemmPhases];
+};
+
 struct GemmTcLaunch {
   int bn, epi, grid;
   const CUtensorMap *mA0, *mA1, *mA2, *mB;
   GemmTcArgs args;
 };
 
-cudaError_t gemm_tc_launch(const GemmTcLaunch& L, cudaStream_t stream, bool pdl);
-uint32_t gemm_tc_smem_bytes(int bn, int epi);
-const void* gemm_tc_function(int bn, int epi);
+cudaError_t gemm_multi_launch(const GemmMultiLaunch& L, cudaStream_t stream, bool pdl);
+cudaError_t gemm_tc_launch(const GemmTcLaunch& L, cudaStream_t stream, bool pdl);  // one phase
+uint32_t gemm_tc_smem_bytes(int bn);
+const void* gemm_tc_function(int bn);
 
 // One verification step, as seen by the kernels.  Node ("row") r in [0, M)
 // belongs to batch entry b with node_off[b] <= r < node_off[b+1]; its local
@@ -130,6 +165,16 @@ cudaError_t launch_swiglu_f32(int M, int F, const float* gu, float* h, cudaStrea
 cudaError_t launch_gemm_simt_f32(const float* A, int lda, const float* W, int K, float* C, int ldc, int M, int N,
                                  cudaStream_t s);
 
+// A strided list of byte ranges to bring into L2: `rows` segments of `seg`
+// bytes at base + i * stride (base, stride and seg multiples of 16).
+struct L2Range {
+  const uint8_t* base;
+  size_t stride;
+  uint32_t seg;
+  int rows;
+};
+constexpr int kMaxL2Ranges = 3;
+
 // attention
 struct AttnArgs {
   StepView sv;
@@ -142,11 +187,28 @@ struct AttnArgs {
   float* part_lse;          // [M*Hq][n_chunks]
   int n_chunks, chunk;      // key chunking of [0, P_b + n_b)
   int max_rows;             // max over batch of n_b * (Hq/Hkv)
-  int* counters;            // [B][Hkv][row blocks] chunk arrivals, zero between launches
+  int q_rows;               // bf16 path: q is [Hkv][q_rows][hd], row node * G + g
+  int* counters;            // bf16 path: [groups][2] chunk arrivals / departures, zero between launches
+  // weights the next kernel streams, brought into L2 while attention (which
+  // moves little data) runs; issued before the wait on the previous kernel
+  L2Range pf[kMaxL2Ranges];
+  int n_pf;
+  uint64_t* trace;          // optional [256 CTAs][16] %globaltimer marks (attention_tc.cu)
 };
-cudaError_t launch_attention(int dtype, const AttnArgs& a, cudaStream_t s, bool pdl);
-size_t attention_smem_bytes();
-cudaError_t attention_configure();
+// fp32 models: one warp per (node, head)
+cudaError_t launch_attention_f32(const AttnArgs& a, cudaStream_t s);
+// bf16 models: tensor-core kernel; q map over [Hkv * q_rows][128] fp16, kv map
+// over the whole cache as [n_layers * 2 * max_batch * Hkv * max_seq][128] fp16,
+// both with 64 x 128 boxes and the 128-byte swizzle
+struct AttnTcMaps {
+  CUtensorMap q, kv;
+};
+constexpr int kAttnTcRows = 128;   // query rows per CTA
+constexpr int kAttnTcKeys = 128;   // keys per block; chunks are multiples of it
+constexpr int kAttnPartCtas = 256; // partial slots: chunked launches stay within this many CTAs
+cudaError_t launch_attention_tc(const AttnArgs& a, const AttnTcMaps& maps, cudaStream_t s, bool pdl);
+size_t attention_tc_smem_bytes();
+cudaError_t attention_tc_configure();
 
 // LM head reductions
 cudaError_t launch_top2_reduce(int M, int tiles, const Top2* part, int top_ld, int32_t* argmax, float* top1,

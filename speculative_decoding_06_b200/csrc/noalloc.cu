@@ -100,10 +100,10 @@ int setup_device(int dev, unsigned char** scratch, int* sms) {
     cudaDeviceProp prop;
     e = cudaGetDeviceProperties(&prop, dev);
     if (e == cudaSuccess)
-      e = cudaFuncSetAttribute(gemm_tc_function(64, GEMM_EPI_ARGMAX), cudaFuncAttributeMaxDynamicSharedMemorySize,
-                               (int)gemm_tc_smem_bytes(64, GEMM_EPI_ARGMAX));
+      e = cudaFuncSetAttribute(gemm_tc_function(64), cudaFuncAttributeMaxDynamicSharedMemorySize,
+                               (int)gemm_tc_smem_bytes(64));
     if (e == cudaSuccess)
-      e = cudaFuncSetAttribute(gemm_tc_function(64, GEMM_EPI_ARGMAX), cudaFuncAttributePreferredSharedMemoryCarveout,
+      e = cudaFuncSetAttribute(gemm_tc_function(64), cudaFuncAttributePreferredSharedMemoryCarveout,
                                (int)cudaSharedmemCarveoutMaxShared);
     if (e != cudaSuccess) {
       return SPEC_ERR_CUDA;

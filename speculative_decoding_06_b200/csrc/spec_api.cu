@@ -34,7 +34,8 @@ namespace {
 constexpr int kMaxNodesLimit = 128;  // ancestor bitmask is two 64-bit words
 constexpr int kMaxSplits = 16;
 constexpr int kGemmCounters = 8192;  // per-tile arrival counters of the split-K GEMMs
-constexpr int kMaxAttnChunks = 8;     // key chunks of one row block = one portable cluster
+constexpr int kMaxAttnChunks = 64;    // key chunks of one (sequence, kv head, row tile)
+constexpr int kCountersPerPhase = 2048; // two ints per split-K tile
 
 size_t align_up(size_t x, size_t a) { return (x + a - 1) / a * a; }
 int ceil_div(int a, int b) { return (a + b - 1) / b; }
@@ -50,8 +51,8 @@ struct WsLayout {
   size_t seq_len, pending, hist, err_sticky;
   // activations
   size_t x, xn, q, attn, hmlp, partial, part_o, part_lse, top_part, argmax, top1, top2, inv_freq;
-  size_t ss, gemm_ctr, attn_ctr;
-  int n_ss = 1, attn_ctr_n = 0;
+  size_t ss, gemm_ctr, attn_ctr, phase_bar;
+  int n_ss = 1, attn_ctr_n = 0, phase_bar_n = 0;
   size_t partial_bytes;
   // outputs (one device->host copy per step)
   size_t o_acc_len, o_acc_nodes, o_acc_tokens, o_bonus, o_end;
@@ -100,13 +101,21 @@ WsLayout make_layout(const spec_config& c) {
   if (c.dtype == SPEC_DTYPE_F32) pcols = std::max<size_t>(pcols, std::max<size_t>(2 * (size_t)c.ffn, c.vocab));
   L.partial_bytes = 4 * (size_t)L.Mpad * pcols;
   L.partial = take(L.partial_bytes);
-  L.part_o = take(4 * (size_t)L.Mmax * c.n_q_heads * L.chunks_cap * c.head_dim);
-  L.part_lse = take(4 * (size_t)L.Mmax * c.n_q_heads * L.chunks_cap);
+  if (c.dtype == SPEC_DTYPE_BF16) {
+    // chunked tensor-core attention: one [128 rows][hd] partial per CTA
+    L.part_o = take(4 * (size_t)kAttnPartCtas * kAttnTcRows * c.head_dim);
+    L.part_lse = take(4 * (size_t)kAttnPartCtas * kAttnTcRows);
+  } else {
+    L.part_o = take(4);
+    L.part_lse = take(4);
+  }
   L.top_part = take(sizeof(Top2) * (size_t)ceil_div(c.vocab, 128) * L.Mpad);
   L.n_ss = std::max(1, c.hidden / 128);
   L.ss = take(4 * (size_t)L.n_ss * L.Mpad);
   L.gemm_ctr = take(4 * (size_t)kGemmCounters);
-  L.attn_ctr_n = c.max_batch * c.n_kv_heads * ceil_div(c.max_nodes * (c.n_q_heads / c.n_kv_heads), 64);
+  L.phase_bar_n = 4 * (c.n_layers + 2);
+  L.phase_bar = take(4 * (size_t)L.phase_bar_n);
+  L.attn_ctr_n = 2 * kAttnPartCtas;
   L.attn_ctr = take(4 * (size_t)L.attn_ctr_n);
   L.argmax = take(4 * (size_t)L.Mpad);
   L.top1 = take(4 * (size_t)L.Mpad);
@@ -167,14 +176,15 @@ EncodeTiledFn get_encode_fn() {
 }
 
 // [rows][cols] bf16, row-major; boxes of 64 columns x box_rows rows, 128-byte swizzle
-bool make_tmap(CUtensorMap* m, const void* ptr, uint64_t rows, uint64_t cols, uint32_t box_rows) {
+bool make_tmap(CUtensorMap* m, const void* ptr, uint64_t rows, uint64_t cols, uint32_t box_rows,
+               CUtensorMapDataType dt = CU_TENSOR_MAP_DATA_TYPE_BFLOAT16) {
   EncodeTiledFn enc = get_encode_fn();
   if (!enc) return false;
   cuuint64_t dims[2] = {cols, rows};
   cuuint64_t strides[1] = {cols * 2};
   cuuint32_t box[2] = {64, box_rows};
   cuuint32_t estr[2] = {1, 1};
-  return enc(m, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, const_cast<void*>(ptr), dims, strides, box, estr,
+  return enc(m, dt, 2, const_cast<void*>(ptr), dims, strides, box, estr,
              CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
              CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
 }
@@ -189,6 +199,7 @@ struct GemmPlan {
 
 struct StepPlan {
   int B, M, max_n, max_lk, n_chunks, chunk, max_rows;
+  int grid_all;  // co-resident CTAs of the multi-phase GEMM launches
   GemmPlan qkv, o, gu, down, lm;
 };
 
@@ -211,6 +222,7 @@ struct spec_handle {
   std::vector<LayerMaps> maps;
   CUtensorMap map_lm;
   CUtensorMap map_xn[2], map_attn[2], map_h[2];  // B operands for BN = 64, 128
+  AttnTcMaps attn_maps;                           // q and the K/V cache (fp16)
   int resident[2][4] = {{0, 0, 0, 0}, {0, 0, 0, 0}};   // co-resident CTAs per SM [bn][epi]
   int occ_api[2][4] = {{0, 0, 0, 0}, {0, 0, 0, 0}};    // what the occupancy query reported
   // host mirror of per-sequence state
@@ -226,8 +238,18 @@ struct spec_handle {
   std::map<GraphKey, cudaGraphExec_t> graphs;
   bool use_pdl = true;
   int max_splits = 16;    // split-K cap
-  int max_chunks = 8;     // attention key-chunk cap (one cluster per row block)
+  int max_chunks = kMaxAttnChunks;  // attention key-chunk cap
   int resident_cap = 0;   // 0: as many CTAs per SM as fit
+  // L2 prefetch of weights ahead of the GEMM that streams them
+  // (all off by default: measured on B200 they only took bandwidth from the
+  // streams they were meant to feed)
+  int pf_next = 0;        // k-blocks of the next phase, per CTA, at the end of a phase's loads
+  int pf_ahead = 0;       // in-phase distance in k-blocks (0: off)
+  int pf_attn_o = 0;      // attention brings the O projection into L2
+  int pf_attn_gu = 0;     // ... and the first columns of every gate/up row
+  uint64_t* trace = nullptr;  // optional GEMM timeline of one layer's launch
+  size_t trace_bytes = 0;
+  int trace_layer = 0;
   std::string err;
   // profiler: an event pair per launch
   bool prof = false;
@@ -318,15 +340,21 @@ StepPlan make_plan(const spec_handle* h, int B, int M, int max_n, int max_lk) {
   s.max_lk = max_lk;
   const int G = c.n_q_heads / c.n_kv_heads;
   s.max_rows = max_n * G;
-  const int rowblocks = ceil_div(s.max_rows, 64);
-  const int ctas_per_chunk = B * c.n_kv_heads * rowblocks;
-  const int ccap = std::min(h->lay.chunks_cap, h->max_chunks);
-  int want = std::max(1, ceil_div(2 * h->sm_count, ctas_per_chunk));
-  want = std::min(want, ccap);
-  int chunk = std::max(256, (int)align_up(ceil_div(max_lk, want), 64));
-  chunk = std::max(chunk, (int)align_up(ceil_div(max_lk, ccap), 64));
-  s.chunk = chunk;
-  s.n_chunks = ceil_div(max_lk, chunk);
+  if (c.dtype == SPEC_DTYPE_BF16) {
+    // Key chunks only while the (sequence, kv head, row tile) groups leave SMs
+    // idle; the chunk CTAs of a group meet, so a chunked grid stays within one
+    // CTA per SM (all co-resident) and within the partial slots.
+    const int groups = B * c.n_kv_heads * ceil_div(s.max_rows, kAttnTcRows);
+    const int blocks = ceil_div(max_lk, kAttnTcKeys);
+    const int cap = std::min(h->sm_count, kAttnPartCtas);
+    int nc = 1;
+    if (2 * groups <= cap) nc = std::max(1, std::min({blocks, cap / groups, h->max_chunks}));
+    s.chunk = ceil_div(blocks, nc) * kAttnTcKeys;
+    s.n_chunks = ceil_div(max_lk, s.chunk);
+  } else {
+    s.chunk = max_lk;
+    s.n_chunks = 1;
+  }
   const int nqkv = (c.n_q_heads + 2 * c.n_kv_heads) * c.head_dim;
   const int qd = c.n_q_heads * c.head_dim;
   s.qkv = plan_gemm(h, 128, nqkv, c.hidden, M, GEMM_EPI_QKV);
@@ -334,6 +362,12 @@ StepPlan make_plan(const spec_handle* h, int B, int M, int max_n, int max_lk) {
   s.gu = plan_gemm(h, 64, c.ffn, c.hidden, M, GEMM_EPI_SWIGLU);
   s.down = plan_gemm(h, 128, c.hidden, c.ffn, M, GEMM_EPI_RESID);
   s.lm = plan_gemm(h, 128, c.vocab, c.hidden, M, GEMM_EPI_ARGMAX);
+  {
+    const int bi = s.qkv.bn == 64 ? 0 : 1;
+    int per_sm = std::max(1, h->resident[bi][0]);
+    if (h->resident_cap > 0) per_sm = std::min(per_sm, h->resident_cap);
+    s.grid_all = per_sm * h->sm_count;
+  }
   return s;
 }
 
@@ -417,6 +451,7 @@ cudaError_t enqueue_step(spec_handle* h, const StepPlan& sp, int mode, bool dbg)
     // arrival counters start every step at zero, whatever an earlier failed step left behind
     cudaError_t e0 = cudaMemsetAsync(gctr, 0, 4 * (size_t)kGemmCounters, st);
     if (e0 == cudaSuccess) e0 = cudaMemsetAsync(h->ws + L.attn_ctr, 0, 4 * (size_t)L.attn_ctr_n, st);
+    if (e0 == cudaSuccess) e0 = cudaMemsetAsync(h->ws + L.phase_bar, 0, 4 * (size_t)L.phase_bar_n, st);
     if (e0 != cudaSuccess) return e0;
   }
   LK(SPEC_PROF_EMBED_META, 1,
@@ -436,77 +471,147 @@ cudaError_t enqueue_step(spec_handle* h, const StepPlan& sp, int mode, bool dbg)
   aa.chunk = sp.chunk;
   aa.max_rows = sp.max_rows;
   aa.counters = h->W<int>(L.attn_ctr);
+  aa.q_rows = L.Mpad * (c.n_q_heads / c.n_kv_heads);
+
+  // ---- GEMM phases of the bf16 path (split-K counters: one region per phase slot)
+  const int bi = sp.qkv.bn == 64 ? 0 : 1;
+  auto as_phase = [](const GemmTcLaunch& g) {
+    GemmPhase q{};
+    q.epi = g.epi;
+    q.mA0 = g.mA0;
+    q.mA1 = g.mA1;
+    q.mA2 = g.mA2;
+    q.mB = g.mB;
+    q.args = g.args;
+    return q;
+  };
+  auto phase_qkv = [&](int l, int slot) {
+    const LayerMaps& mp = h->maps[l];
+    __half* kc = reinterpret_cast<__half*>(h->kv.base) + (size_t)l * h->kv.layer_stride();
+    GemmTcLaunch g = gemm_launch(sp.qkv, GEMM_EPI_QKV, nqkv, d, M, &mp.wq, &mp.wk, &mp.wv, &h->map_xn[bi], qd, kvd,
+                                 kvd, sv.err);
+    g.args.ss_in = ss;
+    g.args.n_ss = L.n_ss;
+    g.args.ss_ld = L.Mpad;
+    g.args.norm_d = d;
+    g.args.eps = c.rms_eps;
+    g.args.part = part;
+    g.args.split_stride = (size_t)L.Mpad * nqkv;
+    g.args.counters = gctr + slot * kCountersPerPhase;
+    g.args.row_seq = sv.row_seq;
+    g.args.row_local = sv.row_local;
+    g.args.P_step = sv.P_step;
+    g.args.seq_ids = sv.seq_ids;
+    g.args.rope_cs = sv.rope_cs;
+    g.args.q_out = reinterpret_cast<__half*>(q);
+    g.args.q_rows = L.Mpad * (c.n_q_heads / c.n_kv_heads);
+    g.args.k_cache = kc;
+    g.args.v_cache = kc + h->kv.kv_stride();
+    g.args.kv_seq_stride = h->kv.seq_stride();
+    g.args.kv_head_stride = h->kv.head_stride();
+    g.args.Hq = c.n_q_heads;
+    g.args.Hkv = c.n_kv_heads;
+    g.args.max_seq = c.max_seq;
+    return as_phase(g);
+  };
+  auto phase_o = [&](int l, int slot) {
+    GemmTcLaunch g = gemm_launch(sp.o, GEMM_EPI_RESID, d, qd, M, &h->maps[l].wo, nullptr, nullptr, &h->map_attn[bi],
+                                 d, 0, 0, sv.err);
+    g.args.part = part;
+    g.args.split_stride = (size_t)L.Mpad * d;
+    g.args.counters = gctr + slot * kCountersPerPhase;
+    g.args.x = x;
+    g.args.norm_w_next = reinterpret_cast<const __nv_bfloat16*>(h->layers[l].mlp_norm);
+    g.args.xn_out = reinterpret_cast<__nv_bfloat16*>(xn);
+    g.args.ss_out = ss;
+    g.args.ss_ld = L.Mpad;
+    return as_phase(g);
+  };
+  auto phase_gu = [&](int l) {
+    GemmTcLaunch g = gemm_launch(sp.gu, GEMM_EPI_SWIGLU, c.ffn, d, M, &h->maps[l].wg, &h->maps[l].wu, nullptr,
+                                 &h->map_xn[bi], 0, 0, 0, sv.err);
+    g.args.ss_in = ss;
+    g.args.n_ss = L.n_ss;
+    g.args.ss_ld = L.Mpad;
+    g.args.norm_d = d;
+    g.args.eps = c.rms_eps;
+    g.args.out_bf16 = reinterpret_cast<__nv_bfloat16*>(hm);
+    g.args.ld_out = c.ffn;
+    return as_phase(g);
+  };
+  auto phase_down = [&](int l, int slot) {
+    const void* next_norm = (l + 1 < c.n_layers) ? h->layers[l + 1].attn_norm : h->final_norm;
+    GemmTcLaunch g = gemm_launch(sp.down, GEMM_EPI_RESID, d, c.ffn, M, &h->maps[l].wd, nullptr, nullptr,
+                                 &h->map_h[bi], d, 0, 0, sv.err);
+    g.args.part = part;
+    g.args.split_stride = (size_t)L.Mpad * d;
+    g.args.counters = gctr + slot * kCountersPerPhase;
+    g.args.x = x;
+    g.args.norm_w_next = reinterpret_cast<const __nv_bfloat16*>(next_norm);
+    g.args.xn_out = reinterpret_cast<__nv_bfloat16*>(xn);
+    g.args.ss_out = ss;
+    g.args.ss_ld = L.Mpad;
+    return as_phase(g);
+  };
+  auto phase_lm = [&]() {
+    GemmTcLaunch g = gemm_launch(sp.lm, GEMM_EPI_ARGMAX, c.vocab, d, M, &h->map_lm, nullptr, nullptr, &h->map_xn[bi],
+                                 c.vocab, 0, 0, sv.err);
+    g.args.top_part = h->W<Top2>(L.top_part);
+    g.args.top_ld = L.Mpad;
+    g.args.dbg_logits = dbg ? h->dbg_logits : nullptr;
+    g.args.ss_in = ss;
+    g.args.n_ss = L.n_ss;
+    g.args.ss_ld = L.Mpad;
+    g.args.norm_d = d;
+    g.args.eps = c.rms_eps;
+    return as_phase(g);
+  };
+  if (dt == 1) {
+    GemmMultiLaunch m{};
+    m.bn = sp.qkv.bn;
+    m.grid = sp.grid_all;
+    m.err = sv.err;
+    m.phase_bar = h->W<int>(L.phase_bar);
+    m.n_phases = 1;
+    m.ph[0] = phase_qkv(0, 0);
+    LK(SPEC_PROF_GEMM_QKV, 1, gemm_multi_launch(m, st, pdl));
+  }
 
   for (int l = 0; l < c.n_layers; ++l) {
     const spec_layer_weights& lw = h->layers[l];
     const void* next_norm = (l + 1 < c.n_layers) ? h->layers[l + 1].attn_norm : h->final_norm;
     aa.layer = l;
     if (dt == 1) {
-      const LayerMaps& mp = h->maps[l];
-      const int bi = sp.qkv.bn == 64 ? 0 : 1;
-      __half* kc = reinterpret_cast<__half*>(h->kv.base) + (size_t)l * h->kv.layer_stride();
-      // QKV (+ norm scale, rotary, q and K/V cache store in the last CTA of each head)
-      GemmTcLaunch g = gemm_launch(sp.qkv, GEMM_EPI_QKV, nqkv, d, M, &mp.wq, &mp.wk, &mp.wv, &h->map_xn[bi], qd,
-                                   kvd, kvd, sv.err);
-      g.args.ss_in = ss;
-      g.args.n_ss = L.n_ss;
-      g.args.ss_ld = L.Mpad;
-      g.args.norm_d = d;
-      g.args.eps = c.rms_eps;
-      g.args.part = part;
-      g.args.split_stride = (size_t)L.Mpad * nqkv;
-      g.args.counters = gctr;
-      g.args.row_seq = sv.row_seq;
-      g.args.row_local = sv.row_local;
-      g.args.P_step = sv.P_step;
-      g.args.seq_ids = sv.seq_ids;
-      g.args.rope_cs = sv.rope_cs;
-      g.args.q_out = reinterpret_cast<__half*>(q);
-      g.args.k_cache = kc;
-      g.args.v_cache = kc + h->kv.kv_stride();
-      g.args.kv_seq_stride = h->kv.seq_stride();
-      g.args.kv_head_stride = h->kv.head_stride();
-      g.args.Hq = c.n_q_heads;
-      g.args.Hkv = c.n_kv_heads;
-      g.args.max_seq = c.max_seq;
-      LK(SPEC_PROF_GEMM_QKV, 1, gemm_tc_launch(g, st, pdl));
-      // attention (chunks + merge in the last chunk's CTA)
-      LK(SPEC_PROF_ATTENTION, 1, launch_attention(dt, aa, st, pdl));
-      // O projection (+ residual, next operand x*w_mlp, sums of squares)
-      GemmTcLaunch go = gemm_launch(sp.o, GEMM_EPI_RESID, d, qd, M, &mp.wo, nullptr, nullptr, &h->map_attn[bi], d,
-                                    0, 0, sv.err);
-      go.args.part = part;
-      go.args.split_stride = (size_t)L.Mpad * d;
-      go.args.counters = gctr;
-      go.args.x = x;
-      go.args.norm_w_next = reinterpret_cast<const __nv_bfloat16*>(lw.mlp_norm);
-      go.args.xn_out = reinterpret_cast<__nv_bfloat16*>(xn);
-      go.args.ss_out = ss;
-      go.args.ss_ld = L.Mpad;
-      LK(SPEC_PROF_GEMM_O, 1, gemm_tc_launch(go, st, pdl));
-      // gate/up (+ norm scale, SwiGLU)
-      GemmTcLaunch gg = gemm_launch(sp.gu, GEMM_EPI_SWIGLU, c.ffn, d, M, &mp.wg, &mp.wu, nullptr, &h->map_xn[bi], 0,
-                                    0, 0, sv.err);
-      gg.args.ss_in = ss;
-      gg.args.n_ss = L.n_ss;
-      gg.args.ss_ld = L.Mpad;
-      gg.args.norm_d = d;
-      gg.args.eps = c.rms_eps;
-      gg.args.out_bf16 = reinterpret_cast<__nv_bfloat16*>(hm);
-      gg.args.ld_out = c.ffn;
-      LK(SPEC_PROF_GEMM_GATE_UP, 1, gemm_tc_launch(gg, st, pdl));
-      // down (+ residual, next operand x*w_next, sums of squares)
-      GemmTcLaunch gd = gemm_launch(sp.down, GEMM_EPI_RESID, d, c.ffn, M, &mp.wd, nullptr, nullptr, &h->map_h[bi],
-                                    d, 0, 0, sv.err);
-      gd.args.part = part;
-      gd.args.split_stride = (size_t)L.Mpad * d;
-      gd.args.counters = gctr;
-      gd.args.x = x;
-      gd.args.norm_w_next = reinterpret_cast<const __nv_bfloat16*>(next_norm);
-      gd.args.xn_out = reinterpret_cast<__nv_bfloat16*>(xn);
-      gd.args.ss_out = ss;
-      gd.args.ss_ld = L.Mpad;
-      LK(SPEC_PROF_GEMM_DOWN, 1, gemm_tc_launch(gd, st, pdl));
+      // attention of layer l (its QKV ran in the previous launch), then one
+      // launch: O, gate/up, down, and the next layer's QKV or the LM head
+      aa.n_pf = 0;
+      if (h->pf_attn_o) {
+        const size_t row = 2 * (size_t)qd;
+        aa.pf[aa.n_pf++] = L2Range{static_cast<const uint8_t*>(lw.wo), row, (uint32_t)row, d};
+      }
+      if (h->pf_attn_gu > 0) {
+        const uint32_t seg = 2 * (uint32_t)std::min(h->pf_attn_gu, d) & ~15u;
+        if (seg > 0) {
+          aa.pf[aa.n_pf++] = L2Range{static_cast<const uint8_t*>(lw.w_gate), 2 * (size_t)d, seg, c.ffn};
+          aa.pf[aa.n_pf++] = L2Range{static_cast<const uint8_t*>(lw.w_up), 2 * (size_t)d, seg, c.ffn};
+        }
+      }
+      aa.trace = (h->trace && l == h->trace_layer) ? h->trace + (size_t)2 * h->sm_count * kMaxGemmPhases * 8 : nullptr;
+      LK(SPEC_PROF_ATTENTION, 1, launch_attention_tc(aa, h->attn_maps, st, pdl));
+      GemmMultiLaunch m{};
+      m.pf_next = h->pf_next;
+      m.pf_ahead = h->pf_ahead;
+      m.bn = sp.qkv.bn;
+      m.grid = sp.grid_all;
+      m.err = sv.err;
+      m.phase_bar = h->W<int>(L.phase_bar) + 4 * (l + 1);
+      m.n_phases = 4;
+      m.ph[0] = phase_o(l, 0);
+      m.ph[1] = phase_gu(l);
+      m.ph[2] = phase_down(l, 2);
+      m.ph[3] = (l + 1 < c.n_layers) ? phase_qkv(l + 1, 3) : phase_lm();
+      if (h->trace && l == h->trace_layer) m.trace = h->trace;
+      LK(SPEC_PROF_GEMM_LAYER, 1, gemm_multi_launch(m, st, pdl));
     } else {
       const float* xf = reinterpret_cast<const float*>(xn);
       LK(SPEC_PROF_GEMM_QKV, 1, launch_gemm_simt_f32(xf, d, (const float*)lw.wq, d, part, nqkv, M, qd, st));
@@ -515,7 +620,7 @@ cudaError_t enqueue_step(spec_handle* h, const StepPlan& sp, int mode, bool dbg)
          launch_gemm_simt_f32(xf, d, (const float*)lw.wv, d, part + qd + kvd, nqkv, M, kvd, st));
       LK(SPEC_PROF_ROPE_KV, 1,
          launch_qkv_rope_store(dt, sv, 1, part, 0, c.n_q_heads, c.n_kv_heads, c.head_dim, q, h->kv, l, st, false));
-      LK(SPEC_PROF_ATTENTION, 1, launch_attention(dt, aa, st, false));
+      LK(SPEC_PROF_ATTENTION, 1, launch_attention_f32(aa, st));
       LK(SPEC_PROF_GEMM_O, 1, launch_gemm_simt_f32((const float*)attn, qd, (const float*)lw.wo, qd, part, d, M, d, st));
       LK(SPEC_PROF_RESID_NORM, 1, launch_residual_norm(dt, M, d, 1, part, 0, x, xn, lw.mlp_norm, c.rms_eps, st, false));
       LK(SPEC_PROF_GEMM_GATE_UP, 1,
@@ -531,18 +636,7 @@ cudaError_t enqueue_step(spec_handle* h, const StepPlan& sp, int mode, bool dbg)
 
   int32_t* amax = h->W<int32_t>(L.argmax);
   if (dt == 1) {
-    const int bi = sp.lm.bn == 64 ? 0 : 1;
-    GemmTcLaunch g = gemm_launch(sp.lm, GEMM_EPI_ARGMAX, c.vocab, d, M, &h->map_lm, nullptr, nullptr, &h->map_xn[bi],
-                                 c.vocab, 0, 0, sv.err);
-    g.args.top_part = h->W<Top2>(L.top_part);
-    g.args.top_ld = L.Mpad;
-    g.args.dbg_logits = dbg ? h->dbg_logits : nullptr;
-    g.args.ss_in = h->W<float>(L.ss);
-    g.args.n_ss = L.n_ss;
-    g.args.ss_ld = L.Mpad;
-    g.args.norm_d = d;
-    g.args.eps = c.rms_eps;
-    LK(SPEC_PROF_LM_HEAD, 1, gemm_tc_launch(g, st, pdl));
+    // the LM head ran as the last phase of the last layer's launch
     LK(SPEC_PROF_LM_REDUCE, 1,
        launch_top2_reduce(M, sp.lm.tiles_o, h->W<Top2>(L.top_part), L.Mpad, amax, h->W<float>(L.top1),
                           h->W<float>(L.top2), st, pdl));
@@ -798,6 +892,10 @@ int spec_init(const spec_config* cfg, const spec_weights* w, void* kv_cache, siz
     if (const char* q = strstr(t, "chunks=")) if (sscanf(q + 7, "%d", &v) == 1 && v >= 1 && v <= kMaxAttnChunks) h->max_chunks = v;
     if (const char* q = strstr(t, "pdl=")) if (sscanf(q + 4, "%d", &v) == 1) h->use_pdl = v != 0;
     if (const char* q = strstr(t, "per_sm=")) if (sscanf(q + 7, "%d", &v) == 1 && v >= 0) h->resident_cap = v;
+    if (const char* q = strstr(t, "pf_next=")) if (sscanf(q + 8, "%d", &v) == 1 && v >= 0) h->pf_next = v;
+    if (const char* q = strstr(t, "pf_ahead=")) if (sscanf(q + 9, "%d", &v) == 1 && v >= 0) h->pf_ahead = v;
+    if (const char* q = strstr(t, "pf_o=")) if (sscanf(q + 5, "%d", &v) == 1) h->pf_attn_o = v != 0;
+    if (const char* q = strstr(t, "pf_gu=")) if (sscanf(q + 6, "%d", &v) == 1 && v >= 0) h->pf_attn_gu = v;
   }
   if (cudaGetDevice(&h->device) != cudaSuccess) return bail(SPEC_ERR_CUDA, "cudaGetDevice");
   cudaDeviceProp prop;
@@ -823,8 +921,24 @@ int spec_init(const spec_config* cfg, const spec_weights* w, void* kv_cache, siz
     return bail(SPEC_ERR_CUDA, "smem attribute");
   if (c.dtype == SPEC_DTYPE_BF16) {
     if (!get_encode_fn()) return bail(SPEC_ERR_CUDA, "cuTensorMapEncodeTiled unavailable");
-    if (attention_configure() != cudaSuccess) return bail(SPEC_ERR_CUDA, "smem attribute");
+    if (attention_tc_configure() != cudaSuccess) return bail(SPEC_ERR_CUDA, "smem attribute");
     const int qd = c.n_q_heads * c.head_dim, kvd = c.n_kv_heads * c.head_dim;
+    {
+      // q as [Hkv * q_rows][128] and the cache as [layers * 2 * batch * Hkv * max_seq][128], fp16;
+      // TMA row coordinates are 32-bit
+      const uint64_t cache_rows = (uint64_t)c.n_layers * 2 * c.max_batch * c.n_kv_heads * c.max_seq;
+      if (cache_rows + 128 >= (1ull << 31)) return bail(SPEC_ERR_CAPACITY, "cache too large for 32-bit rows");
+      const uint64_t q_rows = (uint64_t)c.n_kv_heads * lay.Mpad * (c.n_q_heads / c.n_kv_heads);
+      if (!make_tmap(&h->attn_maps.q, h->ws + lay.q, q_rows, 128, 128, CU_TENSOR_MAP_DATA_TYPE_FLOAT16) ||
+          !make_tmap(&h->attn_maps.kv, kv_cache, cache_rows, 128, 128, CU_TENSOR_MAP_DATA_TYPE_FLOAT16))
+        return bail(SPEC_ERR_CUDA, "tensor map");
+      // attention reads whole 128-key blocks (P = 0 beyond a sequence's keys): every
+      // slot must hold a finite value from the start, and q rows too
+      if (cudaMemsetAsync(kv_cache, 0, kv_bytes_of(c), h->stream) != cudaSuccess ||
+          cudaMemsetAsync(h->ws + lay.q, 0, 2 * (size_t)lay.Mpad * qd, h->stream) != cudaSuccess ||
+          cudaStreamSynchronize(h->stream) != cudaSuccess)
+        return bail(SPEC_ERR_CUDA, "cache init");
+    }
     h->maps.resize(c.n_layers);
     for (int l = 0; l < c.n_layers; ++l) {
       const spec_layer_weights& lw = h->layers[l];
@@ -846,8 +960,8 @@ int spec_init(const spec_config* cfg, const spec_weights* w, void* kv_cache, siz
     }
     for (int i = 0; i < 2; ++i)
       for (int e = 0; e < 4; ++e) {
-        const void* fn = gemm_tc_function(bns[i], e);
-        const int smem = (int)gemm_tc_smem_bytes(bns[i], e);
+        const void* fn = gemm_tc_function(bns[i]);
+        const int smem = (int)gemm_tc_smem_bytes(bns[i]);
         if (cudaFuncSetAttribute(fn, cudaFuncAttributeMaxDynamicSharedMemorySize, smem) != cudaSuccess ||
             cudaFuncSetAttribute(fn, cudaFuncAttributePreferredSharedMemoryCarveout,
                                  (int)cudaSharedmemCarveoutMaxShared) != cudaSuccess)
@@ -1037,6 +1151,23 @@ int spec_profile_read(spec_handle* h, double* ms, int64_t* launches) {
 }
 
 int spec_step_launches(spec_handle* h) { return h ? h->launches : 0; }
+
+// GEMM marks [2 * SMs][phases][8], then attention marks [kAttnPartCtas][16]
+static size_t trace_words(const spec_handle* h) {
+  return (size_t)2 * h->sm_count * kMaxGemmPhases * 8 + (size_t)kAttnPartCtas * 16;
+}
+
+int spec_set_trace(spec_handle* h, uint64_t* device_buf, size_t bytes, int layer) {
+  if (!h) return SPEC_ERR_ARG;
+  if (device_buf && bytes < trace_words(h) * sizeof(uint64_t))
+    return fail(h, SPEC_ERR_CAPACITY, "trace buffer too small");
+  h->trace = device_buf;
+  h->trace_bytes = bytes;
+  h->trace_layer = layer;
+  for (auto& kv : h->graphs) cudaGraphExecDestroy(kv.second);  // graphs bake the pointer in
+  h->graphs.clear();
+  return SPEC_OK;
+}
 
 int spec_info(spec_handle* h, int B, int n_nodes, int prefix, char* buf, size_t n) {
   if (!h || !buf || n == 0) return SPEC_ERR_ARG;

@@ -31,7 +31,7 @@ SPEC_DEBUG_LOGITS = 2
 SPEC_NO_GRAPH = 4
 
 PROF_CLASSES = ("embed_meta", "gemm_qkv", "rope_kv_store", "attention", "gemm_o", "resid_norm", "gemm_gate_up",
-                "gemm_down", "lm_head", "lm_reduce", "accept_walk", "kv_compact")
+                "gemm_down", "lm_head", "lm_reduce", "accept_walk", "kv_compact", "gemm_layer")
 
 ERR_NAMES = {0: "SPEC_OK", -1: "SPEC_ERR_ARG", -2: "SPEC_ERR_TREE", -3: "SPEC_ERR_TOKEN", -4: "SPEC_ERR_CAPACITY",
              -5: "SPEC_ERR_ROOT", -6: "SPEC_ERR_CUDA", -7: "SPEC_ERR_TIMEOUT", -8: "SPEC_ERR_STATE"}
@@ -85,6 +85,7 @@ _SIGNATURES = {
     "spec_profile": (ctypes.c_int, [_h, ctypes.c_int]),
     "spec_profile_read": (ctypes.c_int, [_h, ctypes.POINTER(ctypes.c_double), ctypes.POINTER(ctypes.c_int64)]),
     "spec_step_launches": (ctypes.c_int, [_h]),
+    "spec_set_trace": (ctypes.c_int, [_h, _vp, ctypes.c_size_t, ctypes.c_int]),
     "spec_info": (ctypes.c_int, [_h, ctypes.c_int, ctypes.c_int, ctypes.c_int, ctypes.c_char_p, ctypes.c_size_t]),
     "spec_io_bytes": (ctypes.c_int, [_h, ctypes.POINTER(ctypes.c_size_t), ctypes.POINTER(ctypes.c_size_t)]),
     "spec_lm_head_argmax_noalloc": (ctypes.c_int, [_vp, _vp, _vp, ctypes.c_int, ctypes.c_int, ctypes.c_int,
@@ -143,6 +144,7 @@ spec_validate_tree = _bind("spec_validate_tree")
 spec_profile = _bind("spec_profile")
 spec_profile_read = _bind("spec_profile_read")
 spec_step_launches = _bind("spec_step_launches")
+spec_set_trace = _bind("spec_set_trace")
 spec_info = _bind("spec_info")
 spec_io_bytes = _bind("spec_io_bytes")
 spec_lm_head_argmax_noalloc = _bind("spec_lm_head_argmax_noalloc")
