@@ -210,16 +210,17 @@ SPEC_API int spec_io_bytes(spec_handle* h, size_t* h2d, size_t* d2h);
  * tokens, written to buf (n bytes, NUL-terminated). */
 SPEC_API int spec_info(spec_handle* h, int B, int n_nodes, int prefix, char* buf, size_t n);
 /* Optional timeline of decoder layer `layer` (bf16 models), in %globaltimer
- * stamps (uint64 ns); NULL turns it off.  device_buf holds 2 * SMs * 32 + 4096
- * entries: first the layer's GEMM launch, [2 * SMs CTAs][4 phases][8] (producer
- * starts the phase, may load its activations, has issued its last load;
- * epilogue starts the phase, first accumulator complete, split-K rendezvous
- * passed, units done, phase counted at the grid barrier), then its attention
- * launch, [256 CTAs][16] (start, Q landed, first K/V block landed, first
- * scores ready, output accumulated, partial written, chunk rendezvous passed,
- * merge done, first block's max found, first block's P written, first scores
- * issued, last P seen by the issuer).  Entries of CTAs that did not run stay as
- * they were. */
+ * stamps (uint64 ns); NULL turns it off.  device_buf holds 2 * SMs * 64 + 4096
+ * entries: first the layer's GEMM launch, [2 * SMs CTAs][4 phases][16] (0-7:
+ * producer starts the phase, may load its activations, has issued its last
+ * load; epilogue starts the phase, first accumulator complete, split-K
+ * rendezvous passed, units done, phase counted at the grid barrier; 8-11 for the
+ * first unit: partial stored, split partials summed, finishing stores done,
+ * unit done), then its attention launch, [256 CTAs][16] (start, Q landed,
+ * first K/V block landed, first scores ready, output accumulated, partial
+ * written, chunk rendezvous passed, merge done, first block's max found, first
+ * block's P written, first scores issued, last P seen by the issuer).  Entries
+ * of CTAs that did not run stay as they were. */
 SPEC_API int spec_set_trace(spec_handle* h, uint64_t* device_buf, size_t bytes, int layer);
 /* Number of kernels the most recent step enqueued. */
 SPEC_API int spec_step_launches(spec_handle* h);

@@ -98,13 +98,6 @@ __device__ __forceinline__ void reg_fence32(uint32_t* r) {
 }
 
 
-// 2^x on the special-function unit (PTX ex2.approx: relative error about
-// 2^-22, 2^-inf = +0); the probabilities are rounded to fp16 right after.
-__device__ __forceinline__ float fast_exp2(float x) {
-  float y;
-  asm("ex2.approx.ftz.f32 %0, %1;" : "=f"(y) : "f"(x));
-  return y;
-}
 
 // Bits j = 0..31 of the 128-bit ancestor set (a1:a0) starting at bit s, with
 // zeros for bit positions outside [0, 128); s in [-31, 127].

@@ -185,6 +185,26 @@ __device__ __forceinline__ bool spin_until_geq(const int* p, int target, uint32_
   }
 }
 
+__device__ __forceinline__ int ld_acquire_gpu(const int* p) {
+  int v;
+  asm volatile("ld.acquire.gpu.global.b32 %0, [%1];" : "=r"(v) : "l"(p) : "memory");
+  return v;
+}
+__device__ __forceinline__ int ld_relaxed_gpu(const int* p) {
+  int v;
+  asm volatile("ld.relaxed.gpu.global.b32 %0, [%1];" : "=r"(v) : "l"(p) : "memory");
+  return v;
+}
+__device__ __forceinline__ void fence_acq_rel_gpu() { asm volatile("fence.acq_rel.gpu;" ::: "memory"); }
+__device__ __forceinline__ void st_release_gpu(int* p, int v) {
+  asm volatile("st.release.gpu.global.b32 [%0], %1;" ::"l"(p), "r"(v) : "memory");
+}
+// order this thread's earlier (generic-proxy) global accesses before its later
+// async-proxy (TMA) accesses
+__device__ __forceinline__ void fence_proxy_async_global() {
+  asm volatile("fence.proxy.async.global;" ::: "memory");
+}
+
 // ---------------------------------------------------------------------------
 // TMA (tiled, 2-d, no multicast)
 // ---------------------------------------------------------------------------
@@ -204,16 +224,6 @@ __device__ __forceinline__ void tma_load_2d(void* smem_dst, const void* tmap, ui
       : "memory");
 }
 
-// Bring the box at (x, y) into L2 only (no shared memory, no completion).
-__device__ __forceinline__ void tma_prefetch_l2_2d(const void* tmap, int x, int y) {
-  asm volatile("cp.async.bulk.prefetch.tensor.2d.L2.global.tile [%0, {%1, %2}];" ::"l"(reinterpret_cast<uint64_t>(tmap)),
-               "r"(x), "r"(y)
-               : "memory");
-}
-// Bring `bytes` (multiple of 16, 16-byte aligned) at `p` into L2.
-__device__ __forceinline__ void bulk_prefetch_l2(const void* p, uint32_t bytes) {
-  asm volatile("cp.async.bulk.prefetch.L2.global [%0], %1;" ::"l"(reinterpret_cast<uint64_t>(p)), "r"(bytes) : "memory");
-}
 
 __device__ __forceinline__ uint64_t policy_evict_first() {
   uint64_t p;
@@ -342,6 +352,14 @@ __device__ __forceinline__ void split_store(__nv_bfloat16* base, int t, int ld, 
   const __nv_bfloat16 lo = __float2bfloat16_rn(v - __bfloat162float(hi));
   base[(size_t)split_row(t, 0) * ld + col] = hi;
   base[(size_t)split_row(t, 1) * ld + col] = lo;
+}
+
+// 2^x on the special-function unit (PTX ex2.approx: relative error about
+// 2^-22, 2^-inf = +0)
+__device__ __forceinline__ float fast_exp2(float x) {
+  float y;
+  asm("ex2.approx.ftz.f32 %0, %1;" : "=f"(y) : "f"(x));
+  return y;
 }
 
 // four consecutive columns (col % 4 == 0) of one token, as split bf16

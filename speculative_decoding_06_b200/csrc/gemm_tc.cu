@@ -55,10 +55,10 @@ struct SmemLayout {
   static constexpr uint32_t a_off = 0;
   static constexpr uint32_t b_off = a_off + STAGES * kABytes;
   static constexpr uint32_t epi_off = b_off + STAGES * kBBytes;
-  // per-token norm scale r[BN], then the largest of: SWIGLU up values [64][17]
-  // (padded row: conflict-free), ARGMAX per-warp results [4][BN], RESID per-warp
-  // sums of squares [4][BN]
-  static constexpr uint32_t epi_extra = cmax(64 * 17 * 4, cmax(4 * BN * (uint32_t)sizeof(Top2), 4 * BN * 4));
+  // per-token norm scale r[BN], then the largest of: SWIGLU gate and up values
+  // [128][17] (padded rows: conflict-free), ARGMAX per-warp results [4][BN], RESID
+  // per-warp sums of squares [4][BN]
+  static constexpr uint32_t epi_extra = cmax(128 * 17 * 4, cmax(4 * BN * (uint32_t)sizeof(Top2), 4 * BN * 4));
   static constexpr uint32_t epi_bytes = BN * 4 + epi_extra;
   static constexpr uint32_t bar_off = (epi_off + epi_bytes + 7) & ~7u;
   static constexpr uint32_t n_bars = 2 * STAGES + 4;
@@ -97,7 +97,7 @@ __device__ __forceinline__ UnitIter units_of(const GemmTcArgs& a) {
 // accumulator of the phase complete, 5 split-K rendezvous passed, 6 epilogue
 // done with the phase's units, 7 phase counted at the grid barrier.
 __device__ __forceinline__ void stamp(uint64_t* trace, int p, int k) {
-  if (trace) trace[((size_t)blockIdx.x * kMaxGemmPhases + p) * 8 + k] = global_ns();
+  if (trace) trace[((size_t)blockIdx.x * kMaxGemmPhases + p) * kGemmTraceMarks + k] = global_ns();
 }
 
 __device__ __forceinline__ bool phase_done(const int* bar, int need) {
@@ -108,8 +108,9 @@ __device__ __forceinline__ bool phase_done(const int* bar, int need) {
 
 }  // namespace
 
+// BN = 64: two CTAs per SM (registers capped accordingly); BN = 128: one
 template <int BN, int STAGES>
-__global__ void __launch_bounds__(kThreads, 1)
+__global__ void __launch_bounds__(kThreads, BN == 64 ? 2 : 1)
     gemm_tc_kernel(const __grid_constant__ GemmMaps maps, const __grid_constant__ GemmPhases P) {
   using L = SmemLayout<BN, STAGES>;
   extern __shared__ uint8_t smem_raw[];
@@ -176,33 +177,6 @@ __global__ void __launch_bounds__(kThreads, 1)
       }
     }
   };
-  auto prefetch_a = [&](int p, int kx, int to) {
-    const GemmTcArgs& a = P.ph[p];
-    const CUtensorMap* m = &maps.m[4 * p];
-    if (P.epi[p] == GEMM_EPI_SWIGLU) {
-      tma_prefetch_l2_2d(m + 0, kx, to * 64);
-      tma_prefetch_l2_2d(m + 1, kx, to * 64);
-    } else {
-      const int row = to * kTileO;
-      if (row < a.seg_rows[0]) tma_prefetch_l2_2d(m + 0, kx, row);
-      else if (row < a.seg_rows[0] + a.seg_rows[1]) tma_prefetch_l2_2d(m + 1, kx, row - a.seg_rows[0]);
-      else tma_prefetch_l2_2d(m + 2, kx, row - a.seg_rows[0] - a.seg_rows[1]);
-    }
-  };
-  // L2 prefetch of this CTA's first k-blocks of phase p (issued when the
-  // producer is done with phase p - 1, so that HBM keeps streaming while the
-  // epilogue finishes phase p - 1 and the grid meets at its barrier)
-  auto prefetch_phase_l2 = [&](int p) {
-    const GemmTcArgs& a = P.ph[p];
-    const UnitIter it = units_of(a);
-    const int ut = it.first();
-    if (ut >= it.tiles) return;
-    const int KB = a.K / kTileK;
-    const int kb0 = it.split() * a.kb_per_split;
-    const int kb1 = min(min(kb0 + a.kb_per_split, KB), kb0 + P.pf_next);
-    const int to = ut / a.tiles_t;
-    for (int kb = kb0; kb < kb1; ++kb) prefetch_a(p, kb * kTileK, to);
-  };
   int pre = 0;  // stages whose weight tile was issued before the wait
   if (producer) {
     pol_w = policy_evict_first();
@@ -232,14 +206,55 @@ __global__ void __launch_bounds__(kThreads, 1)
       int stage = 0;
       uint32_t phase = 0;
       int issued = 0;
-      // activation tiles held back until the previous phase has completed
+      // Activation tiles are held back until their producers have finished:
+      // phase 0's come from the previous kernel (waited for above), a later
+      // phase's from the whole previous phase (its grid-barrier count).
       int pend_stage[STAGES], pend_kx[STAGES], pend_row[STAGES];
-      int npend = 0, pend_p = 0;
-      auto flush = [&]() {
-        for (int i = 0; i < npend; ++i)
-          tma_load_2d(smem + L::b_off + pend_stage[i] * L::kBBytes, &maps.m[4 * pend_p + 3], &full[pend_stage[i]],
-                      pend_kx[i], pend_row[i], pol_x);
-        npend = 0;
+      int npend = 0;
+      bool first_b = true;
+      bool phase_ready = false;
+      auto b_ready = [&](int p, int, int) -> bool {
+        if (p == 0) return true;
+        if (!phase_ready) {
+          phase_ready = phase_done(P.phase_bar + p - 1, grid);
+          if (phase_ready) fence_proxy_async_global();  // acquired data is read next by TMA
+        }
+        return phase_ready;
+      };
+      auto issue_b = [&](int p, int st, int kx, int row) {
+        if (first_b) {
+          first_b = false;
+          stamp(P.trace, p, 1);
+        }
+        tma_load_2d(smem + L::b_off + st * L::kBBytes, &maps.m[4 * p + 3], &full[st], kx, row, pol_x);
+      };
+      // issue pending activation loads in k order; `block` waits (bounded) for the first
+      auto drain = [&](int p, int tt, bool block) -> bool {
+        int done = 0;
+        while (done < npend) {
+          if (!b_ready(p, pend_kx[done], tt)) {
+            if (!block) break;
+            const uint64_t t0 = global_ns();
+            while (!b_ready(p, pend_kx[done], tt)) {
+              if (*abort_flag) return false;
+              if (global_ns() - t0 > SPEC_WAIT_NS) {
+                set_error(err, SPEC_DEVERR_TIMEOUT);
+                *abort_flag = 1;
+                return false;
+              }
+              __nanosleep(256);
+            }
+          }
+          issue_b(p, pend_stage[done], pend_kx[done], pend_row[done]);
+          ++done;
+        }
+        for (int i = done; i < npend; ++i) {
+          pend_stage[i - done] = pend_stage[i];
+          pend_kx[i - done] = pend_kx[i];
+          pend_row[i - done] = pend_row[i];
+        }
+        npend -= done;
+        return true;
       };
       for (int p = 0; p < nph && !*abort_flag; ++p) {
         const GemmTcArgs& a = P.ph[p];
@@ -247,9 +262,9 @@ __global__ void __launch_bounds__(kThreads, 1)
         const int KB = a.K / kTileK;
         const int kb0 = it.split() * a.kb_per_split;
         const int kb1 = min(kb0 + a.kb_per_split, KB);
-        bool ready = p == 0;  // phase 0's operand is ready: the kernel waited for its predecessor
         stamp(P.trace, p, 0);
-        if (ready) stamp(P.trace, p, 1);
+        first_b = true;
+        phase_ready = false;
         for (int ut = it.first(); ut < it.tiles && !*abort_flag; ut = it.next(ut)) {
           const int tt = ut % a.tiles_t;
           const int to = ut / a.tiles_t;
@@ -260,47 +275,21 @@ __global__ void __launch_bounds__(kThreads, 1)
               mbar_arrive_expect_tx(&full[stage], kABytes + L::kBBytes);
               load_a(p, smem + L::a_off + stage * kABytes, &full[stage], kx, to);
             }
-            if (P.pf_ahead > 0 && kb + P.pf_ahead < kb1) prefetch_a(p, (kb + P.pf_ahead) * kTileK, to);
-            if (!ready) {
-              ready = phase_done(P.phase_bar + p - 1, grid);
-              if (ready) stamp(P.trace, p, 1);
-            }
-            if (ready) {
-              flush();
-              tma_load_2d(smem + L::b_off + stage * L::kBBytes, &maps.m[4 * p + 3], &full[stage], kx, tt * 2 * BN,
-                          pol_x);
-            } else {
-              pend_stage[npend] = stage;
-              pend_kx[npend] = kx;
-              pend_row[npend] = tt * 2 * BN;
-              pend_p = p;
-              ++npend;
-              if (npend == STAGES) {  // the ring is full of weight tiles: wait for the phase
-                if (!spin_until_geq(P.phase_bar + p - 1, grid, err)) {
-                  *abort_flag = 1;
-                  break;
-                }
-                ready = true;
-                stamp(P.trace, p, 1);
-                flush();
-              }
-            }
+            pend_stage[npend] = stage;
+            pend_kx[npend] = kx;
+            pend_row[npend] = tt * 2 * BN;
+            ++npend;
+            // the ring is full of weight tiles: wait for the oldest activation tile
+            if (!drain(p, tt, npend == STAGES)) break;
             if (++stage == STAGES) {
               stage = 0;
               phase ^= 1;
             }
           }
-        }
-        if (npend > 0 && !*abort_flag) {
-          if (spin_until_geq(P.phase_bar + p - 1, grid, err)) {
-            stamp(P.trace, p, 1);
-            flush();
-          } else {
-            *abort_flag = 1;
-          }
+          // a unit's activation tiles are all issued before the next unit's
+          if (!*abort_flag && npend > 0 && !drain(p, tt, true)) break;
         }
         stamp(P.trace, p, 2);
-        if (p + 1 < nph && !*abort_flag) prefetch_phase_l2(p + 1);
       }
       if (*abort_flag) {
         // let copies already issued land before this CTA's shared memory is released
@@ -435,15 +424,16 @@ __global__ void __launch_bounds__(kThreads, 1)
               if (t < args.M) out[(size_t)t * args.n_out] = v[i] + vl[i];
             }
           }
+          if (first_unit && ep_tid == 0) stamp(P.trace, p, 8);
           tc_fence_before();
           mbar_arrive(&tempty[acc]);  // the accumulator is free for the next unit
           // 2) the S split CTAs of the tile meet at its arrival counter, then all of
           //    them share the finishing work, each taking 1/S of the tile's tokens
           int* ctr = args.counters + 2 * ut;
-          __threadfence();
           named_sync(2, 128);
           if (S > 1) {
             if (ep_tid == 0) {
+              __threadfence();  // the barrier orders every thread's partial stores before it
               atomicAdd(ctr, 1);
               *ep_ok = spin_until_geq(ctr, S, err) ? 1 : 0;
             }
@@ -460,123 +450,158 @@ __global__ void __launch_bounds__(kThreads, 1)
           const float* part = args.part;
           const size_t sst = args.split_stride;
           if (EPI == GEMM_EPI_QKV) {
-            // tile `to` is one head of q|k|v (head_dim 128): rotate-half pairs (c, c+64)
+            // tile `to` is one head of q|k|v (head_dim 128), rotate-half pairs (c, c+64).
+            // lane: 4-column group c4 (columns 4c4.. and 64+4c4..) and one of two
+            // tokens; warp: 2 more token lanes -> 8 tokens per pass
             const int hh = to;
-            const int c = ep_tid & 63;
-            const int par = ep_tid >> 6;
-            for (int tb = t0s; tb < t1s; tb += 8) {
-              float v1[4], v2[4];
+            const int c4 = lane & 15;
+            const int tl8 = ep_warp * 2 + (lane >> 4);
+            const bool is_q = hh < args.Hq;
+            const bool rot = hh < args.Hq + args.Hkv;
+            const int G = args.Hq / args.Hkv;
+            for (int t = t0s + tl8; t < t1s; t += 8) {
+              // independent loads: this token's metadata, rotation and all split partials
+              const int slot = is_q ? 0 : args.row_slot[t];
+              const int sid = is_q ? 0 : args.row_sid[t];
+              float4 cs0 = make_float4(1.f, 0.f, 1.f, 0.f), cs1 = cs0;
+              if (rot) {
+                const float4* csp = reinterpret_cast<const float4*>(args.rope_cs + (size_t)t * 64 + 4 * c4);
+                cs0 = csp[0];
+                cs1 = csp[1];
+              }
+              float4 a = make_float4(0.f, 0.f, 0.f, 0.f), bq = a;
+              constexpr int kQ = 8;
+              for (int q0 = 0; q0 < S; q0 += kQ) {
+                float4 pa[kQ], pb[kQ];
 #pragma unroll
-              for (int i = 0; i < 4; ++i) v1[i] = v2[i] = 0.f;
-              for (int q = 0; q < S; ++q) {  // L2 loads: the peers wrote these
+                for (int qq = 0; qq < kQ; ++qq) {
+                  const bool ok = q0 + qq < S;
+                  const float4* pr = reinterpret_cast<const float4*>(part + (size_t)(q0 + qq) * sst +
+                                                                     (size_t)t * args.n_out + hh * 128 + 4 * c4);
+                  pa[qq] = ok ? __ldcg(pr) : make_float4(0.f, 0.f, 0.f, 0.f);
+                  pb[qq] = ok ? __ldcg(pr + 16) : make_float4(0.f, 0.f, 0.f, 0.f);
+                }
 #pragma unroll
-                for (int i = 0; i < 4; ++i) {
-                  const int t = tb + 2 * i + par;
-                  if (t < t1s) {
-                    const float* pr = part + q * sst + (size_t)t * args.n_out + hh * 128 + c;
-                    v1[i] += __ldcg(pr);
-                    v2[i] += __ldcg(pr + 64);
-                  }
+                for (int qq = 0; qq < kQ; ++qq) {  // fixed order: deterministic
+                  a.x += pa[qq].x; a.y += pa[qq].y; a.z += pa[qq].z; a.w += pa[qq].w;
+                  bq.x += pb[qq].x; bq.y += pb[qq].y; bq.z += pb[qq].z; bq.w += pb[qq].w;
                 }
               }
+              if (first_unit && ep_tid == 0 && t == t0s) stamp(P.trace, p, 9);
+              const float r = r_s[t - t_base];
+              float x1[4] = {a.x * r, a.y * r, a.z * r, a.w * r};
+              float x2[4] = {bq.x * r, bq.y * r, bq.z * r, bq.w * r};
+              const float cs[8] = {cs0.x, cs0.y, cs0.z, cs0.w, cs1.x, cs1.y, cs1.z, cs1.w};
+              if (rot) {
 #pragma unroll
-              for (int i = 0; i < 4; ++i) {
-                const int t = tb + 2 * i + par;
-                if (t >= t1s) continue;
-                const float r = r_s[t - t_base];
-                float a1 = v1[i] * r, a2 = v2[i] * r;
-                if (hh < args.Hq + args.Hkv) {
-                  const float2 cs = args.rope_cs[(size_t)t * 64 + c];
-                  const float o1 = a1 * cs.x - a2 * cs.y;
-                  const float o2 = a2 * cs.x + a1 * cs.y;
-                  a1 = o1;
-                  a2 = o2;
+                for (int i = 0; i < 4; ++i) {  // (cos, sin) pairs
+                  const float co = cs[2 * i], si = cs[2 * i + 1];
+                  const float o1 = x1[i] * co - x2[i] * si;
+                  const float o2 = x2[i] * co + x1[i] * si;
+                  x1[i] = o1;
+                  x2[i] = o2;
                 }
-                if (hh < args.Hq) {
-                  const int G = args.Hq / args.Hkv;
-                  __half* qo = args.q_out + ((size_t)(hh / G) * args.q_rows + (size_t)t * G + hh % G) * 128;
-                  qo[c] = __float2half_rn(a1);
-                  qo[c + 64] = __float2half_rn(a2);
-                } else {
-                  const int b = args.row_seq[t];
-                  const int slot = args.P_step[b] + args.row_local[t];
-                  if (slot < args.max_seq) {
-                    const bool is_k = hh < args.Hq + args.Hkv;
-                    const int kvh = is_k ? hh - args.Hq : hh - args.Hq - args.Hkv;
-                    __half* dst = (is_k ? args.k_cache : args.v_cache) + args.seq_ids[b] * args.kv_seq_stride +
-                                  kvh * args.kv_head_stride + (size_t)slot * 128;
-                    dst[c] = __float2half_rn(a1);
-                    dst[c + 64] = __float2half_rn(a2);
-                  } else if (c == 0) {
-                    set_error(err, SPEC_DEVERR_BOUNDS);
-                  }
-                }
+              }
+              __half* dst = nullptr;
+              if (is_q) {
+                dst = args.q_out + ((size_t)(hh / G) * args.q_rows + (size_t)t * G + hh % G) * 128;
+              } else if (slot >= 0) {
+                const int kvh = rot ? hh - args.Hq : hh - args.Hq - args.Hkv;
+                dst = (rot ? args.k_cache : args.v_cache) + (size_t)sid * args.kv_seq_stride +
+                      (size_t)kvh * args.kv_head_stride + (size_t)slot * 128;
+              } else if (c4 == 0) {
+                set_error(err, SPEC_DEVERR_BOUNDS);
+              }
+              if (dst) {
+                const __half2 h0 = __floats2half2_rn(x1[0], x1[1]), h1 = __floats2half2_rn(x1[2], x1[3]);
+                const __half2 h2 = __floats2half2_rn(x2[0], x2[1]), h3 = __floats2half2_rn(x2[2], x2[3]);
+                uint2 lo, hi;
+                lo.x = *reinterpret_cast<const uint32_t*>(&h0);
+                lo.y = *reinterpret_cast<const uint32_t*>(&h1);
+                hi.x = *reinterpret_cast<const uint32_t*>(&h2);
+                hi.y = *reinterpret_cast<const uint32_t*>(&h3);
+                *reinterpret_cast<uint2*>(dst + 4 * c4) = lo;
+                *reinterpret_cast<uint2*>(dst + 64 + 4 * c4) = hi;
               }
             }
           } else {
             // residual update of this tile's 128 columns for this CTA's tokens, the
-            // next operand x*w (split bf16) and per-token sums of squares of x
-            float* ssw = reinterpret_cast<float*>(epx);  // [4][BN]
-            const int col = to * kTileO + ep_tid;
-            const float w = __bfloat162float(args.norm_w_next[col]);
-            for (int tb = t0s; tb < t1s; tb += 8) {
-              float xv[8];
+            // next operand x*w (split bf16) and per-token sums of squares of x over
+            // the tile.  Warp = token (4 per pass), lane = 4 columns.
+            const int col = to * kTileO + 4 * lane;
+            const float2 w01 = __bfloat1622float2(*reinterpret_cast<const __nv_bfloat162*>(args.norm_w_next + col));
+            const float2 w23 = __bfloat1622float2(*reinterpret_cast<const __nv_bfloat162*>(args.norm_w_next + col + 2));
+            constexpr int kT = 2;  // tokens per warp and pass
+            constexpr int kQ = 8;  // split partials per batch of loads
+            for (int tb = t0s + ep_warp; tb < t1s; tb += 4 * kT) {
+              float4 xv[kT];
 #pragma unroll
-              for (int i = 0; i < 8; ++i)
-                xv[i] = (tb + i < t1s) ? args.x[(size_t)(tb + i) * args.n_out + col] : 0.f;
-              for (int q = 0; q < S; ++q) {
-#pragma unroll
-                for (int i = 0; i < 8; ++i)
-                  if (tb + i < t1s) xv[i] += __ldcg(part + q * sst + (size_t)(tb + i) * args.n_out + col);
+              for (int k = 0; k < kT; ++k) {
+                const int t = tb + 4 * k;
+                xv[k] = t < t1s ? *reinterpret_cast<const float4*>(args.x + (size_t)t * args.n_out + col)
+                                : make_float4(0.f, 0.f, 0.f, 0.f);
               }
+              for (int q0 = 0; q0 < S; q0 += kQ) {
+                float4 pv[kQ][kT];
 #pragma unroll
-              for (int i = 0; i < 8; ++i) {
-                const int t = tb + i;
-                if (t >= t1s) continue;
-                args.x[(size_t)t * args.n_out + col] = xv[i];
-                split_store(args.xn_out, t, args.n_out, col, xv[i] * w);
-                const float sq = warp_sum(xv[i] * xv[i]);
-                if (lane == 0) ssw[ep_warp * BN + (t - t_base)] = sq;
+                for (int qq = 0; qq < kQ; ++qq)
+#pragma unroll
+                  for (int k = 0; k < kT; ++k) {
+                    const int t = tb + 4 * k;
+                    pv[qq][k] = (t < t1s && q0 + qq < S)
+                                    ? __ldcg(reinterpret_cast<const float4*>(part + (size_t)(q0 + qq) * sst +
+                                                                             (size_t)t * args.n_out + col))
+                                    : make_float4(0.f, 0.f, 0.f, 0.f);
+                  }
+#pragma unroll
+                for (int qq = 0; qq < kQ; ++qq)  // fixed order: deterministic
+#pragma unroll
+                  for (int k = 0; k < kT; ++k) {
+                    xv[k].x += pv[qq][k].x;
+                    xv[k].y += pv[qq][k].y;
+                    xv[k].z += pv[qq][k].z;
+                    xv[k].w += pv[qq][k].w;
+                  }
+              }
+              if (first_unit && ep_tid == 0 && tb == t0s) stamp(P.trace, p, 9);
+#pragma unroll
+              for (int k = 0; k < kT; ++k) {
+                const int t = tb + 4 * k;
+                const float4 v = xv[k];
+                const float sq = warp_sum(v.x * v.x + v.y * v.y + v.z * v.z + v.w * v.w);
+                if (t < t1s) {
+                  *reinterpret_cast<float4*>(args.x + (size_t)t * args.n_out + col) = v;
+                  split_store4(args.xn_out, t, args.n_out, col, make_float4(v.x * w01.x, v.y * w01.y, v.z * w23.x, v.w * w23.y));
+                  if (lane == 0) args.ss_out[(size_t)to * args.ss_ld + t] = sq;
+                }
               }
             }
-            named_sync(2, 128);
-            for (int t = t0s + ep_tid; t < t1s; t += 128) {
-              const int c = t - t_base;
-              args.ss_out[(size_t)to * args.ss_ld + t] = ssw[c] + ssw[BN + c] + ssw[2 * BN + c] + ssw[3 * BN + c];
-            }
-          }
-          // the last CTA of the tile to leave resets its counters for the next launch
-          if (S > 1) {
-            named_sync(2, 128);
-            if (ep_tid == 0 && atomicAdd(ctr + 1, 1) == S - 1) {
-              ctr[0] = 0;
-              ctr[1] = 0;
-            }
+            if (first_unit && ep_tid == 0) stamp(P.trace, p, 10);
           }
         } else if (EPI == GEMM_EPI_SWIGLU) {
-          float* stage_up = reinterpret_cast<float*>(epx);  // [64][17]
-          const int f = to * 64 + (row_in_tile & 63);
+          // gate rows 0-63 and up rows 64-127 of the tile meet in shared memory;
+          // every thread then finishes 8 of the 16 tokens of one ffn column
+          float* stage = reinterpret_cast<float*>(epx);  // [128][17]
+          const int fl = ep_tid & 63;
+          const int half = ep_tid >> 6;
+          const int f = to * 64 + fl;
 #pragma unroll 1
           for (int c0 = 0; c0 < BN; c0 += 16) {
             float v[16], vl[16];
             const uint32_t col = (c0 / 64) * 128 + (c0 % 64);
             tmem_ld16x2(taddr + col, taddr + col + 64, v, vl);
 #pragma unroll
-            for (int i = 0; i < 16; ++i) v[i] = (v[i] + vl[i]) * r_s[c0 + i];
-            if (quarter >= 2) {
-#pragma unroll
-              for (int i = 0; i < 16; ++i) stage_up[(row_in_tile - 64) * 17 + i] = v[i];
-            }
+            for (int i = 0; i < 16; ++i) stage[row_in_tile * 17 + i] = (v[i] + vl[i]) * r_s[c0 + i];
             named_sync(1, 128);
-            if (quarter < 2) {
 #pragma unroll
-              for (int i = 0; i < 16; ++i) {
-                const int t = t_base + c0 + i;
-                const float g = v[i];
-                const float up = stage_up[row_in_tile * 17 + i];
-                const float h = g / (1.0f + expf(-g)) * up;
-                if (t < args.M) split_store(args.out_bf16, t, args.ld_out, f, h);
-              }
+            for (int i = 0; i < 8; ++i) {
+              const int ii = half * 8 + i;
+              const int t = t_base + c0 + ii;
+              const float g = stage[fl * 17 + ii];
+              const float up = stage[(64 + fl) * 17 + ii];
+              // silu(g) = g / (1 + 2^(-g log2 e)): special-function exp2 and divide
+              const float h = __fdividef(g, 1.0f + fast_exp2(-1.4426950408889634f * g)) * up;
+              if (t < args.M) split_store(args.out_bf16, t, args.ld_out, f, h);
             }
             named_sync(1, 128);
           }
@@ -616,16 +641,29 @@ __global__ void __launch_bounds__(kThreads, 1)
             if (t < args.M) args.top_part[(size_t)to * args.top_ld + t] = r;
           }
         }
+        // unit done; the last CTA of a split tile to leave resets the tile's
+        // counters for the next launch
         named_sync(2, 128);  // r_s and the staging areas are reused by the next unit
+        if (ep_tid == 0 && S > 1) {
+          int* ctr = args.counters + 2 * ut;
+          if (atomicAdd(ctr + 1, 1) == S - 1) {
+            ctr[0] = 0;
+            ctr[1] = 0;
+          }
+        }
+        if (first_unit && ep_tid == 0) stamp(P.trace, p, 11);
         first_unit = false;
       }
       if (!alive) break;
       if (ep_tid == 0) stamp(P.trace, p, 6);
       // this CTA is done with phase p: make its writes visible, then count it
       if (p + 1 < nph) {
-        __threadfence();
+        fence_proxy_async_global();  // later phases read this phase's outputs with TMA
         named_sync(2, 128);
-        if (ep_tid == 0) atomicAdd(P.phase_bar + p, 1);
+        if (ep_tid == 0) {
+          __threadfence();
+          atomicAdd(P.phase_bar + p, 1);
+        }
       }
       if (ep_tid == 0) stamp(P.trace, p, 7);
     }
@@ -655,8 +693,6 @@ static cudaError_t launch_impl(const GemmMultiLaunch& L_, cudaStream_t stream, b
   ph.phase_bar = L_.phase_bar;
   ph.err = L_.err;
   ph.trace = L_.trace;
-  ph.pf_next = L_.pf_next;
-  ph.pf_ahead = L_.pf_ahead;
   for (int p = 0; p < L_.n_phases; ++p) {
     const GemmPhase& q = L_.ph[p];
     maps.m[4 * p + 0] = *q.mA0;

@@ -51,6 +51,8 @@ struct GemmTcArgs {
   // QKV
   const int32_t* row_seq;
   const int32_t* row_local;
+  const int32_t* row_slot;  // cache slot P_b + local (-1 beyond max_seq)
+  const int32_t* row_sid;   // sequence id
   const int32_t* P_step;
   const int32_t* seq_ids;
   const float2* rope_cs;  // [tokens][64]
@@ -69,6 +71,7 @@ struct GemmTcArgs {
 };
 
 constexpr int kMaxGemmPhases = 4;
+constexpr int kGemmTraceMarks = 16;  // %globaltimer marks per CTA and phase (optional timeline)
 
 // kernel parameters: the tensor maps of every phase (a0, a1, a2, b) and the phases
 struct GemmMaps {
@@ -79,9 +82,7 @@ struct GemmPhases {
   int epi[kMaxGemmPhases];
   int* phase_bar;  // [n_phases - 1] CTAs done with each phase, zero at launch
   uint32_t* err;
-  uint64_t* trace; // optional [grid][kMaxGemmPhases][8] %globaltimer stamps (see gemm_tc.cu)
-  int pf_next;     // k-blocks of the next phase each CTA brings into L2 once its loads for a phase are issued
-  int pf_ahead;    // within a phase, L2 prefetch distance in k-blocks ahead of the shared-memory ring (0: off)
+  uint64_t* trace; // optional [grid][kMaxGemmPhases][kGemmTraceMarks] %globaltimer stamps
   GemmTcArgs ph[kMaxGemmPhases];
 };
 
@@ -97,7 +98,6 @@ struct GemmMultiLaunch {
   int* phase_bar;
   uint32_t* err;
   uint64_t* trace;
-  int pf_next, pf_ahead;
   GemmPhase ph[kMaxGemmPhases];
 };
 
@@ -123,6 +123,8 @@ struct StepView {
   int B, M;
   int32_t* row_seq;         // [M] batch entry
   int32_t* row_local;       // [M] local node index
+  int32_t* row_slot;        // [M] cache slot P_b + local index, -1 when it would pass max_seq
+  int32_t* row_sid;         // [M] sequence id
   int32_t* row_pos;         // [M] position P_b + depth
   uint64_t* row_anc;        // [M][2] ancestor bits over local indices (self included)
   float2* rope_cs;          // [M][head_dim/2] (cos, sin)
@@ -165,16 +167,6 @@ cudaError_t launch_swiglu_f32(int M, int F, const float* gu, float* h, cudaStrea
 cudaError_t launch_gemm_simt_f32(const float* A, int lda, const float* W, int K, float* C, int ldc, int M, int N,
                                  cudaStream_t s);
 
-// A strided list of byte ranges to bring into L2: `rows` segments of `seg`
-// bytes at base + i * stride (base, stride and seg multiples of 16).
-struct L2Range {
-  const uint8_t* base;
-  size_t stride;
-  uint32_t seg;
-  int rows;
-};
-constexpr int kMaxL2Ranges = 3;
-
 // attention
 struct AttnArgs {
   StepView sv;
@@ -189,10 +181,6 @@ struct AttnArgs {
   int max_rows;             // max over batch of n_b * (Hq/Hkv)
   int q_rows;               // bf16 path: q is [Hkv][q_rows][hd], row node * G + g
   int* counters;            // bf16 path: [groups][2] chunk arrivals / departures, zero between launches
-  // weights the next kernel streams, brought into L2 while attention (which
-  // moves little data) runs; issued before the wait on the previous kernel
-  L2Range pf[kMaxL2Ranges];
-  int n_pf;
   uint64_t* trace;          // optional [256 CTAs][16] %globaltimer marks (attention_tc.cu)
 };
 // fp32 models: one warp per (node, head)

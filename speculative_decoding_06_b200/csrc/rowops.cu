@@ -90,6 +90,8 @@ __global__ void __launch_bounds__(256) embed_meta_kernel(StepView sv, const T* _
     }
     sv.row_seq[r] = b;
     sv.row_local[r] = i;
+    sv.row_slot[r] = P + i < sv.max_seq ? P + i : -1;
+    sv.row_sid[r] = seq;
     sv.row_pos[r] = P + depth;
     sv.row_anc[2 * r] = a0;
     sv.row_anc[2 * r + 1] = a1;

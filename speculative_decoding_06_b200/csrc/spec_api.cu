@@ -46,7 +46,7 @@ struct WsLayout {
   // parameter block (one host->device copy per step)
   size_t p_tokens, p_parents, p_node_off, p_seq_ids, p_err, p_end;
   // per-row metadata
-  size_t row_seq, row_local, row_pos, row_anc, rope_cs, P_step;
+  size_t row_seq, row_local, row_slot, row_sid, row_pos, row_anc, rope_cs, P_step;
   // persistent state
   size_t seq_len, pending, hist, err_sticky;
   // activations
@@ -81,6 +81,8 @@ WsLayout make_layout(const spec_config& c) {
   L.p_end = off;
   L.row_seq = take(4 * (size_t)L.Mmax);
   L.row_local = take(4 * (size_t)L.Mmax);
+  L.row_slot = take(4 * (size_t)L.Mmax);
+  L.row_sid = take(4 * (size_t)L.Mmax);
   L.row_pos = take(4 * (size_t)L.Mmax);
   L.row_anc = take(16 * (size_t)L.Mmax);
   L.rope_cs = take(8 * (size_t)L.Mmax * (c.head_dim / 2));
@@ -116,6 +118,7 @@ WsLayout make_layout(const spec_config& c) {
   L.phase_bar_n = 4 * (c.n_layers + 2);
   L.phase_bar = take(4 * (size_t)L.phase_bar_n);
   L.attn_ctr_n = 2 * kAttnPartCtas;
+
   L.attn_ctr = take(4 * (size_t)L.attn_ctr_n);
   L.argmax = take(4 * (size_t)L.Mpad);
   L.top1 = take(4 * (size_t)L.Mpad);
@@ -241,12 +244,6 @@ struct spec_handle {
   int max_chunks = kMaxAttnChunks;  // attention key-chunk cap
   int resident_cap = 0;   // 0: as many CTAs per SM as fit
   // L2 prefetch of weights ahead of the GEMM that streams them
-  // (all off by default: measured on B200 they only took bandwidth from the
-  // streams they were meant to feed)
-  int pf_next = 0;        // k-blocks of the next phase, per CTA, at the end of a phase's loads
-  int pf_ahead = 0;       // in-phase distance in k-blocks (0: off)
-  int pf_attn_o = 0;      // attention brings the O projection into L2
-  int pf_attn_gu = 0;     // ... and the first columns of every gate/up row
   uint64_t* trace = nullptr;  // optional GEMM timeline of one layer's launch
   size_t trace_bytes = 0;
   int trace_layer = 0;
@@ -382,6 +379,8 @@ StepView make_view(spec_handle* h, int B, int M) {
   v.M = M;
   v.row_seq = h->W<int32_t>(L.row_seq);
   v.row_local = h->W<int32_t>(L.row_local);
+  v.row_slot = h->W<int32_t>(L.row_slot);
+  v.row_sid = h->W<int32_t>(L.row_sid);
   v.row_pos = h->W<int32_t>(L.row_pos);
   v.row_anc = h->W<uint64_t>(L.row_anc);
   v.rope_cs = h->W<float2>(L.rope_cs);
@@ -392,6 +391,7 @@ StepView make_view(spec_handle* h, int B, int M) {
   v.max_seq = h->cfg.max_seq;
   v.err = h->W<uint32_t>(L.p_err);
   v.err_sticky = h->W<uint32_t>(L.err_sticky);
+
   return v;
 }
 
@@ -500,6 +500,8 @@ cudaError_t enqueue_step(spec_handle* h, const StepPlan& sp, int mode, bool dbg)
     g.args.counters = gctr + slot * kCountersPerPhase;
     g.args.row_seq = sv.row_seq;
     g.args.row_local = sv.row_local;
+    g.args.row_slot = sv.row_slot;
+    g.args.row_sid = sv.row_sid;
     g.args.P_step = sv.P_step;
     g.args.seq_ids = sv.seq_ids;
     g.args.rope_cs = sv.rope_cs;
@@ -584,23 +586,9 @@ cudaError_t enqueue_step(spec_handle* h, const StepPlan& sp, int mode, bool dbg)
     if (dt == 1) {
       // attention of layer l (its QKV ran in the previous launch), then one
       // launch: O, gate/up, down, and the next layer's QKV or the LM head
-      aa.n_pf = 0;
-      if (h->pf_attn_o) {
-        const size_t row = 2 * (size_t)qd;
-        aa.pf[aa.n_pf++] = L2Range{static_cast<const uint8_t*>(lw.wo), row, (uint32_t)row, d};
-      }
-      if (h->pf_attn_gu > 0) {
-        const uint32_t seg = 2 * (uint32_t)std::min(h->pf_attn_gu, d) & ~15u;
-        if (seg > 0) {
-          aa.pf[aa.n_pf++] = L2Range{static_cast<const uint8_t*>(lw.w_gate), 2 * (size_t)d, seg, c.ffn};
-          aa.pf[aa.n_pf++] = L2Range{static_cast<const uint8_t*>(lw.w_up), 2 * (size_t)d, seg, c.ffn};
-        }
-      }
-      aa.trace = (h->trace && l == h->trace_layer) ? h->trace + (size_t)2 * h->sm_count * kMaxGemmPhases * 8 : nullptr;
+      aa.trace = (h->trace && l == h->trace_layer) ? h->trace + (size_t)2 * h->sm_count * kMaxGemmPhases * kGemmTraceMarks : nullptr;
       LK(SPEC_PROF_ATTENTION, 1, launch_attention_tc(aa, h->attn_maps, st, pdl));
       GemmMultiLaunch m{};
-      m.pf_next = h->pf_next;
-      m.pf_ahead = h->pf_ahead;
       m.bn = sp.qkv.bn;
       m.grid = sp.grid_all;
       m.err = sv.err;
@@ -892,10 +880,6 @@ int spec_init(const spec_config* cfg, const spec_weights* w, void* kv_cache, siz
     if (const char* q = strstr(t, "chunks=")) if (sscanf(q + 7, "%d", &v) == 1 && v >= 1 && v <= kMaxAttnChunks) h->max_chunks = v;
     if (const char* q = strstr(t, "pdl=")) if (sscanf(q + 4, "%d", &v) == 1) h->use_pdl = v != 0;
     if (const char* q = strstr(t, "per_sm=")) if (sscanf(q + 7, "%d", &v) == 1 && v >= 0) h->resident_cap = v;
-    if (const char* q = strstr(t, "pf_next=")) if (sscanf(q + 8, "%d", &v) == 1 && v >= 0) h->pf_next = v;
-    if (const char* q = strstr(t, "pf_ahead=")) if (sscanf(q + 9, "%d", &v) == 1 && v >= 0) h->pf_ahead = v;
-    if (const char* q = strstr(t, "pf_o=")) if (sscanf(q + 5, "%d", &v) == 1) h->pf_attn_o = v != 0;
-    if (const char* q = strstr(t, "pf_gu=")) if (sscanf(q + 6, "%d", &v) == 1 && v >= 0) h->pf_attn_gu = v;
   }
   if (cudaGetDevice(&h->device) != cudaSuccess) return bail(SPEC_ERR_CUDA, "cudaGetDevice");
   cudaDeviceProp prop;
@@ -912,6 +896,7 @@ int spec_init(const spec_config* cfg, const spec_weights* w, void* kv_cache, siz
       cudaMemsetAsync(h->ws + lay.err_sticky, 0, 16, h->stream) != cudaSuccess ||
       cudaMemsetAsync(h->ws + lay.gemm_ctr, 0, 4 * (size_t)kGemmCounters, h->stream) != cudaSuccess ||
       cudaMemsetAsync(h->ws + lay.attn_ctr, 0, 4 * (size_t)lay.attn_ctr_n, h->stream) != cudaSuccess ||
+
       cudaMemcpyAsync(h->ws + lay.inv_freq, inv.data(), 8 * inv.size(), cudaMemcpyHostToDevice, h->stream) !=
           cudaSuccess ||
       cudaStreamSynchronize(h->stream) != cudaSuccess)
@@ -971,8 +956,13 @@ int spec_init(const spec_config* cfg, const spec_weights* w, void* kv_cache, siz
           return bail(SPEC_ERR_CUDA, "occupancy");
         // shared memory per SM (1 KB per CTA is reserved by the system)
         const int by_smem = prop.sharedMemPerMultiprocessor / (smem + (int)prop.reservedSharedMemPerBlock);
+        // registers: allocated per warp in units of 256 (8 per thread)
+        cudaFuncAttributes fa;
+        if (cudaFuncGetAttributes(&fa, fn) != cudaSuccess) return bail(SPEC_ERR_CUDA, "function attributes");
+        const int regs_cta = ((fa.numRegs + 7) / 8) * 8 * 192;
+        const int by_regs = regs_cta > 0 ? prop.regsPerMultiprocessor / regs_cta : 1;
         h->occ_api[i][e] = nb;
-        nb = std::max(nb, by_smem);
+        nb = std::min(std::max(nb, by_smem), by_regs);
         // tensor memory: two accumulators of 2*BN columns (hi and lo) per CTA, 512 columns per SM
         h->resident[i][e] = std::max(1, std::min(nb, 512 / (4 * bns[i])));
       }
@@ -1152,9 +1142,9 @@ int spec_profile_read(spec_handle* h, double* ms, int64_t* launches) {
 
 int spec_step_launches(spec_handle* h) { return h ? h->launches : 0; }
 
-// GEMM marks [2 * SMs][phases][8], then attention marks [kAttnPartCtas][16]
+// GEMM marks [2 * SMs][phases][16], then attention marks [kAttnPartCtas][16]
 static size_t trace_words(const spec_handle* h) {
-  return (size_t)2 * h->sm_count * kMaxGemmPhases * 8 + (size_t)kAttnPartCtas * 16;
+  return (size_t)2 * h->sm_count * kMaxGemmPhases * kGemmTraceMarks + (size_t)kAttnPartCtas * 16;
 }
 
 int spec_set_trace(spec_handle* h, uint64_t* device_buf, size_t bytes, int layer) {
