@@ -78,7 +78,8 @@ typedef struct spec_config {
   int32_t max_batch;    /* sequences held in the cache */
   int32_t max_seq;      /* cache slots per sequence */
   int32_t max_nodes;    /* tree nodes per sequence per step, root included; <= 128 */
-  int32_t draft_head;   /* 1: also size buffers for the EAGLE-3 draft head (bf16 only) */
+  int32_t draft_head;   /* 1: the handle also runs the EAGLE-3 draft head (bf16 only): its weights in
+                           spec_weights, its layer's K/V one more cache layer (counted by spec_kv_bytes) */
 } spec_config;
 
 /* Per-layer weights, device pointers, row-major [out][in] in the model dtype:
@@ -162,6 +163,40 @@ SPEC_API int spec_verify_tree_batch(spec_handle* h, int B, const int32_t* seq_id
 SPEC_API int spec_score_trees(spec_handle* h, int B, const int32_t* seq_ids, const int32_t* tokens, const int32_t* parents,
                      const int32_t* node_offsets, int32_t* argmax, float* top1, float* top2, int flags);
 
+/* ---- EAGLE-3 draft head (cfg.draft_head = 1, bf16 models) ----------------
+ * The draft stage of "EAGLE-3: Scaling up Inference Acceleration of Large
+ * Language Models via Training-Time Test" (summary page, draft-stage section):
+ * the target's low, mid and high features l, m, h of a position (d each) are
+ * concatenated and reduced by one FC layer to the fused feature g = [l|m|h].
+ * W_fuse^T; g is concatenated with the embedding e of the token one step ahead
+ * and reduced by a second FC layer, x = [g|e].W_in^T; one pre-norm decoder layer
+ * of the target's shape (its own K/V cache) turns x into a, and the target's LM
+ * head, after the draft head's final RMSNorm, scores a.  Readings where the page
+ * is silent: concatenation orders [l|m|h] and [g|e]; e from the target's
+ * embedding table; tree nodes attend to the draft prefix and their ancestors
+ * at positions prefix + depth, as in verification.
+ *
+ * feats are DEVICE pointers to bf16 [rows][3][d] (l, m, h per row); tokens,
+ * parents and node_offsets are host arrays as in spec_verify_tree_batch. */
+#define SPEC_DRAFT_TOPK 10     /* draft candidates per node (the pages' tree top-k) */
+
+/* Build the draft layer's K/V for positions 0 .. n-1 of `seq` from n rows of
+ * features and tokens (n <= max_seq), replacing what was there.  Synchronises. */
+SPEC_API int spec_draft_prefill(spec_handle* h, int seq, const void* feats, const int32_t* tokens, int n);
+/* One draft-head step over a batch of trees on the draft prefixes: per node,
+ * the SPEC_DRAFT_TOPK best vocabulary entries of the draft distribution, by
+ * logit descending then index ascending, in top_idx / top_val [nodes][TOPK].
+ * The draft prefixes are not extended (the trees' K/V are scratch).  Flags:
+ * SPEC_DEVICE_OUTPUTS (outputs are device pointers, no synchronisation),
+ * SPEC_DEBUG_LOGITS (also the fp32 draft logits to the debug buffer),
+ * SPEC_NO_GRAPH.  Errors as in spec_verify_tree_batch; SPEC_ERR_STATE when a
+ * sequence has no draft prefix. */
+SPEC_API int spec_draft_step(spec_handle* h, int B, const int32_t* seq_ids, const void* feats, const int32_t* tokens,
+                             const int32_t* parents, const int32_t* node_offsets, int32_t* top_idx, float* top_val,
+                             int flags);
+/* Draft prefix length of `seq` (host output). */
+SPEC_API int spec_draft_len(spec_handle* h, int seq, int32_t* len);
+
 /* Device buffer (fp32, >= max_batch * max_nodes * vocab entries) for SPEC_DEBUG_LOGITS. */
 SPEC_API int spec_set_debug_logits(spec_handle* h, float* device_buf, size_t bytes);
 
@@ -193,7 +228,9 @@ SPEC_API int spec_validate_tree(const int32_t* tokens, const int32_t* parents, i
 #define SPEC_PROF_WALK 10        /* acceptance walk + state update */
 #define SPEC_PROF_COMPACT 11     /* K/V compaction */
 #define SPEC_PROF_GEMM_LAYER 12  /* one launch: O, gate/up, down, then the next QKV or the LM head */
-#define SPEC_PROF_CLASSES 13
+#define SPEC_PROF_DRAFT_FC 13    /* draft head: feature split, fusion FC, input FC */
+#define SPEC_PROF_TOPK 14        /* draft head: top-k over the logits */
+#define SPEC_PROF_CLASSES 15
 
 /* enable != 0: subsequent steps launch kernel by kernel (no graph) with a CUDA
  * event pair around every launch on the handle's stream. */

@@ -607,6 +607,24 @@ __global__ void __launch_bounds__(kThreads, BN == 64 ? 2 : 1)
           }
           tc_fence_before();
           mbar_arrive(&tempty[acc]);
+        } else if (EPI == GEMM_EPI_STORE) {
+          // the accumulator as split bf16 (no split-K): thread = output row, warp
+          // stores of one token are 32 consecutive columns
+          const int o = to * kTileO + row_in_tile;
+          const bool row_ok = o < args.n_out;
+#pragma unroll 1
+          for (int c0 = 0; c0 < BN; c0 += 16) {
+            float v[16], vl[16];
+            const uint32_t col = (c0 / 64) * 128 + (c0 % 64);
+            tmem_ld16x2(taddr + col, taddr + col + 64, v, vl);
+#pragma unroll
+            for (int i = 0; i < 16; ++i) {
+              const int t = t_base + c0 + i;
+              if (row_ok && t < args.M) split_store(args.out_bf16, t, args.ld_out, o, (v[i] + vl[i]) * r_s[c0 + i]);
+            }
+          }
+          tc_fence_before();
+          mbar_arrive(&tempty[acc]);
         } else {  // GEMM_EPI_ARGMAX
           Top2* wres = reinterpret_cast<Top2*>(epx);  // [4][BN]
           const int o = to * kTileO + row_in_tile;

@@ -21,7 +21,7 @@ struct Top2;
 //          x*w (split bf16) and the tile's per-token sums of squares of x
 //   SWIGLU gate rows 0-63, up rows 64-127 of a tile; silu(g)*u as split bf16
 //   ARGMAX per-token (best, index, runner-up) of the tile's vocabulary rows
-enum { GEMM_EPI_QKV = 0, GEMM_EPI_SWIGLU = 1, GEMM_EPI_ARGMAX = 2, GEMM_EPI_RESID = 3 };
+enum { GEMM_EPI_QKV = 0, GEMM_EPI_SWIGLU = 1, GEMM_EPI_ARGMAX = 2, GEMM_EPI_RESID = 3, GEMM_EPI_STORE = 4 };
 
 struct StepView;
 
@@ -41,7 +41,7 @@ struct GemmTcArgs {
   float* part;
   size_t split_stride;
   int* counters;      // [tiles_o * tiles_t], zero between launches
-  // SWIGLU
+  // SWIGLU, STORE (the accumulator itself, no split-K)
   __nv_bfloat16* out_bf16;  // split bf16 [2 x tokens][ld_out]
   int ld_out;
   // ARGMAX
@@ -147,13 +147,24 @@ struct KvView {
   __host__ __device__ size_t layer_stride() const { return 2 * kv_stride(); }
 };
 
-enum { STEP_VERIFY = 0, STEP_PREFILL = 1, STEP_SCORE = 2 };
+enum { STEP_VERIFY = 0, STEP_PREFILL = 1, STEP_SCORE = 2, STEP_DRAFT = 3, STEP_DRAFT_KV = 4 };
 
 // metadata + embedding + first RMSNorm.  bf16 models: xn = split(x*w) (the
 // norm scale is applied by the next GEMM) and ss[0][r] = sum x^2, ss[i>0][r] = 0.
+// With e_out (draft head, bf16): the embedding row goes to e_out as split bf16
+// at columns [e_col, e_col + d) of rows of e_ld elements, and x, xn, ss are
+// left alone.
 cudaError_t launch_embed_meta(int dtype, const StepView& sv, const void* embed, const void* norm_w, int d, float eps,
                               float* x, void* xn, float* ss, int n_ss, int ss_ld, const double* inv_freq, int half,
-                              int mode, cudaStream_t s, bool pdl);
+                              int mode, cudaStream_t s, bool pdl, __nv_bfloat16* e_out = nullptr, int e_ld = 0,
+                              int e_col = 0);
+// bf16 rows [rows][cols] -> split bf16 operand [2 x rows][cols] (lo parts zero)
+cudaError_t launch_split_rows(const __nv_bfloat16* src, int rows, int cols, __nv_bfloat16* dst, cudaStream_t s,
+                              bool pdl);
+// per row: the k largest of V fp32 values, ordered by (value desc, index asc)
+constexpr int kTopKMax = 16;
+cudaError_t launch_topk_rows(int M, int V, const float* logits, size_t ld, int k, int32_t* idx, float* val,
+                             cudaStream_t s, bool pdl);
 // x += sum of split partials; xn = RMSNorm(x) * w
 cudaError_t launch_residual_norm(int dtype, int M, int d, int S, const float* partial, size_t split_stride, float* x,
                                  void* xn, const void* w, float eps, cudaStream_t s, bool pdl);

@@ -59,7 +59,8 @@ __global__ void __launch_bounds__(256) embed_meta_kernel(StepView sv, const T* _
                                                          const T* __restrict__ norm_w, int d, float eps,
                                                          float* __restrict__ x, void* __restrict__ xn,
                                                          float* __restrict__ ss_out, int n_ss, int ss_ld,
-                                                         const double* __restrict__ inv_freq, int half, int mode) {
+                                                         const double* __restrict__ inv_freq, int half, int mode,
+                                                         __nv_bfloat16* __restrict__ e_out, int e_ld, int e_col) {
   __shared__ int s_pos;
   __shared__ float red[8];
   pdl_wait();
@@ -110,6 +111,10 @@ __global__ void __launch_bounds__(256) embed_meta_kernel(StepView sv, const T* _
   }
   const int tok = sv.tokens[r];
   const T* e = embed + (size_t)tok * d;
+  if (SPLIT && e_out) {  // draft head: the embedding is half of the next GEMM's operand
+    for (int k = threadIdx.x; k < d; k += blockDim.x) split_store(e_out, r, e_ld, e_col + k, to_f32(e[k]));
+    return;
+  }
   float* xr = x + (size_t)r * d;
   float ss = 0.f;
   for (int k = threadIdx.x; k < d; k += blockDim.x) {
@@ -131,14 +136,15 @@ __global__ void __launch_bounds__(256) embed_meta_kernel(StepView sv, const T* _
 
 cudaError_t launch_embed_meta(int dtype, const StepView& sv, const void* embed, const void* norm_w, int d, float eps,
                               float* x, void* xn, float* ss, int n_ss, int ss_ld, const double* inv_freq, int half,
-                              int mode, cudaStream_t s, bool pdl) {
+                              int mode, cudaStream_t s, bool pdl, __nv_bfloat16* e_out, int e_ld, int e_col) {
   cudaLaunchAttribute attr[1];
   cudaLaunchConfig_t cfg = make_cfg(dim3(sv.M), dim3(256), 0, s, pdl, attr);
   if (dtype == 0)
     return cudaLaunchKernelEx(&cfg, embed_meta_kernel<float, false>, sv, (const float*)embed, (const float*)norm_w, d,
-                              eps, x, xn, ss, n_ss, ss_ld, inv_freq, half, mode);
+                              eps, x, xn, ss, n_ss, ss_ld, inv_freq, half, mode, (__nv_bfloat16*)nullptr, 0, 0);
   return cudaLaunchKernelEx(&cfg, embed_meta_kernel<__nv_bfloat16, true>, sv, (const __nv_bfloat16*)embed,
-                            (const __nv_bfloat16*)norm_w, d, eps, x, xn, ss, n_ss, ss_ld, inv_freq, half, mode);
+                            (const __nv_bfloat16*)norm_w, d, eps, x, xn, ss, n_ss, ss_ld, inv_freq, half, mode, e_out,
+                            e_ld, e_col);
 }
 
 // ---------------------------------------------------------------------------
@@ -405,6 +411,137 @@ cudaError_t launch_rows_top2_f32(int M, int V, const float* logits, int32_t* arg
                                  cudaStream_t s) {
   rows_top2_f32_kernel<<<(M + 7) / 8, 256, 0, s>>>(M, V, logits, argmax, top1, top2);
   return cudaGetLastError();
+}
+
+// ---------------------------------------------------------------------------
+// bf16 rows -> split-bf16 GEMM operand
+// ---------------------------------------------------------------------------
+// Rows that are already bf16 (the draft head's input features) have a zero lo
+// part.  16 bytes per thread.
+__global__ void __launch_bounds__(256) split_rows_kernel(const uint4* __restrict__ src, int rows, int cols8,
+                                                        uint4* __restrict__ dst) {
+  pdl_wait();
+  pdl_launch_dependents();
+  const size_t n = (size_t)rows * cols8;
+  for (size_t i = blockIdx.x * (size_t)blockDim.x + threadIdx.x; i < n; i += (size_t)gridDim.x * blockDim.x) {
+    const int t = (int)(i / cols8);
+    const int c = (int)(i - (size_t)t * cols8);
+    dst[(size_t)split_row(t, 0) * cols8 + c] = src[i];
+    dst[(size_t)split_row(t, 1) * cols8 + c] = make_uint4(0u, 0u, 0u, 0u);
+  }
+}
+
+cudaError_t launch_split_rows(const __nv_bfloat16* src, int rows, int cols, __nv_bfloat16* dst, cudaStream_t s,
+                              bool pdl) {
+  if (cols % 8) return cudaErrorInvalidValue;
+  const int cols8 = cols / 8;
+  const size_t n = (size_t)rows * cols8;
+  const int grid = (int)std::min<size_t>((n + 255) / 256, 148 * 8);
+  cudaLaunchAttribute attr[1];
+  cudaLaunchConfig_t cfg = make_cfg(dim3(grid), dim3(256), 0, s, pdl, attr);
+  return cudaLaunchKernelEx(&cfg, split_rows_kernel, reinterpret_cast<const uint4*>(src), rows, cols8,
+                            reinterpret_cast<uint4*>(dst));
+}
+
+// ---------------------------------------------------------------------------
+// top-k per row (the draft head's candidate list)
+// ---------------------------------------------------------------------------
+// One CTA per row.  Each thread keeps a sorted list of its best k values over
+// a strided slice of the row; the warps then merge by k rounds of a warp-wide
+// best-of, and warp 0 merges the eight warp lists the same way.  Order: value
+// descending, index ascending.
+namespace {
+__device__ __forceinline__ bool topk_better(float a, int ai, float b, int bi) {
+  return a > b || (a == b && ai < bi);
+}
+// k rounds: each round the best head among the lanes' lists is taken
+__device__ __forceinline__ void warp_merge_topk(const float* lv, const int* li, int k, float* out_v, int* out_i) {
+  const int lane = threadIdx.x & 31;
+  int head = 0;
+  for (int r = 0; r < k; ++r) {
+    float v = head < k ? lv[head] : -INFINITY;
+    int i = head < k ? li[head] : 0x7fffffff;
+    int src = lane;
+#pragma unroll
+    for (int o = 16; o > 0; o >>= 1) {
+      const float v2 = __shfl_xor_sync(0xffffffffu, v, o);
+      const int i2 = __shfl_xor_sync(0xffffffffu, i, o);
+      const int s2 = __shfl_xor_sync(0xffffffffu, src, o);
+      if (topk_better(v2, i2, v, i)) {
+        v = v2;
+        i = i2;
+        src = s2;
+      }
+    }
+    if (lane == src) ++head;
+    if (lane == 0) {
+      out_v[r] = v;
+      out_i[r] = i;
+    }
+  }
+}
+}  // namespace
+
+__global__ void __launch_bounds__(256) topk_rows_kernel(int V, const float* __restrict__ logits, size_t ld, int k,
+                                                       int32_t* __restrict__ out_i, float* __restrict__ out_v) {
+  __shared__ float wv[8][kTopKMax];
+  __shared__ int wi[8][kTopKMax];
+  pdl_wait();
+  pdl_launch_dependents();
+  const int r = blockIdx.x;
+  const float* row = logits + (size_t)r * ld;
+  float lv[kTopKMax];
+  int li[kTopKMax];
+#pragma unroll
+  for (int j = 0; j < kTopKMax; ++j) {
+    lv[j] = -INFINITY;
+    li[j] = 0x7fffffff;
+  }
+  for (int c = threadIdx.x; c < V; c += blockDim.x) {
+    const float x = __ldcs(row + c);
+    if (!topk_better(x, c, lv[k - 1], li[k - 1])) continue;
+    // insert, keeping lv[0..k) sorted
+    float cv = x;
+    int ci = c;
+#pragma unroll
+    for (int j = 0; j < kTopKMax; ++j) {
+      if (j < k && topk_better(cv, ci, lv[j], li[j])) {
+        const float tv = lv[j];
+        const int ti = li[j];
+        lv[j] = cv;
+        li[j] = ci;
+        cv = tv;
+        ci = ti;
+      }
+    }
+  }
+  const int warp = threadIdx.x >> 5;
+  warp_merge_topk(lv, li, k, wv[warp], wi[warp]);
+  __syncthreads();
+  if (warp == 0) {
+    const int lane = threadIdx.x & 31;
+    float mv[kTopKMax];
+    int mi[kTopKMax];
+#pragma unroll
+    for (int j = 0; j < kTopKMax; ++j) {
+      mv[j] = (lane < 8 && j < k) ? wv[lane][j] : -INFINITY;
+      mi[j] = (lane < 8 && j < k) ? wi[lane][j] : 0x7fffffff;
+    }
+    warp_merge_topk(mv, mi, k, wv[0], wi[0]);  // lane 0 writes after reading its own list
+    __syncwarp();
+    if (lane < k) {
+      out_v[(size_t)r * k + lane] = wv[0][lane];
+      out_i[(size_t)r * k + lane] = wi[0][lane];
+    }
+  }
+}
+
+cudaError_t launch_topk_rows(int M, int V, const float* logits, size_t ld, int k, int32_t* idx, float* val,
+                             cudaStream_t s, bool pdl) {
+  if (k < 1 || k > kTopKMax || k > V) return cudaErrorInvalidValue;
+  cudaLaunchAttribute attr[1];
+  cudaLaunchConfig_t cfg = make_cfg(dim3(M), dim3(256), 0, s, pdl, attr);
+  return cudaLaunchKernelEx(&cfg, topk_rows_kernel, V, logits, ld, k, idx, val);
 }
 
 }  // namespace spec

@@ -35,6 +35,7 @@ constexpr int kMaxNodesLimit = 128;  // ancestor bitmask is two 64-bit words
 constexpr int kMaxSplits = 16;
 constexpr int kGemmCounters = 8192;  // per-tile arrival counters of the split-K GEMMs
 constexpr int kMaxAttnChunks = 64;    // key chunks of one (sequence, kv head, row tile)
+constexpr int kDraftTopK = SPEC_DRAFT_TOPK;  // candidates per draft node
 constexpr int kCountersPerPhase = 2048; // two ints per split-K tile
 
 size_t align_up(size_t x, size_t a) { return (x + a - 1) / a * a; }
@@ -44,7 +45,7 @@ struct WsLayout {
   size_t total = 0;
   int Mmax = 0, Mpad = 0, splits_cap = 1, chunks_cap = 1;
   // parameter block (one host->device copy per step)
-  size_t p_tokens, p_parents, p_node_off, p_seq_ids, p_err, p_end;
+  size_t p_tokens, p_parents, p_node_off, p_seq_ids, p_dlen, p_err, p_end;
   // per-row metadata
   size_t row_seq, row_local, row_slot, row_sid, row_pos, row_anc, rope_cs, P_step;
   // persistent state
@@ -52,6 +53,8 @@ struct WsLayout {
   // activations
   size_t x, xn, q, attn, hmlp, partial, part_o, part_lse, top_part, argmax, top1, top2, inv_freq;
   size_t ss, gemm_ctr, attn_ctr, phase_bar;
+  // draft head: split features [2 Mpad][3d], [g|e] operand [2 Mpad][2d], logits, top-k
+  size_t fsplit = 0, ge = 0, dlogits = 0, dtop_i = 0, dtop_v = 0;
   int n_ss = 1, attn_ctr_n = 0, phase_bar_n = 0;
   size_t partial_bytes;
   // outputs (one device->host copy per step)
@@ -77,6 +80,7 @@ WsLayout make_layout(const spec_config& c) {
   L.p_parents = take(4 * (size_t)L.Mmax);
   L.p_node_off = take(4 * (size_t)(c.max_batch + 1));
   L.p_seq_ids = take(4 * (size_t)c.max_batch);
+  L.p_dlen = take(4 * (size_t)c.max_batch);
   L.p_err = take(16);
   L.p_end = off;
   L.row_seq = take(4 * (size_t)L.Mmax);
@@ -123,6 +127,13 @@ WsLayout make_layout(const spec_config& c) {
   L.argmax = take(4 * (size_t)L.Mpad);
   L.top1 = take(4 * (size_t)L.Mpad);
   L.top2 = take(4 * (size_t)L.Mpad);
+  if (c.draft_head) {
+    L.fsplit = take(2 * 2 * (size_t)L.Mpad * 3 * c.hidden);
+    L.ge = take(2 * 2 * (size_t)L.Mpad * 2 * c.hidden);
+    L.dlogits = take(4 * (size_t)L.Mpad * c.vocab);
+    L.dtop_i = take(4 * (size_t)L.Mpad * kDraftTopK);
+    L.dtop_v = take(4 * (size_t)L.Mpad * kDraftTopK);
+  }
   const size_t o0 = off;
   L.o_acc_len = take(4 * (size_t)c.max_batch);
   L.o_acc_nodes = take(4 * (size_t)c.max_batch * c.max_nodes);
@@ -134,9 +145,12 @@ WsLayout make_layout(const spec_config& c) {
   return L;
 }
 
+// decoder layers with a K/V cache: the target's, plus the draft head's one layer
+int cache_layers(const spec_config& c) { return c.n_layers + (c.draft_head ? 1 : 0); }
+
 size_t kv_bytes_of(const spec_config& c) {
   const size_t es = c.dtype == SPEC_DTYPE_BF16 ? 2 : 4;
-  return (size_t)c.n_layers * 2 * c.max_batch * c.n_kv_heads * (size_t)c.max_seq * c.head_dim * es;
+  return (size_t)cache_layers(c) * 2 * c.max_batch * c.n_kv_heads * (size_t)c.max_seq * c.head_dim * es;
 }
 
 std::string check_config(const spec_config* c) {
@@ -226,6 +240,13 @@ struct spec_handle {
   CUtensorMap map_lm;
   CUtensorMap map_xn[2], map_attn[2], map_h[2];  // B operands for BN = 64, 128
   AttnTcMaps attn_maps;                           // q and the K/V cache (fp16)
+  // draft head (cfg.draft_head): its decoder layer is layers[n_layers], maps[n_layers]
+  const void* draft_fc_fuse = nullptr;
+  const void* draft_fc_in = nullptr;
+  const void* draft_final_norm = nullptr;
+  CUtensorMap map_fc_fuse, map_fc_in, map_fsplit[2], map_ge[2];
+  std::vector<int32_t> dlen;        // draft-head prefix length per sequence
+  std::vector<uint8_t> dready;
   int resident[2][4] = {{0, 0, 0, 0}, {0, 0, 0, 0}};   // co-resident CTAs per SM [bn][epi]
   int occ_api[2][4] = {{0, 0, 0, 0}, {0, 0, 0, 0}};    // what the occupancy query reported
   // host mirror of per-sequence state
@@ -308,7 +329,7 @@ GemmPlan plan_gemm(const spec_handle* h, int rows_per_tile, int n_out, int K, in
   GemmPlan p;
   p.bn = M <= 64 ? 64 : 128;
   const int bi = p.bn == 64 ? 0 : 1;
-  int per_sm = std::max(1, h->resident[bi][epi]);
+  int per_sm = std::max(1, h->resident[bi][0]);  // one kernel function for every epilogue
   if (h->resident_cap > 0) per_sm = std::min(per_sm, h->resident_cap);
   const int resident = per_sm * h->sm_count;
   p.tiles_o = ceil_div(n_out, rows_per_tile);
@@ -420,12 +441,131 @@ GemmTcLaunch gemm_launch(const GemmPlan& p, int epi, int n_out, int K, int M, co
   return L;
 }
 
+#define CUDA_RET(expr)                   \
+  do {                                   \
+    cudaError_t e_ = (expr);             \
+    if (e_ != cudaSuccess) return e_;    \
+  } while (0)
+
 // Enqueue the whole step (everything after the parameter upload).
 #define LK(cls, nk, expr)                                                             \
   do {                                                                                \
     cudaError_t e_ = launch_k(h, cls, nk, [&]() { return (expr); });                  \
     if (e_ != cudaSuccess) return e_;                                                 \
   } while (0)
+
+// The GEMM phases of the bf16 path, for decoder layer l (the draft head's
+// layer is index n_layers).  Split-K counters: one region per phase slot.
+struct PhaseBuilder {
+  spec_handle* h;
+  const StepPlan& sp;
+  const StepView& sv;
+  int bi, d, qd, kvd, nqkv, M;
+  PhaseBuilder(spec_handle* h_, const StepPlan& sp_, const StepView& sv_) : h(h_), sp(sp_), sv(sv_) {
+    const spec_config& c = h->cfg;
+    bi = sp.qkv.bn == 64 ? 0 : 1;
+    d = c.hidden;
+    qd = c.n_q_heads * c.head_dim;
+    kvd = c.n_kv_heads * c.head_dim;
+    nqkv = qd + 2 * kvd;
+    M = sp.M;
+  }
+  static GemmPhase as_phase(const GemmTcLaunch& g) {
+    GemmPhase q{};
+    q.epi = g.epi;
+    q.mA0 = g.mA0;
+    q.mA1 = g.mA1;
+    q.mA2 = g.mA2;
+    q.mB = g.mB;
+    q.args = g.args;
+    return q;
+  }
+  int* ctr(int slot) const { return h->W<int>(h->lay.gemm_ctr) + slot * kCountersPerPhase; }
+  GemmPhase qkv(int l, int slot) const {
+    const spec_config& c = h->cfg;
+    const WsLayout& L = h->lay;
+    const LayerMaps& mp = h->maps[l];
+    __half* kc = reinterpret_cast<__half*>(h->kv.base) + (size_t)l * h->kv.layer_stride();
+    GemmTcLaunch g = gemm_launch(sp.qkv, GEMM_EPI_QKV, nqkv, d, M, &mp.wq, &mp.wk, &mp.wv, &h->map_xn[bi], qd, kvd,
+                                 kvd, sv.err);
+    g.args.ss_in = h->W<float>(L.ss);
+    g.args.n_ss = L.n_ss;
+    g.args.ss_ld = L.Mpad;
+    g.args.norm_d = d;
+    g.args.eps = c.rms_eps;
+    g.args.part = h->W<float>(L.partial);
+    g.args.split_stride = (size_t)L.Mpad * nqkv;
+    g.args.counters = ctr(slot);
+    g.args.row_seq = sv.row_seq;
+    g.args.row_local = sv.row_local;
+    g.args.row_slot = sv.row_slot;
+    g.args.row_sid = sv.row_sid;
+    g.args.P_step = sv.P_step;
+    g.args.seq_ids = sv.seq_ids;
+    g.args.rope_cs = sv.rope_cs;
+    g.args.q_out = h->W<__half>(L.q);
+    g.args.q_rows = L.Mpad * (c.n_q_heads / c.n_kv_heads);
+    g.args.k_cache = kc;
+    g.args.v_cache = kc + h->kv.kv_stride();
+    g.args.kv_seq_stride = h->kv.seq_stride();
+    g.args.kv_head_stride = h->kv.head_stride();
+    g.args.Hq = c.n_q_heads;
+    g.args.Hkv = c.n_kv_heads;
+    g.args.max_seq = c.max_seq;
+    return as_phase(g);
+  }
+  // x += A.W^T; xn = split(x * norm_next); ss = per-tile sums of squares
+  GemmPhase resid(const GemmPlan& pl, int K, const CUtensorMap* mw, const CUtensorMap* mb, const void* norm_next,
+                  int slot) const {
+    const WsLayout& L = h->lay;
+    GemmTcLaunch g = gemm_launch(pl, GEMM_EPI_RESID, d, K, M, mw, nullptr, nullptr, mb, d, 0, 0, sv.err);
+    g.args.part = h->W<float>(L.partial);
+    g.args.split_stride = (size_t)L.Mpad * d;
+    g.args.counters = ctr(slot);
+    g.args.x = h->W<float>(L.x);
+    g.args.norm_w_next = reinterpret_cast<const __nv_bfloat16*>(norm_next);
+    g.args.xn_out = h->W<__nv_bfloat16>(L.xn);
+    g.args.ss_out = h->W<float>(L.ss);
+    g.args.ss_ld = L.Mpad;
+    return as_phase(g);
+  }
+  GemmPhase o(int l, int slot) const {
+    return resid(sp.o, qd, &h->maps[l].wo, &h->map_attn[bi], h->layers[l].mlp_norm, slot);
+  }
+  GemmPhase down(int l, int slot, const void* next_norm) const {
+    return resid(sp.down, h->cfg.ffn, &h->maps[l].wd, &h->map_h[bi], next_norm, slot);
+  }
+  GemmPhase gu(int l) const {
+    const spec_config& c = h->cfg;
+    const WsLayout& L = h->lay;
+    GemmTcLaunch g = gemm_launch(sp.gu, GEMM_EPI_SWIGLU, c.ffn, d, M, &h->maps[l].wg, &h->maps[l].wu, nullptr,
+                                 &h->map_xn[bi], 0, 0, 0, sv.err);
+    g.args.ss_in = h->W<float>(L.ss);
+    g.args.n_ss = L.n_ss;
+    g.args.ss_ld = L.Mpad;
+    g.args.norm_d = d;
+    g.args.eps = c.rms_eps;
+    g.args.out_bf16 = h->W<__nv_bfloat16>(L.hmlp);
+    g.args.ld_out = c.ffn;
+    return as_phase(g);
+  }
+  // final norm (folded) + LM head with per-tile top-2; logits also stored when given
+  GemmPhase lm(float* logits) const {
+    const spec_config& c = h->cfg;
+    const WsLayout& L = h->lay;
+    GemmTcLaunch g = gemm_launch(sp.lm, GEMM_EPI_ARGMAX, c.vocab, d, M, &h->map_lm, nullptr, nullptr, &h->map_xn[bi],
+                                 c.vocab, 0, 0, sv.err);
+    g.args.top_part = h->W<Top2>(L.top_part);
+    g.args.top_ld = L.Mpad;
+    g.args.dbg_logits = logits;
+    g.args.ss_in = h->W<float>(L.ss);
+    g.args.n_ss = L.n_ss;
+    g.args.ss_ld = L.Mpad;
+    g.args.norm_d = d;
+    g.args.eps = c.rms_eps;
+    return as_phase(g);
+  }
+};
 
 cudaError_t enqueue_step(spec_handle* h, const StepPlan& sp, int mode, bool dbg) {
   const spec_config& c = h->cfg;
@@ -473,101 +613,7 @@ cudaError_t enqueue_step(spec_handle* h, const StepPlan& sp, int mode, bool dbg)
   aa.counters = h->W<int>(L.attn_ctr);
   aa.q_rows = L.Mpad * (c.n_q_heads / c.n_kv_heads);
 
-  // ---- GEMM phases of the bf16 path (split-K counters: one region per phase slot)
-  const int bi = sp.qkv.bn == 64 ? 0 : 1;
-  auto as_phase = [](const GemmTcLaunch& g) {
-    GemmPhase q{};
-    q.epi = g.epi;
-    q.mA0 = g.mA0;
-    q.mA1 = g.mA1;
-    q.mA2 = g.mA2;
-    q.mB = g.mB;
-    q.args = g.args;
-    return q;
-  };
-  auto phase_qkv = [&](int l, int slot) {
-    const LayerMaps& mp = h->maps[l];
-    __half* kc = reinterpret_cast<__half*>(h->kv.base) + (size_t)l * h->kv.layer_stride();
-    GemmTcLaunch g = gemm_launch(sp.qkv, GEMM_EPI_QKV, nqkv, d, M, &mp.wq, &mp.wk, &mp.wv, &h->map_xn[bi], qd, kvd,
-                                 kvd, sv.err);
-    g.args.ss_in = ss;
-    g.args.n_ss = L.n_ss;
-    g.args.ss_ld = L.Mpad;
-    g.args.norm_d = d;
-    g.args.eps = c.rms_eps;
-    g.args.part = part;
-    g.args.split_stride = (size_t)L.Mpad * nqkv;
-    g.args.counters = gctr + slot * kCountersPerPhase;
-    g.args.row_seq = sv.row_seq;
-    g.args.row_local = sv.row_local;
-    g.args.row_slot = sv.row_slot;
-    g.args.row_sid = sv.row_sid;
-    g.args.P_step = sv.P_step;
-    g.args.seq_ids = sv.seq_ids;
-    g.args.rope_cs = sv.rope_cs;
-    g.args.q_out = reinterpret_cast<__half*>(q);
-    g.args.q_rows = L.Mpad * (c.n_q_heads / c.n_kv_heads);
-    g.args.k_cache = kc;
-    g.args.v_cache = kc + h->kv.kv_stride();
-    g.args.kv_seq_stride = h->kv.seq_stride();
-    g.args.kv_head_stride = h->kv.head_stride();
-    g.args.Hq = c.n_q_heads;
-    g.args.Hkv = c.n_kv_heads;
-    g.args.max_seq = c.max_seq;
-    return as_phase(g);
-  };
-  auto phase_o = [&](int l, int slot) {
-    GemmTcLaunch g = gemm_launch(sp.o, GEMM_EPI_RESID, d, qd, M, &h->maps[l].wo, nullptr, nullptr, &h->map_attn[bi],
-                                 d, 0, 0, sv.err);
-    g.args.part = part;
-    g.args.split_stride = (size_t)L.Mpad * d;
-    g.args.counters = gctr + slot * kCountersPerPhase;
-    g.args.x = x;
-    g.args.norm_w_next = reinterpret_cast<const __nv_bfloat16*>(h->layers[l].mlp_norm);
-    g.args.xn_out = reinterpret_cast<__nv_bfloat16*>(xn);
-    g.args.ss_out = ss;
-    g.args.ss_ld = L.Mpad;
-    return as_phase(g);
-  };
-  auto phase_gu = [&](int l) {
-    GemmTcLaunch g = gemm_launch(sp.gu, GEMM_EPI_SWIGLU, c.ffn, d, M, &h->maps[l].wg, &h->maps[l].wu, nullptr,
-                                 &h->map_xn[bi], 0, 0, 0, sv.err);
-    g.args.ss_in = ss;
-    g.args.n_ss = L.n_ss;
-    g.args.ss_ld = L.Mpad;
-    g.args.norm_d = d;
-    g.args.eps = c.rms_eps;
-    g.args.out_bf16 = reinterpret_cast<__nv_bfloat16*>(hm);
-    g.args.ld_out = c.ffn;
-    return as_phase(g);
-  };
-  auto phase_down = [&](int l, int slot) {
-    const void* next_norm = (l + 1 < c.n_layers) ? h->layers[l + 1].attn_norm : h->final_norm;
-    GemmTcLaunch g = gemm_launch(sp.down, GEMM_EPI_RESID, d, c.ffn, M, &h->maps[l].wd, nullptr, nullptr,
-                                 &h->map_h[bi], d, 0, 0, sv.err);
-    g.args.part = part;
-    g.args.split_stride = (size_t)L.Mpad * d;
-    g.args.counters = gctr + slot * kCountersPerPhase;
-    g.args.x = x;
-    g.args.norm_w_next = reinterpret_cast<const __nv_bfloat16*>(next_norm);
-    g.args.xn_out = reinterpret_cast<__nv_bfloat16*>(xn);
-    g.args.ss_out = ss;
-    g.args.ss_ld = L.Mpad;
-    return as_phase(g);
-  };
-  auto phase_lm = [&]() {
-    GemmTcLaunch g = gemm_launch(sp.lm, GEMM_EPI_ARGMAX, c.vocab, d, M, &h->map_lm, nullptr, nullptr, &h->map_xn[bi],
-                                 c.vocab, 0, 0, sv.err);
-    g.args.top_part = h->W<Top2>(L.top_part);
-    g.args.top_ld = L.Mpad;
-    g.args.dbg_logits = dbg ? h->dbg_logits : nullptr;
-    g.args.ss_in = ss;
-    g.args.n_ss = L.n_ss;
-    g.args.ss_ld = L.Mpad;
-    g.args.norm_d = d;
-    g.args.eps = c.rms_eps;
-    return as_phase(g);
-  };
+  const PhaseBuilder pb(h, sp, sv);
   if (dt == 1) {
     GemmMultiLaunch m{};
     m.bn = sp.qkv.bn;
@@ -575,7 +621,7 @@ cudaError_t enqueue_step(spec_handle* h, const StepPlan& sp, int mode, bool dbg)
     m.err = sv.err;
     m.phase_bar = h->W<int>(L.phase_bar);
     m.n_phases = 1;
-    m.ph[0] = phase_qkv(0, 0);
+    m.ph[0] = pb.qkv(0, 0);
     LK(SPEC_PROF_GEMM_QKV, 1, gemm_multi_launch(m, st, pdl));
   }
 
@@ -594,10 +640,10 @@ cudaError_t enqueue_step(spec_handle* h, const StepPlan& sp, int mode, bool dbg)
       m.err = sv.err;
       m.phase_bar = h->W<int>(L.phase_bar) + 4 * (l + 1);
       m.n_phases = 4;
-      m.ph[0] = phase_o(l, 0);
-      m.ph[1] = phase_gu(l);
-      m.ph[2] = phase_down(l, 2);
-      m.ph[3] = (l + 1 < c.n_layers) ? phase_qkv(l + 1, 3) : phase_lm();
+      m.ph[0] = pb.o(l, 0);
+      m.ph[1] = pb.gu(l);
+      m.ph[2] = pb.down(l, 2, next_norm);
+      m.ph[3] = (l + 1 < c.n_layers) ? pb.qkv(l + 1, 3) : pb.lm(dbg ? h->dbg_logits : nullptr);
       if (h->trace && l == h->trace_layer) m.trace = h->trace;
       LK(SPEC_PROF_GEMM_LAYER, 1, gemm_multi_launch(m, st, pdl));
     } else {
@@ -652,6 +698,91 @@ cudaError_t enqueue_step(spec_handle* h, const StepPlan& sp, int mode, bool dbg)
   if (mode == STEP_VERIFY)
     LK(SPEC_PROF_COMPACT, 1,
        launch_kv_compact(sv, h->kv, c.n_layers, w.acc_len, w.acc_nodes, c.max_nodes, st, pdl && dt == 1));
+  return cudaSuccess;
+}
+
+// The draft head's step (A: its input rows, then its decoder layer, LM head and
+// top-k).  The draft layer is layer n_layers of the cache; prefix lengths come
+// with the parameter block.  With `kv_only` (draft prefill) the step stops once
+// the layer's K/V are stored: they depend on the layer input alone.
+cudaError_t enqueue_draft(spec_handle* h, const StepPlan& sp, bool kv_only, bool dbg) {
+  const spec_config& c = h->cfg;
+  const WsLayout& L = h->lay;
+  cudaStream_t st = h->stream;
+  const bool pdl = h->use_pdl && !h->prof;
+  StepView sv = make_view(h, sp.B, sp.M);
+  sv.seq_len = h->W<int32_t>(L.p_dlen);
+  const int d = c.hidden, M = sp.M, Ld = c.n_layers;
+  const int bi = sp.qkv.bn == 64 ? 0 : 1;
+  h->launches = 0;
+  CUDA_RET(cudaMemsetAsync(h->ws + L.gemm_ctr, 0, 4 * (size_t)kGemmCounters, st));
+  CUDA_RET(cudaMemsetAsync(h->ws + L.attn_ctr, 0, 4 * (size_t)L.attn_ctr_n, st));
+  CUDA_RET(cudaMemsetAsync(h->ws + L.phase_bar, 0, 4 * (size_t)L.phase_bar_n, st));
+  __nv_bfloat16* ge = h->W<__nv_bfloat16>(L.ge);
+  // metadata on the draft prefixes; e = E[token] into the right half of [g|e]
+  LK(SPEC_PROF_EMBED_META, 1,
+     launch_embed_meta(1, sv, h->embed, nullptr, d, c.rms_eps, nullptr, nullptr, nullptr, 0, 0,
+                       h->W<double>(L.inv_freq), c.head_dim / 2, STEP_SCORE, st, pdl, ge, 2 * d, d));
+  const PhaseBuilder pb(h, sp, sv);
+  // g = [l|m|h] . W_fuse^T into the left half of [g|e]
+  {
+    const GemmPlan pf = plan_gemm(h, 128, d, 3 * d, M, GEMM_EPI_STORE);
+    GemmTcLaunch g = gemm_launch(pf, GEMM_EPI_STORE, d, 3 * d, M, &h->map_fc_fuse, nullptr, nullptr,
+                                 &h->map_fsplit[bi], d, 0, 0, sv.err);
+    g.args.out_bf16 = ge;
+    g.args.ld_out = 2 * d;
+    LK(SPEC_PROF_DRAFT_FC, 1, gemm_tc_launch(g, st, pdl));
+  }
+  // x = [g|e] . W_in^T (a residual GEMM on x = 0), xn = split(x * attn_norm), ss
+  CUDA_RET(cudaMemsetAsync(h->ws + L.x, 0, 4 * (size_t)M * d, st));
+  {
+    const GemmPlan pf = plan_gemm(h, 128, d, 2 * d, M, GEMM_EPI_RESID);
+    GemmMultiLaunch m{};
+    m.bn = pf.bn;
+    m.grid = pf.grid;
+    m.err = sv.err;
+    m.phase_bar = h->W<int>(L.phase_bar);
+    m.n_phases = 1;
+    m.ph[0] = pb.resid(pf, 2 * d, &h->map_fc_in, &h->map_ge[bi], h->layers[Ld].attn_norm, 0);
+    LK(SPEC_PROF_DRAFT_FC, 1, gemm_multi_launch(m, st, false));
+  }
+  GemmMultiLaunch m{};
+  m.bn = sp.qkv.bn;
+  m.grid = sp.grid_all;
+  m.err = sv.err;
+  m.phase_bar = h->W<int>(L.phase_bar) + 4 * (c.n_layers + 1);
+  m.n_phases = 1;
+  m.ph[0] = pb.qkv(Ld, 1);
+  LK(SPEC_PROF_GEMM_QKV, 1, gemm_multi_launch(m, st, pdl));
+  if (kv_only) return cudaSuccess;
+
+  AttnArgs aa{};
+  aa.sv = sv;
+  aa.kv = h->kv;
+  aa.layer = Ld;
+  aa.Hq = c.n_q_heads;
+  aa.hd = c.head_dim;
+  aa.q = h->ws + L.q;
+  aa.out = h->ws + L.attn;
+  aa.part_o = h->W<float>(L.part_o);
+  aa.part_lse = h->W<float>(L.part_lse);
+  aa.n_chunks = sp.n_chunks;
+  aa.chunk = sp.chunk;
+  aa.max_rows = sp.max_rows;
+  aa.counters = h->W<int>(L.attn_ctr);
+  aa.q_rows = L.Mpad * (c.n_q_heads / c.n_kv_heads);
+  LK(SPEC_PROF_ATTENTION, 1, launch_attention_tc(aa, h->attn_maps, st, pdl));
+  float* logits = h->W<float>(L.dlogits);
+  m.n_phases = 4;
+  m.ph[0] = pb.o(Ld, 0);
+  m.ph[1] = pb.gu(Ld);
+  m.ph[2] = pb.down(Ld, 2, h->draft_final_norm);
+  m.ph[3] = pb.lm(logits);
+  LK(SPEC_PROF_GEMM_LAYER, 1, gemm_multi_launch(m, st, pdl));
+  LK(SPEC_PROF_TOPK, 1,
+     launch_topk_rows(M, c.vocab, logits, c.vocab, kDraftTopK, h->W<int32_t>(L.dtop_i), h->W<float>(L.dtop_v), st,
+                      pdl));
+  if (dbg) CUDA_RET(cudaMemcpyAsync(h->dbg_logits, logits, 4 * (size_t)M * c.vocab, cudaMemcpyDeviceToDevice, st));
   return cudaSuccess;
 }
 
@@ -774,6 +905,108 @@ int run_step(spec_handle* h, int B, const int32_t* seq_ids, const int32_t* token
   return SPEC_OK;
 }
 
+bool aligned16(const void* p) { return (reinterpret_cast<uintptr_t>(p) & 15u) == 0; }
+
+// Run one draft-head step (or a draft prefill chunk) from host inputs; feats
+// is a device pointer to bf16 [M][3][d].
+int run_draft(spec_handle* h, int B, const int32_t* seq_ids, const void* feats, const int32_t* tokens,
+              const int32_t* parents, const int32_t* node_off, bool kv_only, int flags, int32_t* top_idx,
+              float* top_val) {
+  const spec_config& c = h->cfg;
+  const WsLayout& L = h->lay;
+  if (!c.draft_head) return fail(h, SPEC_ERR_STATE, "the handle was created without the draft head");
+  if (B < 1 || B > c.max_batch) return fail(h, SPEC_ERR_CAPACITY, "batch %d outside [1, %d]", B, c.max_batch);
+  if (!seq_ids || !feats || !tokens || !parents || !node_off) return fail(h, SPEC_ERR_ARG, "null input pointer");
+  if (!aligned16(feats)) return fail(h, SPEC_ERR_ARG, "feats must be 16-byte aligned");
+  if (node_off[0] != 0) return fail(h, SPEC_ERR_ARG, "node_offsets[0] must be 0");
+  std::vector<uint8_t> seen(c.max_batch, 0);
+  int max_n = 0, max_lk = 0;
+  for (int b = 0; b < B; ++b) {
+    const int s = seq_ids[b];
+    if (s < 0 || s >= c.max_batch) return fail(h, SPEC_ERR_ARG, "seq id %d outside [0, %d)", s, c.max_batch);
+    if (seen[s]) return fail(h, SPEC_ERR_ARG, "seq id %d appears twice in one batch", s);
+    seen[s] = 1;
+    const int n = node_off[b + 1] - node_off[b];
+    if (n < 1) return fail(h, SPEC_ERR_ARG, "tree %d is empty", b);
+    if (n > c.max_nodes) return fail(h, SPEC_ERR_CAPACITY, "tree %d has %d nodes > max_nodes %d", b, n, c.max_nodes);
+    if (!kv_only && !h->dready[s]) return fail(h, SPEC_ERR_STATE, "sequence %d has no draft prefix", s);
+    if (h->dlen[s] + n > c.max_seq)
+      return fail(h, SPEC_ERR_CAPACITY, "sequence %d: draft length %d + %d nodes exceeds max_seq %d", s, h->dlen[s], n,
+                  c.max_seq);
+    const int vr = spec_validate_tree(tokens + node_off[b], parents + node_off[b], n, c.vocab, c.max_nodes);
+    if (vr == SPEC_ERR_TREE) return fail(h, vr, "tree %d: parents[0] must be -1 and 0 <= parents[i] < i", b);
+    if (vr) return fail(h, vr, "tree %d rejected", b);
+    max_n = std::max(max_n, n);
+    max_lk = std::max(max_lk, h->dlen[s] + n);
+  }
+  const int M = node_off[B];
+  const bool dbg = (flags & SPEC_DEBUG_LOGITS) != 0 && !kv_only;
+  if (dbg && (!h->dbg_logits || h->dbg_bytes < sizeof(float) * (size_t)M * c.vocab))
+    return fail(h, SPEC_ERR_CAPACITY, "SPEC_DEBUG_LOGITS needs a debug buffer of %zu bytes",
+                sizeof(float) * (size_t)M * c.vocab);
+  uint8_t* pb = h->h_params;
+  std::memcpy(pb + L.p_tokens, tokens, 4 * (size_t)M);
+  std::memcpy(pb + L.p_parents, parents, 4 * (size_t)M);
+  std::memcpy(pb + L.p_node_off, node_off, 4 * (size_t)(B + 1));
+  std::memcpy(pb + L.p_seq_ids, seq_ids, 4 * (size_t)B);
+  std::memcpy(pb + L.p_dlen, h->dlen.data(), 4 * (size_t)c.max_batch);
+  std::memset(pb + L.p_err, 0, 16);
+  CUDA_TRY(h, cudaMemcpyAsync(h->ws, pb, L.p_end, cudaMemcpyHostToDevice, h->stream));
+  // the caller's features become the first GEMM's split operand (outside any graph:
+  // the pointer may change from call to call)
+  CUDA_TRY(h, launch_split_rows(static_cast<const __nv_bfloat16*>(feats), M, 3 * c.hidden,
+                                h->W<__nv_bfloat16>(L.fsplit), h->stream, false));
+  StepPlan sp = make_plan(h, B, M, max_n, max_lk);
+  const int mode = kv_only ? STEP_DRAFT_KV : STEP_DRAFT;
+  const bool graph = !(flags & SPEC_NO_GRAPH) && !h->prof && h->stream != nullptr;
+  if (graph) {
+    GraphKey key{mode, B, M, max_n, sp.n_chunks, sp.chunk, dbg ? 1 : 0, h->use_pdl ? 1 : 0};
+    auto it = h->graphs.find(key);
+    if (it == h->graphs.end()) {
+      cudaGraph_t g = nullptr;
+      CUDA_TRY(h, cudaStreamBeginCapture(h->stream, cudaStreamCaptureModeThreadLocal));
+      cudaError_t e = enqueue_draft(h, sp, kv_only, dbg);
+      cudaError_t e2 = cudaStreamEndCapture(h->stream, &g);
+      if (e != cudaSuccess || e2 != cudaSuccess) {
+        if (g) cudaGraphDestroy(g);
+        return fail(h, SPEC_ERR_CUDA, "graph capture failed: %s", cudaGetErrorString(e != cudaSuccess ? e : e2));
+      }
+      cudaGraphExec_t ex = nullptr;
+      e = cudaGraphInstantiate(&ex, g, 0);
+      cudaGraphDestroy(g);
+      if (e != cudaSuccess) return fail(h, SPEC_ERR_CUDA, "graph instantiate failed: %s", cudaGetErrorString(e));
+      it = h->graphs.emplace(key, ex).first;
+    }
+    CUDA_TRY(h, cudaGraphLaunch(it->second, h->stream));
+  } else {
+    cudaError_t e = enqueue_draft(h, sp, kv_only, dbg);
+    if (e != cudaSuccess) return fail(h, SPEC_ERR_CUDA, "kernel launch failed: %s", cudaGetErrorString(e));
+  }
+  if (!kv_only && (flags & SPEC_DEVICE_OUTPUTS)) {
+    if (top_idx)
+      CUDA_TRY(h, cudaMemcpyAsync(top_idx, h->ws + L.dtop_i, 4 * (size_t)M * kDraftTopK, cudaMemcpyDeviceToDevice,
+                                  h->stream));
+    if (top_val)
+      CUDA_TRY(h, cudaMemcpyAsync(top_val, h->ws + L.dtop_v, 4 * (size_t)M * kDraftTopK, cudaMemcpyDeviceToDevice,
+                                  h->stream));
+    return SPEC_OK;
+  }
+  if (!kv_only) {
+    if (top_idx)
+      CUDA_TRY(h, cudaMemcpyAsync(top_idx, h->ws + L.dtop_i, 4 * (size_t)M * kDraftTopK, cudaMemcpyDeviceToHost,
+                                  h->stream));
+    if (top_val)
+      CUDA_TRY(h, cudaMemcpyAsync(top_val, h->ws + L.dtop_v, 4 * (size_t)M * kDraftTopK, cudaMemcpyDeviceToHost,
+                                  h->stream));
+  }
+  uint32_t errw[2] = {0, 0};
+  CUDA_TRY(h, cudaMemcpyAsync(errw, h->ws + L.p_err, 4, cudaMemcpyDeviceToHost, h->stream));
+  CUDA_TRY(h, cudaStreamSynchronize(h->stream));
+  if (errw[0] & SPEC_DEVERR_TIMEOUT) return fail(h, SPEC_ERR_TIMEOUT, "a bounded wait expired on the device");
+  if (errw[0]) return fail(h, SPEC_ERR_CUDA, "device reported error bits 0x%x", errw[0]);
+  return SPEC_OK;
+}
+
 int refresh_state(spec_handle* h) {
   const WsLayout& L = h->lay;
   const int nb = h->cfg.max_batch;
@@ -795,8 +1028,6 @@ int refresh_state(spec_handle* h) {
   if (sticky) return fail(h, SPEC_ERR_CUDA, "device reported error bits 0x%x", sticky);
   return SPEC_OK;
 }
-
-bool aligned16(const void* p) { return (reinterpret_cast<uintptr_t>(p) & 15u) == 0; }
 
 }  // namespace
 
@@ -841,12 +1072,16 @@ int spec_init(const spec_config* cfg, const spec_weights* w, void* kv_cache, siz
   if (!aligned16(kv_cache) || !aligned16(workspace) || !aligned16(w->embed) || !aligned16(w->lm_head) ||
       !aligned16(w->final_norm))
     return SPEC_ERR_ARG;
-  for (int l = 0; l < c.n_layers; ++l) {
-    const spec_layer_weights& lw = w->layers[l];
+  for (int l = 0; l < cache_layers(c); ++l) {
+    if (l == c.n_layers && !w->draft_layer) return SPEC_ERR_ARG;
+    const spec_layer_weights& lw = l < c.n_layers ? w->layers[l] : *w->draft_layer;
     const void* ps[9] = {lw.wq, lw.wk, lw.wv, lw.wo, lw.w_gate, lw.w_up, lw.w_down, lw.attn_norm, lw.mlp_norm};
     for (const void* p : ps)
       if (!p || !aligned16(p)) return SPEC_ERR_ARG;
   }
+  if (c.draft_head && (!w->draft_fc_fuse || !w->draft_fc_in || !w->draft_final_norm || !aligned16(w->draft_fc_fuse) ||
+                       !aligned16(w->draft_fc_in) || !aligned16(w->draft_final_norm)))
+    return SPEC_ERR_ARG;
 
   spec_handle* h = new spec_handle();
   h->cfg = c;
@@ -856,6 +1091,14 @@ int spec_init(const spec_config* cfg, const spec_weights* w, void* kv_cache, siz
   h->final_norm = w->final_norm;
   h->lm_head = w->lm_head;
   h->layers.assign(w->layers, w->layers + c.n_layers);
+  if (c.draft_head) {
+    h->layers.push_back(*w->draft_layer);
+    h->draft_fc_fuse = w->draft_fc_fuse;
+    h->draft_fc_in = w->draft_fc_in;
+    h->draft_final_norm = w->draft_final_norm;
+  }
+  h->dlen.assign(c.max_batch, 0);
+  h->dready.assign(c.max_batch, 0);
   h->ws = reinterpret_cast<uint8_t*>(workspace);
   h->kv.base = kv_cache;
   h->kv.max_batch = c.max_batch;
@@ -911,7 +1154,7 @@ int spec_init(const spec_config* cfg, const spec_weights* w, void* kv_cache, siz
     {
       // q as [Hkv * q_rows][128] and the cache as [layers * 2 * batch * Hkv * max_seq][128], fp16;
       // TMA row coordinates are 32-bit
-      const uint64_t cache_rows = (uint64_t)c.n_layers * 2 * c.max_batch * c.n_kv_heads * c.max_seq;
+      const uint64_t cache_rows = (uint64_t)cache_layers(c) * 2 * c.max_batch * c.n_kv_heads * c.max_seq;
       if (cache_rows + 128 >= (1ull << 31)) return bail(SPEC_ERR_CAPACITY, "cache too large for 32-bit rows");
       const uint64_t q_rows = (uint64_t)c.n_kv_heads * lay.Mpad * (c.n_q_heads / c.n_kv_heads);
       if (!make_tmap(&h->attn_maps.q, h->ws + lay.q, q_rows, 128, 128, CU_TENSOR_MAP_DATA_TYPE_FLOAT16) ||
@@ -924,8 +1167,8 @@ int spec_init(const spec_config* cfg, const spec_weights* w, void* kv_cache, siz
           cudaStreamSynchronize(h->stream) != cudaSuccess)
         return bail(SPEC_ERR_CUDA, "cache init");
     }
-    h->maps.resize(c.n_layers);
-    for (int l = 0; l < c.n_layers; ++l) {
+    h->maps.resize(h->layers.size());
+    for (int l = 0; l < (int)h->layers.size(); ++l) {
       const spec_layer_weights& lw = h->layers[l];
       LayerMaps& m = h->maps[l];
       bool ok = make_tmap(&m.wq, lw.wq, qd, c.hidden, 128) && make_tmap(&m.wk, lw.wk, kvd, c.hidden, 128) &&
@@ -935,12 +1178,21 @@ int spec_init(const spec_config* cfg, const spec_weights* w, void* kv_cache, siz
       if (!ok) return bail(SPEC_ERR_CUDA, "tensor map");
     }
     if (!make_tmap(&h->map_lm, h->lm_head, c.vocab, c.hidden, 128)) return bail(SPEC_ERR_CUDA, "tensor map");
+    if (c.draft_head &&
+        (!make_tmap(&h->map_fc_fuse, h->draft_fc_fuse, c.hidden, 3 * (uint64_t)c.hidden, 128) ||
+         !make_tmap(&h->map_fc_in, h->draft_fc_in, c.hidden, 2 * (uint64_t)c.hidden, 128)))
+      return bail(SPEC_ERR_CUDA, "tensor map");
     const int bns[2] = {64, 128};
     for (int i = 0; i < 2; ++i) {
       // split activations: a tile of BN tokens is 2*BN rows (hi and lo)
       if (!make_tmap(&h->map_xn[i], h->ws + lay.xn, 2 * (uint64_t)lay.Mpad, c.hidden, 2 * bns[i]) ||
           !make_tmap(&h->map_attn[i], h->ws + lay.attn, 2 * (uint64_t)lay.Mpad, qd, 2 * bns[i]) ||
           !make_tmap(&h->map_h[i], h->ws + lay.hmlp, 2 * (uint64_t)lay.Mpad, c.ffn, 2 * bns[i]))
+        return bail(SPEC_ERR_CUDA, "tensor map");
+      if (c.draft_head &&
+          (!make_tmap(&h->map_fsplit[i], h->ws + lay.fsplit, 2 * (uint64_t)lay.Mpad, 3 * (uint64_t)c.hidden,
+                      2 * bns[i]) ||
+           !make_tmap(&h->map_ge[i], h->ws + lay.ge, 2 * (uint64_t)lay.Mpad, 2 * (uint64_t)c.hidden, 2 * bns[i])))
         return bail(SPEC_ERR_CUDA, "tensor map");
     }
     for (int i = 0; i < 2; ++i)
@@ -1062,6 +1314,55 @@ int spec_score_trees(spec_handle* h, int B, const int32_t* seq_ids, const int32_
   if (argmax) CUDA_TRY(h, cudaMemcpy(argmax, h->ws + L.argmax, 4 * (size_t)M, cudaMemcpyDeviceToHost));
   if (top1) CUDA_TRY(h, cudaMemcpy(top1, h->ws + L.top1, 4 * (size_t)M, cudaMemcpyDeviceToHost));
   if (top2) CUDA_TRY(h, cudaMemcpy(top2, h->ws + L.top2, 4 * (size_t)M, cudaMemcpyDeviceToHost));
+  return SPEC_OK;
+}
+
+int spec_draft_prefill(spec_handle* h, int seq, const void* feats, const int32_t* tokens, int n) {
+  if (!h) return SPEC_ERR_ARG;
+  h->err.clear();
+  const spec_config& c = h->cfg;
+  if (!c.draft_head) return fail(h, SPEC_ERR_STATE, "the handle was created without the draft head");
+  if (!feats || !tokens || n < 1) return fail(h, SPEC_ERR_ARG, "draft prefill needs n >= 1 rows");
+  if (seq < 0 || seq >= c.max_batch) return fail(h, SPEC_ERR_ARG, "seq %d outside [0, %d)", seq, c.max_batch);
+  if (n > c.max_seq) return fail(h, SPEC_ERR_CAPACITY, "draft prefix of %d rows exceeds max_seq %d", n, c.max_seq);
+  if (h->stale) {
+    int rc = refresh_state(h);
+    if (rc) return rc;
+  }
+  // chunks of max_nodes rows as chains: each row's K/V at its own position
+  h->dlen[seq] = 0;
+  h->dready[seq] = 0;
+  const size_t row_bytes = 2 * 3 * (size_t)c.hidden;
+  std::vector<int32_t> par(c.max_nodes);
+  for (int i = 0; i < c.max_nodes; ++i) par[i] = i - 1;
+  for (int i0 = 0; i0 < n; i0 += c.max_nodes) {
+    const int m = std::min(c.max_nodes, n - i0);
+    const int32_t off[2] = {0, m};
+    const int rc = run_draft(h, 1, &seq, static_cast<const uint8_t*>(feats) + (size_t)i0 * row_bytes, tokens + i0,
+                             par.data(), off, true, 0, nullptr, nullptr);
+    if (rc) return rc;
+    h->dlen[seq] += m;
+  }
+  h->dready[seq] = 1;
+  return SPEC_OK;
+}
+
+int spec_draft_step(spec_handle* h, int B, const int32_t* seq_ids, const void* feats, const int32_t* tokens,
+                    const int32_t* parents, const int32_t* node_offsets, int32_t* top_idx, float* top_val,
+                    int flags) {
+  if (!h) return SPEC_ERR_ARG;
+  h->err.clear();
+  if (h->stale) {
+    int rc = refresh_state(h);
+    if (rc) return rc;
+  }
+  return run_draft(h, B, seq_ids, feats, tokens, parents, node_offsets, false, flags, top_idx, top_val);
+}
+
+int spec_draft_len(spec_handle* h, int seq, int32_t* len) {
+  if (!h || !len) return SPEC_ERR_ARG;
+  if (seq < 0 || seq >= h->cfg.max_batch) return fail(h, SPEC_ERR_ARG, "seq %d outside [0, %d)", seq, h->cfg.max_batch);
+  *len = h->dlen[seq];
   return SPEC_OK;
 }
 

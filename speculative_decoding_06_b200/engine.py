@@ -43,14 +43,14 @@ class SpecEngine:
     """One handle of the library over caller-owned (torch) device buffers."""
 
     def __init__(self, dims, weights: Dict, max_batch: int, max_seq: int, max_nodes: int = 128,
-                 stream: Optional[torch.cuda.Stream] = None):
+                 stream: Optional[torch.cuda.Stream] = None, draft: Optional[Dict] = None):
         self.dims = dims
         self.cfg = S.spec_config(
             n_layers=dims.n_layers, hidden=dims.hidden, n_q_heads=dims.n_q_heads, n_kv_heads=dims.n_kv_heads,
             head_dim=dims.head_dim, ffn=dims.ffn, vocab=dims.vocab,
             dtype=S.SPEC_DTYPE_BF16 if dims.dtype == "bf16" else S.SPEC_DTYPE_F32,
             rms_eps=dims.rms_eps, rope_theta=dims.rope_theta, max_batch=max_batch, max_seq=max_seq,
-            max_nodes=max_nodes, draft_head=0)
+            max_nodes=max_nodes, draft_head=1 if draft is not None else 0)
         self.max_nodes = max_nodes
         self.max_batch = max_batch
         kvb = S.spec_kv_bytes(ctypes.byref(self.cfg))
@@ -66,6 +66,15 @@ class SpecEngine:
                 setattr(self._layers[l], k, lw[k].data_ptr())
         self._w = S.spec_weights(embed=weights["embed"].data_ptr(), final_norm=weights["final_norm"].data_ptr(),
                                  lm_head=weights["lm_head"].data_ptr(), layers=self._layers)
+        self._draft = draft
+        if draft is not None:
+            self._dlayer = S.spec_layer_weights()
+            for k in _LAYER_KEYS:
+                setattr(self._dlayer, k, draft["layer"][k].data_ptr())
+            self._w.draft_fc_fuse = draft["fc_fuse"].data_ptr()
+            self._w.draft_fc_in = draft["fc_in"].data_ptr()
+            self._w.draft_layer = ctypes.pointer(self._dlayer)
+            self._w.draft_final_norm = draft["final_norm"].data_ptr()
         # a dedicated stream: the legacy default stream cannot be captured into graphs
         self.stream = stream or torch.cuda.Stream()
         torch.cuda.synchronize()  # weights and buffers were written on torch's stream
@@ -189,8 +198,43 @@ class SpecEngine:
     def sync(self):
         self._check(S.spec_sync(self.h))
 
+    # ------------------------------------------------------------------ draft head
+    def draft_prefill(self, seq: int, feats: torch.Tensor, tokens):
+        """feats: bf16 device tensor [n][3][d]; tokens: the token one step ahead per row."""
+        t = _i32(tokens)
+        f = feats.contiguous()
+        self.stream.wait_stream(torch.cuda.current_stream())
+        self._check(S.spec_draft_prefill(self.h, seq, f.data_ptr(), _ptr(t), len(t)))
+
+    def draft_step(self, seq_ids, feats: torch.Tensor, trees, flags: int = 0):
+        """Host outputs top_idx [nodes][10] int32, top_val [nodes][10] fp32, node offsets."""
+        tok, par, off = pack_trees(trees)
+        ids = _i32(seq_ids)
+        M = int(off[-1])
+        if flags & S.SPEC_DEBUG_LOGITS and (self._dbg is None or self._dbg.numel() < M * self.dims.vocab):
+            self.enable_debug_logits(self.max_batch * self.max_nodes)
+        ti = np.zeros((M, S.SPEC_DRAFT_TOPK), np.int32)
+        tv = np.zeros((M, S.SPEC_DRAFT_TOPK), np.float32)
+        f = feats.contiguous()
+        self.stream.wait_stream(torch.cuda.current_stream())
+        self._check(S.spec_draft_step(self.h, len(ids), _ptr(ids), f.data_ptr(), _ptr(tok), _ptr(par), _ptr(off),
+                                      ti.ctypes.data, tv.ctypes.data, flags & ~S.SPEC_DEVICE_OUTPUTS))
+        return ti, tv, off
+
+    def draft_step_device(self, ids, feats: torch.Tensor, tok, par, off, outputs=None, flags: int = 0):
+        """Queue a draft step without synchronising (outputs: optional int32 / fp32 device tensors)."""
+        ptrs = [None, None] if outputs is None else [o.data_ptr() if o is not None else None for o in outputs]
+        self._check(S.spec_draft_step(self.h, len(ids), _ptr(ids), feats.data_ptr(), _ptr(tok), _ptr(par),
+                                      _ptr(off), ptrs[0], ptrs[1], flags | S.SPEC_DEVICE_OUTPUTS))
+
+    def draft_len(self, seq: int) -> int:
+        ln = np.zeros(1, np.int32)
+        self._check(S.spec_draft_len(self.h, seq, _ptr(ln)))
+        return int(ln[0])
+
     def kv_view(self) -> torch.Tensor:
         """The cache as a tensor [layer][2][max_batch][Hkv][max_seq][hd] (fp16 for bf16 models, else fp32)."""
         d = self.dims
         tdt = torch.float16 if d.dtype == "bf16" else torch.float32
-        return self.kv.view(tdt).view(d.n_layers, 2, self.max_batch, d.n_kv_heads, -1, d.head_dim)
+        layers = d.n_layers + (1 if self._draft is not None else 0)  # the draft head's layer comes last
+        return self.kv.view(tdt).view(layers, 2, self.max_batch, d.n_kv_heads, -1, d.head_dim)

@@ -29,9 +29,10 @@ SPEC_DTYPE_BF16 = 1
 SPEC_DEVICE_OUTPUTS = 1
 SPEC_DEBUG_LOGITS = 2
 SPEC_NO_GRAPH = 4
+SPEC_DRAFT_TOPK = 10
 
 PROF_CLASSES = ("embed_meta", "gemm_qkv", "rope_kv_store", "attention", "gemm_o", "resid_norm", "gemm_gate_up",
-                "gemm_down", "lm_head", "lm_reduce", "accept_walk", "kv_compact", "gemm_layer")
+                "gemm_down", "lm_head", "lm_reduce", "accept_walk", "kv_compact", "gemm_layer", "draft_fc", "topk")
 
 ERR_NAMES = {0: "SPEC_OK", -1: "SPEC_ERR_ARG", -2: "SPEC_ERR_TREE", -3: "SPEC_ERR_TOKEN", -4: "SPEC_ERR_CAPACITY",
              -5: "SPEC_ERR_ROOT", -6: "SPEC_ERR_CUDA", -7: "SPEC_ERR_TIMEOUT", -8: "SPEC_ERR_STATE"}
@@ -90,6 +91,9 @@ _SIGNATURES = {
     "spec_io_bytes": (ctypes.c_int, [_h, ctypes.POINTER(ctypes.c_size_t), ctypes.POINTER(ctypes.c_size_t)]),
     "spec_lm_head_argmax_noalloc": (ctypes.c_int, [_vp, _vp, _vp, ctypes.c_int, ctypes.c_int, ctypes.c_int,
                                                     ctypes.c_float, _vp, _vp, _vp, _vp]),
+    "spec_draft_prefill": (ctypes.c_int, [_h, ctypes.c_int, _vp, _i32p, ctypes.c_int]),
+    "spec_draft_step": (ctypes.c_int, [_h, ctypes.c_int, _i32p, _vp, _i32p, _i32p, _i32p, _vp, _vp, ctypes.c_int]),
+    "spec_draft_len": (ctypes.c_int, [_h, ctypes.c_int, _i32p]),
     "spec_last_error": (ctypes.c_char_p, [_h]),
     "spec_free": (None, [_h]),
 }
@@ -129,24 +133,7 @@ def _bind(name):
     return call
 
 
-spec_kv_bytes = _bind("spec_kv_bytes")
-spec_workspace_bytes = _bind("spec_workspace_bytes")
-spec_init = _bind("spec_init")
-spec_prefill = _bind("spec_prefill")
-spec_verify_tree = _bind("spec_verify_tree")
-spec_verify_tree_batch = _bind("spec_verify_tree_batch")
-spec_score_trees = _bind("spec_score_trees")
-spec_set_debug_logits = _bind("spec_set_debug_logits")
-spec_truncate = _bind("spec_truncate")
-spec_seq_len = _bind("spec_seq_len")
-spec_sync = _bind("spec_sync")
-spec_validate_tree = _bind("spec_validate_tree")
-spec_profile = _bind("spec_profile")
-spec_profile_read = _bind("spec_profile_read")
-spec_step_launches = _bind("spec_step_launches")
-spec_set_trace = _bind("spec_set_trace")
-spec_info = _bind("spec_info")
-spec_io_bytes = _bind("spec_io_bytes")
-spec_lm_head_argmax_noalloc = _bind("spec_lm_head_argmax_noalloc")
-spec_last_error = _bind("spec_last_error")
-spec_free = _bind("spec_free")
+# one Python function per C entry point, same name
+for _name in _SIGNATURES:
+    globals()[_name] = _bind(_name)
+del _name
