@@ -17,8 +17,9 @@
 //                        O += P_j V_j into a third (V is read MN-major);
 //   warps 0-3:           thread r owns query row r: reads S_j from its TMEM
 //                        lane, applies the ancestor mask and the online softmax
-//                        (the running max only moves when it grows by more than
-//                        2^8, which keeps every p <= 256 and rescales O rarely),
+//                        (the running max only moves when a block's max exceeds
+//                        it by more than the slack, 8 in log2 units by default:
+//                        every p stays <= 2^8 and O is rescaled rarely),
 //                        writes P_j into shared memory as the next MMA's A
 //                        operand, and at the end normalises O.
 //
@@ -42,7 +43,6 @@ constexpr int kKeys = 128;                   // keys per block (S's N, P.V's K)
 constexpr int kThreads = 160;                // warps 0-3 rows, warp 4 issue
 constexpr uint32_t kHalf = 128 * 128;        // [128 rows][64 fp16] swizzled: 16 KB
 constexpr uint32_t kTile = 2 * kHalf;        // 128 x 128 fp16: 32 KB
-constexpr float kRescaleLog2 = 8.f;          // running-max slack (log2 units)
 
 enum { B_QFULL = 0, B_KVFULL = 1, B_KVEMPTY = 3, B_SFULL = 5, B_SFREE = 7, B_PFULL = 9, B_PEMPTY = 10, B_OFULL = 11,
        B_DRAIN = 12, kNumBars = 13 };
@@ -353,7 +353,7 @@ __global__ void __launch_bounds__(kThreads, 1) attn_tc_kernel(const __grid_const
       const float mblk = fmaxf(fmaxf(mx4[0], mx4[1]), fmaxf(mx4[2], mx4[3])) * sl2;
       if (j == 0) stamp(a.trace, 8);
       float corr = 1.f;
-      if (mblk > m + kRescaleLog2) {
+      if (mblk > m + a.rescale_slack) {
         corr = fast_exp2(m - mblk);  // 0 while nothing was visible
         m = mblk;
       }

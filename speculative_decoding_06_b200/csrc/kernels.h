@@ -191,6 +191,7 @@ struct AttnArgs {
   int n_chunks, chunk;      // key chunking of [0, P_b + n_b)
   int max_rows;             // max over batch of n_b * (Hq/Hkv)
   int q_rows;               // bf16 path: q is [Hkv][q_rows][hd], row node * G + g
+  float rescale_slack;      // bf16 path: the running max moves only when a block's max exceeds it by this (log2 units)
   int* counters;            // bf16 path: [groups][2] chunk arrivals / departures, zero between launches
   uint64_t* trace;          // optional [256 CTAs][16] %globaltimer marks (attention_tc.cu)
 };

@@ -264,6 +264,7 @@ struct spec_handle {
   int max_splits = 16;    // split-K cap
   int max_chunks = kMaxAttnChunks;  // attention key-chunk cap
   int resident_cap = 0;   // 0: as many CTAs per SM as fit
+  float rescale_slack = 8.f;  // attention: running-max slack in log2 units (p <= 2^slack)
   // L2 prefetch of weights ahead of the GEMM that streams them
   uint64_t* trace = nullptr;  // optional GEMM timeline of one layer's launch
   size_t trace_bytes = 0;
@@ -612,6 +613,7 @@ cudaError_t enqueue_step(spec_handle* h, const StepPlan& sp, int mode, bool dbg)
   aa.max_rows = sp.max_rows;
   aa.counters = h->W<int>(L.attn_ctr);
   aa.q_rows = L.Mpad * (c.n_q_heads / c.n_kv_heads);
+  aa.rescale_slack = h->rescale_slack;
 
   const PhaseBuilder pb(h, sp, sv);
   if (dt == 1) {
@@ -771,6 +773,7 @@ cudaError_t enqueue_draft(spec_handle* h, const StepPlan& sp, bool kv_only, bool
   aa.max_rows = sp.max_rows;
   aa.counters = h->W<int>(L.attn_ctr);
   aa.q_rows = L.Mpad * (c.n_q_heads / c.n_kv_heads);
+  aa.rescale_slack = h->rescale_slack;
   LK(SPEC_PROF_ATTENTION, 1, launch_attention_tc(aa, h->attn_maps, st, pdl));
   float* logits = h->W<float>(L.dlogits);
   m.n_phases = 4;
@@ -1123,6 +1126,8 @@ int spec_init(const spec_config* cfg, const spec_weights* w, void* kv_cache, siz
     if (const char* q = strstr(t, "chunks=")) if (sscanf(q + 7, "%d", &v) == 1 && v >= 1 && v <= kMaxAttnChunks) h->max_chunks = v;
     if (const char* q = strstr(t, "pdl=")) if (sscanf(q + 4, "%d", &v) == 1) h->use_pdl = v != 0;
     if (const char* q = strstr(t, "per_sm=")) if (sscanf(q + 7, "%d", &v) == 1 && v >= 0) h->resident_cap = v;
+    float fv = 0.f;
+    if (const char* q = strstr(t, "rescale=")) if (sscanf(q + 8, "%f", &fv) == 1 && fv >= 0.f && fv <= 15.f) h->rescale_slack = fv;
   }
   if (cudaGetDevice(&h->device) != cudaSuccess) return bail(SPEC_ERR_CUDA, "cudaGetDevice");
   cudaDeviceProp prop;

@@ -8,6 +8,8 @@ GEMM and attention tiles, ragged tails, root-only trees, chains, 128-node
 trees and batches of sequences with different prefix lengths.
 """
 
+import os
+
 import numpy as np
 import pytest
 
@@ -160,3 +162,75 @@ def test_wide_bf16_full_size_tiles():
     shape = synth.tree_from_widths(synth.TREE60_WIDTHS, stream=0)
     toks = planted_tree(om, seq, shape, 0.8, stream=9)
     _check_step(eng, om, 0, seq, shape, toks, "bf16")
+
+
+def _check_batch(eng, om, ids, seqs, trees):
+    """Score and verify a batch; compare logits, outputs and the compacted K/V per sequence."""
+    amax, t1, t2, off = eng.score(ids, trees, flags=2)
+    logits = eng.debug_logits(int(off[-1]))
+    acc_len, acc_nodes, acc_tok, bonus = eng.verify_batch(ids, trees)
+    decided = 0
+    for i, (seq, (toks, par)) in enumerate(zip(seqs, trees)):
+        r = oracle_verify(om, seq, toks, par)
+        lg = logits[off[i]:off[i + 1]]
+        err = float(np.max(np.abs(lg - r["logits"])))
+        assert err <= TOL["bf16"], "sequence %d: max |logit error| %.3g" % (i, err)
+        thr = min(DECISIVE, max(2.5 * err, 1e-6))
+        sure = r["margin"] > thr
+        assert np.array_equal(amax[off[i]:off[i + 1]][sure], r["argmax"][sure])
+        if np.all(r["margin"][decisive_nodes(r, par)] > thr):
+            decided += 1
+            assert acc_len[i] == r["accepted_len"]
+            assert list(acc_nodes[i, :acc_len[i]]) == r["accepted_nodes"]
+            assert list(acc_tok[i, :acc_len[i]]) == r["accepted_tokens"]
+            assert bonus[i] == r["bonus"]
+            ln, _ = eng.seq_len(ids[i])
+            gk, gv = gpu_kv(eng, ids[i], ln)
+            for l in range(om.d.n_layers):
+                assert kv_close(gk[l], seq.k[l], 2e-2) <= 2e-2
+                assert kv_close(gv[l], seq.v[l], 2e-2) <= 2e-2
+    return decided
+
+
+def test_bf16_large_batch_unchunked():
+    """20 sequences (prefixes 150-600) x 61-node trees = 1220 tokens: 128-token GEMM tiles, several token
+    tiles, and attention without key chunks (one CTA walks every 128-key block with the online softmax)."""
+    eng, om = make_pair(synth.SMALL_BF16, max_batch=20, max_seq=1024, max_nodes=64)
+    B = 20
+    Ps = np.random.default_rng(4).integers(150, 601, size=B)
+    seqs, trees = [], []
+    for i in range(B):
+        prefix, seq = decisive_prefix(om, int(Ps[i]), stream0=300 + 7 * i)
+        assert eng.prefill(i, prefix) == seq.pending
+        sh = synth.tree_from_widths(synth.TREE60_WIDTHS, stream=i)
+        trees.append((planted_tree(om, seq, sh, 0.8, stream=60 + i), sh.parents))
+        seqs.append(seq)
+    assert "chunks 1 x" in eng.info(B, 61, int(Ps.max()))
+    assert _check_batch(eng, om, list(range(B)), seqs, trees) >= B // 2
+
+
+def _engine_tuned(dims, tune, **kw):
+    old = os.environ.get("SPEC_TUNE")
+    os.environ["SPEC_TUNE"] = tune
+    try:
+        return make_pair(dims, **kw)
+    finally:
+        if old is None:
+            del os.environ["SPEC_TUNE"]
+        else:
+            os.environ["SPEC_TUNE"] = old
+
+
+@pytest.mark.parametrize("tune", ["chunks=2", "chunks=1", "chunks=2,rescale=0", "chunks=1,rescale=0"])
+def test_bf16_multiblock_attention(tune):
+    """Prefix 700 + 61 nodes = 6 key blocks per (sequence, kv head) in 2 chunks or 1; slack 0 makes every
+    growth of the running max rescale the accumulated output."""
+    eng, om = _engine_tuned(synth.MINI_BF16, tune, max_batch=2, max_seq=1024, max_nodes=64)
+    seqs, trees = [], []
+    for i, P in enumerate((700, 530)):
+        prefix, seq = decisive_prefix(om, P, stream0=500 + 11 * i)
+        assert eng.prefill(i, prefix) == seq.pending
+        sh = synth.tree_from_widths(synth.TREE60_WIDTHS, stream=3 + i)
+        trees.append((planted_tree(om, seq, sh, 0.8, stream=70 + i), sh.parents))
+        seqs.append(seq)
+    _check_batch(eng, om, [0, 1], seqs, trees)
