@@ -369,6 +369,183 @@ def run_ours(args, rank, world, local_rank):
     return 0
 
 
+# ---------------------------------------------------------------------------
+# the other configurations of the pages' workload list (one JSON line each;
+# the default line above stays the batch-1 verification step)
+# ---------------------------------------------------------------------------
+
+def flops_per_token(d):
+    """Dense multiply-adds x 2 per token through every weight matrix (attention scores excluded)."""
+    per_layer = d.q_dim * d.hidden + 2 * d.kv_dim * d.hidden + d.hidden * d.q_dim + 3 * d.ffn * d.hidden
+    return 2 * (d.n_layers * per_layer + d.vocab * d.hidden)
+
+
+def attn_flops(d, rows_keys, layers):
+    """QK and PV: 4 * head_dim flops per (query head, node, visible key) per layer; rows_keys = sum over
+    nodes of their visible keys."""
+    return 4 * d.head_dim * d.n_q_heads * rows_keys * layers
+
+
+def _timed(stream, fn, steps, reset):
+    import torch
+    times = []
+    for _ in range(steps):
+        e0 = torch.cuda.Event(enable_timing=True)
+        e1 = torch.cuda.Event(enable_timing=True)
+        e0.record(stream)
+        fn()
+        e1.record(stream)
+        e1.synchronize()
+        times.append(e0.elapsed_time(e1))
+        reset()
+    return float(np.mean(times))
+
+
+def _roofline(bytes_, flops, ms):
+    hbm, tflops, kind = measured_peaks()
+    t_mem = bytes_ / hbm / 1e6
+    t_fl = flops / tflops / 1e9
+    bound = "hbm" if t_mem >= t_fl else "tensor"
+    return {"bound": bound, "bytes": bytes_, "flops": flops, "roofline_ms": max(t_mem, t_fl),
+            "frac": max(t_mem, t_fl) / ms, "hbm_gbs": hbm, "bf16_tflops": tflops, "peak_source": kind}
+
+
+def run_batch64(args):
+    """64 sequences, prefixes uniform in [512, 4096], each with its own 60-draft tree, p uniform in [0.6, 0.9]."""
+    import torch
+    from speculative_decoding_06_b200.engine import SpecEngine, pack_trees
+    dims = synth.LLAMA8B
+    B = 64
+    lens, ps = synth.batch_prefix_lengths_and_p(B)
+    w = synth.model_weights(dims, seed=0, device="cuda")
+    eng = SpecEngine(dims, w, max_batch=B, max_seq=int(lens.max()) + 64, max_nodes=64)
+    trees = []
+    for b in range(B):
+        pend = eng.prefill(b, synth.prefix_tokens(dims.vocab, int(lens[b]), stream=b))
+        sh = synth.tree_from_widths(synth.TREE60_WIDTHS, stream=b)
+        draws = synth.plant_draws(sh.n, dims.vocab, stream=b)
+        toks = synth.plant_tree(sh, pend, float(ps[b]), draws,
+                                lambda t, p_, b=b: eng.score([b], [(t, p_)])[0])
+        trees.append((toks, sh.parents))
+    tk, pr, off = pack_trees(trees)
+    ids = np.arange(B, dtype=np.int32)
+    acc = torch.zeros(B, dtype=torch.int32, device="cuda")
+
+    def reset():
+        eng.sync()
+        for b in range(B):
+            eng.truncate(b, int(lens[b]))
+
+    for _ in range(max(3, args.warmup)):
+        eng.verify_batch_device(ids, tk, pr, off, outputs=(acc, None, None, None))
+        reset()
+    a_len = eng.verify_batch(list(range(B)), trees)[0]
+    reset()
+    clk = ClockSampler(gpu_uuid(0))
+    ms = _timed(eng.stream, lambda: eng.verify_batch_device(ids, tk, pr, off, outputs=(acc, None, None, None)),
+                args.steps, reset)
+    clocks = clk.stop()
+    M = int(off[-1])
+    kv_tok = dims.n_layers * 2 * dims.kv_dim * 2
+    bytes_ = step_bytes(dims, 0, 0) + int(lens.sum() + M) * kv_tok
+    rk = sum(int(lens[b]) * 61 + 61 * 5 for b in range(B))  # prefix keys per node + ~ancestors
+    fl = flops_per_token(dims) * M + attn_flops(dims, rk, dims.n_layers)
+    tau = float(np.mean(a_len + 1))
+    print(json.dumps({"workload": "llama3.1-8b-shape bf16, batch 64, prefixes U[512,4096], own 60-draft trees,"
+                                  " planted p U[0.6,0.9]", "tokens_per_step": M, "ms_per_step": ms,
+                      "verify_steps_per_s": 1000.0 / ms, "accepted_tokens_per_s": float(np.sum(a_len + 1)) * 1000.0 / ms,
+                      "tau_mean": tau, "roofline": _roofline(bytes_, fl, ms), "plan": eng.info(B, 61, int(lens.max())),
+                      "clocks": clocks, "data": "synthetic"}))
+    eng.close()
+    return 0
+
+
+def run_sweep(args):
+    """Chain-vs-tree sweep at prefix 8192, batch 1, planted p = 0.85."""
+    import torch
+    from speculative_decoding_06_b200.engine import SpecEngine, pack_trees
+    dims = synth.LLAMA8B
+    P = 8192
+    w = synth.model_weights(dims, seed=0, device="cuda")
+    eng = SpecEngine(dims, w, max_batch=1, max_seq=P + 128, max_nodes=128)
+    pend = eng.prefill(0, synth.prefix_tokens(dims.vocab, P, seed=1))
+    shapes = [("chain5", synth.chain(5)), ("chain8", synth.chain(8))]
+    shapes += [("tree%d" % n, synth.tree_from_widths(synth.SWEEP_WIDTHS[n], stream=0)) for n in (16, 32, 60, 80)]
+    kv_tok = dims.n_layers * 2 * dims.kv_dim * 2
+    out = []
+    clk = ClockSampler(gpu_uuid(0))
+    for name, sh in shapes:
+        draws = synth.plant_draws(sh.n, dims.vocab, stream=0)
+        toks = synth.plant_tree(sh, pend, 0.85, draws, lambda t, p_: eng.score([0], [(t, p_)])[0])
+        tk, pr, off = pack_trees([(toks, sh.parents)])
+        ids = np.zeros(1, np.int32)
+
+        def reset():
+            eng.sync()
+            eng.truncate(0, P)
+
+        for _ in range(max(3, args.warmup)):
+            eng.verify_batch_device(ids, tk, pr, off)
+            reset()
+        a, _, _ = eng.verify(0, toks, sh.parents)
+        reset()
+        ms = _timed(eng.stream, lambda: eng.verify_batch_device(ids, tk, pr, off), args.steps, reset)
+        bytes_ = step_bytes(dims, P, sh.n)
+        fl = flops_per_token(dims) * sh.n + attn_flops(dims, P * sh.n, dims.n_layers)
+        out.append({"draft": name, "nodes": sh.n, "ms_per_step": ms, "tau": a + 1,
+                    "accepted_tokens_per_s": (a + 1) * 1000.0 / ms, "roofline_frac": _roofline(bytes_, fl, ms)["frac"]})
+    clocks = clk.stop()
+    print(json.dumps({"workload": "llama3.1-8b-shape bf16, batch 1, prefix 8192, chains 5/8 and trees 16/32/60/80"
+                                  " at depth 8, planted p=0.85", "results": out, "clocks": clocks, "data": "synthetic"}))
+    eng.close()
+    return 0
+
+
+def run_draft(args):
+    """Draft-head step: batch 16, 60-draft trees, draft prefixes of 2048 rows, N(0,1) features."""
+    import torch
+    from speculative_decoding_06_b200.engine import SpecEngine, pack_trees
+    dims = synth.LLAMA8B
+    B, P = 16, 2048
+    w = synth.model_weights(dims, seed=0, device="cuda")
+    dw = synth.draft_head_weights(dims, seed=6, device="cuda")
+    eng = SpecEngine(dims, w, max_batch=B, max_seq=P + 64, max_nodes=64, draft=dw)
+    rng = np.random.default_rng(5)
+    for b in range(B):
+        f = synth.draft_features(P, dims.hidden, seed=100 + b, device="cuda")
+        eng.draft_prefill(b, f, rng.integers(0, dims.vocab, size=P).astype(np.int32))
+    trees = []
+    for b in range(B):
+        sh = synth.tree_from_widths(synth.TREE60_WIDTHS, stream=b)
+        trees.append((rng.integers(0, dims.vocab, size=sh.n).astype(np.int32), sh.parents))
+    tk, pr, off = pack_trees(trees)
+    M = int(off[-1])
+    feats = synth.draft_features(M, dims.hidden, seed=5, device="cuda")
+    ids = np.arange(B, dtype=np.int32)
+    ti = torch.zeros(M, 10, dtype=torch.int32, device="cuda")
+    tv = torch.zeros(M, 10, dtype=torch.float32, device="cuda")
+    step = lambda: eng.draft_step_device(ids, feats, tk, pr, off, outputs=(ti, tv))
+    for _ in range(max(3, args.warmup)):
+        step()
+        eng.sync()
+    clk = ClockSampler(gpu_uuid(0))
+    ms = _timed(eng.stream, step, args.steps, lambda: None)
+    clocks = clk.stop()
+    d = dims
+    layer = d.q_dim * d.hidden + 2 * d.kv_dim * d.hidden + d.hidden * d.q_dim + 3 * d.ffn * d.hidden
+    params = 3 * d.hidden * d.hidden + 2 * d.hidden * d.hidden + layer + d.vocab * d.hidden
+    kv_tok = 2 * d.kv_dim * 2
+    bytes_ = 2 * params + B * (P + 61) * kv_tok + M * 3 * d.hidden * 2
+    fl = 2 * params * M + attn_flops(d, P * M, 1)
+    print(json.dumps({"workload": "EAGLE-3 draft head at 8B shape bf16: batch 16, 60-draft trees, draft prefix 2048,"
+                                  " N(0,1) low/mid/high features, fusion FC + input FC + one tree-masked decoder layer"
+                                  " + LM head + top-10", "tokens_per_step": M, "ms_per_step": ms,
+                      "draft_steps_per_s": 1000.0 / ms, "roofline": _roofline(bytes_, fl, ms), "clocks": clocks,
+                      "data": "synthetic"}))
+    eng.close()
+    return 0
+
+
 def main():
     ap = argparse.ArgumentParser()
     ap.add_argument("--gpus", type=int, default=1)
@@ -379,12 +556,19 @@ def main():
     ap.add_argument("--sample-layers", type=int, default=2)
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--layers", type=int, default=32, help="decoder layers (32 = the 8B shape; fewer only for profiling)")
+    ap.add_argument("--workload", default="verify", choices=["verify", "batch64", "sweep", "draft"],
+                    help="verify: the default line (batch 1, prefix 2048); the others measure the remaining"
+                         " configurations (one GPU, one JSON line each)")
     args = ap.parse_args()
     rank = int(os.environ.get("RANK", "0"))
     world = int(os.environ.get("WORLD_SIZE", "1"))
     local_rank = int(os.environ.get("LOCAL_RANK", "0"))
     if args.impl == "reference":
         return run_reference(args, rank, world)
+    if args.workload != "verify":
+        import torch
+        torch.cuda.set_device(local_rank)
+        return {"batch64": run_batch64, "sweep": run_sweep, "draft": run_draft}[args.workload](args)
     return run_ours(args, rank, world, local_rank)
 
 
