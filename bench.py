@@ -47,6 +47,23 @@ def workload_config(P=2048, layers=32):
             "parallelism": "replicas (one independent verifier per GPU)"}
 
 
+def measured_traffic(cls, bytes_per_launch):
+    """DRAM bytes per launch of kernel class `cls` from the committed ncu record, scaled from the captured
+    (smaller) launch to this workload's launch by algorithmic bytes; None when the kernel source changed
+    since the capture or there is no record."""
+    import hashlib
+    p = os.path.join(ROOT, "profiles", "traffic.json")
+    if not os.path.exists(p):
+        return None
+    rec = json.load(open(p)).get(cls)
+    if not rec:
+        return None
+    src = os.path.join(ROOT, rec["source"])
+    if not os.path.exists(src) or hashlib.sha256(open(src, "rb").read()).hexdigest()[:16] != rec["source_sha256_prefix"]:
+        return None
+    return bytes_per_launch * rec["dram_bytes_per_launch_small"] / rec["algorithmic_bytes_small"]
+
+
 def measured_peaks():
     p = os.path.join(ROOT, "MEASURED_PEAKS.json")
     if os.path.exists(p):
@@ -232,6 +249,21 @@ def run_reference(args, rank, world):
 # our arm
 # ---------------------------------------------------------------------------
 
+def max_over_ranks(value: float, dist=None, device=None) -> float:
+    """The largest `value` over all ranks (every rank calls it, in the same order)."""
+    if dist is None:
+        return float(value)
+    import torch
+    t = torch.tensor([float(value)], dtype=torch.float64, device=device)
+    dist.all_reduce(t, op=dist.ReduceOp.MAX)
+    return float(t.item())
+
+
+def job_throughput(world: int, steps: int, t_total_ms: float) -> float:
+    """Whole-job steps per second: every rank ran `steps` steps; the job took the slowest rank's time."""
+    return world * steps / (t_total_ms / 1000.0)
+
+
 def run_ours(args, rank, world, local_rank):
     import torch
     from speculative_decoding_06_b200.engine import SpecEngine, pack_trees
@@ -296,13 +328,9 @@ def run_ours(args, rank, world, local_rank):
     if dist:
         dist.barrier()
     clocks = clk.stop()
-    t_total = float(sum(times))
-    if dist:
-        tt = torch.tensor([t_total], device="cuda")
-        dist.all_reduce(tt, op=dist.ReduceOp.MAX)
-        t_total = float(tt.item())
+    t_total = max_over_ranks(float(sum(times)), dist, "cuda")
     ms = t_total / args.steps
-    value = world * args.steps / (t_total / 1000.0)
+    value = job_throughput(world, args.steps, t_total)
 
     # ---- end to end through the public API with host buffers (H2D + D2H inside)
     e2e_times = []
@@ -343,7 +371,9 @@ def run_ours(args, rank, world, local_rank):
         "config": workload_config(P, args.layers),
         "accepted_tokens_per_s": value * (a_len + 1), "tau": a_len + 1,
         "roofline": {"bound": "hbm", "kernel": dom, "achieved": achieved, "peak": hbm, "unit": "GB/s",
-                     "frac": achieved / hbm, "traffic": None, "peak_source": peak_kind,
+                     "frac": achieved / hbm, "traffic": measured_traffic(dom, cb[dom] / dom_n),
+                     "traffic_source": "profiles/traffic.json (ncu dram__bytes_read+write, scaled by algorithmic bytes)",
+                     "peak_source": peak_kind,
                      "bytes_per_launch": cb[dom] / dom_n, "launches_per_step": dom_n,
                      "ms_per_launch": dom_ms / dom_n},
         "step_roofline": {"bound": "hbm", "bytes_per_step": sb, "achieved": step_gbs, "peak": hbm, "unit": "GB/s",
