@@ -467,13 +467,13 @@ __global__ void __launch_bounds__(kThreads, 1) attn_tc_kernel(const __grid_const
       float4* po = reinterpret_cast<float4*>(a.part_o + slot * kRows * 128);
       if (ok)
         for (int rr = warp; rr < valid; rr += 4) __stcg(po + rr * 32 + lane, *stage_at(stg, rr, lane));
-      __threadfence();
       named_sync_rows();
       stamp(a.trace, 5);
       int* ctr = a.counters + 2 * grp;
       if (tid == 0) {
         bool met = false;
         if (!*abort_flag) {
+          __threadfence();  // the barrier orders every thread's partial stores before it
           atomicAdd(ctr, 1);
           met = spin_until_geq(ctr, nc_b, err);
         }
@@ -485,53 +485,52 @@ __global__ void __launch_bounds__(kThreads, 1) attn_tc_kernel(const __grid_const
         const int per = (valid + nc_b - 1) / nc_b;
         const int rb = blockIdx.x * per;
         const int R = max(0, min(valid, rb + per) - rb);
-        const float* lse0 = a.part_lse + (size_t)grp * a.n_chunks * kRows;
-        const float4* po0 = reinterpret_cast<const float4*>(a.part_o + (size_t)grp * a.n_chunks * kRows * 128);
-        // chunk weights 2^(lse_c - max) / sum per slice row, in shared memory [R][nc_b]
-        float* wsm = reinterpret_cast<float*>(smem + Smem::v);
-        for (int i = r; i < R * nc_b; i += 128) {
-          const int rr = i / nc_b, c = i - rr * nc_b;
-          wsm[i] = __ldcg(lse0 + c * kRows + rb + rr);
-        }
-        named_sync_rows();
-        if (r < R) {
-          float* wr = wsm + r * nc_b;
-          float mx = -INFINITY;
-          for (int c = 0; c < nc_b; ++c) mx = fmaxf(mx, wr[c]);
-          float sum = 0.f;
-          for (int c = 0; c < nc_b; ++c) {
-            const float w = fast_exp2(wr[c] - mx);  // 2^-inf = 0 for empty chunks
-            wr[c] = w;
-            sum += w;
-          }
-          const float wi = sum > 0.f ? 1.f / sum : 0.f;
-          for (int c = 0; c < nc_b; ++c) wr[c] *= wi;
-        }
-        named_sync_rows();
-        // warp per slice row, lane = 4 columns; all chunks' loads issued together
-        constexpr int kMaxMerge = 16;
-        for (int rr = warp; rr < R; rr += 4) {
-          const float* wr = wsm + rr * nc_b;
-          float4 acc = make_float4(0.f, 0.f, 0.f, 0.f);
-          for (int cb = 0; cb < nc_b; cb += kMaxMerge) {
-            float4 v[kMaxMerge];
+        const float* lse0 = a.part_lse + (size_t)grp * a.n_chunks * kRows + rb;
+        const float4* po0 = reinterpret_cast<const float4*>(a.part_o + (size_t)grp * a.n_chunks * kRows * 128) +
+                            (size_t)rb * 32 + lane;
+        // Two slice rows per warp and round; every chunk's log-sum-exp and
+        // partial of both rows in flight at once (chunks <= kAttnMaxChunks).
+        for (int r0 = warp; r0 < R; r0 += 8) {
+          const int rows2[2] = {r0, r0 + 4};
+          float lv[2][kAttnMaxChunks];
+          float4 pv[2][kAttnMaxChunks];
 #pragma unroll
-            for (int u = 0; u < kMaxMerge; ++u)
-              v[u] = (cb + u < nc_b) ? __ldcg(po0 + ((size_t)(cb + u) * kRows + rb + rr) * 32 + lane)
-                                     : make_float4(0.f, 0.f, 0.f, 0.f);
+          for (int h = 0; h < 2; ++h) {
+            const bool rok = rows2[h] < R;
 #pragma unroll
-            for (int u = 0; u < kMaxMerge; ++u) {
-              const float w = (cb + u < nc_b) ? wr[cb + u] : 0.f;
-              acc.x = fmaf(w, v[u].x, acc.x);
-              acc.y = fmaf(w, v[u].y, acc.y);
-              acc.z = fmaf(w, v[u].z, acc.z);
-              acc.w = fmaf(w, v[u].w, acc.w);
+            for (int c = 0; c < kAttnMaxChunks; ++c) {
+              const bool on = rok && c < nc_b;
+              lv[h][c] = on ? __ldcg(lse0 + (size_t)c * kRows + rows2[h]) : -INFINITY;
+              pv[h][c] = on ? __ldcg(po0 + ((size_t)c * kRows + rows2[h]) * 32) : make_float4(0.f, 0.f, 0.f, 0.f);
             }
           }
-          const int q2 = row0 + rb + rr;
-          const int nd = q2 / G;
-          const int col = (kvh * G + (q2 - nd * G)) * 128 + lane * 4;
-          split_store4(out, base + nd, ld, col, acc);
+#pragma unroll
+          for (int h = 0; h < 2; ++h) {
+            if (rows2[h] >= R) continue;
+            float mx = -INFINITY;
+#pragma unroll
+            for (int c = 0; c < kAttnMaxChunks; ++c) mx = fmaxf(mx, lv[h][c]);
+            float4 acc = make_float4(0.f, 0.f, 0.f, 0.f);
+            float wsum = 0.f;
+#pragma unroll
+            for (int c = 0; c < kAttnMaxChunks; ++c) {
+              const float w = fast_exp2(lv[h][c] - mx);  // 2^-inf = 0 for empty chunks and padding
+              wsum += w;
+              acc.x = fmaf(w, pv[h][c].x, acc.x);
+              acc.y = fmaf(w, pv[h][c].y, acc.y);
+              acc.z = fmaf(w, pv[h][c].z, acc.z);
+              acc.w = fmaf(w, pv[h][c].w, acc.w);
+            }
+            const float wi = wsum > 0.f ? 1.f / wsum : 0.f;
+            acc.x *= wi;
+            acc.y *= wi;
+            acc.z *= wi;
+            acc.w *= wi;
+            const int q2 = row0 + rb + rows2[h];
+            const int nd = q2 / G;
+            const int col = (kvh * G + (q2 - nd * G)) * 128 + lane * 4;
+            split_store4(out, base + nd, ld, col, acc);
+          }
         }
         named_sync_rows();
         stamp(a.trace, 7);

@@ -206,6 +206,7 @@ struct AttnTcMaps {
 constexpr int kAttnTcRows = 128;   // query rows per CTA
 constexpr int kAttnTcKeys = 128;   // keys per block; chunks are multiples of it
 constexpr int kAttnPartCtas = 256; // partial slots: chunked launches stay within this many CTAs
+constexpr int kAttnMaxChunks = 16; // key chunks per (sequence, kv head, row tile) at most
 cudaError_t launch_attention_tc(const AttnArgs& a, const AttnTcMaps& maps, cudaStream_t s, bool pdl);
 size_t attention_tc_smem_bytes();
 cudaError_t attention_tc_configure();

@@ -34,7 +34,7 @@ namespace {
 constexpr int kMaxNodesLimit = 128;  // ancestor bitmask is two 64-bit words
 constexpr int kMaxSplits = 16;
 constexpr int kGemmCounters = 8192;  // per-tile arrival counters of the split-K GEMMs
-constexpr int kMaxAttnChunks = 64;    // key chunks of one (sequence, kv head, row tile)
+constexpr int kMaxAttnChunks = kAttnMaxChunks;  // key chunks of one (sequence, kv head, row tile)
 constexpr int kDraftTopK = SPEC_DRAFT_TOPK;  // candidates per draft node
 constexpr int kCountersPerPhase = 2048; // two ints per split-K tile
 
