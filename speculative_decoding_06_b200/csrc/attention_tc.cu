@@ -40,7 +40,8 @@ namespace {
 
 constexpr int kRows = 128;                   // query rows per CTA (the MMA M)
 constexpr int kKeys = 128;                   // keys per block (S's N, P.V's K)
-constexpr int kThreads = 160;                // warps 0-3 rows, warp 4 issue
+constexpr int kThreads = 288;                // warps 0-7 rows (two per row), warp 8 issue
+constexpr int kCtrlWarp = 8;
 constexpr uint32_t kHalf = 128 * 128;        // [128 rows][64 fp16] swizzled: 16 KB
 constexpr uint32_t kTile = 2 * kHalf;        // 128 x 128 fp16: 32 KB
 
@@ -52,7 +53,8 @@ struct Smem {
   static constexpr uint32_t k = q + kTile;          // 2 stages
   static constexpr uint32_t v = k + 2 * kTile;      // 2 stages
   static constexpr uint32_t p = v + 2 * kTile;
-  static constexpr uint32_t bars = p + kTile;
+  static constexpr uint32_t xchg = p + kTile;        // row maxima [2][2][128] and sums [2][128]
+  static constexpr uint32_t bars = xchg + 6 * 128 * 4;
   static constexpr uint32_t misc = bars + kNumBars * 8;  // tmem slot, abort flag, merge flag
   static constexpr uint32_t end = misc + 16;
   static constexpr uint32_t dyn = end + 1024;            // 1024-byte alignment slack
@@ -89,7 +91,7 @@ __device__ __forceinline__ void stamp_at(uint64_t* trace, int k) {
   if (cta < (unsigned)kAttnPartCtas) trace[cta * kTraceMarks + k] = global_ns();
 }
 
-__device__ __forceinline__ void named_sync_rows() { asm volatile("bar.sync 1, 128;" ::: "memory"); }
+__device__ __forceinline__ void named_sync_rows() { asm volatile("bar.sync 1, 256;" ::: "memory"); }
 
 // keep uses of TMEM-loaded registers after the wait
 __device__ __forceinline__ void reg_fence32(uint32_t* r) {
@@ -179,7 +181,7 @@ __global__ void __launch_bounds__(kThreads, 1) attn_tc_kernel(const __grid_const
   };
   stamp(a.trace, 0);
 
-  if (warp == 4) {
+  if (warp == kCtrlWarp) {
     tmem_alloc(tmem_slot, kTmemCols);
     tmem_relinquish();
   }
@@ -189,9 +191,9 @@ __global__ void __launch_bounds__(kThreads, 1) attn_tc_kernel(const __grid_const
       mbar_init(&bar[B_KVFULL + s], 1);
       mbar_init(&bar[B_KVEMPTY + s], 1);
       mbar_init(&bar[B_SFULL + s], 1);
-      mbar_init(&bar[B_SFREE + s], 4);
+      mbar_init(&bar[B_SFREE + s], 8);
     }
-    mbar_init(&bar[B_PFULL], 4);
+    mbar_init(&bar[B_PFULL], 8);
     mbar_init(&bar[B_PEMPTY], 1);
     mbar_init(&bar[B_OFULL], 1);
     mbar_init(&bar[B_DRAIN], 1);
@@ -203,7 +205,7 @@ __global__ void __launch_bounds__(kThreads, 1) attn_tc_kernel(const __grid_const
   tc_fence_after();
   const uint32_t tmem = *tmem_slot;
 
-  if (warp == 4) {
+  if (warp == kCtrlWarp) {
     // ------------------------------------------------------------ TMA + MMA issue
     if (elect_one()) {
       tma_prefetch_desc(&maps.q);
@@ -304,53 +306,62 @@ __global__ void __launch_bounds__(kThreads, 1) attn_tc_kernel(const __grid_const
     __syncwarp();
   } else {
     // ------------------------------------------------------------ softmax rows
+    // Two threads per query row: warps w and w + 4 read the same TMEM lanes,
+    // w < 4 the columns 0-63 of every block (keys, then output dims), w >= 4
+    // the columns 64-127; they exchange row maxima and sums through shared
+    // memory.  Every thread passes every named barrier, also after a failed
+    // wait (its work is then skipped), so no barrier is left short.
     pdl_wait();
     pdl_launch_dependents();
-    const int r = warp * 32 + lane;
+    const int hf = warp >> 2;
+    const int r = (warp & 3) * 32 + lane;
     const int qr = row0 + r;
     const bool row_ok = qr < rows;
     const int node = row_ok ? qr / G : 0;
     const uint64_t anc0 = sv.row_anc[2 * (base + node)];
     const uint64_t anc1 = sv.row_anc[2 * (base + node) + 1];
-    const uint32_t tl = tmem + ((uint32_t)(warp * 32) << 16);  // this warp's TMEM lanes
-    const float sl2 = 1.4426950408889634f * 0.08838834764831845f;  // log2(e) / sqrt(128)
-    uint8_t* prow = smem + Smem::p + r * 128;
+    const uint32_t tl = tmem + ((uint32_t)((warp & 3) * 32) << 16);  // this warp's TMEM lanes
+    const float sl2 = 1.4426950408889634f * 0.08838834764831845f;      // log2(e) / sqrt(128)
+    uint8_t* prow = smem + Smem::p + hf * kHalf + r * 128;               // this thread's half of P's row
+    float* xmax = reinterpret_cast<float*>(smem + Smem::xchg);           // [parity][half][row]
+    float* xsum = xmax + 4 * 128;                                        // [half][row]
     float m = -INFINITY, l = 0.f;
     bool ok = true;
     for (int j = 0; j < nb; ++j) {
       const int st = j & 1;
       const int key0 = c0 + j * kKeys;
-      const uint32_t ts = tl + st * kKeys;
-      ok = mbar_wait(&bar[B_SFULL + st], (j >> 1) & 1, err, abort_flag);
-      if (!__all_sync(0xffffffffu, ok)) {
-        ok = false;
-        *abort_flag = 1;
-        break;
-      }
+      const uint32_t ts = tl + st * kKeys + hf * 64;
+      if (ok) ok = mbar_wait(&bar[B_SFULL + st], (j >> 1) & 1, err, abort_flag);
+      ok = __all_sync(0xffffffffu, ok);
       if (j == 0) stamp(a.trace, 3);
-      tc_fence_after();
       // visibility word of each 32-key piece (all ones when the whole block is
       // prefix keys of this chunk)
       const bool full = row_ok && key0 + kKeys <= min(P, c1);
       auto vis = [&](int i) {
-        return full ? 0xffffffffu : (row_ok ? visible_word(key0 + 32 * i, P, c1, anc0, anc1) : 0u);
+        const int piece = hf * 2 + i;
+        return full ? 0xffffffffu : (row_ok ? visible_word(key0 + 32 * piece, P, c1, anc0, anc1) : 0u);
       };
-      // pass 1: the block's row max (raw scores; the scale is positive)
+      // pass 1: this half's row max (raw scores; the scale is positive), then both halves'
       float mx4[4] = {-INFINITY, -INFINITY, -INFINITY, -INFINITY};
+      if (ok) {
+        tc_fence_after();
 #pragma unroll 1
-      for (int i = 0; i < 4; ++i) {
-        uint32_t x[32];
-        tmem_ld32_async(ts + 32 * i, x);
-        tmem_wait_ld();
-        reg_fence32(x);
-        const uint32_t w = vis(i);
+        for (int i = 0; i < 2; ++i) {
+          uint32_t x[32];
+          tmem_ld32_async(ts + 32 * i, x);
+          tmem_wait_ld();
+          reg_fence32(x);
+          const uint32_t w = vis(i);
 #pragma unroll
-        for (int c = 0; c < 32; ++c) {
-          const float v = ((w >> c) & 1u) ? __uint_as_float(x[c]) : -INFINITY;
-          mx4[c & 3] = fmaxf(mx4[c & 3], v);
+          for (int c = 0; c < 32; ++c) {
+            const float v = ((w >> c) & 1u) ? __uint_as_float(x[c]) : -INFINITY;
+            mx4[c & 3] = fmaxf(mx4[c & 3], v);
+          }
         }
       }
-      const float mblk = fmaxf(fmaxf(mx4[0], mx4[1]), fmaxf(mx4[2], mx4[3])) * sl2;
+      xmax[(st * 2 + hf) * 128 + r] = fmaxf(fmaxf(mx4[0], mx4[1]), fmaxf(mx4[2], mx4[3]));
+      named_sync_rows();
+      const float mblk = fmaxf(xmax[(st * 2) * 128 + r], xmax[(st * 2 + 1) * 128 + r]) * sl2;
       if (j == 0) stamp(a.trace, 8);
       float corr = 1.f;
       if (mblk > m + a.rescale_slack) {
@@ -358,87 +369,90 @@ __global__ void __launch_bounds__(kThreads, 1) attn_tc_kernel(const __grid_const
         m = mblk;
       }
       const float nm = (m == -INFINITY) ? 0.f : -m;
-      if (j >= 1) {
+      if (j >= 1 && ok) {
         // P.V of the previous block has finished: the P buffer is free and O is current
-        ok = mbar_wait(&bar[B_PEMPTY], (j - 1) & 1, err, abort_flag);
-        if (!__all_sync(0xffffffffu, ok)) {
-          ok = false;
-          *abort_flag = 1;
-          break;
-        }
-        tc_fence_after();
-        if (__any_sync(0xffffffffu, corr != 1.f)) {
+        ok = __all_sync(0xffffffffu, mbar_wait(&bar[B_PEMPTY], (j - 1) & 1, err, abort_flag));
+        if (ok) {
+          tc_fence_after();
+          if (__any_sync(0xffffffffu, corr != 1.f)) {
 #pragma unroll 1
-          for (int i = 0; i < 4; ++i) {
-            uint32_t o[32];
-            tmem_ld32_async(tl + kColO + 32 * i, o);
-            tmem_wait_ld();
-            reg_fence32(o);
+            for (int i = 0; i < 2; ++i) {
+              uint32_t o[32];
+              const uint32_t to_ = tl + kColO + hf * 64 + 32 * i;
+              tmem_ld32_async(to_, o);
+              tmem_wait_ld();
+              reg_fence32(o);
 #pragma unroll
-            for (int c = 0; c < 32; ++c) o[c] = __float_as_uint(__uint_as_float(o[c]) * corr);
-            tmem_st32_async(tl + kColO + 32 * i, o);
+              for (int c = 0; c < 32; ++c) o[c] = __float_as_uint(__uint_as_float(o[c]) * corr);
+              tmem_st32_async(to_, o);
+            }
+            tmem_wait_st();
           }
-          tmem_wait_st();
         }
       }
-      // pass 2: P = 2^(s - m) in fp16 into the K-major, 128-byte-swizzled A
-      // operand (16-byte chunk c of a 128-byte row lands at chunk c ^ (row & 7))
+      // pass 2: P = 2^(s - m) in fp16 into this half of the K-major,
+      // 128-byte-swizzled A operand (16-byte chunk c of a row lands at c ^ (row & 7))
       float ls4[4] = {0.f, 0.f, 0.f, 0.f};
+      if (ok) {
 #pragma unroll 1
-      for (int i = 0; i < 4; ++i) {
-        uint32_t x[32];
-        tmem_ld32_async(ts + 32 * i, x);
-        tmem_wait_ld();
-        reg_fence32(x);
-        const uint32_t w = vis(i);
-        uint32_t pk[16];
+        for (int i = 0; i < 2; ++i) {
+          uint32_t x[32];
+          tmem_ld32_async(ts + 32 * i, x);
+          tmem_wait_ld();
+          reg_fence32(x);
+          const uint32_t w = vis(i);
+          uint32_t pk[16];
 #pragma unroll
-        for (int c = 0; c < 16; ++c) {
-          const float s0 = ((w >> (2 * c)) & 1u) ? __uint_as_float(x[2 * c]) : -INFINITY;
-          const float s1 = ((w >> (2 * c + 1)) & 1u) ? __uint_as_float(x[2 * c + 1]) : -INFINITY;
-          const float p0 = fast_exp2(fmaf(s0, sl2, nm));
-          const float p1 = fast_exp2(fmaf(s1, sl2, nm));
-          ls4[c & 3] += p0 + p1;
-          const __half2 h2 = __floats2half2_rn(p0, p1);
-          pk[c] = *reinterpret_cast<const uint32_t*>(&h2);
-        }
-        uint8_t* dst = prow + (i >> 1) * kHalf;
+          for (int c = 0; c < 16; ++c) {
+            const float s0 = ((w >> (2 * c)) & 1u) ? __uint_as_float(x[2 * c]) : -INFINITY;
+            const float s1 = ((w >> (2 * c + 1)) & 1u) ? __uint_as_float(x[2 * c + 1]) : -INFINITY;
+            const float p0 = fast_exp2(fmaf(s0, sl2, nm));
+            const float p1 = fast_exp2(fmaf(s1, sl2, nm));
+            ls4[c & 3] += p0 + p1;
+            const __half2 h2 = __floats2half2_rn(p0, p1);
+            pk[c] = *reinterpret_cast<const uint32_t*>(&h2);
+          }
 #pragma unroll
-        for (int q4 = 0; q4 < 4; ++q4) {
-          const int chunk = (i & 1) * 4 + q4;
-          *reinterpret_cast<uint4*>(dst + ((chunk ^ (r & 7)) << 4)) =
-              make_uint4(pk[4 * q4], pk[4 * q4 + 1], pk[4 * q4 + 2], pk[4 * q4 + 3]);
+          for (int q4 = 0; q4 < 4; ++q4) {
+            const int chunk = i * 4 + q4;
+            *reinterpret_cast<uint4*>(prow + ((chunk ^ (r & 7)) << 4)) =
+                make_uint4(pk[4 * q4], pk[4 * q4 + 1], pk[4 * q4 + 2], pk[4 * q4 + 3]);
+          }
         }
-      }
-      if (j == 0) stamp(a.trace, 9);
-      tc_fence_before();
-      fence_proxy_async_smem();
-      __syncwarp();
-      if (lane == 0) {
-        mbar_arrive(&bar[B_SFREE + st]);
-        mbar_arrive(&bar[B_PFULL]);
+        if (j == 0) stamp(a.trace, 9);
+        tc_fence_before();
+        fence_proxy_async_smem();
+        __syncwarp();
+        if (lane == 0) {
+          mbar_arrive(&bar[B_SFREE + st]);
+          mbar_arrive(&bar[B_PFULL]);
+        }
       }
       l = l * corr + ((ls4[0] + ls4[1]) + (ls4[2] + ls4[3]));
     }
+    if (!ok) *abort_flag = 1;
     // ---- normalised output of this chunk, staged in shared memory (the K/V
     // ring is idle once the last P.V has completed)
     if (ok) ok = mbar_wait(&bar[B_OFULL], 0, err, abort_flag);
     ok = __all_sync(0xffffffffu, ok);
     stamp(a.trace, 4);
-    const bool any = l > 0.f;
-    const float inv = any ? 1.f / l : 0.f;
+    xsum[hf * 128 + r] = l;
+    named_sync_rows();
+    const float lt = xsum[r] + xsum[128 + r];
+    const bool any = lt > 0.f;
+    const float inv = any ? 1.f / lt : 0.f;
     uint8_t* stg = smem + Smem::k;  // 128 rows x 512 B
     if (ok) {
       tc_fence_after();
 #pragma unroll 1
-      for (int i = 0; i < 4; ++i) {
+      for (int i = 0; i < 2; ++i) {
         uint32_t o[32];
-        tmem_ld32_async(tl + kColO + 32 * i, o);
+        tmem_ld32_async(tl + kColO + hf * 64 + 32 * i, o);
         tmem_wait_ld();
         reg_fence32(o);
 #pragma unroll
         for (int q4 = 0; q4 < 8; ++q4)
-          *stage_at(stg, r, i * 8 + q4) =
+          *stage_at(stg, r, (hf * 2 + i) * 8 + q4) =
               make_float4(__uint_as_float(o[4 * q4]) * inv, __uint_as_float(o[4 * q4 + 1]) * inv,
                           __uint_as_float(o[4 * q4 + 2]) * inv, __uint_as_float(o[4 * q4 + 3]) * inv);
       }
@@ -446,7 +460,7 @@ __global__ void __launch_bounds__(kThreads, 1) attn_tc_kernel(const __grid_const
     const int grp = (b * Hkv + kvh) * gridDim.y + blockIdx.y;
     const size_t slot = (size_t)grp * a.n_chunks + blockIdx.x;
     float* part_lse = a.part_lse + slot * kRows;
-    if (nc_b > 1 && ok) part_lse[r] = any ? m + __log2f(l) : -INFINITY;
+    if (nc_b > 1 && ok && hf == 0) part_lse[r] = any ? m + __log2f(lt) : -INFINITY;
     named_sync_rows();
     __nv_bfloat16* out = reinterpret_cast<__nv_bfloat16*>(a.out);
     const int ld = a.Hq * 128;
@@ -454,7 +468,7 @@ __global__ void __launch_bounds__(kThreads, 1) attn_tc_kernel(const __grid_const
     if (nc_b == 1) {
       // one chunk: each warp writes whole rows, lane = 4 columns, as split bf16
       if (ok) {
-        for (int rr = warp; rr < valid; rr += 4) {
+        for (int rr = warp; rr < valid; rr += 8) {
           const float4 v = *stage_at(stg, rr, lane);
           const int q2 = row0 + rr;
           const int nd = q2 / G;
@@ -466,7 +480,7 @@ __global__ void __launch_bounds__(kThreads, 1) attn_tc_kernel(const __grid_const
       // partial rows, coalesced: lane = 4 columns of one row
       float4* po = reinterpret_cast<float4*>(a.part_o + slot * kRows * 128);
       if (ok)
-        for (int rr = warp; rr < valid; rr += 4) __stcg(po + rr * 32 + lane, *stage_at(stg, rr, lane));
+        for (int rr = warp; rr < valid; rr += 8) __stcg(po + rr * 32 + lane, *stage_at(stg, rr, lane));
       named_sync_rows();
       stamp(a.trace, 5);
       int* ctr = a.counters + 2 * grp;
@@ -488,49 +502,41 @@ __global__ void __launch_bounds__(kThreads, 1) attn_tc_kernel(const __grid_const
         const float* lse0 = a.part_lse + (size_t)grp * a.n_chunks * kRows + rb;
         const float4* po0 = reinterpret_cast<const float4*>(a.part_o + (size_t)grp * a.n_chunks * kRows * 128) +
                             (size_t)rb * 32 + lane;
-        // Two slice rows per warp and round; every chunk's log-sum-exp and
-        // partial of both rows in flight at once (chunks <= kAttnMaxChunks).
-        for (int r0 = warp; r0 < R; r0 += 8) {
-          const int rows2[2] = {r0, r0 + 4};
-          float lv[2][kAttnMaxChunks];
-          float4 pv[2][kAttnMaxChunks];
+        // One slice row per warp and round (8 warps: 16 rows in two rounds);
+        // every chunk's log-sum-exp and partial in flight at once
+        // (chunks <= kAttnMaxChunks).
+        for (int rr = warp; rr < R; rr += 8) {
+          float lv[kAttnMaxChunks];
+          float4 pv[kAttnMaxChunks];
 #pragma unroll
-          for (int h = 0; h < 2; ++h) {
-            const bool rok = rows2[h] < R;
-#pragma unroll
-            for (int c = 0; c < kAttnMaxChunks; ++c) {
-              const bool on = rok && c < nc_b;
-              lv[h][c] = on ? __ldcg(lse0 + (size_t)c * kRows + rows2[h]) : -INFINITY;
-              pv[h][c] = on ? __ldcg(po0 + ((size_t)c * kRows + rows2[h]) * 32) : make_float4(0.f, 0.f, 0.f, 0.f);
-            }
+          for (int c = 0; c < kAttnMaxChunks; ++c) {
+            const bool on = c < nc_b;
+            lv[c] = on ? __ldcg(lse0 + (size_t)c * kRows + rr) : -INFINITY;
+            pv[c] = on ? __ldcg(po0 + ((size_t)c * kRows + rr) * 32) : make_float4(0.f, 0.f, 0.f, 0.f);
           }
+          float mx = -INFINITY;
 #pragma unroll
-          for (int h = 0; h < 2; ++h) {
-            if (rows2[h] >= R) continue;
-            float mx = -INFINITY;
+          for (int c = 0; c < kAttnMaxChunks; ++c) mx = fmaxf(mx, lv[c]);
+          float4 acc = make_float4(0.f, 0.f, 0.f, 0.f);
+          float wsum = 0.f;
 #pragma unroll
-            for (int c = 0; c < kAttnMaxChunks; ++c) mx = fmaxf(mx, lv[h][c]);
-            float4 acc = make_float4(0.f, 0.f, 0.f, 0.f);
-            float wsum = 0.f;
-#pragma unroll
-            for (int c = 0; c < kAttnMaxChunks; ++c) {
-              const float w = fast_exp2(lv[h][c] - mx);  // 2^-inf = 0 for empty chunks and padding
-              wsum += w;
-              acc.x = fmaf(w, pv[h][c].x, acc.x);
-              acc.y = fmaf(w, pv[h][c].y, acc.y);
-              acc.z = fmaf(w, pv[h][c].z, acc.z);
-              acc.w = fmaf(w, pv[h][c].w, acc.w);
-            }
-            const float wi = wsum > 0.f ? 1.f / wsum : 0.f;
-            acc.x *= wi;
-            acc.y *= wi;
-            acc.z *= wi;
-            acc.w *= wi;
-            const int q2 = row0 + rb + rows2[h];
-            const int nd = q2 / G;
-            const int col = (kvh * G + (q2 - nd * G)) * 128 + lane * 4;
-            split_store4(out, base + nd, ld, col, acc);
+          for (int c = 0; c < kAttnMaxChunks; ++c) {
+            const float w = fast_exp2(lv[c] - mx);  // 2^-inf = 0 for empty chunks and padding
+            wsum += w;
+            acc.x = fmaf(w, pv[c].x, acc.x);
+            acc.y = fmaf(w, pv[c].y, acc.y);
+            acc.z = fmaf(w, pv[c].z, acc.z);
+            acc.w = fmaf(w, pv[c].w, acc.w);
           }
+          const float wi = wsum > 0.f ? 1.f / wsum : 0.f;
+          acc.x *= wi;
+          acc.y *= wi;
+          acc.z *= wi;
+          acc.w *= wi;
+          const int q2 = row0 + rb + rr;
+          const int nd = q2 / G;
+          const int col = (kvh * G + (q2 - nd * G)) * 128 + lane * 4;
+          split_store4(out, base + nd, ld, col, acc);
         }
         named_sync_rows();
         stamp(a.trace, 7);
@@ -544,7 +550,7 @@ __global__ void __launch_bounds__(kThreads, 1) attn_tc_kernel(const __grid_const
   }
   tc_fence_before();
   __syncthreads();
-  if (warp == 4) {
+  if (warp == kCtrlWarp) {
     tc_fence_after();
     tmem_dealloc(tmem, kTmemCols);
   }
