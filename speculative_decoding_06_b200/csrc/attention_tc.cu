@@ -54,7 +54,8 @@ struct Smem {
   static constexpr uint32_t v = k + 2 * kTile;      // 2 stages
   static constexpr uint32_t p = v + 2 * kTile;
   static constexpr uint32_t xchg = p + kTile;        // row maxima [2][2][128] and sums [2][128]
-  static constexpr uint32_t bars = xchg + 6 * 128 * 4;
+  static constexpr uint32_t lse = xchg + 6 * 128 * 4; // this chunk's log2-sum-exp per row (cluster merge)
+  static constexpr uint32_t bars = lse + 128 * 4;
   static constexpr uint32_t misc = bars + kNumBars * 8;  // tmem slot, abort flag, merge flag
   static constexpr uint32_t end = misc + 16;
   static constexpr uint32_t dyn = end + 1024;            // 1024-byte alignment slack
@@ -166,14 +167,17 @@ __global__ void __launch_bounds__(kThreads, 1) attn_tc_kernel(const __grid_const
   const int P = sv.P_step[b];
   const int Lk = P + n_b;
   const int c0 = blockIdx.x * a.chunk;
-  if (row0 >= rows || c0 >= Lk) {  // nothing here: no partial, no arrival
+  // (cluster merge: a chunk CTA beyond this sequence's keys stays in its
+  // cluster with an empty partial; the whole cluster shares b and row0)
+  const bool idle = c0 >= Lk;
+  if (row0 >= rows || (idle && !a.cluster_merge)) {  // nothing here: no partial, no arrival
     pdl_wait();
     pdl_launch_dependents();
     return;
   }
-  const int c1 = min(c0 + a.chunk, Lk);
+  const int c1 = idle ? c0 : min(c0 + a.chunk, Lk);
   const int nc_b = (Lk + a.chunk - 1) / a.chunk;  // chunk CTAs of this sequence
-  const int nb = (c1 - c0 + kKeys - 1) / kKeys;
+  const int nb = (c1 - c0 + kKeys - 1) / kKeys;   // 0 when idle
   const int seq = sv.seq_ids[b];
   uint32_t* err = sv.err;
   auto stamp = [&](uint64_t* trace, int k) {
@@ -207,7 +211,10 @@ __global__ void __launch_bounds__(kThreads, 1) attn_tc_kernel(const __grid_const
 
   if (warp == kCtrlWarp) {
     // ------------------------------------------------------------ TMA + MMA issue
-    if (elect_one()) {
+    if (nb == 0) {
+      pdl_wait();
+      pdl_launch_dependents();
+    } else if (elect_one()) {
       tma_prefetch_desc(&maps.q);
       tma_prefetch_desc(&maps.kv);
       // cache rows: [layer][K/V][max_batch][Hkv][max_seq]
@@ -433,7 +440,7 @@ __global__ void __launch_bounds__(kThreads, 1) attn_tc_kernel(const __grid_const
     if (!ok) *abort_flag = 1;
     // ---- normalised output of this chunk, staged in shared memory (the K/V
     // ring is idle once the last P.V has completed)
-    if (ok) ok = mbar_wait(&bar[B_OFULL], 0, err, abort_flag);
+    if (ok && nb > 0) ok = mbar_wait(&bar[B_OFULL], 0, err, abort_flag);  // (an idle CTA issued no MMA)
     ok = __all_sync(0xffffffffu, ok);
     stamp(a.trace, 4);
     xsum[hf * 128 + r] = l;
@@ -442,7 +449,7 @@ __global__ void __launch_bounds__(kThreads, 1) attn_tc_kernel(const __grid_const
     const bool any = lt > 0.f;
     const float inv = any ? 1.f / lt : 0.f;
     uint8_t* stg = smem + Smem::k;  // 128 rows x 512 B
-    if (ok) {
+    if (ok && nb > 0) {
       tc_fence_after();
 #pragma unroll 1
       for (int i = 0; i < 2; ++i) {
@@ -459,15 +466,19 @@ __global__ void __launch_bounds__(kThreads, 1) attn_tc_kernel(const __grid_const
     }
     const int grp = (b * Hkv + kvh) * gridDim.y + blockIdx.y;
     const size_t slot = (size_t)grp * a.n_chunks + blockIdx.x;
-    float* part_lse = a.part_lse + slot * kRows;
-    if (nc_b > 1 && ok && hf == 0) part_lse[r] = any ? m + __log2f(lt) : -INFINITY;
+    const float my_lse = (ok && any && nb > 0) ? m + __log2f(lt) : -INFINITY;
+    if (a.cluster_merge) {
+      if (hf == 0) reinterpret_cast<float*>(smem + Smem::lse)[r] = my_lse;
+    } else if (nc_b > 1 && ok && hf == 0) {
+      a.part_lse[slot * kRows + r] = my_lse;
+    }
     named_sync_rows();
     __nv_bfloat16* out = reinterpret_cast<__nv_bfloat16*>(a.out);
     const int ld = a.Hq * 128;
     const int valid = min(kRows, rows - row0);
     if (nc_b == 1) {
       // one chunk: each warp writes whole rows, lane = 4 columns, as split bf16
-      if (ok) {
+      if (ok && nb > 0) {
         for (int rr = warp; rr < valid; rr += 8) {
           const float4 v = *stage_at(stg, rr, lane);
           const int q2 = row0 + rr;
@@ -476,7 +487,7 @@ __global__ void __launch_bounds__(kThreads, 1) attn_tc_kernel(const __grid_const
           split_store4(out, base + nd, ld, col, v);
         }
       }
-    } else {
+    } else if (!a.cluster_merge) {
       // partial rows, coalesced: lane = 4 columns of one row
       float4* po = reinterpret_cast<float4*>(a.part_o + slot * kRows * 128);
       if (ok)
@@ -548,6 +559,66 @@ __global__ void __launch_bounds__(kThreads, 1) attn_tc_kernel(const __grid_const
       }
     }
   }
+  if (a.cluster_merge) {
+    // every chunk CTA of the cluster has staged its normalised output and
+    // log2-sum-exps in its own shared memory; each merges a slice of the rows
+    // by reading its peers' (distributed shared memory), then the cluster
+    // meets again so that no CTA leaves while a peer still reads it
+    cluster_sync_all();
+    if (warp < 8 && nc_b > 1) {
+      const int valid = min(kRows, rows - row0);
+      const int per = (valid + nc_b - 1) / nc_b;
+      const int rb = blockIdx.x * per;
+      const int R = max(0, min(valid, rb + per) - rb);
+      __nv_bfloat16* out = reinterpret_cast<__nv_bfloat16*>(a.out);
+      const int ld = a.Hq * 128;
+      const uint32_t lse_base = smem_u32(smem + Smem::lse);
+      const uint32_t stg_base = smem_u32(smem + Smem::k);
+      for (int rr = warp; rr < R; rr += 8) {
+        const int row = rb + rr;
+        const uint32_t soff = (uint32_t)(reinterpret_cast<uint8_t*>(stage_at(smem + Smem::k, row, lane)) -
+                                         (smem + Smem::k));
+        float lv[kAttnMaxChunks];
+        float4 pv[kAttnMaxChunks];
+#pragma unroll
+        for (int c = 0; c < kAttnMaxChunks; ++c) {
+          if (c < nc_b) {
+            lv[c] = dsmem_ld_f32(map_peer(lse_base + 4 * row, c));
+            pv[c] = dsmem_ld_f4(map_peer(stg_base + soff, c));
+          } else {
+            lv[c] = -INFINITY;
+            pv[c] = make_float4(0.f, 0.f, 0.f, 0.f);
+          }
+        }
+        float mx = -INFINITY;
+#pragma unroll
+        for (int c = 0; c < kAttnMaxChunks; ++c) mx = fmaxf(mx, lv[c]);
+        float4 acc = make_float4(0.f, 0.f, 0.f, 0.f);
+        float wsum = 0.f;
+#pragma unroll
+        for (int c = 0; c < kAttnMaxChunks; ++c) {
+          if (lv[c] == -INFINITY) continue;  // empty chunk: its staged values are not written
+          const float w = fast_exp2(lv[c] - mx);
+          wsum += w;
+          acc.x = fmaf(w, pv[c].x, acc.x);
+          acc.y = fmaf(w, pv[c].y, acc.y);
+          acc.z = fmaf(w, pv[c].z, acc.z);
+          acc.w = fmaf(w, pv[c].w, acc.w);
+        }
+        const float wi = wsum > 0.f ? 1.f / wsum : 0.f;
+        acc.x *= wi;
+        acc.y *= wi;
+        acc.z *= wi;
+        acc.w *= wi;
+        const int q2 = row0 + row;
+        const int nd = q2 / G;
+        const int col = (kvh * G + (q2 - nd * G)) * 128 + lane * 4;
+        split_store4(out, base + nd, ld, col, acc);
+      }
+    }
+    stamp(a.trace, 7);
+    cluster_sync_all();
+  }
   tc_fence_before();
   __syncthreads();
   if (warp == kCtrlWarp) {
@@ -558,25 +629,59 @@ __global__ void __launch_bounds__(kThreads, 1) attn_tc_kernel(const __grid_const
 
 size_t attention_tc_smem_bytes() { return Smem::dyn; }
 
-cudaError_t attention_tc_configure() {
+cudaError_t attention_tc_configure(int* max_clusters) {
   cudaError_t e = cudaFuncSetAttribute(attn_tc_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
                                        (int)attention_tc_smem_bytes());
   if (e != cudaSuccess) return e;
-  return cudaFuncSetAttribute(attn_tc_kernel, cudaFuncAttributePreferredSharedMemoryCarveout,
-                              (int)cudaSharedmemCarveoutMaxShared);
+  e = cudaFuncSetAttribute(attn_tc_kernel, cudaFuncAttributePreferredSharedMemoryCarveout,
+                           (int)cudaSharedmemCarveoutMaxShared);
+  if (e != cudaSuccess) return e;
+  // how many clusters of cs chunk CTAs the GPU holds at once (0: none)
+  const bool nonportable =
+      cudaFuncSetAttribute(attn_tc_kernel, cudaFuncAttributeNonPortableClusterSizeAllowed, 1) == cudaSuccess;
+  for (int cs = 0; cs <= kAttnMaxChunks; ++cs) {
+    max_clusters[cs] = 0;
+    if (cs < 2 || (cs > 8 && !nonportable)) continue;
+    cudaLaunchConfig_t cfg = {};
+    cfg.gridDim = dim3(cs, 1, 1);
+    cfg.blockDim = dim3(kThreads);
+    cfg.dynamicSmemBytes = attention_tc_smem_bytes();
+    cudaLaunchAttribute at[1];
+    at[0].id = cudaLaunchAttributeClusterDimension;
+    at[0].val.clusterDim.x = cs;
+    at[0].val.clusterDim.y = 1;
+    at[0].val.clusterDim.z = 1;
+    cfg.attrs = at;
+    cfg.numAttrs = 1;
+    int n = 0;
+    if (cudaOccupancyMaxActiveClusters(&n, (void*)attn_tc_kernel, &cfg) == cudaSuccess) max_clusters[cs] = n;
+  }
+  (void)cudaGetLastError();  // a rejected size is not an error of the library
+  return cudaSuccess;
 }
 
 cudaError_t launch_attention_tc(const AttnArgs& a, const AttnTcMaps& maps, cudaStream_t s, bool pdl) {
-  cudaLaunchAttribute attr[1];
-  attr[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
-  attr[0].val.programmaticStreamSerializationAllowed = 1;
+  cudaLaunchAttribute attr[2];
+  int na = 0;
+  if (pdl) {
+    attr[na].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+    attr[na].val.programmaticStreamSerializationAllowed = 1;
+    ++na;
+  }
+  if (a.cluster_merge) {  // the chunk CTAs of a row tile form one cluster
+    attr[na].id = cudaLaunchAttributeClusterDimension;
+    attr[na].val.clusterDim.x = a.n_chunks;
+    attr[na].val.clusterDim.y = 1;
+    attr[na].val.clusterDim.z = 1;
+    ++na;
+  }
   cudaLaunchConfig_t cfg = {};
   cfg.gridDim = dim3(a.n_chunks, (a.max_rows + kRows - 1) / kRows, a.sv.B * a.kv.Hkv);
   cfg.blockDim = dim3(kThreads);
   cfg.dynamicSmemBytes = attention_tc_smem_bytes();
   cfg.stream = s;
   cfg.attrs = attr;
-  cfg.numAttrs = pdl ? 1 : 0;
+  cfg.numAttrs = na;
   return cudaLaunchKernelEx(&cfg, attn_tc_kernel, maps, a);
 }
 

@@ -192,6 +192,7 @@ struct AttnArgs {
   int max_rows;             // max over batch of n_b * (Hq/Hkv)
   int q_rows;               // bf16 path: q is [Hkv][q_rows][hd], row node * G + g
   float rescale_slack;      // bf16 path: the running max moves only when a block's max exceeds it by this (log2 units)
+  int cluster_merge;        // bf16 path: the n_chunks chunk CTAs of a row tile form a cluster and merge through DSMEM
   int* counters;            // bf16 path: [groups][2] chunk arrivals / departures, zero between launches
   uint64_t* trace;          // optional [256 CTAs][16] %globaltimer marks (attention_tc.cu)
 };
@@ -209,7 +210,8 @@ constexpr int kAttnPartCtas = 256; // partial slots: chunked launches stay withi
 constexpr int kAttnMaxChunks = 16; // key chunks per (sequence, kv head, row tile) at most
 cudaError_t launch_attention_tc(const AttnArgs& a, const AttnTcMaps& maps, cudaStream_t s, bool pdl);
 size_t attention_tc_smem_bytes();
-cudaError_t attention_tc_configure();
+// also max_clusters[cs] (cs = 0 .. kAttnMaxChunks): clusters of cs chunk CTAs the GPU holds at once
+cudaError_t attention_tc_configure(int* max_clusters);
 
 // LM head reductions
 cudaError_t launch_top2_reduce(int M, int tiles, const Top2* part, int top_ld, int32_t* argmax, float* top1,

@@ -216,6 +216,7 @@ struct GemmPlan {
 
 struct StepPlan {
   int B, M, max_n, max_lk, n_chunks, chunk, max_rows;
+  int cluster_merge = 0;  // attention chunks merge through DSMEM (all groups' clusters co-resident)
   int grid_all;  // co-resident CTAs of the multi-phase GEMM launches
   GemmPlan qkv, o, gu, down, lm;
 };
@@ -265,6 +266,8 @@ struct spec_handle {
   int max_chunks = kMaxAttnChunks;  // attention key-chunk cap
   int resident_cap = 0;   // 0: as many CTAs per SM as fit
   float rescale_slack = 8.f;  // attention: running-max slack in log2 units (p <= 2^slack)
+  int attn_clusters[kAttnMaxChunks + 1] = {};  // co-resident clusters of n chunk CTAs
+  bool attn_dsmem = true;     // merge chunk partials through distributed shared memory when they fit a cluster
   // L2 prefetch of weights ahead of the GEMM that streams them
   uint64_t* trace = nullptr;  // optional GEMM timeline of one layer's launch
   size_t trace_bytes = 0;
@@ -370,6 +373,10 @@ StepPlan make_plan(const spec_handle* h, int B, int M, int max_n, int max_lk) {
     if (2 * groups <= cap) nc = std::max(1, std::min({blocks, cap / groups, h->max_chunks}));
     s.chunk = ceil_div(blocks, nc) * kAttnTcKeys;
     s.n_chunks = ceil_div(max_lk, s.chunk);
+    // the chunk CTAs of a group merge through distributed shared memory when
+    // every group's cluster fits on the GPU at once (else through global memory)
+    s.cluster_merge = (h->attn_dsmem && s.n_chunks > 1 && s.n_chunks <= kAttnMaxChunks &&
+                       h->attn_clusters[s.n_chunks] >= groups) ? 1 : 0;
   } else {
     s.chunk = max_lk;
     s.n_chunks = 1;
@@ -614,6 +621,7 @@ cudaError_t enqueue_step(spec_handle* h, const StepPlan& sp, int mode, bool dbg)
   aa.counters = h->W<int>(L.attn_ctr);
   aa.q_rows = L.Mpad * (c.n_q_heads / c.n_kv_heads);
   aa.rescale_slack = h->rescale_slack;
+  aa.cluster_merge = sp.cluster_merge;
 
   const PhaseBuilder pb(h, sp, sv);
   if (dt == 1) {
@@ -774,6 +782,7 @@ cudaError_t enqueue_draft(spec_handle* h, const StepPlan& sp, bool kv_only, bool
   aa.counters = h->W<int>(L.attn_ctr);
   aa.q_rows = L.Mpad * (c.n_q_heads / c.n_kv_heads);
   aa.rescale_slack = h->rescale_slack;
+  aa.cluster_merge = sp.cluster_merge;
   LK(SPEC_PROF_ATTENTION, 1, launch_attention_tc(aa, h->attn_maps, st, pdl));
   float* logits = h->W<float>(L.dlogits);
   m.n_phases = 4;
@@ -1125,6 +1134,7 @@ int spec_init(const spec_config* cfg, const spec_weights* w, void* kv_cache, siz
     if (const char* q = strstr(t, "splits=")) if (sscanf(q + 7, "%d", &v) == 1 && v >= 1 && v <= kMaxSplits) h->max_splits = v;
     if (const char* q = strstr(t, "chunks=")) if (sscanf(q + 7, "%d", &v) == 1 && v >= 1 && v <= kMaxAttnChunks) h->max_chunks = v;
     if (const char* q = strstr(t, "pdl=")) if (sscanf(q + 4, "%d", &v) == 1) h->use_pdl = v != 0;
+    if (const char* q = strstr(t, "dsmem=")) if (sscanf(q + 6, "%d", &v) == 1) h->attn_dsmem = v != 0;
     if (const char* q = strstr(t, "per_sm=")) if (sscanf(q + 7, "%d", &v) == 1 && v >= 0) h->resident_cap = v;
     float fv = 0.f;
     if (const char* q = strstr(t, "rescale=")) if (sscanf(q + 8, "%f", &fv) == 1 && fv >= 0.f && fv <= 15.f) h->rescale_slack = fv;
@@ -1154,7 +1164,7 @@ int spec_init(const spec_config* cfg, const spec_weights* w, void* kv_cache, siz
     return bail(SPEC_ERR_CUDA, "smem attribute");
   if (c.dtype == SPEC_DTYPE_BF16) {
     if (!get_encode_fn()) return bail(SPEC_ERR_CUDA, "cuTensorMapEncodeTiled unavailable");
-    if (attention_tc_configure() != cudaSuccess) return bail(SPEC_ERR_CUDA, "smem attribute");
+    if (attention_tc_configure(h->attn_clusters) != cudaSuccess) return bail(SPEC_ERR_CUDA, "smem attribute");
     const int qd = c.n_q_heads * c.head_dim, kvd = c.n_kv_heads * c.head_dim;
     {
       // q as [Hkv * q_rows][128] and the cache as [layers * 2 * batch * Hkv * max_seq][128], fp16;
@@ -1474,12 +1484,15 @@ int spec_info(spec_handle* h, int B, int n_nodes, int prefix, char* buf, size_t 
              p.kbps, p.grid);
     return std::string(t);
   };
-  std::string s = "sms " + std::to_string(h->sm_count) + "; resident/SM [bn64|bn128][qkv,swiglu,argmax,resid] = ";
+  std::string s = "sms " + std::to_string(h->sm_count) + "; attention clusters held [size:count]";
+  for (int cs = 2; cs <= kAttnMaxChunks; ++cs) s += " " + std::to_string(cs) + ":" + std::to_string(h->attn_clusters[cs]);
+  s += "; resident/SM [bn64|bn128][qkv,swiglu,argmax,resid] = ";
   for (int i = 0; i < 2; ++i)
     for (int e = 0; e < 4; ++e)
       s += std::to_string(h->resident[i][e]) + "(" + std::to_string(h->occ_api[i][e]) + ")" + (e < 3 ? "," : "|");
   s += "; qkv " + g(sp.qkv) + "; o " + g(sp.o) + "; gate_up " + g(sp.gu) + "; down " + g(sp.down) + "; lm " +
-       g(sp.lm) + "; attention chunks " + std::to_string(sp.n_chunks) + " x " + std::to_string(sp.chunk);
+       g(sp.lm) + "; attention chunks " + std::to_string(sp.n_chunks) + " x " + std::to_string(sp.chunk) +
+        (sp.cluster_merge ? " (cluster merge)" : " (global merge)");
   snprintf(buf, n, "%s", s.c_str());
   return SPEC_OK;
 }

@@ -221,10 +221,13 @@ def _engine_tuned(dims, tune, **kw):
             os.environ["SPEC_TUNE"] = old
 
 
-@pytest.mark.parametrize("tune", ["chunks=2", "chunks=1", "chunks=2,rescale=0", "chunks=1,rescale=0"])
+@pytest.mark.parametrize("tune", ["chunks=2", "chunks=1", "chunks=2,rescale=0", "chunks=1,rescale=0", "chunks=4,dsmem=0",
+                                  "chunks=4"])
 def test_bf16_multiblock_attention(tune):
-    """Prefix 700 + 61 nodes = 6 key blocks per (sequence, kv head) in 2 chunks or 1; slack 0 makes every
-    growth of the running max rescale the accumulated output."""
+    """Prefix 700 + 61 nodes = 6 key blocks per (sequence, kv head) in 4, 2 or 1 chunks; slack 0 makes every
+    growth of the running max rescale the accumulated output; chunks merge through distributed shared memory
+    (a cluster of chunk CTAs, idle ones included for the shorter sequence) or, with dsmem=0, through global
+    memory."""
     eng, om = _engine_tuned(synth.MINI_BF16, tune, max_batch=2, max_seq=1024, max_nodes=64)
     seqs, trees = [], []
     for i, P in enumerate((700, 530)):
