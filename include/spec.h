@@ -247,13 +247,13 @@ SPEC_API int spec_io_bytes(spec_handle* h, size_t* h2d, size_t* d2h);
  * tokens, written to buf (n bytes, NUL-terminated). */
 SPEC_API int spec_info(spec_handle* h, int B, int n_nodes, int prefix, char* buf, size_t n);
 /* Optional timeline of decoder layer `layer` (bf16 models), in %globaltimer
- * stamps (uint64 ns); NULL turns it off.  device_buf holds 2 * SMs * 64 + 4096
+ * stamps (uint64 ns); NULL turns it off.  device_buf holds 2 * SMs * 64 + 8192
  * entries: first the layer's GEMM launch, [2 * SMs CTAs][4 phases][16] (0-7:
  * producer starts the phase, may load its activations, has issued its last
  * load; epilogue starts the phase, first accumulator complete, split-K
  * rendezvous passed, units done, phase counted at the grid barrier; 8-11 for the
  * first unit: partial stored, split partials summed, finishing stores done,
- * unit done), then its attention launch, [256 CTAs][16] (start, Q landed,
+ * unit done), then its attention launch and the next layer's, [2][256 CTAs][16] (start, Q landed,
  * first K/V block landed, first scores ready, output accumulated, partial
  * written, chunk rendezvous passed, merge done, first block's max found, first
  * block's P written, first scores issued, last P seen by the issuer).  Entries

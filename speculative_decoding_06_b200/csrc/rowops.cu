@@ -362,28 +362,51 @@ cudaError_t launch_gemm_simt_f32(const float* A, int lda, const float* W, int K,
 // LM-head reductions
 // ---------------------------------------------------------------------------
 // one warp per token: merge the per-tile (best, index, runner-up) in tile order
-__global__ void top2_reduce_kernel(int M, int tiles, const Top2* __restrict__ part, int top_ld,
-                                   int32_t* __restrict__ argmax, float* __restrict__ top1, float* __restrict__ top2) {
+// One CTA per token: every thread merges a strided set of the vocabulary
+// tiles' (best, index, runner-up) with its loads issued together, then the
+// warps and the CTA merge (lowest index on equal values).
+__global__ void __launch_bounds__(256) top2_reduce_kernel(int M, int tiles, const Top2* __restrict__ part,
+                                                         int top_ld, int32_t* __restrict__ argmax,
+                                                         float* __restrict__ top1, float* __restrict__ top2) {
+  __shared__ Top2 wbest[8];
   pdl_wait();
   pdl_launch_dependents();
-  const int t = blockIdx.x * (blockDim.x >> 5) + (threadIdx.x >> 5);
-  const int lane = threadIdx.x & 31;
+  const int t = blockIdx.x;
   if (t >= M) return;
+  constexpr int kU = 4;
   Top2 best;
   best.v1 = -INFINITY; best.i1 = 0x7fffffff; best.v2 = -INFINITY;
-  for (int i = lane; i < tiles; i += 32) best = top2_merge(best, part[(size_t)i * top_ld + t]);
+  for (int i0 = threadIdx.x; i0 < tiles; i0 += kU * blockDim.x) {
+    Top2 x[kU];
+#pragma unroll
+    for (int u = 0; u < kU; ++u) {
+      const int i = i0 + u * blockDim.x;
+      if (i < tiles) {
+        x[u] = part[(size_t)i * top_ld + t];
+      } else {
+        x[u].v1 = -INFINITY; x[u].i1 = 0x7fffffff; x[u].v2 = -INFINITY;
+      }
+    }
+#pragma unroll
+    for (int u = 0; u < kU; ++u) best = top2_merge(best, x[u]);
+  }
   best = warp_top2(best);
-  if (lane == 0) {
-    argmax[t] = best.i1;
-    top1[t] = best.v1;
-    top2[t] = best.v2;
+  const int warp = threadIdx.x >> 5;
+  if ((threadIdx.x & 31) == 0) wbest[warp] = best;
+  __syncthreads();
+  if (threadIdx.x == 0) {
+    Top2 r = wbest[0];
+    for (int w = 1; w < (int)(blockDim.x >> 5); ++w) r = top2_merge(r, wbest[w]);
+    argmax[t] = r.i1;
+    top1[t] = r.v1;
+    top2[t] = r.v2;
   }
 }
 
 cudaError_t launch_top2_reduce(int M, int tiles, const Top2* part, int top_ld, int32_t* argmax, float* top1,
                                float* top2, cudaStream_t s, bool pdl) {
   cudaLaunchAttribute attr[1];
-  cudaLaunchConfig_t cfg = make_cfg(dim3((M + 7) / 8), dim3(256), 0, s, pdl, attr);
+  cudaLaunchConfig_t cfg = make_cfg(dim3(M), dim3(256), 0, s, pdl, attr);
   return cudaLaunchKernelEx(&cfg, top2_reduce_kernel, M, tiles, part, top_ld, argmax, top1, top2);
 }
 

@@ -642,7 +642,11 @@ cudaError_t enqueue_step(spec_handle* h, const StepPlan& sp, int mode, bool dbg)
     if (dt == 1) {
       // attention of layer l (its QKV ran in the previous launch), then one
       // launch: O, gate/up, down, and the next layer's QKV or the LM head
-      aa.trace = (h->trace && l == h->trace_layer) ? h->trace + (size_t)2 * h->sm_count * kMaxGemmPhases * kGemmTraceMarks : nullptr;
+      // the traced layer's attention and the next layer's (which follows the traced GEMM launch)
+      aa.trace = (h->trace && (l == h->trace_layer || l == h->trace_layer + 1))
+                     ? h->trace + (size_t)2 * h->sm_count * kMaxGemmPhases * kGemmTraceMarks +
+                           (size_t)(l - h->trace_layer) * kAttnPartCtas * 16
+                     : nullptr;
       LK(SPEC_PROF_ATTENTION, 1, launch_attention_tc(aa, h->attn_maps, st, pdl));
       GemmMultiLaunch m{};
       m.bn = sp.qkv.bn;
@@ -1458,9 +1462,9 @@ int spec_profile_read(spec_handle* h, double* ms, int64_t* launches) {
 
 int spec_step_launches(spec_handle* h) { return h ? h->launches : 0; }
 
-// GEMM marks [2 * SMs][phases][16], then attention marks [kAttnPartCtas][16]
+// GEMM marks [2 * SMs][phases][16], then attention marks [2 layers][kAttnPartCtas][16]
 static size_t trace_words(const spec_handle* h) {
-  return (size_t)2 * h->sm_count * kMaxGemmPhases * kGemmTraceMarks + (size_t)kAttnPartCtas * 16;
+  return (size_t)2 * h->sm_count * kMaxGemmPhases * kGemmTraceMarks + (size_t)2 * kAttnPartCtas * 16;
 }
 
 int spec_set_trace(spec_handle* h, uint64_t* device_buf, size_t bytes, int layer) {
