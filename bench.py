@@ -483,6 +483,11 @@ def run_batch64(args):
     ms = _timed(eng.stream, lambda: eng.verify_batch_device(ids, tk, pr, off, outputs=(acc, None, None, None)),
                 args.steps, reset)
     clocks = clk.stop()
+    eng.profile(True)
+    eng.verify_batch_device(ids, tk, pr, off)
+    reset()
+    prof = {k: round(v[0], 3) for k, v in eng.profile_read().items() if v[1]}
+    eng.profile(False)
     M = int(off[-1])
     kv_tok = dims.n_layers * 2 * dims.kv_dim * 2
     bytes_ = step_bytes(dims, 0, 0) + int(lens.sum() + M) * kv_tok
@@ -492,7 +497,8 @@ def run_batch64(args):
     print(json.dumps({"workload": "llama3.1-8b-shape bf16, batch 64, prefixes U[512,4096], own 60-draft trees,"
                                   " planted p U[0.6,0.9]", "tokens_per_step": M, "ms_per_step": ms,
                       "verify_steps_per_s": 1000.0 / ms, "accepted_tokens_per_s": float(np.sum(a_len + 1)) * 1000.0 / ms,
-                      "tau_mean": tau, "roofline": _roofline(bytes_, fl, ms), "plan": eng.info(B, 61, int(lens.max())),
+                      "tau_mean": tau, "roofline": _roofline(bytes_, fl, ms), "kernel_ms_per_step": prof,
+                      "plan": eng.info(B, 61, int(lens.max())),
                       "clocks": clocks, "data": "synthetic"}))
     eng.close()
     return 0
@@ -569,6 +575,11 @@ def run_draft(args):
     clk = ClockSampler(gpu_uuid(0))
     ms = _timed(eng.stream, step, args.steps, lambda: None)
     clocks = clk.stop()
+    eng.profile(True)
+    step()
+    eng.sync()
+    prof = {k: round(v[0], 3) for k, v in eng.profile_read().items() if v[1]}
+    eng.profile(False)
     d = dims
     layer = d.q_dim * d.hidden + 2 * d.kv_dim * d.hidden + d.hidden * d.q_dim + 3 * d.ffn * d.hidden
     params = 3 * d.hidden * d.hidden + 2 * d.hidden * d.hidden + layer + d.vocab * d.hidden
@@ -578,7 +589,8 @@ def run_draft(args):
     print(json.dumps({"workload": "EAGLE-3 draft head at 8B shape bf16: batch 16, 60-draft trees, draft prefix 2048,"
                                   " N(0,1) low/mid/high features, fusion FC + input FC + one tree-masked decoder layer"
                                   " + LM head + top-10", "tokens_per_step": M, "ms_per_step": ms,
-                      "draft_steps_per_s": 1000.0 / ms, "roofline": _roofline(bytes_, fl, ms), "clocks": clocks,
+                      "draft_steps_per_s": 1000.0 / ms, "roofline": _roofline(bytes_, fl, ms),
+                      "kernel_ms_per_step": prof, "plan": eng.info(B, 61, P), "clocks": clocks,
                       "data": "synthetic"}))
     eng.close()
     return 0
