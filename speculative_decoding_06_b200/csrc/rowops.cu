@@ -469,28 +469,38 @@ cudaError_t launch_split_rows(const __nv_bfloat16* src, int rows, int cols, __nv
 // ---------------------------------------------------------------------------
 // top-k per row (the draft head's candidate list)
 // ---------------------------------------------------------------------------
-// One CTA per row.  Each thread keeps a sorted list of its best k values over
-// a strided slice of the row; the warps then merge by k rounds of a warp-wide
-// best-of, and warp 0 merges the eight warp lists the same way.  Order: value
+// One CTA per row.  Each thread keeps a sorted list of its best K values (in
+// registers: K is a compile-time constant) over a strided slice of the row;
+// each warp then merges its lanes' lists by K rounds of a warp-wide best-of,
+// and warp 0 merges the eight warp lists the same way.  Order: value
 // descending, index ascending.
 namespace {
 __device__ __forceinline__ bool topk_better(float a, int ai, float b, int bi) {
   return a > b || (a == b && ai < bi);
 }
-// k rounds: each round the best head among the lanes' lists is taken
-__device__ __forceinline__ void warp_merge_topk(const float* lv, const int* li, int k, float* out_v, int* out_i) {
+// K rounds: each round the best head among the lanes' lists is taken
+template <int K>
+__device__ __forceinline__ void warp_merge_topk(const float (&lv)[K], const int (&li)[K], float* out_v, int* out_i) {
   const int lane = threadIdx.x & 31;
   int head = 0;
-  for (int r = 0; r < k; ++r) {
-    float v = head < k ? lv[head] : -INFINITY;
-    int i = head < k ? li[head] : 0x7fffffff;
+#pragma unroll
+  for (int r = 0; r < K; ++r) {
+    // this lane's current head, selected without dynamic register indexing
+    float v = -INFINITY;
+    int i = 0x7fffffff;
+#pragma unroll
+    for (int j = 0; j < K; ++j)
+      if (j == head) {
+        v = lv[j];
+        i = li[j];
+      }
     int src = lane;
 #pragma unroll
     for (int o = 16; o > 0; o >>= 1) {
       const float v2 = __shfl_xor_sync(0xffffffffu, v, o);
       const int i2 = __shfl_xor_sync(0xffffffffu, i, o);
       const int s2 = __shfl_xor_sync(0xffffffffu, src, o);
-      if (topk_better(v2, i2, v, i)) {
+      if (topk_better(v2, i2, v, i) || (v2 == v && i2 == i && s2 < src)) {
         v = v2;
         i = i2;
         src = s2;
@@ -505,30 +515,75 @@ __device__ __forceinline__ void warp_merge_topk(const float* lv, const int* li, 
 }
 }  // namespace
 
-__global__ void __launch_bounds__(256) topk_rows_kernel(int V, const float* __restrict__ logits, size_t ld, int k,
+template <int K>
+__global__ void __launch_bounds__(256) topk_rows_kernel(int V, const float* __restrict__ logits, size_t ld,
                                                        int32_t* __restrict__ out_i, float* __restrict__ out_v) {
-  __shared__ float wv[8][kTopKMax];
-  __shared__ int wi[8][kTopKMax];
+  __shared__ float wv[8][K];
+  __shared__ int wi[8][K];
   pdl_wait();
   pdl_launch_dependents();
   const int r = blockIdx.x;
   const float* row = logits + (size_t)r * ld;
-  float lv[kTopKMax];
-  int li[kTopKMax];
+  float lv[K];
+  int li[K];
 #pragma unroll
-  for (int j = 0; j < kTopKMax; ++j) {
+  for (int j = 0; j < K; ++j) {
     lv[j] = -INFINITY;
     li[j] = 0x7fffffff;
   }
-  for (int c = threadIdx.x; c < V; c += blockDim.x) {
-    const float x = __ldcs(row + c);
-    if (!topk_better(x, c, lv[k - 1], li[k - 1])) continue;
-    // insert, keeping lv[0..k) sorted
+  // Pass 1: a lower bound for the row's K-th value.  Each thread takes the
+  // maximum of 64 of the row's values (disjoint sets, strided); the K-th
+  // largest of these 256 maxima is reached by K distinct entries, so the row's
+  // K-th value is at least that.
+  const int warp = threadIdx.x >> 5;
+  const int lane = threadIdx.x & 31;
+  float thr = -INFINITY;
+  {
+    float m = -INFINITY;
+    int mi = 0x7fffffff;
+#pragma unroll 8
+    for (int j = 0; j < 64; ++j) {
+      const int c = threadIdx.x + j * blockDim.x;
+      if (c < V) {
+        const float x = __ldcs(row + c);
+        if (topk_better(x, c, m, mi)) {
+          m = x;
+          mi = c;
+        }
+      }
+    }
+    float sv[K];
+    int si[K];
+#pragma unroll
+    for (int j = 0; j < K; ++j) {
+      sv[j] = j == 0 ? m : -INFINITY;
+      si[j] = j == 0 ? mi : 0x7fffffff;
+    }
+    warp_merge_topk<K>(sv, si, wv[warp], wi[warp]);
+    __syncthreads();
+    if (warp == 0) {
+      float mv[K];
+      int mj[K];
+#pragma unroll
+      for (int j = 0; j < K; ++j) {
+        mv[j] = lane < 8 ? wv[lane][j] : -INFINITY;
+        mj[j] = lane < 8 ? wi[lane][j] : 0x7fffffff;
+      }
+      __syncwarp();
+      warp_merge_topk<K>(mv, mj, wv[0], wi[0]);
+    }
+    __syncthreads();
+    thr = wv[0][K - 1];  // -inf when the row has fewer than K entries
+    __syncthreads();
+  }
+  // Pass 2: the whole row; only values >= thr are offered to the sorted list
+  auto offer = [&](float x, int c) {
+    if (!topk_better(x, c, lv[K - 1], li[K - 1])) return;
     float cv = x;
     int ci = c;
 #pragma unroll
-    for (int j = 0; j < kTopKMax; ++j) {
-      if (j < k && topk_better(cv, ci, lv[j], li[j])) {
+    for (int j = 0; j < K; ++j) {
+      if (topk_better(cv, ci, lv[j], li[j])) {
         const float tv = lv[j];
         const int ti = li[j];
         lv[j] = cv;
@@ -537,24 +592,49 @@ __global__ void __launch_bounds__(256) topk_rows_kernel(int V, const float* __re
         ci = ti;
       }
     }
+  };
+  const bool vec = (ld % 4 == 0) && ((reinterpret_cast<uintptr_t>(logits) & 15u) == 0);
+  const int V4 = vec ? V / 4 : 0;
+  const float4* row4 = reinterpret_cast<const float4*>(row);
+  for (int g0 = threadIdx.x; g0 < V4; g0 += 2 * blockDim.x) {
+    float4 x[2];
+#pragma unroll
+    for (int u = 0; u < 2; ++u) {
+      const int g = g0 + u * blockDim.x;
+      x[u] = g < V4 ? __ldcs(row4 + g) : make_float4(-INFINITY, -INFINITY, -INFINITY, -INFINITY);
+    }
+#pragma unroll
+    for (int u = 0; u < 2; ++u) {
+      const float m = fmaxf(fmaxf(x[u].x, x[u].y), fmaxf(x[u].z, x[u].w));
+      if (m >= thr) {
+        const int c = 4 * (g0 + u * blockDim.x);
+        if (x[u].x >= thr) offer(x[u].x, c);
+        if (x[u].y >= thr) offer(x[u].y, c + 1);
+        if (x[u].z >= thr) offer(x[u].z, c + 2);
+        if (x[u].w >= thr) offer(x[u].w, c + 3);
+      }
+    }
   }
-  const int warp = threadIdx.x >> 5;
-  warp_merge_topk(lv, li, k, wv[warp], wi[warp]);
+  for (int c = 4 * V4 + threadIdx.x; c < V; c += blockDim.x) {
+    const float x = __ldcs(row + c);
+    if (x >= thr) offer(x, c);
+  }
+  warp_merge_topk<K>(lv, li, wv[warp], wi[warp]);
   __syncthreads();
   if (warp == 0) {
-    const int lane = threadIdx.x & 31;
-    float mv[kTopKMax];
-    int mi[kTopKMax];
+    float mv[K];
+    int mi[K];
 #pragma unroll
-    for (int j = 0; j < kTopKMax; ++j) {
-      mv[j] = (lane < 8 && j < k) ? wv[lane][j] : -INFINITY;
-      mi[j] = (lane < 8 && j < k) ? wi[lane][j] : 0x7fffffff;
+    for (int j = 0; j < K; ++j) {
+      mv[j] = lane < 8 ? wv[lane][j] : -INFINITY;
+      mi[j] = lane < 8 ? wi[lane][j] : 0x7fffffff;
     }
-    warp_merge_topk(mv, mi, k, wv[0], wi[0]);  // lane 0 writes after reading its own list
     __syncwarp();
-    if (lane < k) {
-      out_v[(size_t)r * k + lane] = wv[0][lane];
-      out_i[(size_t)r * k + lane] = wi[0][lane];
+    warp_merge_topk<K>(mv, mi, wv[0], wi[0]);
+    __syncwarp();
+    if (lane < K) {
+      out_v[(size_t)r * K + lane] = wv[0][lane];
+      out_i[(size_t)r * K + lane] = wi[0][lane];
     }
   }
 }
@@ -564,7 +644,13 @@ cudaError_t launch_topk_rows(int M, int V, const float* logits, size_t ld, int k
   if (k < 1 || k > kTopKMax || k > V) return cudaErrorInvalidValue;
   cudaLaunchAttribute attr[1];
   cudaLaunchConfig_t cfg = make_cfg(dim3(M), dim3(256), 0, s, pdl, attr);
-  return cudaLaunchKernelEx(&cfg, topk_rows_kernel, V, logits, ld, k, idx, val);
+  switch (k) {  // the list length is a compile-time constant of the kernel
+    case 10: return cudaLaunchKernelEx(&cfg, topk_rows_kernel<10>, V, logits, ld, idx, val);
+    case 16: return cudaLaunchKernelEx(&cfg, topk_rows_kernel<16>, V, logits, ld, idx, val);
+    case 8: return cudaLaunchKernelEx(&cfg, topk_rows_kernel<8>, V, logits, ld, idx, val);
+    case 4: return cudaLaunchKernelEx(&cfg, topk_rows_kernel<4>, V, logits, ld, idx, val);
+    default: return cudaErrorInvalidValue;
+  }
 }
 
 }  // namespace spec
