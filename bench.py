@@ -430,9 +430,11 @@ def _timed(stream, fn, steps, reset):
     for _ in range(steps):
         e0 = torch.cuda.Event(enable_timing=True)
         e1 = torch.cuda.Event(enable_timing=True)
+        torch.cuda.nvtx.range_push("timed_step")
         e0.record(stream)
         fn()
         e1.record(stream)
+        torch.cuda.nvtx.range_pop()
         e1.synchronize()
         times.append(e0.elapsed_time(e1))
         reset()
