@@ -126,6 +126,39 @@ def test_draft_step_topk(which):
     assert [eng.draft_len(i) for i in range(3)] == Ps
 
 
+def test_draft_step_many_token_tiles():
+    """Eight 61-node trees (488 rows): four 128-token tiles in every GEMM of the draft step."""
+    from speculative_decoding_06_b200.engine import SpecEngine
+    _, oh, d = _pair("small")
+    eng = SpecEngine(d, synth.model_weights(d, seed=0, device="cuda"), max_batch=8, max_seq=512, max_nodes=64,
+                     draft=synth.draft_head_weights(d, seed=6, device="cuda"))
+    try:
+        B = 8
+        seqs = []
+        for i in range(B):
+            P = 90 + 17 * i
+            f = _feats(P, d.hidden, seed=60 + i)
+            toks = _tokens(P, d.vocab, 60 + i)
+            eng.draft_prefill(i, f, toks)
+            seqs.append(oh.prefill(_host(f.cpu()), toks))
+        shapes = [synth.tree_from_widths(synth.TREE60_WIDTHS, stream=i) for i in range(B)]
+        trees = [(_tokens(sh.n, d.vocab, 80 + i), sh.parents) for i, sh in enumerate(shapes)]
+        M = sum(sh.n for sh in shapes)
+        assert "bn128 tiles" in eng.info(B, 61, 300) and "x4 " in eng.info(B, 61, 300)
+        fn = _feats(M, d.hidden, seed=70)
+        gi, gv, off = eng.draft_step(list(range(B)), fn, trees, flags=2)
+        logits = eng.debug_logits(M)
+        fh = _host(fn.cpu())
+        for i, (seq, (toks, par)) in enumerate(zip(seqs, trees)):
+            lo, hi = int(off[i]), int(off[i + 1])
+            ref = oh.step_logits(seq, fh[lo:hi], toks, par)
+            err = float(np.max(np.abs(logits[lo:hi] - ref)))
+            assert err <= TOL["bf16"], "sequence %d: max |logit error| %.3g" % (i, err)
+            _check_topk(gi[lo:hi], gv[lo:hi], ref, err)
+    finally:
+        eng.close()
+
+
 def test_draft_errors():
     eng, oh, d = _pair("small")
     f = _feats(8, d.hidden, seed=1)
