@@ -289,6 +289,21 @@ SPEC_API int spec_lm_head_argmax_noalloc(const float* hidden, const void* final_
                                          int d, int V, float eps, int32_t* argmax, float* top1, float* top2,
                                          void* cuda_stream);
 
+/* Self-test of the bounded waits.  Every wait inside the library's kernels
+ * (split-K and attention-chunk rendezvous, grid barriers between GEMM phases,
+ * pipeline mbarriers) gives up after a time limit, records a timeout in the
+ * step's error word and returns; the step then fails with SPEC_ERR_TIMEOUT and
+ * the CUDA context stays usable.  This call runs the same two wait primitives
+ * on one GPU thread against a counter that nothing increments and an mbarrier
+ * that nothing arrives on, each limited to limit_us microseconds (1 .. 10^6).
+ * device_scratch: 16 bytes of device memory, 4-byte aligned, owned by the
+ * caller (overwritten).  On return *expired holds how many of the two waits
+ * gave up (2 when the mechanism works).  Returns SPEC_ERR_TIMEOUT when the
+ * device reported the timeout (the expected outcome), SPEC_OK if it did not,
+ * SPEC_ERR_ARG / SPEC_ERR_CUDA on bad arguments or a CUDA error.  Runs on the
+ * legacy default stream and synchronises the device. */
+SPEC_API int spec_wait_selftest(void* device_scratch, uint32_t limit_us, int32_t* expired);
+
 /* Message of the last error on this handle ("" if none). */
 SPEC_API const char* spec_last_error(spec_handle* h);
 /* Free host-side state (graphs, descriptors); never frees borrowed buffers. */

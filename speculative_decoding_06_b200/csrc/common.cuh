@@ -94,13 +94,13 @@ __device__ __forceinline__ bool mbar_try_wait(uint64_t* bar, uint32_t parity) {
 // Wait for the phase with the given parity to complete; false (and an error
 // bit) if it has not completed within SPEC_WAIT_NS, or if `abort` is raised.
 __device__ __forceinline__ bool mbar_wait(uint64_t* bar, uint32_t parity, uint32_t* err,
-                                          volatile int* abort) {
+                                          volatile int* abort, uint64_t limit_ns = SPEC_WAIT_NS) {
   if (mbar_try_wait(bar, parity)) return true;
   const uint64_t t0 = global_ns();
   while (true) {
     if (mbar_try_wait(bar, parity)) return true;
     if (abort && *abort) return false;
-    if (global_ns() - t0 > SPEC_WAIT_NS) {
+    if (global_ns() - t0 > limit_ns) {
       set_error(err, SPEC_DEVERR_TIMEOUT);
       if (abort) *abort = 1;
       return false;
@@ -190,13 +190,14 @@ __device__ __forceinline__ bool mbar_wait_cluster(uint64_t* bar, uint32_t parity
 
 // Bounded wait until *p >= target (gpu-scope acquire load).  Used only between
 // CTAs of one grid that is sized to be co-resident in full.
-__device__ __forceinline__ bool spin_until_geq(const int* p, int target, uint32_t* err) {
+__device__ __forceinline__ bool spin_until_geq(const int* p, int target, uint32_t* err,
+                                               uint64_t limit_ns = SPEC_WAIT_NS) {
   const uint64_t t0 = global_ns();
   while (true) {
     int v;
     asm volatile("ld.acquire.gpu.global.b32 %0, [%1];" : "=r"(v) : "l"(p) : "memory");
     if (v >= target) return true;
-    if (global_ns() - t0 > SPEC_WAIT_NS) {
+    if (global_ns() - t0 > limit_ns) {
       set_error(err, SPEC_DEVERR_TIMEOUT);
       return false;
     }

@@ -94,6 +94,7 @@ _SIGNATURES = {
     "spec_draft_prefill": (ctypes.c_int, [_h, ctypes.c_int, _vp, _i32p, ctypes.c_int]),
     "spec_draft_step": (ctypes.c_int, [_h, ctypes.c_int, _i32p, _vp, _i32p, _i32p, _i32p, _vp, _vp, ctypes.c_int]),
     "spec_draft_len": (ctypes.c_int, [_h, ctypes.c_int, _i32p]),
+    "spec_wait_selftest": (ctypes.c_int, [_vp, ctypes.c_uint32, _i32p]),
     "spec_last_error": (ctypes.c_char_p, [_h]),
     "spec_free": (None, [_h]),
 }
