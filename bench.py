@@ -105,20 +105,42 @@ def class_bytes(d, M, P, n):
 
 
 class ClockSampler:
-    """nvidia-smi clock / throttle sampling while the timed region runs."""
+    """nvidia-smi clock / throttle sampling around the timed region.
 
-    FIELDS = ("index,clocks.sm,clocks.max.sm,power.draw,clocks_event_reasons.active,"
+    Start it before the warm-up (nvidia-smi needs a moment to come up), mark the
+    timed region with begin() / end(); stop() keeps the samples whose timestamp
+    falls inside the region (50 ms apart), or the nearest one when the region
+    is shorter than the sampling interval."""
+
+    FIELDS = ("timestamp,index,clocks.sm,clocks.max.sm,power.draw,clocks_event_reasons.active,"
               "clocks_event_reasons.hw_slowdown,clocks_event_reasons.hw_thermal_slowdown,"
               "clocks_event_reasons.sw_thermal_slowdown,clocks_event_reasons.sw_power_cap")
 
-    def __init__(self, gpu_id: str):
+    def __init__(self, gpu_id: str, interval_ms: int = 50):
         self.f = tempfile.NamedTemporaryFile("w+", suffix=".csv", delete=False)
+        self.t0 = self.t1 = None
         try:
             self.p = subprocess.Popen(["nvidia-smi", "-i", gpu_id, "--query-gpu=" + self.FIELDS,
-                                       "--format=csv,noheader,nounits", "-lms", "200"],
+                                       "--format=csv,noheader,nounits", "-lms", str(interval_ms)],
                                       stdout=self.f, stderr=subprocess.DEVNULL)
         except Exception:
             self.p = None
+
+    def begin(self):
+        self.t0 = time.time()
+
+    def end(self):
+        self.t1 = time.time()
+
+    @staticmethod
+    def _when(stamp):
+        import datetime
+        for fmt in ("%Y/%m/%d %H:%M:%S.%f", "%Y/%m/%d %H:%M:%S"):
+            try:
+                return datetime.datetime.strptime(stamp, fmt).timestamp()
+            except ValueError:
+                pass
+        return None
 
     def stop(self):
         if self.p is None:
@@ -132,17 +154,28 @@ class ClockSampler:
         rows = []
         for ln in open(self.f.name):
             parts = [x.strip() for x in ln.split(",")]
-            if len(parts) >= 9:
-                rows.append(parts)
+            if len(parts) >= 10 and parts[2].replace(".", "").isdigit():
+                rows.append((self._when(parts[0]), parts))
         os.unlink(self.f.name)
         if not rows:
             return None
-        sm = [float(r[1]) for r in rows if r[1].replace(".", "").isdigit()]
-        mx = [float(r[2]) for r in rows if r[2].replace(".", "").isdigit()]
+        t0 = self.t0 if self.t0 is not None else -float("inf")
+        t1 = self.t1 if self.t1 is not None else float("inf")
+        inside = [r for w, r in rows if w is not None and t0 <= w <= t1]
+        picked = inside
+        if not picked:  # region shorter than the interval: the sample nearest to it
+            mid = 0.5 * (t0 + t1) if self.t0 is not None and self.t1 is not None else None
+            timed = [(abs(w - mid), r) for w, r in rows if w is not None and mid is not None]
+            picked = [min(timed, key=lambda x: x[0])[1]] if timed else [rows[-1][1]]
+        sm = [float(r[2]) for r in picked]
+        mx = [float(r[3]) for r in picked if r[3].replace(".", "").isdigit()]
         names = ["hw_slowdown", "hw_thermal_slowdown", "sw_thermal_slowdown", "sw_power_cap"]
-        reasons = sorted({names[i] for r in rows for i in range(4) if r[5 + i].lower().startswith("active")})
-        return {"sm_mhz": statistics.median(sm) if sm else None, "sm_max_mhz": max(mx) if mx else None,
-                "reasons": reasons, "samples": len(rows)}
+        reasons = sorted({names[i] for r in picked for i in range(4) if r[6 + i].lower().startswith("active")})
+        out = {"sm_mhz": statistics.median(sm), "sm_max_mhz": max(mx) if mx else None, "reasons": reasons,
+               "samples": len(inside)}
+        if self.t0 is not None and self.t1 is not None:
+            out["window_ms"] = round(1000.0 * (self.t1 - self.t0), 1)
+        return out
 
 
 def gpu_uuid(dev):
@@ -301,6 +334,7 @@ def run_ours(args, rank, world, local_rank):
         eng.verify_batch_device(ids, tk, pr, off, outputs=(acc_dev, None, None, None))
 
     # warm-up (also captures the CUDA graph)
+    clk = ClockSampler(gpu_uuid(local_rank))
     for _ in range(max(3, args.warmup)):
         one_step()
         eng.sync()
@@ -310,10 +344,10 @@ def run_ours(args, rank, world, local_rank):
     launches = eng.step_launches()
 
     # ---- timed region: K steps, device time from CUDA events on the launching stream
-    clk = ClockSampler(gpu_uuid(local_rank))
     if dist:
         dist.barrier()
     torch.cuda.synchronize()
+    clk.begin()
     times = []
     for _ in range(args.steps):
         e0 = torch.cuda.Event(enable_timing=True)
@@ -328,6 +362,7 @@ def run_ours(args, rank, world, local_rank):
         eng.sync()
         eng.truncate(0, P)
     torch.cuda.synchronize()
+    clk.end()
     if dist:
         dist.barrier()
     clocks = clk.stop()
@@ -479,14 +514,16 @@ def run_batch64(args):
         for b in range(B):
             eng.truncate(b, int(lens[b]))
 
+    clk = ClockSampler(gpu_uuid(0))
     for _ in range(max(3, args.warmup)):
         eng.verify_batch_device(ids, tk, pr, off, outputs=(acc, None, None, None))
         reset()
     a_len = eng.verify_batch(list(range(B)), trees)[0]
     reset()
-    clk = ClockSampler(gpu_uuid(0))
+    clk.begin()
     ms = _timed(eng.stream, lambda: eng.verify_batch_device(ids, tk, pr, off, outputs=(acc, None, None, None)),
                 args.steps, reset)
+    clk.end()
     clocks = clk.stop()
     eng.profile(True)
     eng.verify_batch_device(ids, tk, pr, off)
@@ -523,6 +560,8 @@ def run_sweep(args):
     kv_tok = dims.n_layers * 2 * dims.kv_dim * 2
     out = []
     clk = ClockSampler(gpu_uuid(0))
+    time.sleep(0.2)
+    clk.begin()
     for name, sh in shapes:
         draws = synth.plant_draws(sh.n, dims.vocab, stream=0)
         toks = synth.plant_tree(sh, pend, 0.85, draws, lambda t, p_: eng.score([0], [(t, p_)])[0])
@@ -543,6 +582,7 @@ def run_sweep(args):
         fl = flops_per_token(dims) * sh.n + attn_flops(dims, P * sh.n, dims.n_layers)
         out.append({"draft": name, "nodes": sh.n, "ms_per_step": ms, "tau": a + 1,
                     "accepted_tokens_per_s": (a + 1) * 1000.0 / ms, "roofline_frac": _roofline(bytes_, fl, ms)["frac"]})
+    clk.end()
     clocks = clk.stop()
     print(json.dumps({"workload": "llama3.1-8b-shape bf16, batch 1, prefix 8192, chains 5/8 and trees 16/32/60/80"
                                   " at depth 8, planted p=0.85", "results": out, "clocks": clocks, "data": "synthetic"}))
@@ -574,11 +614,13 @@ def run_draft(args):
     ti = torch.zeros(M, 10, dtype=torch.int32, device="cuda")
     tv = torch.zeros(M, 10, dtype=torch.float32, device="cuda")
     step = lambda: eng.draft_step_device(ids, feats, tk, pr, off, outputs=(ti, tv))
+    clk = ClockSampler(gpu_uuid(0))
     for _ in range(max(3, args.warmup)):
         step()
         eng.sync()
-    clk = ClockSampler(gpu_uuid(0))
+    clk.begin()
     ms = _timed(eng.stream, step, args.steps, lambda: None)
+    clk.end()
     clocks = clk.stop()
     eng.profile(True)
     step()
