@@ -18,6 +18,7 @@ oracle on a bounded sample of the same workload instead.
 from __future__ import annotations
 
 import argparse
+import dataclasses
 import json
 import os
 import statistics
@@ -311,7 +312,6 @@ def run_ours(args, rank, world, local_rank):
         import datetime
         import torch.distributed as dist
         dist.init_process_group("nccl", timeout=datetime.timedelta(seconds=120), device_id=torch.device("cuda", local_rank))
-    import dataclasses
     dims = dataclasses.replace(synth.LLAMA8B, n_layers=args.layers)
     P = args.prefix
     w = synth.model_weights(dims, seed=0, device="cuda")
@@ -492,7 +492,7 @@ def run_batch64(args):
     """64 sequences, prefixes uniform in [512, 4096], each with its own 60-draft tree, p uniform in [0.6, 0.9]."""
     import torch
     from speculative_decoding_06_b200.engine import SpecEngine, pack_trees
-    dims = synth.LLAMA8B
+    dims = dataclasses.replace(synth.LLAMA8B, n_layers=args.layers)
     B = 64
     lens, ps = synth.batch_prefix_lengths_and_p(B)
     w = synth.model_weights(dims, seed=0, device="cuda")
@@ -536,7 +536,8 @@ def run_batch64(args):
     rk = sum(int(lens[b]) * 61 + 61 * 5 for b in range(B))  # prefix keys per node + ~ancestors
     fl = flops_per_token(dims) * M + attn_flops(dims, rk, dims.n_layers)
     tau = float(np.mean(a_len + 1))
-    print(json.dumps({"workload": "llama3.1-8b-shape bf16, batch 64, prefixes U[512,4096], own 60-draft trees,"
+    print(json.dumps({"layers": dims.n_layers,
+                      "workload": "llama3.1-8b-shape bf16, batch 64, prefixes U[512,4096], own 60-draft trees,"
                                   " planted p U[0.6,0.9]", "tokens_per_step": M, "ms_per_step": ms,
                       "verify_steps_per_s": 1000.0 / ms, "accepted_tokens_per_s": float(np.sum(a_len + 1)) * 1000.0 / ms,
                       "tau_mean": tau, "roofline": _roofline(bytes_, fl, ms, sustained=True), "kernel_ms_per_step": prof,
