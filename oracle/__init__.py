@@ -31,6 +31,6 @@ SwiGLU MLP) is the standard Llama decoder, written out in float64.
 from .tree import tree_meta, accept_walk, ancestor_matrix, root_paths  # noqa: F401
 from .model import (  # noqa: F401
     OracleModel, OracleSeq, oracle_prefill, oracle_tree_logits, oracle_verify,
-    oracle_greedy_ar, causal_logits, top2_margin, argmax_fn_for_planting,
+    oracle_greedy_ar, causal_logits, top2_margin, argmax_fn_for_planting, causal_features, oracle_tree_features,
 )
 from .draft import OracleDraftHead  # noqa: F401

@@ -188,13 +188,32 @@ class OracleModel:
     def forward(self, tokens: Sequence[int], pos: np.ndarray, past: Optional[List[Tuple[np.ndarray, np.ndarray]]],
                 vis_new: np.ndarray):
         """Full forward of new rows on top of a cache.  Returns (logits [n][V], new K/V per layer)."""
+        logits, new_kv, _ = self.forward_features(tokens, pos, past, vis_new, ())
+        return logits, new_kv
+
+    def forward_features(self, tokens: Sequence[int], pos: np.ndarray,
+                         past: Optional[List[Tuple[np.ndarray, np.ndarray]]], vis_new: np.ndarray,
+                         taps: Sequence[int]):
+        """As `forward`, and also the residual stream after taps[f] decoder layers
+        (1 <= taps[f] <= n_layers) for every row: features [n][len(taps)][d].
+
+        EAGLE-3 (draft-stage description) feeds its draft head with the target's
+        low-, mid- and high-level hidden states of each position; these are the
+        residual stream between decoder blocks, before any norm."""
+        L = self.d.n_layers
+        for j in taps:
+            if not 1 <= j <= L:
+                raise ValueError("feature layer %d outside [1, %d]" % (j, L))
         x = self.embed(tokens)
+        after = {}
         new_kv = []
-        for l in range(self.d.n_layers):
+        for l in range(L):
             pk, pv = (None, None) if not past else past[l]
             x, k, v = self.layer_forward(l, x, pos, pk, pv, vis_new)
             new_kv.append((k, v))
-        return self.lm_logits(x), new_kv
+            after[l + 1] = x
+        feats = np.stack([after[j] for j in taps], axis=1) if taps else np.zeros((x.shape[0], 0, x.shape[1]))
+        return self.lm_logits(x), new_kv, feats
 
 
 def causal_logits(model: OracleModel, tokens: Sequence[int]) -> np.ndarray:
@@ -203,6 +222,14 @@ def causal_logits(model: OracleModel, tokens: Sequence[int]) -> np.ndarray:
     vis = np.tril(np.ones((T, T), bool))
     logits, _ = model.forward(tokens, np.arange(T), None, vis)
     return logits
+
+
+def causal_features(model: OracleModel, tokens: Sequence[int], taps: Sequence[int]) -> np.ndarray:
+    """Residual stream after taps[f] layers of a plain causal forward (no cache): [T][len(taps)][d]."""
+    T = len(tokens)
+    vis = np.tril(np.ones((T, T), bool))
+    _, _, feats = model.forward_features(tokens, np.arange(T), None, vis, taps)
+    return feats
 
 
 # ---------------------------------------------------------------------------
@@ -237,24 +264,34 @@ def oracle_tree_logits(model: OracleModel, seq: OracleSeq, tokens: Sequence[int]
     Returns (logits [n][V], per-layer tree K/V).  Node i is at position
     P + depth(i) and sees the prefix plus its ancestors (itself included).
     """
+    logits, kv, _ = oracle_tree_features(model, seq, tokens, parents, ())
+    return logits, kv
+
+
+def oracle_tree_features(model: OracleModel, seq: OracleSeq, tokens: Sequence[int], parents: Sequence[int],
+                         taps: Sequence[int]):
+    """As `oracle_tree_logits`, plus the residual stream after taps[f] layers at every node."""
     depth, _ = tree_meta(parents)
     P = seq.length
     vis = ancestor_matrix(parents)
     past = list(zip(seq.k, seq.v)) if P else None
-    return model.forward(tokens, P + depth, past, vis)
+    return model.forward_features(tokens, P + depth, past, vis, taps)
 
 
 def oracle_verify(model: OracleModel, seq: OracleSeq, tokens: Sequence[int], parents: Sequence[int],
-                  check_root: bool = True) -> dict:
+                  check_root: bool = True, taps: Sequence[int] = ()) -> dict:
     """Tree-verification step; updates `seq` in place (KV compaction, length, pending).
 
     Returns accepted_len (accepted drafts), accepted_nodes, accepted_tokens,
-    bonus, plus argmax / logits / margin per node for parity checks.
+    bonus, plus argmax / logits / margin per node for parity checks.  With
+    `taps`, also "features": the residual stream after taps[f] layers of the
+    root and of each accepted node, in path order ([accepted_len + 1][len(taps)][d]),
+    the draft head's input for the positions the step emits.
     """
     tokens = [int(t) for t in tokens]
     if check_root and tokens[0] != seq.pending:
         raise ValueError("tokens[0] must be the pending token %d" % seq.pending)
-    logits, tree_kv = oracle_tree_logits(model, seq, tokens, parents)
+    logits, tree_kv, feats = oracle_tree_features(model, seq, tokens, parents, taps)
     amax = np.argmax(logits, axis=1)  # first (lowest) index on ties
     acc_nodes, bonus = accept_walk(tokens, parents, amax)
     keep = [0] + acc_nodes
@@ -272,6 +309,7 @@ def oracle_verify(model: OracleModel, seq: OracleSeq, tokens: Sequence[int], par
         "logits": logits,
         "margin": top2_margin(logits),
         "tree_kv": tree_kv,
+        "features": feats[keep],
     }
 
 
