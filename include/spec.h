@@ -63,6 +63,8 @@ extern "C" {
 #define SPEC_DEVICE_OUTPUTS 1  /* outputs are device pointers (or NULL); return without synchronising */
 #define SPEC_DEBUG_LOGITS 2    /* also store fp32 logits [total nodes][vocab] to the buffer of spec_set_debug_logits */
 #define SPEC_NO_GRAPH 4        /* launch kernel by kernel instead of replaying a captured CUDA graph */
+#define SPEC_FEATURES 8        /* also write the draft-head features of the root and the accepted nodes to
+                                  the buffer of spec_set_feature_out (needs cfg.feature_layers) */
 
 typedef struct spec_config {
   int32_t n_layers;
@@ -80,6 +82,11 @@ typedef struct spec_config {
   int32_t max_nodes;    /* tree nodes per sequence per step, root included; <= 128 */
   int32_t draft_head;   /* 1: the handle also runs the EAGLE-3 draft head (bf16 only): its weights in
                            spec_weights, its layer's K/V one more cache layer (counted by spec_kv_bytes) */
+  int32_t feature_layers[3]; /* the low, mid and high features the EAGLE-3 draft head takes (its
+                           draft-stage description: the target's low-, mid- and high-level hidden
+                           states of every position): the residual stream after this many decoder
+                           layers, each in [1, n_layers]; {0, 0, 0}: no feature tap.  The pages name
+                           no layers; 2, n_layers / 2 and n_layers - 3 is one choice. */
 } spec_config;
 
 /* Per-layer weights, device pointers, row-major [out][in] in the model dtype:
@@ -197,6 +204,16 @@ SPEC_API int spec_draft_step(spec_handle* h, int B, const int32_t* seq_ids, cons
 /* Draft prefix length of `seq` (host output). */
 SPEC_API int spec_draft_len(spec_handle* h, int seq, int32_t* len);
 
+/* Device buffer for SPEC_FEATURES, bf16 [B][max_nodes][3][hidden], 16-byte aligned, owned by the
+ * caller.  A verification step with SPEC_FEATURES writes, for batch entry b and k = 0 ..
+ * accepted_len[b], row [b][k] = the residual stream after feature_layers[0], [1] and [2] decoder
+ * layers (rounded to bf16) at the k-th node of the emitted path: the root for k = 0, then the
+ * accepted nodes in order, i.e. the positions P .. P + accepted_len that the step adds to the cache.
+ * Rows beyond accepted_len[b] are left as they were.  bytes must cover the step's batch:
+ * B * max_nodes * 3 * hidden * 2 (checked per step; SPEC_ERR_CAPACITY otherwise).  SPEC_ERR_STATE
+ * when the handle has no feature layers; device_buf NULL detaches the buffer. */
+SPEC_API int spec_set_feature_out(spec_handle* h, void* device_buf, size_t bytes);
+
 /* Device buffer (fp32, >= max_batch * max_nodes * vocab entries) for SPEC_DEBUG_LOGITS. */
 SPEC_API int spec_set_debug_logits(spec_handle* h, float* device_buf, size_t bytes);
 
@@ -230,7 +247,8 @@ SPEC_API int spec_validate_tree(const int32_t* tokens, const int32_t* parents, i
 #define SPEC_PROF_GEMM_LAYER 12  /* one launch: O, gate/up, down, then the next QKV or the LM head */
 #define SPEC_PROF_DRAFT_FC 13    /* draft head: feature split, fusion FC, input FC */
 #define SPEC_PROF_TOPK 14        /* draft head: top-k over the logits */
-#define SPEC_PROF_CLASSES 15
+#define SPEC_PROF_FEATURES 15    /* draft-head feature tap and gather (SPEC_FEATURES) */
+#define SPEC_PROF_CLASSES 16
 
 /* enable != 0: subsequent steps launch kernel by kernel (no graph) with a CUDA
  * event pair around every launch on the handle's stream. */

@@ -156,6 +156,83 @@ cudaError_t launch_kv_compact(const StepView& sv, const KvView& kv, int n_layers
   return cudaLaunchKernelEx(&cfg, kv_compact_kernel, sv, kv, acc_len, acc_nodes, max_nodes);
 }
 
+// ---------------------------------------------------------------------------
+// draft-head features ("EAGLE-3: Scaling up Inference Acceleration of Large
+// Language Models via Training-Time Test", draft-stage description: the draft
+// head takes the target's low-, mid- and high-level hidden states of each
+// position, recorded during prefill and verification)
+// ---------------------------------------------------------------------------
+
+// the residual stream x (fp32 [M][d], d % 4 == 0) after a tap layer, as bf16 rows
+__global__ void feature_tap_kernel(int d, const float* __restrict__ x, __nv_bfloat16* __restrict__ out) {
+  pdl_wait();
+  pdl_launch_dependents();
+  const size_t t = blockIdx.x;
+  const float4* xr = reinterpret_cast<const float4*>(x + t * d);
+  uint2* o = reinterpret_cast<uint2*>(out + t * d);
+  for (int c = threadIdx.x; c < d / 4; c += blockDim.x) {
+    const float4 v = xr[c];
+    const __nv_bfloat162 a = __floats2bfloat162_rn(v.x, v.y);
+    const __nv_bfloat162 b = __floats2bfloat162_rn(v.z, v.w);
+    uint2 u;
+    u.x = *reinterpret_cast<const uint32_t*>(&a);
+    u.y = *reinterpret_cast<const uint32_t*>(&b);
+    o[c] = u;
+  }
+}
+
+cudaError_t launch_feature_tap(int M, int d, const float* x, __nv_bfloat16* out, cudaStream_t s, bool pdl) {
+  if (M < 1 || d % 4) return cudaErrorInvalidValue;
+  cudaLaunchAttribute attr[1];
+  attr[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+  attr[0].val.programmaticStreamSerializationAllowed = 1;
+  cudaLaunchConfig_t cfg = {};
+  cfg.gridDim = dim3(M);
+  cfg.blockDim = dim3(128);
+  cfg.stream = s;
+  cfg.attrs = attr;
+  cfg.numAttrs = pdl ? 1 : 0;
+  return cudaLaunchKernelEx(&cfg, feature_tap_kernel, d, x, out);
+}
+
+// Block (k, b): the k-th node of tree b's emitted path (the root, then the
+// accepted nodes) -> out[b][k][f][:] = tap[f][row of that node][:], f = 0..2.
+// Nothing for k > acc_len[b].  d % 8 == 0; 16-byte copies.
+__global__ void feature_gather_kernel(StepView sv, const int32_t* __restrict__ acc_len,
+                                      const int32_t* __restrict__ acc_nodes, int max_nodes,
+                                      const __nv_bfloat16* __restrict__ tap, int Mpad, int d,
+                                      __nv_bfloat16* __restrict__ out) {
+  pdl_wait();
+  pdl_launch_dependents();
+  const int b = blockIdx.y, k = blockIdx.x;
+  const int a = acc_len[b];
+  if (k > a) return;
+  const int node = k == 0 ? 0 : acc_nodes[(size_t)b * max_nodes + k - 1];
+  const size_t row = (size_t)sv.node_off[b] + node;
+  const int nv = d / 8;
+  for (int f = 0; f < 3; ++f) {
+    const uint4* src = reinterpret_cast<const uint4*>(tap + ((size_t)f * Mpad + row) * d);
+    uint4* dst = reinterpret_cast<uint4*>(out + (((size_t)b * max_nodes + k) * 3 + f) * d);
+    for (int i = threadIdx.x; i < nv; i += blockDim.x) dst[i] = src[i];
+  }
+}
+
+cudaError_t launch_feature_gather(const StepView& sv, const int32_t* acc_len, const int32_t* acc_nodes,
+                                  int max_nodes, const __nv_bfloat16* tap, int Mpad, int d, __nv_bfloat16* out,
+                                  cudaStream_t s, bool pdl) {
+  if (d % 8 || max_nodes < 1) return cudaErrorInvalidValue;
+  cudaLaunchAttribute attr[1];
+  attr[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+  attr[0].val.programmaticStreamSerializationAllowed = 1;
+  cudaLaunchConfig_t cfg = {};
+  cfg.gridDim = dim3(max_nodes, sv.B);
+  cfg.blockDim = dim3(128);
+  cfg.stream = s;
+  cfg.attrs = attr;
+  cfg.numAttrs = pdl ? 1 : 0;
+  return cudaLaunchKernelEx(&cfg, feature_gather_kernel, sv, acc_len, acc_nodes, max_nodes, tap, Mpad, d, out);
+}
+
 // draft head: out[r] = [g[r] | E[tokens[r]]]  (bf16, 2d wide)
 __global__ void gather_concat_kernel(int d, const __nv_bfloat16* __restrict__ g, const int32_t* __restrict__ tokens,
                                      const __nv_bfloat16* __restrict__ embed, __nv_bfloat16* __restrict__ out) {

@@ -55,6 +55,8 @@ struct WsLayout {
   size_t ss, gemm_ctr, attn_ctr, phase_bar;
   // draft head: split features [2 Mpad][3d], [g|e] operand [2 Mpad][2d], logits, top-k
   size_t fsplit = 0, ge = 0, dlogits = 0, dtop_i = 0, dtop_v = 0;
+  // feature tap: bf16 residual stream after the three feature layers [3][Mpad][d]
+  size_t tap = 0;
   int n_ss = 1, attn_ctr_n = 0, phase_bar_n = 0;
   size_t partial_bytes;
   // outputs (one device->host copy per step)
@@ -127,6 +129,7 @@ WsLayout make_layout(const spec_config& c) {
   L.argmax = take(4 * (size_t)L.Mpad);
   L.top1 = take(4 * (size_t)L.Mpad);
   L.top2 = take(4 * (size_t)L.Mpad);
+  if (c.feature_layers[0] > 0) L.tap = take(2 * 3 * (size_t)L.Mpad * c.hidden);
   if (c.draft_head) {
     L.fsplit = take(2 * 2 * (size_t)L.Mpad * 3 * c.hidden);
     L.ge = take(2 * 2 * (size_t)L.Mpad * 2 * c.hidden);
@@ -173,6 +176,12 @@ std::string check_config(const spec_config* c) {
     if (c->hidden % 4) return "fp32 models need hidden % 4 == 0";
   }
   if (c->draft_head && c->dtype != SPEC_DTYPE_BF16) return "the draft head is bf16 only";
+  const int* fl = c->feature_layers;
+  if (fl[0] || fl[1] || fl[2]) {
+    for (int f = 0; f < 3; ++f)
+      if (fl[f] < 1 || fl[f] > c->n_layers) return "feature_layers must all be 0 or each in [1, n_layers]";
+    if (c->hidden % 8) return "feature taps need hidden % 8 == 0";
+  }
   return "";
 }
 
@@ -260,6 +269,8 @@ struct spec_handle {
   uint8_t* h_out = nullptr;
   float* dbg_logits = nullptr;
   size_t dbg_bytes = 0;
+  void* feat_out = nullptr;  // SPEC_FEATURES destination, bf16 [B][max_nodes][3][d]
+  size_t feat_bytes = 0;
   std::map<GraphKey, cudaGraphExec_t> graphs;
   bool use_pdl = true;
   int max_splits = 16;    // split-K cap
@@ -575,7 +586,7 @@ struct PhaseBuilder {
   }
 };
 
-cudaError_t enqueue_step(spec_handle* h, const StepPlan& sp, int mode, bool dbg) {
+cudaError_t enqueue_step(spec_handle* h, const StepPlan& sp, int mode, bool dbg, bool feat) {
   const spec_config& c = h->cfg;
   const WsLayout& L = h->lay;
   cudaStream_t st = h->stream;
@@ -595,6 +606,15 @@ cudaError_t enqueue_step(spec_handle* h, const StepPlan& sp, int mode, bool dbg)
 
   float* ss = h->W<float>(L.ss);
   int* gctr = h->W<int>(L.gemm_ctr);
+  // feature tap: after the layer that completes the residual stream of feature layer f
+  __nv_bfloat16* tap = feat ? h->W<__nv_bfloat16>(L.tap) : nullptr;
+  auto tap_after = [&](int layers_done, bool tpdl) -> cudaError_t {
+    if (!feat) return cudaSuccess;
+    for (int f = 0; f < 3; ++f)
+      if (c.feature_layers[f] == layers_done)
+        LK(SPEC_PROF_FEATURES, 1, launch_feature_tap(M, d, x, tap + (size_t)f * L.Mpad * d, st, tpdl));
+    return cudaSuccess;
+  };
   if (dt == 1) {
     // arrival counters start every step at zero, whatever an earlier failed step left behind
     cudaError_t e0 = cudaMemsetAsync(gctr, 0, 4 * (size_t)kGemmCounters, st);
@@ -660,6 +680,7 @@ cudaError_t enqueue_step(spec_handle* h, const StepPlan& sp, int mode, bool dbg)
       m.ph[3] = (l + 1 < c.n_layers) ? pb.qkv(l + 1, 3) : pb.lm(dbg ? h->dbg_logits : nullptr);
       if (h->trace && l == h->trace_layer) m.trace = h->trace;
       LK(SPEC_PROF_GEMM_LAYER, 1, gemm_multi_launch(m, st, pdl));
+      CUDA_RET(tap_after(l + 1, pdl));
     } else {
       const float* xf = reinterpret_cast<const float*>(xn);
       LK(SPEC_PROF_GEMM_QKV, 1, launch_gemm_simt_f32(xf, d, (const float*)lw.wq, d, part, nqkv, M, qd, st));
@@ -679,6 +700,7 @@ cudaError_t enqueue_step(spec_handle* h, const StepPlan& sp, int mode, bool dbg)
       LK(SPEC_PROF_GEMM_DOWN, 1,
          launch_gemm_simt_f32((const float*)hm, c.ffn, (const float*)lw.w_down, c.ffn, part, d, M, d, st));
       LK(SPEC_PROF_RESID_NORM, 1, launch_residual_norm(dt, M, d, 1, part, 0, x, xn, next_norm, c.rms_eps, st, false));
+      CUDA_RET(tap_after(l + 1, false));
     }
   }
 
@@ -712,6 +734,10 @@ cudaError_t enqueue_step(spec_handle* h, const StepPlan& sp, int mode, bool dbg)
   if (mode == STEP_VERIFY)
     LK(SPEC_PROF_COMPACT, 1,
        launch_kv_compact(sv, h->kv, c.n_layers, w.acc_len, w.acc_nodes, c.max_nodes, st, pdl && dt == 1));
+  if (feat)
+    LK(SPEC_PROF_FEATURES, 1,
+       launch_feature_gather(sv, w.acc_len, w.acc_nodes, c.max_nodes, tap, L.Mpad, d,
+                             static_cast<__nv_bfloat16*>(h->feat_out), st, pdl && dt == 1));
   return cudaSuccess;
 }
 
@@ -851,6 +877,14 @@ int run_step(spec_handle* h, int B, const int32_t* seq_ids, const int32_t* token
   if (dbg && (!h->dbg_logits || h->dbg_bytes < sizeof(float) * (size_t)M * h->cfg.vocab))
     return fail(h, SPEC_ERR_CAPACITY, "SPEC_DEBUG_LOGITS needs a debug buffer of %zu bytes",
                 sizeof(float) * (size_t)M * h->cfg.vocab);
+  const bool feat = (flags & SPEC_FEATURES) != 0;
+  if (feat) {
+    if (mode != STEP_VERIFY) return fail(h, SPEC_ERR_ARG, "SPEC_FEATURES applies to verification steps");
+    if (h->cfg.feature_layers[0] < 1) return fail(h, SPEC_ERR_STATE, "the handle was created without feature layers");
+    const size_t need = 2 * 3 * (size_t)B * h->cfg.max_nodes * h->cfg.hidden;
+    if (!h->feat_out || h->feat_bytes < need)
+      return fail(h, SPEC_ERR_CAPACITY, "SPEC_FEATURES needs a feature buffer of %zu bytes", need);
+  }
   // pack the parameter block
   uint8_t* pb = h->h_params;
   std::memcpy(pb + L.p_tokens, tokens, 4 * (size_t)M);
@@ -864,12 +898,12 @@ int run_step(spec_handle* h, int B, const int32_t* seq_ids, const int32_t* token
   // the legacy default stream cannot be captured: launch directly there
   const bool graph = !(flags & SPEC_NO_GRAPH) && !h->prof && h->stream != nullptr;
   if (graph) {
-    GraphKey key{mode, B, M, max_n, sp.n_chunks, sp.chunk, dbg ? 1 : 0, h->use_pdl ? 1 : 0};
+    GraphKey key{mode, B, M, max_n, sp.n_chunks, sp.chunk, (dbg ? 1 : 0) | (feat ? 2 : 0), h->use_pdl ? 1 : 0};
     auto it = h->graphs.find(key);
     if (it == h->graphs.end()) {
       cudaGraph_t g = nullptr;
       CUDA_TRY(h, cudaStreamBeginCapture(h->stream, cudaStreamCaptureModeThreadLocal));
-      cudaError_t e = enqueue_step(h, sp, mode, dbg);
+      cudaError_t e = enqueue_step(h, sp, mode, dbg, feat);
       cudaError_t e2 = cudaStreamEndCapture(h->stream, &g);
       if (e != cudaSuccess || e2 != cudaSuccess) {
         if (g) cudaGraphDestroy(g);
@@ -883,7 +917,7 @@ int run_step(spec_handle* h, int B, const int32_t* seq_ids, const int32_t* token
     }
     CUDA_TRY(h, cudaGraphLaunch(it->second, h->stream));
   } else {
-    cudaError_t e = enqueue_step(h, sp, mode, dbg);
+    cudaError_t e = enqueue_step(h, sp, mode, dbg, feat);
     if (e != cudaSuccess) return fail(h, SPEC_ERR_CUDA, "kernel launch failed: %s", cudaGetErrorString(e));
   }
 
@@ -1382,6 +1416,18 @@ int spec_draft_len(spec_handle* h, int seq, int32_t* len) {
   if (!h || !len) return SPEC_ERR_ARG;
   if (seq < 0 || seq >= h->cfg.max_batch) return fail(h, SPEC_ERR_ARG, "seq %d outside [0, %d)", seq, h->cfg.max_batch);
   *len = h->dlen[seq];
+  return SPEC_OK;
+}
+
+int spec_set_feature_out(spec_handle* h, void* device_buf, size_t bytes) {
+  if (!h) return SPEC_ERR_ARG;
+  if (h->cfg.feature_layers[0] < 1) return fail(h, SPEC_ERR_STATE, "the handle was created without feature layers");
+  if (device_buf && !aligned16(device_buf)) return fail(h, SPEC_ERR_ARG, "the feature buffer must be 16-byte aligned");
+  h->feat_out = device_buf;
+  h->feat_bytes = device_buf ? bytes : 0;
+  // graphs bake the pointer in
+  for (auto& kv : h->graphs) cudaGraphExecDestroy(kv.second);
+  h->graphs.clear();
   return SPEC_OK;
 }
 

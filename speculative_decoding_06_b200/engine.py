@@ -43,7 +43,10 @@ class SpecEngine:
     """One handle of the library over caller-owned (torch) device buffers."""
 
     def __init__(self, dims, weights: Dict, max_batch: int, max_seq: int, max_nodes: int = 128,
-                 stream: Optional[torch.cuda.Stream] = None, draft: Optional[Dict] = None):
+                 stream: Optional[torch.cuda.Stream] = None, draft: Optional[Dict] = None,
+                 feature_layers: Optional[Sequence[int]] = None):
+        """feature_layers: (low, mid, high) layer counts whose residual streams a
+        verification step can return for the draft head (see verify_batch)."""
         self.dims = dims
         self.cfg = S.spec_config(
             n_layers=dims.n_layers, hidden=dims.hidden, n_q_heads=dims.n_q_heads, n_kv_heads=dims.n_kv_heads,
@@ -51,6 +54,9 @@ class SpecEngine:
             dtype=S.SPEC_DTYPE_BF16 if dims.dtype == "bf16" else S.SPEC_DTYPE_F32,
             rms_eps=dims.rms_eps, rope_theta=dims.rope_theta, max_batch=max_batch, max_seq=max_seq,
             max_nodes=max_nodes, draft_head=1 if draft is not None else 0)
+        if feature_layers is not None:
+            self.cfg.feature_layers[:] = [int(j) for j in feature_layers]
+        self._feat = None
         self.max_nodes = max_nodes
         self.max_batch = max_batch
         kvb = S.spec_kv_bytes(ctypes.byref(self.cfg))
@@ -119,8 +125,10 @@ class SpecEngine:
         a = int(acc_len[0])
         return a, [int(x) for x in acc_tok[:a]], int(bonus[0])
 
-    def verify_batch(self, seq_ids, trees, flags: int = 0):
-        """Host outputs: (accepted_len[B], accepted_nodes[B][max_nodes], accepted_tokens, bonus[B])."""
+    def verify_batch(self, seq_ids, trees, flags: int = 0, features: bool = False):
+        """Host outputs: (accepted_len[B], accepted_nodes[B][max_nodes], accepted_tokens, bonus[B]);
+        with `features`, also the draft-head features of each emitted path as a bf16 device
+        tensor [B][max_nodes][3][hidden] (rows 0 .. accepted_len[b] valid)."""
         tok, par, off = pack_trees(trees)
         ids = _i32(seq_ids)
         B = len(ids)
@@ -128,10 +136,23 @@ class SpecEngine:
         acc_nodes = np.zeros((B, self.max_nodes), np.int32)
         acc_tok = np.zeros((B, self.max_nodes), np.int32)
         bonus = np.zeros(B, np.int32)
+        if features:
+            self.feature_buffer()
+            flags |= S.SPEC_FEATURES
         self._check(S.spec_verify_tree_batch(self.h, B, _ptr(ids), _ptr(tok), _ptr(par), _ptr(off),
                                              acc_len.ctypes.data, acc_nodes.ctypes.data, acc_tok.ctypes.data,
                                              bonus.ctypes.data, flags & ~S.SPEC_DEVICE_OUTPUTS))
+        if features:
+            return acc_len, acc_nodes, acc_tok, bonus, self._feat[:B]
         return acc_len, acc_nodes, acc_tok, bonus
+
+    def feature_buffer(self) -> torch.Tensor:
+        """The SPEC_FEATURES destination, bf16 [max_batch][max_nodes][3][hidden] (allocated once)."""
+        if self._feat is None:
+            self._feat = torch.zeros(self.max_batch, self.max_nodes, 3, self.dims.hidden, dtype=torch.bfloat16,
+                                     device="cuda")
+            self._check(S.spec_set_feature_out(self.h, self._feat.data_ptr(), self._feat.numel() * 2))
+        return self._feat
 
     def verify_batch_device(self, ids: np.ndarray, tok: np.ndarray, par: np.ndarray, off: np.ndarray,
                             outputs: Optional[Tuple[torch.Tensor, ...]] = None, flags: int = 0):

@@ -29,10 +29,12 @@ SPEC_DTYPE_BF16 = 1
 SPEC_DEVICE_OUTPUTS = 1
 SPEC_DEBUG_LOGITS = 2
 SPEC_NO_GRAPH = 4
+SPEC_FEATURES = 8
 SPEC_DRAFT_TOPK = 10
 
 PROF_CLASSES = ("embed_meta", "gemm_qkv", "rope_kv_store", "attention", "gemm_o", "resid_norm", "gemm_gate_up",
-                "gemm_down", "lm_head", "lm_reduce", "accept_walk", "kv_compact", "gemm_layer", "draft_fc", "topk")
+                "gemm_down", "lm_head", "lm_reduce", "accept_walk", "kv_compact", "gemm_layer", "draft_fc", "topk",
+                "features")
 
 ERR_NAMES = {0: "SPEC_OK", -1: "SPEC_ERR_ARG", -2: "SPEC_ERR_TREE", -3: "SPEC_ERR_TOKEN", -4: "SPEC_ERR_CAPACITY",
              -5: "SPEC_ERR_ROOT", -6: "SPEC_ERR_CUDA", -7: "SPEC_ERR_TIMEOUT", -8: "SPEC_ERR_STATE"}
@@ -45,6 +47,7 @@ class spec_config(ctypes.Structure):
         ("vocab", ctypes.c_int32), ("dtype", ctypes.c_int32), ("rms_eps", ctypes.c_float),
         ("rope_theta", ctypes.c_float), ("max_batch", ctypes.c_int32), ("max_seq", ctypes.c_int32),
         ("max_nodes", ctypes.c_int32), ("draft_head", ctypes.c_int32),
+        ("feature_layers", ctypes.c_int32 * 3),
     ]
 
 
@@ -79,6 +82,7 @@ _SIGNATURES = {
     "spec_score_trees": (ctypes.c_int, [_h, ctypes.c_int, _i32p, _i32p, _i32p, _i32p, _i32p, _f32p, _f32p,
                                         ctypes.c_int]),
     "spec_set_debug_logits": (ctypes.c_int, [_h, _vp, ctypes.c_size_t]),
+    "spec_set_feature_out": (ctypes.c_int, [_h, _vp, ctypes.c_size_t]),
     "spec_truncate": (ctypes.c_int, [_h, ctypes.c_int, ctypes.c_int]),
     "spec_seq_len": (ctypes.c_int, [_h, ctypes.c_int, _i32p, _i32p]),
     "spec_sync": (ctypes.c_int, [_h]),

@@ -21,7 +21,7 @@ def gpu_available() -> bool:
     return torch.cuda.is_available()
 
 
-def make_pair(dims, max_batch=1, max_seq=1024, max_nodes=128, seed=0, device_gen=False):
+def make_pair(dims, max_batch=1, max_seq=1024, max_nodes=128, seed=0, device_gen=False, **engine_kw):
     """Engine (GPU) and oracle (CPU) over the same seeded weights."""
     from speculative_decoding_06_b200.engine import SpecEngine
     if device_gen:
@@ -32,7 +32,7 @@ def make_pair(dims, max_batch=1, max_seq=1024, max_nodes=128, seed=0, device_gen
         host = synth.weights_to_host(wcpu)
         wdev = {k: v.cuda() for k, v in wcpu.items() if k != "layers"}
         wdev["layers"] = [{k: v.cuda() for k, v in lw.items()} for lw in wcpu["layers"]]
-    eng = SpecEngine(dims, wdev, max_batch=max_batch, max_seq=max_seq, max_nodes=max_nodes)
+    eng = SpecEngine(dims, wdev, max_batch=max_batch, max_seq=max_seq, max_nodes=max_nodes, **engine_kw)
     return eng, OracleModel(dims, host)
 
 

@@ -46,6 +46,23 @@ def test_kv_bytes_matches_layout():
     assert 0 < ws < 512 << 20
 
 
+@pytest.mark.parametrize("layers,ok", [((0, 0, 0), True), ((1, 1, 2), True), ((2, 1, 2), True),
+                                       ((0, 1, 2), False), ((1, 3, 2), False), ((-1, 1, 1), False)])
+def test_feature_layers_checked_and_sized(layers, ok):
+    """feature_layers: all zero (no tap) or each in [1, n_layers]; a tap adds [3][Mpad][d] bf16 of workspace."""
+    d = synth.MINI_BF16  # 2 layers
+    base = S.spec_workspace_bytes(ctypes.byref(cfg_of(d, max_batch=2, max_nodes=64)))
+    c = cfg_of(d, max_batch=2, max_nodes=64)
+    c.feature_layers[:] = list(layers)
+    ws = S.spec_workspace_bytes(ctypes.byref(c))
+    if not ok:
+        assert ws == 0 and S.spec_kv_bytes(ctypes.byref(c)) == 0
+    elif layers == (0, 0, 0):
+        assert ws == base
+    else:
+        assert ws >= base + 3 * 128 * d.hidden * 2  # Mpad = 128 for 2 x 64 nodes
+
+
 @pytest.mark.parametrize("field,value", [
     ("n_kv_heads", 3), ("head_dim", 64), ("hidden", 4000), ("max_nodes", 129), ("max_nodes", 0), ("dtype", 7),
     ("ffn", 100), ("rope_theta", 0.5),
