@@ -279,6 +279,7 @@ struct spec_handle {
   float rescale_slack = 8.f;  // attention: running-max slack in log2 units (p <= 2^slack)
   int attn_clusters[kAttnMaxChunks + 1] = {};  // co-resident clusters of n chunk CTAs
   bool attn_dsmem = true;     // merge chunk partials through distributed shared memory when they fit a cluster
+  int bn64_max = 64;          // largest token count planned with 64-token tiles (several token tiles above 64)
   // L2 prefetch of weights ahead of the GEMM that streams them
   uint64_t* trace = nullptr;  // optional GEMM timeline of one layer's launch
   size_t trace_bytes = 0;
@@ -342,7 +343,7 @@ cudaError_t launch_k(spec_handle* h, int cls, int n_kernels, F&& fn) {
 
 GemmPlan plan_gemm(const spec_handle* h, int rows_per_tile, int n_out, int K, int M, int epi) {
   GemmPlan p;
-  p.bn = M <= 64 ? 64 : 128;
+  p.bn = M <= h->bn64_max ? 64 : 128;
   const int bi = p.bn == 64 ? 0 : 1;
   int per_sm = std::max(1, h->resident[bi][0]);  // one kernel function for every epilogue
   if (h->resident_cap > 0) per_sm = std::min(per_sm, h->resident_cap);
@@ -1173,6 +1174,7 @@ int spec_init(const spec_config* cfg, const spec_weights* w, void* kv_cache, siz
     if (const char* q = strstr(t, "chunks=")) if (sscanf(q + 7, "%d", &v) == 1 && v >= 1 && v <= kMaxAttnChunks) h->max_chunks = v;
     if (const char* q = strstr(t, "pdl=")) if (sscanf(q + 4, "%d", &v) == 1) h->use_pdl = v != 0;
     if (const char* q = strstr(t, "dsmem=")) if (sscanf(q + 6, "%d", &v) == 1) h->attn_dsmem = v != 0;
+    if (const char* q = strstr(t, "bn64max=")) if (sscanf(q + 8, "%d", &v) == 1 && v >= 64) h->bn64_max = v;
     if (const char* q = strstr(t, "per_sm=")) if (sscanf(q + 7, "%d", &v) == 1 && v >= 0) h->resident_cap = v;
     float fv = 0.f;
     if (const char* q = strstr(t, "rescale=")) if (sscanf(q + 8, "%f", &fv) == 1 && fv >= 0.f && fv <= 15.f) h->rescale_slack = fv;
