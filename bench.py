@@ -644,6 +644,56 @@ def run_draft(args):
     return 0
 
 
+def run_draft_tree(args):
+    """Dynamic draft tree: batch 16, draft prefixes of 2048 rows, 8 drafting steps, top-10, 60 nodes."""
+    import torch
+    from speculative_decoding_06_b200.engine import SpecEngine
+    dims = synth.LLAMA8B
+    B, P, steps, K, total = 16, 2048, 8, 10, 60
+    w = synth.model_weights(dims, seed=0, device="cuda")
+    dw = synth.draft_head_weights(dims, seed=6, device="cuda")
+    eng = SpecEngine(dims, w, max_batch=B, max_seq=P + 128, max_nodes=128, draft=dw)
+    rng = np.random.default_rng(5)
+    for b in range(B):
+        f = synth.draft_features(P, dims.hidden, seed=100 + b, device="cuda")
+        eng.draft_prefill(b, f, rng.integers(0, dims.vocab, size=P).astype(np.int32))
+    root_feats = synth.draft_features(B, dims.hidden, seed=7, device="cuda")
+    roots = rng.integers(0, dims.vocab, size=B).astype(np.int32)
+    ids = list(range(B))
+    step = lambda: eng.draft_tree(ids, root_feats, roots, steps=steps, topk=K, total=total)
+    clk = ClockSampler(gpu_uuid(0))
+    for _ in range(max(3, args.warmup)):
+        step()
+    clk.begin()
+    ms = _timed(eng.stream, step, args.steps, lambda: None)
+    clk.end()
+    clocks = clk.stop()
+    eng.profile(True)
+    step()
+    prof = {k: round(v[0], 3) for k, v in eng.profile_read().items() if v[1]}
+    eng.profile(False)
+    d = dims
+    layer = d.q_dim * d.hidden + 2 * d.kv_dim * d.hidden + d.hidden * d.q_dim + 3 * d.ffn * d.hidden
+    per_step = 2 * d.hidden * d.hidden + layer + d.vocab * d.hidden  # input FC, decoder layer, LM head
+    hbm, tflops, kind = measured_peaks()
+    roof = 0.0
+    fl_all = 0.0
+    for t in range(steps):
+        M = B * (1 + t * K)  # every step recomputes the tree built so far
+        fl = 2.0 * per_step * M + (2.0 * 3 * d.hidden * d.hidden * B if t == 0 else 0.0) + attn_flops(d, P * M, 1)
+        by = 2.0 * per_step + B * (P + M // B) * 2 * d.kv_dim * 2
+        roof += max(by / hbm / 1e6, fl / tflops / 1e9)
+        fl_all += fl
+    print(json.dumps({"workload": "EAGLE-3 dynamic draft tree at 8B shape bf16: batch 16, draft prefix 2048, "
+                                  "8 drafting steps, top-10 offers, 60 nodes (every step recomputes the tree so far)",
+                      "ms_per_tree_batch": ms, "trees_per_s": B * 1000.0 / ms,
+                      "roofline": {"bound": "per step: max(hbm, tensor)", "roofline_ms": roof, "frac": roof / ms,
+                                   "flops": fl_all, "hbm_gbs": hbm, "bf16_tflops": tflops, "peak_source": kind},
+                      "kernel_ms_per_tree_batch": prof, "clocks": clocks, "data": "synthetic"}))
+    eng.close()
+    return 0
+
+
 def main():
     ap = argparse.ArgumentParser()
     ap.add_argument("--gpus", type=int, default=1)
@@ -654,7 +704,7 @@ def main():
     ap.add_argument("--sample-layers", type=int, default=2)
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--layers", type=int, default=32, help="decoder layers (32 = the 8B shape; fewer only for profiling)")
-    ap.add_argument("--workload", default="verify", choices=["verify", "batch64", "sweep", "draft"],
+    ap.add_argument("--workload", default="verify", choices=["verify", "batch64", "sweep", "draft", "draft_tree"],
                     help="verify: the default line (batch 1, prefix 2048); the others measure the remaining"
                          " configurations (one GPU, one JSON line each)")
     args = ap.parse_args()
@@ -666,7 +716,8 @@ def main():
     if args.workload != "verify":
         import torch
         torch.cuda.set_device(local_rank)
-        return {"batch64": run_batch64, "sweep": run_sweep, "draft": run_draft}[args.workload](args)
+        return {"batch64": run_batch64, "sweep": run_sweep, "draft": run_draft,
+                "draft_tree": run_draft_tree}[args.workload](args)
     return run_ours(args, rank, world, local_rank)
 
 

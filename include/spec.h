@@ -204,6 +204,30 @@ SPEC_API int spec_draft_step(spec_handle* h, int B, const int32_t* seq_ids, cons
 /* Draft prefix length of `seq` (host output). */
 SPEC_API int spec_draft_len(spec_handle* h, int seq, int32_t* len);
 
+/* Dynamic draft tree for B sequences ("EAGLE-3: Scaling up Inference Acceleration of Large
+ * Language Models via Training-Time Test", draft-stage description: multi-step drafting, where
+ * from the second step on the draft's own output a replaces the target feature; and its account
+ * of EAGLE-2: the draft's confidence stands in for the acceptance rate and shapes the tree).
+ * Reading taken where the pages leave steps open: a node's value is the sum of the draft's
+ * log-probabilities (full-vocabulary softmax) along its root path; step t = 0 .. steps-1 runs
+ * the draft head over the tree built so far (the root's feature is the fused target feature,
+ * every other node's the output a of its parent); the nodes that joined last (the root at step
+ * 0) offer their topk best tokens and the topk best offers join (ties: earlier offer); after the
+ * last step the `total` best offers, joined or not (ties: lower depth, then earlier offer), form
+ * the tree, which is closed under ancestors.
+ * root_feats: device bf16 [B][3][hidden], 16-byte aligned, the low/mid/high target features of
+ * each sequence's last verified position (as SPEC_FEATURES returns them); root_tokens: host
+ * int32 [B], the pending tokens (the roots).  Each sequence needs a draft prefix (the rows up to
+ * the last verified position, spec_draft_prefill), which the call leaves unchanged.  topk is 4,
+ * 8, 10 or 16; 1 + (steps-1)*topk <= max_nodes, 1 + steps*topk <= 128, topk + (steps-1)*topk^2
+ * <= 1024 offers, total <= that and total + 1 <= max_nodes (SPEC_ERR_CAPACITY otherwise).
+ * Outputs (host): out_tokens / out_parents int32 [B][total+1], root first, nodes by depth and
+ * then value, parents[i] < i (a tree spec_verify_tree_batch accepts); out_values (may be NULL)
+ * float [B][total+1], each node's value (0 for the root).  Synchronises. */
+SPEC_API int spec_draft_tree(spec_handle* h, int B, const int32_t* seq_ids, const void* root_feats,
+                             const int32_t* root_tokens, int steps, int topk, int total, int32_t* out_tokens,
+                             int32_t* out_parents, float* out_values);
+
 /* Device buffer for SPEC_FEATURES, bf16 [B][max_nodes][3][hidden], 16-byte aligned, owned by the
  * caller.  A verification step with SPEC_FEATURES writes, for batch entry b and k = 0 ..
  * accepted_len[b], row [b][k] = the residual stream after feature_layers[0], [1] and [2] decoder
@@ -248,7 +272,8 @@ SPEC_API int spec_validate_tree(const int32_t* tokens, const int32_t* parents, i
 #define SPEC_PROF_DRAFT_FC 13    /* draft head: feature split, fusion FC, input FC */
 #define SPEC_PROF_TOPK 14        /* draft head: top-k over the logits */
 #define SPEC_PROF_FEATURES 15    /* draft-head feature tap and gather (SPEC_FEATURES) */
-#define SPEC_PROF_CLASSES 16
+#define SPEC_PROF_TREE 16        /* dynamic draft tree: root features, expansion, rerank */
+#define SPEC_PROF_CLASSES 17
 
 /* enable != 0: subsequent steps launch kernel by kernel (no graph) with a CUDA
  * event pair around every launch on the handle's stream. */

@@ -163,8 +163,50 @@ cudaError_t launch_split_rows(const __nv_bfloat16* src, int rows, int cols, __nv
                               bool pdl);
 // per row: the k largest of V fp32 values, ordered by (value desc, index asc)
 constexpr int kTopKMax = 16;
+// top-k per row (value desc, index asc), k in {4, 8, 10, 16}; with lse != NULL also
+// the row's log-sum-exp (natural log)
 cudaError_t launch_topk_rows(int M, int V, const float* logits, size_t ld, int k, int32_t* idx, float* val,
-                             cudaStream_t s, bool pdl);
+                             float* lse, cudaStream_t s, bool pdl);
+
+// a launch configuration with programmatic dependent launch when pdl (attr: 1 slot)
+cudaLaunchConfig_t make_cfg(dim3 grid, dim3 block, size_t smem, cudaStream_t s, bool pdl, cudaLaunchAttribute* attr);
+
+// ---------------------------------------------------------------------------
+// dynamic draft tree (draft_tree.cu)
+// ---------------------------------------------------------------------------
+constexpr int kTreeMaxOffers = 1024;  // candidates offered over all steps, per tree
+constexpr int kTreeMaxNodes = 128;    // nodes joined over all steps, per tree (root included)
+
+struct TreeOffer {
+  float v;      // cumulative log-probability
+  int depth;    // the offered node's depth
+  int order;    // offer order within the tree (ties)
+  int parent;   // offering node (joined node id)
+  int token;
+  int node;     // joined node id, or -1
+};
+
+struct TreeArgs {
+  int K;            // top-k per offering node, and nodes joining per step
+  int max_nodes;    // stride of the per-tree node arrays
+  int write_next;   // 1: write the next step's tree into the parameter block
+  int32_t* tok;     // [B][max_nodes] joined nodes
+  int32_t* par;
+  float* val;
+  TreeOffer* offers;  // [B][kTreeMaxOffers]
+  int32_t* n_offers;  // [B]
+};
+
+cudaError_t launch_tree_save_root(int B, int d, int ld, const __nv_bfloat16* ge, __nv_bfloat16* groot,
+                                  const int32_t* tokens, const TreeArgs& a, cudaStream_t s, bool pdl);
+cudaError_t launch_tree_feature_rows(int M, int d, int ld, int n, int n_prev, const int32_t* parents,
+                                     const __nv_bfloat16* groot, const float* x_prev, __nv_bfloat16* ge,
+                                     cudaStream_t s, bool pdl);
+cudaError_t launch_tree_expand(const TreeArgs& a, int B, int t, int n, int nf, const int32_t* top_i,
+                               const float* top_v, const float* lse, int32_t* tokens_io, int32_t* parents_io,
+                               cudaStream_t s, bool pdl);
+cudaError_t launch_tree_rerank(const TreeArgs& a, int B, int total, int32_t* out_tok, int32_t* out_par,
+                               float* out_val, cudaStream_t s, bool pdl);
 // x += sum of split partials; xn = RMSNorm(x) * w
 cudaError_t launch_residual_norm(int dtype, int M, int d, int S, const float* partial, size_t split_stride, float* x,
                                  void* xn, const void* w, float eps, cudaStream_t s, bool pdl);

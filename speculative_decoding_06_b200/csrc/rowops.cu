@@ -30,6 +30,9 @@ __device__ __forceinline__ float block_sum(float v, float* red) {
   return t;
 }
 
+
+}  // namespace
+
 cudaLaunchConfig_t make_cfg(dim3 grid, dim3 block, size_t smem, cudaStream_t s, bool pdl, cudaLaunchAttribute* attr) {
   cudaLaunchConfig_t cfg = {};
   cfg.gridDim = grid;
@@ -42,8 +45,6 @@ cudaLaunchConfig_t make_cfg(dim3 grid, dim3 block, size_t smem, cudaStream_t s, 
   cfg.numAttrs = pdl ? 1 : 0;
   return cfg;
 }
-
-}  // namespace
 
 // ---------------------------------------------------------------------------
 // tree metadata + embedding + RMSNorm
@@ -515,9 +516,10 @@ __device__ __forceinline__ void warp_merge_topk(const float (&lv)[K], const int 
 }
 }  // namespace
 
-template <int K>
+template <int K, bool LSE>
 __global__ void __launch_bounds__(256) topk_rows_kernel(int V, const float* __restrict__ logits, size_t ld,
-                                                       int32_t* __restrict__ out_i, float* __restrict__ out_v) {
+                                                       int32_t* __restrict__ out_i, float* __restrict__ out_v,
+                                                       float* __restrict__ out_lse) {
   __shared__ float wv[8][K];
   __shared__ int wi[8][K];
   pdl_wait();
@@ -596,6 +598,17 @@ __global__ void __launch_bounds__(256) topk_rows_kernel(int V, const float* __re
   const bool vec = (ld % 4 == 0) && ((reinterpret_cast<uintptr_t>(logits) & 15u) == 0);
   const int V4 = vec ? V / 4 : 0;
   const float4* row4 = reinterpret_cast<const float4*>(row);
+  // optional log-sum-exp: a running (max, sum of 2^((x - max) log2 e)) per thread
+  constexpr float kLog2e = 1.4426950408889634f;
+  float lm = -INFINITY, ls = 0.f;
+  auto lse_add = [&](float mx, float e0, float e1, float e2, float e3) {
+    if (mx > lm) {
+      ls = (lm == -INFINITY ? 0.f : ls * fast_exp2((lm - mx) * kLog2e));
+      lm = mx;
+    }
+    ls += fast_exp2((e0 - lm) * kLog2e) + fast_exp2((e1 - lm) * kLog2e) + fast_exp2((e2 - lm) * kLog2e) +
+          fast_exp2((e3 - lm) * kLog2e);
+  };
   for (int g0 = threadIdx.x; g0 < V4; g0 += 2 * blockDim.x) {
     float4 x[2];
 #pragma unroll
@@ -606,6 +619,7 @@ __global__ void __launch_bounds__(256) topk_rows_kernel(int V, const float* __re
 #pragma unroll
     for (int u = 0; u < 2; ++u) {
       const float m = fmaxf(fmaxf(x[u].x, x[u].y), fmaxf(x[u].z, x[u].w));
+      if (LSE && m > -INFINITY) lse_add(m, x[u].x, x[u].y, x[u].z, x[u].w);
       if (m >= thr) {
         const int c = 4 * (g0 + u * blockDim.x);
         if (x[u].x >= thr) offer(x[u].x, c);
@@ -617,7 +631,35 @@ __global__ void __launch_bounds__(256) topk_rows_kernel(int V, const float* __re
   }
   for (int c = 4 * V4 + threadIdx.x; c < V; c += blockDim.x) {
     const float x = __ldcs(row + c);
+    if (LSE) lse_add(x, x, -INFINITY, -INFINITY, -INFINITY);
     if (x >= thr) offer(x, c);
+  }
+  if (LSE) {
+    // combine the threads' (max, sum) pairs: warp shuffles, then the 8 warps
+    __shared__ float lse_m[8], lse_s[8];
+    for (int o = 16; o > 0; o >>= 1) {
+      const float m2 = __shfl_xor_sync(0xffffffffu, lm, o);
+      const float s2 = __shfl_xor_sync(0xffffffffu, ls, o);
+      const float mm = fmaxf(lm, m2);
+      if (mm > -INFINITY) {
+        ls = (lm == -INFINITY ? 0.f : ls * fast_exp2((lm - mm) * kLog2e)) +
+             (m2 == -INFINITY ? 0.f : s2 * fast_exp2((m2 - mm) * kLog2e));
+        lm = mm;
+      }
+    }
+    if (lane == 0) {
+      lse_m[warp] = lm;
+      lse_s[warp] = ls;
+    }
+    __syncthreads();
+    if (threadIdx.x == 0) {
+      float M0 = -INFINITY;
+      for (int w = 0; w < 8; ++w) M0 = fmaxf(M0, lse_m[w]);
+      float S0 = 0.f;
+      for (int w = 0; w < 8; ++w)
+        if (lse_m[w] > -INFINITY) S0 += lse_s[w] * fast_exp2((lse_m[w] - M0) * kLog2e);
+      out_lse[r] = M0 + __logf(S0);
+    }
   }
   warp_merge_topk<K>(lv, li, wv[warp], wi[warp]);
   __syncthreads();
@@ -640,15 +682,23 @@ __global__ void __launch_bounds__(256) topk_rows_kernel(int V, const float* __re
 }
 
 cudaError_t launch_topk_rows(int M, int V, const float* logits, size_t ld, int k, int32_t* idx, float* val,
-                             cudaStream_t s, bool pdl) {
+                             float* lse, cudaStream_t s, bool pdl) {
   if (k < 1 || k > kTopKMax || k > V) return cudaErrorInvalidValue;
   cudaLaunchAttribute attr[1];
   cudaLaunchConfig_t cfg = make_cfg(dim3(M), dim3(256), 0, s, pdl, attr);
   switch (k) {  // the list length is a compile-time constant of the kernel
-    case 10: return cudaLaunchKernelEx(&cfg, topk_rows_kernel<10>, V, logits, ld, idx, val);
-    case 16: return cudaLaunchKernelEx(&cfg, topk_rows_kernel<16>, V, logits, ld, idx, val);
-    case 8: return cudaLaunchKernelEx(&cfg, topk_rows_kernel<8>, V, logits, ld, idx, val);
-    case 4: return cudaLaunchKernelEx(&cfg, topk_rows_kernel<4>, V, logits, ld, idx, val);
+    case 10:
+      return lse ? cudaLaunchKernelEx(&cfg, topk_rows_kernel<10, true>, V, logits, ld, idx, val, lse)
+                 : cudaLaunchKernelEx(&cfg, topk_rows_kernel<10, false>, V, logits, ld, idx, val, lse);
+    case 16:
+      return lse ? cudaLaunchKernelEx(&cfg, topk_rows_kernel<16, true>, V, logits, ld, idx, val, lse)
+                 : cudaLaunchKernelEx(&cfg, topk_rows_kernel<16, false>, V, logits, ld, idx, val, lse);
+    case 8:
+      return lse ? cudaLaunchKernelEx(&cfg, topk_rows_kernel<8, true>, V, logits, ld, idx, val, lse)
+                 : cudaLaunchKernelEx(&cfg, topk_rows_kernel<8, false>, V, logits, ld, idx, val, lse);
+    case 4:
+      return lse ? cudaLaunchKernelEx(&cfg, topk_rows_kernel<4, true>, V, logits, ld, idx, val, lse)
+                 : cudaLaunchKernelEx(&cfg, topk_rows_kernel<4, false>, V, logits, ld, idx, val, lse);
     default: return cudaErrorInvalidValue;
   }
 }

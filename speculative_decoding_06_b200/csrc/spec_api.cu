@@ -57,6 +57,9 @@ struct WsLayout {
   size_t fsplit = 0, ge = 0, dlogits = 0, dtop_i = 0, dtop_v = 0;
   // feature tap: bf16 residual stream after the three feature layers [3][Mpad][d]
   size_t tap = 0;
+  // dynamic draft tree: per-tree nodes and offers, saved root features, per-row top-k and log-sum-exp, output
+  size_t tr_tok = 0, tr_par = 0, tr_val = 0, tr_offers = 0, tr_noff = 0, tr_groot = 0, tr_lse = 0, tr_top_i = 0,
+         tr_top_v = 0, tr_out_tok = 0, tr_out_par = 0, tr_out_val = 0;
   int n_ss = 1, attn_ctr_n = 0, phase_bar_n = 0;
   size_t partial_bytes;
   // outputs (one device->host copy per step)
@@ -136,6 +139,19 @@ WsLayout make_layout(const spec_config& c) {
     L.dlogits = take(4 * (size_t)L.Mpad * c.vocab);
     L.dtop_i = take(4 * (size_t)L.Mpad * kDraftTopK);
     L.dtop_v = take(4 * (size_t)L.Mpad * kDraftTopK);
+    const size_t tn = (size_t)c.max_batch * kTreeMaxNodes;
+    L.tr_tok = take(4 * tn);
+    L.tr_par = take(4 * tn);
+    L.tr_val = take(4 * tn);
+    L.tr_offers = take(sizeof(TreeOffer) * (size_t)c.max_batch * kTreeMaxOffers);
+    L.tr_noff = take(4 * (size_t)c.max_batch);
+    L.tr_groot = take(2 * 2 * (size_t)c.max_batch * c.hidden);
+    L.tr_lse = take(4 * (size_t)L.Mpad);
+    L.tr_top_i = take(4 * (size_t)L.Mpad * kTopKMax);
+    L.tr_top_v = take(4 * (size_t)L.Mpad * kTopKMax);
+    L.tr_out_tok = take(4 * tn);
+    L.tr_out_par = take(4 * tn);
+    L.tr_out_val = take(4 * tn);
   }
   const size_t o0 = off;
   L.o_acc_len = take(4 * (size_t)c.max_batch);
@@ -746,7 +762,14 @@ cudaError_t enqueue_step(spec_handle* h, const StepPlan& sp, int mode, bool dbg,
 // top-k).  The draft layer is layer n_layers of the cache; prefix lengths come
 // with the parameter block.  With `kv_only` (draft prefill) the step stops once
 // the layer's K/V are stored: they depend on the layer input alone.
-cudaError_t enqueue_draft(spec_handle* h, const StepPlan& sp, bool kv_only, bool dbg) {
+// One step of the dynamic draft tree: step t over trees of n nodes (n_prev at
+// step t - 1), top-k K per row, the tree state.
+struct TreeStep {
+  int t, n, n_prev, K;
+  TreeArgs args;
+};
+
+cudaError_t enqueue_draft(spec_handle* h, const StepPlan& sp, bool kv_only, bool dbg, const TreeStep* ts = nullptr) {
   const spec_config& c = h->cfg;
   const WsLayout& L = h->lay;
   cudaStream_t st = h->stream;
@@ -765,14 +788,24 @@ cudaError_t enqueue_draft(spec_handle* h, const StepPlan& sp, bool kv_only, bool
      launch_embed_meta(1, sv, h->embed, nullptr, d, c.rms_eps, nullptr, nullptr, nullptr, 0, 0,
                        h->W<double>(L.inv_freq), c.head_dim / 2, STEP_SCORE, st, pdl, ge, 2 * d, d));
   const PhaseBuilder pb(h, sp, sv);
-  // g = [l|m|h] . W_fuse^T into the left half of [g|e]
-  {
+  __nv_bfloat16* groot = h->W<__nv_bfloat16>(L.tr_groot);
+  if (ts && ts->t > 0) {
+    // a later drafting step: the root keeps its fused target feature, every other
+    // node takes its parent's draft output a (the previous step's x)
+    LK(SPEC_PROF_DRAFT_FC, 1,
+       launch_tree_feature_rows(M, d, 2 * d, ts->n, ts->n_prev, h->W<int32_t>(L.p_parents), groot, h->W<float>(L.x),
+                                ge, st, pdl));
+  } else {
+    // g = [l|m|h] . W_fuse^T into the left half of [g|e]
     const GemmPlan pf = plan_gemm(h, 128, d, 3 * d, M, GEMM_EPI_STORE);
     GemmTcLaunch g = gemm_launch(pf, GEMM_EPI_STORE, d, 3 * d, M, &h->map_fc_fuse, nullptr, nullptr,
                                  &h->map_fsplit[bi], d, 0, 0, sv.err);
     g.args.out_bf16 = ge;
     g.args.ld_out = 2 * d;
     LK(SPEC_PROF_DRAFT_FC, 1, gemm_tc_launch(g, st, pdl));
+    if (ts)
+      LK(SPEC_PROF_TREE, 1,
+         launch_tree_save_root(sp.B, d, 2 * d, ge, groot, h->W<int32_t>(L.p_tokens), ts->args, st, pdl));
   }
   // x = [g|e] . W_in^T (a residual GEMM on x = 0), xn = split(x * attn_norm), ss
   CUDA_RET(cudaMemsetAsync(h->ws + L.x, 0, 4 * (size_t)M * d, st));
@@ -822,9 +855,14 @@ cudaError_t enqueue_draft(spec_handle* h, const StepPlan& sp, bool kv_only, bool
   m.ph[2] = pb.down(Ld, 2, h->draft_final_norm);
   m.ph[3] = pb.lm(logits);
   LK(SPEC_PROF_GEMM_LAYER, 1, gemm_multi_launch(m, st, pdl));
-  LK(SPEC_PROF_TOPK, 1,
-     launch_topk_rows(M, c.vocab, logits, c.vocab, kDraftTopK, h->W<int32_t>(L.dtop_i), h->W<float>(L.dtop_v), st,
-                      pdl));
+  if (ts)
+    LK(SPEC_PROF_TOPK, 1,
+       launch_topk_rows(M, c.vocab, logits, c.vocab, ts->K, h->W<int32_t>(L.tr_top_i), h->W<float>(L.tr_top_v),
+                        h->W<float>(L.tr_lse), st, pdl));
+  else
+    LK(SPEC_PROF_TOPK, 1,
+       launch_topk_rows(M, c.vocab, logits, c.vocab, kDraftTopK, h->W<int32_t>(L.dtop_i), h->W<float>(L.dtop_v),
+                        nullptr, st, pdl));
   if (dbg) CUDA_RET(cudaMemcpyAsync(h->dbg_logits, logits, 4 * (size_t)M * c.vocab, cudaMemcpyDeviceToDevice, st));
   return cudaSuccess;
 }
@@ -1412,6 +1450,113 @@ int spec_draft_step(spec_handle* h, int B, const int32_t* seq_ids, const void* f
     if (rc) return rc;
   }
   return run_draft(h, B, seq_ids, feats, tokens, parents, node_offsets, false, flags, top_idx, top_val);
+}
+
+int spec_draft_tree(spec_handle* h, int B, const int32_t* seq_ids, const void* root_feats, const int32_t* root_tokens,
+                    int steps, int topk, int total, int32_t* out_tokens, int32_t* out_parents, float* out_values) {
+  if (!h) return SPEC_ERR_ARG;
+  h->err.clear();
+  if (h->stale) {
+    int rc = refresh_state(h);
+    if (rc) return rc;
+  }
+  const spec_config& c = h->cfg;
+  const WsLayout& L = h->lay;
+  cudaStream_t st = h->stream;
+  if (!c.draft_head) return fail(h, SPEC_ERR_STATE, "the handle was created without the draft head");
+  if (B < 1 || B > c.max_batch) return fail(h, SPEC_ERR_CAPACITY, "batch %d outside [1, %d]", B, c.max_batch);
+  if (!seq_ids || !root_feats || !root_tokens || !out_tokens || !out_parents)
+    return fail(h, SPEC_ERR_ARG, "null pointer");
+  if (!aligned16(root_feats)) return fail(h, SPEC_ERR_ARG, "root_feats must be 16-byte aligned");
+  if (topk != 4 && topk != 8 && topk != 10 && topk != 16) return fail(h, SPEC_ERR_ARG, "topk must be 4, 8, 10 or 16");
+  if (steps < 1 || total < 1) return fail(h, SPEC_ERR_ARG, "steps and total must be positive");
+  const int n_last = 1 + (steps - 1) * topk;       // rows per tree in the last step
+  const int joined = 1 + steps * topk;             // nodes joined over all steps
+  const int n_offers = topk + (steps - 1) * topk * topk;
+  if (n_last > c.max_nodes || joined > kTreeMaxNodes || n_offers > kTreeMaxOffers)
+    return fail(h, SPEC_ERR_CAPACITY, "%d steps of top-%d exceed the tree limits (max_nodes %d)", steps, topk,
+                c.max_nodes);
+  if (total > n_offers || total + 1 > c.max_nodes)
+    return fail(h, SPEC_ERR_CAPACITY, "total %d exceeds the offers (%d) or max_nodes - 1", total, n_offers);
+  std::vector<uint8_t> seen(c.max_batch, 0);
+  int max_dlen = 0;
+  for (int b = 0; b < B; ++b) {
+    const int s = seq_ids[b];
+    if (s < 0 || s >= c.max_batch) return fail(h, SPEC_ERR_ARG, "seq id %d outside [0, %d)", s, c.max_batch);
+    if (seen[s]) return fail(h, SPEC_ERR_ARG, "seq id %d appears twice in one batch", s);
+    seen[s] = 1;
+    if (!h->dready[s]) return fail(h, SPEC_ERR_STATE, "sequence %d has no draft prefix", s);
+    if (h->dlen[s] + n_last > c.max_seq)
+      return fail(h, SPEC_ERR_CAPACITY, "sequence %d: draft length %d + %d nodes exceeds max_seq %d", s, h->dlen[s],
+                  n_last, c.max_seq);
+    if (root_tokens[b] < 0 || root_tokens[b] >= c.vocab) return fail(h, SPEC_ERR_TOKEN, "root token outside [0, vocab)");
+    max_dlen = std::max(max_dlen, h->dlen[s]);
+  }
+  TreeArgs ta{};
+  ta.K = topk;
+  ta.max_nodes = kTreeMaxNodes;
+  ta.tok = h->W<int32_t>(L.tr_tok);
+  ta.par = h->W<int32_t>(L.tr_par);
+  ta.val = h->W<float>(L.tr_val);
+  ta.offers = h->W<TreeOffer>(L.tr_offers);
+  ta.n_offers = h->W<int32_t>(L.tr_noff);
+  for (int t = 0; t < steps; ++t) {
+    const int n = 1 + t * topk, M = B * n;
+    uint8_t* pb = h->h_params;
+    int32_t* no = reinterpret_cast<int32_t*>(pb + L.p_node_off);
+    for (int b = 0; b <= B; ++b) no[b] = b * n;
+    std::memcpy(pb + L.p_seq_ids, seq_ids, 4 * (size_t)B);
+    std::memcpy(pb + L.p_dlen, h->dlen.data(), 4 * (size_t)c.max_batch);
+    std::memset(pb + L.p_err, 0, 16);
+    if (t == 0) {
+      // step 0: one root per tree; a later step's tokens and parents were written on
+      // the device by the previous expansion
+      int32_t* tk = reinterpret_cast<int32_t*>(pb + L.p_tokens);
+      int32_t* pr = reinterpret_cast<int32_t*>(pb + L.p_parents);
+      for (int b = 0; b < B; ++b) {
+        tk[b] = root_tokens[b];
+        pr[b] = -1;
+      }
+      CUDA_TRY(h, cudaMemcpyAsync(h->ws, pb, L.p_end, cudaMemcpyHostToDevice, st));
+      CUDA_TRY(h, launch_split_rows(static_cast<const __nv_bfloat16*>(root_feats), B, 3 * c.hidden,
+                                    h->W<__nv_bfloat16>(L.fsplit), st, false));
+    } else {
+      CUDA_TRY(h, cudaMemcpyAsync(h->ws + L.p_node_off, pb + L.p_node_off, L.p_end - L.p_node_off,
+                                  cudaMemcpyHostToDevice, st));
+    }
+    const StepPlan sp = make_plan(h, B, M, n, max_dlen + n);
+    TreeStep ts{t, n, t ? 1 + (t - 1) * topk : 0, topk, ta};
+    ts.args.write_next = t + 1 < steps ? 1 : 0;
+    cudaError_t e = enqueue_draft(h, sp, false, false, &ts);
+    if (e == cudaSuccess)
+      e = launch_k(h, SPEC_PROF_TREE, 1, [&]() {
+        return launch_tree_expand(ts.args, B, t, n, t == 0 ? 1 : topk, h->W<int32_t>(L.tr_top_i),
+                                  h->W<float>(L.tr_top_v), h->W<float>(L.tr_lse), h->W<int32_t>(L.p_tokens),
+                                  h->W<int32_t>(L.p_parents), st, false);
+      });
+    if (e != cudaSuccess) return fail(h, SPEC_ERR_CUDA, "kernel launch failed: %s", cudaGetErrorString(e));
+    // the host parameter block is rewritten by the next step: let this step's copy finish
+    uint32_t errw[2] = {0, 0};
+    CUDA_TRY(h, cudaMemcpyAsync(errw, h->ws + L.p_err, 4, cudaMemcpyDeviceToHost, st));
+    CUDA_TRY(h, cudaStreamSynchronize(st));
+    if (errw[0] & SPEC_DEVERR_TIMEOUT) return fail(h, SPEC_ERR_TIMEOUT, "a bounded wait expired on the device");
+    if (errw[0]) return fail(h, SPEC_ERR_CUDA, "device reported error bits 0x%x", errw[0]);
+  }
+  const size_t no_ = (size_t)B * (total + 1);
+  cudaError_t e = launch_k(h, SPEC_PROF_TREE, 1, [&]() {
+    return launch_tree_rerank(ta, B, total, h->W<int32_t>(L.tr_out_tok), h->W<int32_t>(L.tr_out_par),
+                              h->W<float>(L.tr_out_val), st, false);
+  });
+  if (e != cudaSuccess) return fail(h, SPEC_ERR_CUDA, "kernel launch failed: %s", cudaGetErrorString(e));
+  CUDA_TRY(h, cudaMemcpyAsync(out_tokens, h->ws + L.tr_out_tok, 4 * no_, cudaMemcpyDeviceToHost, st));
+  CUDA_TRY(h, cudaMemcpyAsync(out_parents, h->ws + L.tr_out_par, 4 * no_, cudaMemcpyDeviceToHost, st));
+  if (out_values) CUDA_TRY(h, cudaMemcpyAsync(out_values, h->ws + L.tr_out_val, 4 * no_, cudaMemcpyDeviceToHost, st));
+  CUDA_TRY(h, cudaStreamSynchronize(st));
+  for (int b = 0; b < B; ++b)
+    if (spec_validate_tree(out_tokens + (size_t)b * (total + 1), out_parents + (size_t)b * (total + 1), total + 1,
+                           c.vocab, c.max_nodes) != SPEC_OK)
+      return fail(h, SPEC_ERR_CUDA, "tree %d came out malformed", b);
+  return SPEC_OK;
 }
 
 int spec_draft_len(spec_handle* h, int seq, int32_t* len) {

@@ -248,6 +248,21 @@ class SpecEngine:
         self._check(S.spec_draft_step(self.h, len(ids), _ptr(ids), feats.data_ptr(), _ptr(tok), _ptr(par),
                                       _ptr(off), ptrs[0], ptrs[1], flags | S.SPEC_DEVICE_OUTPUTS))
 
+    def draft_tree(self, seq_ids, root_feats: torch.Tensor, root_tokens, steps: int = 8, topk: int = 10,
+                   total: int = 60):
+        """Dynamic draft tree per sequence: (tokens [B][total+1], parents [B][total+1], values)."""
+        ids = _i32(seq_ids)
+        B = len(ids)
+        rt = _i32(root_tokens)
+        tok = np.zeros((B, total + 1), np.int32)
+        par = np.zeros((B, total + 1), np.int32)
+        val = np.zeros((B, total + 1), np.float32)
+        f = root_feats.contiguous()
+        self.stream.wait_stream(torch.cuda.current_stream())
+        self._check(S.spec_draft_tree(self.h, B, _ptr(ids), f.data_ptr(), _ptr(rt), steps, topk, total,
+                                      _ptr(tok), _ptr(par), _fptr(val)))
+        return tok, par, val
+
     def draft_len(self, seq: int) -> int:
         ln = np.zeros(1, np.int32)
         self._check(S.spec_draft_len(self.h, seq, _ptr(ln)))

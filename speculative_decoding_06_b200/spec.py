@@ -34,7 +34,7 @@ SPEC_DRAFT_TOPK = 10
 
 PROF_CLASSES = ("embed_meta", "gemm_qkv", "rope_kv_store", "attention", "gemm_o", "resid_norm", "gemm_gate_up",
                 "gemm_down", "lm_head", "lm_reduce", "accept_walk", "kv_compact", "gemm_layer", "draft_fc", "topk",
-                "features")
+                "features", "draft_tree")
 
 ERR_NAMES = {0: "SPEC_OK", -1: "SPEC_ERR_ARG", -2: "SPEC_ERR_TREE", -3: "SPEC_ERR_TOKEN", -4: "SPEC_ERR_CAPACITY",
              -5: "SPEC_ERR_ROOT", -6: "SPEC_ERR_CUDA", -7: "SPEC_ERR_TIMEOUT", -8: "SPEC_ERR_STATE"}
@@ -98,6 +98,8 @@ _SIGNATURES = {
     "spec_draft_prefill": (ctypes.c_int, [_h, ctypes.c_int, _vp, _i32p, ctypes.c_int]),
     "spec_draft_step": (ctypes.c_int, [_h, ctypes.c_int, _i32p, _vp, _i32p, _i32p, _i32p, _vp, _vp, ctypes.c_int]),
     "spec_draft_len": (ctypes.c_int, [_h, ctypes.c_int, _i32p]),
+    "spec_draft_tree": (ctypes.c_int, [_h, ctypes.c_int, _i32p, _vp, _i32p, ctypes.c_int, ctypes.c_int, ctypes.c_int,
+                                       _i32p, _i32p, _f32p]),
     "spec_wait_selftest": (ctypes.c_int, [_vp, ctypes.c_uint32, _i32p]),
     "spec_last_error": (ctypes.c_char_p, [_h]),
     "spec_free": (None, [_h]),
