@@ -142,6 +142,13 @@ SPEC_API int spec_init(const spec_config* cfg, const spec_weights* w, void* kv_c
  * *pending_token (host) receives the argmax at the last position: the root of
  * the next tree.  Synchronises the stream. */
 SPEC_API int spec_prefill(spec_handle* h, int seq, const int32_t* tokens, int n, int32_t* pending_token);
+/* spec_prefill that also writes the draft-head features of every prompt position (the
+ * residual stream after feature_layers[0], [1] and [2] decoder layers, rounded to bf16) to
+ * feats_out: device bf16 [n][3][hidden], 16-byte aligned, owned by the caller.  These are
+ * the features the EAGLE-3 draft head records during prefill (its draft-stage description).
+ * SPEC_ERR_STATE when the handle has no feature layers. */
+SPEC_API int spec_prefill_features(spec_handle* h, int seq, const int32_t* tokens, int n, int32_t* pending_token,
+                                   void* feats_out);
 
 /* One verification step for one sequence (host pointers, synchronises).
  * tokens[0] must be the pending token; parents[0] == -1 and 0 <= parents[i] < i.
@@ -190,6 +197,10 @@ SPEC_API int spec_score_trees(spec_handle* h, int B, const int32_t* seq_ids, con
 /* Build the draft layer's K/V for positions 0 .. n-1 of `seq` from n rows of
  * features and tokens (n <= max_seq), replacing what was there.  Synchronises. */
 SPEC_API int spec_draft_prefill(spec_handle* h, int seq, const void* feats, const int32_t* tokens, int n);
+/* As spec_draft_prefill, but the n rows extend the draft prefix of `seq` (positions len ..
+ * len + n - 1, attending to the rows before them): the rows a verification step adds.
+ * SPEC_ERR_STATE when the sequence has no draft prefix; SPEC_ERR_CAPACITY past max_seq. */
+SPEC_API int spec_draft_append(spec_handle* h, int seq, const void* feats, const int32_t* tokens, int n);
 /* One draft-head step over a batch of trees on the draft prefixes: per node,
  * the SPEC_DRAFT_TOPK best vocabulary entries of the draft distribution, by
  * logit descending then index ascending, in top_idx / top_val [nodes][TOPK].

@@ -217,6 +217,35 @@ __global__ void feature_gather_kernel(StepView sv, const int32_t* __restrict__ a
   }
 }
 
+// Prefill: every row in order, out[r][f][:] = tap[f][r][:].
+__global__ void feature_rows_out_kernel(const __nv_bfloat16* __restrict__ tap, int Mpad, int d,
+                                        __nv_bfloat16* __restrict__ out) {
+  pdl_wait();
+  pdl_launch_dependents();
+  const size_t r = blockIdx.x;
+  const int nv = d / 8;
+  for (int f = 0; f < 3; ++f) {
+    const uint4* src = reinterpret_cast<const uint4*>(tap + ((size_t)f * Mpad + r) * d);
+    uint4* dst = reinterpret_cast<uint4*>(out + (r * 3 + f) * d);
+    for (int i = threadIdx.x; i < nv; i += blockDim.x) dst[i] = src[i];
+  }
+}
+
+cudaError_t launch_feature_rows_out(int M, const __nv_bfloat16* tap, int Mpad, int d, __nv_bfloat16* out,
+                                    cudaStream_t s, bool pdl) {
+  if (d % 8 || M < 1) return cudaErrorInvalidValue;
+  cudaLaunchAttribute attr[1];
+  attr[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+  attr[0].val.programmaticStreamSerializationAllowed = 1;
+  cudaLaunchConfig_t cfg = {};
+  cfg.gridDim = dim3(M);
+  cfg.blockDim = dim3(128);
+  cfg.stream = s;
+  cfg.attrs = attr;
+  cfg.numAttrs = pdl ? 1 : 0;
+  return cudaLaunchKernelEx(&cfg, feature_rows_out_kernel, tap, Mpad, d, out);
+}
+
 cudaError_t launch_feature_gather(const StepView& sv, const int32_t* acc_len, const int32_t* acc_nodes,
                                   int max_nodes, const __nv_bfloat16* tap, int Mpad, int d, __nv_bfloat16* out,
                                   cudaStream_t s, bool pdl) {

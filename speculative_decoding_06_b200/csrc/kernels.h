@@ -278,6 +278,8 @@ cudaError_t kv_compact_configure(size_t smem);
 // draft-head features: the residual stream (fp32 [M][d]) as bf16 rows of out, and the rows of
 // each tree's emitted path (root, accepted nodes) from tap [3][Mpad][d] to out [B][max_nodes][3][d]
 cudaError_t launch_feature_tap(int M, int d, const float* x, __nv_bfloat16* out, cudaStream_t s, bool pdl);
+cudaError_t launch_feature_rows_out(int M, const __nv_bfloat16* tap, int Mpad, int d, __nv_bfloat16* out,
+                                    cudaStream_t s, bool pdl);
 cudaError_t launch_feature_gather(const StepView& sv, const int32_t* acc_len, const int32_t* acc_nodes,
                                   int max_nodes, const __nv_bfloat16* tap, int Mpad, int d, __nv_bfloat16* out,
                                   cudaStream_t s, bool pdl);

@@ -287,6 +287,7 @@ struct spec_handle {
   size_t dbg_bytes = 0;
   void* feat_out = nullptr;  // SPEC_FEATURES destination, bf16 [B][max_nodes][3][d]
   size_t feat_bytes = 0;
+  void* pf_feat_out = nullptr;  // features of the prefill chunk being run, bf16 [rows][3][d]
   std::map<GraphKey, cudaGraphExec_t> graphs;
   bool use_pdl = true;
   int max_splits = 16;    // split-K cap
@@ -751,10 +752,13 @@ cudaError_t enqueue_step(spec_handle* h, const StepPlan& sp, int mode, bool dbg,
   if (mode == STEP_VERIFY)
     LK(SPEC_PROF_COMPACT, 1,
        launch_kv_compact(sv, h->kv, c.n_layers, w.acc_len, w.acc_nodes, c.max_nodes, st, pdl && dt == 1));
-  if (feat)
+  if (feat && mode == STEP_VERIFY)
     LK(SPEC_PROF_FEATURES, 1,
        launch_feature_gather(sv, w.acc_len, w.acc_nodes, c.max_nodes, tap, L.Mpad, d,
                              static_cast<__nv_bfloat16*>(h->feat_out), st, pdl && dt == 1));
+  else if (feat && mode == STEP_PREFILL)
+    LK(SPEC_PROF_FEATURES, 1,
+       launch_feature_rows_out(M, tap, L.Mpad, d, static_cast<__nv_bfloat16*>(h->pf_feat_out), st, pdl && dt == 1));
   return cudaSuccess;
 }
 
@@ -918,10 +922,11 @@ int run_step(spec_handle* h, int B, const int32_t* seq_ids, const int32_t* token
                 sizeof(float) * (size_t)M * h->cfg.vocab);
   const bool feat = (flags & SPEC_FEATURES) != 0;
   if (feat) {
-    if (mode != STEP_VERIFY) return fail(h, SPEC_ERR_ARG, "SPEC_FEATURES applies to verification steps");
+    if (mode != STEP_VERIFY && !(mode == STEP_PREFILL && h->pf_feat_out))
+      return fail(h, SPEC_ERR_ARG, "SPEC_FEATURES applies to verification steps");
     if (h->cfg.feature_layers[0] < 1) return fail(h, SPEC_ERR_STATE, "the handle was created without feature layers");
     const size_t need = 2 * 3 * (size_t)B * h->cfg.max_nodes * h->cfg.hidden;
-    if (!h->feat_out || h->feat_bytes < need)
+    if (mode == STEP_VERIFY && (!h->feat_out || h->feat_bytes < need))
       return fail(h, SPEC_ERR_CAPACITY, "SPEC_FEATURES needs a feature buffer of %zu bytes", need);
   }
   // pack the parameter block
@@ -1316,10 +1321,14 @@ int spec_init(const spec_config* cfg, const spec_weights* w, void* kv_cache, siz
   return SPEC_OK;
 }
 
-int spec_prefill(spec_handle* h, int seq, const int32_t* tokens, int n, int32_t* pending_token) {
+static int prefill_impl(spec_handle* h, int seq, const int32_t* tokens, int n, int32_t* pending_token,
+                        void* feats_out) {
   if (!h) return SPEC_ERR_ARG;
   h->err.clear();
   const spec_config& c = h->cfg;
+  if (feats_out && c.feature_layers[0] < 1)
+    return fail(h, SPEC_ERR_STATE, "the handle was created without feature layers");
+  if (feats_out && !aligned16(feats_out)) return fail(h, SPEC_ERR_ARG, "feats_out must be 16-byte aligned");
   if (!tokens || n < 1) return fail(h, SPEC_ERR_ARG, "prefill needs n >= 1 tokens");
   if (seq < 0 || seq >= c.max_batch) return fail(h, SPEC_ERR_ARG, "seq %d outside [0, %d)", seq, c.max_batch);
   if (n > c.max_seq) return fail(h, SPEC_ERR_CAPACITY, "prompt of %d tokens exceeds max_seq %d", n, c.max_seq);
@@ -1342,12 +1351,27 @@ int spec_prefill(spec_handle* h, int seq, const int32_t* tokens, int n, int32_t*
   for (int s0 = 0; s0 < n; s0 += c.max_nodes) {
     const int m = std::min(c.max_nodes, n - s0);
     const int32_t off[2] = {0, m};
-    int rc = run_step(h, 1, ids, tokens + s0, parents.data(), off, STEP_PREFILL, 0, true);
+    // with features: this chunk's rows go to feats_out at its offset (no graph: the
+    // destination changes from chunk to chunk)
+    h->pf_feat_out = feats_out ? static_cast<uint8_t*>(feats_out) + (size_t)s0 * 3 * c.hidden * 2 : nullptr;
+    int rc = run_step(h, 1, ids, tokens + s0, parents.data(), off, STEP_PREFILL,
+                      feats_out ? (SPEC_FEATURES | SPEC_NO_GRAPH) : 0, true);
+    h->pf_feat_out = nullptr;
     if (rc) return rc;
   }
   h->ready[seq] = 1;
   if (pending_token) *pending_token = h->pending[seq];
   return SPEC_OK;
+}
+
+int spec_prefill(spec_handle* h, int seq, const int32_t* tokens, int n, int32_t* pending_token) {
+  return prefill_impl(h, seq, tokens, n, pending_token, nullptr);
+}
+
+int spec_prefill_features(spec_handle* h, int seq, const int32_t* tokens, int n, int32_t* pending_token,
+                          void* feats_out) {
+  if (!feats_out) return h ? fail(h, SPEC_ERR_ARG, "feats_out is NULL") : SPEC_ERR_ARG;
+  return prefill_impl(h, seq, tokens, n, pending_token, feats_out);
 }
 
 int spec_verify_tree_batch(spec_handle* h, int B, const int32_t* seq_ids, const int32_t* tokens,
@@ -1410,20 +1434,23 @@ int spec_score_trees(spec_handle* h, int B, const int32_t* seq_ids, const int32_
   return SPEC_OK;
 }
 
-int spec_draft_prefill(spec_handle* h, int seq, const void* feats, const int32_t* tokens, int n) {
+static int draft_rows_impl(spec_handle* h, int seq, const void* feats, const int32_t* tokens, int n, bool reset) {
   if (!h) return SPEC_ERR_ARG;
   h->err.clear();
   const spec_config& c = h->cfg;
   if (!c.draft_head) return fail(h, SPEC_ERR_STATE, "the handle was created without the draft head");
   if (!feats || !tokens || n < 1) return fail(h, SPEC_ERR_ARG, "draft prefill needs n >= 1 rows");
   if (seq < 0 || seq >= c.max_batch) return fail(h, SPEC_ERR_ARG, "seq %d outside [0, %d)", seq, c.max_batch);
-  if (n > c.max_seq) return fail(h, SPEC_ERR_CAPACITY, "draft prefix of %d rows exceeds max_seq %d", n, c.max_seq);
+  const int start = reset ? 0 : h->dlen[seq];
+  if (!reset && !h->dready[seq]) return fail(h, SPEC_ERR_STATE, "sequence %d has no draft prefix", seq);
+  if (start + n > c.max_seq)
+    return fail(h, SPEC_ERR_CAPACITY, "draft prefix of %d rows exceeds max_seq %d", start + n, c.max_seq);
   if (h->stale) {
     int rc = refresh_state(h);
     if (rc) return rc;
   }
-  // chunks of max_nodes rows as chains: each row's K/V at its own position
-  h->dlen[seq] = 0;
+  // chunks of max_nodes rows as chains: each row's K/V at its own position, after the rows before it
+  h->dlen[seq] = start;
   h->dready[seq] = 0;
   const size_t row_bytes = 2 * 3 * (size_t)c.hidden;
   std::vector<int32_t> par(c.max_nodes);
@@ -1438,6 +1465,14 @@ int spec_draft_prefill(spec_handle* h, int seq, const void* feats, const int32_t
   }
   h->dready[seq] = 1;
   return SPEC_OK;
+}
+
+int spec_draft_prefill(spec_handle* h, int seq, const void* feats, const int32_t* tokens, int n) {
+  return draft_rows_impl(h, seq, feats, tokens, n, true);
+}
+
+int spec_draft_append(spec_handle* h, int seq, const void* feats, const int32_t* tokens, int n) {
+  return draft_rows_impl(h, seq, feats, tokens, n, false);
 }
 
 int spec_draft_step(spec_handle* h, int B, const int32_t* seq_ids, const void* feats, const int32_t* tokens,

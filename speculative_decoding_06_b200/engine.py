@@ -115,6 +115,16 @@ class SpecEngine:
         self._check(S.spec_prefill(self.h, seq, _ptr(t), len(t), _ptr(pend)))
         return int(pend[0])
 
+    def prefill_features(self, seq: int, tokens):
+        """Prefill that also returns the draft-head features of every prompt position,
+        a bf16 device tensor [n][3][hidden] (needs feature_layers)."""
+        t = _i32(tokens)
+        feats = torch.empty(len(t), 3, self.dims.hidden, dtype=torch.bfloat16, device="cuda")
+        pend = np.zeros(1, np.int32)
+        self.stream.wait_stream(torch.cuda.current_stream())
+        self._check(S.spec_prefill_features(self.h, seq, _ptr(t), len(t), _ptr(pend), feats.data_ptr()))
+        return int(pend[0]), feats
+
     def verify(self, seq: int, tokens, parents):
         t, p = _i32(tokens), _i32(parents)
         acc_len = np.zeros(1, np.int32)
@@ -226,6 +236,43 @@ class SpecEngine:
         f = feats.contiguous()
         self.stream.wait_stream(torch.cuda.current_stream())
         self._check(S.spec_draft_prefill(self.h, seq, f.data_ptr(), _ptr(t), len(t)))
+
+    def draft_append(self, seq: int, feats: torch.Tensor, tokens):
+        """Extend the draft prefix by rows of features [n][3][d] and their next tokens."""
+        t = _i32(tokens)
+        f = feats.contiguous()
+        self.stream.wait_stream(torch.cuda.current_stream())
+        self._check(S.spec_draft_append(self.h, seq, f.data_ptr(), _ptr(t), len(t)))
+
+    def speculative_decode(self, seq: int, prompt, n_new: int, steps: int = 8, topk: int = 10, total: int = 60):
+        """Greedy EAGLE-3 decoding of one sequence through the library.
+
+        Prefill with features; the draft prefix holds one row per position but the
+        last: row p is the fused features of position p with the embedding of token
+        p + 1.  Each decoding step drafts a tree rooted at the pending token from the
+        features of the last verified position, verifies it (returning the features
+        of the root and the accepted nodes), and appends the rows the step verified.
+        Returns (emitted tokens, accepted draft tokens per step), the first emitted
+        token being the prefill's pending token."""
+        p = _i32(prompt)
+        T = len(p)
+        if T < 2:
+            raise ValueError("the prompt needs at least two tokens")
+        pend, feats = self.prefill_features(seq, p)
+        self.draft_prefill(seq, feats[:T - 1], p[1:])
+        last = feats[T - 1:T].clone()
+        emitted, accepted = [pend], []
+        while len(emitted) < n_new + 1:
+            tok, par, _ = self.draft_tree([seq], last, [pend], steps=steps, topk=topk, total=total)
+            acc_len, _, acc_tok, bonus, F = self.verify_batch([seq], [(tok[0], par[0])], features=True)
+            a = int(acc_len[0])
+            acc = [int(x) for x in acc_tok[0, :a]]
+            self.draft_append(seq, torch.cat([last, F[0, :a]], dim=0), [pend] + acc)
+            last = F[0, a:a + 1].clone()
+            pend = int(bonus[0])
+            emitted += acc + [pend]
+            accepted.append(a)
+        return emitted, accepted
 
     def draft_step(self, seq_ids, feats: torch.Tensor, trees, flags: int = 0):
         """Host outputs top_idx [nodes][10] int32, top_val [nodes][10] fp32, node offsets."""

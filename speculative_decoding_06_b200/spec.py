@@ -76,6 +76,7 @@ _SIGNATURES = {
     "spec_init": (ctypes.c_int, [ctypes.POINTER(spec_config), ctypes.POINTER(spec_weights), _vp, ctypes.c_size_t,
                                  _vp, ctypes.c_size_t, _vp, ctypes.POINTER(_h)]),
     "spec_prefill": (ctypes.c_int, [_h, ctypes.c_int, _i32p, ctypes.c_int, _i32p]),
+    "spec_prefill_features": (ctypes.c_int, [_h, ctypes.c_int, _i32p, ctypes.c_int, _i32p, _vp]),
     "spec_verify_tree": (ctypes.c_int, [_h, ctypes.c_int, _i32p, _i32p, ctypes.c_int, _i32p, _i32p, _i32p]),
     "spec_verify_tree_batch": (ctypes.c_int, [_h, ctypes.c_int, _i32p, _i32p, _i32p, _i32p, _vp, _vp, _vp, _vp,
                                               ctypes.c_int]),
@@ -98,6 +99,7 @@ _SIGNATURES = {
     "spec_draft_prefill": (ctypes.c_int, [_h, ctypes.c_int, _vp, _i32p, ctypes.c_int]),
     "spec_draft_step": (ctypes.c_int, [_h, ctypes.c_int, _i32p, _vp, _i32p, _i32p, _i32p, _vp, _vp, ctypes.c_int]),
     "spec_draft_len": (ctypes.c_int, [_h, ctypes.c_int, _i32p]),
+    "spec_draft_append": (ctypes.c_int, [_h, ctypes.c_int, _vp, _i32p, ctypes.c_int]),
     "spec_draft_tree": (ctypes.c_int, [_h, ctypes.c_int, _i32p, _vp, _i32p, ctypes.c_int, ctypes.c_int, ctypes.c_int,
                                        _i32p, _i32p, _f32p]),
     "spec_wait_selftest": (ctypes.c_int, [_vp, ctypes.c_uint32, _i32p]),
