@@ -719,6 +719,9 @@ def run_decode(args):
         e0 = torch.cuda.Event(enable_timing=True)
         e1 = torch.cuda.Event(enable_timing=True)
         torch.cuda.synchronize()
+        timed = i >= max(3, args.warmup)
+        if timed:
+            torch.cuda.nvtx.range_push("timed_step")
         e0.record(eng.stream)
         tok, par, _ = eng.draft_tree([0], last, [pend], steps=steps, topk=K, total=total)
         acc_len, _, acc_tok, bonus, F = eng.verify_batch([0], [(tok[0], par[0])], features=True)
@@ -728,8 +731,10 @@ def run_decode(args):
         last = F[0, a:a + 1].clone()
         pend = int(bonus[0])
         e1.record(eng.stream)
+        if timed:
+            torch.cuda.nvtx.range_pop()
         e1.synchronize()
-        if i >= max(3, args.warmup):
+        if timed:
             times.append(e0.elapsed_time(e1))
             accs.append(a)
     clk.end()

@@ -101,11 +101,13 @@ __device__ __forceinline__ bool offer_before(float va, int oa, float vb, int ob)
 
 // One CTA per tree.  Step t: tree b has n nodes (rows b * n .. b * n + n - 1 of
 // this step); the nodes n - nf .. n - 1 joined last and offer their K best
-// tokens; the K best offers join as nodes n .. n + K - 1; the next step's tree
-// (n + K nodes) is written to tokens_next / parents_next at rows b * (n + K).
+// tokens; the K best offers join as nodes n .. n + K - 1; the next step's trees
+// (n + K nodes each) go to the parameter block: tokens and parents at rows
+// b * (n + K), node offsets b * (n + K).
 __global__ void tree_expand_kernel(TreeArgs a, int t, int n, int nf, const int32_t* __restrict__ top_i,
                                    const float* __restrict__ top_v, const float* __restrict__ lse,
-                                   int32_t* __restrict__ tokens_io, int32_t* __restrict__ parents_io) {
+                                   int32_t* __restrict__ tokens_io, int32_t* __restrict__ parents_io,
+                                   int32_t* __restrict__ node_off_io) {
   pdl_wait();
   pdl_launch_dependents();
   const int b = blockIdx.x;
@@ -175,16 +177,19 @@ __global__ void tree_expand_kernel(TreeArgs a, int t, int n, int nf, const int32
       tokens_io[(size_t)b * nn + i] = tok[i];
       parents_io[(size_t)b * nn + i] = par[i];
     }
+    if (b == 0)
+      for (int i = q; i <= (int)gridDim.x; i += blockDim.x) node_off_io[i] = i * nn;
   }
 }
 
 cudaError_t launch_tree_expand(const TreeArgs& a, int B, int t, int n, int nf, const int32_t* top_i,
                                const float* top_v, const float* lse, int32_t* tokens_io, int32_t* parents_io,
-                               cudaStream_t s, bool pdl) {
+                               int32_t* node_off_io, cudaStream_t s, bool pdl) {
   if (nf * a.K > 256 || a.K > kTopKMax || n + a.K > a.max_nodes) return cudaErrorInvalidValue;
   cudaLaunchAttribute attr[1];
   cudaLaunchConfig_t cfg = make_cfg(dim3(B), dim3(256), 0, s, pdl, attr);
-  return cudaLaunchKernelEx(&cfg, tree_expand_kernel, a, t, n, nf, top_i, top_v, lse, tokens_io, parents_io);
+  return cudaLaunchKernelEx(&cfg, tree_expand_kernel, a, t, n, nf, top_i, top_v, lse, tokens_io, parents_io,
+                            node_off_io);
 }
 
 // ---------------------------------------------------------------------------

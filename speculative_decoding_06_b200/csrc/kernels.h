@@ -204,7 +204,7 @@ cudaError_t launch_tree_feature_rows(int M, int d, int ld, int n, int n_prev, co
                                      cudaStream_t s, bool pdl);
 cudaError_t launch_tree_expand(const TreeArgs& a, int B, int t, int n, int nf, const int32_t* top_i,
                                const float* top_v, const float* lse, int32_t* tokens_io, int32_t* parents_io,
-                               cudaStream_t s, bool pdl);
+                               int32_t* node_off_io, cudaStream_t s, bool pdl);
 cudaError_t launch_tree_rerank(const TreeArgs& a, int B, int total, int32_t* out_tok, int32_t* out_par,
                                float* out_val, cudaStream_t s, bool pdl);
 // x += sum of split partials; xn = RMSNorm(x) * w

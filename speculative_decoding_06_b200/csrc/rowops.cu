@@ -516,7 +516,7 @@ __device__ __forceinline__ void warp_merge_topk(const float (&lv)[K], const int 
 }
 }  // namespace
 
-template <int K, bool LSE>
+template <int K, bool LSE, int U>
 __global__ void __launch_bounds__(256) topk_rows_kernel(int V, const float* __restrict__ logits, size_t ld,
                                                        int32_t* __restrict__ out_i, float* __restrict__ out_v,
                                                        float* __restrict__ out_lse) {
@@ -609,15 +609,16 @@ __global__ void __launch_bounds__(256) topk_rows_kernel(int V, const float* __re
     ls += fast_exp2((e0 - lm) * kLog2e) + fast_exp2((e1 - lm) * kLog2e) + fast_exp2((e2 - lm) * kLog2e) +
           fast_exp2((e3 - lm) * kLog2e);
   };
-  for (int g0 = threadIdx.x; g0 < V4; g0 += 2 * blockDim.x) {
-    float4 x[2];
+  constexpr int kU = U;  // float4 loads in flight per thread (more when few rows leave SMs idle)
+  for (int g0 = threadIdx.x; g0 < V4; g0 += kU * blockDim.x) {
+    float4 x[kU];
 #pragma unroll
-    for (int u = 0; u < 2; ++u) {
+    for (int u = 0; u < kU; ++u) {
       const int g = g0 + u * blockDim.x;
       x[u] = g < V4 ? __ldcs(row4 + g) : make_float4(-INFINITY, -INFINITY, -INFINITY, -INFINITY);
     }
 #pragma unroll
-    for (int u = 0; u < 2; ++u) {
+    for (int u = 0; u < kU; ++u) {
       const float m = fmaxf(fmaxf(x[u].x, x[u].y), fmaxf(x[u].z, x[u].w));
       if (LSE && m > -INFINITY) lse_add(m, x[u].x, x[u].y, x[u].z, x[u].w);
       if (m >= thr) {
@@ -686,19 +687,33 @@ cudaError_t launch_topk_rows(int M, int V, const float* logits, size_t ld, int k
   if (k < 1 || k > kTopKMax || k > V) return cudaErrorInvalidValue;
   cudaLaunchAttribute attr[1];
   cudaLaunchConfig_t cfg = make_cfg(dim3(M), dim3(256), 0, s, pdl, attr);
+  // few rows leave SMs idle: each CTA then keeps more of its row in flight
+  const bool few = M <= 256;
   switch (k) {  // the list length is a compile-time constant of the kernel
     case 10:
-      return lse ? cudaLaunchKernelEx(&cfg, topk_rows_kernel<10, true>, V, logits, ld, idx, val, lse)
-                 : cudaLaunchKernelEx(&cfg, topk_rows_kernel<10, false>, V, logits, ld, idx, val, lse);
+      if (few)
+        return lse ? cudaLaunchKernelEx(&cfg, topk_rows_kernel<10, true, 4>, V, logits, ld, idx, val, lse)
+                   : cudaLaunchKernelEx(&cfg, topk_rows_kernel<10, false, 4>, V, logits, ld, idx, val, lse);
+      return lse ? cudaLaunchKernelEx(&cfg, topk_rows_kernel<10, true, 2>, V, logits, ld, idx, val, lse)
+                 : cudaLaunchKernelEx(&cfg, topk_rows_kernel<10, false, 2>, V, logits, ld, idx, val, lse);
     case 16:
-      return lse ? cudaLaunchKernelEx(&cfg, topk_rows_kernel<16, true>, V, logits, ld, idx, val, lse)
-                 : cudaLaunchKernelEx(&cfg, topk_rows_kernel<16, false>, V, logits, ld, idx, val, lse);
+      if (few)
+        return lse ? cudaLaunchKernelEx(&cfg, topk_rows_kernel<16, true, 4>, V, logits, ld, idx, val, lse)
+                   : cudaLaunchKernelEx(&cfg, topk_rows_kernel<16, false, 4>, V, logits, ld, idx, val, lse);
+      return lse ? cudaLaunchKernelEx(&cfg, topk_rows_kernel<16, true, 2>, V, logits, ld, idx, val, lse)
+                 : cudaLaunchKernelEx(&cfg, topk_rows_kernel<16, false, 2>, V, logits, ld, idx, val, lse);
     case 8:
-      return lse ? cudaLaunchKernelEx(&cfg, topk_rows_kernel<8, true>, V, logits, ld, idx, val, lse)
-                 : cudaLaunchKernelEx(&cfg, topk_rows_kernel<8, false>, V, logits, ld, idx, val, lse);
+      if (few)
+        return lse ? cudaLaunchKernelEx(&cfg, topk_rows_kernel<8, true, 4>, V, logits, ld, idx, val, lse)
+                   : cudaLaunchKernelEx(&cfg, topk_rows_kernel<8, false, 4>, V, logits, ld, idx, val, lse);
+      return lse ? cudaLaunchKernelEx(&cfg, topk_rows_kernel<8, true, 2>, V, logits, ld, idx, val, lse)
+                 : cudaLaunchKernelEx(&cfg, topk_rows_kernel<8, false, 2>, V, logits, ld, idx, val, lse);
     case 4:
-      return lse ? cudaLaunchKernelEx(&cfg, topk_rows_kernel<4, true>, V, logits, ld, idx, val, lse)
-                 : cudaLaunchKernelEx(&cfg, topk_rows_kernel<4, false>, V, logits, ld, idx, val, lse);
+      if (few)
+        return lse ? cudaLaunchKernelEx(&cfg, topk_rows_kernel<4, true, 4>, V, logits, ld, idx, val, lse)
+                   : cudaLaunchKernelEx(&cfg, topk_rows_kernel<4, false, 4>, V, logits, ld, idx, val, lse);
+      return lse ? cudaLaunchKernelEx(&cfg, topk_rows_kernel<4, true, 2>, V, logits, ld, idx, val, lse)
+                 : cudaLaunchKernelEx(&cfg, topk_rows_kernel<4, false, 2>, V, logits, ld, idx, val, lse);
     default: return cudaErrorInvalidValue;
   }
 }

@@ -1535,30 +1535,27 @@ int spec_draft_tree(spec_handle* h, int B, const int32_t* seq_ids, const void* r
   ta.val = h->W<float>(L.tr_val);
   ta.offers = h->W<TreeOffer>(L.tr_offers);
   ta.n_offers = h->W<int32_t>(L.tr_noff);
-  for (int t = 0; t < steps; ++t) {
-    const int n = 1 + t * topk, M = B * n;
+  // the parameter block is uploaded once: each expansion writes the next step's
+  // trees and node offsets on the device, so the steps queue back to back
+  {
     uint8_t* pb = h->h_params;
+    int32_t* tk = reinterpret_cast<int32_t*>(pb + L.p_tokens);
+    int32_t* pr = reinterpret_cast<int32_t*>(pb + L.p_parents);
     int32_t* no = reinterpret_cast<int32_t*>(pb + L.p_node_off);
-    for (int b = 0; b <= B; ++b) no[b] = b * n;
+    for (int b = 0; b < B; ++b) {
+      tk[b] = root_tokens[b];
+      pr[b] = -1;
+    }
+    for (int b = 0; b <= B; ++b) no[b] = b;
     std::memcpy(pb + L.p_seq_ids, seq_ids, 4 * (size_t)B);
     std::memcpy(pb + L.p_dlen, h->dlen.data(), 4 * (size_t)c.max_batch);
     std::memset(pb + L.p_err, 0, 16);
-    if (t == 0) {
-      // step 0: one root per tree; a later step's tokens and parents were written on
-      // the device by the previous expansion
-      int32_t* tk = reinterpret_cast<int32_t*>(pb + L.p_tokens);
-      int32_t* pr = reinterpret_cast<int32_t*>(pb + L.p_parents);
-      for (int b = 0; b < B; ++b) {
-        tk[b] = root_tokens[b];
-        pr[b] = -1;
-      }
-      CUDA_TRY(h, cudaMemcpyAsync(h->ws, pb, L.p_end, cudaMemcpyHostToDevice, st));
-      CUDA_TRY(h, launch_split_rows(static_cast<const __nv_bfloat16*>(root_feats), B, 3 * c.hidden,
-                                    h->W<__nv_bfloat16>(L.fsplit), st, false));
-    } else {
-      CUDA_TRY(h, cudaMemcpyAsync(h->ws + L.p_node_off, pb + L.p_node_off, L.p_end - L.p_node_off,
-                                  cudaMemcpyHostToDevice, st));
-    }
+    CUDA_TRY(h, cudaMemcpyAsync(h->ws, pb, L.p_end, cudaMemcpyHostToDevice, st));
+    CUDA_TRY(h, launch_split_rows(static_cast<const __nv_bfloat16*>(root_feats), B, 3 * c.hidden,
+                                  h->W<__nv_bfloat16>(L.fsplit), st, false));
+  }
+  for (int t = 0; t < steps; ++t) {
+    const int n = 1 + t * topk, M = B * n;
     const StepPlan sp = make_plan(h, B, M, n, max_dlen + n);
     TreeStep ts{t, n, t ? 1 + (t - 1) * topk : 0, topk, ta};
     ts.args.write_next = t + 1 < steps ? 1 : 0;
@@ -1567,15 +1564,9 @@ int spec_draft_tree(spec_handle* h, int B, const int32_t* seq_ids, const void* r
       e = launch_k(h, SPEC_PROF_TREE, 1, [&]() {
         return launch_tree_expand(ts.args, B, t, n, t == 0 ? 1 : topk, h->W<int32_t>(L.tr_top_i),
                                   h->W<float>(L.tr_top_v), h->W<float>(L.tr_lse), h->W<int32_t>(L.p_tokens),
-                                  h->W<int32_t>(L.p_parents), st, false);
+                                  h->W<int32_t>(L.p_parents), h->W<int32_t>(L.p_node_off), st, false);
       });
     if (e != cudaSuccess) return fail(h, SPEC_ERR_CUDA, "kernel launch failed: %s", cudaGetErrorString(e));
-    // the host parameter block is rewritten by the next step: let this step's copy finish
-    uint32_t errw[2] = {0, 0};
-    CUDA_TRY(h, cudaMemcpyAsync(errw, h->ws + L.p_err, 4, cudaMemcpyDeviceToHost, st));
-    CUDA_TRY(h, cudaStreamSynchronize(st));
-    if (errw[0] & SPEC_DEVERR_TIMEOUT) return fail(h, SPEC_ERR_TIMEOUT, "a bounded wait expired on the device");
-    if (errw[0]) return fail(h, SPEC_ERR_CUDA, "device reported error bits 0x%x", errw[0]);
   }
   const size_t no_ = (size_t)B * (total + 1);
   cudaError_t e = launch_k(h, SPEC_PROF_TREE, 1, [&]() {
@@ -1586,7 +1577,11 @@ int spec_draft_tree(spec_handle* h, int B, const int32_t* seq_ids, const void* r
   CUDA_TRY(h, cudaMemcpyAsync(out_tokens, h->ws + L.tr_out_tok, 4 * no_, cudaMemcpyDeviceToHost, st));
   CUDA_TRY(h, cudaMemcpyAsync(out_parents, h->ws + L.tr_out_par, 4 * no_, cudaMemcpyDeviceToHost, st));
   if (out_values) CUDA_TRY(h, cudaMemcpyAsync(out_values, h->ws + L.tr_out_val, 4 * no_, cudaMemcpyDeviceToHost, st));
+  uint32_t errw[2] = {0, 0};
+  CUDA_TRY(h, cudaMemcpyAsync(errw, h->ws + L.p_err, 4, cudaMemcpyDeviceToHost, st));
   CUDA_TRY(h, cudaStreamSynchronize(st));
+  if (errw[0] & SPEC_DEVERR_TIMEOUT) return fail(h, SPEC_ERR_TIMEOUT, "a bounded wait expired on the device");
+  if (errw[0]) return fail(h, SPEC_ERR_CUDA, "device reported error bits 0x%x", errw[0]);
   for (int b = 0; b < B; ++b)
     if (spec_validate_tree(out_tokens + (size_t)b * (total + 1), out_parents + (size_t)b * (total + 1), total + 1,
                            c.vocab, c.max_nodes) != SPEC_OK)
