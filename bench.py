@@ -695,8 +695,9 @@ def run_draft_tree(args):
 
 
 def run_decode(args):
-    """The closed loop at the 8B shape, batch 1, prefix 2048: per step a dynamic draft tree
-    (8 steps of top-10, 60 nodes), its verification with features, the draft-prefix update."""
+    """The closed loop at the 8B shape, prefix 2048, `--batch` sequences: per step one dynamic
+    draft tree per sequence (8 steps of top-10, 60 nodes), their verification with features,
+    the draft-prefix updates."""
     import torch
     from speculative_decoding_06_b200.engine import SpecEngine
     dims = synth.LLAMA8B
@@ -705,12 +706,17 @@ def run_decode(args):
     w = synth.model_weights(dims, seed=0, device="cuda")
     dw = synth.draft_head_weights(dims, seed=6, device="cuda")
     L = dims.n_layers
-    eng = SpecEngine(dims, w, max_batch=1, max_seq=P + 64 * (n_steps + 2), max_nodes=128, draft=dw,
+    B = args.batch
+    eng = SpecEngine(dims, w, max_batch=B, max_seq=P + 64 * (n_steps + 2), max_nodes=128, draft=dw,
                      feature_layers=(2, L // 2, L - 3))
-    prompt = synth.prefix_tokens(dims.vocab, P, seed=1)
-    pend, feats = eng.prefill_features(0, prompt)
-    eng.draft_prefill(0, feats[:P - 1], prompt[1:])
-    last = feats[P - 1:P].clone()
+    ids = list(range(B))
+    pend, last = [], []
+    for b in ids:
+        prompt = synth.prefix_tokens(dims.vocab, P, seed=1, stream=b)
+        pb, feats = eng.prefill_features(b, prompt)
+        eng.draft_prefill(b, feats[:P - 1], prompt[1:])
+        pend.append(pb)
+        last.append(feats[P - 1:P].clone())
     times, accs = [], []
     clk = ClockSampler(gpu_uuid(0))
     for i in range(n_steps):
@@ -723,13 +729,15 @@ def run_decode(args):
         if timed:
             torch.cuda.nvtx.range_push("timed_step")
         e0.record(eng.stream)
-        tok, par, _ = eng.draft_tree([0], last, [pend], steps=steps, topk=K, total=total)
-        acc_len, _, acc_tok, bonus, F = eng.verify_batch([0], [(tok[0], par[0])], features=True)
-        a = int(acc_len[0])
-        acc = [int(x) for x in acc_tok[0, :a]]
-        eng.draft_append(0, torch.cat([last, F[0, :a]], dim=0), [pend] + acc)
-        last = F[0, a:a + 1].clone()
-        pend = int(bonus[0])
+        tok, par, _ = eng.draft_tree(ids, torch.cat(last, dim=0), pend, steps=steps, topk=K, total=total)
+        acc_len, _, acc_tok, bonus, F = eng.verify_batch(ids, [(tok[b], par[b]) for b in ids], features=True)
+        for b in ids:
+            a = int(acc_len[b])
+            acc = [int(x) for x in acc_tok[b, :a]]
+            eng.draft_append(b, torch.cat([last[b], F[b, :a]], dim=0), [pend[b]] + acc)
+            last[b] = F[b, a:a + 1].clone()
+            pend[b] = int(bonus[b])
+        a = float(np.mean(acc_len[:B]))
         e1.record(eng.stream)
         if timed:
             torch.cuda.nvtx.range_pop()
@@ -741,10 +749,11 @@ def run_decode(args):
     clocks = clk.stop()
     ms = float(np.mean(times))
     tau = float(np.mean(accs)) + 1.0
-    print(json.dumps({"workload": "EAGLE-3 greedy decoding loop at 8B shape bf16, batch 1, prefix 2048: dynamic "
-                                  "draft tree (8 steps, top-10, 60 nodes) + verification with features + draft-prefix "
-                                  "update per step; random-init draft head, so few drafts are accepted",
-                      "ms_per_decode_step": ms, "tau": tau, "tokens_per_s": tau * 1000.0 / ms,
+    print(json.dumps({"workload": "EAGLE-3 greedy decoding loop at 8B shape bf16, batch %d, prefix 2048: dynamic "
+                                  "draft tree (8 steps, top-10, 60 nodes) per sequence + verification with features + "
+                                  "draft-prefix update per step; random-init draft head, so few drafts are "
+                                  "accepted" % B,
+                      "batch": B, "ms_per_decode_step": ms, "tau": tau, "tokens_per_s": B * tau * 1000.0 / ms,
                       "steps": len(times), "clocks": clocks,
                       "data": "synthetic"}))
     eng.close()
@@ -760,6 +769,7 @@ def main():
     ap.add_argument("--prefix", type=int, default=2048)
     ap.add_argument("--sample-layers", type=int, default=2)
     ap.add_argument("--no-cpu-baseline", action="store_true")
+    ap.add_argument("--batch", type=int, default=1, help="sequences decoded together (--workload decode)")
     ap.add_argument("--layers", type=int, default=32, help="decoder layers (32 = the 8B shape; fewer only for profiling)")
     ap.add_argument("--workload", default="verify", choices=["verify", "batch64", "sweep", "draft", "draft_tree", "decode"],
                     help="verify: the default line (batch 1, prefix 2048); the others measure the remaining"

@@ -245,34 +245,51 @@ class SpecEngine:
         self._check(S.spec_draft_append(self.h, seq, f.data_ptr(), _ptr(t), len(t)))
 
     def speculative_decode(self, seq: int, prompt, n_new: int, steps: int = 8, topk: int = 10, total: int = 60):
-        """Greedy EAGLE-3 decoding of one sequence through the library.
+        """Greedy EAGLE-3 decoding of one sequence (see speculative_decode_batch)."""
+        emitted, accepted = self.speculative_decode_batch([seq], [prompt], n_new, steps, topk, total)
+        return emitted[0], accepted[0]
 
-        Prefill with features; the draft prefix holds one row per position but the
-        last: row p is the fused features of position p with the embedding of token
-        p + 1.  Each decoding step drafts a tree rooted at the pending token from the
-        features of the last verified position, verifies it (returning the features
-        of the root and the accepted nodes), and appends the rows the step verified.
-        Returns (emitted tokens, accepted draft tokens per step), the first emitted
-        token being the prefill's pending token."""
-        p = _i32(prompt)
-        T = len(p)
-        if T < 2:
-            raise ValueError("the prompt needs at least two tokens")
-        pend, feats = self.prefill_features(seq, p)
-        self.draft_prefill(seq, feats[:T - 1], p[1:])
-        last = feats[T - 1:T].clone()
-        emitted, accepted = [pend], []
-        while len(emitted) < n_new + 1:
-            tok, par, _ = self.draft_tree([seq], last, [pend], steps=steps, topk=topk, total=total)
-            acc_len, _, acc_tok, bonus, F = self.verify_batch([seq], [(tok[0], par[0])], features=True)
-            a = int(acc_len[0])
-            acc = [int(x) for x in acc_tok[0, :a]]
-            self.draft_append(seq, torch.cat([last, F[0, :a]], dim=0), [pend] + acc)
-            last = F[0, a:a + 1].clone()
-            pend = int(bonus[0])
-            emitted += acc + [pend]
-            accepted.append(a)
-        return emitted, accepted
+    def speculative_decode_batch(self, seq_ids, prompts, n_new: int, steps: int = 8, topk: int = 10,
+                                 total: int = 60):
+        """Greedy EAGLE-3 decoding of several sequences at once, through the library.
+
+        Prefill each prompt with features; a sequence's draft prefix holds one row per
+        position but the last: row p is the fused features of position p with the
+        embedding of token p + 1.  Each decoding step drafts one tree per sequence
+        (rooted at its pending token, from the features of its last verified position),
+        verifies the batch (returning the features of each root and its accepted nodes)
+        and appends to every draft prefix the rows the step verified.  Sequences that
+        have emitted n_new + 1 tokens drop out of later steps.  Returns (emitted tokens
+        per sequence, accepted draft tokens per step per sequence); the first emitted
+        token of a sequence is its prefill's pending token."""
+        ids = [int(s) for s in seq_ids]
+        pend, last, emitted, accepted = {}, {}, {}, {}
+        for s, prompt in zip(ids, prompts):
+            p = _i32(prompt)
+            T = len(p)
+            if T < 2:
+                raise ValueError("every prompt needs at least two tokens")
+            pend[s], feats = self.prefill_features(s, p)
+            self.draft_prefill(s, feats[:T - 1], p[1:])
+            last[s] = feats[T - 1:T].clone()
+            emitted[s], accepted[s] = [pend[s]], []
+        live = [s for s in ids if len(emitted[s]) < n_new + 1]
+        while live:
+            root_feats = torch.cat([last[s] for s in live], dim=0)
+            tok, par, _ = self.draft_tree(live, root_feats, [pend[s] for s in live], steps=steps, topk=topk,
+                                          total=total)
+            acc_len, _, acc_tok, bonus, F = self.verify_batch(live, [(tok[b], par[b]) for b in range(len(live))],
+                                                              features=True)
+            for b, s in enumerate(live):
+                a = int(acc_len[b])
+                acc = [int(x) for x in acc_tok[b, :a]]
+                self.draft_append(s, torch.cat([last[s], F[b, :a]], dim=0), [pend[s]] + acc)
+                last[s] = F[b, a:a + 1].clone()
+                pend[s] = int(bonus[b])
+                emitted[s] += acc + [pend[s]]
+                accepted[s].append(a)
+            live = [s for s in live if len(emitted[s]) < n_new + 1]
+        return [emitted[s] for s in ids], [accepted[s] for s in ids]
 
     def draft_step(self, seq_ids, feats: torch.Tensor, trees, flags: int = 0):
         """Host outputs top_idx [nodes][10] int32, top_val [nodes][10] fp32, node offsets."""

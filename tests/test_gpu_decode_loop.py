@@ -74,3 +74,35 @@ def test_speculative_decode_is_lossless(loop_pair):
     assert ln == len(prompt) + len(emitted) - 1 and pending == emitted[-1]
     assert eng.draft_len(0) == ln - 1
     print("steps %d, accepted per step %s, compared %d tokens" % (len(accepted), accepted, m))
+
+
+def test_speculative_decode_batch_is_lossless():
+    """Two sequences decoded together: each equals its own greedy continuation."""
+    from speculative_decoding_06_b200.engine import SpecEngine
+    d = synth.SMALL_BF16
+    w = synth.model_weights(d, seed=0, device="cuda")
+    dw = synth.draft_head_weights(d, seed=6, device="cuda")
+    eng = SpecEngine(d, w, max_batch=2, max_seq=512, max_nodes=64, draft=dw, feature_layers=TAPS)
+    om = OracleModel(d, synth.weights_to_host(w))
+    try:
+        n = 16
+        prompts, greedys, safes = [], [], []
+        stream = 40
+        while len(prompts) < 2 and stream < 400:
+            prompt = synth.prefix_tokens(om.d.vocab, 30 + 9 * len(prompts), seed=2, stream=stream)
+            greedy, safe = _greedy(om, prompt, n)
+            if safe >= 8:
+                prompts.append(prompt)
+                greedys.append(greedy)
+                safes.append(safe)
+            stream += 1
+        assert len(prompts) == 2
+        emitted, accepted = eng.speculative_decode_batch([1, 0], prompts, n, steps=2, topk=4, total=8)
+        for e, g, safe in zip(emitted, greedys, safes):
+            m = min(len(e), safe)
+            assert e[:m] == g[:m]
+        for s, e in zip([1, 0], emitted):
+            ln, pending = eng.seq_len(s)
+            assert pending == e[-1] and eng.draft_len(s) == ln - 1
+    finally:
+        eng.close()
