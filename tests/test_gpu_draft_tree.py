@@ -56,13 +56,14 @@ def _decisive(tree, steps, topk, total, tol):
     return not (len(v) > total and v[total - 1] - v[total] <= tol)
 
 
-@pytest.mark.parametrize("steps,topk,total", [(3, 4, 8), (2, 8, 12)])
+@pytest.mark.parametrize("steps,topk,total", [(3, 4, 8), (2, 8, 12), (8, 10, 60)])
 def test_draft_tree_matches_oracle(steps, topk, total):
+    """(8, 10, 60) is the pages' evaluated setting: 8 drafting steps, top-10, 60 draft tokens."""
     from speculative_decoding_06_b200.engine import SpecEngine
     d = synth.SMALL_BF16
     wdev = synth.model_weights(d, seed=0, device="cuda")
     dwdev = synth.draft_head_weights(d, seed=6, device="cuda")
-    eng = SpecEngine(d, wdev, max_batch=3, max_seq=512, max_nodes=64, draft=dwdev)
+    eng = SpecEngine(d, wdev, max_batch=3, max_seq=512, max_nodes=128, draft=dwdev)
     oh = OracleDraftHead(d, synth.weights_to_host(wdev),
                          {"fc_fuse": _host(dwdev["fc_fuse"]), "fc_in": _host(dwdev["fc_in"]),
                           "final_norm": _host(dwdev["final_norm"]),
