@@ -102,3 +102,15 @@ def test_validate_tree():
     assert _validate([1, -4], [-1, 0]) == S.SPEC_ERR_TOKEN
     assert _validate(list(range(65)), [-1] + list(range(64))) == S.SPEC_ERR_CAPACITY
     assert _validate([], []) == S.SPEC_ERR_CAPACITY
+
+
+def test_new_entry_points_reject_bad_arguments_without_gpu():
+    """NULL handles and buffers are refused before any CUDA call."""
+    i32 = ctypes.c_int32(0)
+    assert S.spec_draft_tree(None, 1, None, None, None, 8, 10, 60, None, None, None) == S.SPEC_ERR_ARG
+    assert S.spec_prefill_features(None, 0, None, 1, None, None) == S.SPEC_ERR_ARG
+    assert S.spec_draft_append(None, 0, None, None, 1) == S.SPEC_ERR_ARG
+    assert S.spec_set_feature_out(None, None, 0) == S.SPEC_ERR_ARG
+    assert S.spec_wait_selftest(None, 1000, ctypes.byref(i32)) == S.SPEC_ERR_ARG
+    assert S.spec_wait_selftest(ctypes.c_void_p(16), 0, ctypes.byref(i32)) == S.SPEC_ERR_ARG
+    assert S.spec_wait_selftest(ctypes.c_void_p(18), 1000, ctypes.byref(i32)) == S.SPEC_ERR_ARG  # misaligned
