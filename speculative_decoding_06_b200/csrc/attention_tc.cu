@@ -551,11 +551,7 @@ __global__ void __launch_bounds__(kThreads, 1) attn_tc_kernel(const __grid_const
         }
         named_sync_rows();
         stamp(a.trace, 7);
-        // the last chunk CTA to leave resets the group's counters for the next layer
-        if (tid == 0 && atomicAdd(ctr + 1, 1) == nc_b - 1) {
-          ctr[0] = 0;
-          ctr[1] = 0;
-        }
+        // (each layer has its own counters, zeroed with the step: nothing to reset)
       }
     }
   }

@@ -659,16 +659,9 @@ __global__ void __launch_bounds__(kThreads, BN == 64 ? 2 : 1)
             if (t < args.M) args.top_part[(size_t)to * args.top_ld + t] = r;
           }
         }
-        // unit done; the last CTA of a split tile to leave resets the tile's
-        // counters for the next launch
+        // unit done (a phase's arrival counters serve it alone and are zeroed with
+        // the step, so nothing is reset here)
         named_sync(2, 128);  // r_s and the staging areas are reused by the next unit
-        if (ep_tid == 0 && S > 1) {
-          int* ctr = args.counters + 2 * ut;
-          if (atomicAdd(ctr + 1, 1) == S - 1) {
-            ctr[0] = 0;
-            ctr[1] = 0;
-          }
-        }
         if (first_unit && ep_tid == 0) stamp(P.trace, p, 11);
         first_unit = false;
       }

@@ -40,7 +40,7 @@ struct GemmTcArgs {
   // split-K partials [splits][tokens][n_out] and per-tile arrival counters
   float* part;
   size_t split_stride;
-  int* counters;      // [tiles_o * tiles_t], zero between launches
+  int* counters;      // [2 * tiles_o * tiles_t], zero at launch; a phase's own (never reused within a step)
   // SWIGLU, STORE (the accumulator itself, no split-K)
   __nv_bfloat16* out_bf16;  // split bf16 [2 x tokens][ld_out]
   int ld_out;
@@ -235,7 +235,7 @@ struct AttnArgs {
   int q_rows;               // bf16 path: q is [Hkv][q_rows][hd], row node * G + g
   float rescale_slack;      // bf16 path: the running max moves only when a block's max exceeds it by this (log2 units)
   int cluster_merge;        // bf16 path: the n_chunks chunk CTAs of a row tile form a cluster and merge through DSMEM
-  int* counters;            // bf16 path: [groups][2] chunk arrivals / departures, zero between launches
+  int* counters;            // bf16 path: [groups][2] chunk arrivals, zero at launch; a layer's own within a step
   uint64_t* trace;          // optional [256 CTAs][16] %globaltimer marks (attention_tc.cu)
 };
 // fp32 models: one warp per (node, head)

@@ -33,10 +33,11 @@ namespace {
 
 constexpr int kMaxNodesLimit = 128;  // ancestor bitmask is two 64-bit words
 constexpr int kMaxSplits = 16;
-constexpr int kGemmCounters = 8192;  // per-tile arrival counters of the split-K GEMMs
+// split-K arrival counters: one region per (launch, phase) of a step, all zeroed
+// when the step starts, so no kernel has to reset them
 constexpr int kMaxAttnChunks = kAttnMaxChunks;  // key chunks of one (sequence, kv head, row tile)
 constexpr int kDraftTopK = SPEC_DRAFT_TOPK;  // candidates per draft node
-constexpr int kCountersPerPhase = 2048; // two ints per split-K tile
+constexpr int kCountersPerPhase = 1024;  // two ints per split-K tile (<= 2 x 296 resident CTAs)
 
 size_t align_up(size_t x, size_t a) { return (x + a - 1) / a * a; }
 int ceil_div(int a, int b) { return (a + b - 1) / b; }
@@ -53,6 +54,7 @@ struct WsLayout {
   // activations
   size_t x, xn, q, attn, hmlp, partial, part_o, part_lse, top_part, argmax, top1, top2, inv_freq;
   size_t ss, gemm_ctr, attn_ctr, phase_bar;
+  int gemm_ctr_n = 0;  // ints: 4 phases x launches of a step x kCountersPerPhase
   // draft head: split features [2 Mpad][3d], [g|e] operand [2 Mpad][2d], logits, top-k
   size_t fsplit = 0, ge = 0, dlogits = 0, dtop_i = 0, dtop_v = 0;
   // feature tap: bf16 residual stream after the three feature layers [3][Mpad][d]
@@ -123,10 +125,12 @@ WsLayout make_layout(const spec_config& c) {
   L.top_part = take(sizeof(Top2) * (size_t)ceil_div(c.vocab, 128) * L.Mpad);
   L.n_ss = std::max(1, c.hidden / 128);
   L.ss = take(4 * (size_t)L.n_ss * L.Mpad);
-  L.gemm_ctr = take(4 * (size_t)kGemmCounters);
+  // launches of a step: the first QKV and one per layer (verification); three (draft step)
+  L.gemm_ctr_n = 4 * std::max(c.n_layers + 1, 3) * kCountersPerPhase;
+  L.gemm_ctr = take(4 * (size_t)L.gemm_ctr_n);
   L.phase_bar_n = 4 * (c.n_layers + 2);
   L.phase_bar = take(4 * (size_t)L.phase_bar_n);
-  L.attn_ctr_n = 2 * kAttnPartCtas;
+  L.attn_ctr_n = 2 * kAttnPartCtas * (c.n_layers + 1);  // per layer, the draft head's last
 
   L.attn_ctr = take(4 * (size_t)L.attn_ctr_n);
   L.argmax = take(4 * (size_t)L.Mpad);
@@ -517,7 +521,8 @@ struct PhaseBuilder {
     q.args = g.args;
     return q;
   }
-  int* ctr(int slot) const { return h->W<int>(h->lay.gemm_ctr) + slot * kCountersPerPhase; }
+  // counters of phase `slot` of launch `launch` within the step
+  int* ctr(int region) const { return h->W<int>(h->lay.gemm_ctr) + region * kCountersPerPhase; }
   GemmPhase qkv(int l, int slot) const {
     const spec_config& c = h->cfg;
     const WsLayout& L = h->lay;
@@ -635,7 +640,7 @@ cudaError_t enqueue_step(spec_handle* h, const StepPlan& sp, int mode, bool dbg,
   };
   if (dt == 1) {
     // arrival counters start every step at zero, whatever an earlier failed step left behind
-    cudaError_t e0 = cudaMemsetAsync(gctr, 0, 4 * (size_t)kGemmCounters, st);
+    cudaError_t e0 = cudaMemsetAsync(gctr, 0, 4 * (size_t)L.gemm_ctr_n, st);
     if (e0 == cudaSuccess) e0 = cudaMemsetAsync(h->ws + L.attn_ctr, 0, 4 * (size_t)L.attn_ctr_n, st);
     if (e0 == cudaSuccess) e0 = cudaMemsetAsync(h->ws + L.phase_bar, 0, 4 * (size_t)L.phase_bar_n, st);
     if (e0 != cudaSuccess) return e0;
@@ -677,6 +682,7 @@ cudaError_t enqueue_step(spec_handle* h, const StepPlan& sp, int mode, bool dbg,
     const spec_layer_weights& lw = h->layers[l];
     const void* next_norm = (l + 1 < c.n_layers) ? h->layers[l + 1].attn_norm : h->final_norm;
     aa.layer = l;
+    aa.counters = h->W<int>(L.attn_ctr) + (size_t)l * 2 * kAttnPartCtas;  // this layer's own
     if (dt == 1) {
       // attention of layer l (its QKV ran in the previous launch), then one
       // launch: O, gate/up, down, and the next layer's QKV or the LM head
@@ -692,10 +698,11 @@ cudaError_t enqueue_step(spec_handle* h, const StepPlan& sp, int mode, bool dbg,
       m.err = sv.err;
       m.phase_bar = h->W<int>(L.phase_bar) + 4 * (l + 1);
       m.n_phases = 4;
-      m.ph[0] = pb.o(l, 0);
+      // split-K counter regions 4 * (l + 1) + phase (region 0 is the first QKV launch's)
+      m.ph[0] = pb.o(l, 4 * (l + 1) + 0);
       m.ph[1] = pb.gu(l);
-      m.ph[2] = pb.down(l, 2, next_norm);
-      m.ph[3] = (l + 1 < c.n_layers) ? pb.qkv(l + 1, 3) : pb.lm(dbg ? h->dbg_logits : nullptr);
+      m.ph[2] = pb.down(l, 4 * (l + 1) + 2, next_norm);
+      m.ph[3] = (l + 1 < c.n_layers) ? pb.qkv(l + 1, 4 * (l + 1) + 3) : pb.lm(dbg ? h->dbg_logits : nullptr);
       if (h->trace && l == h->trace_layer) m.trace = h->trace;
       LK(SPEC_PROF_GEMM_LAYER, 1, gemm_multi_launch(m, st, pdl));
       CUDA_RET(tap_after(l + 1, pdl));
@@ -783,7 +790,7 @@ cudaError_t enqueue_draft(spec_handle* h, const StepPlan& sp, bool kv_only, bool
   const int d = c.hidden, M = sp.M, Ld = c.n_layers;
   const int bi = sp.qkv.bn == 64 ? 0 : 1;
   h->launches = 0;
-  CUDA_RET(cudaMemsetAsync(h->ws + L.gemm_ctr, 0, 4 * (size_t)kGemmCounters, st));
+  CUDA_RET(cudaMemsetAsync(h->ws + L.gemm_ctr, 0, 4 * (size_t)L.gemm_ctr_n, st));
   CUDA_RET(cudaMemsetAsync(h->ws + L.attn_ctr, 0, 4 * (size_t)L.attn_ctr_n, st));
   CUDA_RET(cudaMemsetAsync(h->ws + L.phase_bar, 0, 4 * (size_t)L.phase_bar_n, st));
   __nv_bfloat16* ge = h->W<__nv_bfloat16>(L.ge);
@@ -830,7 +837,7 @@ cudaError_t enqueue_draft(spec_handle* h, const StepPlan& sp, bool kv_only, bool
   m.err = sv.err;
   m.phase_bar = h->W<int>(L.phase_bar) + 4 * (c.n_layers + 1);
   m.n_phases = 1;
-  m.ph[0] = pb.qkv(Ld, 1);
+  m.ph[0] = pb.qkv(Ld, 4 + 1);
   LK(SPEC_PROF_GEMM_QKV, 1, gemm_multi_launch(m, st, pdl));
   if (kv_only) return cudaSuccess;
 
@@ -847,16 +854,16 @@ cudaError_t enqueue_draft(spec_handle* h, const StepPlan& sp, bool kv_only, bool
   aa.n_chunks = sp.n_chunks;
   aa.chunk = sp.chunk;
   aa.max_rows = sp.max_rows;
-  aa.counters = h->W<int>(L.attn_ctr);
+  aa.counters = h->W<int>(L.attn_ctr) + (size_t)Ld * 2 * kAttnPartCtas;  // the draft layer's own
   aa.q_rows = L.Mpad * (c.n_q_heads / c.n_kv_heads);
   aa.rescale_slack = h->rescale_slack;
   aa.cluster_merge = sp.cluster_merge;
   LK(SPEC_PROF_ATTENTION, 1, launch_attention_tc(aa, h->attn_maps, st, pdl));
   float* logits = h->W<float>(L.dlogits);
   m.n_phases = 4;
-  m.ph[0] = pb.o(Ld, 0);
+  m.ph[0] = pb.o(Ld, 8 + 0);
   m.ph[1] = pb.gu(Ld);
-  m.ph[2] = pb.down(Ld, 2, h->draft_final_norm);
+  m.ph[2] = pb.down(Ld, 8 + 2, h->draft_final_norm);
   m.ph[3] = pb.lm(logits);
   LK(SPEC_PROF_GEMM_LAYER, 1, gemm_multi_launch(m, st, pdl));
   if (ts)
@@ -1235,7 +1242,7 @@ int spec_init(const spec_config* cfg, const spec_weights* w, void* kv_cache, siz
   if (cudaMemsetAsync(h->ws + lay.seq_len, 0, 4 * (size_t)c.max_batch, h->stream) != cudaSuccess ||
       cudaMemsetAsync(h->ws + lay.pending, 0xff, 4 * (size_t)c.max_batch, h->stream) != cudaSuccess ||
       cudaMemsetAsync(h->ws + lay.err_sticky, 0, 16, h->stream) != cudaSuccess ||
-      cudaMemsetAsync(h->ws + lay.gemm_ctr, 0, 4 * (size_t)kGemmCounters, h->stream) != cudaSuccess ||
+      cudaMemsetAsync(h->ws + lay.gemm_ctr, 0, 4 * (size_t)lay.gemm_ctr_n, h->stream) != cudaSuccess ||
       cudaMemsetAsync(h->ws + lay.attn_ctr, 0, 4 * (size_t)lay.attn_ctr_n, h->stream) != cudaSuccess ||
 
       cudaMemcpyAsync(h->ws + lay.inv_freq, inv.data(), 8 * inv.size(), cudaMemcpyHostToDevice, h->stream) !=
