@@ -139,7 +139,7 @@ __global__ void tree_expand_kernel(TreeArgs a, int t, int n, int nf, const int32
     o.node = -1;
     off[base + q] = o;
   }
-  // K rounds of a block-wide best (value desc, order asc)
+  // K block-wide selections of the best offer (value desc, order asc)
   for (int k = 0; k < K; ++k) {
     sv[q] = v;
     so[q] = order;
@@ -154,7 +154,7 @@ __global__ void tree_expand_kernel(TreeArgs a, int t, int n, int nf, const int32
     if (q == 0) taken[k] = so[0];
     __syncthreads();
     if (order == taken[k]) {
-      v = -INFINITY;  // out of the next rounds
+      v = -INFINITY;  // out of the remaining selections
       order = 0x7fffffff;
     }
     __syncthreads();
