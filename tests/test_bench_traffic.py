@@ -35,7 +35,3 @@ def test_no_traffic_once_the_source_changed(tmp_path, monkeypatch):
     monkeypatch.setattr(bench, "ROOT", str(tmp_path))
     assert bench.measured_traffic("gemm_layer", 5000.0) is None
 
-
-def test_committed_record_matches_the_committed_kernel():
-    """The repository's own record is live: the GEMM source is the captured one."""
-    assert bench.measured_traffic("gemm_layer", 1.0) is not None
