@@ -199,7 +199,9 @@ SPEC_API int spec_score_trees(spec_handle* h, int B, const int32_t* seq_ids, con
 SPEC_API int spec_draft_prefill(spec_handle* h, int seq, const void* feats, const int32_t* tokens, int n);
 /* As spec_draft_prefill, but the n rows extend the draft prefix of `seq` (positions len ..
  * len + n - 1, attending to the rows before them): the rows a verification step adds.
- * SPEC_ERR_STATE when the sequence has no draft prefix; SPEC_ERR_CAPACITY past max_seq. */
+ * SPEC_ERR_STATE when the sequence has no draft prefix; SPEC_ERR_CAPACITY past max_seq (both
+ * before any work, the prefix unchanged).  An error during the work leaves the prefix marked
+ * unusable: rebuild it with spec_draft_prefill.  Synchronises. */
 SPEC_API int spec_draft_append(spec_handle* h, int seq, const void* feats, const int32_t* tokens, int n);
 /* One draft-head step over a batch of trees on the draft prefixes: per node,
  * the SPEC_DRAFT_TOPK best vocabulary entries of the draft distribution, by
