@@ -256,8 +256,10 @@ size_t attention_tc_smem_bytes();
 cudaError_t attention_tc_configure(int* max_clusters);
 
 // LM head reductions
+// with err (optional): when the error word is non-zero (an earlier kernel gave up on a
+// wait), every row gets argmax -1 and top1 = top2 = NaN instead
 cudaError_t launch_top2_reduce(int M, int tiles, const Top2* part, int top_ld, int32_t* argmax, float* top1,
-                               float* top2, cudaStream_t s, bool pdl);
+                               float* top2, cudaStream_t s, bool pdl, const uint32_t* err = nullptr);
 cudaError_t launch_rows_top2_f32(int M, int V, const float* logits, int32_t* argmax, float* top1, float* top2,
                                  cudaStream_t s);
 

@@ -30,7 +30,8 @@ constexpr int kNoallocMaxVocab = 262144; // V
 constexpr size_t kSplitBytes = (size_t)2 * kNoallocMaxRows * kNoallocMaxHidden * 2;  // hi + lo rows, bf16
 constexpr size_t kTop2Bytes = (size_t)(kNoallocMaxVocab / 128) * kNoallocMaxRows * 12;  // one Top2 per tile x row
 constexpr size_t kSsBytes = (size_t)kNoallocMaxRows * 4;
-constexpr size_t kScratchBytes = kSplitBytes + kTop2Bytes + kSsBytes;  // 3.5 MiB + 256 B
+constexpr size_t kErrBytes = 256;  // the call's device error word (4 bytes used)
+constexpr size_t kScratchBytes = kSplitBytes + kTop2Bytes + kSsBytes + kErrBytes;  // 3.5 MiB + 512 B
 
 // The scratch.  In host code this name is only a stand-in for the device
 // array: its device address comes from cudaGetSymbolAddress, once per device.
@@ -64,16 +65,12 @@ typedef CUresult (*EncodeTiledFn)(CUtensorMap*, CUtensorMapDataType, cuuint32_t,
                                   const cuuint64_t*, const cuuint32_t*, const cuuint32_t*, CUtensorMapInterleave,
                                   CUtensorMapSwizzle, CUtensorMapL2promotion, CUtensorMapFloatOOBfill);
 
+// resolved once, in setup_device under g_setup_mu, before any encode() call
+EncodeTiledFn g_encode = nullptr;
+
 bool encode(CUtensorMap* m, const void* ptr, uint64_t rows, uint64_t cols, uint32_t box_rows) {
-  static EncodeTiledFn fn = nullptr;
-  if (!fn) {
-    void* p = nullptr;
-    cudaDriverEntryPointQueryResult q;
-    if (cudaGetDriverEntryPointByVersion("cuTensorMapEncodeTiled", &p, 12000, cudaEnableDefault, &q) != cudaSuccess ||
-        q != cudaDriverEntryPointSuccess)
-      return false;
-    fn = reinterpret_cast<EncodeTiledFn>(p);
-  }
+  const EncodeTiledFn fn = g_encode;
+  if (!fn) return false;
   cuuint64_t dims[2] = {cols, rows};
   cuuint64_t strides[1] = {cols * 2};
   cuuint32_t box[2] = {64, box_rows};
@@ -91,6 +88,14 @@ int g_sm_count[kMaxDevices] = {};
 
 int setup_device(int dev, unsigned char** scratch, int* sms) {
   std::lock_guard<std::mutex> lock(g_setup_mu);
+  if (!g_encode) {
+    void* p = nullptr;
+    cudaDriverEntryPointQueryResult q;
+    if (cudaGetDriverEntryPointByVersion("cuTensorMapEncodeTiled", &p, 12000, cudaEnableDefault, &q) != cudaSuccess ||
+        q != cudaDriverEntryPointSuccess)
+      return SPEC_ERR_CUDA;
+    g_encode = reinterpret_cast<EncodeTiledFn>(p);
+  }
   if (!g_scratch_ptr[dev]) {
     void* p = nullptr;
     cudaError_t e = cudaGetSymbolAddress(&p, g_noalloc_scratch);
@@ -146,11 +151,17 @@ int spec_lm_head_argmax_noalloc(const float* hidden, const void* final_norm, con
   __nv_bfloat16* split = reinterpret_cast<__nv_bfloat16*>(scratch);
   Top2* top_part = reinterpret_cast<Top2*>(scratch + kSplitBytes);
   float* ss = reinterpret_cast<float*>(scratch + kSplitBytes + kTop2Bytes);
+  uint32_t* err = reinterpret_cast<uint32_t*>(scratch + kSplitBytes + kTop2Bytes + kSsBytes);
   cudaStream_t st = reinterpret_cast<cudaStream_t>(cuda_stream);
 
   CUtensorMap map_lm, map_x;
   if (!encode(&map_lm, lm_head, (uint64_t)V, (uint64_t)d, 128) ||
       !encode(&map_x, split, 2 * (uint64_t)kNoallocMaxRows, (uint64_t)d, 128)) {
+    return SPEC_ERR_CUDA;
+  }
+  // the error word starts every call at zero (a memset needs no allocation)
+  e = cudaMemsetAsync(err, 0, sizeof(uint32_t), st);
+  if (e != cudaSuccess) {
     return SPEC_ERR_CUDA;
   }
   noalloc_prep_kernel<<<M, 256, 0, st>>>(hidden, reinterpret_cast<const __nv_bfloat16*>(final_norm), d, split, ss);
@@ -178,9 +189,11 @@ int spec_lm_head_argmax_noalloc(const float* hidden, const void* final_norm, con
   g.args.eps = eps;
   g.args.top_part = top_part;
   g.args.top_ld = kNoallocMaxRows;
+  g.args.err = err;
   g.grid = g.args.tiles_o < 2 * sms ? g.args.tiles_o : 2 * sms;
   e = gemm_tc_launch(g, st, false);
-  if (e == cudaSuccess) e = launch_top2_reduce(M, g.args.tiles_o, top_part, kNoallocMaxRows, argmax, top1, top2, st, false);
+  if (e == cudaSuccess) e = launch_top2_reduce(M, g.args.tiles_o, top_part, kNoallocMaxRows, argmax, top1, top2, st, false,
+                                                  err);
   if (e != cudaSuccess) {
     return SPEC_ERR_CUDA;
   }

@@ -368,12 +368,21 @@ cudaError_t launch_gemm_simt_f32(const float* A, int lda, const float* W, int K,
 // warps and the CTA merge (lowest index on equal values).
 __global__ void __launch_bounds__(256) top2_reduce_kernel(int M, int tiles, const Top2* __restrict__ part,
                                                          int top_ld, int32_t* __restrict__ argmax,
-                                                         float* __restrict__ top1, float* __restrict__ top2) {
+                                                         float* __restrict__ top1, float* __restrict__ top2,
+                                                         const uint32_t* __restrict__ err) {
   __shared__ Top2 wbest[8];
   pdl_wait();
   pdl_launch_dependents();
   const int t = blockIdx.x;
   if (t >= M) return;
+  if (err && *err) {  // the partials may be stale: say so instead of reducing them
+    if (threadIdx.x == 0) {
+      argmax[t] = -1;
+      top1[t] = __int_as_float(0x7fc00000);
+      top2[t] = __int_as_float(0x7fc00000);
+    }
+    return;
+  }
   constexpr int kU = 4;
   Top2 best;
   best.v1 = -INFINITY; best.i1 = 0x7fffffff; best.v2 = -INFINITY;
@@ -405,10 +414,10 @@ __global__ void __launch_bounds__(256) top2_reduce_kernel(int M, int tiles, cons
 }
 
 cudaError_t launch_top2_reduce(int M, int tiles, const Top2* part, int top_ld, int32_t* argmax, float* top1,
-                               float* top2, cudaStream_t s, bool pdl) {
+                               float* top2, cudaStream_t s, bool pdl, const uint32_t* err) {
   cudaLaunchAttribute attr[1];
   cudaLaunchConfig_t cfg = make_cfg(dim3(M), dim3(256), 0, s, pdl, attr);
-  return cudaLaunchKernelEx(&cfg, top2_reduce_kernel, M, tiles, part, top_ld, argmax, top1, top2);
+  return cudaLaunchKernelEx(&cfg, top2_reduce_kernel, M, tiles, part, top_ld, argmax, top1, top2, err);
 }
 
 __global__ void rows_top2_f32_kernel(int M, int V, const float* __restrict__ logits, int32_t* __restrict__ argmax,
