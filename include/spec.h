@@ -53,11 +53,16 @@ extern "C" {
 #define SPEC_ERR_CUDA (-6)     /* a CUDA call failed; the message names the cudaError_t */
 #define SPEC_ERR_TIMEOUT (-7)  /* a bounded wait inside a kernel expired */
 #define SPEC_ERR_STATE (-8)    /* sequence not prefilled, or truncation beyond its length */
+#define SPEC_ERR_RANGE (-9)    /* bf16 models: a q / K / V value outside the fp16 range of the cache (|v| > 65504) */
 
 /* model dtypes */
 #define SPEC_DTYPE_F32 0       /* weights, activations and K/V in fp32; plain FFMA arithmetic */
 #define SPEC_DTYPE_BF16 1      /* weights bf16; GEMM activations as split bf16 (hi + lo); q, K/V cache and
-                                  attention probabilities fp16; fp32 accumulation, residual and softmax */
+                                  attention probabilities fp16; fp32 accumulation, residual and softmax.
+                                  q, K and V (after the rotary embedding) must lie within the fp16 range,
+                                  |v| <= 65504: a step that meets a value beyond it (or a NaN) stores it
+                                  saturated, leaves every sequence's state as it was, and fails with
+                                  SPEC_ERR_RANGE */
 
 /* flags of spec_verify_tree_batch */
 #define SPEC_DEVICE_OUTPUTS 1  /* outputs are device pointers (or NULL); return without synchronising */
@@ -336,10 +341,18 @@ SPEC_API int spec_step_launches(spec_handle* h);
  * any GPU work.  Work is queued on cuda_stream (NULL: legacy default stream);
  * the call does not synchronise.
  *
+ * Device-side failure: every wait inside the call is bounded (2 s).  If one
+ * gives up, the GPU stays usable and every row gets argmax = -1 and
+ * top1 = top2 = NaN; the return code cannot say so, because the call returns
+ * before the GPU runs.  After synchronising the stream, argmax[0] < 0 means
+ * the outputs are void.  The error word behind this is part of the scratch and
+ * is cleared at the start of each call.
+ *
  * The first call on a device looks up the scratch array's device address and
  * sets kernel attributes, so make that first call before any stream capture.
- * Every call uses the same scratch and leaves its contents behind; nothing in
- * it has to start at zero.  Calls that overlap on the GPU (on different
+ * Every call uses the same scratch and leaves its contents behind; only the
+ * error word has to start at zero, and the call clears it itself (a memset on
+ * cuda_stream, no allocation).  Calls that overlap on the GPU (on different
  * streams, or from different threads) race on the scratch: serialise them. */
 SPEC_API int spec_lm_head_argmax_noalloc(const float* hidden, const void* final_norm, const void* lm_head, int M,
                                          int d, int V, float eps, int32_t* argmax, float* top1, float* top2,

@@ -21,6 +21,7 @@ enum : uint32_t {
   SPEC_DEVERR_ROOT = 1u,      // tokens[0] is not the sequence's pending token
   SPEC_DEVERR_TIMEOUT = 2u,   // a bounded wait expired
   SPEC_DEVERR_BOUNDS = 4u,    // a kernel saw an index outside its buffers and skipped it
+  SPEC_DEVERR_RANGE = 8u,     // a q / K / V value outside the fp16 range (|v| > 65504 or NaN), stored saturated
 };
 
 #ifndef SPEC_WAIT_NS

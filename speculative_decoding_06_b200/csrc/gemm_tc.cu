@@ -513,6 +513,16 @@ __global__ void __launch_bounds__(kThreads, BN == 64 ? 2 : 1)
                 set_error(err, SPEC_DEVERR_BOUNDS);
               }
               if (dst) {
+                // q and the K/V cache are fp16: a value beyond its range (or NaN) is
+                // stored saturated and fails the step instead of turning into inf / NaN
+                bool in_range = true;
+#pragma unroll
+                for (int i = 0; i < 4; ++i) {
+                  in_range = in_range && fabsf(x1[i]) <= 65504.f && fabsf(x2[i]) <= 65504.f;
+                  x1[i] = fminf(fmaxf(x1[i], -65504.f), 65504.f);
+                  x2[i] = fminf(fmaxf(x2[i], -65504.f), 65504.f);
+                }
+                if (!in_range) set_error(err, SPEC_DEVERR_RANGE);
                 const __half2 h0 = __floats2half2_rn(x1[0], x1[1]), h1 = __floats2half2_rn(x1[2], x1[3]);
                 const __half2 h2 = __floats2half2_rn(x2[0], x2[1]), h3 = __floats2half2_rn(x2[2], x2[3]);
                 uint2 lo, hi;

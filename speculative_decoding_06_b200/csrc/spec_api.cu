@@ -991,6 +991,7 @@ int run_step(spec_handle* h, int B, const int32_t* seq_ids, const int32_t* token
   CUDA_TRY(h, cudaStreamSynchronize(h->stream));
   if (errw[0] & SPEC_DEVERR_TIMEOUT) return fail(h, SPEC_ERR_TIMEOUT, "a bounded wait expired on the device");
   if (errw[0] & SPEC_DEVERR_ROOT) return fail(h, SPEC_ERR_ROOT, "tokens[0] is not the pending token (device check)");
+  if (errw[0] & SPEC_DEVERR_RANGE) return fail(h, SPEC_ERR_RANGE, "a q / K / V value exceeded the fp16 range");
   if (errw[0]) return fail(h, SPEC_ERR_CUDA, "device reported error bits 0x%x", errw[0]);
   // mirror the state update done on the device
   if (mode != STEP_SCORE) {
@@ -1104,6 +1105,7 @@ int run_draft(spec_handle* h, int B, const int32_t* seq_ids, const void* feats, 
   CUDA_TRY(h, cudaMemcpyAsync(errw, h->ws + L.p_err, 4, cudaMemcpyDeviceToHost, h->stream));
   CUDA_TRY(h, cudaStreamSynchronize(h->stream));
   if (errw[0] & SPEC_DEVERR_TIMEOUT) return fail(h, SPEC_ERR_TIMEOUT, "a bounded wait expired on the device");
+  if (errw[0] & SPEC_DEVERR_RANGE) return fail(h, SPEC_ERR_RANGE, "a q / K / V value exceeded the fp16 range");
   if (errw[0]) return fail(h, SPEC_ERR_CUDA, "device reported error bits 0x%x", errw[0]);
   return SPEC_OK;
 }
@@ -1126,6 +1128,7 @@ int refresh_state(spec_handle* h) {
   h->stale = false;
   if (sticky & SPEC_DEVERR_TIMEOUT) return fail(h, SPEC_ERR_TIMEOUT, "a bounded wait expired on the device");
   if (sticky & SPEC_DEVERR_ROOT) return fail(h, SPEC_ERR_ROOT, "a queued step had tokens[0] != pending token");
+  if (sticky & SPEC_DEVERR_RANGE) return fail(h, SPEC_ERR_RANGE, "a queued step exceeded the fp16 range of q / K / V");
   if (sticky) return fail(h, SPEC_ERR_CUDA, "device reported error bits 0x%x", sticky);
   return SPEC_OK;
 }
@@ -1588,6 +1591,7 @@ int spec_draft_tree(spec_handle* h, int B, const int32_t* seq_ids, const void* r
   CUDA_TRY(h, cudaMemcpyAsync(errw, h->ws + L.p_err, 4, cudaMemcpyDeviceToHost, st));
   CUDA_TRY(h, cudaStreamSynchronize(st));
   if (errw[0] & SPEC_DEVERR_TIMEOUT) return fail(h, SPEC_ERR_TIMEOUT, "a bounded wait expired on the device");
+  if (errw[0] & SPEC_DEVERR_RANGE) return fail(h, SPEC_ERR_RANGE, "a q / K / V value exceeded the fp16 range");
   if (errw[0]) return fail(h, SPEC_ERR_CUDA, "device reported error bits 0x%x", errw[0]);
   for (int b = 0; b < B; ++b)
     if (spec_validate_tree(out_tokens + (size_t)b * (total + 1), out_parents + (size_t)b * (total + 1), total + 1,

@@ -22,6 +22,7 @@ SPEC_ERR_ROOT = -5
 SPEC_ERR_CUDA = -6
 SPEC_ERR_TIMEOUT = -7
 SPEC_ERR_STATE = -8
+SPEC_ERR_RANGE = -9
 
 SPEC_DTYPE_F32 = 0
 SPEC_DTYPE_BF16 = 1
@@ -37,7 +38,8 @@ PROF_CLASSES = ("embed_meta", "gemm_qkv", "rope_kv_store", "attention", "gemm_o"
                 "features", "draft_tree")
 
 ERR_NAMES = {0: "SPEC_OK", -1: "SPEC_ERR_ARG", -2: "SPEC_ERR_TREE", -3: "SPEC_ERR_TOKEN", -4: "SPEC_ERR_CAPACITY",
-             -5: "SPEC_ERR_ROOT", -6: "SPEC_ERR_CUDA", -7: "SPEC_ERR_TIMEOUT", -8: "SPEC_ERR_STATE"}
+             -5: "SPEC_ERR_ROOT", -6: "SPEC_ERR_CUDA", -7: "SPEC_ERR_TIMEOUT", -8: "SPEC_ERR_STATE",
+             -9: "SPEC_ERR_RANGE"}
 
 
 class spec_config(ctypes.Structure):
