@@ -15,8 +15,8 @@ import pytest
 
 import synth
 from oracle import oracle_verify, top2_margin
-from gpu_common import (DECISIVE, TOL, decisive_nodes, decisive_prefix, gpu_kv, kv_close, make_pair,
-                        planted_tree)
+from gpu_common import (DECISIVE, TOL, decided_case, decided_tree, decisive_nodes, decisive_prefix, gpu_kv,
+                        kv_close, make_pair)
 
 pytestmark = pytest.mark.gpu
 
@@ -61,24 +61,26 @@ def test_tiny_fp32_config():
     assert pend == seq.pending
     gk, gv = gpu_kv(eng, 0, 64)
     assert kv_close(gk[0], seq.k[0], 1e-5) <= 1e-5
-    decided = 0
     for step in range(4):
         shape = synth.tiny_tree()
-        toks = planted_tree(om, seq, shape, 0.8, stream=step)
+        toks, _ = decided_tree(om, seq, shape, 0.8, stream=step, min_margin=1e-3)
+        assert toks is not None
         d, err = _check_step(eng, om, 0, seq, shape, toks, "f32")
-        decided += d
+        assert d, "step %d was not decided" % step
         assert err < 1e-4
-    assert decided >= 3
 
 
+# (model, prefix length, tree, prefix stream, planting stream): the streams are the
+# first ones from which gpu_common.decided_case finds a decided step (the search
+# runs again in each test and ends at its first candidate)
 BF16_CASES = [
-    ("mini", 37, "root"),
-    ("mini", 37, "chain2"),
-    ("mini", 300, "tiny"),
-    ("mini", 1000, "tree60"),
-    ("mini", 129, "tree127"),
-    ("small", 700, "tree60"),
-    ("small", 64, "chain8"),
+    ("mini", 37, "root", 37, 37),
+    ("mini", 37, "chain2", 37, 37),
+    ("mini", 300, "tiny", 300, 300),
+    ("mini", 1000, "tree60", 1000, 3000),
+    ("mini", 129, "tree127", 133, 133),
+    ("small", 700, "tree60", 700, 2700),
+    ("small", 64, "chain8", 64, 64),
 ]
 
 
@@ -108,18 +110,18 @@ def _pair(which):
     return _pairs[which]
 
 
-@pytest.mark.parametrize("which,P,kind", BF16_CASES)
-def test_bf16_verify_parity(which, P, kind):
+@pytest.mark.parametrize("which,P,kind,s_prefix,s_plant", BF16_CASES)
+def test_bf16_verify_parity(which, P, kind, s_prefix, s_plant):
     eng, om = _pair(which)
-    prefix, seq = decisive_prefix(om, P, stream0=P)
+    shape = _shape(kind)
+    prefix, seq, toks = decided_case(om, P, shape, 0.8, stream0=s_prefix, plant0=s_plant)
     pend = eng.prefill(0, prefix)
     assert pend == seq.pending
     gk, gv = gpu_kv(eng, 0, P)
     for l in range(om.d.n_layers):
         assert kv_close(gk[l], seq.k[l], 2e-2) <= 2e-2
-    shape = _shape(kind)
-    toks = planted_tree(om, seq, shape, 0.8, stream=P)
-    _check_step(eng, om, 0, seq, shape, toks, "bf16")
+    decided, _ = _check_step(eng, om, 0, seq, shape, toks, "bf16")
+    assert decided, "the step was not decided: outputs and K/V went unchecked"
 
 
 def test_bf16_batch_of_sequences():
@@ -129,9 +131,8 @@ def test_bf16_batch_of_sequences():
     shapes = [synth.tree_from_widths((3, 3, 2), stream=1), synth.tiny_tree(), synth.chain(5)]
     seqs, trees = [], []
     for i, (P, sh) in enumerate(zip(Ps, shapes)):
-        prefix, seq = decisive_prefix(om, P, stream0=100 + 10 * i)
+        prefix, seq, toks = decided_case(om, P, sh, 0.8, stream0=(101, 112, 120)[i])
         assert eng.prefill(i, prefix) == seq.pending
-        toks = planted_tree(om, seq, sh, 0.8, stream=50 + i)
         seqs.append(seq)
         trees.append((toks, sh.parents))
     amax, t1, t2, off = eng.score([0, 1, 2], trees, flags=2)
@@ -142,26 +143,30 @@ def test_bf16_batch_of_sequences():
         lg = logits[off[i]:off[i + 1]]
         err = float(np.max(np.abs(lg - r["logits"])))
         assert err <= TOL["bf16"]
-        thr = min(DECISIVE, 2.5 * err)
-        if np.all(r["margin"][decisive_nodes(r, par)] > thr):
-            assert acc_len[i] == r["accepted_len"]
-            assert list(acc_nodes[i, :acc_len[i]]) == r["accepted_nodes"]
-            assert list(acc_tok[i, :acc_len[i]]) == r["accepted_tokens"]
-            assert bonus[i] == r["bonus"]
-            ln, _ = eng.seq_len(i)
-            gk, gv = gpu_kv(eng, i, ln)
-            for l in range(om.d.n_layers):
-                assert kv_close(gk[l], seq.k[l], 2e-2) <= 2e-2
+        thr = min(DECISIVE, max(2.5 * err, 1e-6))
+        assert np.all(r["margin"][decisive_nodes(r, par)] > thr), "sequence %d was not decided" % i
+        assert acc_len[i] == r["accepted_len"]
+        assert list(acc_nodes[i, :acc_len[i]]) == r["accepted_nodes"]
+        assert list(acc_tok[i, :acc_len[i]]) == r["accepted_tokens"]
+        assert bonus[i] == r["bonus"]
+        ln, _ = eng.seq_len(i)
+        gk, gv = gpu_kv(eng, i, ln)
+        for l in range(om.d.n_layers):
+            assert kv_close(gk[l], seq.k[l], 2e-2) <= 2e-2
+            assert kv_close(gv[l], seq.v[l], 2e-2) <= 2e-2
+
+
+WIDE_STREAMS = (7, 7)  # (prefix, planting) streams of the decided step on the 8B-layer-shape model
 
 
 def test_wide_bf16_full_size_tiles():
     """8B layer shapes (d 4096, 32/8 heads, ffn 14336), 2 layers, vocab 16384: full-size tiles and splits."""
-    eng, om = make_pair(synth.WIDE_BF16, max_batch=1, max_seq=512, max_nodes=64, device_gen=True)
-    prefix, seq = decisive_prefix(om, 200, stream0=7, tries=6)
-    assert eng.prefill(0, prefix) == seq.pending
+    eng, om = make_pair(synth.WIDE_BF16, max_batch=1, max_seq=512, max_nodes=64)
     shape = synth.tree_from_widths(synth.TREE60_WIDTHS, stream=0)
-    toks = planted_tree(om, seq, shape, 0.8, stream=9)
-    _check_step(eng, om, 0, seq, shape, toks, "bf16")
+    prefix, seq, toks = decided_case(om, 200, shape, 0.8, stream0=WIDE_STREAMS[0], plant0=WIDE_STREAMS[1])
+    assert eng.prefill(0, prefix) == seq.pending
+    decided, _ = _check_step(eng, om, 0, seq, shape, toks, "bf16")
+    assert decided
 
 
 def _check_batch(eng, om, ids, seqs, trees):
@@ -192,6 +197,12 @@ def _check_batch(eng, om, ids, seqs, trees):
     return decided
 
 
+# per sequence: (prefix stream, planting stream) of a decided step
+LARGE_STREAMS = [(302, 3302), (308, 308), (320, 320), (322, 322), (328, 1328), (335, 335), (350, 350), (350, 350),
+                 (360, 360), (364, 364), (370, 370), (377, 377), (384, 1384), (392, 3392), (399, 2399), (405, 405),
+                 (412, 412), (419, 419), (427, 427), (433, 1433)]
+
+
 def test_bf16_large_batch_unchunked():
     """20 sequences (prefixes 150-600) x 61-node trees = 1220 tokens: 128-token GEMM tiles, several token
     tiles, and attention without key chunks (one CTA walks every 128-key block with the online softmax)."""
@@ -200,13 +211,14 @@ def test_bf16_large_batch_unchunked():
     Ps = np.random.default_rng(4).integers(150, 601, size=B)
     seqs, trees = [], []
     for i in range(B):
-        prefix, seq = decisive_prefix(om, int(Ps[i]), stream0=300 + 7 * i)
-        assert eng.prefill(i, prefix) == seq.pending
         sh = synth.tree_from_widths(synth.TREE60_WIDTHS, stream=i)
-        trees.append((planted_tree(om, seq, sh, 0.8, stream=60 + i), sh.parents))
+        prefix, seq, toks = decided_case(om, int(Ps[i]), sh, 0.8, stream0=LARGE_STREAMS[i][0],
+                                         plant0=LARGE_STREAMS[i][1])
+        assert eng.prefill(i, prefix) == seq.pending
+        trees.append((toks, sh.parents))
         seqs.append(seq)
     assert "chunks 1 x" in eng.info(B, 61, int(Ps.max()))
-    assert _check_batch(eng, om, list(range(B)), seqs, trees) >= B // 2
+    assert _check_batch(eng, om, list(range(B)), seqs, trees) == B
 
 
 def _engine_tuned(dims, tune, **kw):
@@ -231,9 +243,9 @@ def test_bf16_multiblock_attention(tune):
     eng, om = _engine_tuned(synth.MINI_BF16, tune, max_batch=2, max_seq=1024, max_nodes=64)
     seqs, trees = [], []
     for i, P in enumerate((700, 530)):
-        prefix, seq = decisive_prefix(om, P, stream0=500 + 11 * i)
-        assert eng.prefill(i, prefix) == seq.pending
         sh = synth.tree_from_widths(synth.TREE60_WIDTHS, stream=3 + i)
-        trees.append((planted_tree(om, seq, sh, 0.8, stream=70 + i), sh.parents))
+        prefix, seq, toks = decided_case(om, P, sh, 0.8, stream0=(501, 512)[i], plant0=(1501, 512)[i])
+        assert eng.prefill(i, prefix) == seq.pending
+        trees.append((toks, sh.parents))
         seqs.append(seq)
-    _check_batch(eng, om, [0, 1], seqs, trees)
+    assert _check_batch(eng, om, [0, 1], seqs, trees) == 2
