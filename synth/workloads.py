@@ -315,3 +315,37 @@ def draft_head_weights(d: ModelDims, seed: int = 6, device: str = "cpu") -> dict
     w["layer"] = lw
     w["final_norm"] = torch.ones(d.hidden, device=device, dtype=tdt)
     return w
+
+
+# ---------------------------------------------------------------------------
+# fingerprints of generated inputs
+# ---------------------------------------------------------------------------
+
+def weights_fingerprint(w: dict, row_stride: int = 509) -> str:
+    """sha256 (hex, 16 digits) over every `row_stride`-th row of each matrix's raw bits.
+
+    Stored beside precomputed expected values, so that a machine that draws
+    different weights from the same seed (another torch build or CPU code
+    path) is detected before any comparison is made."""
+    import hashlib
+    h = hashlib.sha256()
+
+    def add(name, t):
+        a = tensor_to_host(t)
+        a2 = a.reshape(a.shape[0], -1) if a.ndim > 1 else a.reshape(1, -1)
+        h.update(name.encode())
+        h.update(np.ascontiguousarray(a2[::row_stride]).tobytes())
+
+    for k in ("embed", "lm_head", "final_norm"):
+        if k in w:
+            add(k, w[k])
+    for i, lw in enumerate(w.get("layers", [])):
+        for k in LAYER_KEYS:
+            add("%d.%s" % (i, k), lw[k])
+    for k in ("fc_fuse", "fc_in"):
+        if k in w:
+            add(k, w[k])
+    if "layer" in w:
+        for k in LAYER_KEYS:
+            add("layer." + k, w["layer"][k])
+    return h.hexdigest()[:16]
