@@ -64,3 +64,23 @@ def test_reference_arm_other_ranks_exit_without_work():
         pass
     # rank 1 of a torchrun launch returns at once (rank 0 alone times the oracle)
     assert bench.run_reference(A(), 1, 2) == 0
+
+
+def test_replica_launcher_starts_n_ranks(capfd):
+    """bench.py --gpus N without a launcher starts N ranks through torchrun; rank 0 alone prints, with
+    n_gpus = N and the job's throughput over the slowest rank's time."""
+    sys.path.insert(0, ROOT)
+    import json
+    import bench
+    cmd = bench.replica_command(2, "x.py", ["--steps", "3"], 12345)
+    assert cmd[1:4] == ["-m", "torch.distributed.run", "--nnodes=1"]
+    assert cmd[cmd.index("--nproc-per-node") + 1] == "2" and cmd[cmd.index("--master-addr") + 1] == "127.0.0.1"
+    assert cmd[-3:] == ["x.py", "--steps", "3"]
+    rc = bench.run_replicas(2, [], script=os.path.join(ROOT, "tests", "rank_probe.py"), timeout_s=300)
+    assert rc == 0
+    lines = [ln for ln in capfd.readouterr().out.splitlines() if ln.startswith("{")]
+    assert len(lines) == 1
+    rec = json.loads(lines[0])
+    assert rec["n_gpus"] == 2
+    assert rec["ms_per_step"] == pytest.approx(12.5)          # the slower rank: 125 ms over 10 steps
+    assert rec["value"] == pytest.approx(2 * 10 / 0.125)
