@@ -256,6 +256,26 @@ SPEC_API int spec_draft_tree(spec_handle* h, int B, const int32_t* seq_ids, cons
  * when the handle has no feature layers; device_buf NULL detaches the buffer. */
 SPEC_API int spec_set_feature_out(spec_handle* h, void* device_buf, size_t bytes);
 
+/* Temperature sampling instead of greedy choices (both leave the target's output distribution
+ * unchanged: "EAGLE-3投机解码：树验证器方法", section 验证-接受语义, and the sampling rule of
+ * Leviathan et al., "Fast Inference from Transformers via Speculative Decoding", which that page
+ * cites).  temperature = 0 (the default) restores greedy decoding.
+ *
+ * With temperature T > 0, every token the target chooses -- the pending token of a prefill, the
+ * choice at each tree node of a verification or scoring step -- is a draw from softmax(logits / T),
+ * taken as argmax_v(logit_v / T + g_v) with g_v a standard Gumbel variable.  The noise of a row
+ * depends only on (seed, sequence id, the row's position, v): g_v = -ln(-ln u) with
+ * u = (2 (x >> 9) + 1) 2^-24 and x word 0 of Philox4x32-10 (Salmon et al., SC 2011) at counter
+ * (v, position, sequence id, 0) and key (seed & 0xffffffff, seed >> 32).  A tree node at position
+ * P + depth accepts, as in the greedy walk, the first child whose token equals its draw; the bonus is
+ * the draw at the last accepted node.  Each draft token thus acts as a point-mass proposal in the
+ * speculative-sampling rule (accepted with probability p(x) given the earlier siblings' rejections),
+ * and the emitted stream is exactly autoregressive sampling with the same noise.  spec_score_trees
+ * then returns the draws as "argmax" and the perturbed scores logit / T + g as top1 / top2.  The
+ * draft head's top-k is unaffected.  SPEC_ERR_ARG for a negative, infinite or NaN temperature or
+ * one whose reciprocal overflows.  Takes effect for calls made after it (cached graphs are rebuilt). */
+SPEC_API int spec_set_sampling(spec_handle* h, float temperature, uint64_t seed);
+
 /* Device buffer (fp32, >= max_batch * max_nodes * vocab entries) for SPEC_DEBUG_LOGITS. */
 SPEC_API int spec_set_debug_logits(spec_handle* h, float* device_buf, size_t bytes);
 

@@ -38,6 +38,34 @@ __device__ __forceinline__ uint64_t global_ns() {
   return t;
 }
 
+// ---------------------------------------------------------------------------
+// sampling noise
+// ---------------------------------------------------------------------------
+// Philox4x32 with 10 rounds (Salmon, Moraes, Dror and Shaw, "Parallel Random
+// Numbers: As Easy as 1, 2, 3", SC 2011): per round the full 64-bit products
+// M0 * c0 and M1 * c2 give c' = (hi1 ^ c1 ^ k0, lo1, hi0 ^ c3 ^ k1, lo0), and the
+// key advances by the Weyl increments between rounds.
+__device__ __forceinline__ uint4 philox4x32_10(uint4 c, uint32_t k0, uint32_t k1) {
+#pragma unroll
+  for (int r = 0; r < 10; ++r) {
+    const uint32_t hi0 = __umulhi(0xD2511F53u, c.x), lo0 = 0xD2511F53u * c.x;
+    const uint32_t hi1 = __umulhi(0xCD9E8D57u, c.z), lo1 = 0xCD9E8D57u * c.z;
+    c = make_uint4(hi1 ^ c.y ^ k0, lo1, hi0 ^ c.w ^ k1, lo0);
+    k0 += 0x9E3779B9u;
+    k1 += 0xBB67AE85u;
+  }
+  return c;
+}
+
+// Standard Gumbel variable of vocabulary entry v for (seed, sequence, position):
+// word 0 of Philox(counter (v, pos, seq, 0), key seed) gives u = (2 (x >> 9) + 1) 2^-24,
+// and g = -ln(-ln u), evaluated through w = 1 - u (exact) as -ln(-log1p(-w)).
+__device__ __forceinline__ float gumbel_noise(uint32_t seed_lo, uint32_t seed_hi, int seq, int pos, int v) {
+  const uint32_t x = philox4x32_10(make_uint4((uint32_t)v, (uint32_t)pos, (uint32_t)seq, 0u), seed_lo, seed_hi).x;
+  const float w = (float)(2u * (8388607u - (x >> 9)) + 1u) * 5.9604644775390625e-08f;
+  return -logf(-log1pf(-w));
+}
+
 __device__ __forceinline__ uint32_t smem_u32(const void* p) {
   return static_cast<uint32_t>(__cvta_generic_to_shared(p));
 }

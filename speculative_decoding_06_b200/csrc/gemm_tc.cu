@@ -650,6 +650,9 @@ __global__ void __launch_bounds__(kThreads, BN == 64 ? 2 : 1)
             for (int i = 0; i < 16; ++i) {
               const int t = t_base + c0 + i;
               if (args.dbg_logits && row_ok && t < args.M) args.dbg_logits[(size_t)t * args.n_out + o] = v[i];
+              if (args.inv_temp > 0.f && row_ok && t < args.M)  // temperature sampling: Gumbel-max
+                v[i] = fmaf(v[i], args.inv_temp,
+                            gumbel_noise(args.seed_lo, args.seed_hi, args.row_sid[t], args.row_pos[t], o));
               Top2 x;
               x.v1 = row_ok ? v[i] : -INFINITY;
               x.i1 = row_ok ? o : 0x7fffffff;

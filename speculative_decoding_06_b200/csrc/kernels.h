@@ -47,7 +47,12 @@ struct GemmTcArgs {
   // ARGMAX
   Top2* top_part;     // [tiles_o][top_ld]
   int top_ld;
-  float* dbg_logits;  // optional [M][n_out]
+  float* dbg_logits;  // optional [M][n_out] (the logits themselves, before any sampling noise)
+  // sampling (inv_temp > 0): the row's choice is argmax_v(logit_v * inv_temp + gumbel(seed, sid, pos, v))
+  // with sid = row_sid[t] and pos = row_pos[t]; inv_temp = 0: the plain argmax
+  const int32_t* row_pos;
+  float inv_temp;
+  uint32_t seed_lo, seed_hi;
   // QKV
   const int32_t* row_seq;
   const int32_t* row_local;
@@ -260,8 +265,10 @@ cudaError_t attention_tc_configure(int* max_clusters);
 // wait), every row gets argmax -1 and top1 = top2 = NaN instead
 cudaError_t launch_top2_reduce(int M, int tiles, const Top2* part, int top_ld, int32_t* argmax, float* top1,
                                float* top2, cudaStream_t s, bool pdl, const uint32_t* err = nullptr);
+// (with inv_temp > 0, the sampled choice of each row as in GemmTcArgs)
 cudaError_t launch_rows_top2_f32(int M, int V, const float* logits, int32_t* argmax, float* top1, float* top2,
-                                 cudaStream_t s);
+                                 cudaStream_t s, float inv_temp = 0.f, uint32_t seed_lo = 0, uint32_t seed_hi = 0,
+                                 const int32_t* row_sid = nullptr, const int32_t* row_pos = nullptr);
 
 // acceptance walk (or commit-all for prefill chains) + state update
 struct WalkArgs {

@@ -421,15 +421,22 @@ cudaError_t launch_top2_reduce(int M, int tiles, const Top2* part, int top_ld, i
 }
 
 __global__ void rows_top2_f32_kernel(int M, int V, const float* __restrict__ logits, int32_t* __restrict__ argmax,
-                                     float* __restrict__ top1, float* __restrict__ top2) {
+                                     float* __restrict__ top1, float* __restrict__ top2, float inv_temp,
+                                     uint32_t seed_lo, uint32_t seed_hi, const int32_t* __restrict__ row_sid,
+                                     const int32_t* __restrict__ row_pos) {
   const int t = blockIdx.x * (blockDim.x >> 5) + (threadIdx.x >> 5);
   const int lane = threadIdx.x & 31;
   if (t >= M) return;
+  const bool sample = inv_temp > 0.f;
+  const int sid = sample ? row_sid[t] : 0;
+  const int pos = sample ? row_pos[t] : 0;
   Top2 best;
   best.v1 = -INFINITY; best.i1 = 0x7fffffff; best.v2 = -INFINITY;
   for (int v = lane; v < V; v += 32) {
     Top2 x;
-    x.v1 = logits[(size_t)t * V + v]; x.i1 = v; x.v2 = -INFINITY;
+    const float l = logits[(size_t)t * V + v];
+    x.v1 = sample ? fmaf(l, inv_temp, gumbel_noise(seed_lo, seed_hi, sid, pos, v)) : l;
+    x.i1 = v; x.v2 = -INFINITY;
     best = top2_merge(best, x);
   }
   best = warp_top2(best);
@@ -441,8 +448,11 @@ __global__ void rows_top2_f32_kernel(int M, int V, const float* __restrict__ log
 }
 
 cudaError_t launch_rows_top2_f32(int M, int V, const float* logits, int32_t* argmax, float* top1, float* top2,
-                                 cudaStream_t s) {
-  rows_top2_f32_kernel<<<(M + 7) / 8, 256, 0, s>>>(M, V, logits, argmax, top1, top2);
+                                 cudaStream_t s, float inv_temp, uint32_t seed_lo, uint32_t seed_hi,
+                                 const int32_t* row_sid, const int32_t* row_pos) {
+  if (inv_temp > 0.f && (!row_sid || !row_pos)) return cudaErrorInvalidValue;
+  rows_top2_f32_kernel<<<(M + 7) / 8, 256, 0, s>>>(M, V, logits, argmax, top1, top2, inv_temp, seed_lo, seed_hi,
+                                                   row_sid, row_pos);
   return cudaGetLastError();
 }
 

@@ -289,6 +289,8 @@ struct spec_handle {
   uint8_t* h_out = nullptr;
   float* dbg_logits = nullptr;
   size_t dbg_bytes = 0;
+  float temperature = 0.f;  // > 0: tokens are sampled (spec_set_sampling); 0: greedy
+  uint64_t seed = 0;
   void* feat_out = nullptr;  // SPEC_FEATURES destination, bf16 [B][max_nodes][3][d]
   size_t feat_bytes = 0;
   void* pf_feat_out = nullptr;  // features of the prefill chunk being run, bf16 [rows][3][d]
@@ -591,8 +593,9 @@ struct PhaseBuilder {
     g.args.ld_out = c.ffn;
     return as_phase(g);
   }
-  // final norm (folded) + LM head with per-tile top-2; logits also stored when given
-  GemmPhase lm(float* logits) const {
+  // final norm (folded) + LM head with per-tile top-2; logits also stored when given;
+  // with `sample`, the top-2 is of the temperature-scaled logits plus the Gumbel noise
+  GemmPhase lm(float* logits, bool sample) const {
     const spec_config& c = h->cfg;
     const WsLayout& L = h->lay;
     GemmTcLaunch g = gemm_launch(sp.lm, GEMM_EPI_ARGMAX, c.vocab, d, M, &h->map_lm, nullptr, nullptr, &h->map_xn[bi],
@@ -600,6 +603,13 @@ struct PhaseBuilder {
     g.args.top_part = h->W<Top2>(L.top_part);
     g.args.top_ld = L.Mpad;
     g.args.dbg_logits = logits;
+    if (sample) {
+      g.args.inv_temp = 1.f / h->temperature;
+      g.args.seed_lo = (uint32_t)h->seed;
+      g.args.seed_hi = (uint32_t)(h->seed >> 32);
+      g.args.row_sid = sv.row_sid;
+      g.args.row_pos = sv.row_pos;
+    }
     g.args.ss_in = h->W<float>(L.ss);
     g.args.n_ss = L.n_ss;
     g.args.ss_ld = L.Mpad;
@@ -702,7 +712,7 @@ cudaError_t enqueue_step(spec_handle* h, const StepPlan& sp, int mode, bool dbg,
       m.ph[0] = pb.o(l, 4 * (l + 1) + 0);
       m.ph[1] = pb.gu(l);
       m.ph[2] = pb.down(l, 4 * (l + 1) + 2, next_norm);
-      m.ph[3] = (l + 1 < c.n_layers) ? pb.qkv(l + 1, 4 * (l + 1) + 3) : pb.lm(dbg ? h->dbg_logits : nullptr);
+      m.ph[3] = (l + 1 < c.n_layers) ? pb.qkv(l + 1, 4 * (l + 1) + 3) : pb.lm(dbg ? h->dbg_logits : nullptr, h->temperature > 0.f);
       if (h->trace && l == h->trace_layer) m.trace = h->trace;
       LK(SPEC_PROF_GEMM_LAYER, 1, gemm_multi_launch(m, st, pdl));
       CUDA_RET(tap_after(l + 1, pdl));
@@ -738,7 +748,10 @@ cudaError_t enqueue_step(spec_handle* h, const StepPlan& sp, int mode, bool dbg,
   } else {
     LK(SPEC_PROF_LM_HEAD, 1,
        launch_gemm_simt_f32((const float*)xn, d, (const float*)h->lm_head, d, part, c.vocab, M, c.vocab, st));
-    LK(SPEC_PROF_LM_REDUCE, 1, launch_rows_top2_f32(M, c.vocab, part, amax, h->W<float>(L.top1), h->W<float>(L.top2), st));
+    LK(SPEC_PROF_LM_REDUCE, 1,
+       launch_rows_top2_f32(M, c.vocab, part, amax, h->W<float>(L.top1), h->W<float>(L.top2), st,
+                            h->temperature > 0.f ? 1.f / h->temperature : 0.f, (uint32_t)h->seed,
+                            (uint32_t)(h->seed >> 32), sv.row_sid, sv.row_pos));
     if (dbg && h->dbg_logits) {
       cudaError_t e = cudaMemcpyAsync(h->dbg_logits, part, sizeof(float) * (size_t)M * c.vocab,
                                       cudaMemcpyDeviceToDevice, st);
@@ -864,7 +877,7 @@ cudaError_t enqueue_draft(spec_handle* h, const StepPlan& sp, bool kv_only, bool
   m.ph[0] = pb.o(Ld, 8 + 0);
   m.ph[1] = pb.gu(Ld);
   m.ph[2] = pb.down(Ld, 8 + 2, h->draft_final_norm);
-  m.ph[3] = pb.lm(logits);
+  m.ph[3] = pb.lm(logits, false);  // the draft head's own top-k reads the logits
   LK(SPEC_PROF_GEMM_LAYER, 1, gemm_multi_launch(m, st, pdl));
   if (ts)
     LK(SPEC_PROF_TOPK, 1,
@@ -1614,6 +1627,21 @@ int spec_set_feature_out(spec_handle* h, void* device_buf, size_t bytes) {
   h->feat_out = device_buf;
   h->feat_bytes = device_buf ? bytes : 0;
   // graphs bake the pointer in
+  for (auto& kv : h->graphs) cudaGraphExecDestroy(kv.second);
+  h->graphs.clear();
+  return SPEC_OK;
+}
+
+int spec_set_sampling(spec_handle* h, float temperature, uint64_t seed) {
+  if (!h) return SPEC_ERR_ARG;
+  h->err.clear();
+  if (!(temperature >= 0.f) || !std::isfinite(temperature))
+    return fail(h, SPEC_ERR_ARG, "temperature %g must be finite and >= 0", (double)temperature);
+  if (temperature > 0.f && !std::isfinite(1.f / temperature))
+    return fail(h, SPEC_ERR_ARG, "temperature %g is too small (1/T overflows)", (double)temperature);
+  h->temperature = temperature;
+  h->seed = seed;
+  // graphs bake the launch arguments in
   for (auto& kv : h->graphs) cudaGraphExecDestroy(kv.second);
   h->graphs.clear();
   return SPEC_OK;

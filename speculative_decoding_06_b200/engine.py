@@ -186,6 +186,10 @@ class SpecEngine:
                                        _fptr(t1), _fptr(t2), flags))
         return amax, t1, t2, off
 
+    def set_sampling(self, temperature: float, seed: int = 0):
+        """Temperature sampling (T > 0) or greedy choices (T = 0) for later calls (spec_set_sampling)."""
+        self._check(S.spec_set_sampling(self.h, float(temperature), int(seed)))
+
     def enable_debug_logits(self, rows: int):
         self._dbg = torch.empty(rows * self.dims.vocab, dtype=torch.float32, device="cuda")
         self._check(S.spec_set_debug_logits(self.h, self._dbg.data_ptr(), self._dbg.numel() * 4))

@@ -85,6 +85,7 @@ _SIGNATURES = {
     "spec_score_trees": (ctypes.c_int, [_h, ctypes.c_int, _i32p, _i32p, _i32p, _i32p, _i32p, _f32p, _f32p,
                                         ctypes.c_int]),
     "spec_set_debug_logits": (ctypes.c_int, [_h, _vp, ctypes.c_size_t]),
+    "spec_set_sampling": (ctypes.c_int, [_h, ctypes.c_float, ctypes.c_uint64]),
     "spec_set_feature_out": (ctypes.c_int, [_h, _vp, ctypes.c_size_t]),
     "spec_truncate": (ctypes.c_int, [_h, ctypes.c_int, ctypes.c_int]),
     "spec_seq_len": (ctypes.c_int, [_h, ctypes.c_int, _i32p, _i32p]),

@@ -114,3 +114,7 @@ def test_new_entry_points_reject_bad_arguments_without_gpu():
     assert S.spec_wait_selftest(None, 1000, ctypes.byref(i32)) == S.SPEC_ERR_ARG
     assert S.spec_wait_selftest(ctypes.c_void_p(16), 0, ctypes.byref(i32)) == S.SPEC_ERR_ARG
     assert S.spec_wait_selftest(ctypes.c_void_p(18), 1000, ctypes.byref(i32)) == S.SPEC_ERR_ARG  # misaligned
+
+
+def test_sampling_setter_without_handle():
+    assert S.spec_set_sampling(None, 0.7, 1) == S.SPEC_ERR_ARG
