@@ -368,6 +368,8 @@ def run_ours(args, rank, world, local_rank):
     P = args.prefix
     w = synth.model_weights(dims, seed=0, device="cuda")
     eng = SpecEngine(dims, w, max_batch=1, max_seq=P + 256, max_nodes=64)
+    if args.temperature > 0:
+        eng.set_sampling(args.temperature, 1)  # tokens are draws at temperature T (planting included)
     prefix = synth.prefix_tokens(dims.vocab, P, seed=1)
     pend = eng.prefill(0, prefix)
     shape = synth.tree_from_widths(synth.TREE60_WIDTHS, stream=0)
@@ -459,7 +461,8 @@ def run_ours(args, rank, world, local_rank):
         "metric": METRIC, "value": value, "unit": UNIT, "n_gpus": world, "steps": args.steps,
         "warmup": max(3, args.warmup), "ms_per_step": ms, "higher_is_better": True, "scaling": "weak",
         "vs_baseline": None, "dtype": "bf16", "data": "synthetic (random-init weights, uniform prefix, planted tree)",
-        "config": workload_config(P, args.layers),
+        "config": dict(workload_config(P, args.layers), **({"temperature": args.temperature}
+                                                           if args.temperature > 0 else {})),
         "accepted_tokens_per_s": value * (a_len + 1), "tau": a_len + 1,
         "roofline": {"bound": "hbm", "kernel": dom, "achieved": achieved, "peak": hbm, "unit": "GB/s",
                      "frac": achieved / hbm, "traffic": measured_traffic(dom, cb[dom] / dom_n),
@@ -824,6 +827,8 @@ def main():
     ap.add_argument("--sample-layers", type=int, default=2)
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--batch", type=int, default=1, help="sequences decoded together (--workload decode)")
+    ap.add_argument("--temperature", type=float, default=0.0,
+                    help="verify workload: sample at this temperature instead of greedy choices (0: greedy)")
     ap.add_argument("--layers", type=int, default=32, help="decoder layers (32 = the 8B shape; fewer only for profiling)")
     ap.add_argument("--workload", default="verify", choices=["verify", "batch64", "sweep", "draft", "draft_tree", "decode"],
                     help="verify: the default line (batch 1, prefix 2048); the others measure the remaining"
