@@ -230,7 +230,7 @@ __device__ __forceinline__ bool spin_until_geq(const int* p, int target, uint32_
       set_error(err, SPEC_DEVERR_TIMEOUT);
       return false;
     }
-    __nanosleep(64);
+    __nanosleep(20);
   }
 }
 
@@ -389,10 +389,12 @@ __device__ __forceinline__ void fence_proxy_async_smem() {
 // A bf16 model's GEMM activations are stored as two bf16 parts, hi = bf16(v)
 // and lo = bf16(v - hi), which together carry ~16 mantissa bits; the weights
 // are exact bf16, so W.hi + W.lo reproduces W.v to fp32-accumulation accuracy.
-// Layout: tokens in groups of 64; group g occupies 128 rows, its 64 hi rows
-// followed by its 64 lo rows.  A GEMM tile of BN tokens (BN a multiple of 64)
-// is one contiguous box of 2*BN rows.
-constexpr int kSplitGroup = 64;
+// Layout: tokens in groups of 32; group g occupies 64 rows, its 32 hi rows
+// followed by its 32 lo rows.  A GEMM tile of BN tokens (BN a multiple of 32:
+// 64, 96, 128) is one contiguous box of 2*BN rows, and in the tile's
+// accumulator token c's hi column is (c / 32) * 64 + c % 32, its lo column 32
+// further.
+constexpr int kSplitGroup = 32;
 __host__ __device__ __forceinline__ int split_row(int t, int part) {
   return (t / kSplitGroup) * (2 * kSplitGroup) + part * kSplitGroup + (t % kSplitGroup);
 }

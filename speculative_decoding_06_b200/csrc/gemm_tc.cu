@@ -66,7 +66,8 @@ struct SmemLayout {
   static constexpr uint32_t total = misc_off + 16;
   static constexpr uint32_t dyn_bytes = total + 1024;  // slack to align the base to 1024
   static constexpr uint32_t acc_cols = 2 * BN;             // one accumulator: hi and lo columns
-  static constexpr uint32_t tmem_cols = 2 * acc_cols;       // two accumulators
+  // two accumulators, allocated as a power of two of at least 32 columns
+  static constexpr uint32_t tmem_cols = 2 * acc_cols <= 256 ? 256u : 512u;
 };
 
 __device__ __forceinline__ void named_sync(int id, int n) {
@@ -242,7 +243,7 @@ __global__ void __launch_bounds__(kThreads, BN == 64 ? 2 : 1)
                 *abort_flag = 1;
                 return false;
               }
-              __nanosleep(256);
+              __nanosleep(32);
             }
           }
           issue_b(p, pend_stage[done], pend_kx[done], pend_row[done]);
@@ -414,14 +415,17 @@ __global__ void __launch_bounds__(kThreads, BN == 64 ? 2 : 1)
           const int o = to * kTileO + row_in_tile;
           float* out = args.part + (size_t)sp * args.split_stride + o;
 #pragma unroll 1
-          for (int c0 = 0; c0 < BN; c0 += 16) {
-            float v[16], vl[16];
-            const uint32_t col = (c0 / 64) * 128 + (c0 % 64);
-            tmem_ld16x2(taddr + col, taddr + col + 64, v, vl);
+          for (int c0 = 0; c0 < BN; c0 += 32) {
+            // 32 tokens' hi and lo columns in two loads and one wait
+            uint32_t v[32], vl[32];
+            const uint32_t col = (c0 / kSplitGroup) * (2 * kSplitGroup) + (c0 % kSplitGroup);
+            tmem_ld32_async(taddr + col, v);
+            tmem_ld32_async(taddr + col + kSplitGroup, vl);
+            tmem_wait_ld();
 #pragma unroll
-            for (int i = 0; i < 16; ++i) {
+            for (int i = 0; i < 32; ++i) {
               const int t = t_base + c0 + i;
-              if (t < args.M) out[(size_t)t * args.n_out] = v[i] + vl[i];
+              if (t < args.M) out[(size_t)t * args.n_out] = __uint_as_float(v[i]) + __uint_as_float(vl[i]);
             }
           }
           if (first_unit && ep_tid == 0) stamp(P.trace, p, 8);
@@ -598,8 +602,8 @@ __global__ void __launch_bounds__(kThreads, BN == 64 ? 2 : 1)
 #pragma unroll 1
           for (int c0 = 0; c0 < BN; c0 += 16) {
             float v[16], vl[16];
-            const uint32_t col = (c0 / 64) * 128 + (c0 % 64);
-            tmem_ld16x2(taddr + col, taddr + col + 64, v, vl);
+            const uint32_t col = (c0 / kSplitGroup) * (2 * kSplitGroup) + (c0 % kSplitGroup);
+            tmem_ld16x2(taddr + col, taddr + col + kSplitGroup, v, vl);
 #pragma unroll
             for (int i = 0; i < 16; ++i) stage[row_in_tile * 17 + i] = (v[i] + vl[i]) * r_s[c0 + i];
             named_sync(1, 128);
@@ -625,8 +629,8 @@ __global__ void __launch_bounds__(kThreads, BN == 64 ? 2 : 1)
 #pragma unroll 1
           for (int c0 = 0; c0 < BN; c0 += 16) {
             float v[16], vl[16];
-            const uint32_t col = (c0 / 64) * 128 + (c0 % 64);
-            tmem_ld16x2(taddr + col, taddr + col + 64, v, vl);
+            const uint32_t col = (c0 / kSplitGroup) * (2 * kSplitGroup) + (c0 % kSplitGroup);
+            tmem_ld16x2(taddr + col, taddr + col + kSplitGroup, v, vl);
 #pragma unroll
             for (int i = 0; i < 16; ++i) {
               const int t = t_base + c0 + i;
@@ -642,8 +646,8 @@ __global__ void __launch_bounds__(kThreads, BN == 64 ? 2 : 1)
 #pragma unroll 1
           for (int c0 = 0; c0 < BN; c0 += 16) {
             float v[16], vl[16];
-            const uint32_t col = (c0 / 64) * 128 + (c0 % 64);
-            tmem_ld16x2(taddr + col, taddr + col + 64, v, vl);
+            const uint32_t col = (c0 / kSplitGroup) * (2 * kSplitGroup) + (c0 % kSplitGroup);
+            tmem_ld16x2(taddr + col, taddr + col + kSplitGroup, v, vl);
 #pragma unroll
             for (int i = 0; i < 16; ++i) v[i] = (v[i] + vl[i]) * r_s[c0 + i];
 #pragma unroll
@@ -705,10 +709,13 @@ __global__ void __launch_bounds__(kThreads, BN == 64 ? 2 : 1)
 // host-side launch helpers
 // ---------------------------------------------------------------------------
 
-// BN = 64 tokens: 3 stages of 32 KB (two CTAs per SM); BN = 128: 4 stages of 48 KB (one per SM)
+// BN = 64 tokens: 3 stages of 32 KB (two CTAs per SM); BN = 96: 5 stages of 40 KB and BN = 128:
+// 4 stages of 48 KB (one CTA per SM)
 template <int BN, int STAGES>
 static cudaError_t launch_impl(const GemmMultiLaunch& L_, cudaStream_t stream, bool pdl) {
   using L = SmemLayout<BN, STAGES>;
+  static_assert(L::dyn_bytes <= 227 * 1024, "shared memory per CTA");
+  static_assert(BN % kSplitGroup == 0 && 2 * BN <= 256, "token tile: whole split groups, one TMA box");
   GemmMaps maps;
   GemmPhases ph;
   memset(&maps, 0, sizeof(maps));
@@ -740,17 +747,20 @@ static cudaError_t launch_impl(const GemmMultiLaunch& L_, cudaStream_t stream, b
 }
 
 uint32_t gemm_tc_smem_bytes(int bn) {
-  return bn == 64 ? SmemLayout<64, 3>::dyn_bytes : SmemLayout<128, 4>::dyn_bytes;
+  return bn == 64 ? SmemLayout<64, 3>::dyn_bytes
+                  : bn == 96 ? SmemLayout<96, 5>::dyn_bytes : SmemLayout<128, 4>::dyn_bytes;
 }
 
 const void* gemm_tc_function(int bn) {
-  return bn == 64 ? (const void*)gemm_tc_kernel<64, 3> : (const void*)gemm_tc_kernel<128, 4>;
+  return bn == 64 ? (const void*)gemm_tc_kernel<64, 3>
+                  : bn == 96 ? (const void*)gemm_tc_kernel<96, 5> : (const void*)gemm_tc_kernel<128, 4>;
 }
 
 cudaError_t gemm_multi_launch(const GemmMultiLaunch& L, cudaStream_t stream, bool pdl) {
   if (L.n_phases < 1 || L.n_phases > kMaxGemmPhases) return cudaErrorInvalidValue;
   if (L.n_phases > 1 && !L.phase_bar) return cudaErrorInvalidValue;
   if (L.bn == 64) return launch_impl<64, 3>(L, stream, pdl);
+  if (L.bn == 96) return launch_impl<96, 5>(L, stream, pdl);
   if (L.bn == 128) return launch_impl<128, 4>(L, stream, pdl);
   return cudaErrorInvalidValue;
 }

@@ -268,17 +268,17 @@ struct spec_handle {
   uint8_t* ws = nullptr;
   std::vector<LayerMaps> maps;
   CUtensorMap map_lm;
-  CUtensorMap map_xn[2], map_attn[2], map_h[2];  // B operands for BN = 64, 128
+  CUtensorMap map_xn[3], map_attn[3], map_h[3];  // B operands for BN = 64, 128, 96 (bn_slot)
   AttnTcMaps attn_maps;                           // q and the K/V cache (fp16)
   // draft head (cfg.draft_head): its decoder layer is layers[n_layers], maps[n_layers]
   const void* draft_fc_fuse = nullptr;
   const void* draft_fc_in = nullptr;
   const void* draft_final_norm = nullptr;
-  CUtensorMap map_fc_fuse, map_fc_in, map_fsplit[2], map_ge[2];
+  CUtensorMap map_fc_fuse, map_fc_in, map_fsplit[3], map_ge[3];
   std::vector<int32_t> dlen;        // draft-head prefix length per sequence
   std::vector<uint8_t> dready;
-  int resident[2][4] = {{0, 0, 0, 0}, {0, 0, 0, 0}};   // co-resident CTAs per SM [bn][epi]
-  int occ_api[2][4] = {{0, 0, 0, 0}, {0, 0, 0, 0}};    // what the occupancy query reported
+  int resident[3][4] = {};  // co-resident CTAs per SM [bn_slot][epi]
+  int occ_api[3][4] = {};   // what the occupancy query reported
   // host mirror of per-sequence state
   std::vector<int32_t> len, pending;
   std::vector<int32_t> len_hi;  // upper bound while device-output steps are in flight
@@ -303,6 +303,7 @@ struct spec_handle {
   int attn_clusters[kAttnMaxChunks + 1] = {};  // co-resident clusters of n chunk CTAs
   bool attn_dsmem = true;     // merge chunk partials through distributed shared memory when they fit a cluster
   int bn64_max = 64;          // largest token count planned with 64-token tiles (several token tiles above 64)
+  bool bn96 = true;           // 96-token tiles for 65 .. 96 tokens (else 128)
   // L2 prefetch of weights ahead of the GEMM that streams them
   uint64_t* trace = nullptr;  // optional GEMM timeline of one layer's launch
   size_t trace_bytes = 0;
@@ -364,10 +365,14 @@ cudaError_t launch_k(spec_handle* h, int cls, int n_kernels, F&& fn) {
   return cudaSuccess;
 }
 
+// index of a token-tile width in the per-width tables (tensor maps, residency)
+int bn_slot(int bn) { return bn == 64 ? 0 : bn == 128 ? 1 : 2; }
+constexpr int kTileWidths[3] = {64, 128, 96};
+
 GemmPlan plan_gemm(const spec_handle* h, int rows_per_tile, int n_out, int K, int M, int epi) {
   GemmPlan p;
-  p.bn = M <= h->bn64_max ? 64 : 128;
-  const int bi = p.bn == 64 ? 0 : 1;
+  p.bn = M <= h->bn64_max ? 64 : (h->bn96 && M <= 96 ? 96 : 128);
+  const int bi = bn_slot(p.bn);
   int per_sm = std::max(1, h->resident[bi][0]);  // one kernel function for every epilogue
   if (h->resident_cap > 0) per_sm = std::min(per_sm, h->resident_cap);
   const int resident = per_sm * h->sm_count;
@@ -424,7 +429,7 @@ StepPlan make_plan(const spec_handle* h, int B, int M, int max_n, int max_lk) {
   s.down = plan_gemm(h, 128, c.hidden, c.ffn, M, GEMM_EPI_RESID);
   s.lm = plan_gemm(h, 128, c.vocab, c.hidden, M, GEMM_EPI_ARGMAX);
   {
-    const int bi = s.qkv.bn == 64 ? 0 : 1;
+    const int bi = bn_slot(s.qkv.bn);
     int per_sm = std::max(1, h->resident[bi][0]);
     if (h->resident_cap > 0) per_sm = std::min(per_sm, h->resident_cap);
     s.grid_all = per_sm * h->sm_count;
@@ -506,7 +511,7 @@ struct PhaseBuilder {
   int bi, d, qd, kvd, nqkv, M;
   PhaseBuilder(spec_handle* h_, const StepPlan& sp_, const StepView& sv_) : h(h_), sp(sp_), sv(sv_) {
     const spec_config& c = h->cfg;
-    bi = sp.qkv.bn == 64 ? 0 : 1;
+    bi = bn_slot(sp.qkv.bn);
     d = c.hidden;
     qd = c.n_q_heads * c.head_dim;
     kvd = c.n_kv_heads * c.head_dim;
@@ -801,7 +806,7 @@ cudaError_t enqueue_draft(spec_handle* h, const StepPlan& sp, bool kv_only, bool
   StepView sv = make_view(h, sp.B, sp.M);
   sv.seq_len = h->W<int32_t>(L.p_dlen);
   const int d = c.hidden, M = sp.M, Ld = c.n_layers;
-  const int bi = sp.qkv.bn == 64 ? 0 : 1;
+  const int bi = bn_slot(sp.qkv.bn);
   h->launches = 0;
   CUDA_RET(cudaMemsetAsync(h->ws + L.gemm_ctr, 0, 4 * (size_t)L.gemm_ctr_n, st));
   CUDA_RET(cudaMemsetAsync(h->ws + L.attn_ctr, 0, 4 * (size_t)L.attn_ctr_n, st));
@@ -1241,6 +1246,7 @@ int spec_init(const spec_config* cfg, const spec_weights* w, void* kv_cache, siz
     if (const char* q = strstr(t, "pdl=")) if (sscanf(q + 4, "%d", &v) == 1) h->use_pdl = v != 0;
     if (const char* q = strstr(t, "dsmem=")) if (sscanf(q + 6, "%d", &v) == 1) h->attn_dsmem = v != 0;
     if (const char* q = strstr(t, "bn64max=")) if (sscanf(q + 8, "%d", &v) == 1 && v >= 64) h->bn64_max = v;
+    if (const char* q = strstr(t, "bn96=")) if (sscanf(q + 5, "%d", &v) == 1) h->bn96 = v != 0;
     if (const char* q = strstr(t, "per_sm=")) if (sscanf(q + 7, "%d", &v) == 1 && v >= 0) h->resident_cap = v;
     float fv = 0.f;
     if (const char* q = strstr(t, "rescale=")) if (sscanf(q + 8, "%f", &fv) == 1 && fv >= 0.f && fv <= 15.f) h->rescale_slack = fv;
@@ -1303,8 +1309,8 @@ int spec_init(const spec_config* cfg, const spec_weights* w, void* kv_cache, siz
         (!make_tmap(&h->map_fc_fuse, h->draft_fc_fuse, c.hidden, 3 * (uint64_t)c.hidden, 128) ||
          !make_tmap(&h->map_fc_in, h->draft_fc_in, c.hidden, 2 * (uint64_t)c.hidden, 128)))
       return bail(SPEC_ERR_CUDA, "tensor map");
-    const int bns[2] = {64, 128};
-    for (int i = 0; i < 2; ++i) {
+    const int* bns = kTileWidths;
+    for (int i = 0; i < 3; ++i) {
       // split activations: a tile of BN tokens is 2*BN rows (hi and lo)
       if (!make_tmap(&h->map_xn[i], h->ws + lay.xn, 2 * (uint64_t)lay.Mpad, c.hidden, 2 * bns[i]) ||
           !make_tmap(&h->map_attn[i], h->ws + lay.attn, 2 * (uint64_t)lay.Mpad, qd, 2 * bns[i]) ||
@@ -1316,7 +1322,7 @@ int spec_init(const spec_config* cfg, const spec_weights* w, void* kv_cache, siz
            !make_tmap(&h->map_ge[i], h->ws + lay.ge, 2 * (uint64_t)lay.Mpad, 2 * (uint64_t)c.hidden, 2 * bns[i])))
         return bail(SPEC_ERR_CUDA, "tensor map");
     }
-    for (int i = 0; i < 2; ++i)
+    for (int i = 0; i < 3; ++i)
       for (int e = 0; e < 4; ++e) {
         const void* fn = gemm_tc_function(bns[i]);
         const int smem = (int)gemm_tc_smem_bytes(bns[i]);
@@ -1752,8 +1758,8 @@ int spec_info(spec_handle* h, int B, int n_nodes, int prefix, char* buf, size_t 
   };
   std::string s = "sms " + std::to_string(h->sm_count) + "; attention clusters held [size:count]";
   for (int cs = 2; cs <= kAttnMaxChunks; ++cs) s += " " + std::to_string(cs) + ":" + std::to_string(h->attn_clusters[cs]);
-  s += "; resident/SM [bn64|bn128][qkv,swiglu,argmax,resid] = ";
-  for (int i = 0; i < 2; ++i)
+  s += "; resident/SM [bn64|bn128|bn96][qkv,swiglu,argmax,resid] = ";
+  for (int i = 0; i < 3; ++i)
     for (int e = 0; e < 4; ++e)
       s += std::to_string(h->resident[i][e]) + "(" + std::to_string(h->occ_api[i][e]) + ")" + (e < 3 ? "," : "|");
   s += "; qkv " + g(sp.qkv) + "; o " + g(sp.o) + "; gate_up " + g(sp.gu) + "; down " + g(sp.down) + "; lm " +

@@ -81,6 +81,7 @@ BF16_CASES = [
     ("mini", 129, "tree127", 133, 133),
     ("small", 700, "tree60", 700, 2700),
     ("small", 64, "chain8", 64, 64),
+    ("small", 500, "tree80", 500, 500),  # 81 tokens: 96-token GEMM tiles
 ]
 
 
@@ -97,6 +98,8 @@ def _shape(kind):
         return synth.tree_from_widths(synth.TREE60_WIDTHS, stream=4)
     if kind == "tree127":
         return synth.tree_from_widths((10, 12, 16, 20, 20, 20, 16, 13), stream=5)
+    if kind == "tree80":
+        return synth.tree_from_widths(synth.SWEEP_WIDTHS[80], stream=6)
     raise KeyError(kind)
 
 
