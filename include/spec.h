@@ -127,8 +127,10 @@ typedef struct spec_weights {
 
 typedef struct spec_handle spec_handle;
 
-/* Bytes of device memory for the K/V cache (layout [layer][K|V][seq][kv head][slot][hd];
- * fp16 elements for bf16 models, fp32 for fp32 models). */
+/* Bytes of device memory for the K/V cache.  Layout [layer][plane][seq][kv head][slot][hd]:
+ * fp32 models hold planes K, V (fp32); bf16 models hold K, V and K_lo in fp16, where
+ * K_lo = fp16(k - fp16(k)) carries the rounding error of K so that the attention
+ * scores see ~22 bits of each key. */
 SPEC_API size_t spec_kv_bytes(const spec_config* cfg);
 /* Bytes of device workspace (activations, split-K partials, per-sequence state). */
 SPEC_API size_t spec_workspace_bytes(const spec_config* cfg);

@@ -109,10 +109,10 @@ __global__ void __launch_bounds__(256) kv_compact_kernel(StepView sv, KvView kv,
   const int b = blockIdx.y;
   const int a = acc_len[b];
   if (a <= 0) return;
-  const int lk = blockIdx.x;  // layer * 2 * Hkv + kvsel * Hkv + head
+  const int lk = blockIdx.x;  // (layer * planes + plane) * Hkv + head
   const int head = lk % kv.Hkv;
-  const int kvsel = (lk / kv.Hkv) & 1;
-  const int layer = lk / (2 * kv.Hkv);
+  const int kvsel = (lk / kv.Hkv) % kv.planes;
+  const int layer = lk / (kv.planes * kv.Hkv);
   const int P = sv.P_step[b];
   const int seq = sv.seq_ids[b];
   uint8_t* base = reinterpret_cast<uint8_t*>(kv.base) +
@@ -147,7 +147,7 @@ cudaError_t launch_kv_compact(const StepView& sv, const KvView& kv, int n_layers
   attr[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
   attr[0].val.programmaticStreamSerializationAllowed = 1;
   cudaLaunchConfig_t cfg = {};
-  cfg.gridDim = dim3(n_layers * 2 * kv.Hkv, sv.B);
+  cfg.gridDim = dim3(n_layers * kv.planes * kv.Hkv, sv.B);
   cfg.blockDim = dim3(256);
   cfg.dynamicSmemBytes = smem;
   cfg.stream = s;

@@ -8,27 +8,38 @@
 //
 // One CTA handles one (sequence, kv head, tile of 128 query rows, key chunk).
 // The query rows of a kv head are its G = Hq/Hkv heads for every tree node
-// (row = node * G + g), so one K/V block serves all of them.  q and the K/V
-// cache are fp16; the probabilities P are rounded to fp16 for the P.V product;
-// scores and outputs accumulate in fp32 in tensor memory.
+// (row = node * G + g), so one K/V block serves all of them.
 //
-//   warp 4 (one thread): TMA loads of Q and of 128-key K/V blocks (two stages),
-//                        S_j = Q K_j^T into one of two 128-column TMEM buffers,
-//                        O += P_j V_j into a third (V is read MN-major);
-//   warps 0-3:           thread r owns query row r: reads S_j from its TMEM
-//                        lane, applies the ancestor mask and the online softmax
-//                        (the running max only moves when a block's max exceeds
-//                        it by more than the slack, 8 in log2 units by default:
-//                        every p stays <= 2^8 and O is rescaled rarely),
-//                        writes P_j into shared memory as the next MMA's A
-//                        operand, and at the end normalises O.
+// Precision: the scores carry ~22 bits.  q and K come in two fp16 parts each
+// (hi, and lo = the rounding error of hi; the cache holds K, V and K_lo
+// planes), and S = Q_hi K_hi^T + Q_hi K_lo^T + Q_lo K_hi^T accumulates in fp32
+// in tensor memory; the probabilities come in two fp16 parts too,
+// O += P_hi V + P_lo V, with V single fp16 and O accumulating in fp32.  (With
+// one fp16 part for q and K the scores' rounding dominated the logit error of a
+// 32-layer model of the 8B shape; P's rounding made a node's logits depend on
+// where key chunks start.)
+//
+//   warp 8 (one thread): TMA loads of Q (hi, lo) and of 64-key blocks of K, K_lo
+//                        and V (two stages), the three S MMAs of a block into
+//                        one of two 64-column TMEM buffers, O += P_j V_j into a
+//                        128-column buffer (V read MN-major);
+//   warps 0-7:           two threads per query row (warps w and w + 4 share the
+//                        row's TMEM lane; each takes 32 of the block's keys):
+//                        read S_j, apply the ancestor mask and the online
+//                        softmax (the running max moves only when a block's max
+//                        exceeds it by more than the slack, 8 in log2 units by
+//                        default: every p stays <= 2^8 and O is rescaled
+//                        rarely), write P_j (hi and lo) into shared memory as
+//                        the next MMAs' A operands, and at the end normalise O.
 //
 // A sequence's keys are cut into chunks so that short-prefix, small-batch steps
 // still occupy the GPU; the chunk CTAs of one (sequence, kv head, row tile)
 // are co-resident (the plan keeps the grid within one CTA per SM), publish
-// fp32 partials (normalised O and log2-sum-exp), meet at a bounded counter, and
-// each merges a slice of the rows.  With one chunk the CTA writes its rows
-// directly.  The output is split bf16 (hi, lo) for the O-projection GEMM.
+// fp32 partials (normalised O and log2-sum-exp) and merge them through global
+// memory (a bounded counter, then each CTA merges a slice of the rows) or,
+// when every group's cluster fits on the GPU at once, through distributed
+// shared memory.  With one chunk the CTA writes its rows directly.  The output
+// is split bf16 (hi, lo) for the O-projection GEMM.
 #include <cuda.h>
 
 #include "common.cuh"
@@ -39,21 +50,28 @@ namespace spec {
 namespace {
 
 constexpr int kRows = 128;                   // query rows per CTA (the MMA M)
-constexpr int kKeys = 128;                   // keys per block (S's N, P.V's K)
+constexpr int kKeys = kAttnTcKeys;           // keys per block (S's N, P.V's K): 64
 constexpr int kThreads = 288;                // warps 0-7 rows (two per row), warp 8 issue
 constexpr int kCtrlWarp = 8;
-constexpr uint32_t kHalf = 128 * 128;        // [128 rows][64 fp16] swizzled: 16 KB
-constexpr uint32_t kTile = 2 * kHalf;        // 128 x 128 fp16: 32 KB
+constexpr uint32_t kQHalf = kRows * 128;     // [128 rows][64 fp16] swizzled: 16 KB
+constexpr uint32_t kQTile = 2 * kQHalf;      // 128 x 128 fp16: 32 KB
+constexpr uint32_t kKHalf = kKeys * 128;     // [64 keys][64 fp16] swizzled: 8 KB
+constexpr uint32_t kKTile = 2 * kKHalf;      // 64 x 128 fp16: 16 KB
+constexpr uint32_t kPTile = kRows * kKeys * 2;  // [128 rows][64 keys] fp16, one 128-byte row each: 16 KB
+static_assert(kKeys == 64, "a P row is one 128-byte swizzled row; two 32-key pieces per block");
 
 enum { B_QFULL = 0, B_KVFULL = 1, B_KVEMPTY = 3, B_SFULL = 5, B_SFREE = 7, B_PFULL = 9, B_PEMPTY = 10, B_OFULL = 11,
        B_DRAIN = 12, kNumBars = 13 };
 
 struct Smem {
-  static constexpr uint32_t q = 0;
-  static constexpr uint32_t k = q + kTile;          // 2 stages
-  static constexpr uint32_t v = k + 2 * kTile;      // 2 stages
-  static constexpr uint32_t p = v + 2 * kTile;
-  static constexpr uint32_t xchg = p + kTile;        // row maxima [2][2][128] and sums [2][128]
+  static constexpr uint32_t q = 0;                   // Q hi
+  static constexpr uint32_t qlo = q + kQTile;        // Q lo
+  static constexpr uint32_t k = qlo + kQTile;        // 2 stages; with klo, 64 KB of output staging at the end
+  static constexpr uint32_t klo = k + 2 * kKTile;    // 2 stages
+  static constexpr uint32_t v = klo + 2 * kKTile;    // 2 stages
+  static constexpr uint32_t p = v + 2 * kKTile;      // P hi
+  static constexpr uint32_t plo = p + kPTile;        // P lo
+  static constexpr uint32_t xchg = plo + kPTile;     // row maxima [2][2][128] and sums [2][128]
   static constexpr uint32_t lse = xchg + 6 * 128 * 4; // this chunk's log2-sum-exp per row (cluster merge)
   static constexpr uint32_t bars = lse + 128 * 4;
   static constexpr uint32_t misc = bars + kNumBars * 8;  // tmem slot, abort flag, merge flag
@@ -62,13 +80,15 @@ struct Smem {
 };
 static_assert(Smem::dyn <= 227 * 1024, "shared memory");
 
-// tensor-memory columns: S buffers at 0 and 128, O at 256
-constexpr uint32_t kTmemCols = 512;
-constexpr uint32_t kColO = 256;
+// tensor-memory columns: S buffers at 0 and 64, O at 128
+constexpr uint32_t kTmemCols = 256;
+constexpr uint32_t kColO = 2 * kKeys;
+static_assert(kColO + 128 <= kTmemCols, "tensor memory");
+static_assert(Smem::xchg - Smem::k >= 128 * 512, "output staging (128 rows x 512 B) fits in the K / K_lo ring");
 
-// fp16 A and B, f32 D, M = 128, N = 128; bit 16 marks B as MN-major
+// fp16 A and B, f32 D, M = 128; S: N = 64 keys; P.V: N = 128 dims, B MN-major (bit 16)
 constexpr uint32_t kIdescS = (1u << 4) | ((uint32_t)(kKeys >> 3) << 17) | ((uint32_t)(kRows >> 4) << 24);
-constexpr uint32_t kIdescPV = kIdescS | (1u << 16);
+constexpr uint32_t kIdescPV = (1u << 4) | (1u << 16) | ((uint32_t)(128 >> 3) << 17) | ((uint32_t)(kRows >> 4) << 24);
 
 // MN-major operand with the 128-byte swizzle: 64 fp16 along N per 128-byte row,
 // 8-row (K) groups 1024 B apart (stride byte offset), N atoms `lbo` bytes apart
@@ -217,23 +237,29 @@ __global__ void __launch_bounds__(kThreads, 1) attn_tc_kernel(const __grid_const
     } else if (elect_one()) {
       tma_prefetch_desc(&maps.q);
       tma_prefetch_desc(&maps.kv);
-      // cache rows: [layer][K/V][max_batch][Hkv][max_seq]
-      const int krow = (((a.layer * 2 + 0) * a.kv.max_batch + seq) * Hkv + kvh) * a.kv.max_seq;
-      const int vrow = (((a.layer * 2 + 1) * a.kv.max_batch + seq) * Hkv + kvh) * a.kv.max_seq;
+      // cache rows: [layer][K | V | K_lo][max_batch][Hkv][max_seq]
+      const int planes = a.kv.planes;
+      const int krow = (((a.layer * planes + 0) * a.kv.max_batch + seq) * Hkv + kvh) * a.kv.max_seq;
+      const int vrow = (((a.layer * planes + 1) * a.kv.max_batch + seq) * Hkv + kvh) * a.kv.max_seq;
+      const int klrow = (((a.layer * planes + 2) * a.kv.max_batch + seq) * Hkv + kvh) * a.kv.max_seq;
       const int qrow = kvh * a.q_rows + base * G + row0;
+      const int qlrow = qrow + Hkv * a.q_rows;  // the lo part follows all kv heads' hi parts
       const uint64_t pol_q = policy_evict_first();
       const uint64_t pol = policy_evict_normal();  // the other row tiles read the same K/V blocks
       int loaded = 0;
       auto load_kv = [&](int j) {
         const int st = j & 1;
         const int key = c0 + j * kKeys;
-        uint8_t* sk = smem + Smem::k + st * kTile;
-        uint8_t* svb = smem + Smem::v + st * kTile;
-        mbar_arrive_expect_tx(&bar[B_KVFULL + st], 2 * kTile);
+        uint8_t* sk = smem + Smem::k + st * kKTile;
+        uint8_t* skl = smem + Smem::klo + st * kKTile;
+        uint8_t* svb = smem + Smem::v + st * kKTile;
+        mbar_arrive_expect_tx(&bar[B_KVFULL + st], 3 * kKTile);
         tma_load_2d(sk, &maps.kv, &bar[B_KVFULL + st], 0, krow + key, pol);
-        tma_load_2d(sk + kHalf, &maps.kv, &bar[B_KVFULL + st], 64, krow + key, pol);
+        tma_load_2d(sk + kKHalf, &maps.kv, &bar[B_KVFULL + st], 64, krow + key, pol);
+        tma_load_2d(skl, &maps.kv, &bar[B_KVFULL + st], 0, klrow + key, pol);
+        tma_load_2d(skl + kKHalf, &maps.kv, &bar[B_KVFULL + st], 64, klrow + key, pol);
         tma_load_2d(svb, &maps.kv, &bar[B_KVFULL + st], 0, vrow + key, pol);
-        tma_load_2d(svb + kHalf, &maps.kv, &bar[B_KVFULL + st], 64, vrow + key, pol);
+        tma_load_2d(svb + kKHalf, &maps.kv, &bar[B_KVFULL + st], 64, vrow + key, pol);
         loaded = j + 1;
       };
       // blocks made only of prefix keys were written by earlier steps: load
@@ -243,19 +269,25 @@ __global__ void __launch_bounds__(kThreads, 1) attn_tc_kernel(const __grid_const
       while (pre < first && c0 + (pre + 1) * kKeys <= P) load_kv(pre++);
       pdl_wait();
       pdl_launch_dependents();
-      mbar_arrive_expect_tx(&bar[B_QFULL], kTile);
+      mbar_arrive_expect_tx(&bar[B_QFULL], 2 * kQTile);
       tma_load_2d(smem + Smem::q, &maps.q, &bar[B_QFULL], 0, qrow, pol_q);
-      tma_load_2d(smem + Smem::q + kHalf, &maps.q, &bar[B_QFULL], 64, qrow, pol_q);
+      tma_load_2d(smem + Smem::q + kQHalf, &maps.q, &bar[B_QFULL], 64, qrow, pol_q);
+      tma_load_2d(smem + Smem::qlo, &maps.q, &bar[B_QFULL], 0, qlrow, pol_q);
+      tma_load_2d(smem + Smem::qlo + kQHalf, &maps.q, &bar[B_QFULL], 64, qlrow, pol_q);
       for (int j = pre; j < first; ++j) load_kv(j);
       const uint32_t sq = smem_u32(smem + Smem::q);
+      const uint32_t sql = smem_u32(smem + Smem::qlo);
       const uint32_t sp = smem_u32(smem + Smem::p);
+      const uint32_t spl = smem_u32(smem + Smem::plo);
       auto issue_pv = [&](int j) {
-        const uint32_t svv = smem_u32(smem + Smem::v + (j & 1) * kTile);
+        const uint32_t svv = smem_u32(smem + Smem::v + (j & 1) * kKTile);
 #pragma unroll
         for (int kk = 0; kk < kKeys / 16; ++kk) {
-          const uint64_t ad = sw128_kmajor_desc(sp + (kk >> 2) * kHalf + (kk & 3) * 32);
-          const uint64_t bd = sw128_mnmajor_desc(svv + kk * 16 * 128, kHalf);
-          tc_mma_bf16(tmem + kColO, ad, bd, kIdescPV, (j > 0 || kk > 0) ? 1u : 0u);
+          // P: one 128-byte row of 64 keys per query row; V: 16 keys (rows) per step,
+          // its two 64-dim halves kKHalf apart (the N atoms of the MN-major operand)
+          const uint64_t bd = sw128_mnmajor_desc(svv + kk * 16 * 128, kKHalf);
+          tc_mma_bf16(tmem + kColO, sw128_kmajor_desc(sp + kk * 32), bd, kIdescPV, (j > 0 || kk > 0) ? 1u : 0u);
+          tc_mma_bf16(tmem + kColO, sw128_kmajor_desc(spl + kk * 32), bd, kIdescPV, 1u);
         }
       };
       bool ok = mbar_wait(&bar[B_QFULL], 0, err, abort_flag);
@@ -270,12 +302,16 @@ __global__ void __launch_bounds__(kThreads, 1) attn_tc_kernel(const __grid_const
         if (j >= 2) ok = mbar_wait(&bar[B_SFREE + st], ((j - 2) >> 1) & 1, err, abort_flag);
         if (!ok) break;
         tc_fence_after();
-        const uint32_t sk = smem_u32(smem + Smem::k + st * kTile);
+        const uint32_t sk = smem_u32(smem + Smem::k + st * kKTile);
+        const uint32_t skl = smem_u32(smem + Smem::klo + st * kKTile);
 #pragma unroll
-        for (int ks = 0; ks < 8; ++ks) {
-          const uint32_t off = (ks >> 2) * kHalf + (ks & 3) * 32;
-          tc_mma_bf16(tmem + st * kKeys, sw128_kmajor_desc(sq + off), sw128_kmajor_desc(sk + off), kIdescS,
-                      ks > 0 ? 1u : 0u);
+        for (int ks = 0; ks < 8; ++ks) {  // 16 head dims per step
+          const uint32_t oq = (ks >> 2) * kQHalf + (ks & 3) * 32;
+          const uint32_t okey = (ks >> 2) * kKHalf + (ks & 3) * 32;
+          const uint64_t dq = sw128_kmajor_desc(sq + oq), dk = sw128_kmajor_desc(sk + okey);
+          tc_mma_bf16(tmem + st * kKeys, dq, dk, kIdescS, ks > 0 ? 1u : 0u);
+          tc_mma_bf16(tmem + st * kKeys, dq, sw128_kmajor_desc(skl + okey), kIdescS, 1u);
+          tc_mma_bf16(tmem + st * kKeys, sw128_kmajor_desc(sql + oq), dk, kIdescS, 1u);
         }
         tc_commit(&bar[B_SFULL + st]);
         if (j == 0) stamp_at(a.trace, 11);
@@ -314,10 +350,10 @@ __global__ void __launch_bounds__(kThreads, 1) attn_tc_kernel(const __grid_const
   } else {
     // ------------------------------------------------------------ softmax rows
     // Two threads per query row: warps w and w + 4 read the same TMEM lanes,
-    // w < 4 the columns 0-63 of every block (keys, then output dims), w >= 4
-    // the columns 64-127; they exchange row maxima and sums through shared
-    // memory.  Every thread passes every named barrier, also after a failed
-    // wait (its work is then skipped), so no barrier is left short.
+    // w < 4 the first 32 keys of every block and output dims 0-63, w >= 4 the
+    // other 32 keys and dims 64-127; they exchange row maxima and sums through
+    // shared memory.  Every thread passes every named barrier, also after a
+    // failed wait (its work is then skipped), so no barrier is left short.
     pdl_wait();
     pdl_launch_dependents();
     const int hf = warp >> 2;
@@ -329,7 +365,8 @@ __global__ void __launch_bounds__(kThreads, 1) attn_tc_kernel(const __grid_const
     const uint64_t anc1 = sv.row_anc[2 * (base + node) + 1];
     const uint32_t tl = tmem + ((uint32_t)((warp & 3) * 32) << 16);  // this warp's TMEM lanes
     const float sl2 = 1.4426950408889634f * 0.08838834764831845f;      // log2(e) / sqrt(128)
-    uint8_t* prow = smem + Smem::p + hf * kHalf + r * 128;               // this thread's half of P's row
+    uint8_t* prow = smem + Smem::p + r * 128;                            // P's row (64 keys, 128 bytes)
+    uint8_t* plrow = smem + Smem::plo + r * 128;                         // P_lo's row
     float* xmax = reinterpret_cast<float*>(smem + Smem::xchg);           // [parity][half][row]
     float* xsum = xmax + 4 * 128;                                        // [half][row]
     float m = -INFINITY, l = 0.f;
@@ -337,33 +374,26 @@ __global__ void __launch_bounds__(kThreads, 1) attn_tc_kernel(const __grid_const
     for (int j = 0; j < nb; ++j) {
       const int st = j & 1;
       const int key0 = c0 + j * kKeys;
-      const uint32_t ts = tl + st * kKeys + hf * 64;
+      const uint32_t ts = tl + st * kKeys + hf * 32;  // this thread's 32 keys of S
       if (ok) ok = mbar_wait(&bar[B_SFULL + st], (j >> 1) & 1, err, abort_flag);
       ok = __all_sync(0xffffffffu, ok);
       if (j == 0) stamp(a.trace, 3);
-      // visibility word of each 32-key piece (all ones when the whole block is
-      // prefix keys of this chunk)
+      // visibility word of this thread's 32 keys (all ones when the whole block
+      // is prefix keys of this chunk)
       const bool full = row_ok && key0 + kKeys <= min(P, c1);
-      auto vis = [&](int i) {
-        const int piece = hf * 2 + i;
-        return full ? 0xffffffffu : (row_ok ? visible_word(key0 + 32 * piece, P, c1, anc0, anc1) : 0u);
-      };
+      const uint32_t w = full ? 0xffffffffu : (row_ok ? visible_word(key0 + 32 * hf, P, c1, anc0, anc1) : 0u);
       // pass 1: this half's row max (raw scores; the scale is positive), then both halves'
       float mx4[4] = {-INFINITY, -INFINITY, -INFINITY, -INFINITY};
       if (ok) {
         tc_fence_after();
-#pragma unroll 1
-        for (int i = 0; i < 2; ++i) {
-          uint32_t x[32];
-          tmem_ld32_async(ts + 32 * i, x);
-          tmem_wait_ld();
-          reg_fence32(x);
-          const uint32_t w = vis(i);
+        uint32_t x[32];
+        tmem_ld32_async(ts, x);
+        tmem_wait_ld();
+        reg_fence32(x);
 #pragma unroll
-          for (int c = 0; c < 32; ++c) {
-            const float v = ((w >> c) & 1u) ? __uint_as_float(x[c]) : -INFINITY;
-            mx4[c & 3] = fmaxf(mx4[c & 3], v);
-          }
+        for (int c = 0; c < 32; ++c) {
+          const float v = ((w >> c) & 1u) ? __uint_as_float(x[c]) : -INFINITY;
+          mx4[c & 3] = fmaxf(mx4[c & 3], v);
         }
       }
       xmax[(st * 2 + hf) * 128 + r] = fmaxf(fmaxf(mx4[0], mx4[1]), fmaxf(mx4[2], mx4[3]));
@@ -397,34 +427,34 @@ __global__ void __launch_bounds__(kThreads, 1) attn_tc_kernel(const __grid_const
           }
         }
       }
-      // pass 2: P = 2^(s - m) in fp16 into this half of the K-major,
-      // 128-byte-swizzled A operand (16-byte chunk c of a row lands at c ^ (row & 7))
+      // pass 2: P = 2^(s - m) in fp16 into this thread's half of the row of the
+      // K-major, 128-byte-swizzled A operand (16-byte chunk c of a row lands at c ^ (row & 7))
       float ls4[4] = {0.f, 0.f, 0.f, 0.f};
       if (ok) {
-#pragma unroll 1
-        for (int i = 0; i < 2; ++i) {
-          uint32_t x[32];
-          tmem_ld32_async(ts + 32 * i, x);
-          tmem_wait_ld();
-          reg_fence32(x);
-          const uint32_t w = vis(i);
-          uint32_t pk[16];
+        uint32_t x[32];
+        tmem_ld32_async(ts, x);
+        tmem_wait_ld();
+        reg_fence32(x);
+        uint32_t pk[16], pl[16];
 #pragma unroll
-          for (int c = 0; c < 16; ++c) {
-            const float s0 = ((w >> (2 * c)) & 1u) ? __uint_as_float(x[2 * c]) : -INFINITY;
-            const float s1 = ((w >> (2 * c + 1)) & 1u) ? __uint_as_float(x[2 * c + 1]) : -INFINITY;
-            const float p0 = fast_exp2(fmaf(s0, sl2, nm));
-            const float p1 = fast_exp2(fmaf(s1, sl2, nm));
-            ls4[c & 3] += p0 + p1;
-            const __half2 h2 = __floats2half2_rn(p0, p1);
-            pk[c] = *reinterpret_cast<const uint32_t*>(&h2);
-          }
+        for (int c = 0; c < 16; ++c) {
+          const float s0 = ((w >> (2 * c)) & 1u) ? __uint_as_float(x[2 * c]) : -INFINITY;
+          const float s1 = ((w >> (2 * c + 1)) & 1u) ? __uint_as_float(x[2 * c + 1]) : -INFINITY;
+          const float p0 = fast_exp2(fmaf(s0, sl2, nm));
+          const float p1 = fast_exp2(fmaf(s1, sl2, nm));
+          ls4[c & 3] += p0 + p1;
+          const __half2 h2 = __floats2half2_rn(p0, p1);
+          const float2 hf2 = __half22float2(h2);
+          const __half2 l2 = __floats2half2_rn(p0 - hf2.x, p1 - hf2.y);
+          pk[c] = *reinterpret_cast<const uint32_t*>(&h2);
+          pl[c] = *reinterpret_cast<const uint32_t*>(&l2);
+        }
 #pragma unroll
-          for (int q4 = 0; q4 < 4; ++q4) {
-            const int chunk = i * 4 + q4;
-            *reinterpret_cast<uint4*>(prow + ((chunk ^ (r & 7)) << 4)) =
-                make_uint4(pk[4 * q4], pk[4 * q4 + 1], pk[4 * q4 + 2], pk[4 * q4 + 3]);
-          }
+        for (int q4 = 0; q4 < 4; ++q4) {
+          const int chunk = hf * 4 + q4;
+          const int at = (chunk ^ (r & 7)) << 4;
+          *reinterpret_cast<uint4*>(prow + at) = make_uint4(pk[4 * q4], pk[4 * q4 + 1], pk[4 * q4 + 2], pk[4 * q4 + 3]);
+          *reinterpret_cast<uint4*>(plrow + at) = make_uint4(pl[4 * q4], pl[4 * q4 + 1], pl[4 * q4 + 2], pl[4 * q4 + 3]);
         }
         if (j == 0) stamp(a.trace, 9);
         tc_fence_before();

@@ -506,13 +506,19 @@ __global__ void __launch_bounds__(kThreads, BN == 64 ? 2 : 1)
                   x2[i] = o2;
                 }
               }
+              // q and K are stored as two fp16 parts (hi, then lo = the rounding
+              // error of hi): the attention scores use both; V keeps one part
               __half* dst = nullptr;
+              __half* dst_lo = nullptr;
               if (is_q) {
                 dst = args.q_out + ((size_t)(hh / G) * args.q_rows + (size_t)t * G + hh % G) * 128;
+                dst_lo = dst + (size_t)args.Hkv * args.q_rows * 128;
               } else if (slot >= 0) {
                 const int kvh = rot ? hh - args.Hq : hh - args.Hq - args.Hkv;
-                dst = (rot ? args.k_cache : args.v_cache) + (size_t)sid * args.kv_seq_stride +
-                      (size_t)kvh * args.kv_head_stride + (size_t)slot * 128;
+                const size_t off = (size_t)sid * args.kv_seq_stride + (size_t)kvh * args.kv_head_stride +
+                                   (size_t)slot * 128;
+                dst = (rot ? args.k_cache : args.v_cache) + off;
+                if (rot) dst_lo = args.klo_cache + off;
               } else if (c4 == 0) {
                 set_error(err, SPEC_DEVERR_BOUNDS);
               }
@@ -536,6 +542,21 @@ __global__ void __launch_bounds__(kThreads, BN == 64 ? 2 : 1)
                 hi.y = *reinterpret_cast<const uint32_t*>(&h3);
                 *reinterpret_cast<uint2*>(dst + 4 * c4) = lo;
                 *reinterpret_cast<uint2*>(dst + 64 + 4 * c4) = hi;
+                if (dst_lo) {
+                  const float2 f0 = __half22float2(h0), f1 = __half22float2(h1);
+                  const float2 f2 = __half22float2(h2), f3 = __half22float2(h3);
+                  const __half2 e0 = __floats2half2_rn(x1[0] - f0.x, x1[1] - f0.y);
+                  const __half2 e1 = __floats2half2_rn(x1[2] - f1.x, x1[3] - f1.y);
+                  const __half2 e2 = __floats2half2_rn(x2[0] - f2.x, x2[1] - f2.y);
+                  const __half2 e3 = __floats2half2_rn(x2[2] - f3.x, x2[3] - f3.y);
+                  uint2 el, eh;
+                  el.x = *reinterpret_cast<const uint32_t*>(&e0);
+                  el.y = *reinterpret_cast<const uint32_t*>(&e1);
+                  eh.x = *reinterpret_cast<const uint32_t*>(&e2);
+                  eh.y = *reinterpret_cast<const uint32_t*>(&e3);
+                  *reinterpret_cast<uint2*>(dst_lo + 4 * c4) = el;
+                  *reinterpret_cast<uint2*>(dst_lo + 64 + 4 * c4) = eh;
+                }
               }
             }
           } else {

@@ -61,9 +61,11 @@ struct GemmTcArgs {
   const int32_t* P_step;
   const int32_t* seq_ids;
   const float2* rope_cs;  // [tokens][64]
-  __half* q_out;          // [Hkv][q_rows][128]: row t*G + g holds head kvh*G + g of token t
+  __half* q_out;          // [2][Hkv][q_rows][128]: part 0 = fp16(q), part 1 = fp16(q - part 0);
+                          // row t*G + g holds head kvh*G + g of token t
   int q_rows;             // rows per kv head in q_out (>= tokens * G)
   __half* k_cache;        // this layer's K base: [max_batch][Hkv][max_seq][128]
+  __half* klo_cache;      // this layer's K_lo plane (fp16(k - fp16(k))), same layout
   __half* v_cache;
   size_t kv_seq_stride, kv_head_stride;
   int Hq, Hkv, max_seq;
@@ -143,13 +145,14 @@ struct StepView {
 };
 
 struct KvView {
-  void* base;               // [layer][2][max_batch][Hkv][max_seq][hd]
+  void* base;               // [layer][plane][max_batch][Hkv][max_seq][hd]
   int max_batch, Hkv, max_seq, hd;
-  size_t elem;              // 2 (bf16) or 4 (fp32)
+  size_t elem;              // 2 (bf16 models: fp16 planes) or 4 (fp32)
+  int planes;               // K, V (fp32 models); K, V, K_lo (bf16 models: K = K + K_lo to ~22 bits)
   __host__ __device__ size_t head_stride() const { return (size_t)max_seq * hd; }
   __host__ __device__ size_t seq_stride() const { return (size_t)Hkv * max_seq * hd; }
   __host__ __device__ size_t kv_stride() const { return (size_t)max_batch * seq_stride(); }
-  __host__ __device__ size_t layer_stride() const { return 2 * kv_stride(); }
+  __host__ __device__ size_t layer_stride() const { return (size_t)planes * kv_stride(); }
 };
 
 enum { STEP_VERIFY = 0, STEP_PREFILL = 1, STEP_SCORE = 2, STEP_DRAFT = 3, STEP_DRAFT_KV = 4 };
@@ -252,7 +255,7 @@ struct AttnTcMaps {
   CUtensorMap q, kv;
 };
 constexpr int kAttnTcRows = 128;   // query rows per CTA
-constexpr int kAttnTcKeys = 128;   // keys per block; chunks are multiples of it
+constexpr int kAttnTcKeys = 64;    // keys per block; chunks are multiples of it
 constexpr int kAttnPartCtas = 256; // partial slots: chunked launches stay within this many CTAs
 constexpr int kAttnMaxChunks = 16; // key chunks per (sequence, kv head, row tile) at most
 cudaError_t launch_attention_tc(const AttnArgs& a, const AttnTcMaps& maps, cudaStream_t s, bool pdl);

@@ -107,7 +107,7 @@ WsLayout make_layout(const spec_config& c) {
   // bf16 models keep GEMM activations as split bf16 (hi and lo rows): 2 x Mpad rows of 2 bytes
   const size_t arows = c.dtype == SPEC_DTYPE_BF16 ? 2 * (size_t)L.Mpad : (size_t)L.Mpad;
   L.xn = take(es * arows * c.hidden);
-  L.q = take(es * (size_t)L.Mpad * qd);
+  L.q = take(es * (size_t)L.Mpad * qd * (c.dtype == SPEC_DTYPE_BF16 ? 2 : 1));  // bf16 models: hi and lo parts
   L.attn = take(es * arows * qd);
   L.hmlp = take(es * arows * c.ffn);
   size_t pcols = (size_t)std::max(nqkv, c.hidden) * (c.dtype == SPEC_DTYPE_BF16 ? L.splits_cap : 1);
@@ -171,9 +171,12 @@ WsLayout make_layout(const spec_config& c) {
 // decoder layers with a K/V cache: the target's, plus the draft head's one layer
 int cache_layers(const spec_config& c) { return c.n_layers + (c.draft_head ? 1 : 0); }
 
+// planes per cache layer: K and V; bf16 models add K_lo = fp16(k - fp16(k)) for the attention scores
+int cache_planes(const spec_config& c) { return c.dtype == SPEC_DTYPE_BF16 ? 3 : 2; }
+
 size_t kv_bytes_of(const spec_config& c) {
   const size_t es = c.dtype == SPEC_DTYPE_BF16 ? 2 : 4;
-  return (size_t)cache_layers(c) * 2 * c.max_batch * c.n_kv_heads * (size_t)c.max_seq * c.head_dim * es;
+  return (size_t)cache_layers(c) * cache_planes(c) * c.max_batch * c.n_kv_heads * (size_t)c.max_seq * c.head_dim * es;
 }
 
 std::string check_config(const spec_config* c) {
@@ -556,6 +559,7 @@ struct PhaseBuilder {
     g.args.q_rows = L.Mpad * (c.n_q_heads / c.n_kv_heads);
     g.args.k_cache = kc;
     g.args.v_cache = kc + h->kv.kv_stride();
+    g.args.klo_cache = kc + 2 * h->kv.kv_stride();
     g.args.kv_seq_stride = h->kv.seq_stride();
     g.args.kv_head_stride = h->kv.head_stride();
     g.args.Hq = c.n_q_heads;
@@ -1228,6 +1232,7 @@ int spec_init(const spec_config* cfg, const spec_weights* w, void* kv_cache, siz
   h->kv.max_seq = c.max_seq;
   h->kv.hd = c.head_dim;
   h->kv.elem = c.dtype == SPEC_DTYPE_BF16 ? 2 : 4;
+  h->kv.planes = cache_planes(c);
   h->len.assign(c.max_batch, 0);
   h->pending.assign(c.max_batch, -1);
   h->len_hi.assign(c.max_batch, 0);
@@ -1279,18 +1284,18 @@ int spec_init(const spec_config* cfg, const spec_weights* w, void* kv_cache, siz
     if (attention_tc_configure(h->attn_clusters) != cudaSuccess) return bail(SPEC_ERR_CUDA, "smem attribute");
     const int qd = c.n_q_heads * c.head_dim, kvd = c.n_kv_heads * c.head_dim;
     {
-      // q as [Hkv * q_rows][128] and the cache as [layers * 2 * batch * Hkv * max_seq][128], fp16;
-      // TMA row coordinates are 32-bit
-      const uint64_t cache_rows = (uint64_t)cache_layers(c) * 2 * c.max_batch * c.n_kv_heads * c.max_seq;
+      // q as [2 * Hkv * q_rows][128] (hi part, then lo part) and the cache as
+      // [layers * planes * batch * Hkv * max_seq][128], fp16; TMA row coordinates are 32-bit
+      const uint64_t cache_rows = (uint64_t)cache_layers(c) * cache_planes(c) * c.max_batch * c.n_kv_heads * c.max_seq;
       if (cache_rows + 128 >= (1ull << 31)) return bail(SPEC_ERR_CAPACITY, "cache too large for 32-bit rows");
       const uint64_t q_rows = (uint64_t)c.n_kv_heads * lay.Mpad * (c.n_q_heads / c.n_kv_heads);
-      if (!make_tmap(&h->attn_maps.q, h->ws + lay.q, q_rows, 128, 128, CU_TENSOR_MAP_DATA_TYPE_FLOAT16) ||
-          !make_tmap(&h->attn_maps.kv, kv_cache, cache_rows, 128, 128, CU_TENSOR_MAP_DATA_TYPE_FLOAT16))
+      if (!make_tmap(&h->attn_maps.q, h->ws + lay.q, 2 * q_rows, 128, 128, CU_TENSOR_MAP_DATA_TYPE_FLOAT16) ||
+          !make_tmap(&h->attn_maps.kv, kv_cache, cache_rows, 128, kAttnTcKeys, CU_TENSOR_MAP_DATA_TYPE_FLOAT16))
         return bail(SPEC_ERR_CUDA, "tensor map");
-      // attention reads whole 128-key blocks (P = 0 beyond a sequence's keys): every
+      // attention reads whole key blocks (P = 0 beyond a sequence's keys): every
       // slot must hold a finite value from the start, and q rows too
       if (cudaMemsetAsync(kv_cache, 0, kv_bytes_of(c), h->stream) != cudaSuccess ||
-          cudaMemsetAsync(h->ws + lay.q, 0, 2 * (size_t)lay.Mpad * qd, h->stream) != cudaSuccess ||
+          cudaMemsetAsync(h->ws + lay.q, 0, 2 * 2 * (size_t)lay.Mpad * qd, h->stream) != cudaSuccess ||
           cudaStreamSynchronize(h->stream) != cudaSuccess)
         return bail(SPEC_ERR_CUDA, "cache init");
     }

@@ -337,8 +337,10 @@ class SpecEngine:
         return int(ln[0])
 
     def kv_view(self) -> torch.Tensor:
-        """The cache as a tensor [layer][2][max_batch][Hkv][max_seq][hd] (fp16 for bf16 models, else fp32)."""
+        """The cache as a tensor [layer][plane][max_batch][Hkv][max_seq][hd]: planes K, V (fp32 models) or
+        K, V, K_lo in fp16 (bf16 models; the key is K + K_lo)."""
         d = self.dims
         tdt = torch.float16 if d.dtype == "bf16" else torch.float32
+        planes = 3 if d.dtype == "bf16" else 2
         layers = d.n_layers + (1 if self._draft is not None else 0)  # the draft head's layer comes last
-        return self.kv.view(tdt).view(layers, 2, self.max_batch, d.n_kv_heads, -1, d.head_dim)
+        return self.kv.view(tdt).view(layers, planes, self.max_batch, d.n_kv_heads, -1, d.head_dim)

@@ -140,7 +140,12 @@ def decided_case(om, P, shape, p, stream0, plant_tries=3, prefix_tries=40, seed=
 
 
 def decided_tree_on(om, seq, shape, p, stream, tries=12):
-    """As decided_case, for a fixed prefix state (the sweep's drafts share one prefix)."""
+    """As decided_case, for a fixed prefix state (the sweep's drafts share one prefix).  None when the
+    root itself is a near-tie (no planting can help) or no planting stream is decided."""
+    lg_root, _ = oracle_tree_logits(om, seq, [seq.pending], [-1])
+    if float(top2_margin(lg_root)[0]) <= DECISIVE:
+        log("  root near-tie: margin %.4f" % float(top2_margin(lg_root)[0]))
+        return None
     for kt in range(tries):
         st = stream + STREAM_STEP * kt
         t0 = time.time()

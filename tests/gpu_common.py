@@ -111,8 +111,9 @@ def kv_close(gpu, ref, tol):
 
 
 def gpu_kv(eng, seq, length):
-    """Cached K and V of one sequence as float64 arrays [layer][pos][Hkv][hd]."""
+    """Cached K and V of one sequence as float64 arrays [layer][pos][Hkv][hd] (bf16 models: K = K + K_lo)."""
     kv = eng.kv_view()[:, :, seq, :, :length, :].to(torch.float64).cpu().numpy()
-    k = np.transpose(kv[:, 0], (0, 2, 1, 3))
+    kk = kv[:, 0] + kv[:, 2] if kv.shape[1] == 3 else kv[:, 0]
+    k = np.transpose(kk, (0, 2, 1, 3))
     v = np.transpose(kv[:, 1], (0, 2, 1, 3))
     return k, v

@@ -40,8 +40,11 @@ def cfg_of(d, max_batch=1, max_seq=512, max_nodes=64):
 def test_kv_bytes_matches_layout():
     d = synth.LLAMA8B
     c = cfg_of(d, max_batch=1, max_seq=4096, max_nodes=64)
-    # [layer][K|V][seq][kv head][slot][hd] bf16
-    assert S.spec_kv_bytes(ctypes.byref(c)) == 32 * 2 * 1 * 8 * 4096 * 128 * 2
+    # [layer][K|V|K_lo][seq][kv head][slot][hd] fp16
+    assert S.spec_kv_bytes(ctypes.byref(c)) == 32 * 3 * 1 * 8 * 4096 * 128 * 2
+    cf = cfg_of(synth.TINY, max_batch=2, max_seq=512, max_nodes=16)
+    # fp32 models: [layer][K|V][seq][kv head][slot][hd] fp32
+    assert S.spec_kv_bytes(ctypes.byref(cf)) == 2 * 2 * 2 * 4 * 512 * 64 * 4
     ws = S.spec_workspace_bytes(ctypes.byref(c))
     assert 0 < ws < 512 << 20
 

@@ -86,6 +86,7 @@ def _check_scored(g, rec, pre, amax, t1, t2, cols):
     gc = g[:, torch.as_tensor(cols.astype(np.int64), device="cuda")].double().cpu().numpy()
     err = max(float(np.max(np.abs(gt - rec[pre + "topk_val"]))),
               float(np.max(np.abs(gc - rec[pre + "logit_cols"].astype(np.float64)))))
+    print("%s max |logit error| vs the oracle: %.4g" % (pre or "step", err))
     assert err <= TOL["bf16"], "%s: max |logit error| %.4g" % (pre, err)
     np.testing.assert_allclose(t1, rec[pre + "topk_val"][:, 0], atol=TOL["bf16"])
     np.testing.assert_allclose(t2, rec[pre + "topk_val"][:, 1], atol=TOL["bf16"])
@@ -236,6 +237,7 @@ def test_fullsize_draft_head_batch16(target):
         gt = torch.gather(g, 1, torch.as_tensor(oi.astype(np.int64), device="cuda")).double().cpu().numpy()
         gc = g[:, torch.as_tensor(rec["cols"].astype(np.int64), device="cuda")].double().cpu().numpy()
         err = max(float(np.max(np.abs(gt - ov))), float(np.max(np.abs(gc - rec["logit_cols"]))))
+        print("draft step max |logit error| vs the oracle: %.4g" % err)
         assert err <= TOL["bf16"], "draft logits: max error %.4g" % err
         thr = min(DECISIVE, max(2.5 * err, 1e-6))
         K = gi.shape[1]
