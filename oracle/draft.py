@@ -12,6 +12,15 @@ table; the decoder layer is a pre-norm Llama layer of the target's shape with
 its own prefix K/V; a final RMSNorm precedes the LM head; the tree nodes
 attend to the draft prefix and to their ancestors, as in verification.
 
+Reduced draft vocabulary (VocabTrim / FR-Spec / SpecVocab in the aitangshan.cn
+walkthrough, sections 1 and 3.2: the draft model's output covers a trimmed
+vocabulary, which shrinks its search space and LM head): with `vocab_ids` the
+draft head's LM head is the target's rows at those token ids (ascending), the
+draft distribution is the softmax over that subset, and every drafted token is
+one of them.  Verification is unchanged, so the output is still the target's.
+Which tokens to keep is a property of a training corpus the pages do not give;
+the subset is an input here.
+
 Parity unpinned by the pages beyond these definitions: the pages give no
 numbers for the draft head.
 """
@@ -50,18 +59,32 @@ def top_k_rows(logits: np.ndarray, k: int):
 
 
 class OracleDraftHead:
-    def __init__(self, dims, target_weights: dict, draft_weights: dict):
+    def __init__(self, dims, target_weights: dict, draft_weights: dict, vocab_ids=None):
+        """vocab_ids: ascending token ids of a reduced draft vocabulary (None: the whole vocabulary)."""
         self.d = dims
+        lm = target_weights["lm_head"]
+        self.vocab_ids = None
+        if vocab_ids is not None:
+            ids = np.asarray(vocab_ids, dtype=np.int64)
+            if ids.ndim != 1 or ids.size < 2 or np.any(np.diff(ids) <= 0) or ids[0] < 0 or ids[-1] >= lm.shape[0]:
+                raise ValueError("vocab_ids must be strictly increasing token ids")
+            self.vocab_ids = ids
+            lm = lm[ids]  # the target's LM-head rows of the kept tokens
         # a one-layer model that reuses the generic decoder layer; its embed / lm_head
         # entries are the target's (the draft head has no table of its own)
         self.layer_model = OracleModel(dims, {
             "embed": target_weights["embed"],
-            "lm_head": target_weights["lm_head"],
+            "lm_head": lm,
             "final_norm": draft_weights["final_norm"],
             "layers": [draft_weights["layer"]],
         })
         self.fc_fuse = draft_weights["fc_fuse"]
         self.fc_in = draft_weights["fc_in"]
+
+    def token_of(self, idx):
+        """Token ids of draft-vocabulary indices (identity without a reduced vocabulary)."""
+        idx = np.asarray(idx, dtype=np.int64)
+        return idx if self.vocab_ids is None else self.vocab_ids[idx]
 
     def fuse(self, feats: np.ndarray) -> np.ndarray:
         """feats [n][3][k] (storage format) -> fused feature g [n][k]."""
@@ -105,9 +128,10 @@ class OracleDraftHead:
         return self.layer_model.lm_logits(a), a
 
     def step_topk(self, seq: DraftSeq, feats, tokens, parents, k: int = 10):
+        """Top-k per node as token ids; logits over the draft vocabulary."""
         logits = self.step_logits(seq, feats, tokens, parents)
         idx, val = top_k_rows(logits, k)
-        return idx, val, logits
+        return self.token_of(idx), val, logits
 
 
 # ---------------------------------------------------------------------------
@@ -139,7 +163,7 @@ def greedy_draft_chain(head: OracleDraftHead, seq: DraftSeq, g_root: np.ndarray,
         vis = np.tril(np.ones((T, T), bool))
         a, _, _ = head.layer_model.layer_forward(0, x, P + np.arange(T), seq.k, seq.v, vis)
         logits = head.layer_model.lm_logits(a[-1:])
-        t = int(np.argmax(logits[0]))
+        t = int(head.token_of(np.argmax(logits[0])))
         out.append(t)
         toks.append(t)
         gs.append(a[-1])
@@ -193,7 +217,7 @@ def build_draft_tree(head: OracleDraftHead, seq: DraftSeq, g_root: np.ndarray, r
         for f in frontier:
             idx, _ = top_k_rows(logits[f:f + 1], topk)
             for t in idx[0]:
-                offers.append((val[f] + lp[f, t], dep[f] + 1, order, f, int(t)))
+                offers.append((val[f] + lp[f, t], dep[f] + 1, order, f, int(head.token_of(t))))
                 order += 1
         offered.extend(offers)
         frontier = []

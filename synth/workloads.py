@@ -349,3 +349,13 @@ def weights_fingerprint(w: dict, row_stride: int = 509) -> str:
         for k in LAYER_KEYS:
             add("layer." + k, w["layer"][k])
     return h.hexdigest()[:16]
+
+
+def draft_vocab_ids(vocab: int, n: int, seed: int = 8) -> np.ndarray:
+    """A reduced draft vocabulary: n distinct token ids, ascending, drawn uniformly (seed 8).
+
+    Reduced draft vocabularies (VocabTrim, FR-Spec, SpecVocab) keep the tokens a
+    corpus uses most; no corpus is available here, so a seeded uniform subset
+    stands in for the frequency-ranked one."""
+    rng = np.random.default_rng([seed, vocab, n])
+    return np.sort(rng.choice(vocab, size=n, replace=False)).astype(np.int32)
