@@ -648,6 +648,15 @@ def run_sweep(args):
     return 0
 
 
+def reduce_draft_vocab(dw, w, vocab, n):
+    """Give the draft head a reduced vocabulary of n seeded token ids (the target's LM-head rows of them)."""
+    import torch
+    if n:
+        dw["vocab_ids"] = torch.as_tensor(synth.draft_vocab_ids(vocab, n), device="cuda")
+        dw["lm_head"] = w["lm_head"][dw["vocab_ids"].long()].contiguous()
+    return dw
+
+
 def run_draft(args):
     """Draft-head step: batch 16, 60-draft trees, draft prefixes of 2048 rows, N(0,1) features."""
     import torch
@@ -655,7 +664,7 @@ def run_draft(args):
     dims = synth.LLAMA8B
     B, P = 16, 2048
     w = synth.model_weights(dims, seed=0, device="cuda")
-    dw = synth.draft_head_weights(dims, seed=6, device="cuda")
+    dw = reduce_draft_vocab(synth.draft_head_weights(dims, seed=6, device="cuda"), w, dims.vocab, args.draft_vocab)
     eng = SpecEngine(dims, w, max_batch=B, max_seq=P + 64, max_nodes=64, draft=dw)
     rng = np.random.default_rng(5)
     for b in range(B):
@@ -686,14 +695,16 @@ def run_draft(args):
     prof = {k: round(v[0], 3) for k, v in eng.profile_read().items() if v[1]}
     eng.profile(False)
     d = dims
+    Vd = args.draft_vocab or d.vocab
     layer = d.q_dim * d.hidden + 2 * d.kv_dim * d.hidden + d.hidden * d.q_dim + 3 * d.ffn * d.hidden
-    params = 3 * d.hidden * d.hidden + 2 * d.hidden * d.hidden + layer + d.vocab * d.hidden
+    params = 3 * d.hidden * d.hidden + 2 * d.hidden * d.hidden + layer + Vd * d.hidden
     kv_tok = 2 * d.kv_dim * 2
     bytes_ = 2 * params + B * (P + 61) * kv_tok + M * 3 * d.hidden * 2
     fl = 2 * params * M + attn_flops(d, P * M, 1)
     print(json.dumps({"workload": "EAGLE-3 draft head at 8B shape bf16: batch 16, 60-draft trees, draft prefix 2048,"
                                   " N(0,1) low/mid/high features, fusion FC + input FC + one tree-masked decoder layer"
-                                  " + LM head + top-10", "tokens_per_step": M, "ms_per_step": ms,
+                                  " + LM head + top-10" + (" over a reduced draft vocabulary of %d tokens" % Vd
+                                                           if args.draft_vocab else ""), "tokens_per_step": M, "ms_per_step": ms,
                       "draft_steps_per_s": 1000.0 / ms, "roofline": _roofline(bytes_, fl, ms),
                       "kernel_ms_per_step": prof, "plan": eng.info(B, 61, P), "clocks": clocks,
                       "data": "synthetic"}))
@@ -708,7 +719,7 @@ def run_draft_tree(args):
     dims = synth.LLAMA8B
     B, P, steps, K, total = 16, 2048, 8, 10, 60
     w = synth.model_weights(dims, seed=0, device="cuda")
-    dw = synth.draft_head_weights(dims, seed=6, device="cuda")
+    dw = reduce_draft_vocab(synth.draft_head_weights(dims, seed=6, device="cuda"), w, dims.vocab, args.draft_vocab)
     eng = SpecEngine(dims, w, max_batch=B, max_seq=P + 128, max_nodes=128, draft=dw)
     rng = np.random.default_rng(5)
     for b in range(B):
@@ -731,7 +742,7 @@ def run_draft_tree(args):
     eng.profile(False)
     d = dims
     layer = d.q_dim * d.hidden + 2 * d.kv_dim * d.hidden + d.hidden * d.q_dim + 3 * d.ffn * d.hidden
-    per_step = 2 * d.hidden * d.hidden + layer + d.vocab * d.hidden  # input FC, decoder layer, LM head
+    per_step = 2 * d.hidden * d.hidden + layer + (args.draft_vocab or d.vocab) * d.hidden  # input FC, layer, LM head
     hbm, tflops, kind = measured_peaks()
     roof = 0.0
     fl_all = 0.0
@@ -742,7 +753,9 @@ def run_draft_tree(args):
         roof += max(by / hbm / 1e6, fl / tflops / 1e9)
         fl_all += fl
     print(json.dumps({"workload": "EAGLE-3 dynamic draft tree at 8B shape bf16: batch 16, draft prefix 2048, "
-                                  "8 drafting steps, top-10 offers, 60 nodes (every step recomputes the tree so far)",
+                                  "8 drafting steps, top-10 offers, 60 nodes (every step recomputes the tree so far)"
+                                  + (", reduced draft vocabulary of %d tokens" % args.draft_vocab
+                                     if args.draft_vocab else ""),
                       "ms_per_tree_batch": ms, "trees_per_s": B * 1000.0 / ms,
                       "roofline": {"bound": "per step: max(hbm, tensor)", "roofline_ms": roof, "frac": roof / ms,
                                    "flops": fl_all, "hbm_gbs": hbm, "bf16_tflops": tflops, "peak_source": kind},
@@ -827,6 +840,8 @@ def main():
     ap.add_argument("--sample-layers", type=int, default=2)
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--batch", type=int, default=1, help="sequences decoded together (--workload decode)")
+    ap.add_argument("--draft-vocab", type=int, default=0,
+                    help="draft / draft_tree workloads: a reduced draft vocabulary of this many seeded token ids")
     ap.add_argument("--temperature", type=float, default=0.0,
                     help="verify workload: sample at this temperature instead of greedy choices (0: greedy)")
     ap.add_argument("--layers", type=int, default=32, help="decoder layers (32 = the 8B shape; fewer only for profiling)")

@@ -92,6 +92,11 @@ typedef struct spec_config {
                            states of every position): the residual stream after this many decoder
                            layers, each in [1, n_layers]; {0, 0, 0}: no feature tap.  The pages name
                            no layers; 2, n_layers / 2 and n_layers - 3 is one choice. */
+  int32_t draft_vocab;  /* reduced draft vocabulary (VocabTrim / FR-Spec / SpecVocab in the aitangshan.cn
+                           walkthrough, sections 1 and 3.2): 0 = the draft head scores the whole vocabulary;
+                           2 .. vocab = its LM head is spec_weights.draft_lm_head, the target's rows of the
+                           token ids draft_vocab_ids, its softmax and its drafts cover only those tokens
+                           (verification is unchanged).  Needs draft_head. */
 } spec_config;
 
 /* Per-layer weights, device pointers, row-major [out][in] in the model dtype:
@@ -123,6 +128,9 @@ typedef struct spec_weights {
   const void* draft_fc_in;
   const spec_layer_weights* draft_layer;
   const void* draft_final_norm;
+  const void* draft_lm_head;        /* cfg.draft_vocab > 0: [draft_vocab][d], device, 16-byte aligned */
+  const int32_t* draft_vocab_ids;   /* cfg.draft_vocab > 0: [draft_vocab] token ids, device, strictly
+                                       increasing in [0, vocab) (checked by spec_init: SPEC_ERR_ARG) */
 } spec_weights;
 
 typedef struct spec_handle spec_handle;

@@ -170,16 +170,17 @@ __global__ void __launch_bounds__(kThreads, 1) attn_tc_kernel(const __grid_const
   const int Hkv = a.kv.Hkv;
   const int G = a.Hq / Hkv;
   const int bk = blockIdx.z;
-  const int b = bk / Hkv;
-  const int kvh = bk - b * Hkv;
+  const int bi = bk / Hkv;  // position in the work order (longest sequences first)
+  const int kvh = bk - bi * Hkv;
   const int tid = threadIdx.x;
   const int warp = tid >> 5;
   const int lane = tid & 31;
-  if (b >= sv.B) {
+  if (bi >= sv.B) {
     pdl_wait();
     pdl_launch_dependents();
     return;
   }
+  const int b = sv.order ? sv.order[bi] : bi;
   const int base = sv.node_off[b];
   const int n_b = sv.node_off[b + 1] - base;
   const int rows = n_b * G;
@@ -382,11 +383,12 @@ __global__ void __launch_bounds__(kThreads, 1) attn_tc_kernel(const __grid_const
       // is prefix keys of this chunk)
       const bool full = row_ok && key0 + kKeys <= min(P, c1);
       const uint32_t w = full ? 0xffffffffu : (row_ok ? visible_word(key0 + 32 * hf, P, c1, anc0, anc1) : 0u);
-      // pass 1: this half's row max (raw scores; the scale is positive), then both halves'
+      // pass 1: this half's row max (raw scores; the scale is positive), then both
+      // halves'; the 32 scores stay in registers for pass 2
       float mx4[4] = {-INFINITY, -INFINITY, -INFINITY, -INFINITY};
+      uint32_t x[32];
       if (ok) {
         tc_fence_after();
-        uint32_t x[32];
         tmem_ld32_async(ts, x);
         tmem_wait_ld();
         reg_fence32(x);
@@ -431,10 +433,6 @@ __global__ void __launch_bounds__(kThreads, 1) attn_tc_kernel(const __grid_const
       // K-major, 128-byte-swizzled A operand (16-byte chunk c of a row lands at c ^ (row & 7))
       float ls4[4] = {0.f, 0.f, 0.f, 0.f};
       if (ok) {
-        uint32_t x[32];
-        tmem_ld32_async(ts, x);
-        tmem_wait_ld();
-        reg_fence32(x);
         uint32_t pk[16], pl[16];
 #pragma unroll
         for (int c = 0; c < 16; ++c) {

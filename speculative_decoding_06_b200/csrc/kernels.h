@@ -127,6 +127,7 @@ struct StepView {
   const int32_t* parents;   // [M]
   const int32_t* node_off;  // [B+1]
   const int32_t* seq_ids;   // [B]
+  const int32_t* order;     // [B] batch entries by decreasing key count (attention's work order)
   int B, M;
   int32_t* row_seq;         // [M] batch entry
   int32_t* row_local;       // [M] local node index
@@ -173,8 +174,9 @@ cudaError_t launch_split_rows(const __nv_bfloat16* src, int rows, int cols, __nv
 constexpr int kTopKMax = 16;
 // top-k per row (value desc, index asc), k in {4, 8, 10, 16}; with lse != NULL also
 // the row's log-sum-exp (natural log)
+// (id_map: token id of each of the V columns; the indices written are id_map[column])
 cudaError_t launch_topk_rows(int M, int V, const float* logits, size_t ld, int k, int32_t* idx, float* val,
-                             float* lse, cudaStream_t s, bool pdl);
+                             float* lse, cudaStream_t s, bool pdl, const int32_t* id_map = nullptr);
 
 // a launch configuration with programmatic dependent launch when pdl (attr: 1 slot)
 cudaLaunchConfig_t make_cfg(dim3 grid, dim3 block, size_t smem, cudaStream_t s, bool pdl, cudaLaunchAttribute* attr);

@@ -538,7 +538,8 @@ __device__ __forceinline__ void warp_merge_topk(const float (&lv)[K], const int 
 template <int K, bool LSE, int U>
 __global__ void __launch_bounds__(256) topk_rows_kernel(int V, const float* __restrict__ logits, size_t ld,
                                                        int32_t* __restrict__ out_i, float* __restrict__ out_v,
-                                                       float* __restrict__ out_lse) {
+                                                       float* __restrict__ out_lse,
+                                                       const int32_t* __restrict__ id_map) {
   __shared__ float wv[8][K];
   __shared__ int wi[8][K];
   pdl_wait();
@@ -696,13 +697,13 @@ __global__ void __launch_bounds__(256) topk_rows_kernel(int V, const float* __re
     __syncwarp();
     if (lane < K) {
       out_v[(size_t)r * K + lane] = wv[0][lane];
-      out_i[(size_t)r * K + lane] = wi[0][lane];
+      out_i[(size_t)r * K + lane] = id_map ? id_map[wi[0][lane]] : wi[0][lane];
     }
   }
 }
 
 cudaError_t launch_topk_rows(int M, int V, const float* logits, size_t ld, int k, int32_t* idx, float* val,
-                             float* lse, cudaStream_t s, bool pdl) {
+                             float* lse, cudaStream_t s, bool pdl, const int32_t* id_map) {
   if (k < 1 || k > kTopKMax || k > V) return cudaErrorInvalidValue;
   cudaLaunchAttribute attr[1];
   cudaLaunchConfig_t cfg = make_cfg(dim3(M), dim3(256), 0, s, pdl, attr);
@@ -711,28 +712,28 @@ cudaError_t launch_topk_rows(int M, int V, const float* logits, size_t ld, int k
   switch (k) {  // the list length is a compile-time constant of the kernel
     case 10:
       if (few)
-        return lse ? cudaLaunchKernelEx(&cfg, topk_rows_kernel<10, true, 4>, V, logits, ld, idx, val, lse)
-                   : cudaLaunchKernelEx(&cfg, topk_rows_kernel<10, false, 4>, V, logits, ld, idx, val, lse);
-      return lse ? cudaLaunchKernelEx(&cfg, topk_rows_kernel<10, true, 2>, V, logits, ld, idx, val, lse)
-                 : cudaLaunchKernelEx(&cfg, topk_rows_kernel<10, false, 2>, V, logits, ld, idx, val, lse);
+        return lse ? cudaLaunchKernelEx(&cfg, topk_rows_kernel<10, true, 4>, V, logits, ld, idx, val, lse, id_map)
+                   : cudaLaunchKernelEx(&cfg, topk_rows_kernel<10, false, 4>, V, logits, ld, idx, val, lse, id_map);
+      return lse ? cudaLaunchKernelEx(&cfg, topk_rows_kernel<10, true, 2>, V, logits, ld, idx, val, lse, id_map)
+                 : cudaLaunchKernelEx(&cfg, topk_rows_kernel<10, false, 2>, V, logits, ld, idx, val, lse, id_map);
     case 16:
       if (few)
-        return lse ? cudaLaunchKernelEx(&cfg, topk_rows_kernel<16, true, 4>, V, logits, ld, idx, val, lse)
-                   : cudaLaunchKernelEx(&cfg, topk_rows_kernel<16, false, 4>, V, logits, ld, idx, val, lse);
-      return lse ? cudaLaunchKernelEx(&cfg, topk_rows_kernel<16, true, 2>, V, logits, ld, idx, val, lse)
-                 : cudaLaunchKernelEx(&cfg, topk_rows_kernel<16, false, 2>, V, logits, ld, idx, val, lse);
+        return lse ? cudaLaunchKernelEx(&cfg, topk_rows_kernel<16, true, 4>, V, logits, ld, idx, val, lse, id_map)
+                   : cudaLaunchKernelEx(&cfg, topk_rows_kernel<16, false, 4>, V, logits, ld, idx, val, lse, id_map);
+      return lse ? cudaLaunchKernelEx(&cfg, topk_rows_kernel<16, true, 2>, V, logits, ld, idx, val, lse, id_map)
+                 : cudaLaunchKernelEx(&cfg, topk_rows_kernel<16, false, 2>, V, logits, ld, idx, val, lse, id_map);
     case 8:
       if (few)
-        return lse ? cudaLaunchKernelEx(&cfg, topk_rows_kernel<8, true, 4>, V, logits, ld, idx, val, lse)
-                   : cudaLaunchKernelEx(&cfg, topk_rows_kernel<8, false, 4>, V, logits, ld, idx, val, lse);
-      return lse ? cudaLaunchKernelEx(&cfg, topk_rows_kernel<8, true, 2>, V, logits, ld, idx, val, lse)
-                 : cudaLaunchKernelEx(&cfg, topk_rows_kernel<8, false, 2>, V, logits, ld, idx, val, lse);
+        return lse ? cudaLaunchKernelEx(&cfg, topk_rows_kernel<8, true, 4>, V, logits, ld, idx, val, lse, id_map)
+                   : cudaLaunchKernelEx(&cfg, topk_rows_kernel<8, false, 4>, V, logits, ld, idx, val, lse, id_map);
+      return lse ? cudaLaunchKernelEx(&cfg, topk_rows_kernel<8, true, 2>, V, logits, ld, idx, val, lse, id_map)
+                 : cudaLaunchKernelEx(&cfg, topk_rows_kernel<8, false, 2>, V, logits, ld, idx, val, lse, id_map);
     case 4:
       if (few)
-        return lse ? cudaLaunchKernelEx(&cfg, topk_rows_kernel<4, true, 4>, V, logits, ld, idx, val, lse)
-                   : cudaLaunchKernelEx(&cfg, topk_rows_kernel<4, false, 4>, V, logits, ld, idx, val, lse);
-      return lse ? cudaLaunchKernelEx(&cfg, topk_rows_kernel<4, true, 2>, V, logits, ld, idx, val, lse)
-                 : cudaLaunchKernelEx(&cfg, topk_rows_kernel<4, false, 2>, V, logits, ld, idx, val, lse);
+        return lse ? cudaLaunchKernelEx(&cfg, topk_rows_kernel<4, true, 4>, V, logits, ld, idx, val, lse, id_map)
+                   : cudaLaunchKernelEx(&cfg, topk_rows_kernel<4, false, 4>, V, logits, ld, idx, val, lse, id_map);
+      return lse ? cudaLaunchKernelEx(&cfg, topk_rows_kernel<4, true, 2>, V, logits, ld, idx, val, lse, id_map)
+                 : cudaLaunchKernelEx(&cfg, topk_rows_kernel<4, false, 2>, V, logits, ld, idx, val, lse, id_map);
     default: return cudaErrorInvalidValue;
   }
 }

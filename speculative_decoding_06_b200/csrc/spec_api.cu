@@ -46,7 +46,7 @@ struct WsLayout {
   size_t total = 0;
   int Mmax = 0, Mpad = 0, splits_cap = 1, chunks_cap = 1;
   // parameter block (one host->device copy per step)
-  size_t p_tokens, p_parents, p_node_off, p_seq_ids, p_dlen, p_err, p_end;
+  size_t p_tokens, p_parents, p_node_off, p_seq_ids, p_dlen, p_order, p_err, p_end;
   // per-row metadata
   size_t row_seq, row_local, row_slot, row_sid, row_pos, row_anc, rope_cs, P_step;
   // persistent state
@@ -88,6 +88,7 @@ WsLayout make_layout(const spec_config& c) {
   L.p_node_off = take(4 * (size_t)(c.max_batch + 1));
   L.p_seq_ids = take(4 * (size_t)c.max_batch);
   L.p_dlen = take(4 * (size_t)c.max_batch);
+  L.p_order = take(4 * (size_t)c.max_batch);
   L.p_err = take(16);
   L.p_end = off;
   L.row_seq = take(4 * (size_t)L.Mmax);
@@ -199,6 +200,9 @@ std::string check_config(const spec_config* c) {
     if (c->hidden % 4) return "fp32 models need hidden % 4 == 0";
   }
   if (c->draft_head && c->dtype != SPEC_DTYPE_BF16) return "the draft head is bf16 only";
+  if (c->draft_vocab < 0 || c->draft_vocab == 1 || c->draft_vocab > c->vocab)
+    return "draft_vocab must be 0 or in [2, vocab]";
+  if (c->draft_vocab && !c->draft_head) return "draft_vocab needs the draft head";
   const int* fl = c->feature_layers;
   if (fl[0] || fl[1] || fl[2]) {
     for (int f = 0; f < 3; ++f)
@@ -277,6 +281,9 @@ struct spec_handle {
   const void* draft_fc_fuse = nullptr;
   const void* draft_fc_in = nullptr;
   const void* draft_final_norm = nullptr;
+  const void* draft_lm_head = nullptr;     // reduced draft vocabulary: [draft_vocab][d]
+  const int32_t* draft_ids = nullptr;      // its token ids (device)
+  CUtensorMap map_lm_draft;
   CUtensorMap map_fc_fuse, map_fc_in, map_fsplit[3], map_ge[3];
   std::vector<int32_t> dlen;        // draft-head prefix length per sequence
   std::vector<uint8_t> dready;
@@ -447,6 +454,7 @@ StepView make_view(spec_handle* h, int B, int M) {
   v.parents = h->W<int32_t>(L.p_parents);
   v.node_off = h->W<int32_t>(L.p_node_off);
   v.seq_ids = h->W<int32_t>(L.p_seq_ids);
+  v.order = h->W<int32_t>(L.p_order);
   v.B = B;
   v.M = M;
   v.row_seq = h->W<int32_t>(L.row_seq);
@@ -604,11 +612,13 @@ struct PhaseBuilder {
   }
   // final norm (folded) + LM head with per-tile top-2; logits also stored when given;
   // with `sample`, the top-2 is of the temperature-scaled logits plus the Gumbel noise
-  GemmPhase lm(float* logits, bool sample) const {
+  GemmPhase lm(float* logits, bool sample) const { return lm_rows(logits, sample, sp.lm, &h->map_lm, h->cfg.vocab); }
+  // the same over a given set of LM-head rows (the reduced draft vocabulary)
+  GemmPhase lm_rows(float* logits, bool sample, const GemmPlan& plan, const CUtensorMap* map, int rows) const {
     const spec_config& c = h->cfg;
     const WsLayout& L = h->lay;
-    GemmTcLaunch g = gemm_launch(sp.lm, GEMM_EPI_ARGMAX, c.vocab, d, M, &h->map_lm, nullptr, nullptr, &h->map_xn[bi],
-                                 c.vocab, 0, 0, sv.err);
+    GemmTcLaunch g = gemm_launch(plan, GEMM_EPI_ARGMAX, rows, d, M, map, nullptr, nullptr, &h->map_xn[bi], rows, 0, 0,
+                                 sv.err);
     g.args.top_part = h->W<Top2>(L.top_part);
     g.args.top_ld = L.Mpad;
     g.args.dbg_logits = logits;
@@ -886,18 +896,38 @@ cudaError_t enqueue_draft(spec_handle* h, const StepPlan& sp, bool kv_only, bool
   m.ph[0] = pb.o(Ld, 8 + 0);
   m.ph[1] = pb.gu(Ld);
   m.ph[2] = pb.down(Ld, 8 + 2, h->draft_final_norm);
-  m.ph[3] = pb.lm(logits, false);  // the draft head's own top-k reads the logits
+  // the draft head's own top-k reads the logits (over the reduced vocabulary when there is one)
+  const int Vd = c.draft_vocab ? c.draft_vocab : c.vocab;
+  if (c.draft_vocab) {
+    const GemmPlan pl = plan_gemm(h, 128, Vd, d, M, GEMM_EPI_ARGMAX);
+    m.ph[3] = pb.lm_rows(logits, false, pl, &h->map_lm_draft, Vd);
+  } else {
+    m.ph[3] = pb.lm(logits, false);
+  }
   LK(SPEC_PROF_GEMM_LAYER, 1, gemm_multi_launch(m, st, pdl));
   if (ts)
     LK(SPEC_PROF_TOPK, 1,
-       launch_topk_rows(M, c.vocab, logits, c.vocab, ts->K, h->W<int32_t>(L.tr_top_i), h->W<float>(L.tr_top_v),
-                        h->W<float>(L.tr_lse), st, pdl));
+       launch_topk_rows(M, Vd, logits, Vd, ts->K, h->W<int32_t>(L.tr_top_i), h->W<float>(L.tr_top_v),
+                        h->W<float>(L.tr_lse), st, pdl, h->draft_ids));
   else
     LK(SPEC_PROF_TOPK, 1,
-       launch_topk_rows(M, c.vocab, logits, c.vocab, kDraftTopK, h->W<int32_t>(L.dtop_i), h->W<float>(L.dtop_v),
-                        nullptr, st, pdl));
-  if (dbg) CUDA_RET(cudaMemcpyAsync(h->dbg_logits, logits, 4 * (size_t)M * c.vocab, cudaMemcpyDeviceToDevice, st));
+       launch_topk_rows(M, Vd, logits, Vd, kDraftTopK, h->W<int32_t>(L.dtop_i), h->W<float>(L.dtop_v),
+                        nullptr, st, pdl, h->draft_ids));
+  if (dbg) CUDA_RET(cudaMemcpyAsync(h->dbg_logits, logits, 4 * (size_t)M * Vd, cudaMemcpyDeviceToDevice, st));
   return cudaSuccess;
+}
+
+// Batch entries by decreasing key count (cached length + tree nodes): attention
+// takes its (sequence, kv head) work in this order, so that the longest
+// sequences start first and the shortest fill the tail.  Only the speed depends
+// on it; an approximate length (while device-output steps are in flight) is fine.
+void key_order(const spec_handle* h, int B, const int32_t* seq_ids, const int32_t* node_off,
+               const std::vector<int32_t>& len, int32_t* out) {
+  (void)h;
+  std::vector<std::pair<int, int>> keys((size_t)B);
+  for (int b = 0; b < B; ++b) keys[b] = {-(len[seq_ids[b]] + node_off[b + 1] - node_off[b]), b};
+  std::stable_sort(keys.begin(), keys.end());
+  for (int b = 0; b < B; ++b) out[b] = keys[b].second;
 }
 
 // Validate a batch of trees on the host (before anything is queued).
@@ -964,6 +994,7 @@ int run_step(spec_handle* h, int B, const int32_t* seq_ids, const int32_t* token
   std::memcpy(pb + L.p_parents, parents, 4 * (size_t)M);
   std::memcpy(pb + L.p_node_off, node_off, 4 * (size_t)(B + 1));
   std::memcpy(pb + L.p_seq_ids, seq_ids, 4 * (size_t)B);
+  key_order(h, B, seq_ids, node_off, h->stale ? h->len_hi : h->len, reinterpret_cast<int32_t*>(pb + L.p_order));
   std::memset(pb + L.p_err, 0, 16);
   CUDA_TRY(h, cudaMemcpyAsync(h->ws, pb, L.p_end, cudaMemcpyHostToDevice, h->stream));
 
@@ -1074,6 +1105,7 @@ int run_draft(spec_handle* h, int B, const int32_t* seq_ids, const void* feats, 
   std::memcpy(pb + L.p_node_off, node_off, 4 * (size_t)(B + 1));
   std::memcpy(pb + L.p_seq_ids, seq_ids, 4 * (size_t)B);
   std::memcpy(pb + L.p_dlen, h->dlen.data(), 4 * (size_t)c.max_batch);
+  key_order(h, B, seq_ids, node_off, h->dlen, reinterpret_cast<int32_t*>(pb + L.p_order));
   std::memset(pb + L.p_err, 0, 16);
   CUDA_TRY(h, cudaMemcpyAsync(h->ws, pb, L.p_end, cudaMemcpyHostToDevice, h->stream));
   // the caller's features become the first GEMM's split operand (outside any graph:
@@ -1208,6 +1240,15 @@ int spec_init(const spec_config* cfg, const spec_weights* w, void* kv_cache, siz
   if (c.draft_head && (!w->draft_fc_fuse || !w->draft_fc_in || !w->draft_final_norm || !aligned16(w->draft_fc_fuse) ||
                        !aligned16(w->draft_fc_in) || !aligned16(w->draft_final_norm)))
     return SPEC_ERR_ARG;
+  if (c.draft_vocab) {
+    if (!w->draft_lm_head || !aligned16(w->draft_lm_head) || !w->draft_vocab_ids) return SPEC_ERR_ARG;
+    // the token ids must be strictly increasing in [0, vocab): the top-k's tie order follows them
+    std::vector<int32_t> ids((size_t)c.draft_vocab);
+    if (cudaMemcpy(ids.data(), w->draft_vocab_ids, 4 * ids.size(), cudaMemcpyDeviceToHost) != cudaSuccess)
+      return SPEC_ERR_CUDA;
+    for (size_t i = 0; i < ids.size(); ++i)
+      if (ids[i] < 0 || ids[i] >= c.vocab || (i && ids[i] <= ids[i - 1])) return SPEC_ERR_ARG;
+  }
 
   spec_handle* h = new spec_handle();
   h->cfg = c;
@@ -1222,6 +1263,10 @@ int spec_init(const spec_config* cfg, const spec_weights* w, void* kv_cache, siz
     h->draft_fc_fuse = w->draft_fc_fuse;
     h->draft_fc_in = w->draft_fc_in;
     h->draft_final_norm = w->draft_final_norm;
+    if (c.draft_vocab) {
+      h->draft_lm_head = w->draft_lm_head;
+      h->draft_ids = w->draft_vocab_ids;
+    }
   }
   h->dlen.assign(c.max_batch, 0);
   h->dready.assign(c.max_batch, 0);
@@ -1313,6 +1358,8 @@ int spec_init(const spec_config* cfg, const spec_weights* w, void* kv_cache, siz
     if (c.draft_head &&
         (!make_tmap(&h->map_fc_fuse, h->draft_fc_fuse, c.hidden, 3 * (uint64_t)c.hidden, 128) ||
          !make_tmap(&h->map_fc_in, h->draft_fc_in, c.hidden, 2 * (uint64_t)c.hidden, 128)))
+      return bail(SPEC_ERR_CUDA, "tensor map");
+    if (c.draft_vocab && !make_tmap(&h->map_lm_draft, h->draft_lm_head, c.draft_vocab, c.hidden, 128))
       return bail(SPEC_ERR_CUDA, "tensor map");
     const int* bns = kTileWidths;
     for (int i = 0; i < 3; ++i) {
@@ -1583,6 +1630,8 @@ int spec_draft_tree(spec_handle* h, int B, const int32_t* seq_ids, const void* r
     for (int b = 0; b <= B; ++b) no[b] = b;
     std::memcpy(pb + L.p_seq_ids, seq_ids, 4 * (size_t)B);
     std::memcpy(pb + L.p_dlen, h->dlen.data(), 4 * (size_t)c.max_batch);
+    // every tree has the same node count at every step: the draft prefixes decide the order
+    key_order(h, B, seq_ids, no, h->dlen, reinterpret_cast<int32_t*>(pb + L.p_order));
     std::memset(pb + L.p_err, 0, 16);
     CUDA_TRY(h, cudaMemcpyAsync(h->ws, pb, L.p_end, cudaMemcpyHostToDevice, st));
     CUDA_TRY(h, launch_split_rows(static_cast<const __nv_bfloat16*>(root_feats), B, 3 * c.hidden,

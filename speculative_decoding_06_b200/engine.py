@@ -46,14 +46,19 @@ class SpecEngine:
                  stream: Optional[torch.cuda.Stream] = None, draft: Optional[Dict] = None,
                  feature_layers: Optional[Sequence[int]] = None):
         """feature_layers: (low, mid, high) layer counts whose residual streams a
-        verification step can return for the draft head (see verify_batch)."""
+        verification step can return for the draft head (see verify_batch).
+        draft: the draft head's weights; with "vocab_ids" (int32 device tensor, ascending
+        token ids) and "lm_head" (bf16 [len(vocab_ids)][d]: the target's rows of those ids)
+        it scores a reduced vocabulary."""
         self.dims = dims
         self.cfg = S.spec_config(
             n_layers=dims.n_layers, hidden=dims.hidden, n_q_heads=dims.n_q_heads, n_kv_heads=dims.n_kv_heads,
             head_dim=dims.head_dim, ffn=dims.ffn, vocab=dims.vocab,
             dtype=S.SPEC_DTYPE_BF16 if dims.dtype == "bf16" else S.SPEC_DTYPE_F32,
             rms_eps=dims.rms_eps, rope_theta=dims.rope_theta, max_batch=max_batch, max_seq=max_seq,
-            max_nodes=max_nodes, draft_head=1 if draft is not None else 0)
+            max_nodes=max_nodes, draft_head=1 if draft is not None else 0,
+            draft_vocab=int(draft["vocab_ids"].numel()) if draft is not None and "vocab_ids" in draft else 0)
+        self.draft_vocab = self.cfg.draft_vocab or dims.vocab
         if feature_layers is not None:
             self.cfg.feature_layers[:] = [int(j) for j in feature_layers]
         self._feat = None
@@ -81,6 +86,9 @@ class SpecEngine:
             self._w.draft_fc_in = draft["fc_in"].data_ptr()
             self._w.draft_layer = ctypes.pointer(self._dlayer)
             self._w.draft_final_norm = draft["final_norm"].data_ptr()
+            if "vocab_ids" in draft:
+                self._w.draft_lm_head = draft["lm_head"].data_ptr()
+                self._w.draft_vocab_ids = draft["vocab_ids"].data_ptr()
         # a dedicated stream: the legacy default stream cannot be captured into graphs
         self.stream = stream or torch.cuda.Stream()
         torch.cuda.synchronize()  # weights and buffers were written on torch's stream
@@ -195,9 +203,12 @@ class SpecEngine:
         self._check(S.spec_set_debug_logits(self.h, self._dbg.data_ptr(), self._dbg.numel() * 4))
         return self._dbg
 
-    def debug_logits(self, rows: int) -> np.ndarray:
+    def debug_logits(self, rows: int, width: Optional[int] = None) -> np.ndarray:
+        """The SPEC_DEBUG_LOGITS rows [rows][width] (width: the vocabulary, or the draft vocabulary
+        after a draft step)."""
         torch.cuda.synchronize()
-        return self._dbg[: rows * self.dims.vocab].view(rows, self.dims.vocab).cpu().numpy()
+        w = width or self.dims.vocab
+        return self._dbg[: rows * w].view(rows, w).cpu().numpy()
 
     def truncate(self, seq: int, new_len: int):
         self._check(S.spec_truncate(self.h, seq, new_len))

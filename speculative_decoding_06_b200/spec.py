@@ -49,7 +49,7 @@ class spec_config(ctypes.Structure):
         ("vocab", ctypes.c_int32), ("dtype", ctypes.c_int32), ("rms_eps", ctypes.c_float),
         ("rope_theta", ctypes.c_float), ("max_batch", ctypes.c_int32), ("max_seq", ctypes.c_int32),
         ("max_nodes", ctypes.c_int32), ("draft_head", ctypes.c_int32),
-        ("feature_layers", ctypes.c_int32 * 3),
+        ("feature_layers", ctypes.c_int32 * 3), ("draft_vocab", ctypes.c_int32),
     ]
 
 
@@ -64,6 +64,7 @@ class spec_weights(ctypes.Structure):
         ("layers", ctypes.POINTER(spec_layer_weights)),
         ("draft_fc_fuse", ctypes.c_void_p), ("draft_fc_in", ctypes.c_void_p),
         ("draft_layer", ctypes.POINTER(spec_layer_weights)), ("draft_final_norm", ctypes.c_void_p),
+        ("draft_lm_head", ctypes.c_void_p), ("draft_vocab_ids", ctypes.c_void_p),
     ]
 
 

@@ -68,7 +68,7 @@ def test_feature_layers_checked_and_sized(layers, ok):
 
 @pytest.mark.parametrize("field,value", [
     ("n_kv_heads", 3), ("head_dim", 64), ("hidden", 4000), ("max_nodes", 129), ("max_nodes", 0), ("dtype", 7),
-    ("ffn", 100), ("rope_theta", 0.5),
+    ("ffn", 100), ("rope_theta", 0.5), ("draft_vocab", 1), ("draft_vocab", 100),
 ])
 def test_bad_bf16_config_rejected(field, value):
     c = cfg_of(synth.MINI_BF16)
