@@ -241,6 +241,19 @@ def make_sweep_p8192():
         log("prefill P=8192 stream %d: %.0f s, last margin %.4f" % (s, time.time() - t0, m))
         if m <= DECISIVE:
             continue
+        # the trees' deciding paths start along the greedy continuation: skip a prefix
+        # whose first greedy tokens hold a near-tie (no planting of a wide tree avoids it)
+        toks, par, near = [seq.pending], [-1], False
+        for depth in range(3):
+            lg, _ = oracle_tree_logits(om, seq, toks, par)
+            if float(top2_margin(lg[-1:])[0]) <= DECISIVE:
+                near = True
+                break
+            toks.append(int(np.argmax(lg[-1])))
+            par.append(len(toks) - 2)
+        if near:
+            log("  greedy continuation near-tie at depth %d" % depth)
+            continue
         P = len(prefix)
         cols = sampled_columns(dims.vocab, N_COLS, 8192)
         rec = {"fingerprint": np.array(fp), "P": np.int32(P), "prefix": prefix, "prefix_stream": np.int32(s),
