@@ -636,10 +636,17 @@ def run_sweep(args):
         a, _, _ = eng.verify(0, toks, sh.parents)
         reset()
         ms = _timed(eng.stream, lambda: eng.verify_batch_device(ids, tk, pr, off), args.steps, reset)
+        # per-kernel time of one step (launches serialised by the profiler's events)
+        eng.profile(True)
+        eng.verify_batch_device(ids, tk, pr, off)
+        reset()
+        prof = {k: round(v[0], 3) for k, v in eng.profile_read().items() if v[1]}
+        eng.profile(False)
         bytes_ = step_bytes(dims, P, sh.n)
         fl = flops_per_token(dims) * sh.n + attn_flops(dims, P * sh.n, dims.n_layers)
         out.append({"draft": name, "nodes": sh.n, "ms_per_step": ms, "tau": a + 1,
-                    "accepted_tokens_per_s": (a + 1) * 1000.0 / ms, "roofline_frac": _roofline(bytes_, fl, ms)["frac"]})
+                    "accepted_tokens_per_s": (a + 1) * 1000.0 / ms, "roofline_frac": _roofline(bytes_, fl, ms)["frac"],
+                    "kernel_ms_per_step": prof})
     clk.end()
     clocks = clk.stop()
     print(json.dumps({"workload": "llama3.1-8b-shape bf16, batch 1, prefix 8192, chains 5/8 and trees 16/32/60/80"

@@ -19,18 +19,20 @@
 // 32-layer model of the 8B shape; P's rounding made a node's logits depend on
 // where key chunks start.)
 //
-//   warp 8 (one thread): TMA loads of Q (hi, lo) and of 64-key blocks of K, K_lo
-//                        and V (two stages), the three S MMAs of a block into
-//                        one of two 64-column TMEM buffers, O += P_j V_j into a
+//   warp 16 (one thread): TMA loads of Q (hi, lo) and of 64-key blocks of K,
+//                        K_lo and V (two stages each; the later blocks of the
+//                        chunk are brought into L2 up front), the S MMAs of a
+//                        block into one of two TMEM buffers, O += P_j V_j into a
 //                        128-column buffer (V read MN-major);
-//   warps 0-7:           two threads per query row (warps w and w + 4 share the
-//                        row's TMEM lane; each takes 32 of the block's keys):
-//                        read S_j, apply the ancestor mask and the online
-//                        softmax (the running max moves only when a block's max
-//                        exceeds it by more than the slack, 8 in log2 units by
-//                        default: every p stays <= 2^8 and O is rescaled
-//                        rarely), write P_j (hi and lo) into shared memory as
-//                        the next MMAs' A operands, and at the end normalise O.
+//   warps 0-15:          four threads per query row (warps w, w + 4, w + 8 and
+//                        w + 12 share the row's TMEM lane; each takes 16 of the
+//                        block's keys and 32 output dims): read S_j, apply the
+//                        ancestor mask and the online softmax (the running max
+//                        moves only when a block's max exceeds it by more than
+//                        the slack, 8 in log2 units by default: every p stays
+//                        <= 2^8 and O is rescaled rarely), write P_j (hi and lo)
+//                        into shared memory as the next MMAs' A operands, and at
+//                        the end normalise O.
 //
 // A sequence's keys are cut into chunks so that short-prefix, small-batch steps
 // still occupy the GPU; the chunk CTAs of one (sequence, kv head, row tile)
@@ -51,28 +53,37 @@ namespace {
 
 constexpr int kRows = 128;                   // query rows per CTA (the MMA M)
 constexpr int kKeys = kAttnTcKeys;           // keys per block (S's N, P.V's K): 64
-constexpr int kThreads = 288;                // warps 0-7 rows (two per row), warp 8 issue
-constexpr int kCtrlWarp = 8;
+constexpr int kRowWarps = 16;                // softmax warps: four threads per query row
+constexpr int kPerRow = kRowWarps / 4;       // threads of a row (warps w, w + 4, w + 8, w + 12 share its TMEM lane)
+constexpr int kKeysPT = 64 / kPerRow;        // keys of a block per thread: 16
+constexpr int kDimsPT = 128 / kPerRow;       // output dims per thread: 32
+constexpr int kThreads = 32 * (kRowWarps + 2);  // + warp 16: MMA issue, warp 17: TMA loads
+constexpr int kCtrlWarp = kRowWarps;
+constexpr int kLoadWarp = kRowWarps + 1;
 constexpr uint32_t kQHalf = kRows * 128;     // [128 rows][64 fp16] swizzled: 16 KB
 constexpr uint32_t kQTile = 2 * kQHalf;      // 128 x 128 fp16: 32 KB
 constexpr uint32_t kKHalf = kKeys * 128;     // [64 keys][64 fp16] swizzled: 8 KB
 constexpr uint32_t kKTile = 2 * kKHalf;      // 64 x 128 fp16: 16 KB
+// a K stage holds, per 64-dim half, K's 64 rows then K_lo's 64 rows: one 128-row
+// operand [K; K_lo] per half, so Q_hi [K; K_lo]^T is one N = 128 product
+constexpr uint32_t kKStage = 2 * kKTile;     // 32 KB
 constexpr uint32_t kPTile = kRows * kKeys * 2;  // [128 rows][64 keys] fp16, one 128-byte row each: 16 KB
 static_assert(kKeys == 64, "a P row is one 128-byte swizzled row; two 32-key pieces per block");
 
-enum { B_QFULL = 0, B_KVFULL = 1, B_KVEMPTY = 3, B_SFULL = 5, B_SFREE = 7, B_PFULL = 9, B_PEMPTY = 10, B_OFULL = 11,
-       B_DRAIN = 12, kNumBars = 13 };
+// K and V stages are filled and released separately: a K stage is free once the
+// scores that read it are done, a V stage once P.V is
+enum { B_QFULL = 0, B_KFULL = 1, B_VFULL = 3, B_KEMPTY = 5, B_VEMPTY = 7, B_SFULL = 9, B_SFREE = 11, B_PFULL = 13,
+       B_PEMPTY = 14, B_OFULL = 15, B_DRAIN = 16, kNumBars = 17 };
 
 struct Smem {
   static constexpr uint32_t q = 0;                   // Q hi
   static constexpr uint32_t qlo = q + kQTile;        // Q lo
-  static constexpr uint32_t k = qlo + kQTile;        // 2 stages; with klo, 64 KB of output staging at the end
-  static constexpr uint32_t klo = k + 2 * kKTile;    // 2 stages
-  static constexpr uint32_t v = klo + 2 * kKTile;    // 2 stages
+  static constexpr uint32_t k = qlo + kQTile;        // 2 stages of [K; K_lo]; 64 KB of output staging at the end
+  static constexpr uint32_t v = k + 2 * kKStage;     // 2 stages
   static constexpr uint32_t p = v + 2 * kKTile;      // P hi
   static constexpr uint32_t plo = p + kPTile;        // P lo
-  static constexpr uint32_t xchg = plo + kPTile;     // row maxima [2][2][128] and sums [2][128]
-  static constexpr uint32_t lse = xchg + 6 * 128 * 4; // this chunk's log2-sum-exp per row (cluster merge)
+  static constexpr uint32_t xchg = plo + kPTile;     // row maxima [2][kPerRow][128] and sums [kPerRow][128]
+  static constexpr uint32_t lse = xchg + 3 * kPerRow * 128 * 4; // this chunk's log2-sum-exp per row (cluster merge)
   static constexpr uint32_t bars = lse + 128 * 4;
   static constexpr uint32_t misc = bars + kNumBars * 8;  // tmem slot, abort flag, merge flag
   static constexpr uint32_t end = misc + 16;
@@ -80,14 +91,17 @@ struct Smem {
 };
 static_assert(Smem::dyn <= 227 * 1024, "shared memory");
 
-// tensor-memory columns: S buffers at 0 and 64, O at 128
-constexpr uint32_t kTmemCols = 256;
-constexpr uint32_t kColO = 2 * kKeys;
+// tensor-memory columns: two S buffers of 128 (keys 0-63: Q_hi K^T + Q_lo K^T, 64-127:
+// Q_hi K_lo^T, added by the softmax) at 0 and 128, O at 256
+constexpr uint32_t kTmemCols = 512;
+constexpr uint32_t kSCols = 2 * kKeys;
+constexpr uint32_t kColO = 2 * kSCols;
 static_assert(kColO + 128 <= kTmemCols, "tensor memory");
-static_assert(Smem::xchg - Smem::k >= 128 * 512, "output staging (128 rows x 512 B) fits in the K / K_lo ring");
+static_assert(Smem::v - Smem::k >= 128 * 512, "output staging (128 rows x 512 B) fits in the K ring");
 
-// fp16 A and B, f32 D, M = 128; S: N = 64 keys; P.V: N = 128 dims, B MN-major (bit 16)
+// fp16 A and B, f32 D, M = 128; S: N = 128 ([K; K_lo]) and N = 64 (K); P.V: N = 128 dims, B MN-major (bit 16)
 constexpr uint32_t kIdescS = (1u << 4) | ((uint32_t)(kKeys >> 3) << 17) | ((uint32_t)(kRows >> 4) << 24);
+constexpr uint32_t kIdescS2 = (1u << 4) | ((uint32_t)(2 * kKeys >> 3) << 17) | ((uint32_t)(kRows >> 4) << 24);
 constexpr uint32_t kIdescPV = (1u << 4) | (1u << 16) | ((uint32_t)(128 >> 3) << 17) | ((uint32_t)(kRows >> 4) << 24);
 
 // MN-major operand with the 128-byte swizzle: 64 fp16 along N per 128-byte row,
@@ -112,13 +126,8 @@ __device__ __forceinline__ void stamp_at(uint64_t* trace, int k) {
   if (cta < (unsigned)kAttnPartCtas) trace[cta * kTraceMarks + k] = global_ns();
 }
 
-__device__ __forceinline__ void named_sync_rows() { asm volatile("bar.sync 1, 256;" ::: "memory"); }
+__device__ __forceinline__ void named_sync_rows() { asm volatile("bar.sync 1, %0;" ::"n"(32 * kRowWarps) : "memory"); }
 
-// keep uses of TMEM-loaded registers after the wait
-__device__ __forceinline__ void reg_fence32(uint32_t* r) {
-#pragma unroll
-  for (int i = 0; i < 32; ++i) asm volatile("" : "+r"(r[i]));
-}
 
 
 
@@ -213,12 +222,14 @@ __global__ void __launch_bounds__(kThreads, 1) attn_tc_kernel(const __grid_const
   if (tid == 0) {
     mbar_init(&bar[B_QFULL], 1);
     for (int s = 0; s < 2; ++s) {
-      mbar_init(&bar[B_KVFULL + s], 1);
-      mbar_init(&bar[B_KVEMPTY + s], 1);
+      mbar_init(&bar[B_KFULL + s], 1);
+      mbar_init(&bar[B_VFULL + s], 1);
+      mbar_init(&bar[B_KEMPTY + s], 1);
+      mbar_init(&bar[B_VEMPTY + s], 1);
       mbar_init(&bar[B_SFULL + s], 1);
-      mbar_init(&bar[B_SFREE + s], 8);
+      mbar_init(&bar[B_SFREE + s], kRowWarps);
     }
-    mbar_init(&bar[B_PFULL], 8);
+    mbar_init(&bar[B_PFULL], kRowWarps);
     mbar_init(&bar[B_PEMPTY], 1);
     mbar_init(&bar[B_OFULL], 1);
     mbar_init(&bar[B_DRAIN], 1);
@@ -230,8 +241,8 @@ __global__ void __launch_bounds__(kThreads, 1) attn_tc_kernel(const __grid_const
   tc_fence_after();
   const uint32_t tmem = *tmem_slot;
 
-  if (warp == kCtrlWarp) {
-    // ------------------------------------------------------------ TMA + MMA issue
+  if (warp == kLoadWarp) {
+    // ------------------------------------------------------------ TMA loads
     if (nb == 0) {
       pdl_wait();
       pdl_launch_dependents();
@@ -247,27 +258,49 @@ __global__ void __launch_bounds__(kThreads, 1) attn_tc_kernel(const __grid_const
       const int qlrow = qrow + Hkv * a.q_rows;  // the lo part follows all kv heads' hi parts
       const uint64_t pol_q = policy_evict_first();
       const uint64_t pol = policy_evict_normal();  // the other row tiles read the same K/V blocks
-      int loaded = 0;
-      auto load_kv = [&](int j) {
+      int kloaded = 0, vloaded = 0;  // blocks whose K (K_lo) / V copies were issued
+      auto load_k = [&](int j) {
         const int st = j & 1;
         const int key = c0 + j * kKeys;
-        uint8_t* sk = smem + Smem::k + st * kKTile;
-        uint8_t* skl = smem + Smem::klo + st * kKTile;
+        uint8_t* sk = smem + Smem::k + st * kKStage;
+        mbar_arrive_expect_tx(&bar[B_KFULL + st], 2 * kKTile);
+        tma_load_2d(sk, &maps.kv, &bar[B_KFULL + st], 0, krow + key, pol);
+        tma_load_2d(sk + kKHalf, &maps.kv, &bar[B_KFULL + st], 0, klrow + key, pol);
+        tma_load_2d(sk + kKTile, &maps.kv, &bar[B_KFULL + st], 64, krow + key, pol);
+        tma_load_2d(sk + kKTile + kKHalf, &maps.kv, &bar[B_KFULL + st], 64, klrow + key, pol);
+        kloaded = j + 1;
+      };
+      auto load_v = [&](int j) {
+        const int st = j & 1;
+        const int key = c0 + j * kKeys;
         uint8_t* svb = smem + Smem::v + st * kKTile;
-        mbar_arrive_expect_tx(&bar[B_KVFULL + st], 3 * kKTile);
-        tma_load_2d(sk, &maps.kv, &bar[B_KVFULL + st], 0, krow + key, pol);
-        tma_load_2d(sk + kKHalf, &maps.kv, &bar[B_KVFULL + st], 64, krow + key, pol);
-        tma_load_2d(skl, &maps.kv, &bar[B_KVFULL + st], 0, klrow + key, pol);
-        tma_load_2d(skl + kKHalf, &maps.kv, &bar[B_KVFULL + st], 64, klrow + key, pol);
-        tma_load_2d(svb, &maps.kv, &bar[B_KVFULL + st], 0, vrow + key, pol);
-        tma_load_2d(svb + kKHalf, &maps.kv, &bar[B_KVFULL + st], 64, vrow + key, pol);
-        loaded = j + 1;
+        mbar_arrive_expect_tx(&bar[B_VFULL + st], kKTile);
+        tma_load_2d(svb, &maps.kv, &bar[B_VFULL + st], 0, vrow + key, pol);
+        tma_load_2d(svb + kKHalf, &maps.kv, &bar[B_VFULL + st], 64, vrow + key, pol);
+        vloaded = j + 1;
+      };
+      // the blocks beyond the two stages go into L2 now, so that their copies into
+      // shared memory later wait on L2 rather than on HBM
+      auto prefetch_kv = [&](int j) {
+        const int key = c0 + j * kKeys;
+        tma_prefetch_l2_2d(&maps.kv, 0, krow + key);
+        tma_prefetch_l2_2d(&maps.kv, 64, krow + key);
+        tma_prefetch_l2_2d(&maps.kv, 0, klrow + key);
+        tma_prefetch_l2_2d(&maps.kv, 64, klrow + key);
+        tma_prefetch_l2_2d(&maps.kv, 0, vrow + key);
+        tma_prefetch_l2_2d(&maps.kv, 64, vrow + key);
       };
       // blocks made only of prefix keys were written by earlier steps: load
       // them before waiting for the previous kernel
       const int first = min(nb, 2);
       int pre = 0;
-      while (pre < first && c0 + (pre + 1) * kKeys <= P) load_kv(pre++);
+      while (pre < first && c0 + (pre + 1) * kKeys <= P) {
+        load_k(pre);
+        load_v(pre);
+        ++pre;
+      }
+      int pf = first;
+      while (pf < nb && c0 + (pf + 1) * kKeys <= P) prefetch_kv(pf++);
       pdl_wait();
       pdl_launch_dependents();
       mbar_arrive_expect_tx(&bar[B_QFULL], 2 * kQTile);
@@ -275,7 +308,43 @@ __global__ void __launch_bounds__(kThreads, 1) attn_tc_kernel(const __grid_const
       tma_load_2d(smem + Smem::q + kQHalf, &maps.q, &bar[B_QFULL], 64, qrow, pol_q);
       tma_load_2d(smem + Smem::qlo, &maps.q, &bar[B_QFULL], 0, qlrow, pol_q);
       tma_load_2d(smem + Smem::qlo + kQHalf, &maps.q, &bar[B_QFULL], 64, qlrow, pol_q);
-      for (int j = pre; j < first; ++j) load_kv(j);
+      for (int j = pre; j < first; ++j) {
+        load_k(j);
+        load_v(j);
+      }
+      while (pf < nb) prefetch_kv(pf++);
+      // block j >= 2 into the stages of block j - 2: K once its scores are done,
+      // V once its P.V is done (the MMA issuer commits both)
+      bool ok = true;
+      for (int j = 2; j < nb && ok; ++j) {
+        ok = mbar_wait(&bar[B_KEMPTY + (j & 1)], ((j - 2) >> 1) & 1, err, abort_flag);
+        if (ok) load_k(j);
+        if (ok) ok = mbar_wait(&bar[B_VEMPTY + (j & 1)], ((j - 2) >> 1) & 1, err, abort_flag);
+        if (ok) load_v(j);
+      }
+      if (!ok) {
+        *abort_flag = 1;
+        // let this thread's copies land before the CTA's shared memory is released:
+        // only the last copy into each stage can be outstanding (an earlier one was
+        // consumed before the stage was refilled)
+        for (int j = max(0, kloaded - 2); j < kloaded; ++j)
+          mbar_wait(&bar[B_KFULL + (j & 1)], (j >> 1) & 1, nullptr, nullptr);
+        for (int j = max(0, vloaded - 2); j < vloaded; ++j)
+          mbar_wait(&bar[B_VFULL + (j & 1)], (j >> 1) & 1, nullptr, nullptr);
+      }
+    } else {
+      pdl_wait();
+      pdl_launch_dependents();
+    }
+    __syncwarp();
+  } else if (warp == kCtrlWarp) {
+    // ------------------------------------------------------------ MMA issue
+    if (nb == 0) {
+      pdl_wait();
+      pdl_launch_dependents();
+    } else if (elect_one()) {
+      pdl_wait();
+      pdl_launch_dependents();
       const uint32_t sq = smem_u32(smem + Smem::q);
       const uint32_t sql = smem_u32(smem + Smem::qlo);
       const uint32_t sp = smem_u32(smem + Smem::p);
@@ -291,57 +360,49 @@ __global__ void __launch_bounds__(kThreads, 1) attn_tc_kernel(const __grid_const
           tc_mma_bf16(tmem + kColO, sw128_kmajor_desc(spl + kk * 32), bd, kIdescPV, 1u);
         }
       };
+      // P.V of block j (its P written, its V landed)
+      auto pv_step = [&](int j) -> bool {
+        if (!mbar_wait(&bar[B_PFULL], j & 1, err, abort_flag)) return false;
+        if (!mbar_wait(&bar[B_VFULL + (j & 1)], (j >> 1) & 1, err, abort_flag)) return false;
+        tc_fence_after();
+        issue_pv(j);
+        tc_commit(&bar[B_PEMPTY]);
+        tc_commit(&bar[B_VEMPTY + (j & 1)]);
+        return true;
+      };
       bool ok = mbar_wait(&bar[B_QFULL], 0, err, abort_flag);
       stamp_at(a.trace, 1);
-      int waited = 0;  // K/V blocks whose arrival this thread has seen
       for (int j = 0; j < nb && ok; ++j) {
         const int st = j & 1;
-        ok = mbar_wait(&bar[B_KVFULL + st], (j >> 1) & 1, err, abort_flag);
+        ok = mbar_wait(&bar[B_KFULL + st], (j >> 1) & 1, err, abort_flag);
         if (!ok) break;
-        waited = j + 1;
         if (j == 0) stamp_at(a.trace, 2);
         if (j >= 2) ok = mbar_wait(&bar[B_SFREE + st], ((j - 2) >> 1) & 1, err, abort_flag);
         if (!ok) break;
         tc_fence_after();
-        const uint32_t sk = smem_u32(smem + Smem::k + st * kKTile);
-        const uint32_t skl = smem_u32(smem + Smem::klo + st * kKTile);
+        const uint32_t sk = smem_u32(smem + Smem::k + st * kKStage);
 #pragma unroll
         for (int ks = 0; ks < 8; ++ks) {  // 16 head dims per step
           const uint32_t oq = (ks >> 2) * kQHalf + (ks & 3) * 32;
-          const uint32_t okey = (ks >> 2) * kKHalf + (ks & 3) * 32;
-          const uint64_t dq = sw128_kmajor_desc(sq + oq), dk = sw128_kmajor_desc(sk + okey);
-          tc_mma_bf16(tmem + st * kKeys, dq, dk, kIdescS, ks > 0 ? 1u : 0u);
-          tc_mma_bf16(tmem + st * kKeys, dq, sw128_kmajor_desc(skl + okey), kIdescS, 1u);
-          tc_mma_bf16(tmem + st * kKeys, sw128_kmajor_desc(sql + oq), dk, kIdescS, 1u);
+          const uint32_t okey = (ks >> 2) * kKTile + (ks & 3) * 32;  // [K; K_lo] rows of this dim half
+          const uint64_t dk2 = sw128_kmajor_desc(sk + okey);         // N = 128: K then K_lo
+          tc_mma_bf16(tmem + st * kSCols, sw128_kmajor_desc(sq + oq), dk2, kIdescS2, ks > 0 ? 1u : 0u);
+          tc_mma_bf16(tmem + st * kSCols, sw128_kmajor_desc(sql + oq), dk2, kIdescS, 1u);  // N = 64: K only
         }
         tc_commit(&bar[B_SFULL + st]);
+        tc_commit(&bar[B_KEMPTY + st]);
         if (j == 0) stamp_at(a.trace, 11);
-        if (j >= 1) {
-          ok = mbar_wait(&bar[B_PFULL], (j - 1) & 1, err, abort_flag);
-          if (!ok) break;
-          tc_fence_after();
-          issue_pv(j - 1);
-          tc_commit(&bar[B_PEMPTY]);
-          tc_commit(&bar[B_KVEMPTY + ((j - 1) & 1)]);
-          if (j + 1 < nb) {
-            ok = mbar_wait(&bar[B_KVEMPTY + ((j - 1) & 1)], ((j - 1) >> 1) & 1, err, abort_flag);
-            if (!ok) break;
-            load_kv(j + 1);
-          }
-        }
+        if (j >= 1) ok = pv_step(j - 1);
       }
-      if (ok) ok = mbar_wait(&bar[B_PFULL], (nb - 1) & 1, err, abort_flag);
       stamp_at(a.trace, 12);
+      if (ok && nb > 0) ok = pv_step(nb - 1);
       if (ok) {
-        tc_fence_after();
-        issue_pv(nb - 1);
         tc_commit(&bar[B_OFULL]);
       } else {
         *abort_flag = 1;
-        // let issued MMAs and copies finish before the CTA's memory is released
+        // let issued MMAs finish before the CTA's memory is released
         tc_commit(&bar[B_DRAIN]);
         mbar_wait(&bar[B_DRAIN], 0, nullptr, nullptr);
-        for (int j = waited; j < loaded; ++j) mbar_wait(&bar[B_KVFULL + (j & 1)], (j >> 1) & 1, nullptr, nullptr);
       }
     } else {
       pdl_wait();
@@ -350,14 +411,14 @@ __global__ void __launch_bounds__(kThreads, 1) attn_tc_kernel(const __grid_const
     __syncwarp();
   } else {
     // ------------------------------------------------------------ softmax rows
-    // Two threads per query row: warps w and w + 4 read the same TMEM lanes,
-    // w < 4 the first 32 keys of every block and output dims 0-63, w >= 4 the
-    // other 32 keys and dims 64-127; they exchange row maxima and sums through
-    // shared memory.  Every thread passes every named barrier, also after a
-    // failed wait (its work is then skipped), so no barrier is left short.
+    // Four threads per query row: warps w, w + 4, w + 8 and w + 12 read the same
+    // TMEM lanes; quarter q = warp / 4 takes keys 16q .. 16q + 15 of every block
+    // and output dims 32q .. 32q + 31, and the four exchange row maxima and sums
+    // through shared memory.  Every thread passes every named barrier, also after
+    // a failed wait (its work is then skipped), so no barrier is left short.
     pdl_wait();
     pdl_launch_dependents();
-    const int hf = warp >> 2;
+    const int qtr = warp >> 2;
     const int r = (warp & 3) * 32 + lane;
     const int qr = row0 + r;
     const bool row_ok = qr < rows;
@@ -368,39 +429,43 @@ __global__ void __launch_bounds__(kThreads, 1) attn_tc_kernel(const __grid_const
     const float sl2 = 1.4426950408889634f * 0.08838834764831845f;      // log2(e) / sqrt(128)
     uint8_t* prow = smem + Smem::p + r * 128;                            // P's row (64 keys, 128 bytes)
     uint8_t* plrow = smem + Smem::plo + r * 128;                         // P_lo's row
-    float* xmax = reinterpret_cast<float*>(smem + Smem::xchg);           // [parity][half][row]
-    float* xsum = xmax + 4 * 128;                                        // [half][row]
+    float* xmax = reinterpret_cast<float*>(smem + Smem::xchg);           // [parity][quarter][row]
+    float* xsum = xmax + 2 * kPerRow * 128;                              // [quarter][row]
+    const uint32_t kmask = (1u << kKeysPT) - 1u;
     float m = -INFINITY, l = 0.f;
     bool ok = true;
     for (int j = 0; j < nb; ++j) {
       const int st = j & 1;
       const int key0 = c0 + j * kKeys;
-      const uint32_t ts = tl + st * kKeys + hf * 32;  // this thread's 32 keys of S
+      const uint32_t ts = tl + st * kSCols + qtr * kKeysPT;  // this thread's keys of S (+ kKeys: the K_lo part)
       if (ok) ok = mbar_wait(&bar[B_SFULL + st], (j >> 1) & 1, err, abort_flag);
       ok = __all_sync(0xffffffffu, ok);
       if (j == 0) stamp(a.trace, 3);
-      // visibility word of this thread's 32 keys (all ones when the whole block
-      // is prefix keys of this chunk)
+      // visibility bits of this thread's keys (all ones when the whole block is
+      // prefix keys of this chunk)
       const bool full = row_ok && key0 + kKeys <= min(P, c1);
-      const uint32_t w = full ? 0xffffffffu : (row_ok ? visible_word(key0 + 32 * hf, P, c1, anc0, anc1) : 0u);
-      // pass 1: this half's row max (raw scores; the scale is positive), then both
-      // halves'; the 32 scores stay in registers for pass 2
+      const uint32_t w =
+          full ? kmask : (row_ok ? visible_word(key0 + kKeysPT * qtr, P, c1, anc0, anc1) & kmask : 0u);
+      // pass 1: this quarter's row max (raw scores; the scale is positive), then the
+      // row's; the scores stay in registers for pass 2
+      float x[kKeysPT];
       float mx4[4] = {-INFINITY, -INFINITY, -INFINITY, -INFINITY};
-      uint32_t x[32];
       if (ok) {
         tc_fence_after();
-        tmem_ld32_async(ts, x);
-        tmem_wait_ld();
-        reg_fence32(x);
+        float xl[kKeysPT];
+        tmem_ld16x2(ts, ts + kKeys, x, xl);
 #pragma unroll
-        for (int c = 0; c < 32; ++c) {
-          const float v = ((w >> c) & 1u) ? __uint_as_float(x[c]) : -INFINITY;
-          mx4[c & 3] = fmaxf(mx4[c & 3], v);
+        for (int c = 0; c < kKeysPT; ++c) {
+          x[c] += xl[c];
+          mx4[c & 3] = fmaxf(mx4[c & 3], ((w >> c) & 1u) ? x[c] : -INFINITY);
         }
       }
-      xmax[(st * 2 + hf) * 128 + r] = fmaxf(fmaxf(mx4[0], mx4[1]), fmaxf(mx4[2], mx4[3]));
+      xmax[(st * kPerRow + qtr) * 128 + r] = fmaxf(fmaxf(mx4[0], mx4[1]), fmaxf(mx4[2], mx4[3]));
       named_sync_rows();
-      const float mblk = fmaxf(xmax[(st * 2) * 128 + r], xmax[(st * 2 + 1) * 128 + r]) * sl2;
+      float mraw = xmax[(st * kPerRow) * 128 + r];
+#pragma unroll
+      for (int q = 1; q < kPerRow; ++q) mraw = fmaxf(mraw, xmax[(st * kPerRow + q) * 128 + r]);
+      const float mblk = mraw * sl2;
       if (j == 0) stamp(a.trace, 8);
       float corr = 1.f;
       if (mblk > m + a.rescale_slack) {
@@ -408,48 +473,46 @@ __global__ void __launch_bounds__(kThreads, 1) attn_tc_kernel(const __grid_const
         m = mblk;
       }
       const float nm = (m == -INFINITY) ? 0.f : -m;
+      // pass 2: P = 2^(s - m) as two fp16 parts, in registers until the P buffer is free
+      float ls4[4] = {0.f, 0.f, 0.f, 0.f};
+      uint32_t pk[kKeysPT / 2], pl[kKeysPT / 2];
+#pragma unroll
+      for (int c = 0; c < kKeysPT / 2; ++c) {
+        const float s0 = ((w >> (2 * c)) & 1u) ? x[2 * c] : -INFINITY;
+        const float s1 = ((w >> (2 * c + 1)) & 1u) ? x[2 * c + 1] : -INFINITY;
+        const float p0 = ok ? fast_exp2(fmaf(s0, sl2, nm)) : 0.f;
+        const float p1 = ok ? fast_exp2(fmaf(s1, sl2, nm)) : 0.f;
+        ls4[c & 3] += p0 + p1;
+        const __half2 h2 = __floats2half2_rn(p0, p1);
+        const float2 hf2 = __half22float2(h2);
+        const __half2 l2 = __floats2half2_rn(p0 - hf2.x, p1 - hf2.y);
+        pk[c] = *reinterpret_cast<const uint32_t*>(&h2);
+        pl[c] = *reinterpret_cast<const uint32_t*>(&l2);
+      }
       if (j >= 1 && ok) {
         // P.V of the previous block has finished: the P buffer is free and O is current
         ok = __all_sync(0xffffffffu, mbar_wait(&bar[B_PEMPTY], (j - 1) & 1, err, abort_flag));
         if (ok) {
           tc_fence_after();
           if (__any_sync(0xffffffffu, corr != 1.f)) {
-#pragma unroll 1
-            for (int i = 0; i < 2; ++i) {
-              uint32_t o[32];
-              const uint32_t to_ = tl + kColO + hf * 64 + 32 * i;
-              tmem_ld32_async(to_, o);
-              tmem_wait_ld();
-              reg_fence32(o);
+            uint32_t o[32];
+            const uint32_t to_ = tl + kColO + qtr * kDimsPT;
+            tmem_ld32_async(to_, o);
+            tmem_wait_ld();
+            tmem_reg_fence32(o);
 #pragma unroll
-              for (int c = 0; c < 32; ++c) o[c] = __float_as_uint(__uint_as_float(o[c]) * corr);
-              tmem_st32_async(to_, o);
-            }
+            for (int c = 0; c < 32; ++c) o[c] = __float_as_uint(__uint_as_float(o[c]) * corr);
+            tmem_st32_async(to_, o);
             tmem_wait_st();
           }
         }
       }
-      // pass 2: P = 2^(s - m) in fp16 into this thread's half of the row of the
-      // K-major, 128-byte-swizzled A operand (16-byte chunk c of a row lands at c ^ (row & 7))
-      float ls4[4] = {0.f, 0.f, 0.f, 0.f};
+      // this thread's 32 bytes of the row of the K-major, 128-byte-swizzled A
+      // operand (16-byte chunk c of a row lands at c ^ (row & 7))
       if (ok) {
-        uint32_t pk[16], pl[16];
 #pragma unroll
-        for (int c = 0; c < 16; ++c) {
-          const float s0 = ((w >> (2 * c)) & 1u) ? __uint_as_float(x[2 * c]) : -INFINITY;
-          const float s1 = ((w >> (2 * c + 1)) & 1u) ? __uint_as_float(x[2 * c + 1]) : -INFINITY;
-          const float p0 = fast_exp2(fmaf(s0, sl2, nm));
-          const float p1 = fast_exp2(fmaf(s1, sl2, nm));
-          ls4[c & 3] += p0 + p1;
-          const __half2 h2 = __floats2half2_rn(p0, p1);
-          const float2 hf2 = __half22float2(h2);
-          const __half2 l2 = __floats2half2_rn(p0 - hf2.x, p1 - hf2.y);
-          pk[c] = *reinterpret_cast<const uint32_t*>(&h2);
-          pl[c] = *reinterpret_cast<const uint32_t*>(&l2);
-        }
-#pragma unroll
-        for (int q4 = 0; q4 < 4; ++q4) {
-          const int chunk = hf * 4 + q4;
+        for (int q4 = 0; q4 < kKeysPT / 8; ++q4) {
+          const int chunk = qtr * (kKeysPT / 8) + q4;
           const int at = (chunk ^ (r & 7)) << 4;
           *reinterpret_cast<uint4*>(prow + at) = make_uint4(pk[4 * q4], pk[4 * q4 + 1], pk[4 * q4 + 2], pk[4 * q4 + 3]);
           *reinterpret_cast<uint4*>(plrow + at) = make_uint4(pl[4 * q4], pl[4 * q4 + 1], pl[4 * q4 + 2], pl[4 * q4 + 3]);
@@ -471,33 +534,32 @@ __global__ void __launch_bounds__(kThreads, 1) attn_tc_kernel(const __grid_const
     if (ok && nb > 0) ok = mbar_wait(&bar[B_OFULL], 0, err, abort_flag);  // (an idle CTA issued no MMA)
     ok = __all_sync(0xffffffffu, ok);
     stamp(a.trace, 4);
-    xsum[hf * 128 + r] = l;
+    xsum[qtr * 128 + r] = l;
     named_sync_rows();
-    const float lt = xsum[r] + xsum[128 + r];
+    float lt = 0.f;
+#pragma unroll
+    for (int q = 0; q < kPerRow; ++q) lt += xsum[q * 128 + r];
     const bool any = lt > 0.f;
     const float inv = any ? 1.f / lt : 0.f;
     uint8_t* stg = smem + Smem::k;  // 128 rows x 512 B
     if (ok && nb > 0) {
       tc_fence_after();
-#pragma unroll 1
-      for (int i = 0; i < 2; ++i) {
-        uint32_t o[32];
-        tmem_ld32_async(tl + kColO + hf * 64 + 32 * i, o);
-        tmem_wait_ld();
-        reg_fence32(o);
+      uint32_t o[32];
+      tmem_ld32_async(tl + kColO + qtr * kDimsPT, o);
+      tmem_wait_ld();
+      tmem_reg_fence32(o);
 #pragma unroll
-        for (int q4 = 0; q4 < 8; ++q4)
-          *stage_at(stg, r, (hf * 2 + i) * 8 + q4) =
-              make_float4(__uint_as_float(o[4 * q4]) * inv, __uint_as_float(o[4 * q4 + 1]) * inv,
-                          __uint_as_float(o[4 * q4 + 2]) * inv, __uint_as_float(o[4 * q4 + 3]) * inv);
-      }
+      for (int q4 = 0; q4 < 8; ++q4)
+        *stage_at(stg, r, qtr * 8 + q4) =
+            make_float4(__uint_as_float(o[4 * q4]) * inv, __uint_as_float(o[4 * q4 + 1]) * inv,
+                        __uint_as_float(o[4 * q4 + 2]) * inv, __uint_as_float(o[4 * q4 + 3]) * inv);
     }
     const int grp = (b * Hkv + kvh) * gridDim.y + blockIdx.y;
     const size_t slot = (size_t)grp * a.n_chunks + blockIdx.x;
     const float my_lse = (ok && any && nb > 0) ? m + __log2f(lt) : -INFINITY;
     if (a.cluster_merge) {
-      if (hf == 0) reinterpret_cast<float*>(smem + Smem::lse)[r] = my_lse;
-    } else if (nc_b > 1 && ok && hf == 0) {
+      if (qtr == 0) reinterpret_cast<float*>(smem + Smem::lse)[r] = my_lse;
+    } else if (nc_b > 1 && ok && qtr == 0) {
       a.part_lse[slot * kRows + r] = my_lse;
     }
     named_sync_rows();
@@ -507,7 +569,7 @@ __global__ void __launch_bounds__(kThreads, 1) attn_tc_kernel(const __grid_const
     if (nc_b == 1) {
       // one chunk: each warp writes whole rows, lane = 4 columns, as split bf16
       if (ok && nb > 0) {
-        for (int rr = warp; rr < valid; rr += 8) {
+        for (int rr = warp; rr < valid; rr += kRowWarps) {
           const float4 v = *stage_at(stg, rr, lane);
           const int q2 = row0 + rr;
           const int nd = q2 / G;
@@ -519,7 +581,7 @@ __global__ void __launch_bounds__(kThreads, 1) attn_tc_kernel(const __grid_const
       // partial rows, coalesced: lane = 4 columns of one row
       float4* po = reinterpret_cast<float4*>(a.part_o + slot * kRows * 128);
       if (ok)
-        for (int rr = warp; rr < valid; rr += 8) __stcg(po + rr * 32 + lane, *stage_at(stg, rr, lane));
+        for (int rr = warp; rr < valid; rr += kRowWarps) __stcg(po + rr * 32 + lane, *stage_at(stg, rr, lane));
       named_sync_rows();
       stamp(a.trace, 5);
       int* ctr = a.counters + 2 * grp;
@@ -541,10 +603,10 @@ __global__ void __launch_bounds__(kThreads, 1) attn_tc_kernel(const __grid_const
         const float* lse0 = a.part_lse + (size_t)grp * a.n_chunks * kRows + rb;
         const float4* po0 = reinterpret_cast<const float4*>(a.part_o + (size_t)grp * a.n_chunks * kRows * 128) +
                             (size_t)rb * 32 + lane;
-        // One slice row per warp and round (8 warps: 16 rows in two rounds);
+        // One slice row per warp and round;
         // every chunk's log-sum-exp and partial in flight at once
         // (chunks <= kAttnMaxChunks).
-        for (int rr = warp; rr < R; rr += 8) {
+        for (int rr = warp; rr < R; rr += kRowWarps) {
           float lv[kAttnMaxChunks];
           float4 pv[kAttnMaxChunks];
 #pragma unroll
@@ -589,7 +651,7 @@ __global__ void __launch_bounds__(kThreads, 1) attn_tc_kernel(const __grid_const
     // by reading its peers' (distributed shared memory), then the cluster
     // meets again so that no CTA leaves while a peer still reads it
     cluster_sync_all();
-    if (warp < 8 && nc_b > 1) {
+    if (warp < kRowWarps && nc_b > 1) {
       const int valid = min(kRows, rows - row0);
       const int per = (valid + nc_b - 1) / nc_b;
       const int rb = blockIdx.x * per;
@@ -598,7 +660,7 @@ __global__ void __launch_bounds__(kThreads, 1) attn_tc_kernel(const __grid_const
       const int ld = a.Hq * 128;
       const uint32_t lse_base = smem_u32(smem + Smem::lse);
       const uint32_t stg_base = smem_u32(smem + Smem::k);
-      for (int rr = warp; rr < R; rr += 8) {
+      for (int rr = warp; rr < R; rr += kRowWarps) {
         const int row = rb + rr;
         const uint32_t soff = (uint32_t)(reinterpret_cast<uint8_t*>(stage_at(smem + Smem::k, row, lane)) -
                                          (smem + Smem::k));

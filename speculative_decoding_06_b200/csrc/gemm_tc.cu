@@ -92,6 +92,59 @@ __device__ __forceinline__ UnitIter units_of(const GemmTcArgs& a) {
   return it;
 }
 
+// The work units of a phase that a CTA takes, in order: tile `ut` over k-blocks
+// [kb0, kb1).  Plain and split-K phases: UnitIter's tiles over this CTA's split
+// range.  Stream-K phases (GemmTcArgs::streamk): the phase's tiles x KB
+// k-blocks in tile-major order, cut into one contiguous share per CTA,
+// [W b / grid, W (b + 1) / grid) with W = tiles x KB, whose pieces (one per
+// tile it touches) are the units.  Every CTA then streams the same number of
+// weight k-blocks, whatever the tile count; the CTA holding a tile's first
+// k-block finishes the tile, the CTAs whose shares start inside the tile hand
+// it fp32 partial sums.
+struct WorkIter {
+  int KB, kb0s, kb1s, tiles, grid, S, ut;
+  long long g, w1;  // stream-K cursor and end
+  bool sk;
+  __device__ bool next(int& t, int& k0, int& k1) {
+    if (sk) {
+      if (g >= w1) return false;
+      t = (int)(g / KB);
+      k0 = (int)(g - (long long)t * KB);
+      k1 = (int)min((long long)KB, k0 + (w1 - g));
+      g += k1 - k0;
+      return true;
+    }
+    if (ut >= tiles) return false;
+    t = ut;
+    k0 = kb0s;
+    k1 = kb1s;
+    ut = S > 1 ? tiles : ut + grid;
+    return true;
+  }
+};
+
+__device__ __forceinline__ WorkIter work_of(const GemmTcArgs& a) {
+  const UnitIter it = units_of(a);
+  WorkIter w;
+  w.KB = a.K / kTileK;
+  w.tiles = it.tiles;
+  w.grid = it.grid;
+  w.S = it.S;
+  w.ut = it.first();
+  w.kb0s = it.split() * a.kb_per_split;
+  w.kb1s = min(w.kb0s + a.kb_per_split, w.KB);
+  w.sk = a.streamk != 0;
+  const long long W = (long long)w.tiles * w.KB;
+  w.g = W * it.b / it.grid;
+  w.w1 = W * (it.b + 1) / it.grid;
+  return w;
+}
+
+// stream-K: the CTA whose share holds k-block index g of the phase (W in all, over grid CTAs)
+__device__ __forceinline__ int sk_cta_of(long long W, long long g, int grid) {
+  return (int)(((g + 1) * grid - 1) / W);
+}
+
 // Optional timeline: stamp k of phase p of this CTA.  Stamps: 0 producer
 // starts the phase, 1 producer may load the phase's activations, 2 producer
 // has issued the phase's last load, 3 epilogue starts the phase, 4 first
@@ -182,13 +235,10 @@ __global__ void __launch_bounds__(kThreads, BN == 64 ? 2 : 1)
   if (producer) {
     pol_w = policy_evict_first();
     pol_x = policy_evict_last();
-    const UnitIter it = units_of(P.ph[0]);
-    const int ut = it.first();
-    if (ut < it.tiles) {
+    WorkIter wi = work_of(P.ph[0]);
+    int ut, kb0, kb1;
+    if (wi.next(ut, kb0, kb1)) {
       const GemmTcArgs& a = P.ph[0];
-      const int KB = a.K / kTileK;
-      const int kb0 = it.split() * a.kb_per_split;
-      const int kb1 = min(kb0 + a.kb_per_split, KB);
       const int to = ut / a.tiles_t;
       pre = min(STAGES, kb1 - kb0);
       for (int s = 0; s < pre; ++s) {
@@ -259,14 +309,12 @@ __global__ void __launch_bounds__(kThreads, BN == 64 ? 2 : 1)
       };
       for (int p = 0; p < nph && !*abort_flag; ++p) {
         const GemmTcArgs& a = P.ph[p];
-        const UnitIter it = units_of(a);
-        const int KB = a.K / kTileK;
-        const int kb0 = it.split() * a.kb_per_split;
-        const int kb1 = min(kb0 + a.kb_per_split, KB);
+        WorkIter wi = work_of(a);
+        int ut, kb0, kb1;
         stamp(P.trace, p, 0);
         first_b = true;
         phase_ready = false;
-        for (int ut = it.first(); ut < it.tiles && !*abort_flag; ut = it.next(ut)) {
+        while (!*abort_flag && wi.next(ut, kb0, kb1)) {
           const int tt = ut % a.tiles_t;
           const int to = ut / a.tiles_t;
           for (int kb = kb0; kb < kb1 && !*abort_flag; ++kb, ++issued) {
@@ -312,12 +360,9 @@ __global__ void __launch_bounds__(kThreads, BN == 64 ? 2 : 1)
       uint32_t last_phase = 0;
       bool ok = true;
       for (int p = 0; p < nph && ok && !*abort_flag; ++p) {
-        const GemmTcArgs& a = P.ph[p];
-        const UnitIter it = units_of(a);
-        const int KB = a.K / kTileK;
-        const int kb0 = it.split() * a.kb_per_split;
-        const int kb1 = min(kb0 + a.kb_per_split, KB);
-        for (int ut = it.first(); ut < it.tiles && ok && !*abort_flag; ut = it.next(ut), ++j) {
+        WorkIter wi = work_of(P.ph[p]);
+        int ut, kb0, kb1;
+        for (; ok && !*abort_flag && wi.next(ut, kb0, kb1); ++j) {
           const int acc = j & 1;
           const uint32_t acc_phase = (j >> 1) & 1;
           if (!mbar_wait(&tempty[acc], acc_phase ^ 1, err, abort_flag)) {
@@ -367,8 +412,10 @@ __global__ void __launch_bounds__(kThreads, BN == 64 ? 2 : 1)
       const GemmTcArgs& args = P.ph[p];
       const int EPI = P.epi[p];
       const UnitIter it = units_of(args);
+      WorkIter wi = work_of(args);
       const int S = args.splits;
       const int sp = it.split();
+      const int KB = args.K / kTileK;
       if (p > 0) {
         // the previous phase wrote this phase's norm statistics and operands
         if (ep_tid == 0) *ep_ok = spin_until_geq(P.phase_bar + p - 1, grid, err) ? 1 : 0;
@@ -380,7 +427,8 @@ __global__ void __launch_bounds__(kThreads, BN == 64 ? 2 : 1)
       }
       if (ep_tid == 0) stamp(P.trace, p, 3);
       bool first_unit = true;
-      for (int ut = it.first(); ut < it.tiles; ut = it.next(ut), ++j) {
+      int ut, kb0, kb1;
+      for (; wi.next(ut, kb0, kb1); ++j) {
         const int tt = ut % args.tiles_t;
         const int to = ut / args.tiles_t;
         const int acc = j & 1;
@@ -409,6 +457,64 @@ __global__ void __launch_bounds__(kThreads, BN == 64 ? 2 : 1)
         tc_fence_after();
         if (first_unit && ep_tid == 0) stamp(P.trace, p, 4);
         const uint32_t taddr = tmem_base + ((uint32_t)(quarter * 32) << 16) + acc * L::acc_cols;
+
+        if (args.streamk && kb0 > 0) {
+          // stream-K, a share that starts inside tile ut: its fp32 sums (hi + lo
+          // columns) go to this CTA's slot [BN tokens][128 rows] for the CTA that
+          // holds the tile's first k-block, which finishes the tile
+          float* slot = args.part + (size_t)blockIdx.x * kTileO * BN + row_in_tile;
+#pragma unroll 1
+          for (int c0 = 0; c0 < BN; c0 += 32) {
+            uint32_t v[32], vl[32];
+            const uint32_t col = (c0 / kSplitGroup) * (2 * kSplitGroup) + (c0 % kSplitGroup);
+            tmem_ld32_async(taddr + col, v);
+            tmem_ld32_async(taddr + col + kSplitGroup, vl);
+            tmem_wait_ld();
+            tmem_reg_fence32(v);
+            tmem_reg_fence32(vl);
+#pragma unroll
+            for (int i = 0; i < 32; ++i)
+              __stcg(slot + (size_t)(c0 + i) * kTileO, __uint_as_float(v[i]) + __uint_as_float(vl[i]));
+          }
+          tc_fence_before();
+          mbar_arrive(&tempty[acc]);
+          named_sync(2, 128);  // every thread's stores precede the arrival
+          if (ep_tid == 0) {
+            __threadfence();
+            atomicAdd(args.counters + ut, 1);
+          }
+          first_unit = false;
+          continue;
+        }
+        if (args.streamk && kb1 < KB) {
+          // stream-K, the tile's first k-blocks, not all of them: the CTAs after this
+          // one up to `last` hold the rest (each its share's first unit, which waits
+          // on nothing); add their sums to this accumulator's hi columns
+          const long long W = (long long)(args.tiles_o * args.tiles_t) * KB;
+          const int last = sk_cta_of(W, (long long)ut * KB + KB - 1, grid);
+          if (ep_tid == 0) *ep_ok = spin_until_geq(args.counters + ut, last - (int)blockIdx.x, err) ? 1 : 0;
+          named_sync(2, 128);
+          if (!*ep_ok) {
+            alive = false;
+            break;
+          }
+#pragma unroll 1
+          for (int c0 = 0; c0 < BN; c0 += 32) {
+            uint32_t v[32];
+            const uint32_t col = (c0 / kSplitGroup) * (2 * kSplitGroup) + (c0 % kSplitGroup);
+            tmem_ld32_async(taddr + col, v);
+            tmem_wait_ld();
+            tmem_reg_fence32(v);
+            for (int c = (int)blockIdx.x + 1; c <= last; ++c) {
+              const float* slot = args.part + (size_t)c * kTileO * BN + row_in_tile;
+#pragma unroll
+              for (int i = 0; i < 32; ++i)
+                v[i] = __float_as_uint(__uint_as_float(v[i]) + __ldcg(slot + (size_t)(c0 + i) * kTileO));
+            }
+            tmem_st32_async(taddr + col, v);
+          }
+          tmem_wait_st();
+        }
 
         if (EPI == GEMM_EPI_QKV || EPI == GEMM_EPI_RESID) {
           // 1) this split's partial sums

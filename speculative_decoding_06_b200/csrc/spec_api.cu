@@ -37,7 +37,8 @@ constexpr int kMaxSplits = 16;
 // when the step starts, so no kernel has to reset them
 constexpr int kMaxAttnChunks = kAttnMaxChunks;  // key chunks of one (sequence, kv head, row tile)
 constexpr int kDraftTopK = SPEC_DRAFT_TOPK;  // candidates per draft node
-constexpr int kCountersPerPhase = 1024;  // two ints per split-K tile (<= 2 x 296 resident CTAs)
+constexpr int kCountersPerPhase = 1024;  // two ints per split-K tile (<= 2 x 296 resident CTAs), one per stream-K tile
+constexpr int kSkMaxCtas = 320;          // stream-K phases run on at most this many CTAs (their partial slots)
 
 size_t align_up(size_t x, size_t a) { return (x + a - 1) / a * a; }
 int ceil_div(int a, int b) { return (a + b - 1) / b; }
@@ -114,6 +115,8 @@ WsLayout make_layout(const spec_config& c) {
   size_t pcols = (size_t)std::max(nqkv, c.hidden) * (c.dtype == SPEC_DTYPE_BF16 ? L.splits_cap : 1);
   if (c.dtype == SPEC_DTYPE_F32) pcols = std::max<size_t>(pcols, std::max<size_t>(2 * (size_t)c.ffn, c.vocab));
   L.partial_bytes = 4 * (size_t)L.Mpad * pcols;
+  // stream-K hand-over slots: [resident CTAs][128 rows][BN <= 128 tokens] fp32
+  if (c.dtype == SPEC_DTYPE_BF16) L.partial_bytes = std::max(L.partial_bytes, 4 * (size_t)kSkMaxCtas * 128 * 128);
   L.partial = take(L.partial_bytes);
   if (c.dtype == SPEC_DTYPE_BF16) {
     // chunked tensor-core attention: one [128 rows][hd] partial per CTA
@@ -248,6 +251,7 @@ struct LayerMaps {
 
 struct GemmPlan {
   int bn, tiles_o, tiles_t, splits, kbps, grid;
+  int sk = 0;  // stream-K over all resident CTAs (GemmTcArgs::streamk)
 };
 
 struct StepPlan {
@@ -309,6 +313,7 @@ struct spec_handle {
   int max_splits = 16;    // split-K cap
   int max_chunks = kMaxAttnChunks;  // attention key-chunk cap
   int resident_cap = 0;   // 0: as many CTAs per SM as fit
+  bool streamk = true;    // stream-K for the SWIGLU and ARGMAX phases when whole tiles leave CTAs idle
   float rescale_slack = 8.f;  // attention: running-max slack in log2 units (p <= 2^slack)
   int attn_clusters[kAttnMaxChunks + 1] = {};  // co-resident clusters of n chunk CTAs
   bool attn_dsmem = true;     // merge chunk partials through distributed shared memory when they fit a cluster
@@ -400,6 +405,18 @@ GemmPlan plan_gemm(const spec_handle* h, int rows_per_tile, int n_out, int K, in
   p.kbps = ceil_div(KB, S);
   p.splits = ceil_div(KB, p.kbps);  // no empty split
   p.grid = p.splits > 1 ? base * p.splits : std::min(base, resident);
+  // Stream-K for the phases without split-K when whole tiles would leave CTAs
+  // idle in the last round (more than 2 % of the CTA-rounds): every resident
+  // CTA then streams the same number of weight k-blocks.
+  if (h->streamk && (epi == GEMM_EPI_SWIGLU || epi == GEMM_EPI_ARGMAX) && p.splits == 1 &&
+      resident <= kSkMaxCtas && base <= kCountersPerPhase && (long long)base * KB >= 2LL * resident &&
+      (size_t)resident * 128 * p.bn * 4 <= h->lay.partial_bytes) {
+    const long long rounds = ceil_div(base, resident);
+    if (rounds * resident * 100 > 102LL * base) {
+      p.sk = 1;
+      p.grid = resident;
+    }
+  }
   return p;
 }
 
@@ -493,6 +510,7 @@ GemmTcLaunch gemm_launch(const GemmPlan& p, int epi, int n_out, int K, int M, co
   L.args.tiles_t = p.tiles_t;
   L.args.splits = p.splits;
   L.args.kb_per_split = p.kbps;
+  L.args.streamk = p.sk;
   L.args.seg_rows[0] = s0;
   L.args.seg_rows[1] = s1;
   L.args.seg_rows[2] = s2;
@@ -596,11 +614,13 @@ struct PhaseBuilder {
   GemmPhase down(int l, int slot, const void* next_norm) const {
     return resid(sp.down, h->cfg.ffn, &h->maps[l].wd, &h->map_h[bi], next_norm, slot);
   }
-  GemmPhase gu(int l) const {
+  GemmPhase gu(int l, int slot) const {
     const spec_config& c = h->cfg;
     const WsLayout& L = h->lay;
     GemmTcLaunch g = gemm_launch(sp.gu, GEMM_EPI_SWIGLU, c.ffn, d, M, &h->maps[l].wg, &h->maps[l].wu, nullptr,
                                  &h->map_xn[bi], 0, 0, 0, sv.err);
+    g.args.part = h->W<float>(L.partial);  // stream-K hand-over slots
+    g.args.counters = ctr(slot);
     g.args.ss_in = h->W<float>(L.ss);
     g.args.n_ss = L.n_ss;
     g.args.ss_ld = L.Mpad;
@@ -612,13 +632,18 @@ struct PhaseBuilder {
   }
   // final norm (folded) + LM head with per-tile top-2; logits also stored when given;
   // with `sample`, the top-2 is of the temperature-scaled logits plus the Gumbel noise
-  GemmPhase lm(float* logits, bool sample) const { return lm_rows(logits, sample, sp.lm, &h->map_lm, h->cfg.vocab); }
+  GemmPhase lm(float* logits, bool sample, int slot) const {
+    return lm_rows(logits, sample, sp.lm, &h->map_lm, h->cfg.vocab, slot);
+  }
   // the same over a given set of LM-head rows (the reduced draft vocabulary)
-  GemmPhase lm_rows(float* logits, bool sample, const GemmPlan& plan, const CUtensorMap* map, int rows) const {
+  GemmPhase lm_rows(float* logits, bool sample, const GemmPlan& plan, const CUtensorMap* map, int rows,
+                    int slot) const {
     const spec_config& c = h->cfg;
     const WsLayout& L = h->lay;
     GemmTcLaunch g = gemm_launch(plan, GEMM_EPI_ARGMAX, rows, d, M, map, nullptr, nullptr, &h->map_xn[bi], rows, 0, 0,
                                  sv.err);
+    g.args.part = h->W<float>(L.partial);  // stream-K hand-over slots
+    g.args.counters = ctr(slot);
     g.args.top_part = h->W<Top2>(L.top_part);
     g.args.top_ld = L.Mpad;
     g.args.dbg_logits = logits;
@@ -729,9 +754,10 @@ cudaError_t enqueue_step(spec_handle* h, const StepPlan& sp, int mode, bool dbg,
       m.n_phases = 4;
       // split-K counter regions 4 * (l + 1) + phase (region 0 is the first QKV launch's)
       m.ph[0] = pb.o(l, 4 * (l + 1) + 0);
-      m.ph[1] = pb.gu(l);
+      m.ph[1] = pb.gu(l, 4 * (l + 1) + 1);
       m.ph[2] = pb.down(l, 4 * (l + 1) + 2, next_norm);
-      m.ph[3] = (l + 1 < c.n_layers) ? pb.qkv(l + 1, 4 * (l + 1) + 3) : pb.lm(dbg ? h->dbg_logits : nullptr, h->temperature > 0.f);
+      m.ph[3] = (l + 1 < c.n_layers) ? pb.qkv(l + 1, 4 * (l + 1) + 3)
+                                     : pb.lm(dbg ? h->dbg_logits : nullptr, h->temperature > 0.f, 4 * (l + 1) + 3);
       if (h->trace && l == h->trace_layer) m.trace = h->trace;
       LK(SPEC_PROF_GEMM_LAYER, 1, gemm_multi_launch(m, st, pdl));
       CUDA_RET(tap_after(l + 1, pdl));
@@ -894,15 +920,15 @@ cudaError_t enqueue_draft(spec_handle* h, const StepPlan& sp, bool kv_only, bool
   float* logits = h->W<float>(L.dlogits);
   m.n_phases = 4;
   m.ph[0] = pb.o(Ld, 8 + 0);
-  m.ph[1] = pb.gu(Ld);
+  m.ph[1] = pb.gu(Ld, 8 + 1);
   m.ph[2] = pb.down(Ld, 8 + 2, h->draft_final_norm);
   // the draft head's own top-k reads the logits (over the reduced vocabulary when there is one)
   const int Vd = c.draft_vocab ? c.draft_vocab : c.vocab;
   if (c.draft_vocab) {
     const GemmPlan pl = plan_gemm(h, 128, Vd, d, M, GEMM_EPI_ARGMAX);
-    m.ph[3] = pb.lm_rows(logits, false, pl, &h->map_lm_draft, Vd);
+    m.ph[3] = pb.lm_rows(logits, false, pl, &h->map_lm_draft, Vd, 8 + 3);
   } else {
-    m.ph[3] = pb.lm(logits, false);
+    m.ph[3] = pb.lm(logits, false, 8 + 3);
   }
   LK(SPEC_PROF_GEMM_LAYER, 1, gemm_multi_launch(m, st, pdl));
   if (ts)
@@ -1298,6 +1324,7 @@ int spec_init(const spec_config* cfg, const spec_weights* w, void* kv_cache, siz
     if (const char* q = strstr(t, "bn64max=")) if (sscanf(q + 8, "%d", &v) == 1 && v >= 64) h->bn64_max = v;
     if (const char* q = strstr(t, "bn96=")) if (sscanf(q + 5, "%d", &v) == 1) h->bn96 = v != 0;
     if (const char* q = strstr(t, "per_sm=")) if (sscanf(q + 7, "%d", &v) == 1 && v >= 0) h->resident_cap = v;
+    if (const char* q = strstr(t, "sk=")) if (sscanf(q + 3, "%d", &v) == 1) h->streamk = v != 0;
     float fv = 0.f;
     if (const char* q = strstr(t, "rescale=")) if (sscanf(q + 8, "%f", &fv) == 1 && fv >= 0.f && fv <= 15.f) h->rescale_slack = fv;
   }
