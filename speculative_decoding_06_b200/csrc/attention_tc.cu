@@ -483,9 +483,12 @@ __global__ void __launch_bounds__(kThreads, 1) attn_tc_kernel(const __grid_const
         const float p0 = ok ? fast_exp2(fmaf(s0, sl2, nm)) : 0.f;
         const float p1 = ok ? fast_exp2(fmaf(s1, sl2, nm)) : 0.f;
         ls4[c & 3] += p0 + p1;
-        const __half2 h2 = __floats2half2_rn(p0, p1);
-        const float2 hf2 = __half22float2(h2);
-        const __half2 l2 = __floats2half2_rn(p0 - hf2.x, p1 - hf2.y);
+        // hi: p truncated to fp16's 11 significant bits (exact in fp16 for p >= 2^-14,
+        // so one conversion per pair instead of a round trip), lo: the exact remainder
+        const float t0 = __uint_as_float(__float_as_uint(p0) & 0xFFFFE000u);
+        const float t1 = __uint_as_float(__float_as_uint(p1) & 0xFFFFE000u);
+        const __half2 h2 = __floats2half2_rn(t0, t1);
+        const __half2 l2 = __floats2half2_rn(p0 - t0, p1 - t1);
         pk[c] = *reinterpret_cast<const uint32_t*>(&h2);
         pl[c] = *reinterpret_cast<const uint32_t*>(&l2);
       }

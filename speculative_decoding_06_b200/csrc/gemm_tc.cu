@@ -58,7 +58,8 @@ struct SmemLayout {
   // per-token norm scale r[BN], then the largest of: SWIGLU gate and up values
   // [128][17] (padded rows: conflict-free), ARGMAX per-warp results [4][BN], RESID
   // per-warp sums of squares [4][BN]
-  static constexpr uint32_t epi_extra = cmax(128 * 17 * 4, cmax(4 * BN * (uint32_t)sizeof(Top2), 4 * BN * 4));
+  static constexpr uint32_t epi_extra =
+      cmax(cmax(128 * 17 * 4, 16 * 129 * 4), cmax(4 * BN * (uint32_t)sizeof(Top2), 4 * BN * 4));
   static constexpr uint32_t epi_bytes = BN * 4 + epi_extra;
   static constexpr uint32_t bar_off = (epi_off + epi_bytes + 7) & ~7u;
   static constexpr uint32_t n_bars = 2 * STAGES + 4;
@@ -138,6 +139,17 @@ __device__ __forceinline__ WorkIter work_of(const GemmTcArgs& a) {
   w.g = W * it.b / it.grid;
   w.w1 = W * (it.b + 1) / it.grid;
   return w;
+}
+
+// float -> unsigned key with the same order (for integer warp reductions)
+__device__ __forceinline__ uint32_t order_key(float v) {
+  const uint32_t u = __float_as_uint(v);
+  return (u & 0x80000000u) ? ~u : (u | 0x80000000u);
+}
+
+// (value desc, index asc)
+__device__ __forceinline__ bool topk_better(float a, int ai, float b, int bi) {
+  return a > b || (a == b && ai < bi);
 }
 
 // stream-K: the CTA whose share holds k-block index g of the phase (W in all, over grid CTAs)
@@ -762,6 +774,151 @@ __global__ void __launch_bounds__(kThreads, BN == 64 ? 2 : 1)
             for (int i = 0; i < 16; ++i) {
               const int t = t_base + c0 + i;
               if (row_ok && t < args.M) split_store(args.out_bf16, t, args.ld_out, o, (v[i] + vl[i]) * r_s[c0 + i]);
+            }
+          }
+          tc_fence_before();
+          mbar_arrive(&tempty[acc]);
+        } else if (EPI == GEMM_EPI_TOPK) {
+          // Per 16 tokens: the tile's 128 x 16 logits go to shared memory token-major;
+          // warp w then takes tokens 4w .. 4w + 3 of the 16 side by side, each lane 4
+          // of a token's 128 rows (lane + 32u), sorted.  T = the k-th largest of the
+          // 32 lane maxima (a bitonic sort across the warp) is a lower bound for the
+          // tile's k-th largest value, so the values >= T (a prefix of each lane's
+          // four) hold the tile's k best: they become the tile's candidates (at most
+          // kCandSlots; ties at T that would overflow them fall back to k rounds of an
+          // exact warp-wide selection).  Also the tile's (max, sum of exp(l - max)).
+          float* sT = reinterpret_cast<float*>(epx);  // [16][129]
+          const int o = to * kTileO + row_in_tile;
+          const bool row_ok = o < args.n_out;
+          const int K = args.topk;
+          const uint32_t lt_mask = (1u << lane) - 1u;
+#pragma unroll 1
+          for (int c0 = 0; c0 < BN; c0 += 16) {
+            float v[16], vl[16];
+            const uint32_t col = (c0 / kSplitGroup) * (2 * kSplitGroup) + (c0 % kSplitGroup);
+            tmem_ld16x2(taddr + col, taddr + col + kSplitGroup, v, vl);
+#pragma unroll
+            for (int i = 0; i < 16; ++i) {
+              const float x = (v[i] + vl[i]) * r_s[c0 + i];
+              const int t = t_base + c0 + i;
+              if (args.dbg_logits && row_ok && t < args.M) args.dbg_logits[(size_t)t * args.n_out + o] = x;
+              sT[i * 129 + row_in_tile] = row_ok ? x : -INFINITY;
+            }
+            named_sync(1, 128);
+            float a[4][4];
+            int ai[4][4];
+#pragma unroll
+            for (int q = 0; q < 4; ++q) {
+              const int i = ep_warp * 4 + q;
+#pragma unroll
+              for (int u = 0; u < 4; ++u) {
+                a[q][u] = sT[i * 129 + lane + 32 * u];
+                const int oo = to * kTileO + lane + 32 * u;
+                ai[q][u] = oo < args.n_out ? oo : 0x7fffffff;
+              }
+            }
+            named_sync(1, 128);  // the staging area is free for the next 16 tokens
+            auto cx = [&](int q, int x, int y) {
+              if (topk_better(a[q][y], ai[q][y], a[q][x], ai[q][x])) {
+                const float tv = a[q][x];
+                const int ti = ai[q][x];
+                a[q][x] = a[q][y];
+                ai[q][x] = ai[q][y];
+                a[q][y] = tv;
+                ai[q][y] = ti;
+              }
+            };
+#pragma unroll
+            for (int q = 0; q < 4; ++q) {
+              cx(q, 0, 1);
+              cx(q, 2, 3);
+              cx(q, 0, 2);
+              cx(q, 1, 3);
+              cx(q, 1, 2);
+            }
+            // bitonic sort (descending) of the lane maxima: lane r ends with the r-th largest
+            float srt[4];
+#pragma unroll
+            for (int q = 0; q < 4; ++q) srt[q] = a[q][0];
+#pragma unroll
+            for (int kk = 2; kk <= 32; kk <<= 1)
+#pragma unroll
+              for (int jj = kk >> 1; jj > 0; jj >>= 1) {
+                const bool keep_max = ((lane & jj) == 0) == ((lane & kk) == 0);
+#pragma unroll
+                for (int q = 0; q < 4; ++q) {
+                  const float y = __shfl_xor_sync(0xffffffffu, srt[q], jj);
+                  srt[q] = keep_max ? fmaxf(srt[q], y) : fminf(srt[q], y);
+                }
+              }
+            float thr[4], mx[4], se[4];
+#pragma unroll
+            for (int q = 0; q < 4; ++q) {
+              thr[q] = __shfl_sync(0xffffffffu, srt[q], K - 1);
+              mx[q] = __shfl_sync(0xffffffffu, srt[q], 0);
+              se[q] = 0.f;
+              if (mx[q] > -INFINITY) {
+#pragma unroll
+                for (int u = 0; u < 4; ++u) se[q] += fast_exp2((a[q][u] - mx[q]) * 1.4426950408889634f);
+              }
+            }
+#pragma unroll
+            for (int off = 16; off > 0; off >>= 1)
+#pragma unroll
+              for (int q = 0; q < 4; ++q) se[q] += __shfl_xor_sync(0xffffffffu, se[q], off);
+#pragma unroll
+            for (int q = 0; q < 4; ++q) {
+              const int t = t_base + c0 + ep_warp * 4 + q;
+              if (t >= args.M) continue;  // (the same for the whole warp)
+              const size_t cb = (size_t)t * args.cand_ld + to;
+              float* cv = args.cand_v + cb * kCandSlots;
+              int32_t* ci = args.cand_i + cb * kCandSlots;
+              // candidates: this lane's values >= T, a prefix of its sorted four
+              const int c = (a[q][0] >= thr[q]) + (a[q][1] >= thr[q]) + (a[q][2] >= thr[q]) + (a[q][3] >= thr[q]);
+              const uint32_t b0 = __ballot_sync(0xffffffffu, c & 1);
+              const uint32_t b1 = __ballot_sync(0xffffffffu, c & 2);
+              const uint32_t b2 = __ballot_sync(0xffffffffu, c & 4);
+              const int tot = __popc(b0) + 2 * __popc(b1) + 4 * __popc(b2);
+              if (tot <= kCandSlots) {
+                const int pre = __popc(b0 & lt_mask) + 2 * __popc(b1 & lt_mask) + 4 * __popc(b2 & lt_mask);
+#pragma unroll
+                for (int u = 0; u < 4; ++u)
+                  if (u < c) {
+                    cv[pre + u] = a[q][u];
+                    ci[pre + u] = ai[q][u];
+                  }
+                if (lane >= tot && lane < kCandSlots) {
+                  cv[lane] = -INFINITY;
+                  ci[lane] = 0x7fffffff;
+                }
+              } else {
+                // many values tie at T: the k best by k rounds of a warp-wide maximum
+                int head = 0;
+                float rv = -INFINITY;
+                int ri = 0x7fffffff;
+                for (int rr = 0; rr < K; ++rr) {
+                  const float hv = head == 0 ? a[q][0] : head == 1 ? a[q][1] : head == 2 ? a[q][2]
+                                 : head == 3 ? a[q][3] : -INFINITY;
+                  const int hi = head == 0 ? ai[q][0] : head == 1 ? ai[q][1] : head == 2 ? ai[q][2]
+                               : head == 3 ? ai[q][3] : 0x7fffffff;
+                  const uint32_t key = order_key(hv);
+                  const uint32_t kmax = __reduce_max_sync(0xffffffffu, key);
+                  const uint32_t imin = __reduce_min_sync(0xffffffffu, key == kmax ? (uint32_t)hi : 0xffffffffu);
+                  const int wl = __ffs(__ballot_sync(0xffffffffu, key == kmax && (uint32_t)hi == imin)) - 1;
+                  const float wv = __shfl_sync(0xffffffffu, hv, wl);
+                  const int wi = __shfl_sync(0xffffffffu, hi, wl);
+                  if (lane == wl) ++head;
+                  if (lane == rr) {
+                    rv = wv;
+                    ri = wi;
+                  }
+                }
+                if (lane < kCandSlots) {
+                  cv[lane] = lane < K ? rv : -INFINITY;
+                  ci[lane] = lane < K ? ri : 0x7fffffff;
+                }
+              }
+              if (lane == 0) args.cand_lse[cb] = make_float2(mx[q], se[q]);
             }
           }
           tc_fence_before();

@@ -21,7 +21,9 @@ struct Top2;
 //          x*w (split bf16) and the tile's per-token sums of squares of x
 //   SWIGLU gate rows 0-63, up rows 64-127 of a tile; silu(g)*u as split bf16
 //   ARGMAX per-token (best, index, runner-up) of the tile's vocabulary rows
-enum { GEMM_EPI_QKV = 0, GEMM_EPI_SWIGLU = 1, GEMM_EPI_ARGMAX = 2, GEMM_EPI_RESID = 3, GEMM_EPI_STORE = 4 };
+//   TOPK   per token, the tile's k best logits and (max, sum of exp) (draft LM head)
+enum { GEMM_EPI_QKV = 0, GEMM_EPI_SWIGLU = 1, GEMM_EPI_ARGMAX = 2, GEMM_EPI_RESID = 3, GEMM_EPI_STORE = 4,
+       GEMM_EPI_TOPK = 5 };
 
 struct StepView;
 
@@ -53,7 +55,14 @@ struct GemmTcArgs {
   // ARGMAX
   Top2* top_part;     // [tiles_o][top_ld]
   int top_ld;
-  float* dbg_logits;  // optional [M][n_out] (the logits themselves, before any sampling noise)
+  float* dbg_logits;  // optional [M][n_out] (the logits themselves, before any sampling noise; ARGMAX, TOPK)
+  // TOPK: per token and tile, kCandSlots candidates that hold the tile's `topk` (<= 16)
+  // best logits (unused slots -inf) into cand_v / cand_i [tokens][cand_ld][kCandSlots]
+  // and (max, sum of exp(l - max)) into cand_lse [tokens][cand_ld]; cand_ld = tiles_o
+  int topk, cand_ld;
+  float* cand_v;
+  int32_t* cand_i;
+  float2* cand_lse;
   // sampling (inv_temp > 0): the row's choice is argmax_v(logit_v * inv_temp + gumbel(seed, sid, pos, v))
   // with sid = row_sid[t] and pos = row_pos[t]; inv_temp = 0: the plain argmax
   const int32_t* row_pos;
@@ -84,6 +93,7 @@ struct GemmTcArgs {
 };
 
 constexpr int kMaxGemmPhases = 4;
+constexpr int kCandSlots = 24;  // TOPK candidates per (token, vocabulary tile)
 constexpr int kGemmTraceMarks = 16;  // %globaltimer marks per CTA and phase (optional timeline)
 
 // kernel parameters: the tensor maps of every phase (a0, a1, a2, b) and the phases
@@ -183,6 +193,14 @@ constexpr int kTopKMax = 16;
 // (id_map: token id of each of the V columns; the indices written are id_map[column])
 cudaError_t launch_topk_rows(int M, int V, const float* logits, size_t ld, int k, int32_t* idx, float* val,
                              float* lse, cudaStream_t s, bool pdl, const int32_t* id_map = nullptr);
+
+// top-k per row (k in {4, 8, 10, 16}) from the LM head's TOPK candidates: cand_v / cand_i
+// [M][tiles][kCandSlots] (a superset of each tile's k best), cand_lse [M][tiles] (max, sum of
+// exp(l - max));
+// with lse != NULL also the row's log-sum-exp; indices mapped through id_map when given
+cudaError_t launch_topk_merge(int M, int tiles, int k, const float* cand_v, const int32_t* cand_i,
+                              const float2* cand_lse, int32_t* idx, float* val, float* lse, cudaStream_t s, bool pdl,
+                              const int32_t* id_map = nullptr);
 
 // a launch configuration with programmatic dependent launch when pdl (attr: 1 slot)
 cudaLaunchConfig_t make_cfg(dim3 grid, dim3 block, size_t smem, cudaStream_t s, bool pdl, cudaLaunchAttribute* attr);

@@ -738,4 +738,131 @@ cudaError_t launch_topk_rows(int M, int V, const float* logits, size_t ld, int k
   }
 }
 
+// Top-k of a row from the per-tile candidates of the LM head's TOPK epilogue: each
+// 128-row vocabulary tile gave kCandSlots candidates holding its k best (in no
+// particular order; unused slots -inf) and its (max, sum of exp(l - max)).  The
+// row's k best are among the tiles' k best; its log-sum-exp combines the tiles'
+// pairs.  One CTA per row; thread j takes tiles j, j + 256, ...
+template <int K, bool LSE>
+__global__ void __launch_bounds__(256) topk_merge_kernel(int tiles, const float* __restrict__ cand_v,
+                                                        const int32_t* __restrict__ cand_i,
+                                                        const float2* __restrict__ cand_lse,
+                                                        int32_t* __restrict__ out_i, float* __restrict__ out_v,
+                                                        float* __restrict__ out_lse,
+                                                        const int32_t* __restrict__ id_map) {
+  __shared__ float wv[8][K];
+  __shared__ int wi[8][K];
+  __shared__ float lse_m[8], lse_s[8];
+  pdl_wait();
+  pdl_launch_dependents();
+  const int r = blockIdx.x;
+  const int warp = threadIdx.x >> 5;
+  const int lane = threadIdx.x & 31;
+  constexpr float kLog2e = 1.4426950408889634f;
+  float lv[K];
+  int li[K];
+#pragma unroll
+  for (int j = 0; j < K; ++j) {
+    lv[j] = -INFINITY;
+    li[j] = 0x7fffffff;
+  }
+  float lm = -INFINITY, ls = 0.f;
+  for (int t = threadIdx.x; t < tiles; t += blockDim.x) {
+    const size_t b = (size_t)r * tiles + t;
+    const float* cv = cand_v + b * kCandSlots;
+    const int32_t* ci = cand_i + b * kCandSlots;
+    for (int j = 0; j < kCandSlots; ++j) {
+      float x = __ldcs(cv + j);
+      int c = __ldcs(ci + j);
+      if (!topk_better(x, c, lv[K - 1], li[K - 1])) continue;
+#pragma unroll
+      for (int q = 0; q < K; ++q) {
+        if (topk_better(x, c, lv[q], li[q])) {
+          const float tv = lv[q];
+          const int ti = li[q];
+          lv[q] = x;
+          li[q] = c;
+          x = tv;
+          c = ti;
+        }
+      }
+    }
+    if (LSE) {
+      const float2 pr = __ldcs(cand_lse + b);
+      if (pr.x > -INFINITY) {
+        if (pr.x > lm) {
+          ls = (lm == -INFINITY ? 0.f : ls * fast_exp2((lm - pr.x) * kLog2e));
+          lm = pr.x;
+        }
+        ls += pr.y * fast_exp2((pr.x - lm) * kLog2e);
+      }
+    }
+  }
+  if (LSE) {
+    for (int o = 16; o > 0; o >>= 1) {
+      const float m2 = __shfl_xor_sync(0xffffffffu, lm, o);
+      const float s2 = __shfl_xor_sync(0xffffffffu, ls, o);
+      const float mm = fmaxf(lm, m2);
+      if (mm > -INFINITY) {
+        ls = (lm == -INFINITY ? 0.f : ls * fast_exp2((lm - mm) * kLog2e)) +
+             (m2 == -INFINITY ? 0.f : s2 * fast_exp2((m2 - mm) * kLog2e));
+        lm = mm;
+      }
+    }
+    if (lane == 0) {
+      lse_m[warp] = lm;
+      lse_s[warp] = ls;
+    }
+  }
+  warp_merge_topk<K>(lv, li, wv[warp], wi[warp]);
+  __syncthreads();
+  if (warp == 0) {
+    float mv[K];
+    int mi[K];
+#pragma unroll
+    for (int j = 0; j < K; ++j) {
+      mv[j] = lane < 8 ? wv[lane][j] : -INFINITY;
+      mi[j] = lane < 8 ? wi[lane][j] : 0x7fffffff;
+    }
+    __syncwarp();
+    warp_merge_topk<K>(mv, mi, wv[0], wi[0]);
+    __syncwarp();
+    if (lane < K) {
+      out_v[(size_t)r * K + lane] = wv[0][lane];
+      out_i[(size_t)r * K + lane] = id_map ? id_map[wi[0][lane]] : wi[0][lane];
+    }
+    if (LSE && lane == 0) {
+      float M0 = -INFINITY;
+      for (int w = 0; w < 8; ++w) M0 = fmaxf(M0, lse_m[w]);
+      float S0 = 0.f;
+      for (int w = 0; w < 8; ++w)
+        if (lse_m[w] > -INFINITY) S0 += lse_s[w] * fast_exp2((lse_m[w] - M0) * kLog2e);
+      out_lse[r] = M0 + __logf(S0);
+    }
+  }
+}
+
+cudaError_t launch_topk_merge(int M, int tiles, int k, const float* cand_v, const int32_t* cand_i,
+                              const float2* cand_lse, int32_t* idx, float* val, float* lse, cudaStream_t s, bool pdl,
+                              const int32_t* id_map) {
+  if (M < 1 || tiles < 1 || k < 1 || k > kTopKMax) return cudaErrorInvalidValue;
+  cudaLaunchAttribute attr[1];
+  cudaLaunchConfig_t cfg = make_cfg(dim3(M), dim3(256), 0, s, pdl, attr);
+  const bool l = lse != nullptr;
+  switch (k) {
+#define SPEC_TOPK_MERGE(KK)                                                                                         \
+  case KK:                                                                                                          \
+    return l ? cudaLaunchKernelEx(&cfg, topk_merge_kernel<KK, true>, tiles, cand_v, cand_i, cand_lse, idx, val, lse, \
+                                  id_map)                                                                           \
+             : cudaLaunchKernelEx(&cfg, topk_merge_kernel<KK, false>, tiles, cand_v, cand_i, cand_lse, idx, val, lse, \
+                                  id_map);
+    SPEC_TOPK_MERGE(4)
+    SPEC_TOPK_MERGE(8)
+    SPEC_TOPK_MERGE(10)
+    SPEC_TOPK_MERGE(16)
+#undef SPEC_TOPK_MERGE
+    default: return cudaErrorInvalidValue;
+  }
+}
+
 }  // namespace spec

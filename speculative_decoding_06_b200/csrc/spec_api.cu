@@ -57,7 +57,7 @@ struct WsLayout {
   size_t ss, gemm_ctr, attn_ctr, phase_bar;
   int gemm_ctr_n = 0;  // ints: 4 phases x launches of a step x kCountersPerPhase
   // draft head: split features [2 Mpad][3d], [g|e] operand [2 Mpad][2d], logits, top-k
-  size_t fsplit = 0, ge = 0, dlogits = 0, dtop_i = 0, dtop_v = 0;
+  size_t fsplit = 0, ge = 0, cand_v = 0, cand_i = 0, cand_lse = 0, dtop_i = 0, dtop_v = 0;
   // feature tap: bf16 residual stream after the three feature layers [3][Mpad][d]
   size_t tap = 0;
   // dynamic draft tree: per-tree nodes and offers, saved root features, per-row top-k and log-sum-exp, output
@@ -144,7 +144,12 @@ WsLayout make_layout(const spec_config& c) {
   if (c.draft_head) {
     L.fsplit = take(2 * 2 * (size_t)L.Mpad * 3 * c.hidden);
     L.ge = take(2 * 2 * (size_t)L.Mpad * 2 * c.hidden);
-    L.dlogits = take(4 * (size_t)L.Mpad * c.vocab);
+    // the draft LM head's top-k candidates: per row and 128-row vocabulary tile,
+    // kCandSlots (value, index) holding the tile's k <= 16 best, and (max, sum of exp)
+    const size_t vtiles = ((size_t)c.vocab + 127) / 128;
+    L.cand_v = take(4 * (size_t)L.Mpad * vtiles * kCandSlots);
+    L.cand_i = take(4 * (size_t)L.Mpad * vtiles * kCandSlots);
+    L.cand_lse = take(8 * (size_t)L.Mpad * vtiles);
     L.dtop_i = take(4 * (size_t)L.Mpad * kDraftTopK);
     L.dtop_v = take(4 * (size_t)L.Mpad * kDraftTopK);
     const size_t tn = (size_t)c.max_batch * kTreeMaxNodes;
@@ -408,7 +413,7 @@ GemmPlan plan_gemm(const spec_handle* h, int rows_per_tile, int n_out, int K, in
   // Stream-K for the phases without split-K when whole tiles would leave CTAs
   // idle in the last round (more than 2 % of the CTA-rounds): every resident
   // CTA then streams the same number of weight k-blocks.
-  if (h->streamk && (epi == GEMM_EPI_SWIGLU || epi == GEMM_EPI_ARGMAX) && p.splits == 1 &&
+  if (h->streamk && (epi == GEMM_EPI_SWIGLU || epi == GEMM_EPI_ARGMAX || epi == GEMM_EPI_TOPK) && p.splits == 1 &&
       resident <= kSkMaxCtas && base <= kCountersPerPhase && (long long)base * KB >= 2LL * resident &&
       (size_t)resident * 128 * p.bn * 4 <= h->lay.partial_bytes) {
     const long long rounds = ceil_div(base, resident);
@@ -632,6 +637,19 @@ struct PhaseBuilder {
   }
   // final norm (folded) + LM head with per-tile top-2; logits also stored when given;
   // with `sample`, the top-2 is of the temperature-scaled logits plus the Gumbel noise
+  // the draft head's LM head: per row and vocabulary tile, the tile's k best and (max,
+  // sum of exp) for launch_topk_merge; logits (optional) get the logits themselves
+  GemmPhase lm_topk(float* logits, const GemmPlan& plan, const CUtensorMap* map, int rows, int k, int slot) const {
+    const WsLayout& L = h->lay;
+    GemmPhase q = lm_rows(logits, false, plan, map, rows, slot);
+    q.epi = GEMM_EPI_TOPK;
+    q.args.topk = k;
+    q.args.cand_ld = plan.tiles_o;
+    q.args.cand_v = h->W<float>(L.cand_v);
+    q.args.cand_i = h->W<int32_t>(L.cand_i);
+    q.args.cand_lse = h->W<float2>(L.cand_lse);
+    return q;
+  }
   GemmPhase lm(float* logits, bool sample, int slot) const {
     return lm_rows(logits, sample, sp.lm, &h->map_lm, h->cfg.vocab, slot);
   }
@@ -917,29 +935,22 @@ cudaError_t enqueue_draft(spec_handle* h, const StepPlan& sp, bool kv_only, bool
   aa.rescale_slack = h->rescale_slack;
   aa.cluster_merge = sp.cluster_merge;
   LK(SPEC_PROF_ATTENTION, 1, launch_attention_tc(aa, h->attn_maps, st, pdl));
-  float* logits = h->W<float>(L.dlogits);
   m.n_phases = 4;
   m.ph[0] = pb.o(Ld, 8 + 0);
   m.ph[1] = pb.gu(Ld, 8 + 1);
   m.ph[2] = pb.down(Ld, 8 + 2, h->draft_final_norm);
-  // the draft head's own top-k reads the logits (over the reduced vocabulary when there is one)
+  // the LM head (over the reduced vocabulary when there is one) keeps, per row and
+  // 128-row tile, the tile's k best and (max, sum of exp); the logits are never stored
+  // (except into the debug buffer), and a small kernel merges the tiles
   const int Vd = c.draft_vocab ? c.draft_vocab : c.vocab;
-  if (c.draft_vocab) {
-    const GemmPlan pl = plan_gemm(h, 128, Vd, d, M, GEMM_EPI_ARGMAX);
-    m.ph[3] = pb.lm_rows(logits, false, pl, &h->map_lm_draft, Vd, 8 + 3);
-  } else {
-    m.ph[3] = pb.lm(logits, false, 8 + 3);
-  }
+  const int K = ts ? ts->K : kDraftTopK;
+  const GemmPlan pl = c.draft_vocab ? plan_gemm(h, 128, Vd, d, M, GEMM_EPI_TOPK) : sp.lm;
+  m.ph[3] = pb.lm_topk(dbg ? h->dbg_logits : nullptr, pl, c.draft_vocab ? &h->map_lm_draft : &h->map_lm, Vd, K, 8 + 3);
   LK(SPEC_PROF_GEMM_LAYER, 1, gemm_multi_launch(m, st, pdl));
-  if (ts)
-    LK(SPEC_PROF_TOPK, 1,
-       launch_topk_rows(M, Vd, logits, Vd, ts->K, h->W<int32_t>(L.tr_top_i), h->W<float>(L.tr_top_v),
-                        h->W<float>(L.tr_lse), st, pdl, h->draft_ids));
-  else
-    LK(SPEC_PROF_TOPK, 1,
-       launch_topk_rows(M, Vd, logits, Vd, kDraftTopK, h->W<int32_t>(L.dtop_i), h->W<float>(L.dtop_v),
-                        nullptr, st, pdl, h->draft_ids));
-  if (dbg) CUDA_RET(cudaMemcpyAsync(h->dbg_logits, logits, 4 * (size_t)M * Vd, cudaMemcpyDeviceToDevice, st));
+  LK(SPEC_PROF_TOPK, 1,
+     launch_topk_merge(M, pl.tiles_o, K, h->W<float>(L.cand_v), h->W<int32_t>(L.cand_i), h->W<float2>(L.cand_lse),
+                       h->W<int32_t>(ts ? L.tr_top_i : L.dtop_i), h->W<float>(ts ? L.tr_top_v : L.dtop_v),
+                       ts ? h->W<float>(L.tr_lse) : nullptr, st, pdl, h->draft_ids));
   return cudaSuccess;
 }
 
