@@ -67,22 +67,19 @@ constexpr uint32_t kKTile = 2 * kKHalf;      // 64 x 128 fp16: 16 KB
 // a K stage holds, per 64-dim half, K's 64 rows then K_lo's 64 rows: one 128-row
 // operand [K; K_lo] per half, so Q_hi [K; K_lo]^T is one N = 128 product
 constexpr uint32_t kKStage = 2 * kKTile;     // 32 KB
-constexpr uint32_t kPTile = kRows * kKeys * 2;  // [128 rows][64 keys] fp16, one 128-byte row each: 16 KB
 static_assert(kKeys == 64, "a P row is one 128-byte swizzled row; two 32-key pieces per block");
 
 // K and V stages are filled and released separately: a K stage is free once the
 // scores that read it are done, a V stage once P.V is
 enum { B_QFULL = 0, B_KFULL = 1, B_VFULL = 3, B_KEMPTY = 5, B_VEMPTY = 7, B_SFULL = 9, B_SFREE = 11, B_PFULL = 13,
-       B_PEMPTY = 14, B_OFULL = 15, B_DRAIN = 16, kNumBars = 17 };
+       B_PEMPTY = 15, B_OFULL = 17, B_DRAIN = 18, kNumBars = 19 };
 
 struct Smem {
   static constexpr uint32_t q = 0;                   // Q hi
   static constexpr uint32_t qlo = q + kQTile;        // Q lo
   static constexpr uint32_t k = qlo + kQTile;        // 2 stages of [K; K_lo]; 64 KB of output staging at the end
   static constexpr uint32_t v = k + 2 * kKStage;     // 2 stages
-  static constexpr uint32_t p = v + 2 * kKTile;      // P hi
-  static constexpr uint32_t plo = p + kPTile;        // P lo
-  static constexpr uint32_t xchg = plo + kPTile;     // row maxima [2][kPerRow][128] and sums [kPerRow][128]
+  static constexpr uint32_t xchg = v + 2 * kKTile;   // row maxima [2][kPerRow][128] and sums [kPerRow][128]
   static constexpr uint32_t lse = xchg + 3 * kPerRow * 128 * 4; // this chunk's log2-sum-exp per row (cluster merge)
   static constexpr uint32_t bars = lse + 128 * 4;
   static constexpr uint32_t misc = bars + kNumBars * 8;  // tmem slot, abort flag, merge flag
@@ -92,11 +89,15 @@ struct Smem {
 static_assert(Smem::dyn <= 227 * 1024, "shared memory");
 
 // tensor-memory columns: two S buffers of 128 (keys 0-63: Q_hi K^T + Q_lo K^T, 64-127:
-// Q_hi K_lo^T, added by the softmax) at 0 and 128, O at 256
+// Q_hi K_lo^T, added by the softmax) at 0 and 128, O at 256, and two P buffers of 64
+// at 384 and 448: the P.V MMAs' A operand (P_hi in 32 columns, then P_lo; two fp16 keys
+// per 32-bit column, the even key in the low half)
 constexpr uint32_t kTmemCols = 512;
 constexpr uint32_t kSCols = 2 * kKeys;
 constexpr uint32_t kColO = 2 * kSCols;
-static_assert(kColO + 128 <= kTmemCols, "tensor memory");
+constexpr uint32_t kColP = kColO + 128;
+constexpr uint32_t kPCols = kKeys;  // one buffer: 32 columns of P_hi, 32 of P_lo
+static_assert(kColP + 2 * kPCols <= kTmemCols, "tensor memory");
 static_assert(Smem::v - Smem::k >= 128 * 512, "output staging (128 rows x 512 B) fits in the K ring");
 
 // fp16 A and B, f32 D, M = 128; S: N = 128 ([K; K_lo]) and N = 64 (K); P.V: N = 128 dims, B MN-major (bit 16)
@@ -229,8 +230,10 @@ __global__ void __launch_bounds__(kThreads, 1) attn_tc_kernel(const __grid_const
       mbar_init(&bar[B_SFULL + s], 1);
       mbar_init(&bar[B_SFREE + s], kRowWarps);
     }
-    mbar_init(&bar[B_PFULL], kRowWarps);
-    mbar_init(&bar[B_PEMPTY], 1);
+    for (int s = 0; s < 2; ++s) {
+      mbar_init(&bar[B_PFULL + s], kRowWarps);
+      mbar_init(&bar[B_PEMPTY + s], 1);
+    }
     mbar_init(&bar[B_OFULL], 1);
     mbar_init(&bar[B_DRAIN], 1);
     *abort_flag = 0;
@@ -347,8 +350,6 @@ __global__ void __launch_bounds__(kThreads, 1) attn_tc_kernel(const __grid_const
       pdl_launch_dependents();
       const uint32_t sq = smem_u32(smem + Smem::q);
       const uint32_t sql = smem_u32(smem + Smem::qlo);
-      const uint32_t sp = smem_u32(smem + Smem::p);
-      const uint32_t spl = smem_u32(smem + Smem::plo);
       auto issue_pv = [&](int j) {
         const uint32_t svv = smem_u32(smem + Smem::v + (j & 1) * kKTile);
 #pragma unroll
@@ -356,17 +357,18 @@ __global__ void __launch_bounds__(kThreads, 1) attn_tc_kernel(const __grid_const
           // P: one 128-byte row of 64 keys per query row; V: 16 keys (rows) per step,
           // its two 64-dim halves kKHalf apart (the N atoms of the MN-major operand)
           const uint64_t bd = sw128_mnmajor_desc(svv + kk * 16 * 128, kKHalf);
-          tc_mma_bf16(tmem + kColO, sw128_kmajor_desc(sp + kk * 32), bd, kIdescPV, (j > 0 || kk > 0) ? 1u : 0u);
-          tc_mma_bf16(tmem + kColO, sw128_kmajor_desc(spl + kk * 32), bd, kIdescPV, 1u);
+          const uint32_t pa = tmem + kColP + (j & 1) * kPCols + kk * 8;  // 16 keys: 8 columns
+          tc_mma_ts(tmem + kColO, pa, bd, kIdescPV, (j > 0 || kk > 0) ? 1u : 0u);
+          tc_mma_ts(tmem + kColO, pa + kPCols / 2, bd, kIdescPV, 1u);
         }
       };
       // P.V of block j (its P written, its V landed)
       auto pv_step = [&](int j) -> bool {
-        if (!mbar_wait(&bar[B_PFULL], j & 1, err, abort_flag)) return false;
+        if (!mbar_wait(&bar[B_PFULL + (j & 1)], (j >> 1) & 1, err, abort_flag)) return false;
         if (!mbar_wait(&bar[B_VFULL + (j & 1)], (j >> 1) & 1, err, abort_flag)) return false;
         tc_fence_after();
         issue_pv(j);
-        tc_commit(&bar[B_PEMPTY]);
+        tc_commit(&bar[B_PEMPTY + (j & 1)]);
         tc_commit(&bar[B_VEMPTY + (j & 1)]);
         return true;
       };
@@ -427,8 +429,6 @@ __global__ void __launch_bounds__(kThreads, 1) attn_tc_kernel(const __grid_const
     const uint64_t anc1 = sv.row_anc[2 * (base + node) + 1];
     const uint32_t tl = tmem + ((uint32_t)((warp & 3) * 32) << 16);  // this warp's TMEM lanes
     const float sl2 = 1.4426950408889634f * 0.08838834764831845f;      // log2(e) / sqrt(128)
-    uint8_t* prow = smem + Smem::p + r * 128;                            // P's row (64 keys, 128 bytes)
-    uint8_t* plrow = smem + Smem::plo + r * 128;                         // P_lo's row
     float* xmax = reinterpret_cast<float*>(smem + Smem::xchg);           // [parity][quarter][row]
     float* xsum = xmax + 2 * kPerRow * 128;                              // [quarter][row]
     const uint32_t kmask = (1u << kKeysPT) - 1u;
@@ -492,12 +492,13 @@ __global__ void __launch_bounds__(kThreads, 1) attn_tc_kernel(const __grid_const
         pk[c] = *reinterpret_cast<const uint32_t*>(&h2);
         pl[c] = *reinterpret_cast<const uint32_t*>(&l2);
       }
-      if (j >= 1 && ok) {
-        // P.V of the previous block has finished: the P buffer is free and O is current
-        ok = __all_sync(0xffffffffu, mbar_wait(&bar[B_PEMPTY], (j - 1) & 1, err, abort_flag));
+      // a larger running max rescales O: P.V of block j - 1 must have finished
+      if (j >= 1 && ok && __any_sync(0xffffffffu, corr != 1.f)) {
+        ok = __all_sync(0xffffffffu,
+                        mbar_wait(&bar[B_PEMPTY + ((j - 1) & 1)], ((j - 1) >> 1) & 1, err, abort_flag));
         if (ok) {
           tc_fence_after();
-          if (__any_sync(0xffffffffu, corr != 1.f)) {
+          {
             uint32_t o[32];
             const uint32_t to_ = tl + kColO + qtr * kDimsPT;
             tmem_ld32_async(to_, o);
@@ -510,23 +511,23 @@ __global__ void __launch_bounds__(kThreads, 1) attn_tc_kernel(const __grid_const
           }
         }
       }
-      // this thread's 32 bytes of the row of the K-major, 128-byte-swizzled A
-      // operand (16-byte chunk c of a row lands at c ^ (row & 7))
+      // P buffer j & 1 is free once P.V of block j - 2 has finished
+      if (j >= 2 && ok) {
+        ok = __all_sync(0xffffffffu, mbar_wait(&bar[B_PEMPTY + (j & 1)], ((j - 2) >> 1) & 1, err, abort_flag));
+        if (ok) tc_fence_after();
+      }
+      // this thread's 16 keys: 8 columns of P_hi and 8 of P_lo in its TMEM lane
       if (ok) {
-#pragma unroll
-        for (int q4 = 0; q4 < kKeysPT / 8; ++q4) {
-          const int chunk = qtr * (kKeysPT / 8) + q4;
-          const int at = (chunk ^ (r & 7)) << 4;
-          *reinterpret_cast<uint4*>(prow + at) = make_uint4(pk[4 * q4], pk[4 * q4 + 1], pk[4 * q4 + 2], pk[4 * q4 + 3]);
-          *reinterpret_cast<uint4*>(plrow + at) = make_uint4(pl[4 * q4], pl[4 * q4 + 1], pl[4 * q4 + 2], pl[4 * q4 + 3]);
-        }
+        const uint32_t tp = tl + kColP + (j & 1) * kPCols + qtr * (kKeysPT / 2);
+        tmem_st8_async(tp, pk);
+        tmem_st8_async(tp + kPCols / 2, pl);
+        tmem_wait_st();
         if (j == 0) stamp(a.trace, 9);
         tc_fence_before();
-        fence_proxy_async_smem();
         __syncwarp();
         if (lane == 0) {
           mbar_arrive(&bar[B_SFREE + st]);
-          mbar_arrive(&bar[B_PFULL]);
+          mbar_arrive(&bar[B_PFULL + (j & 1)]);
         }
       }
       l = l * corr + ((ls4[0] + ls4[1]) + (ls4[2] + ls4[3]));
