@@ -128,6 +128,10 @@ __device__ __forceinline__ void stamp_at(uint64_t* trace, int k) {
 }
 
 __device__ __forceinline__ void named_sync_rows() { asm volatile("bar.sync 1, %0;" ::"n"(32 * kRowWarps) : "memory"); }
+// the kPerRow warps whose threads share TMEM lanes 32 q .. 32 q + 31 (warps q, q + 4, ...)
+__device__ __forceinline__ void named_sync_quad(int q) {
+  asm volatile("bar.sync %0, %1;" ::"r"(2 + q), "n"(32 * kPerRow) : "memory");
+}
 
 
 
@@ -461,7 +465,7 @@ __global__ void __launch_bounds__(kThreads, 1) attn_tc_kernel(const __grid_const
         }
       }
       xmax[(st * kPerRow + qtr) * 128 + r] = fmaxf(fmaxf(mx4[0], mx4[1]), fmaxf(mx4[2], mx4[3]));
-      named_sync_rows();
+      named_sync_quad(warp & 3);  // the four warps that share these rows
       float mraw = xmax[(st * kPerRow) * 128 + r];
 #pragma unroll
       for (int q = 1; q < kPerRow; ++q) mraw = fmaxf(mraw, xmax[(st * kPerRow + q) * 128 + r]);
