@@ -220,7 +220,9 @@ SPEC_API int spec_draft_prefill(spec_handle* h, int seq, const void* feats, cons
 SPEC_API int spec_draft_append(spec_handle* h, int seq, const void* feats, const int32_t* tokens, int n);
 /* One draft-head step over a batch of trees on the draft prefixes: per node,
  * the SPEC_DRAFT_TOPK best vocabulary entries of the draft distribution, by
- * logit descending then index ascending, in top_idx / top_val [nodes][TOPK].
+ * logit descending then index ascending, in top_idx / top_val [nodes][TOPK]
+ * (selected inside the LM-head GEMM, per 128-row vocabulary tile, then merged:
+ * the draft logits are not stored).
  * The draft prefixes are not extended (the trees' K/V are scratch).  Flags:
  * SPEC_DEVICE_OUTPUTS (outputs are device pointers, no synchronisation),
  * SPEC_DEBUG_LOGITS (also the fp32 draft logits to the debug buffer),
@@ -318,7 +320,7 @@ SPEC_API int spec_validate_tree(const int32_t* tokens, const int32_t* parents, i
 #define SPEC_PROF_COMPACT 11     /* K/V compaction */
 #define SPEC_PROF_GEMM_LAYER 12  /* one launch: O, gate/up, down, then the next QKV or the LM head */
 #define SPEC_PROF_DRAFT_FC 13    /* draft head: feature split, fusion FC, input FC */
-#define SPEC_PROF_TOPK 14        /* draft head: top-k over the logits */
+#define SPEC_PROF_TOPK 14        /* draft head: merge of the LM-head tiles' top-k candidates */
 #define SPEC_PROF_FEATURES 15    /* draft-head feature tap and gather (SPEC_FEATURES) */
 #define SPEC_PROF_TREE 16        /* dynamic draft tree: root features, expansion, rerank */
 #define SPEC_PROF_CLASSES 17
