@@ -318,7 +318,8 @@ struct spec_handle {
   int max_splits = 16;    // split-K cap
   int max_chunks = kMaxAttnChunks;  // attention key-chunk cap
   int resident_cap = 0;   // 0: as many CTAs per SM as fit
-  bool streamk = true;    // stream-K for the SWIGLU and ARGMAX phases when whole tiles leave CTAs idle
+  bool streamk = false;   // stream-K for the SWIGLU / ARGMAX / TOPK phases when whole tiles leave CTAs idle
+                          // (SPEC_TUNE sk=1; measured 0.3-2 % slower end to end, so off by default)
   float rescale_slack = 8.f;  // attention: running-max slack in log2 units (p <= 2^slack)
   int attn_clusters[kAttnMaxChunks + 1] = {};  // co-resident clusters of n chunk CTAs
   bool attn_dsmem = true;     // merge chunk partials through distributed shared memory when they fit a cluster
@@ -1844,8 +1845,8 @@ int spec_info(spec_handle* h, int B, int n_nodes, int prefix, char* buf, size_t 
   const StepPlan sp = make_plan(h, B, B * n_nodes, n_nodes, prefix + n_nodes);
   auto g = [](const GemmPlan& p) {
     char t[96];
-    snprintf(t, sizeof(t), "bn%d tiles%dx%d splits%d kb/split%d grid%d", p.bn, p.tiles_o, p.tiles_t, p.splits,
-             p.kbps, p.grid);
+    snprintf(t, sizeof(t), "bn%d tiles%dx%d splits%d kb/split%d grid%d%s", p.bn, p.tiles_o, p.tiles_t, p.splits,
+             p.kbps, p.grid, p.sk ? " stream-K" : "");
     return std::string(t);
   };
   std::string s = "sms " + std::to_string(h->sm_count) + "; attention clusters held [size:count]";
