@@ -318,8 +318,9 @@ struct spec_handle {
   int max_splits = 16;    // split-K cap
   int max_chunks = kMaxAttnChunks;  // attention key-chunk cap
   int resident_cap = 0;   // 0: as many CTAs per SM as fit
-  bool streamk = false;   // stream-K for the SWIGLU / ARGMAX / TOPK phases when whole tiles leave CTAs idle
-                          // (SPEC_TUNE sk=1; measured 0.3-2 % slower end to end, so off by default)
+  int streamk = -1;       // stream-K when whole tiles leave CTAs idle: 1 for the SWIGLU, ARGMAX and TOPK
+                          // phases, 2 for SWIGLU only, 0 off, -1 (default, the measured best) SWIGLU at
+                          // 96- and 128-token tiles, where one CTA per SM leaves the most idle (SPEC_TUNE sk=)
   float rescale_slack = 8.f;  // attention: running-max slack in log2 units (p <= 2^slack)
   int attn_clusters[kAttnMaxChunks + 1] = {};  // co-resident clusters of n chunk CTAs
   bool attn_dsmem = true;     // merge chunk partials through distributed shared memory when they fit a cluster
@@ -414,7 +415,10 @@ GemmPlan plan_gemm(const spec_handle* h, int rows_per_tile, int n_out, int K, in
   // Stream-K for the phases without split-K when whole tiles would leave CTAs
   // idle in the last round (more than 2 % of the CTA-rounds): every resident
   // CTA then streams the same number of weight k-blocks.
-  if (h->streamk && (epi == GEMM_EPI_SWIGLU || epi == GEMM_EPI_ARGMAX || epi == GEMM_EPI_TOPK) && p.splits == 1 &&
+  const bool sk_epi = h->streamk == 1   ? (epi == GEMM_EPI_SWIGLU || epi == GEMM_EPI_ARGMAX || epi == GEMM_EPI_TOPK)
+                      : h->streamk == 2 ? epi == GEMM_EPI_SWIGLU
+                                        : h->streamk < 0 && epi == GEMM_EPI_SWIGLU && p.bn > 64;
+  if (sk_epi && p.splits == 1 &&
       resident <= kSkMaxCtas && base <= kCountersPerPhase && (long long)base * KB >= 2LL * resident &&
       (size_t)resident * 128 * p.bn * 4 <= h->lay.partial_bytes) {
     const long long rounds = ceil_div(base, resident);
@@ -1336,7 +1340,7 @@ int spec_init(const spec_config* cfg, const spec_weights* w, void* kv_cache, siz
     if (const char* q = strstr(t, "bn64max=")) if (sscanf(q + 8, "%d", &v) == 1 && v >= 64) h->bn64_max = v;
     if (const char* q = strstr(t, "bn96=")) if (sscanf(q + 5, "%d", &v) == 1) h->bn96 = v != 0;
     if (const char* q = strstr(t, "per_sm=")) if (sscanf(q + 7, "%d", &v) == 1 && v >= 0) h->resident_cap = v;
-    if (const char* q = strstr(t, "sk=")) if (sscanf(q + 3, "%d", &v) == 1) h->streamk = v != 0;
+    if (const char* q = strstr(t, "sk=")) if (sscanf(q + 3, "%d", &v) == 1 && v >= -1 && v <= 2) h->streamk = v;
     float fv = 0.f;
     if (const char* q = strstr(t, "rescale=")) if (sscanf(q + 8, "%f", &fv) == 1 && fv >= 0.f && fv <= 15.f) h->rescale_slack = fv;
   }
