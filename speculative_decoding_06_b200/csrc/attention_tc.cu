@@ -19,11 +19,13 @@
 // 32-layer model of the 8B shape; P's rounding made a node's logits depend on
 // where key chunks start.)
 //
-//   warp 16 (one thread): TMA loads of Q (hi, lo) and of 64-key blocks of K,
-//                        K_lo and V (two stages each; the later blocks of the
-//                        chunk are brought into L2 up front), the S MMAs of a
-//                        block into one of two TMEM buffers, O += P_j V_j into a
-//                        128-column buffer (V read MN-major);
+//   warp 17 (one thread): TMA loads of Q (hi, lo) and of 64-key blocks of K,
+//                        K_lo and V (two K stages and two V stages, each
+//                        refilled once its MMAs are done; the later blocks of
+//                        the chunk are brought into L2 up front);
+//   warp 16 (one thread): the S MMAs of a block into one of two TMEM buffers and
+//                        O += P_j V_j into a 128-column TMEM buffer (P_j read
+//                        from tensor memory, V from shared memory MN-major);
 //   warps 0-15:          four threads per query row (warps w, w + 4, w + 8 and
 //                        w + 12 share the row's TMEM lane; each takes 16 of the
 //                        block's keys and 32 output dims): read S_j, apply the
@@ -31,8 +33,8 @@
 //                        moves only when a block's max exceeds it by more than
 //                        the slack, 8 in log2 units by default: every p stays
 //                        <= 2^8 and O is rescaled rarely), write P_j (hi and lo)
-//                        into shared memory as the next MMAs' A operands, and at
-//                        the end normalise O.
+//                        into one of two P buffers in tensor memory, and at the
+//                        end normalise O.
 //
 // A sequence's keys are cut into chunks so that short-prefix, small-batch steps
 // still occupy the GPU; the chunk CTAs of one (sequence, kv head, row tile)
