@@ -56,10 +56,9 @@ struct SmemLayout {
   static constexpr uint32_t b_off = a_off + STAGES * kABytes;
   static constexpr uint32_t epi_off = b_off + STAGES * kBBytes;
   // per-token norm scale r[BN], then the largest of: SWIGLU gate and up values
-  // [128][17] (padded rows: conflict-free), ARGMAX per-warp results [4][BN], RESID
-  // per-warp sums of squares [4][BN]
-  static constexpr uint32_t epi_extra =
-      cmax(cmax(128 * 17 * 4, 16 * 129 * 4), cmax(4 * BN * (uint32_t)sizeof(Top2), 4 * BN * 4));
+  // [128][17] (padded rows: conflict-free), the ARGMAX and TOPK token-major staging
+  // [16][136] / [16][129], RESID per-warp sums of squares [4][BN]
+  static constexpr uint32_t epi_extra = cmax(cmax(128 * 17 * 4, 16 * 136 * 4), 4 * BN * 4);
   static constexpr uint32_t epi_bytes = BN * 4 + epi_extra;
   static constexpr uint32_t bar_off = (epi_off + epi_bytes + 7) & ~7u;
   static constexpr uint32_t n_bars = 2 * STAGES + 4;
@@ -76,11 +75,10 @@ __device__ __forceinline__ void named_sync(int id, int n) {
 }
 
 // Units of a phase done by CTA b: with split-K one unit (b / S, b % S) if
-// b < tiles * S; otherwise tiles b, b + grid, ...
+// b < tiles * S; otherwise tiles b, b + grid, ... (WorkIter walks them)
 struct UnitIter {
   int tiles, S, grid, b;
   __device__ int first() const { return S > 1 ? (b < tiles * S ? b / S : tiles) : b; }
-  __device__ int next(int ut) const { return S > 1 ? tiles : ut + grid; }
   __device__ int split() const { return S > 1 ? b % S : 0; }
 };
 
@@ -924,9 +922,16 @@ __global__ void __launch_bounds__(kThreads, BN == 64 ? 2 : 1)
           tc_fence_before();
           mbar_arrive(&tempty[acc]);
         } else {  // GEMM_EPI_ARGMAX
-          Top2* wres = reinterpret_cast<Top2*>(epx);  // [4][BN]
+          // Per 16 tokens: the tile's 128 x 16 scores (logits, or logit / T + Gumbel
+          // noise) go to shared memory token-major; then eight threads per token take
+          // rows p, p + 8, ... (p = 0..7) each, keep their (best, index, runner-up),
+          // and meet in three shuffle rounds.  (Rows 136 floats apart: the reads of a
+          // warp's 4 tokens x 8 threads hit 32 different banks.)
+          float* sT = reinterpret_cast<float*>(epx);  // [16][136]
           const int o = to * kTileO + row_in_tile;
           const bool row_ok = o < args.n_out;
+          const int tok = ep_tid >> 3;  // this thread's token of the 16
+          const int part = ep_tid & 7;
 #pragma unroll 1
           for (int c0 = 0; c0 < BN; c0 += 16) {
             float v[16], vl[16];
@@ -941,24 +946,40 @@ __global__ void __launch_bounds__(kThreads, BN == 64 ? 2 : 1)
               if (args.inv_temp > 0.f && row_ok && t < args.M)  // temperature sampling: Gumbel-max
                 v[i] = fmaf(v[i], args.inv_temp,
                             gumbel_noise(args.seed_lo, args.seed_hi, args.row_sid[t], args.row_pos[t], o));
-              Top2 x;
-              x.v1 = row_ok ? v[i] : -INFINITY;
-              x.i1 = row_ok ? o : 0x7fffffff;
-              x.v2 = -INFINITY;
-              x = warp_top2(x);
-              if (lane == i) wres[quarter * BN + c0 + i] = x;
+              sT[i * 136 + row_in_tile] = row_ok ? v[i] : -INFINITY;
             }
+            named_sync(1, 128);
+            Top2 x;
+            x.v1 = -INFINITY;
+            x.i1 = 0x7fffffff;
+            x.v2 = -INFINITY;
+#pragma unroll
+            for (int u = 0; u < 16; ++u) {
+              const int r = part + 8 * u;
+              const float val = sT[tok * 136 + r];
+              const int idx = to * kTileO + r < args.n_out ? to * kTileO + r : 0x7fffffff;
+              if (val > x.v1 || (val == x.v1 && idx < x.i1)) {
+                x.v2 = x.v1;
+                x.v1 = val;
+                x.i1 = idx;
+              } else {
+                x.v2 = fmaxf(x.v2, val);
+              }
+            }
+#pragma unroll
+            for (int off = 4; off > 0; off >>= 1) {
+              Top2 y;
+              y.v1 = __shfl_xor_sync(0xffffffffu, x.v1, off);
+              y.i1 = __shfl_xor_sync(0xffffffffu, x.i1, off);
+              y.v2 = __shfl_xor_sync(0xffffffffu, x.v2, off);
+              x = top2_merge(x, y);
+            }
+            const int t = t_base + c0 + tok;
+            if (part == 0 && t < args.M) args.top_part[(size_t)to * args.top_ld + t] = x;
+            named_sync(1, 128);  // the staging area is free for the next 16 tokens
           }
           tc_fence_before();
           mbar_arrive(&tempty[acc]);
-          named_sync(1, 128);
-          for (int c = ep_tid; c < BN; c += 128) {
-            Top2 r = wres[c];
-#pragma unroll
-            for (int q = 1; q < 4; ++q) r = top2_merge(r, wres[q * BN + c]);
-            const int t = t_base + c;
-            if (t < args.M) args.top_part[(size_t)to * args.top_ld + t] = r;
-          }
         }
         // unit done (a phase's arrival counters serve it alone and are zeroed with
         // the step, so nothing is reset here)
