@@ -119,5 +119,17 @@ def test_new_entry_points_reject_bad_arguments_without_gpu():
     assert S.spec_wait_selftest(ctypes.c_void_p(18), 1000, ctypes.byref(i32)) == S.SPEC_ERR_ARG  # misaligned
 
 
+def test_draft_head_workspace_holds_no_logits():
+    """The draft head's top-10 is selected inside the LM-head GEMM: at batch 16 x 64 nodes the
+    workspace holds per-tile candidates (24 slots x 1002 tiles per row), not [1024][128256]
+    fp32 logits (525 MB)."""
+    c = cfg_of(synth.LLAMA8B, max_batch=16, max_seq=2112, max_nodes=64)
+    base = S.spec_workspace_bytes(ctypes.byref(c))
+    c.draft_head = 1
+    with_draft = S.spec_workspace_bytes(ctypes.byref(c))
+    assert 0 < base < with_draft
+    assert with_draft - base < 1024 * 128256 * 4
+
+
 def test_sampling_setter_without_handle():
     assert S.spec_set_sampling(None, 0.7, 1) == S.SPEC_ERR_ARG
