@@ -186,14 +186,8 @@ cudaError_t launch_embed_meta(int dtype, const StepView& sv, const void* embed, 
 // bf16 rows [rows][cols] -> split bf16 operand [2 x rows][cols] (lo parts zero)
 cudaError_t launch_split_rows(const __nv_bfloat16* src, int rows, int cols, __nv_bfloat16* dst, cudaStream_t s,
                               bool pdl);
-// per row: the k largest of V fp32 values, ordered by (value desc, index asc)
+// the longest top-k list of the draft head (value desc, index asc)
 constexpr int kTopKMax = 16;
-// top-k per row (value desc, index asc), k in {4, 8, 10, 16}; with lse != NULL also
-// the row's log-sum-exp (natural log)
-// (id_map: token id of each of the V columns; the indices written are id_map[column])
-cudaError_t launch_topk_rows(int M, int V, const float* logits, size_t ld, int k, int32_t* idx, float* val,
-                             float* lse, cudaStream_t s, bool pdl, const int32_t* id_map = nullptr);
-
 // top-k per row (k in {4, 8, 10, 16}) from the LM head's TOPK candidates: cand_v / cand_i
 // [M][tiles][kCandSlots] (a superset of each tile's k best), cand_lse [M][tiles] (max, sum of
 // exp(l - max));

@@ -535,209 +535,6 @@ __device__ __forceinline__ void warp_merge_topk(const float (&lv)[K], const int 
 }
 }  // namespace
 
-template <int K, bool LSE, int U>
-__global__ void __launch_bounds__(256) topk_rows_kernel(int V, const float* __restrict__ logits, size_t ld,
-                                                       int32_t* __restrict__ out_i, float* __restrict__ out_v,
-                                                       float* __restrict__ out_lse,
-                                                       const int32_t* __restrict__ id_map) {
-  __shared__ float wv[8][K];
-  __shared__ int wi[8][K];
-  pdl_wait();
-  pdl_launch_dependents();
-  const int r = blockIdx.x;
-  const float* row = logits + (size_t)r * ld;
-  float lv[K];
-  int li[K];
-#pragma unroll
-  for (int j = 0; j < K; ++j) {
-    lv[j] = -INFINITY;
-    li[j] = 0x7fffffff;
-  }
-  // Pass 1: a lower bound for the row's K-th value.  Each thread takes the
-  // maximum of 64 of the row's values (disjoint sets, strided); the K-th
-  // largest of these 256 maxima is reached by K distinct entries, so the row's
-  // K-th value is at least that.
-  const int warp = threadIdx.x >> 5;
-  const int lane = threadIdx.x & 31;
-  float thr = -INFINITY;
-  {
-    float m = -INFINITY;
-    int mi = 0x7fffffff;
-#pragma unroll 8
-    for (int j = 0; j < 64; ++j) {
-      const int c = threadIdx.x + j * blockDim.x;
-      if (c < V) {
-        const float x = __ldcs(row + c);
-        if (topk_better(x, c, m, mi)) {
-          m = x;
-          mi = c;
-        }
-      }
-    }
-    float sv[K];
-    int si[K];
-#pragma unroll
-    for (int j = 0; j < K; ++j) {
-      sv[j] = j == 0 ? m : -INFINITY;
-      si[j] = j == 0 ? mi : 0x7fffffff;
-    }
-    warp_merge_topk<K>(sv, si, wv[warp], wi[warp]);
-    __syncthreads();
-    if (warp == 0) {
-      float mv[K];
-      int mj[K];
-#pragma unroll
-      for (int j = 0; j < K; ++j) {
-        mv[j] = lane < 8 ? wv[lane][j] : -INFINITY;
-        mj[j] = lane < 8 ? wi[lane][j] : 0x7fffffff;
-      }
-      __syncwarp();
-      warp_merge_topk<K>(mv, mj, wv[0], wi[0]);
-    }
-    __syncthreads();
-    thr = wv[0][K - 1];  // -inf when the row has fewer than K entries
-    __syncthreads();
-  }
-  // Pass 2: the whole row; only values >= thr are offered to the sorted list
-  auto offer = [&](float x, int c) {
-    if (!topk_better(x, c, lv[K - 1], li[K - 1])) return;
-    float cv = x;
-    int ci = c;
-#pragma unroll
-    for (int j = 0; j < K; ++j) {
-      if (topk_better(cv, ci, lv[j], li[j])) {
-        const float tv = lv[j];
-        const int ti = li[j];
-        lv[j] = cv;
-        li[j] = ci;
-        cv = tv;
-        ci = ti;
-      }
-    }
-  };
-  const bool vec = (ld % 4 == 0) && ((reinterpret_cast<uintptr_t>(logits) & 15u) == 0);
-  const int V4 = vec ? V / 4 : 0;
-  const float4* row4 = reinterpret_cast<const float4*>(row);
-  // optional log-sum-exp: a running (max, sum of 2^((x - max) log2 e)) per thread
-  constexpr float kLog2e = 1.4426950408889634f;
-  float lm = -INFINITY, ls = 0.f;
-  auto lse_add = [&](float mx, float e0, float e1, float e2, float e3) {
-    if (mx > lm) {
-      ls = (lm == -INFINITY ? 0.f : ls * fast_exp2((lm - mx) * kLog2e));
-      lm = mx;
-    }
-    ls += fast_exp2((e0 - lm) * kLog2e) + fast_exp2((e1 - lm) * kLog2e) + fast_exp2((e2 - lm) * kLog2e) +
-          fast_exp2((e3 - lm) * kLog2e);
-  };
-  constexpr int kU = U;  // float4 loads in flight per thread (more when few rows leave SMs idle)
-  for (int g0 = threadIdx.x; g0 < V4; g0 += kU * blockDim.x) {
-    float4 x[kU];
-#pragma unroll
-    for (int u = 0; u < kU; ++u) {
-      const int g = g0 + u * blockDim.x;
-      x[u] = g < V4 ? __ldcs(row4 + g) : make_float4(-INFINITY, -INFINITY, -INFINITY, -INFINITY);
-    }
-#pragma unroll
-    for (int u = 0; u < kU; ++u) {
-      const float m = fmaxf(fmaxf(x[u].x, x[u].y), fmaxf(x[u].z, x[u].w));
-      if (LSE && m > -INFINITY) lse_add(m, x[u].x, x[u].y, x[u].z, x[u].w);
-      if (m >= thr) {
-        const int c = 4 * (g0 + u * blockDim.x);
-        if (x[u].x >= thr) offer(x[u].x, c);
-        if (x[u].y >= thr) offer(x[u].y, c + 1);
-        if (x[u].z >= thr) offer(x[u].z, c + 2);
-        if (x[u].w >= thr) offer(x[u].w, c + 3);
-      }
-    }
-  }
-  for (int c = 4 * V4 + threadIdx.x; c < V; c += blockDim.x) {
-    const float x = __ldcs(row + c);
-    if (LSE) lse_add(x, x, -INFINITY, -INFINITY, -INFINITY);
-    if (x >= thr) offer(x, c);
-  }
-  if (LSE) {
-    // combine the threads' (max, sum) pairs: warp shuffles, then the 8 warps
-    __shared__ float lse_m[8], lse_s[8];
-    for (int o = 16; o > 0; o >>= 1) {
-      const float m2 = __shfl_xor_sync(0xffffffffu, lm, o);
-      const float s2 = __shfl_xor_sync(0xffffffffu, ls, o);
-      const float mm = fmaxf(lm, m2);
-      if (mm > -INFINITY) {
-        ls = (lm == -INFINITY ? 0.f : ls * fast_exp2((lm - mm) * kLog2e)) +
-             (m2 == -INFINITY ? 0.f : s2 * fast_exp2((m2 - mm) * kLog2e));
-        lm = mm;
-      }
-    }
-    if (lane == 0) {
-      lse_m[warp] = lm;
-      lse_s[warp] = ls;
-    }
-    __syncthreads();
-    if (threadIdx.x == 0) {
-      float M0 = -INFINITY;
-      for (int w = 0; w < 8; ++w) M0 = fmaxf(M0, lse_m[w]);
-      float S0 = 0.f;
-      for (int w = 0; w < 8; ++w)
-        if (lse_m[w] > -INFINITY) S0 += lse_s[w] * fast_exp2((lse_m[w] - M0) * kLog2e);
-      out_lse[r] = M0 + __logf(S0);
-    }
-  }
-  warp_merge_topk<K>(lv, li, wv[warp], wi[warp]);
-  __syncthreads();
-  if (warp == 0) {
-    float mv[K];
-    int mi[K];
-#pragma unroll
-    for (int j = 0; j < K; ++j) {
-      mv[j] = lane < 8 ? wv[lane][j] : -INFINITY;
-      mi[j] = lane < 8 ? wi[lane][j] : 0x7fffffff;
-    }
-    __syncwarp();
-    warp_merge_topk<K>(mv, mi, wv[0], wi[0]);
-    __syncwarp();
-    if (lane < K) {
-      out_v[(size_t)r * K + lane] = wv[0][lane];
-      out_i[(size_t)r * K + lane] = id_map ? id_map[wi[0][lane]] : wi[0][lane];
-    }
-  }
-}
-
-cudaError_t launch_topk_rows(int M, int V, const float* logits, size_t ld, int k, int32_t* idx, float* val,
-                             float* lse, cudaStream_t s, bool pdl, const int32_t* id_map) {
-  if (k < 1 || k > kTopKMax || k > V) return cudaErrorInvalidValue;
-  cudaLaunchAttribute attr[1];
-  cudaLaunchConfig_t cfg = make_cfg(dim3(M), dim3(256), 0, s, pdl, attr);
-  // few rows leave SMs idle: each CTA then keeps more of its row in flight
-  const bool few = M <= 256;
-  switch (k) {  // the list length is a compile-time constant of the kernel
-    case 10:
-      if (few)
-        return lse ? cudaLaunchKernelEx(&cfg, topk_rows_kernel<10, true, 4>, V, logits, ld, idx, val, lse, id_map)
-                   : cudaLaunchKernelEx(&cfg, topk_rows_kernel<10, false, 4>, V, logits, ld, idx, val, lse, id_map);
-      return lse ? cudaLaunchKernelEx(&cfg, topk_rows_kernel<10, true, 2>, V, logits, ld, idx, val, lse, id_map)
-                 : cudaLaunchKernelEx(&cfg, topk_rows_kernel<10, false, 2>, V, logits, ld, idx, val, lse, id_map);
-    case 16:
-      if (few)
-        return lse ? cudaLaunchKernelEx(&cfg, topk_rows_kernel<16, true, 4>, V, logits, ld, idx, val, lse, id_map)
-                   : cudaLaunchKernelEx(&cfg, topk_rows_kernel<16, false, 4>, V, logits, ld, idx, val, lse, id_map);
-      return lse ? cudaLaunchKernelEx(&cfg, topk_rows_kernel<16, true, 2>, V, logits, ld, idx, val, lse, id_map)
-                 : cudaLaunchKernelEx(&cfg, topk_rows_kernel<16, false, 2>, V, logits, ld, idx, val, lse, id_map);
-    case 8:
-      if (few)
-        return lse ? cudaLaunchKernelEx(&cfg, topk_rows_kernel<8, true, 4>, V, logits, ld, idx, val, lse, id_map)
-                   : cudaLaunchKernelEx(&cfg, topk_rows_kernel<8, false, 4>, V, logits, ld, idx, val, lse, id_map);
-      return lse ? cudaLaunchKernelEx(&cfg, topk_rows_kernel<8, true, 2>, V, logits, ld, idx, val, lse, id_map)
-                 : cudaLaunchKernelEx(&cfg, topk_rows_kernel<8, false, 2>, V, logits, ld, idx, val, lse, id_map);
-    case 4:
-      if (few)
-        return lse ? cudaLaunchKernelEx(&cfg, topk_rows_kernel<4, true, 4>, V, logits, ld, idx, val, lse, id_map)
-                   : cudaLaunchKernelEx(&cfg, topk_rows_kernel<4, false, 4>, V, logits, ld, idx, val, lse, id_map);
-      return lse ? cudaLaunchKernelEx(&cfg, topk_rows_kernel<4, true, 2>, V, logits, ld, idx, val, lse, id_map)
-                 : cudaLaunchKernelEx(&cfg, topk_rows_kernel<4, false, 2>, V, logits, ld, idx, val, lse, id_map);
-    default: return cudaErrorInvalidValue;
-  }
-}
-
 // Top-k of a row from the per-tile candidates of the LM head's TOPK epilogue: each
 // 128-row vocabulary tile gave kCandSlots candidates holding its k best (in no
 // particular order; unused slots -inf) and its (max, sum of exp(l - max)).  The
