@@ -447,26 +447,31 @@ __global__ void __launch_bounds__(kThreads, 1) attn_tc_kernel(const __grid_const
       if (ok) ok = mbar_wait(&bar[B_SFULL + st], (j >> 1) & 1, err, abort_flag);
       ok = __all_sync(0xffffffffu, ok);
       if (j == 0) stamp(a.trace, 3);
-      // visibility bits of this thread's keys (all ones when the whole block is
-      // prefix keys of this chunk)
-      const bool full = row_ok && key0 + kKeys <= min(P, c1);
-      const uint32_t w =
-          full ? kmask : (row_ok ? visible_word(key0 + kKeysPT * qtr, P, c1, anc0, anc1) & kmask : 0u);
-      // pass 1: this quarter's row max (raw scores; the scale is positive), then the
-      // row's; the scores stay in registers for pass 2
+      // a block of prefix keys of this chunk is visible to every row of the warp
+      const bool wfull = __all_sync(0xffffffffu, row_ok && key0 + kKeys <= min(P, c1));
+      // pass 1: this thread's scores (hidden keys set to -inf, so that pass 2 needs
+      // no mask) and their max (raw scores; the scale is positive), then the row's
       float x[kKeysPT];
-      float mx4[4] = {-INFINITY, -INFINITY, -INFINITY, -INFINITY};
       if (ok) {
         tc_fence_after();
         float xl[kKeysPT];
         tmem_ld16x2(ts, ts + kKeys, x, xl);
 #pragma unroll
-        for (int c = 0; c < kKeysPT; ++c) {
-          x[c] += xl[c];
-          mx4[c & 3] = fmaxf(mx4[c & 3], ((w >> c) & 1u) ? x[c] : -INFINITY);
+        for (int c = 0; c < kKeysPT; c += 2)
+          f2_unpack(f2_add(f2_pack(x[c], x[c + 1]), f2_pack(xl[c], xl[c + 1])), x[c], x[c + 1]);
+        if (!wfull) {
+          const uint32_t w = row_ok ? visible_word(key0 + kKeysPT * qtr, P, c1, anc0, anc1) & kmask : 0u;
+#pragma unroll
+          for (int c = 0; c < kKeysPT; ++c) x[c] = ((w >> c) & 1u) ? x[c] : -INFINITY;
         }
+      } else {
+#pragma unroll
+        for (int c = 0; c < kKeysPT; ++c) x[c] = -INFINITY;
       }
-      xmax[(st * kPerRow + qtr) * 128 + r] = fmaxf(fmaxf(mx4[0], mx4[1]), fmaxf(mx4[2], mx4[3]));
+      static_assert(kKeysPT == 16, "max tree over 16 scores");
+      xmax[(st * kPerRow + qtr) * 128 + r] =
+          fmaxf(fmax3(fmax3(x[0], x[1], x[2]), fmax3(x[3], x[4], x[5]), fmax3(x[6], x[7], x[8])),
+                fmax3(fmax3(x[9], x[10], x[11]), fmax3(x[12], x[13], x[14]), x[15]));
       named_sync_quad(warp & 3);  // the four warps that share these rows
       float mraw = xmax[(st * kPerRow) * 128 + r];
 #pragma unroll
@@ -479,25 +484,32 @@ __global__ void __launch_bounds__(kThreads, 1) attn_tc_kernel(const __grid_const
         m = mblk;
       }
       const float nm = (m == -INFINITY) ? 0.f : -m;
-      // pass 2: P = 2^(s - m) as two fp16 parts, in registers until the P buffer is free
-      float ls4[4] = {0.f, 0.f, 0.f, 0.f};
+      // pass 2: P = 2^(s - m) as two fp16 parts, in registers until the P buffer is
+      // free (2^-inf = 0 for hidden keys; the scale and the sums go two keys at a time)
+      const uint64_t sc2 = f2_pack(sl2, sl2), nm2 = f2_pack(nm, nm);
+      uint64_t lsa = f2_pack(0.f, 0.f), lsb = lsa;
       uint32_t pk[kKeysPT / 2], pl[kKeysPT / 2];
 #pragma unroll
       for (int c = 0; c < kKeysPT / 2; ++c) {
-        const float s0 = ((w >> (2 * c)) & 1u) ? x[2 * c] : -INFINITY;
-        const float s1 = ((w >> (2 * c + 1)) & 1u) ? x[2 * c + 1] : -INFINITY;
-        const float p0 = ok ? fast_exp2(fmaf(s0, sl2, nm)) : 0.f;
-        const float p1 = ok ? fast_exp2(fmaf(s1, sl2, nm)) : 0.f;
-        ls4[c & 3] += p0 + p1;
+        float y0, y1;
+        f2_unpack(f2_fma(f2_pack(x[2 * c], x[2 * c + 1]), sc2, nm2), y0, y1);
+        const float p0 = fast_exp2(y0), p1 = fast_exp2(y1);
+        const uint64_t p2 = f2_pack(p0, p1);
+        if (c & 1) lsb = f2_add(lsb, p2);
+        else lsa = f2_add(lsa, p2);
         // hi: p truncated to fp16's 11 significant bits (exact in fp16 for p >= 2^-14,
         // so one conversion per pair instead of a round trip), lo: the exact remainder
         const float t0 = __uint_as_float(__float_as_uint(p0) & 0xFFFFE000u);
         const float t1 = __uint_as_float(__float_as_uint(p1) & 0xFFFFE000u);
+        float d0, d1;
+        f2_unpack(f2_sub(p2, f2_pack(t0, t1)), d0, d1);
         const __half2 h2 = __floats2half2_rn(t0, t1);
-        const __half2 l2 = __floats2half2_rn(p0 - t0, p1 - t1);
+        const __half2 l2 = __floats2half2_rn(d0, d1);
         pk[c] = *reinterpret_cast<const uint32_t*>(&h2);
         pl[c] = *reinterpret_cast<const uint32_t*>(&l2);
       }
+      float la0, la1;
+      f2_unpack(f2_add(lsa, lsb), la0, la1);
       // a larger running max rescales O: P.V of block j - 1 must have finished
       if (j >= 1 && ok && __any_sync(0xffffffffu, corr != 1.f)) {
         ok = __all_sync(0xffffffffu,
@@ -536,7 +548,7 @@ __global__ void __launch_bounds__(kThreads, 1) attn_tc_kernel(const __grid_const
           mbar_arrive(&bar[B_PFULL + (j & 1)]);
         }
       }
-      l = l * corr + ((ls4[0] + ls4[1]) + (ls4[2] + ls4[3]));
+      l = l * corr + (la0 + la1);
     }
     if (!ok) *abort_flag = 1;
     // ---- normalised output of this chunk, staged in shared memory (the K/V
