@@ -487,6 +487,7 @@ __global__ void __launch_bounds__(kThreads, 1) attn_tc_kernel(const __grid_const
       // pass 2: P = 2^(s - m) as two fp16 parts, in registers until the P buffer is
       // free (2^-inf = 0 for hidden keys; the scale and the sums go two keys at a time)
       const uint64_t sc2 = f2_pack(sl2, sl2), nm2 = f2_pack(nm, nm);
+      const uint64_t dn2 = f2_pack(0x1p-112f, 0x1p-112f), up2 = f2_pack(0x1p112f, 0x1p112f);
       uint64_t lsa = f2_pack(0.f, 0.f), lsb = lsa;
       uint32_t pk[kKeysPT / 2], pl[kKeysPT / 2];
 #pragma unroll
@@ -497,15 +498,18 @@ __global__ void __launch_bounds__(kThreads, 1) attn_tc_kernel(const __grid_const
         const uint64_t p2 = f2_pack(p0, p1);
         if (c & 1) lsb = f2_add(lsb, p2);
         else lsa = f2_add(lsa, p2);
-        // hi: p truncated to fp16's 11 significant bits (exact in fp16 for p >= 2^-14,
-        // so one conversion per pair instead of a round trip), lo: the exact remainder
-        const float t0 = __uint_as_float(__float_as_uint(p0) & 0xFFFFE000u);
-        const float t1 = __uint_as_float(__float_as_uint(p1) & 0xFFFFE000u);
+        // hi: p truncated to fp16's 11 significant bits, formed without a conversion:
+        // p * 2^-112 carries fp16's exponent bias (127 - 112 = 15), so its bits 13-27
+        // are the fp16 bits (p < 2^-14, below fp16's normal range, flushes to zero and
+        // goes wholly into lo); lo: the exact remainder p - hi, rounded to fp16
+        uint32_t u0, u1;
+        u2_unpack(f2_mul_ftz(p2, dn2), u0, u1);
+        u0 &= 0xFFFFE000u;
+        u1 &= 0xFFFFE000u;
+        pk[c] = (u0 >> 13) | (u1 << 3);
         float d0, d1;
-        f2_unpack(f2_sub(p2, f2_pack(t0, t1)), d0, d1);
-        const __half2 h2 = __floats2half2_rn(t0, t1);
+        f2_unpack(f2_sub(p2, f2_mul(u2_pack(u0, u1), up2)), d0, d1);
         const __half2 l2 = __floats2half2_rn(d0, d1);
-        pk[c] = *reinterpret_cast<const uint32_t*>(&h2);
         pl[c] = *reinterpret_cast<const uint32_t*>(&l2);
       }
       float la0, la1;
