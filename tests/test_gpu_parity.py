@@ -256,3 +256,21 @@ def test_bf16_multiblock_attention(tune):
         trees.append((toks, sh.parents))
         seqs.append(seq)
     assert _check_batch(eng, om, [0, 1], seqs, trees) == 2
+
+
+@pytest.mark.parametrize("tune", ["chunks=4,dsmem=0", "chunks=4"])
+def test_bf16_chunk_merge_mixed_lengths(tune):
+    """A batch whose sequences split into different chunk counts: prefix 90 + 61 nodes fits one key chunk (its
+    rows are written by its CTA directly), prefix 700 + 61 takes four whose partials are merged through global
+    memory (dsmem=0) or a cluster; the longer sequence comes second in the batch and first in the attention's
+    work order."""
+    eng, om = _engine_tuned(synth.MINI_BF16, tune, max_batch=2, max_seq=1024, max_nodes=64)
+    assert ("(global merge)" if "dsmem=0" in tune else "(cluster merge)") in eng.info(2, 61, 700)
+    seqs, trees = [], []
+    for i, P in enumerate((90, 700)):
+        sh = synth.tree_from_widths(synth.TREE60_WIDTHS, stream=7 + i)
+        prefix, seq, toks = decided_case(om, P, sh, 0.8, stream0=(601, 501)[i])
+        assert eng.prefill(i, prefix) == seq.pending
+        trees.append((toks, sh.parents))
+        seqs.append(seq)
+    assert _check_batch(eng, om, [0, 1], seqs, trees) == 2
