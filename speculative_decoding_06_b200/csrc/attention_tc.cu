@@ -614,8 +614,7 @@ __global__ void __launch_bounds__(kThreads, 1) attn_tc_kernel(const __grid_const
       if (tid == 0) {
         bool met = false;
         if (!*abort_flag) {
-          __threadfence();  // the barrier orders every thread's partial stores before it
-          atomicAdd(ctr, 1);
+          red_release_add_gpu(ctr, 1);  // the barrier orders every thread's partial stores before it
           met = spin_until_geq(ctr, nc_b, err);
         }
         *merge_ok = met ? 1 : 0;

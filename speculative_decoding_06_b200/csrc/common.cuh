@@ -245,6 +245,12 @@ __device__ __forceinline__ int ld_relaxed_gpu(const int* p) {
   return v;
 }
 __device__ __forceinline__ void fence_acq_rel_gpu() { asm volatile("fence.acq_rel.gpu;" ::: "memory"); }
+// Count an arrival with release semantics and no returned value: writes ordered
+// before it (this thread's, and the CTA's through a preceding barrier) are
+// visible at gpu scope to a thread that acquires the count.
+__device__ __forceinline__ void red_release_add_gpu(int* p, int v) {
+  asm volatile("red.release.gpu.global.add.s32 [%0], %1;" ::"l"(p), "r"(v) : "memory");
+}
 __device__ __forceinline__ void st_release_gpu(int* p, int v) {
   asm volatile("st.release.gpu.global.b32 [%0], %1;" ::"l"(p), "r"(v) : "memory");
 }

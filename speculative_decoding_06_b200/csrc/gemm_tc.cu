@@ -489,10 +489,7 @@ __global__ void __launch_bounds__(kThreads, BN == 64 ? 2 : 1)
           tc_fence_before();
           mbar_arrive(&tempty[acc]);
           named_sync(2, 128);  // every thread's stores precede the arrival
-          if (ep_tid == 0) {
-            __threadfence();
-            atomicAdd(args.counters + ut, 1);
-          }
+          if (ep_tid == 0) red_release_add_gpu(args.counters + ut, 1);
           first_unit = false;
           continue;
         }
@@ -553,8 +550,7 @@ __global__ void __launch_bounds__(kThreads, BN == 64 ? 2 : 1)
           named_sync(2, 128);
           if (S > 1) {
             if (ep_tid == 0) {
-              __threadfence();  // the barrier orders every thread's partial stores before it
-              atomicAdd(ctr, 1);
+              red_release_add_gpu(ctr, 1);  // the barrier orders every thread's partial stores before it
               *ep_ok = spin_until_geq(ctr, S, err) ? 1 : 0;
             }
             named_sync(2, 128);
@@ -993,10 +989,7 @@ __global__ void __launch_bounds__(kThreads, BN == 64 ? 2 : 1)
       if (p + 1 < nph) {
         fence_proxy_async_global();  // later phases read this phase's outputs with TMA
         named_sync(2, 128);
-        if (ep_tid == 0) {
-          __threadfence();
-          atomicAdd(P.phase_bar + p, 1);
-        }
+        if (ep_tid == 0) red_release_add_gpu(P.phase_bar + p, 1);
       }
       if (ep_tid == 0) stamp(P.trace, p, 7);
     }
