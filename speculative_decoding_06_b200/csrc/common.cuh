@@ -408,6 +408,15 @@ __device__ __forceinline__ void tmem_st32_async(uint32_t taddr, const uint32_t* 
                ::"r"(taddr), "r"(r[0]), "r"(r[1]), "r"(r[2]), "r"(r[3]), "r"(r[4]), "r"(r[5]), "r"(r[6]), "r"(r[7]), "r"(r[8]), "r"(r[9]), "r"(r[10]), "r"(r[11]), "r"(r[12]), "r"(r[13]), "r"(r[14]), "r"(r[15]), "r"(r[16]), "r"(r[17]), "r"(r[18]), "r"(r[19]), "r"(r[20]), "r"(r[21]), "r"(r[22]), "r"(r[23]), "r"(r[24]), "r"(r[25]), "r"(r[26]), "r"(r[27]), "r"(r[28]), "r"(r[29]), "r"(r[30]), "r"(r[31])
                : "memory");
 }
+// Each thread of the warp writes 16 consecutive 32-bit columns of its own lane.
+__device__ __forceinline__ void tmem_st16_async(uint32_t taddr, const uint32_t* r) {
+  asm volatile(
+      "tcgen05.st.sync.aligned.32x32b.x16.b32 [%0], {%1,%2,%3,%4,%5,%6,%7,%8,%9,%10,%11,%12,%13,%14,%15,%16};" ::"r"(
+          taddr),
+      "r"(r[0]), "r"(r[1]), "r"(r[2]), "r"(r[3]), "r"(r[4]), "r"(r[5]), "r"(r[6]), "r"(r[7]), "r"(r[8]), "r"(r[9]),
+      "r"(r[10]), "r"(r[11]), "r"(r[12]), "r"(r[13]), "r"(r[14]), "r"(r[15])
+      : "memory");
+}
 // Each thread of the warp writes 8 consecutive 32-bit columns of its own lane.
 __device__ __forceinline__ void tmem_st8_async(uint32_t taddr, const uint32_t* r) {
   asm volatile("tcgen05.st.sync.aligned.32x32b.x8.b32 [%0], {%1,%2,%3,%4,%5,%6,%7,%8};" ::"r"(taddr), "r"(r[0]),
@@ -427,12 +436,12 @@ __device__ __forceinline__ void fence_proxy_async_smem() {
 // A bf16 model's GEMM activations are stored as two bf16 parts, hi = bf16(v)
 // and lo = bf16(v - hi), which together carry ~16 mantissa bits; the weights
 // are exact bf16, so W.hi + W.lo reproduces W.v to fp32-accumulation accuracy.
-// Layout: tokens in groups of 32; group g occupies 64 rows, its 32 hi rows
-// followed by its 32 lo rows.  A GEMM tile of BN tokens (BN a multiple of 32:
-// 64, 96, 128) is one contiguous box of 2*BN rows, and in the tile's
-// accumulator token c's hi column is (c / 32) * 64 + c % 32, its lo column 32
+// Layout: tokens in groups of 16; group g occupies 32 rows, its 16 hi rows
+// followed by its 16 lo rows.  A GEMM tile of BN tokens (BN a multiple of 16:
+// 64, 80, 96, 128) is one contiguous box of 2*BN rows, and in the tile's
+// accumulator token c's hi column is (c / 16) * 32 + c % 16, its lo column 16
 // further.
-constexpr int kSplitGroup = 32;
+constexpr int kSplitGroup = 16;
 __host__ __device__ __forceinline__ int split_row(int t, int part) {
   return (t / kSplitGroup) * (2 * kSplitGroup) + part * kSplitGroup + (t % kSplitGroup);
 }

@@ -164,6 +164,30 @@ __device__ __forceinline__ void stamp(uint64_t* trace, int p, int k) {
   if (trace) trace[((size_t)blockIdx.x * kMaxGemmPhases + p) * kGemmTraceMarks + k] = global_ns();
 }
 
+// hi + lo of the accumulator's tokens c0 .. c0 + 31 (c0 % 32 == 0): split groups
+// of 16 tokens (16 hi columns, then 16 lo columns), so the 32 tokens are the 64
+// columns from 2 * c0; `two` is false when only tokens c0 .. c0 + 15 exist (the
+// last chunk of an 80-token tile)
+__device__ __forceinline__ void acc_sums32(uint32_t taddr, int c0, bool two, float* s) {
+  static_assert(kSplitGroup == 16, "accumulator column layout");
+  uint32_t a[32], b[32];
+  tmem_ld32_async(taddr + 2 * c0, a);
+  if (two) {
+    tmem_ld32_async(taddr + 2 * c0 + 32, b);
+  } else {
+#pragma unroll
+    for (int i = 0; i < 32; ++i) b[i] = 0u;
+  }
+  tmem_wait_ld();
+  tmem_reg_fence32(a);
+  tmem_reg_fence32(b);
+#pragma unroll
+  for (int i = 0; i < 16; ++i) {
+    s[i] = __uint_as_float(a[i]) + __uint_as_float(a[16 + i]);
+    s[16 + i] = __uint_as_float(b[i]) + __uint_as_float(b[16 + i]);
+  }
+}
+
 __device__ __forceinline__ bool phase_done(const int* bar, int need) {
   int v;
   asm volatile("ld.acquire.gpu.global.b32 %0, [%1];" : "=r"(v) : "l"(bar) : "memory");
@@ -475,16 +499,12 @@ __global__ void __launch_bounds__(kThreads, BN == 64 ? 2 : 1)
           float* slot = args.part + (size_t)blockIdx.x * kTileO * BN + row_in_tile;
 #pragma unroll 1
           for (int c0 = 0; c0 < BN; c0 += 32) {
-            uint32_t v[32], vl[32];
-            const uint32_t col = (c0 / kSplitGroup) * (2 * kSplitGroup) + (c0 % kSplitGroup);
-            tmem_ld32_async(taddr + col, v);
-            tmem_ld32_async(taddr + col + kSplitGroup, vl);
-            tmem_wait_ld();
-            tmem_reg_fence32(v);
-            tmem_reg_fence32(vl);
+            float v[32];
+            const bool two = c0 + 16 < BN;
+            acc_sums32(taddr, c0, two, v);
 #pragma unroll
             for (int i = 0; i < 32; ++i)
-              __stcg(slot + (size_t)(c0 + i) * kTileO, __uint_as_float(v[i]) + __uint_as_float(vl[i]));
+              if (i < 16 || two) __stcg(slot + (size_t)(c0 + i) * kTileO, v[i]);
           }
           tc_fence_before();
           mbar_arrive(&tempty[acc]);
@@ -506,19 +526,19 @@ __global__ void __launch_bounds__(kThreads, BN == 64 ? 2 : 1)
             break;
           }
 #pragma unroll 1
-          for (int c0 = 0; c0 < BN; c0 += 32) {
-            uint32_t v[32];
-            const uint32_t col = (c0 / kSplitGroup) * (2 * kSplitGroup) + (c0 % kSplitGroup);
-            tmem_ld32_async(taddr + col, v);
-            tmem_wait_ld();
-            tmem_reg_fence32(v);
+          for (int c0 = 0; c0 < BN; c0 += kSplitGroup) {
+            float vf[kSplitGroup];
+            const uint32_t col = (c0 / kSplitGroup) * (2 * kSplitGroup);  // the group's hi columns
+            tmem_ld16(taddr + col, vf);
             for (int c = (int)blockIdx.x + 1; c <= last; ++c) {
               const float* slot = args.part + (size_t)c * kTileO * BN + row_in_tile;
 #pragma unroll
-              for (int i = 0; i < 32; ++i)
-                v[i] = __float_as_uint(__uint_as_float(v[i]) + __ldcg(slot + (size_t)(c0 + i) * kTileO));
+              for (int i = 0; i < kSplitGroup; ++i) vf[i] += __ldcg(slot + (size_t)(c0 + i) * kTileO);
             }
-            tmem_st32_async(taddr + col, v);
+            uint32_t v[kSplitGroup];
+#pragma unroll
+            for (int i = 0; i < kSplitGroup; ++i) v[i] = __float_as_uint(vf[i]);
+            tmem_st16_async(taddr + col, v);
           }
           tmem_wait_st();
         }
@@ -530,15 +550,13 @@ __global__ void __launch_bounds__(kThreads, BN == 64 ? 2 : 1)
 #pragma unroll 1
           for (int c0 = 0; c0 < BN; c0 += 32) {
             // 32 tokens' hi and lo columns in two loads and one wait
-            uint32_t v[32], vl[32];
-            const uint32_t col = (c0 / kSplitGroup) * (2 * kSplitGroup) + (c0 % kSplitGroup);
-            tmem_ld32_async(taddr + col, v);
-            tmem_ld32_async(taddr + col + kSplitGroup, vl);
-            tmem_wait_ld();
+            float v[32];
+            const bool two = c0 + 16 < BN;
+            acc_sums32(taddr, c0, two, v);
 #pragma unroll
             for (int i = 0; i < 32; ++i) {
               const int t = t_base + c0 + i;
-              if (t < args.M) out[(size_t)t * args.n_out] = __uint_as_float(v[i]) + __uint_as_float(vl[i]);
+              if ((i < 16 || two) && t < args.M) out[(size_t)t * args.n_out] = v[i];
             }
           }
           if (first_unit && ep_tid == 0) stamp(P.trace, p, 8);
@@ -1007,8 +1025,9 @@ __global__ void __launch_bounds__(kThreads, BN == 64 ? 2 : 1)
 // host-side launch helpers
 // ---------------------------------------------------------------------------
 
-// BN = 64 tokens: 3 stages of 32 KB (two CTAs per SM); BN = 96: 5 stages of 40 KB and BN = 128:
-// 4 stages of 48 KB (one CTA per SM)
+// BN = 64 tokens: 3 stages of 32 KB (two CTAs per SM); BN = 80: 6 stages of 36 KB, BN = 96: 5
+// stages of 40 KB and BN = 128: 4 stages of 48 KB (one CTA per SM).  96 KB of weight tiles are in
+// flight per SM at 64 and 80 tokens, 80 KB at 96 and 64 KB at 128.
 template <int BN, int STAGES>
 static cudaError_t launch_impl(const GemmMultiLaunch& L_, cudaStream_t stream, bool pdl) {
   using L = SmemLayout<BN, STAGES>;
@@ -1045,19 +1064,24 @@ static cudaError_t launch_impl(const GemmMultiLaunch& L_, cudaStream_t stream, b
 }
 
 uint32_t gemm_tc_smem_bytes(int bn) {
-  return bn == 64 ? SmemLayout<64, 3>::dyn_bytes
-                  : bn == 96 ? SmemLayout<96, 5>::dyn_bytes : SmemLayout<128, 4>::dyn_bytes;
+  return bn == 64   ? SmemLayout<64, 3>::dyn_bytes
+         : bn == 80 ? SmemLayout<80, 6>::dyn_bytes
+         : bn == 96 ? SmemLayout<96, 5>::dyn_bytes
+                    : SmemLayout<128, 4>::dyn_bytes;
 }
 
 const void* gemm_tc_function(int bn) {
-  return bn == 64 ? (const void*)gemm_tc_kernel<64, 3>
-                  : bn == 96 ? (const void*)gemm_tc_kernel<96, 5> : (const void*)gemm_tc_kernel<128, 4>;
+  return bn == 64   ? (const void*)gemm_tc_kernel<64, 3>
+         : bn == 80 ? (const void*)gemm_tc_kernel<80, 6>
+         : bn == 96 ? (const void*)gemm_tc_kernel<96, 5>
+                    : (const void*)gemm_tc_kernel<128, 4>;
 }
 
 cudaError_t gemm_multi_launch(const GemmMultiLaunch& L, cudaStream_t stream, bool pdl) {
   if (L.n_phases < 1 || L.n_phases > kMaxGemmPhases) return cudaErrorInvalidValue;
   if (L.n_phases > 1 && !L.phase_bar) return cudaErrorInvalidValue;
   if (L.bn == 64) return launch_impl<64, 3>(L, stream, pdl);
+  if (L.bn == 80) return launch_impl<80, 6>(L, stream, pdl);
   if (L.bn == 96) return launch_impl<96, 5>(L, stream, pdl);
   if (L.bn == 128) return launch_impl<128, 4>(L, stream, pdl);
   return cudaErrorInvalidValue;

@@ -284,7 +284,7 @@ struct spec_handle {
   uint8_t* ws = nullptr;
   std::vector<LayerMaps> maps;
   CUtensorMap map_lm;
-  CUtensorMap map_xn[3], map_attn[3], map_h[3];  // B operands for BN = 64, 128, 96 (bn_slot)
+  CUtensorMap map_xn[4], map_attn[4], map_h[4];  // B operands for BN = 64, 128, 96, 80 (bn_slot)
   AttnTcMaps attn_maps;                           // q and the K/V cache (fp16)
   // draft head (cfg.draft_head): its decoder layer is layers[n_layers], maps[n_layers]
   const void* draft_fc_fuse = nullptr;
@@ -293,11 +293,11 @@ struct spec_handle {
   const void* draft_lm_head = nullptr;     // reduced draft vocabulary: [draft_vocab][d]
   const int32_t* draft_ids = nullptr;      // its token ids (device)
   CUtensorMap map_lm_draft;
-  CUtensorMap map_fc_fuse, map_fc_in, map_fsplit[3], map_ge[3];
+  CUtensorMap map_fc_fuse, map_fc_in, map_fsplit[4], map_ge[4];
   std::vector<int32_t> dlen;        // draft-head prefix length per sequence
   std::vector<uint8_t> dready;
-  int resident[3][4] = {};  // co-resident CTAs per SM [bn_slot][epi]
-  int occ_api[3][4] = {};   // what the occupancy query reported
+  int resident[4][4] = {};  // co-resident CTAs per SM [bn_slot][epi]
+  int occ_api[4][4] = {};   // what the occupancy query reported
   // host mirror of per-sequence state
   std::vector<int32_t> len, pending;
   std::vector<int32_t> len_hi;  // upper bound while device-output steps are in flight
@@ -325,7 +325,8 @@ struct spec_handle {
   int attn_clusters[kAttnMaxChunks + 1] = {};  // co-resident clusters of n chunk CTAs
   bool attn_dsmem = true;     // merge chunk partials through distributed shared memory when they fit a cluster
   int bn64_max = 64;          // largest token count planned with 64-token tiles (several token tiles above 64)
-  bool bn96 = true;           // 96-token tiles for 65 .. 96 tokens (else 128)
+  bool bn80 = true;           // 80-token tiles for 65 .. 80 tokens (6 stages: as many weight bytes in flight as at 64)
+  bool bn96 = true;           // 96-token tiles for 65 (81) .. 96 tokens (else 128)
   // L2 prefetch of weights ahead of the GEMM that streams them
   uint64_t* trace = nullptr;  // optional GEMM timeline of one layer's launch
   size_t trace_bytes = 0;
@@ -388,12 +389,13 @@ cudaError_t launch_k(spec_handle* h, int cls, int n_kernels, F&& fn) {
 }
 
 // index of a token-tile width in the per-width tables (tensor maps, residency)
-int bn_slot(int bn) { return bn == 64 ? 0 : bn == 128 ? 1 : 2; }
-constexpr int kTileWidths[3] = {64, 128, 96};
+int bn_slot(int bn) { return bn == 64 ? 0 : bn == 128 ? 1 : bn == 96 ? 2 : 3; }
+constexpr int kNumTileWidths = 4;
+constexpr int kTileWidths[kNumTileWidths] = {64, 128, 96, 80};
 
 GemmPlan plan_gemm(const spec_handle* h, int rows_per_tile, int n_out, int K, int M, int epi) {
   GemmPlan p;
-  p.bn = M <= h->bn64_max ? 64 : (h->bn96 && M <= 96 ? 96 : 128);
+  p.bn = M <= h->bn64_max ? 64 : (h->bn80 && M <= 80 ? 80 : (h->bn96 && M <= 96 ? 96 : 128));
   const int bi = bn_slot(p.bn);
   int per_sm = std::max(1, h->resident[bi][0]);  // one kernel function for every epilogue
   if (h->resident_cap > 0) per_sm = std::min(per_sm, h->resident_cap);
@@ -1339,6 +1341,7 @@ int spec_init(const spec_config* cfg, const spec_weights* w, void* kv_cache, siz
     if (const char* q = strstr(t, "dsmem=")) if (sscanf(q + 6, "%d", &v) == 1) h->attn_dsmem = v != 0;
     if (const char* q = strstr(t, "bn64max=")) if (sscanf(q + 8, "%d", &v) == 1 && v >= 64) h->bn64_max = v;
     if (const char* q = strstr(t, "bn96=")) if (sscanf(q + 5, "%d", &v) == 1) h->bn96 = v != 0;
+    if (const char* q = strstr(t, "bn80=")) if (sscanf(q + 5, "%d", &v) == 1) h->bn80 = v != 0;
     if (const char* q = strstr(t, "per_sm=")) if (sscanf(q + 7, "%d", &v) == 1 && v >= 0) h->resident_cap = v;
     if (const char* q = strstr(t, "sk=")) if (sscanf(q + 3, "%d", &v) == 1 && v >= -1 && v <= 2) h->streamk = v;
     float fv = 0.f;
@@ -1405,7 +1408,7 @@ int spec_init(const spec_config* cfg, const spec_weights* w, void* kv_cache, siz
     if (c.draft_vocab && !make_tmap(&h->map_lm_draft, h->draft_lm_head, c.draft_vocab, c.hidden, 128))
       return bail(SPEC_ERR_CUDA, "tensor map");
     const int* bns = kTileWidths;
-    for (int i = 0; i < 3; ++i) {
+    for (int i = 0; i < kNumTileWidths; ++i) {
       // split activations: a tile of BN tokens is 2*BN rows (hi and lo)
       if (!make_tmap(&h->map_xn[i], h->ws + lay.xn, 2 * (uint64_t)lay.Mpad, c.hidden, 2 * bns[i]) ||
           !make_tmap(&h->map_attn[i], h->ws + lay.attn, 2 * (uint64_t)lay.Mpad, qd, 2 * bns[i]) ||
@@ -1417,7 +1420,7 @@ int spec_init(const spec_config* cfg, const spec_weights* w, void* kv_cache, siz
            !make_tmap(&h->map_ge[i], h->ws + lay.ge, 2 * (uint64_t)lay.Mpad, 2 * (uint64_t)c.hidden, 2 * bns[i])))
         return bail(SPEC_ERR_CUDA, "tensor map");
     }
-    for (int i = 0; i < 3; ++i)
+    for (int i = 0; i < kNumTileWidths; ++i)
       for (int e = 0; e < 4; ++e) {
         const void* fn = gemm_tc_function(bns[i]);
         const int smem = (int)gemm_tc_smem_bytes(bns[i]);
@@ -1855,8 +1858,8 @@ int spec_info(spec_handle* h, int B, int n_nodes, int prefix, char* buf, size_t 
   };
   std::string s = "sms " + std::to_string(h->sm_count) + "; attention clusters held [size:count]";
   for (int cs = 2; cs <= kAttnMaxChunks; ++cs) s += " " + std::to_string(cs) + ":" + std::to_string(h->attn_clusters[cs]);
-  s += "; resident/SM [bn64|bn128|bn96][qkv,swiglu,argmax,resid] = ";
-  for (int i = 0; i < 3; ++i)
+  s += "; resident/SM [bn64|bn128|bn96|bn80][qkv,swiglu,argmax,resid] = ";
+  for (int i = 0; i < kNumTileWidths; ++i)
     for (int e = 0; e < 4; ++e)
       s += std::to_string(h->resident[i][e]) + "(" + std::to_string(h->occ_api[i][e]) + ")" + (e < 3 ? "," : "|");
   s += "; qkv " + g(sp.qkv) + "; o " + g(sp.o) + "; gate_up " + g(sp.gu) + "; down " + g(sp.down) + "; lm " +

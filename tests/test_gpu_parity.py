@@ -82,6 +82,8 @@ BF16_CASES = [
     ("small", 700, "tree60", 700, 2700),
     ("small", 64, "chain8", 64, 64),
     ("small", 500, "tree80", 500, 500),  # 81 tokens: 96-token GEMM tiles
+    ("small", 400, "tree72", 400, 400),  # 73 tokens: 80-token GEMM tiles
+    ("mini", 200, "tree72", 200, 200),
 ]
 
 
@@ -100,6 +102,8 @@ def _shape(kind):
         return synth.tree_from_widths((10, 12, 16, 20, 20, 20, 16, 13), stream=5)
     if kind == "tree80":
         return synth.tree_from_widths(synth.SWEEP_WIDTHS[80], stream=6)
+    if kind == "tree72":
+        return synth.tree_from_widths((10, 10, 10, 10, 10, 8, 8, 6), stream=7)
     raise KeyError(kind)
 
 
@@ -117,6 +121,8 @@ def _pair(which):
 def test_bf16_verify_parity(which, P, kind, s_prefix, s_plant):
     eng, om = _pair(which)
     shape = _shape(kind)
+    if kind == "tree72":
+        assert "qkv bn80 " in eng.info(1, shape.n, P)
     prefix, seq, toks = decided_case(om, P, shape, 0.8, stream0=s_prefix, plant0=s_plant)
     pend = eng.prefill(0, prefix)
     assert pend == seq.pending
