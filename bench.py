@@ -126,6 +126,12 @@ class ClockSampler:
                                       stdout=self.f, stderr=subprocess.DEVNULL)
         except Exception:
             self.p = None
+        # a short run can end before nvidia-smi's first sample: wait (at most 5 s) for it
+        t_end = time.time() + 5.0
+        while self.p is not None and time.time() < t_end and self.p.poll() is None:
+            if os.path.getsize(self.f.name) > 0:
+                break
+            time.sleep(0.02)
 
     def begin(self):
         self.t0 = time.time()
