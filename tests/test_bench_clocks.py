@@ -55,3 +55,21 @@ def test_nearest_sample_when_the_region_is_short():
     out = _sampler(rows, T, T + 0.02).stop()
     assert out["samples"] == 0
     assert out["sm_mhz"] == 1950 and out["reasons"] == []
+
+
+def test_a_short_run_waits_for_the_first_sample(tmp_path, monkeypatch):
+    """nvidia-smi can take longer to print its first sample than a short timed run
+    lasts: the sampler waits (at most 5 s) for it before the warm-up, so the record
+    is never empty."""
+    fake = tmp_path / "nvidia-smi"
+    fake.write_text("#!/bin/sh\nsleep 0.5\nwhile true; do\n"
+                    "  echo '2026/12/03 12:00:00.000, 0, 1965, 1965, 700.0, 0x0, Not Active, Not Active, "
+                    "Not Active, Not Active'\n  sleep 0.05\ndone\n")
+    fake.chmod(0o755)
+    monkeypatch.setenv("PATH", str(tmp_path) + os.pathsep + os.environ.get("PATH", ""))
+    cs = bench.ClockSampler("0")
+    assert os.path.getsize(cs.f.name) > 0
+    cs.begin()
+    cs.end()
+    out = cs.stop()
+    assert out is not None and out["sm_mhz"] == 1965 and out["reasons"] == []
