@@ -93,24 +93,31 @@ __device__ __forceinline__ UnitIter units_of(const GemmTcArgs& a) {
 
 // The work units of a phase that a CTA takes, in order: tile `ut` over k-blocks
 // [kb0, kb1).  Plain and split-K phases: UnitIter's tiles over this CTA's split
-// range.  Stream-K phases (GemmTcArgs::streamk): the phase's tiles x KB
-// k-blocks in tile-major order, cut into one contiguous share per CTA,
-// [W b / grid, W (b + 1) / grid) with W = tiles x KB, whose pieces (one per
-// tile it touches) are the units.  Every CTA then streams the same number of
-// weight k-blocks, whatever the tile count; the CTA holding a tile's first
-// k-block finishes the tile, the CTAs whose shares start inside the tile hand
-// it fp32 partial sums.
+// range.  Stream-K phases (GemmTcArgs::streamk): the shared tiles' sk_tiles x
+// KB k-blocks in tile-major order, cut into one contiguous share per CTA,
+// [W b / grid, W (b + 1) / grid) with W = sk_tiles x KB, whose pieces (one per
+// tile it touches) are the first units; the CTA holding a tile's first k-block
+// finishes the tile, the CTAs whose shares start inside the tile hand it fp32
+// partial sums.  Then the remaining tiles, whole, round-robin from sk_tiles + b:
+// every CTA streams the same number of weight k-blocks, whatever the tile count.
 struct WorkIter {
   int KB, kb0s, kb1s, tiles, grid, S, ut;
-  long long g, w1;  // stream-K cursor and end
+  long long g, w1;  // stream-K cursor and end (over the shared tiles' k-blocks)
   bool sk;
   __device__ bool next(int& t, int& k0, int& k1) {
     if (sk) {
-      if (g >= w1) return false;
-      t = (int)(g / KB);
-      k0 = (int)(g - (long long)t * KB);
-      k1 = (int)min((long long)KB, k0 + (w1 - g));
-      g += k1 - k0;
+      if (g < w1) {
+        t = (int)(g / KB);
+        k0 = (int)(g - (long long)t * KB);
+        k1 = (int)min((long long)KB, k0 + (w1 - g));
+        g += k1 - k0;
+        return true;
+      }
+      if (ut >= tiles) return false;  // then whole tiles, round-robin
+      t = ut;
+      k0 = 0;
+      k1 = KB;
+      ut += grid;
       return true;
     }
     if (ut >= tiles) return false;
@@ -133,9 +140,10 @@ __device__ __forceinline__ WorkIter work_of(const GemmTcArgs& a) {
   w.kb0s = it.split() * a.kb_per_split;
   w.kb1s = min(w.kb0s + a.kb_per_split, w.KB);
   w.sk = a.streamk != 0;
-  const long long W = (long long)w.tiles * w.KB;
+  const long long W = (long long)a.sk_tiles * w.KB;
   w.g = W * it.b / it.grid;
   w.w1 = W * (it.b + 1) / it.grid;
+  if (w.sk) w.ut = a.sk_tiles + it.b;
   return w;
 }
 
@@ -517,7 +525,7 @@ __global__ void __launch_bounds__(kThreads, BN == 64 ? 2 : 1)
           // stream-K, the tile's first k-blocks, not all of them: the CTAs after this
           // one up to `last` hold the rest (each its share's first unit, which waits
           // on nothing); add their sums to this accumulator's hi columns
-          const long long W = (long long)(args.tiles_o * args.tiles_t) * KB;
+          const long long W = (long long)args.sk_tiles * KB;
           const int last = sk_cta_of(W, (long long)ut * KB + KB - 1, grid);
           if (ep_tid == 0) *ep_ok = spin_until_geq(args.counters + ut, last - (int)blockIdx.x, err) ? 1 : 0;
           named_sync(2, 128);

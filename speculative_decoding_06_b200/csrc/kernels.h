@@ -32,12 +32,15 @@ struct GemmTcArgs {
   int K;              // reduction length, multiple of 64
   int M;              // valid tokens (columns); token rows >= M are ignored
   int tiles_o, tiles_t, splits, kb_per_split;
-  // stream-K (SWIGLU, ARGMAX; splits = 1): every CTA takes an equal contiguous
-  // share of the tiles x K/64 k-blocks; a share that starts inside a tile writes
-  // fp32 sums to part + CTA * 128 * BN ([BN tokens][128 rows]) and counts itself
-  // at counters[tile]; the CTA holding the tile's first k-block adds them and
-  // finishes the tile.  Needs tiles x K/64 >= 2 x grid.
-  int streamk;
+  // stream-K (SWIGLU, ARGMAX, TOPK; splits = 1): tiles [0, sk_tiles) are shared
+  // out, every CTA taking an equal contiguous share of their sk_tiles x K/64
+  // k-blocks first; a share that starts inside a tile writes fp32 sums to part +
+  // CTA * 128 * BN ([BN tokens][128 rows]) and counts itself at counters[tile];
+  // the CTA holding the tile's first k-block adds them and finishes the tile.
+  // The other tiles go round-robin, whole (sk_tiles = all the tiles when they are
+  // fewer than the CTAs, else the last round's remainder).  Needs sk_tiles x
+  // K/64 >= 2 x grid.
+  int streamk, sk_tiles;
   int seg_rows[3];    // rows served by mA0, mA1, mA2; unused for SWIGLU
   // RMSNorm folded into the epilogue: the operand rows are x*w, not yet
   // normalised; the result is scaled per token by rsqrt(sum(ss)/norm_d + eps)

@@ -257,6 +257,7 @@ struct LayerMaps {
 struct GemmPlan {
   int bn, tiles_o, tiles_t, splits, kbps, grid;
   int sk = 0;  // stream-K over all resident CTAs (GemmTcArgs::streamk)
+  int sk_tiles = 0;  // the tiles it shares out (the others go whole, round-robin)
 };
 
 struct StepPlan {
@@ -324,6 +325,7 @@ struct spec_handle {
   float rescale_slack = 8.f;  // attention: running-max slack in log2 units (p <= 2^slack)
   int attn_clusters[kAttnMaxChunks + 1] = {};  // co-resident clusters of n chunk CTAs
   bool attn_dsmem = true;     // merge chunk partials through distributed shared memory when they fit a cluster
+  bool sk_hybrid = true;      // stream-K shares only the last round's tiles (else every tile)
   int bn64_max = 64;          // largest token count planned with 64-token tiles (several token tiles above 64)
   bool bn80 = true;           // 80-token tiles for 65 .. 80 tokens (6 stages: as many weight bytes in flight as at 64)
   bool bn96 = true;           // 96-token tiles for 65 (81) .. 96 tokens (else 128)
@@ -415,17 +417,21 @@ GemmPlan plan_gemm(const spec_handle* h, int rows_per_tile, int n_out, int K, in
   p.splits = ceil_div(KB, p.kbps);  // no empty split
   p.grid = p.splits > 1 ? base * p.splits : std::min(base, resident);
   // Stream-K for the phases without split-K when whole tiles would leave CTAs
-  // idle in the last round (more than 2 % of the CTA-rounds): every resident
-  // CTA then streams the same number of weight k-blocks.
+  // idle in the last round (more than 2 % of the CTA-rounds): the last round's
+  // tiles (all of them when there are fewer tiles than CTAs) are shared out so
+  // that every resident CTA streams the same number of weight k-blocks; the
+  // earlier rounds' tiles go whole.
   const bool sk_epi = h->streamk == 1   ? (epi == GEMM_EPI_SWIGLU || epi == GEMM_EPI_ARGMAX || epi == GEMM_EPI_TOPK)
                       : h->streamk == 2 ? epi == GEMM_EPI_SWIGLU
                                         : h->streamk < 0 && epi == GEMM_EPI_SWIGLU && p.bn > 64;
-  if (sk_epi && p.splits == 1 &&
-      resident <= kSkMaxCtas && base <= kCountersPerPhase && (long long)base * KB >= 2LL * resident &&
+  const int sk_tiles = (base < resident || !h->sk_hybrid) ? base : base % resident;
+  if (sk_epi && p.splits == 1 && sk_tiles > 0 &&
+      resident <= kSkMaxCtas && base <= kCountersPerPhase && (long long)sk_tiles * KB >= 2LL * resident &&
       (size_t)resident * 128 * p.bn * 4 <= h->lay.partial_bytes) {
     const long long rounds = ceil_div(base, resident);
     if (rounds * resident * 100 > 102LL * base) {
       p.sk = 1;
+      p.sk_tiles = sk_tiles;
       p.grid = resident;
     }
   }
@@ -523,6 +529,7 @@ GemmTcLaunch gemm_launch(const GemmPlan& p, int epi, int n_out, int K, int M, co
   L.args.splits = p.splits;
   L.args.kb_per_split = p.kbps;
   L.args.streamk = p.sk;
+  L.args.sk_tiles = p.sk_tiles;
   L.args.seg_rows[0] = s0;
   L.args.seg_rows[1] = s1;
   L.args.seg_rows[2] = s2;
@@ -1344,6 +1351,7 @@ int spec_init(const spec_config* cfg, const spec_weights* w, void* kv_cache, siz
     if (const char* q = strstr(t, "bn80=")) if (sscanf(q + 5, "%d", &v) == 1) h->bn80 = v != 0;
     if (const char* q = strstr(t, "per_sm=")) if (sscanf(q + 7, "%d", &v) == 1 && v >= 0) h->resident_cap = v;
     if (const char* q = strstr(t, "sk=")) if (sscanf(q + 3, "%d", &v) == 1 && v >= -1 && v <= 2) h->streamk = v;
+    if (const char* q = strstr(t, "skh=")) if (sscanf(q + 4, "%d", &v) == 1) h->sk_hybrid = v != 0;
     float fv = 0.f;
     if (const char* q = strstr(t, "rescale=")) if (sscanf(q + 8, "%f", &fv) == 1 && fv >= 0.f && fv <= 15.f) h->rescale_slack = fv;
   }
