@@ -168,13 +168,16 @@ def test_bf16_batch_of_sequences():
 WIDE_STREAMS = (7, 7)  # (prefix, planting) streams of the decided step on the 8B-layer-shape model
 
 
-@pytest.mark.parametrize("tune", ["", "sk=1"])
+@pytest.mark.parametrize("tune", ["sk=0", "", "sk=1"])
 def test_wide_bf16_full_size_tiles(tune, monkeypatch):
     """8B layer shapes (d 4096, 32/8 heads, ffn 14336), 2 layers, vocab 16384: full-size tiles and splits;
-    with sk=1 the gate/up and LM-head phases run stream-K (equal k-block shares, partial sums handed over)."""
+    whole tiles everywhere with sk=0, the LM head on stream-K by default (its 128 tiles on 296 CTAs: equal
+    k-block shares, partial sums handed over), gate/up too with sk=1."""
     monkeypatch.setenv("SPEC_TUNE", tune)
     eng, om = make_pair(synth.WIDE_BF16, max_batch=1, max_seq=512, max_nodes=64)
-    assert ("stream-K" in eng.info(1, 61, 200)) == (tune == "sk=1")
+    plan = eng.info(1, 61, 200)
+    assert ("stream-K" in plan.split("; lm ")[1]) == (tune != "sk=0")
+    assert ("stream-K" in plan.split("; gate_up ")[1].split(";")[0]) == (tune == "sk=1")
     shape = synth.tree_from_widths(synth.TREE60_WIDTHS, stream=0)
     prefix, seq, toks = decided_case(om, 200, shape, 0.8, stream0=WIDE_STREAMS[0], plant0=WIDE_STREAMS[1])
     assert eng.prefill(0, prefix) == seq.pending
