@@ -320,9 +320,9 @@ struct spec_handle {
   int max_chunks = kMaxAttnChunks;  // attention key-chunk cap
   int resident_cap = 0;   // 0: as many CTAs per SM as fit
   int streamk = -1;       // stream-K when whole tiles leave CTAs idle: 1 for the SWIGLU, ARGMAX and TOPK
-                          // phases, 2 for SWIGLU only, 0 off, -1 (default, the measured best) the LM head's
-                          // ARGMAX and SWIGLU at 80- to 128-token tiles, where one CTA per SM leaves the most
-                          // idle (SPEC_TUNE sk=)
+                          // phases, 2 for SWIGLU only, 0 off, -1 (default, the measured best) the LM heads'
+                          // ARGMAX and TOPK and SWIGLU at 80- to 128-token tiles, where one CTA per SM leaves
+                          // the most idle (SPEC_TUNE sk=)
   float rescale_slack = 8.f;  // attention: running-max slack in log2 units (p <= 2^slack)
   int attn_clusters[kAttnMaxChunks + 1] = {};  // co-resident clusters of n chunk CTAs
   bool attn_dsmem = true;     // merge chunk partials through distributed shared memory when they fit a cluster
@@ -424,7 +424,8 @@ GemmPlan plan_gemm(const spec_handle* h, int rows_per_tile, int n_out, int K, in
   // earlier rounds' tiles go whole.
   const bool sk_epi = h->streamk == 1   ? (epi == GEMM_EPI_SWIGLU || epi == GEMM_EPI_ARGMAX || epi == GEMM_EPI_TOPK)
                       : h->streamk == 2 ? epi == GEMM_EPI_SWIGLU
-                                        : h->streamk < 0 && (epi == GEMM_EPI_ARGMAX || (epi == GEMM_EPI_SWIGLU && p.bn > 64));
+                                        : h->streamk < 0 && (epi == GEMM_EPI_ARGMAX || epi == GEMM_EPI_TOPK ||
+                                                             (epi == GEMM_EPI_SWIGLU && p.bn > 64));
   const int sk_tiles = (base < resident || !h->sk_hybrid) ? base : base % resident;
   if (sk_epi && p.splits == 1 && sk_tiles > 0 &&
       resident <= kSkMaxCtas && base <= kCountersPerPhase && (long long)sk_tiles * KB >= 2LL * resident &&
